@@ -1,0 +1,234 @@
+/* gpt2.h -- C ABI of the B200 (sm_100a) GPT-2 pre-LayerNorm training step.
+ *
+ * The library computes one training step of a GPT-2 decoder: token + position
+ * embedding, L pre-LN blocks (causal multi-head attention, 4x tanh-GELU MLP,
+ * residual connections), final LayerNorm, a bias-free head tied to the token
+ * embedding (or a separate head), mean next-token cross-entropy, the backward
+ * pass, gradient accumulation over micro-batches, global-norm clipping at 1.0 and
+ * AdamW with weight decay on >= 2-D tensors only.
+ * Sources (page titles and sections): "gpt/docs/LLM.md" Architecture Details
+ * (Embedding Layer, Transformer Blocks, Output Layer); "GPT From Scratch" Key
+ * decisions (pre-norm blocks, tanh-GELU, tying, padding 50,257 -> 50,304, decay
+ * groups, clipping, accumulation); "AxonLM" Key Features and Training Recipe
+ * (1/sqrt(2L) init, betas 0.9/0.95, decay 0.1, clip 1.0); "Genesis" Model Specs
+ * (untied head, 163,009,536 parameters).
+ *
+ * Conventions for every call:
+ *  - Return value: 0 (GPT2_OK) or a negative GPT2_ERR_* code; the message of the
+ *    last failure on a handle is in gpt2_last_error(). Op-level calls (gpt2_op_*)
+ *    have no handle; their last message is in gpt2_op_last_error().
+ *  - Pointers are plain host or device addresses; sizes are element counts. No
+ *    call keeps a caller pointer after it returns.
+ *  - A handle is not thread-safe: one thread at a time per handle.
+ *  - All GPU work of a handle is enqueued on its stream (gpt2_set_stream); calls
+ *    that return data to host memory synchronise that stream.
+ *  - Kernels never trap. Bad token ids are caught on the device (recorded in a
+ *    device error word and replaced by id 0 so that all accesses stay in bounds)
+ *    and reported as GPT2_ERR_TOKEN_RANGE at the next call that synchronises.
+ *    Every mbarrier wait inside a kernel is bounded; one that gives up is
+ *    reported as GPT2_ERR_TIMEOUT.
+ */
+#ifndef GPT2_B200_H
+#define GPT2_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  GPT2_OK = 0,
+  GPT2_ERR_CONFIG = -1,       /* invalid configuration or argument */
+  GPT2_ERR_OOM = -2,          /* device allocation failed */
+  GPT2_ERR_SEQ_TOO_LONG = -3, /* T > cfg.T (the block size) */
+  GPT2_ERR_TOKEN_RANGE = -4,  /* a token or target id outside [0, V) */
+  GPT2_ERR_BATCH = -5,        /* B > B_max, B differs between accumulated micro-batches, or B*T too large */
+  GPT2_ERR_NO_GRAD = -6,      /* gpt2_step / gpt2_get_grads with no accumulated micro-batch */
+  GPT2_ERR_CUDA = -7,         /* a CUDA runtime or driver call failed */
+  GPT2_ERR_TIMEOUT = -8       /* a bounded device-side wait gave up */
+};
+
+enum { GPT2_FP32 = 0, GPT2_BF16 = 1 };
+
+/* Model configuration.
+ *  L layers, H heads, C width (C % H == 0; bf16 mode needs C / H == 64), T block
+ *  size (maximum sequence length), V logical vocabulary (stored padded to a
+ *  multiple of 64; padding rows are zero, excluded from the softmax, receive no
+ *  gradient and are not counted as parameters), tied = 1 ties the head to wte,
+ *  qkv_bias = 1 gives the QKV projection a bias (0 matches the untied
+ *  163,009,536-parameter count), dtype GPT2_FP32 (fp32 everywhere) or GPT2_BF16
+ *  (bf16 GEMM/attention operands, fp32 residual stream, LayerNorm, softmax and
+ *  cross-entropy statistics, fp32 gradients, master weights and Adam state),
+ *  B_max the largest micro-batch the handle's activation arena is sized for. */
+typedef struct {
+  int L, H, C, T, V, tied, qkv_bias, dtype, B_max;
+} gpt2_config;
+
+typedef struct gpt2 gpt2; /* opaque; the library owns all device memory it uses */
+
+/* Create a model on the current CUDA device. Weights: N(0, 0.02), attention-out
+ * and MLP-projection weights N(0, 0.02 / sqrt(2L)), biases 0, LayerNorm gains 1
+ * and biases 0 ("AxonLM", Key Features: 1/sqrt(2L) for residual projections).
+ * The draws follow the init stream of the design notes: element j of tensor i
+ * (canonical order) takes two splitmix64 outputs of seed ^ (i << 40) ^ 2j and
+ * ^ (2j + 1), maps them to u1 in (0, 1] and u2 in [0, 1), and uses the cos branch
+ * of Box-Muller, computed on the host in double and rounded to fp32.
+ * Allocates parameters, gradients, Adam state, the bf16 shadow and the
+ * activation arena for B_max * T tokens. On failure *out is NULL. */
+int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out);
+
+/* Use `stream` (a cudaStream_t, e.g. torch.cuda.current_stream().cuda_stream) for
+ * all later work; NULL selects the library's own stream. */
+int gpt2_set_stream(gpt2* m, void* stream);
+
+/* Forward + backward of one micro-batch of B sequences of length T (T <= cfg.T).
+ * tokens, targets: int32 [B, T], host or device memory (detected), copied in
+ * before the call returns. Gradients of the micro-batch's mean cross-entropy
+ * are ADDED to the accumulated gradients; the micro-batch count k grows by 1.
+ * All micro-batches accumulated before one step must have the same B and T.
+ * loss_out (nullable, host): mean cross-entropy of this micro-batch; when
+ * given, the call synchronises the stream. */
+int gpt2_forward_backward(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T, float* loss_out);
+
+/* Forward only (no gradients, no change to k). loss_out as above (nullable). */
+int gpt2_forward(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T, float* loss_out);
+
+/* Optimizer step on the accumulated gradients: G = (sum of micro-batch
+ * gradients) / k; global-norm clip to 1.0 (coefficient 1 / (||G|| + 1e-6) when
+ * below 1); AdamW with eps 1e-8, bias correction, decoupled decay
+ * p <- p (1 - lr wd) on >= 2-D tensors only; t += 1; gradients zeroed; k = 0.
+ * grad_norm_out (nullable, host): the pre-clip ||G||; when given, the call
+ * synchronises. Returns GPT2_ERR_NO_GRAD when k == 0. */
+int gpt2_step(gpt2* m, float lr, float wd, float beta1, float beta2, float* grad_norm_out);
+
+/* Zero the accumulated gradients; k = 0. */
+int gpt2_zero_grad(gpt2* m);
+
+/* Logical parameter count (V rows, not the padded rows). */
+int gpt2_num_params(const gpt2* m, int64_t* out);
+
+/* Canonical tensor i: name (NUL-terminated, truncated to name_len), shape
+ * (rows, cols; cols = 1 and ndim = 1 for vectors), offset in the canonical flat
+ * order. Canonical order (PyTorch Linear convention W[out][in]): wte[V,C],
+ * wpe[T,C]; per layer ln1_g, ln1_b, qkv_w[3C,C], qkv_b[3C] (if qkv_bias),
+ * ao_w[C,C], ao_b, ln2_g, ln2_b, fc_w[4C,C], fc_b[4C], pj_w[C,4C], pj_b; lnf_g,
+ * lnf_b; head_w[V,C] if untied. Returns GPT2_ERR_CONFIG past the last tensor. */
+int gpt2_tensor_info(const gpt2* m, int i, char* name, int name_len, int64_t* rows, int64_t* cols, int* ndim,
+                     int64_t* offset);
+
+/* Copy parameters, averaged gradients ((1/k) sum, GPT2_ERR_NO_GRAD if k == 0)
+ * or Adam moments between the device and n floats of HOST memory in canonical
+ * order; n must equal gpt2_num_params. Synchronises. */
+int gpt2_get_params(gpt2* m, float* host, int64_t n);
+int gpt2_set_params(gpt2* m, const float* host, int64_t n); /* also refreshes the bf16 shadow */
+int gpt2_get_grads(gpt2* m, float* host, int64_t n);
+int gpt2_get_adam(gpt2* m, float* m_host, float* v_host, int64_t n, int64_t* t_out);
+
+/* Device address and length (floats) of the flat fp32 gradient storage (the
+ * library's internal, padded layout), e.g. for a data-parallel all-reduce of the
+ * accumulated gradients between gpt2_forward_backward and gpt2_step. The buffer
+ * holds the SUM over the k accumulated micro-batches; padding entries are zero.
+ * Owned by the handle; valid until gpt2_destroy. */
+int gpt2_grad_buffer(gpt2* m, float** dev, int64_t* n);
+
+/* Per-kernel-category timing with CUDA events on the handle's stream.
+ * gpt2_profile(m, 1) clears old records and starts recording an event pair around
+ * every launch; gpt2_profile(m, 0) stops. gpt2_profile_read(m, cat, ...) waits for
+ * the stream and returns, for category cat (0 .. count-1), its name, total device
+ * milliseconds, launch count and the algorithmic FLOPs and bytes of those launches
+ * (2*M*N*K per GEMM; causal attention 4*B*H*hd*T(T+1)/2 forward and 2.5 times
+ * that backward; bytes a kernel must move for the memory-bound ones). Returns
+ * GPT2_ERR_CONFIG past the last category. */
+int gpt2_profile(gpt2* m, int enable);
+int gpt2_profile_read(gpt2* m, int cat, char* name, int name_len, double* ms, int64_t* launches, double* flops,
+                      double* bytes);
+
+/* Number of kernel launches the handle has issued since creation (for reports). */
+int gpt2_launch_count(const gpt2* m, int64_t* out);
+
+const char* gpt2_last_error(const gpt2* m);
+void gpt2_destroy(gpt2* m);
+
+/* ------------------------------------------------------------------------
+ * Op-level entry points: single kernels on caller-owned DEVICE buffers, for
+ * per-kernel checks and measurement. `stream` is a cudaStream_t (NULL = the
+ * legacy default stream). dtype selects the activation type: GPT2_BF16 for
+ * bf16 (__nv_bfloat16) buffers, GPT2_FP32 for float. fp32 buffers named f32_*
+ * are float in both modes. Calls are asynchronous unless stated otherwise;
+ * those that need scratch memory allocate it with cudaMallocAsync on the stream
+ * and free it the same way.
+ * ------------------------------------------------------------------------ */
+
+/* Epilogues of gpt2_op_gemm (D = accumulator, fp32):
+ *  0 out(act) = D + bias                     qkv / logits
+ *  1 out(act) = D + bias, out2(act) = gelu_tanh(D + bias)   fc + GELU
+ *  2 out(f32) = aux(f32) + D + bias          residual add
+ *  3 out(act) = D * gelu_tanh'(aux(act))     GELU backward
+ *  4 out(f32) = D, or out += D when accumulate   dX / dW
+ * D[M, N] = sum_k A(m, k) B(n, k), with A(m, k) = A[m*lda + k] (a_mn = 0) or
+ * A[k*lda + m] (a_mn = 1), and B(n, k) likewise with b_mn. bias (nullable) is
+ * f32 [N]. ksplit > 1 (bf16 only, epilogue 4 only) splits K into ksplit slices
+ * reduced in a fixed order. bf16 needs lda, ldb, ldo multiples of 8 and 16-byte
+ * aligned base pointers (tensor-memory-accelerator tiles). */
+int gpt2_op_gemm(int dtype, const void* A, int64_t lda, int a_mn, const void* B, int64_t ldb, int b_mn, int M, int N,
+                 int K, int epilogue, void* out, int64_t ldo, void* out2, int64_t ldo2, const float* bias,
+                 const void* aux, int64_t ld_aux, int accumulate, int ksplit, void* stream);
+
+/* LayerNorm forward over rows of f32_x [N, C]: y(act) [N, C], f32 mean and rstd
+ * [N]. eps 1e-5, biased variance. C % 4 == 0, C <= 2048. */
+int gpt2_op_layernorm_fwd(int dtype, const float* f32_x, const float* f32_g, const float* f32_b, int N, int C, void* y,
+                          float* f32_mean, float* f32_rstd, void* stream);
+
+/* LayerNorm backward: f32_dres (+)= dx (accumulate = 1 adds), dres_act (nullable)
+ * = copy of the new f32_dres in the activation type, f32_dg and f32_db (+)= the
+ * parameter gradients (accumulate_params = 1 adds). */
+int gpt2_op_layernorm_bwd(int dtype, const float* f32_dy, const float* f32_x, const float* f32_g,
+                          const float* f32_mean, const float* f32_rstd, int N, int C, float* f32_dres, void* dres_act,
+                          int accumulate, float* f32_dg, float* f32_db, int accumulate_params, void* stream);
+
+/* Causal attention forward: qkv(act) [B*T, 3*NH*hd] -> out(act) [B*T, NH*hd],
+ * f32_lse [B, NH, T] (natural log). bf16 requires hd == 64; fp32 requires hd a
+ * multiple of 32, at most 128. */
+int gpt2_op_attention_fwd(int dtype, const void* qkv, int B, int T, int NH, int hd, void* out, float* f32_lse,
+                          void* stream);
+
+/* Causal attention backward: dqkv(act) [B*T, 3*NH*hd] from qkv, out, dout(act)
+ * and f32_lse. Deterministic (no atomics). */
+int gpt2_op_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* f32_lse, int B,
+                          int T, int NH, int hd, void* dqkv, void* stream);
+
+/* Embedding forward: f32_x0[b*T + t, :] = wte[tokens[b*T + t], :] + wpe[t, :]
+ * (wte [V, C], wpe [>= T, C], f32). Ids outside [0, V) raise
+ * GPT2_ERR_TOKEN_RANGE (this call synchronises to report it). */
+int gpt2_op_embedding_fwd(const int32_t* tokens, const float* f32_wte, const float* f32_wpe, int B, int T, int C, int V,
+                          float* f32_x0, void* stream);
+
+/* Stable bucketing of token positions by id (the atomic-free embedding
+ * backward's first stage). tokens [N] device, N <= 32768, ids in [0, V).
+ * Outputs (device): sorted_pos [N] (positions ordered by (id, position)),
+ * seg_id [N] and seg_start [N + 1] (distinct ids in increasing order and the
+ * index in sorted_pos where each id's positions begin; seg_start[nseg] = N).
+ * *nseg_out (host) = number of distinct ids. Synchronises. */
+int gpt2_op_token_buckets(const int32_t* tokens, int N, int V, int32_t* sorted_pos, int32_t* seg_id,
+                          int32_t* seg_start, int32_t* nseg_out, void* stream);
+
+/* Embedding backward, atomic-free and deterministic: f32_dwte[v] += sum of
+ * f32_dx0 rows at positions with tokens == v; f32_dwpe[t] += sum_b
+ * f32_dx0[b*T + t]. B*T <= 32768. */
+int gpt2_op_embedding_bwd(const int32_t* tokens, const float* f32_dx0, int B, int T, int C, int V, float* f32_dwte,
+                          float* f32_dwpe, void* stream);
+
+/* Cross-entropy over rows of logits(act) [N, ld] (first V columns; ld % 8 == 0,
+ * ld <= 65536): f32_row_loss[n] = logsumexp - z[target]; logits overwritten by
+ * (softmax - onehot) * scale (padding columns set to 0). */
+int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, const int32_t* targets, float scale,
+                          float* f32_row_loss, void* stream);
+
+const char* gpt2_op_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT2_B200_H */

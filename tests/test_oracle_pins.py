@@ -323,6 +323,22 @@ def test_accumulation_equals_big_batch():
     assert np.max(np.abs(G - Gbig)) <= 1e-10 * np.max(np.abs(Gbig))
 
 
+def test_key_bias_gradient_vanishes():
+    """Adding q.b_k to every score of a row leaves the softmax unchanged, so the
+    gradient of the key third of the QKV bias is identically zero while the query
+    and value parts are not."""
+    p = rand_params(TINY, 15)
+    tok, tgt = batch(TINY, 2)
+    _, g = oracle.forward_backward(TINY, p, tok, tgt)
+    C = TINY.C
+    for t in oracle.tensors(TINY):
+        if t.name.endswith("qkv_b"):
+            gb = g[t.offset:t.offset + t.size]
+            scale = np.max(np.abs(gb))
+            assert np.max(np.abs(gb[C:2 * C])) <= 1e-12 * scale
+            assert np.max(np.abs(gb[:C])) > 1e-6 * scale and np.max(np.abs(gb[2 * C:])) > 1e-3 * scale
+
+
 def test_tying_gradient_is_sum_of_embedding_and_head_parts():
     tied = oracle.Config(2, 2, 16, 8, 23, 1, 1)
     untied = oracle.Config(2, 2, 16, 8, 23, 0, 1)

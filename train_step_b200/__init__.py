@@ -1,0 +1,321 @@
+"""Python binding of the B200 GPT-2 training-step library (include/gpt2.h).
+
+Argument marshalling only: every step of the training step runs in the CUDA
+kernels of ``libgpt2_b200.so``. PyTorch supplies device memory and streams. If
+the shared library is missing this module raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgpt2_b200.so")
+
+FP32, BF16 = 0, 1
+EPI_BIAS, EPI_BIAS_GELU, EPI_RESID, EPI_DGELU, EPI_F32 = 0, 1, 2, 3, 4
+
+ERRORS = {
+    -1: "GPT2_ERR_CONFIG", -2: "GPT2_ERR_OOM", -3: "GPT2_ERR_SEQ_TOO_LONG", -4: "GPT2_ERR_TOKEN_RANGE",
+    -5: "GPT2_ERR_BATCH", -6: "GPT2_ERR_NO_GRAD", -7: "GPT2_ERR_CUDA", -8: "GPT2_ERR_TIMEOUT",
+}
+
+
+class Gpt2Error(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{ERRORS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class _Config(ct.Structure):
+    _fields_ = [(n, ct.c_int) for n in ("L", "H", "C", "T", "V", "tied", "qkv_bias", "dtype", "B_max")]
+
+
+_lib = None
+_SYMBOLS = {
+    "gpt2_create": ([ct.POINTER(_Config), ct.c_uint64, ct.POINTER(ct.c_void_p)], ct.c_int),
+    "gpt2_set_stream": ([ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_forward_backward": ([ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_void_p], ct.c_int),
+    "gpt2_forward": ([ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_void_p], ct.c_int),
+    "gpt2_step": ([ct.c_void_p, ct.c_float, ct.c_float, ct.c_float, ct.c_float, ct.c_void_p], ct.c_int),
+    "gpt2_zero_grad": ([ct.c_void_p], ct.c_int),
+    "gpt2_num_params": ([ct.c_void_p, ct.POINTER(ct.c_int64)], ct.c_int),
+    "gpt2_tensor_info": ([ct.c_void_p, ct.c_int, ct.c_char_p, ct.c_int, ct.POINTER(ct.c_int64),
+                          ct.POINTER(ct.c_int64), ct.POINTER(ct.c_int), ct.POINTER(ct.c_int64)], ct.c_int),
+    "gpt2_get_params": ([ct.c_void_p, ct.c_void_p, ct.c_int64], ct.c_int),
+    "gpt2_set_params": ([ct.c_void_p, ct.c_void_p, ct.c_int64], ct.c_int),
+    "gpt2_get_grads": ([ct.c_void_p, ct.c_void_p, ct.c_int64], ct.c_int),
+    "gpt2_get_adam": ([ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int64, ct.POINTER(ct.c_int64)], ct.c_int),
+    "gpt2_launch_count": ([ct.c_void_p, ct.POINTER(ct.c_int64)], ct.c_int),
+    "gpt2_grad_buffer": ([ct.c_void_p, ct.POINTER(ct.c_void_p), ct.POINTER(ct.c_int64)], ct.c_int),
+    "gpt2_profile": ([ct.c_void_p, ct.c_int], ct.c_int),
+    "gpt2_profile_read": ([ct.c_void_p, ct.c_int, ct.c_char_p, ct.c_int, ct.POINTER(ct.c_double),
+                           ct.POINTER(ct.c_int64), ct.POINTER(ct.c_double), ct.POINTER(ct.c_double)], ct.c_int),
+    "gpt2_last_error": ([ct.c_void_p], ct.c_char_p),
+    "gpt2_destroy": ([ct.c_void_p], None),
+    "gpt2_op_gemm": ([ct.c_int, ct.c_void_p, ct.c_int64, ct.c_int, ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int,
+                      ct.c_int, ct.c_int, ct.c_int, ct.c_void_p, ct.c_int64, ct.c_void_p, ct.c_int64, ct.c_void_p,
+                      ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_void_p], ct.c_int),
+    "gpt2_op_layernorm_fwd": ([ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_void_p,
+                               ct.c_void_p, ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_layernorm_bwd": ([ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int,
+                               ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_int,
+                               ct.c_void_p], ct.c_int),
+    "gpt2_op_attention_fwd": ([ct.c_int, ct.c_void_p, ct.c_int, ct.c_int, ct.c_int, ct.c_int, ct.c_void_p,
+                               ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_attention_bwd": ([ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int,
+                               ct.c_int, ct.c_int, ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_embedding_fwd": ([ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_int, ct.c_int,
+                               ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_token_buckets": ([ct.c_void_p, ct.c_int, ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p,
+                               ct.POINTER(ct.c_int32), ct.c_void_p], ct.c_int),
+    "gpt2_op_embedding_bwd": ([ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_int, ct.c_int, ct.c_void_p,
+                               ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_cross_entropy": ([ct.c_int, ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_void_p, ct.c_float,
+                               ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_last_error": ([], ct.c_char_p),
+}
+
+
+def lib() -> ct.CDLL:
+    """Load libgpt2_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m train_step_b200.build` "
+                               "(there is no CPU fallback)")
+        L = ct.CDLL(LIB_PATH)
+        for name, (args, res) in _SYMBOLS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SYMBOLS)
+
+
+def _ptr(x):
+    """Address of a torch tensor, numpy array or None."""
+    if x is None:
+        return None
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    return x.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is not None:
+        return stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _op(code: int) -> None:
+    if code != 0:
+        raise Gpt2Error(code, lib().gpt2_op_last_error().decode())
+
+
+@dataclass
+class Config:
+    L: int
+    H: int
+    C: int
+    T: int
+    V: int
+    tied: int = 1
+    qkv_bias: int = 1
+    dtype: int = BF16
+    B_max: int = 1
+
+    def c(self) -> _Config:
+        return _Config(self.L, self.H, self.C, self.T, self.V, self.tied, self.qkv_bias, self.dtype, self.B_max)
+
+
+class GPT2:
+    """One model handle: parameters, gradients, Adam state and activations on the GPU."""
+
+    def __init__(self, cfg: Config, seed: int = 42, stream=None):
+        self.cfg = cfg
+        h = ct.c_void_p()
+        c = cfg.c()
+        rc = lib().gpt2_create(ct.byref(c), seed, ct.byref(h))
+        if rc != 0:
+            raise Gpt2Error(rc, "gpt2_create failed")
+        self.h = h
+        if stream is not None:
+            self._check(lib().gpt2_set_stream(self.h, stream))
+
+    def _check(self, rc: int) -> None:
+        if rc != 0:
+            raise Gpt2Error(rc, lib().gpt2_last_error(self.h).decode())
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            lib().gpt2_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_stream(self, stream) -> None:
+        self._check(lib().gpt2_set_stream(self.h, stream))
+
+    def forward_backward(self, tokens, targets, want_loss: bool = True):
+        B, T = tokens.shape
+        loss = ct.c_float()
+        self._check(lib().gpt2_forward_backward(self.h, _ptr(tokens), _ptr(targets), B, T,
+                                                ct.byref(loss) if want_loss else None))
+        return loss.value if want_loss else None
+
+    def forward(self, tokens, targets):
+        B, T = tokens.shape
+        loss = ct.c_float()
+        self._check(lib().gpt2_forward(self.h, _ptr(tokens), _ptr(targets), B, T, ct.byref(loss)))
+        return loss.value
+
+    def step(self, lr: float, wd: float, beta1: float = 0.9, beta2: float = 0.95, want_norm: bool = True):
+        n = ct.c_float()
+        self._check(lib().gpt2_step(self.h, lr, wd, beta1, beta2, ct.byref(n) if want_norm else None))
+        return n.value if want_norm else None
+
+    def zero_grad(self) -> None:
+        self._check(lib().gpt2_zero_grad(self.h))
+
+    @property
+    def num_params(self) -> int:
+        n = ct.c_int64()
+        self._check(lib().gpt2_num_params(self.h, ct.byref(n)))
+        return n.value
+
+    def tensors(self):
+        out = []
+        name = ct.create_string_buffer(64)
+        r, c, o = ct.c_int64(), ct.c_int64(), ct.c_int64()
+        nd = ct.c_int()
+        i = 0
+        while lib().gpt2_tensor_info(self.h, i, name, 64, ct.byref(r), ct.byref(c), ct.byref(nd), ct.byref(o)) == 0:
+            shape = (r.value, c.value) if nd.value == 2 else (r.value,)
+            out.append((name.value.decode(), shape, o.value))
+            i += 1
+        return out
+
+    def get_params(self) -> np.ndarray:
+        out = np.empty(self.num_params, np.float32)
+        self._check(lib().gpt2_get_params(self.h, out.ctypes.data, out.size))
+        return out
+
+    def set_params(self, p) -> None:
+        p = np.ascontiguousarray(p, np.float32)
+        self._check(lib().gpt2_set_params(self.h, p.ctypes.data, p.size))
+
+    def get_grads(self) -> np.ndarray:
+        out = np.empty(self.num_params, np.float32)
+        self._check(lib().gpt2_get_grads(self.h, out.ctypes.data, out.size))
+        return out
+
+    def get_adam(self):
+        m = np.empty(self.num_params, np.float32)
+        v = np.empty(self.num_params, np.float32)
+        t = ct.c_int64()
+        self._check(lib().gpt2_get_adam(self.h, m.ctypes.data, v.ctypes.data, m.size, ct.byref(t)))
+        return m, v, t.value
+
+    def grad_buffer(self):
+        """(device address, length in floats) of the flat gradient storage."""
+        p = ct.c_void_p()
+        n = ct.c_int64()
+        self._check(lib().gpt2_grad_buffer(self.h, ct.byref(p), ct.byref(n)))
+        return p.value, n.value
+
+    def profile(self, enable: bool) -> None:
+        self._check(lib().gpt2_profile(self.h, int(enable)))
+
+    def profile_read(self) -> dict:
+        """{category: (ms, launches, flops, bytes)} of the recorded launches."""
+        out = {}
+        name = ct.create_string_buffer(64)
+        ms, fl, by = ct.c_double(), ct.c_double(), ct.c_double()
+        n = ct.c_int64()
+        i = 0
+        while lib().gpt2_profile_read(self.h, i, name, 64, ct.byref(ms), ct.byref(n), ct.byref(fl), ct.byref(by)) == 0:
+            out[name.value.decode()] = (ms.value, n.value, fl.value, by.value)
+            i += 1
+        return out
+
+    def launch_count(self) -> int:
+        n = ct.c_int64()
+        self._check(lib().gpt2_launch_count(self.h, ct.byref(n)))
+        return n.value
+
+
+# ---------------------------------------------------------------------------
+# op-level wrappers (torch CUDA tensors in, results written in place)
+# ---------------------------------------------------------------------------
+def _dt(t) -> int:
+    import torch
+    return BF16 if t.dtype == torch.bfloat16 else FP32
+
+
+def gemm(A, B, out, *, M, N, K, lda, ldb, ldo, a_mn=False, b_mn=False, epilogue=EPI_F32, out2=None, ldo2=0,
+         bias=None, aux=None, ld_aux=0, accumulate=False, ksplit=1, stream=None):
+    _op(lib().gpt2_op_gemm(_dt(A), _ptr(A), lda, int(a_mn), _ptr(B), ldb, int(b_mn), M, N, K, epilogue, _ptr(out),
+                           ldo, _ptr(out2), ldo2, _ptr(bias), _ptr(aux), ld_aux, int(accumulate), ksplit,
+                           _stream(stream)))
+
+
+def layernorm_fwd(x, g, b, y, mean, rstd, stream=None):
+    N, C = x.shape
+    _op(lib().gpt2_op_layernorm_fwd(_dt(y), _ptr(x), _ptr(g), _ptr(b), N, C, _ptr(y), _ptr(mean), _ptr(rstd),
+                                    _stream(stream)))
+
+
+def layernorm_bwd(dy, x, g, mean, rstd, dres, dres_act, dg, db, accumulate=False, accumulate_params=False,
+                  dtype=None, stream=None):
+    N, C = x.shape
+    dt = dtype if dtype is not None else (_dt(dres_act) if dres_act is not None else FP32)
+    _op(lib().gpt2_op_layernorm_bwd(dt, _ptr(dy), _ptr(x), _ptr(g), _ptr(mean), _ptr(rstd), N, C, _ptr(dres),
+                                    _ptr(dres_act), int(accumulate), _ptr(dg), _ptr(db), int(accumulate_params),
+                                    _stream(stream)))
+
+
+def attention_fwd(qkv, out, lse, B, T, NH, hd, stream=None):
+    _op(lib().gpt2_op_attention_fwd(_dt(qkv), _ptr(qkv), B, T, NH, hd, _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def attention_bwd(qkv, out, dout, lse, dqkv, B, T, NH, hd, stream=None):
+    _op(lib().gpt2_op_attention_bwd(_dt(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), B, T, NH, hd,
+                                    _ptr(dqkv), _stream(stream)))
+
+
+def embedding_fwd(tokens, wte, wpe, x0, stream=None):
+    B, T = tokens.shape
+    V, C = wte.shape
+    _op(lib().gpt2_op_embedding_fwd(_ptr(tokens), _ptr(wte), _ptr(wpe), B, T, C, V, _ptr(x0), _stream(stream)))
+
+
+def token_buckets(tokens, V, sorted_pos, seg_id, seg_start, stream=None) -> int:
+    n = ct.c_int32()
+    _op(lib().gpt2_op_token_buckets(_ptr(tokens), tokens.numel(), V, _ptr(sorted_pos), _ptr(seg_id), _ptr(seg_start),
+                                    ct.byref(n), _stream(stream)))
+    return n.value
+
+
+def embedding_bwd(tokens, dx0, dwte, dwpe, stream=None):
+    B, T = tokens.shape
+    V, C = dwte.shape
+    _op(lib().gpt2_op_embedding_bwd(_ptr(tokens), _ptr(dx0), B, T, C, V, _ptr(dwte), _ptr(dwpe), _stream(stream)))
+
+
+def cross_entropy(logits, V, targets, scale, row_loss, stream=None):
+    N, ld = logits.shape
+    _op(lib().gpt2_op_cross_entropy(_dt(logits), _ptr(logits), ld, N, V, _ptr(targets), scale, _ptr(row_loss),
+                                    _stream(stream)))

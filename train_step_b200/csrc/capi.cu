@@ -1,0 +1,916 @@
+// capi.cu -- the C ABI of include/gpt2.h: handle, device arena, initialisation and
+// the orchestration of one micro-batch (forward, backward) and of the optimizer
+// step, all enqueued on one CUDA stream.
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "launch.cuh"
+
+using namespace g2;
+
+namespace {
+
+constexpr int HEAD_CHUNK_ROWS = 4096;  // rows of logits materialised at once
+
+struct TensorSlot {
+  std::string name;
+  int64_t rows, cols;       // logical shape (cols = 1 for vectors)
+  int ndim;
+  double sigma, fill;       // init
+  int64_t canon_off;        // offset in the canonical (logical) flat order
+  int64_t dev_off;          // offset in device storage
+  int64_t dev_rows;         // rows in storage (vocabulary tensors padded to Vp)
+};
+
+struct LayerP {
+  float *ln1_g, *ln1_b, *qkv_w, *qkv_b, *ao_w, *ao_b, *ln2_g, *ln2_b, *fc_w, *fc_b, *pj_w, *pj_b;
+};
+
+thread_local std::string g_op_error;
+
+uint64_t splitmix64_at(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+}  // namespace
+
+struct gpt2 {
+  gpt2_config cfg{};
+  int Vp = 0, C = 0, F = 0, NH = 0, hd = 0, L = 0, T = 0, Nmax = 0;
+  int act_bytes = 4;
+  std::vector<TensorSlot> tensors;
+  int64_t n_logical = 0, n_store = 0, n_decay = 0;
+  // parameter state (device)
+  float *p = nullptr, *g = nullptr, *m = nullptr, *v = nullptr;
+  bf16* shadow = nullptr;
+  // views into p (master) and g, and the GEMM operand view (shadow or master)
+  float *wte = nullptr, *wpe = nullptr, *lnf_g = nullptr, *lnf_b = nullptr, *head = nullptr;
+  std::vector<LayerP> lp, lg;
+  float *g_wte = nullptr, *g_wpe = nullptr, *g_lnf_g = nullptr, *g_lnf_b = nullptr, *g_head = nullptr;
+  // activations
+  char* arena = nullptr;
+  size_t arena_bytes = 0;
+  float *x = nullptr, *stat_mean = nullptr, *stat_rstd = nullptr, *lse = nullptr;
+  char *h1 = nullptr, *qkv = nullptr, *att = nullptr, *h2 = nullptr, *u = nullptr, *a = nullptr, *xf = nullptr;
+  char *logits = nullptr, *dres_act = nullptr, *du = nullptr, *datt = nullptr, *dqkv = nullptr;
+  float *dres = nullptr, *dh = nullptr, *Dattn = nullptr, *row_loss = nullptr, *part = nullptr, *splitk = nullptr;
+  size_t part_floats = 0, splitk_floats = 0;
+  int *tok = nullptr, *tgt = nullptr;
+  void* emb_scratch = nullptr;
+  // scalars
+  int* d_err = nullptr;
+  float* d_loss = nullptr;
+  float* d_gnorm = nullptr;
+  double* d_norm_part = nullptr;
+  int norm_parts = 0;
+  // state
+  cudaStream_t stream = nullptr;
+  bool own_stream = false;
+  int k = 0, k_B = 0, k_T = 0;
+  int64_t t = 0;
+  long long launches = 0;
+  int num_sms = 148;
+  std::string err;
+  Profiler prof;
+
+  LaunchCtx ctx() {
+    LaunchCtx c;
+    c.prof = &prof;
+    c.stream = stream;
+    c.d_err = d_err;
+    c.msg = &err;
+    c.launches = &launches;
+    c.splitk_ws = splitk;
+    c.splitk_cap = splitk_floats;
+    c.num_sms = num_sms;
+    return c;
+  }
+  float* P(const std::string& n) { return p + find(n).dev_off; }
+  float* G(const std::string& n) { return g + find(n).dev_off; }
+  const TensorSlot& find(const std::string& n) const {
+    for (auto& s : tensors)
+      if (s.name == n) return s;
+    static TensorSlot none{};
+    return none;
+  }
+  bool has(const std::string& n) const {
+    for (auto& s : tensors)
+      if (s.name == n) return true;
+    return false;
+  }
+  // GEMM operand for a weight: the bf16 shadow in bf16 mode, the master otherwise
+  const void* W(const float* master) const {
+    if (cfg.dtype == GPT2_BF16) return shadow + (master - p);
+    return master;
+  }
+  char* act(char* base, int64_t layer, int64_t per_layer_elems) const {
+    return base + layer * per_layer_elems * act_bytes;
+  }
+};
+
+namespace {
+
+int set_err(gpt2* m, int code, const std::string& msg) {
+  if (m) m->err = msg;
+  return code;
+}
+
+int cuda_err(gpt2* m, cudaError_t e, const char* what) {
+  return set_err(m, GPT2_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define CK(m, call)                                  \
+  do {                                               \
+    cudaError_t e_ = (call);                         \
+    if (e_ != cudaSuccess) return cuda_err(m, e_, #call); \
+  } while (0)
+#define RK(call)            \
+  do {                      \
+    int r_ = (call);        \
+    if (r_) return r_;      \
+  } while (0)
+
+int64_t align64(int64_t x) { return (x + 63) & ~int64_t(63); }
+
+void build_tensors(gpt2* m) {
+  const gpt2_config& c = m->cfg;
+  const int64_t C = c.C, F = 4LL * c.C;
+  const double s = 0.02, sr = 0.02 / std::sqrt(2.0 * c.L);
+  auto& t = m->tensors;
+  t.clear();
+  auto add = [&](const std::string& n, int64_t r, int64_t cc, int nd, double sg, double fill, int64_t dev_rows) {
+    t.push_back(TensorSlot{n, r, cc, nd, sg, fill, 0, 0, dev_rows});
+  };
+  add("wte", c.V, C, 2, s, 0, m->Vp);
+  add("wpe", c.T, C, 2, s, 0, c.T);
+  for (int l = 0; l < c.L; ++l) {
+    std::string p = "h" + std::to_string(l) + ".";
+    add(p + "ln1_g", C, 1, 1, 0, 1, C);
+    add(p + "ln1_b", C, 1, 1, 0, 0, C);
+    add(p + "qkv_w", 3 * C, C, 2, s, 0, 3 * C);
+    if (c.qkv_bias) add(p + "qkv_b", 3 * C, 1, 1, 0, 0, 3 * C);
+    add(p + "ao_w", C, C, 2, sr, 0, C);
+    add(p + "ao_b", C, 1, 1, 0, 0, C);
+    add(p + "ln2_g", C, 1, 1, 0, 1, C);
+    add(p + "ln2_b", C, 1, 1, 0, 0, C);
+    add(p + "fc_w", F, C, 2, s, 0, F);
+    add(p + "fc_b", F, 1, 1, 0, 0, F);
+    add(p + "pj_w", C, F, 2, sr, 0, C);
+    add(p + "pj_b", C, 1, 1, 0, 0, C);
+  }
+  add("lnf_g", C, 1, 1, 0, 1, C);
+  add("lnf_b", C, 1, 1, 0, 0, C);
+  if (!c.tied) add("head_w", c.V, C, 2, s, 0, m->Vp);
+  int64_t off = 0;
+  for (auto& x : t) {
+    x.canon_off = off;
+    off += x.rows * x.cols;
+  }
+  m->n_logical = off;
+  // storage: all >= 2-D tensors first (weight decay and the bf16 shadow cover
+  // exactly that prefix), each tensor 64-element aligned
+  int64_t d = 0;
+  for (auto& x : t)
+    if (x.ndim == 2) {
+      x.dev_off = d;
+      d = align64(d + x.dev_rows * x.cols);
+    }
+  m->n_decay = d;
+  for (auto& x : t)
+    if (x.ndim == 1) {
+      x.dev_off = d;
+      d = align64(d + x.dev_rows * x.cols);
+    }
+  m->n_store = d;
+}
+
+void host_init(const gpt2* m, uint64_t seed, std::vector<float>& out) {
+  out.assign(m->n_logical, 0.f);
+  for (size_t i = 0; i < m->tensors.size(); ++i) {
+    const TensorSlot& t = m->tensors[i];
+    const int64_t n = t.rows * t.cols;
+    float* o = out.data() + t.canon_off;
+    if (t.sigma == 0) {
+      for (int64_t j = 0; j < n; ++j) o[j] = (float)t.fill;
+      continue;
+    }
+    const uint64_t base = seed ^ ((uint64_t)i << 40);
+    for (int64_t j = 0; j < n; ++j) {
+      const uint64_t x1 = splitmix64_at(base ^ (uint64_t)(2 * j));
+      const uint64_t x2 = splitmix64_at(base ^ (uint64_t)(2 * j + 1));
+      const double u1 = ((double)(x1 >> 11) + 1.0) * 0x1.0p-53;
+      const double u2 = (double)(x2 >> 11) * 0x1.0p-53;
+      const double z = std::sqrt(-2.0 * std::log(u1)) * std::cos(2.0 * M_PI * u2);
+      o[j] = (float)(t.sigma * z);
+    }
+  }
+}
+
+int check_device_error(gpt2* m) {
+  int h = 0;
+  CK(m, cudaMemcpyAsync(&h, m->d_err, sizeof(int), cudaMemcpyDeviceToHost, m->stream));
+  CK(m, cudaStreamSynchronize(m->stream));
+  if (h) {
+    CK(m, cudaMemsetAsync(m->d_err, 0, sizeof(int), m->stream));
+    if (h == DEV_TOKEN_RANGE) return set_err(m, GPT2_ERR_TOKEN_RANGE, "a token or target id is outside [0, V)");
+    if (h == DEV_TIMEOUT) return set_err(m, GPT2_ERR_TIMEOUT, "a bounded device-side wait gave up");
+    return set_err(m, GPT2_ERR_CUDA, "device error word set");
+  }
+  return GPT2_OK;
+}
+
+int copy_tokens(gpt2* m, int* dst, const int32_t* src, size_t n) {
+  cudaPointerAttributes at;
+  cudaMemcpyKind kind = cudaMemcpyHostToDevice;
+  if (cudaPointerGetAttributes(&at, src) == cudaSuccess &&
+      (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged))
+    kind = cudaMemcpyDeviceToDevice;
+  cudaGetLastError();
+  CK(m, cudaMemcpyAsync(dst, src, n * sizeof(int32_t), kind, m->stream));
+  return GPT2_OK;
+}
+
+// Forward of one micro-batch; with `backward`, also the backward pass that adds
+// the gradients of this micro-batch's mean loss into m->g.
+int run_micro_batch(gpt2* m, int B, int T, bool backward) {
+  LaunchCtx c = m->ctx();
+  const int dt = m->cfg.dtype;
+  const int N = B * T, C = m->C, F = m->F, L = m->L, NH = m->NH, hd = m->hd, Vp = m->Vp;
+  const int64_t NC = (int64_t)m->Nmax * C, NF = (int64_t)m->Nmax * F, N3C = 3 * NC;
+  const int64_t NLSE = (int64_t)m->cfg.B_max * NH * m->T;
+  const int ab = m->act_bytes;
+  auto xs = [&](int i) { return m->x + (int64_t)i * NC; };
+  auto mean = [&](int i) { return m->stat_mean + (int64_t)i * m->Nmax; };
+  auto rstd = [&](int i) { return m->stat_rstd + (int64_t)i * m->Nmax; };
+  auto ACT = [&](char* base, int l, int64_t per) -> void* { return base + (int64_t)l * per * ab; };
+  auto LN_F = [&](const float* x, const float* gg, const float* bb, void* y, float* mu, float* rs) {
+    return dt == GPT2_BF16 ? layernorm_fwd_t<bf16>(c, x, gg, bb, N, C, (bf16*)y, mu, rs)
+                           : layernorm_fwd_t<float>(c, x, gg, bb, N, C, (float*)y, mu, rs);
+  };
+
+  // ---------------- forward ----------------
+  RK(embedding_fwd(c, m->tok, m->wte, m->wpe, N, T, C, m->cfg.V, xs(0)));
+  for (int l = 0; l < L; ++l) {
+    const LayerP& w = m->lp[l];
+    void* h1 = ACT(m->h1, l, NC);
+    void* qkv = ACT(m->qkv, l, N3C);
+    void* att = ACT(m->att, l, NC);
+    void* h2 = ACT(m->h2, l, NC);
+    void* u = ACT(m->u, l, NF);
+    void* a = ACT(m->a, l, NF);
+    float* lse = m->lse + l * NLSE;
+    RK(LN_F(xs(2 * l), w.ln1_g, w.ln1_b, h1, mean(2 * l), rstd(2 * l)));
+    RK(gemm(c, dt, GemmDesc{h1, C, false, m->W(w.qkv_w), C, false, N, 3 * C, C, EPI_BF16, qkv, 3 * C, nullptr, 0,
+                            w.qkv_b, nullptr, 0, 0, 1}));
+    RK(attention_fwd(c, dt, qkv, B, T, NH, hd, att, lse));
+    RK(gemm(c, dt, GemmDesc{att, C, false, m->W(w.ao_w), C, false, N, C, C, EPI_F32_RESID, xs(2 * l + 1), C, nullptr,
+                            0, w.ao_b, xs(2 * l), C, 0, 1}));
+    RK(LN_F(xs(2 * l + 1), w.ln2_g, w.ln2_b, h2, mean(2 * l + 1), rstd(2 * l + 1)));
+    RK(gemm(c, dt, GemmDesc{h2, C, false, m->W(w.fc_w), C, false, N, F, C, EPI_BF16_GELU, u, F, a, F, w.fc_b, nullptr,
+                            0, 0, 1}));
+    RK(gemm(c, dt, GemmDesc{a, F, false, m->W(w.pj_w), F, false, N, C, F, EPI_F32_RESID, xs(2 * l + 2), C, nullptr, 0,
+                            w.pj_b, xs(2 * l + 1), C, 0, 1}));
+  }
+  RK(LN_F(xs(2 * L), m->lnf_g, m->lnf_b, m->xf, mean(2 * L), rstd(2 * L)));
+
+  // ---------------- head + cross-entropy, chunk by chunk ----------------
+  const float* headw = m->cfg.tied ? m->wte : m->head;
+  float* g_head = m->cfg.tied ? m->g_wte : m->g_head;
+  const int chunk = N < HEAD_CHUNK_ROWS ? N : HEAD_CHUNK_ROWS;
+  for (int r0 = 0; r0 < N; r0 += chunk) {
+    const int rows = (N - r0) < chunk ? (N - r0) : chunk;
+    char* xf_c = m->xf + (int64_t)r0 * C * ab;
+    RK(gemm(c, dt, GemmDesc{xf_c, C, false, m->W(headw), C, false, rows, Vp, C, EPI_BF16, m->logits, Vp, nullptr, 0,
+                            nullptr, nullptr, 0, 0, 1}));
+    RK(cross_entropy(c, dt, m->logits, Vp, rows, m->cfg.V, m->tgt + r0, 1.0f / (float)N, m->row_loss + r0));
+    if (backward) {
+      // dxf = dlogits W ; dW += dlogits^T xf
+      RK(gemm(c, dt, GemmDesc{m->logits, Vp, false, m->W(headw), C, true, rows, C, Vp, EPI_F32, m->dh + (int64_t)r0 * C,
+                              C, nullptr, 0, nullptr, nullptr, 0, 0, 0}));
+      RK(gemm(c, dt, GemmDesc{m->logits, Vp, true, xf_c, C, true, Vp, C, rows, EPI_F32, g_head, C, nullptr, 0, nullptr,
+                              nullptr, 0, 1, 0}));
+    }
+  }
+  sum_rows_kernel<<<1, 1024, 0, m->stream>>>(m->row_loss, N, 1.0f / (float)N, m->d_loss, 0);
+  RK(check_launch(c, "sum_rows"));
+  if (!backward) return GPT2_OK;
+
+  // ---------------- backward ----------------
+  void* dres_act = dt == GPT2_BF16 ? (void*)m->dres_act : (void*)m->dres;
+  auto LN_B = [&](const float* dy, const float* x, const float* gg, float* mu, float* rs, int accumulate, float* dg,
+                  float* db) -> int {
+    const int grid = ln_bwd_grid(N);
+    int r = dt == GPT2_BF16 ? layernorm_bwd_t<bf16>(c, dy, x, gg, mu, rs, N, C, m->dres, (bf16*)m->dres_act,
+                                                    accumulate, m->part)
+                            : layernorm_bwd_t<float>(c, dy, x, gg, mu, rs, N, C, m->dres, (float*)nullptr, accumulate,
+                                                     m->part);
+    if (r) return r;
+    r = reduce_partials(c, m->part, grid, C, dg, 1);
+    if (r) return r;
+    return reduce_partials(c, m->part + (size_t)grid * C, grid, C, db, 1);
+  };
+  auto COLSUM_ACT = [&](const void* y, int ncols, float* out) -> int {
+    return dt == GPT2_BF16 ? colsum_t<bf16>(c, (const bf16*)y, ncols, N, ncols, m->part, out)
+                           : colsum_t<float>(c, (const float*)y, ncols, N, ncols, m->part, out);
+  };
+  RK(LN_B(m->dh, xs(2 * L), m->lnf_g, mean(2 * L), rstd(2 * L), 0, m->g_lnf_g, m->g_lnf_b));
+  for (int l = L - 1; l >= 0; --l) {
+    const LayerP& w = m->lp[l];
+    const LayerP& gw = m->lg[l];
+    void* h1 = ACT(m->h1, l, NC);
+    void* qkv = ACT(m->qkv, l, N3C);
+    void* att = ACT(m->att, l, NC);
+    void* h2 = ACT(m->h2, l, NC);
+    void* u = ACT(m->u, l, NF);
+    void* a = ACT(m->a, l, NF);
+    float* lse = m->lse + l * NLSE;
+    // MLP: x_out = x_mid + pj(gelu(fc(ln2(x_mid))))
+    RK(gemm(c, dt, GemmDesc{dres_act, C, true, a, F, true, C, F, N, EPI_F32, gw.pj_w, F, nullptr, 0, nullptr, nullptr,
+                            0, 1, 0}));
+    RK(colsum_t<float>(c, m->dres, C, N, C, m->part, gw.pj_b));
+    RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.pj_w), F, true, N, F, C, EPI_BF16_DGELU, m->du, F, nullptr, 0,
+                            nullptr, u, F, 0, 1}));
+    RK(gemm(c, dt, GemmDesc{m->du, F, true, h2, C, true, F, C, N, EPI_F32, gw.fc_w, C, nullptr, 0, nullptr, nullptr, 0,
+                            1, 0}));
+    RK(COLSUM_ACT(m->du, F, gw.fc_b));
+    RK(gemm(c, dt, GemmDesc{m->du, F, false, m->W(w.fc_w), C, true, N, C, F, EPI_F32, m->dh, C, nullptr, 0, nullptr,
+                            nullptr, 0, 0, 1}));
+    RK(LN_B(m->dh, xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), 1, gw.ln2_g, gw.ln2_b));
+    // attention: x_mid = x_in + ao(attn(ln1(x_in)))
+    RK(gemm(c, dt, GemmDesc{dres_act, C, true, att, C, true, C, C, N, EPI_F32, gw.ao_w, C, nullptr, 0, nullptr, nullptr,
+                            0, 1, 0}));
+    RK(colsum_t<float>(c, m->dres, C, N, C, m->part, gw.ao_b));
+    RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.ao_w), C, true, N, C, C, EPI_BF16, m->datt, C, nullptr, 0,
+                            nullptr, nullptr, 0, 0, 1}));
+    RK(attention_bwd(c, dt, qkv, att, m->datt, lse, B, T, NH, hd, m->dqkv, m->Dattn));
+    RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, true, h1, C, true, 3 * C, C, N, EPI_F32, gw.qkv_w, C, nullptr, 0, nullptr,
+                            nullptr, 0, 1, 0}));
+    if (gw.qkv_b) RK(COLSUM_ACT(m->dqkv, 3 * C, gw.qkv_b));
+    RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, false, m->W(w.qkv_w), C, true, N, C, 3 * C, EPI_F32, m->dh, C, nullptr, 0,
+                            nullptr, nullptr, 0, 0, 1}));
+    RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b));
+  }
+  EmbScratch es = emb_scratch_carve(m->emb_scratch, N, C);
+  RK(embedding_bwd(c, m->tok, m->dres, B, T, C, m->cfg.V, m->g_wte, m->g_wpe, es));
+  return GPT2_OK;
+}
+
+int validate_batch(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T) {
+  if (!m) return GPT2_ERR_CONFIG;
+  if (!tokens || !targets) return set_err(m, GPT2_ERR_CONFIG, "tokens and targets are required");
+  if (T <= 0 || B <= 0) return set_err(m, GPT2_ERR_CONFIG, "B and T must be positive");
+  if (T > m->cfg.T) return set_err(m, GPT2_ERR_SEQ_TOO_LONG, "sequence length exceeds the block size");
+  if (B > m->cfg.B_max) return set_err(m, GPT2_ERR_BATCH, "B exceeds B_max");
+  return GPT2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
+  if (!out) return GPT2_ERR_CONFIG;
+  *out = nullptr;
+  if (!cfg) return GPT2_ERR_CONFIG;
+  const gpt2_config c = *cfg;
+  if (c.L <= 0 || c.H <= 0 || c.C <= 0 || c.T <= 0 || c.V <= 0 || c.B_max <= 0 || c.C % c.H ||
+      (c.dtype != GPT2_FP32 && c.dtype != GPT2_BF16) || c.C % 64 || c.V > (1 << 17))
+    return GPT2_ERR_CONFIG;
+  const int hd = c.C / c.H;
+  if (c.dtype == GPT2_BF16 && hd != 64) return GPT2_ERR_CONFIG;
+  if (c.dtype == GPT2_FP32 && (hd % 32 || hd > 128)) return GPT2_ERR_CONFIG;
+  if ((int64_t)c.B_max * c.T > EMB_MAX_TOKENS) return GPT2_ERR_BATCH;
+  gpt2* m = new gpt2();
+  m->cfg = c;
+  m->C = c.C;
+  m->F = 4 * c.C;
+  m->NH = c.H;
+  m->hd = hd;
+  m->L = c.L;
+  m->T = c.T;
+  m->Vp = (c.V + 63) / 64 * 64;
+  m->Nmax = c.B_max * c.T;
+  m->act_bytes = c.dtype == GPT2_BF16 ? 2 : 4;
+  m->num_sms = device_sm_count();
+  build_tensors(m);
+  auto bail = [&](int code, const char* what) {
+    std::string msg = what;
+    gpt2_destroy(m);
+    (void)msg;
+    return code;
+  };
+  if (cudaStreamCreateWithFlags(&m->stream, cudaStreamNonBlocking) != cudaSuccess) return bail(GPT2_ERR_CUDA, "stream");
+  m->own_stream = true;
+  const size_t S = (size_t)m->n_store;
+  if (cudaMalloc(&m->p, S * 4) || cudaMalloc(&m->g, S * 4) || cudaMalloc(&m->m, S * 4) || cudaMalloc(&m->v, S * 4))
+    return bail(GPT2_ERR_OOM, "state");
+  if (c.dtype == GPT2_BF16 && cudaMalloc(&m->shadow, (size_t)m->n_decay * 2)) return bail(GPT2_ERR_OOM, "shadow");
+  cudaMemset(m->p, 0, S * 4);
+  cudaMemset(m->g, 0, S * 4);
+  cudaMemset(m->m, 0, S * 4);
+  cudaMemset(m->v, 0, S * 4);
+  // views
+  m->wte = m->P("wte");
+  m->wpe = m->P("wpe");
+  m->lnf_g = m->P("lnf_g");
+  m->lnf_b = m->P("lnf_b");
+  m->head = c.tied ? nullptr : m->P("head_w");
+  m->g_wte = m->G("wte");
+  m->g_wpe = m->G("wpe");
+  m->g_lnf_g = m->G("lnf_g");
+  m->g_lnf_b = m->G("lnf_b");
+  m->g_head = c.tied ? nullptr : m->G("head_w");
+  m->lp.resize(c.L);
+  m->lg.resize(c.L);
+  for (int l = 0; l < c.L; ++l) {
+    const std::string p = "h" + std::to_string(l) + ".";
+    auto fill = [&](LayerP& L, bool grad) {
+      auto X = [&](const char* n) -> float* {
+        if (!m->has(p + n)) return nullptr;
+        return grad ? m->G(p + n) : m->P(p + n);
+      };
+      L = LayerP{X("ln1_g"), X("ln1_b"), X("qkv_w"), X("qkv_b"), X("ao_w"), X("ao_b"),
+                 X("ln2_g"), X("ln2_b"), X("fc_w"),  X("fc_b"),  X("pj_w"), X("pj_b")};
+    };
+    fill(m->lp[l], false);
+    fill(m->lg[l], true);
+  }
+  // activation arena
+  const int64_t N = m->Nmax, C = c.C, F = m->F, L = c.L, ab = m->act_bytes;
+  const int64_t chunk = N < HEAD_CHUNK_ROWS ? N : HEAD_CHUNK_ROWS;
+  int gx, R, rp;
+  colsum_shape((int)N, (int)(3 * C > F ? 3 * C : F), gx, R, rp);
+  const int64_t colsum_floats = (int64_t)(R + 1) * (3 * C > F ? 3 * C : F);
+  // colsum partials never exceed 1184 row chunks x 512 columns per chunk of columns
+  m->part_floats = (size_t)std::max<int64_t>(std::max<int64_t>(2LL * ln_bwd_grid((int)N) * C, colsum_floats),
+                                             1184LL * 512 + 4096);
+  m->splitk_floats = (size_t)std::max<int64_t>(16LL * F * C, 16LL * chunk * C);
+  std::vector<std::pair<void**, size_t>> plan = {
+      {(void**)&m->x, (size_t)(2 * L + 1) * N * C * 4},
+      {(void**)&m->stat_mean, (size_t)(2 * L + 1) * N * 4},
+      {(void**)&m->stat_rstd, (size_t)(2 * L + 1) * N * 4},
+      {(void**)&m->lse, (size_t)L * c.B_max * c.H * c.T * 4},
+      {(void**)&m->h1, (size_t)L * N * C * ab},
+      {(void**)&m->qkv, (size_t)L * N * 3 * C * ab},
+      {(void**)&m->att, (size_t)L * N * C * ab},
+      {(void**)&m->h2, (size_t)L * N * C * ab},
+      {(void**)&m->u, (size_t)L * N * F * ab},
+      {(void**)&m->a, (size_t)L * N * F * ab},
+      {(void**)&m->xf, (size_t)N * C * ab},
+      {(void**)&m->logits, (size_t)chunk * m->Vp * ab},
+      {(void**)&m->dres_act, (size_t)N * C * ab},
+      {(void**)&m->du, (size_t)N * F * ab},
+      {(void**)&m->datt, (size_t)N * C * ab},
+      {(void**)&m->dqkv, (size_t)N * 3 * C * ab},
+      {(void**)&m->dres, (size_t)N * C * 4},
+      {(void**)&m->dh, (size_t)N * C * 4},
+      {(void**)&m->Dattn, (size_t)c.B_max * c.H * c.T * 4},
+      {(void**)&m->row_loss, (size_t)N * 4},
+      {(void**)&m->part, m->part_floats * 4},
+      {(void**)&m->splitk, m->splitk_floats * 4},
+      {(void**)&m->tok, (size_t)N * 4},
+      {(void**)&m->tgt, (size_t)N * 4},
+      {(void**)&m->emb_scratch, emb_scratch_bytes((int)N, (int)C)},
+      {(void**)&m->d_err, 256},
+      {(void**)&m->d_loss, 256},
+      {(void**)&m->d_gnorm, 256},
+  };
+  m->norm_parts = 8 * m->num_sms;
+  plan.push_back({(void**)&m->d_norm_part, (size_t)m->norm_parts * 8});
+  size_t total = 0;
+  for (auto& e : plan) total += (e.second + 255) & ~size_t(255);
+  if (cudaMalloc(&m->arena, total) != cudaSuccess) return bail(GPT2_ERR_OOM, "arena");
+  m->arena_bytes = total;
+  cudaMemset(m->arena, 0, total);
+  size_t off = 0;
+  for (auto& e : plan) {
+    *e.first = m->arena + off;
+    off += (e.second + 255) & ~size_t(255);
+  }
+  std::vector<float> init;
+  host_init(m, seed, init);
+  int r = gpt2_set_params(m, init.data(), m->n_logical);
+  if (r) {
+    gpt2_destroy(m);
+    return r;
+  }
+  *out = m;
+  return GPT2_OK;
+}
+
+int gpt2_set_stream(gpt2* m, void* stream) {
+  if (!m) return GPT2_ERR_CONFIG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (!s) {
+    if (!m->own_stream) {
+      CK(m, cudaStreamCreateWithFlags(&m->stream, cudaStreamNonBlocking));
+      m->own_stream = true;
+    }
+    return GPT2_OK;
+  }
+  if (m->own_stream) {
+    CK(m, cudaStreamSynchronize(m->stream));
+    cudaStreamDestroy(m->stream);
+    m->own_stream = false;
+  }
+  m->stream = s;
+  return GPT2_OK;
+}
+
+int gpt2_forward_backward(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T, float* loss_out) {
+  RK(validate_batch(m, tokens, targets, B, T));
+  if (m->k > 0 && (B != m->k_B || T != m->k_T))
+    return set_err(m, GPT2_ERR_BATCH, "all accumulated micro-batches must have the same B and T");
+  RK(copy_tokens(m, m->tok, tokens, (size_t)B * T));
+  RK(copy_tokens(m, m->tgt, targets, (size_t)B * T));
+  RK(run_micro_batch(m, B, T, true));
+  m->k += 1;
+  m->k_B = B;
+  m->k_T = T;
+  if (loss_out) {
+    CK(m, cudaMemcpyAsync(loss_out, m->d_loss, 4, cudaMemcpyDeviceToHost, m->stream));
+    RK(check_device_error(m));
+  }
+  return GPT2_OK;
+}
+
+int gpt2_forward(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T, float* loss_out) {
+  RK(validate_batch(m, tokens, targets, B, T));
+  RK(copy_tokens(m, m->tok, tokens, (size_t)B * T));
+  RK(copy_tokens(m, m->tgt, targets, (size_t)B * T));
+  RK(run_micro_batch(m, B, T, false));
+  if (loss_out) {
+    CK(m, cudaMemcpyAsync(loss_out, m->d_loss, 4, cudaMemcpyDeviceToHost, m->stream));
+    RK(check_device_error(m));
+  }
+  return GPT2_OK;
+}
+
+int gpt2_step(gpt2* m, float lr, float wd, float beta1, float beta2, float* grad_norm_out) {
+  if (!m) return GPT2_ERR_CONFIG;
+  if (m->k == 0) return set_err(m, GPT2_ERR_NO_GRAD, "step without an accumulated micro-batch");
+  LaunchCtx c = m->ctx();
+  m->t += 1;
+  ProfScope ps(c, CAT_ADAMW, 0.0, (double)m->n_store * 36 + (m->cfg.dtype == GPT2_BF16 ? 2.0 * m->n_decay : 0.0));
+  sumsq_partial_kernel<<<m->norm_parts, ADAM_THREADS, 0, m->stream>>>(m->g, m->n_store, m->d_norm_part);
+  RK(check_launch(c, "sumsq_partial"));
+  AdamArgs a{};
+  a.p = m->p;
+  a.g = m->g;
+  a.m = m->m;
+  a.v = m->v;
+  a.shadow = m->cfg.dtype == GPT2_BF16 ? m->shadow : nullptr;
+  a.n = m->n_store;
+  a.n_decay = m->n_decay;
+  a.partial = m->d_norm_part;
+  a.nparts = m->norm_parts;
+  a.inv_k = 1.0f / (float)m->k;
+  a.lr = lr;
+  a.wd = wd;
+  a.b1 = beta1;
+  a.b2 = beta2;
+  a.step_size = (float)(lr / (1.0 - std::pow((double)beta1, (double)m->t)));
+  a.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(1.0 - std::pow((double)beta2, (double)m->t)));
+  a.gnorm_out = m->d_gnorm;
+  adamw_kernel<<<8 * m->num_sms, ADAM_THREADS, 0, m->stream>>>(a);
+  RK(check_launch(c, "adamw"));
+  m->k = 0;
+  if (grad_norm_out) {
+    CK(m, cudaMemcpyAsync(grad_norm_out, m->d_gnorm, 4, cudaMemcpyDeviceToHost, m->stream));
+    RK(check_device_error(m));
+  }
+  return GPT2_OK;
+}
+
+int gpt2_zero_grad(gpt2* m) {
+  if (!m) return GPT2_ERR_CONFIG;
+  CK(m, cudaMemsetAsync(m->g, 0, (size_t)m->n_store * 4, m->stream));
+  m->k = 0;
+  return GPT2_OK;
+}
+
+int gpt2_num_params(const gpt2* m, int64_t* out) {
+  if (!m || !out) return GPT2_ERR_CONFIG;
+  *out = m->n_logical;
+  return GPT2_OK;
+}
+
+int gpt2_tensor_info(const gpt2* m, int i, char* name, int name_len, int64_t* rows, int64_t* cols, int* ndim,
+                     int64_t* offset) {
+  if (!m || i < 0 || i >= (int)m->tensors.size()) return GPT2_ERR_CONFIG;
+  const TensorSlot& t = m->tensors[i];
+  if (name && name_len > 0) std::snprintf(name, name_len, "%s", t.name.c_str());
+  if (rows) *rows = t.rows;
+  if (cols) *cols = t.cols;
+  if (ndim) *ndim = t.ndim;
+  if (offset) *offset = t.canon_off;
+  return GPT2_OK;
+}
+
+namespace {
+// Copy between canonical host order and device storage for one state buffer.
+int xfer(gpt2* m, float* dev, float* host, const float* host_in, int64_t n, bool to_host, float scale) {
+  if (n != m->n_logical) return set_err(m, GPT2_ERR_CONFIG, "n must equal the logical parameter count");
+  for (auto& t : m->tensors) {
+    const size_t bytes = (size_t)(t.rows * t.cols) * 4;
+    if (to_host)
+      CK(m, cudaMemcpyAsync(host + t.canon_off, dev + t.dev_off, bytes, cudaMemcpyDeviceToHost, m->stream));
+    else
+      CK(m, cudaMemcpyAsync(dev + t.dev_off, host_in + t.canon_off, bytes, cudaMemcpyHostToDevice, m->stream));
+  }
+  CK(m, cudaStreamSynchronize(m->stream));
+  if (to_host && scale != 1.0f)
+    for (int64_t i = 0; i < n; ++i) host[i] *= scale;
+  return GPT2_OK;
+}
+}  // namespace
+
+int gpt2_get_params(gpt2* m, float* host, int64_t n) {
+  if (!m || !host) return GPT2_ERR_CONFIG;
+  RK(xfer(m, m->p, host, nullptr, n, true, 1.0f));
+  return check_device_error(m);
+}
+
+int gpt2_set_params(gpt2* m, const float* host, int64_t n) {
+  if (!m || !host) return GPT2_ERR_CONFIG;
+  RK(xfer(m, m->p, nullptr, host, n, false, 1.0f));
+  if (m->cfg.dtype == GPT2_BF16) {
+    cast_shadow_kernel<<<8 * m->num_sms, 256, 0, m->stream>>>(m->p, m->shadow, m->n_decay);
+    LaunchCtx c = m->ctx();
+    RK(check_launch(c, "cast_shadow"));
+    CK(m, cudaStreamSynchronize(m->stream));
+  }
+  return GPT2_OK;
+}
+
+int gpt2_get_grads(gpt2* m, float* host, int64_t n) {
+  if (!m || !host) return GPT2_ERR_CONFIG;
+  if (m->k == 0) return set_err(m, GPT2_ERR_NO_GRAD, "no accumulated micro-batch");
+  RK(xfer(m, m->g, host, nullptr, n, true, 1.0f / (float)m->k));
+  return check_device_error(m);
+}
+
+int gpt2_get_adam(gpt2* m, float* m_host, float* v_host, int64_t n, int64_t* t_out) {
+  if (!m || !m_host || !v_host) return GPT2_ERR_CONFIG;
+  RK(xfer(m, m->m, m_host, nullptr, n, true, 1.0f));
+  RK(xfer(m, m->v, v_host, nullptr, n, true, 1.0f));
+  if (t_out) *t_out = m->t;
+  return check_device_error(m);
+}
+
+int gpt2_grad_buffer(gpt2* m, float** dev, int64_t* n) {
+  if (!m || !dev || !n) return GPT2_ERR_CONFIG;
+  *dev = m->g;
+  *n = m->n_store;
+  return GPT2_OK;
+}
+
+int gpt2_profile(gpt2* m, int enable) {
+  if (!m) return GPT2_ERR_CONFIG;
+  if (enable) m->prof.reset();
+  m->prof.on = enable != 0;
+  return GPT2_OK;
+}
+
+int gpt2_profile_read(gpt2* m, int cat, char* name, int name_len, double* ms, int64_t* launches, double* flops,
+                      double* bytes) {
+  if (!m || cat < 0 || cat >= CAT_COUNT) return GPT2_ERR_CONFIG;
+  CK(m, cudaStreamSynchronize(m->stream));
+  double t = 0, f = 0, b = 0;
+  int64_t n = 0;
+  for (auto& r : m->prof.recs) {
+    if (r.cat != cat) continue;
+    float e = 0.f;
+    CK(m, cudaEventElapsedTime(&e, r.a, r.b));
+    t += e;
+    f += r.flops;
+    b += r.bytes;
+    ++n;
+  }
+  if (name && name_len > 0) std::snprintf(name, name_len, "%s", prof_cat_name(cat));
+  if (ms) *ms = t;
+  if (launches) *launches = n;
+  if (flops) *flops = f;
+  if (bytes) *bytes = b;
+  return GPT2_OK;
+}
+
+int gpt2_launch_count(const gpt2* m, int64_t* out) {
+  if (!m || !out) return GPT2_ERR_CONFIG;
+  *out = m->launches;
+  return GPT2_OK;
+}
+
+const char* gpt2_last_error(const gpt2* m) { return m ? m->err.c_str() : "null handle"; }
+
+void gpt2_destroy(gpt2* m) {
+  if (!m) return;
+  if (m->stream) cudaStreamSynchronize(m->stream);
+  cudaFree(m->arena);
+  cudaFree(m->p);
+  cudaFree(m->g);
+  cudaFree(m->m);
+  cudaFree(m->v);
+  cudaFree(m->shadow);
+  if (m->own_stream && m->stream) cudaStreamDestroy(m->stream);
+  delete m;
+}
+
+// ---------------------------------------------------------------------------
+// op-level entry points
+// ---------------------------------------------------------------------------
+namespace {
+struct OpCtx {
+  LaunchCtx c;
+  int* d_err = nullptr;
+  cudaStream_t s;
+  explicit OpCtx(void* stream) : s((cudaStream_t)stream) {
+    c.stream = s;
+    c.msg = &g_op_error;
+    c.num_sms = device_sm_count();
+  }
+  int alloc_err() {
+    if (cudaMallocAsync((void**)&d_err, sizeof(int), s) != cudaSuccess) return GPT2_ERR_OOM;
+    cudaMemsetAsync(d_err, 0, sizeof(int), s);
+    c.d_err = d_err;
+    return GPT2_OK;
+  }
+  // synchronise and translate the device error word; frees it
+  int finish() {
+    int h = 0;
+    if (d_err) {
+      cudaMemcpyAsync(&h, d_err, sizeof(int), cudaMemcpyDeviceToHost, s);
+      cudaFreeAsync(d_err, s);
+      d_err = nullptr;
+    }
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+      g_op_error = cudaGetErrorString(e);
+      return GPT2_ERR_CUDA;
+    }
+    if (h == DEV_TOKEN_RANGE) {
+      g_op_error = "token or target id outside [0, V)";
+      return GPT2_ERR_TOKEN_RANGE;
+    }
+    if (h == DEV_TIMEOUT) {
+      g_op_error = "a bounded device-side wait gave up";
+      return GPT2_ERR_TIMEOUT;
+    }
+    return GPT2_OK;
+  }
+};
+}  // namespace
+
+int gpt2_op_gemm(int dtype, const void* A, int64_t lda, int a_mn, const void* B, int64_t ldb, int b_mn, int M, int N,
+                 int K, int epilogue, void* out, int64_t ldo, void* out2, int64_t ldo2, const float* bias,
+                 const void* aux, int64_t ld_aux, int accumulate, int ksplit, void* stream) {
+  OpCtx o(stream);
+  RK(o.alloc_err());
+  float* ws = nullptr;
+  if (dtype == GPT2_BF16 && epilogue == EPI_F32 && ksplit > 1) {
+    const size_t n = (size_t)ksplit * M * N;
+    if (cudaMallocAsync((void**)&ws, n * 4, o.s) != cudaSuccess) return GPT2_ERR_OOM;
+    o.c.splitk_ws = ws;
+    o.c.splitk_cap = n;
+  }
+  int r = gemm(o.c, dtype,
+               GemmDesc{A, lda, a_mn != 0, B, ldb, b_mn != 0, M, N, K, epilogue, out, ldo, out2, ldo2, bias, aux,
+                        ld_aux, accumulate, ksplit <= 0 ? 1 : ksplit});
+  if (ws) cudaFreeAsync(ws, o.s);
+  int r2 = o.finish();
+  return r ? r : r2;
+}
+
+int gpt2_op_layernorm_fwd(int dtype, const float* x, const float* g, const float* b, int N, int C, void* y,
+                          float* mean, float* rstd, void* stream) {
+  OpCtx o(stream);
+  if (C % 4 || C > 2048 || N <= 0) {
+    g_op_error = "layernorm: C % 4 == 0, C <= 2048, N > 0 required";
+    return GPT2_ERR_CONFIG;
+  }
+  return dtype == GPT2_BF16 ? layernorm_fwd_t<bf16>(o.c, x, g, b, N, C, (bf16*)y, mean, rstd)
+                            : layernorm_fwd_t<float>(o.c, x, g, b, N, C, (float*)y, mean, rstd);
+}
+
+int gpt2_op_layernorm_bwd(int dtype, const float* dy, const float* x, const float* g, const float* mean,
+                          const float* rstd, int N, int C, float* dres, void* dres_act, int accumulate, float* dg,
+                          float* db, int accumulate_params, void* stream) {
+  OpCtx o(stream);
+  if (C % 4 || C > 2048 || N <= 0) {
+    g_op_error = "layernorm: C % 4 == 0, C <= 2048, N > 0 required";
+    return GPT2_ERR_CONFIG;
+  }
+  const int grid = ln_bwd_grid(N);
+  float* part = nullptr;
+  if (cudaMallocAsync((void**)&part, (size_t)2 * grid * C * 4, o.s) != cudaSuccess) return GPT2_ERR_OOM;
+  int r = dtype == GPT2_BF16
+              ? layernorm_bwd_t<bf16>(o.c, dy, x, g, mean, rstd, N, C, dres, (bf16*)dres_act, accumulate, part)
+              : layernorm_bwd_t<float>(o.c, dy, x, g, mean, rstd, N, C, dres, (float*)dres_act, accumulate, part);
+  if (!r) r = reduce_partials(o.c, part, grid, C, dg, accumulate_params);
+  if (!r) r = reduce_partials(o.c, part + (size_t)grid * C, grid, C, db, accumulate_params);
+  cudaFreeAsync(part, o.s);
+  return r;
+}
+
+int gpt2_op_attention_fwd(int dtype, const void* qkv, int B, int T, int NH, int hd, void* out, float* lse,
+                          void* stream) {
+  OpCtx o(stream);
+  if (B <= 0 || T <= 0 || NH <= 0) {
+    g_op_error = "attention: empty shape";
+    return GPT2_ERR_CONFIG;
+  }
+  return attention_fwd(o.c, dtype, qkv, B, T, NH, hd, out, lse);
+}
+
+int gpt2_op_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse, int B,
+                          int T, int NH, int hd, void* dqkv, void* stream) {
+  OpCtx o(stream);
+  if (B <= 0 || T <= 0 || NH <= 0) {
+    g_op_error = "attention: empty shape";
+    return GPT2_ERR_CONFIG;
+  }
+  float* D = nullptr;
+  if (cudaMallocAsync((void**)&D, (size_t)B * NH * T * 4, o.s) != cudaSuccess) return GPT2_ERR_OOM;
+  int r = attention_bwd(o.c, dtype, qkv, out, dout, lse, B, T, NH, hd, dqkv, D);
+  cudaFreeAsync(D, o.s);
+  return r;
+}
+
+int gpt2_op_embedding_fwd(const int32_t* tokens, const float* wte, const float* wpe, int B, int T, int C, int V,
+                          float* x0, void* stream) {
+  OpCtx o(stream);
+  RK(o.alloc_err());
+  int r = embedding_fwd(o.c, tokens, wte, wpe, B * T, T, C, V, x0);
+  int r2 = o.finish();
+  return r ? r : r2;
+}
+
+int gpt2_op_token_buckets(const int32_t* tokens, int N, int V, int32_t* sorted_pos, int32_t* seg_id,
+                          int32_t* seg_start, int32_t* nseg_out, void* stream) {
+  OpCtx o(stream);
+  if (N <= 0 || N > EMB_MAX_TOKENS) {
+    g_op_error = "token_buckets: 0 < N <= 32768 required";
+    return GPT2_ERR_BATCH;
+  }
+  RK(o.alloc_err());
+  void* scratch = nullptr;
+  if (cudaMallocAsync(&scratch, emb_scratch_bytes(N, 4), o.s) != cudaSuccess) return GPT2_ERR_OOM;
+  EmbScratch es = emb_scratch_carve(scratch, N, 4);
+  int r = token_sort(o.c, tokens, N, V, es);
+  int counts[2] = {0, 0};
+  std::vector<int> chunk_start, seg_chunk0;
+  if (!r) {
+    cudaMemcpyAsync(counts, es.counts, 8, cudaMemcpyDeviceToHost, o.s);
+    cudaStreamSynchronize(o.s);
+    chunk_start.resize(counts[1] + 1);
+    seg_chunk0.resize(counts[0] + 1);
+    cudaMemcpyAsync(chunk_start.data(), es.chunk_start, (counts[1] + 1) * 4, cudaMemcpyDeviceToHost, o.s);
+    cudaMemcpyAsync(seg_chunk0.data(), es.seg_chunk0, (counts[0] + 1) * 4, cudaMemcpyDeviceToHost, o.s);
+    cudaMemcpyAsync(sorted_pos, es.sorted_pos, (size_t)N * 4, cudaMemcpyDeviceToDevice, o.s);
+    cudaMemcpyAsync(seg_id, es.seg_id, (size_t)counts[0] * 4, cudaMemcpyDeviceToDevice, o.s);
+    cudaStreamSynchronize(o.s);
+    std::vector<int> starts(counts[0] + 1);
+    for (int s = 0; s <= counts[0]; ++s) starts[s] = chunk_start[seg_chunk0[s]];
+    cudaMemcpyAsync(seg_start, starts.data(), (counts[0] + 1) * 4, cudaMemcpyHostToDevice, o.s);
+    if (nseg_out) *nseg_out = counts[0];
+  }
+  cudaFreeAsync(scratch, o.s);
+  int r2 = o.finish();
+  return r ? r : r2;
+}
+
+int gpt2_op_embedding_bwd(const int32_t* tokens, const float* dx0, int B, int T, int C, int V, float* dwte,
+                          float* dwpe, void* stream) {
+  OpCtx o(stream);
+  const int N = B * T;
+  if (N <= 0 || N > EMB_MAX_TOKENS || C % 4) {
+    g_op_error = "embedding_bwd: 0 < B*T <= 32768 and C % 4 == 0 required";
+    return GPT2_ERR_CONFIG;
+  }
+  RK(o.alloc_err());
+  void* scratch = nullptr;
+  if (cudaMallocAsync(&scratch, emb_scratch_bytes(N, C), o.s) != cudaSuccess) return GPT2_ERR_OOM;
+  EmbScratch es = emb_scratch_carve(scratch, N, C);
+  int r = embedding_bwd(o.c, tokens, dx0, B, T, C, V, dwte, dwpe, es);
+  cudaFreeAsync(scratch, o.s);
+  int r2 = o.finish();
+  return r ? r : r2;
+}
+
+int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, const int32_t* targets, float scale,
+                          float* row_loss, void* stream) {
+  OpCtx o(stream);
+  RK(o.alloc_err());
+  int r = cross_entropy(o.c, dtype, logits, ld, N, V, targets, scale, row_loss);
+  int r2 = o.finish();
+  return r ? r : r2;
+}
+
+const char* gpt2_op_last_error(void) { return g_op_error.c_str(); }
+
+}  // extern "C"

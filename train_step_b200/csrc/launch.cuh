@@ -1,0 +1,539 @@
+// launch.cuh -- host-side launchers for the kernels (shape checks, grid sizing,
+// tensor-map encoding). Every launcher returns 0 or a negative GPT2_ERR_* code
+// and writes a message into `msg` on failure.
+#pragma once
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <string>
+#include <vector>
+
+#include "../../include/gpt2.h"
+#include "adamw.cuh"
+#include "attention.cuh"
+#include "common.cuh"
+#include "cross_entropy.cuh"
+#include "embedding.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "layernorm.cuh"
+
+namespace g2 {
+
+// Kernel categories for the per-launch CUDA-event profiler.
+enum ProfCat : int {
+  CAT_GEMM = 0,
+  CAT_SPLITK,
+  CAT_ATTN_FWD,
+  CAT_ATTN_BWD,
+  CAT_LN_FWD,
+  CAT_LN_BWD,
+  CAT_REDUCE,
+  CAT_EMB_FWD,
+  CAT_EMB_BWD,
+  CAT_CE,
+  CAT_ADAMW,
+  CAT_COUNT
+};
+inline const char* prof_cat_name(int c) {
+  static const char* n[CAT_COUNT] = {"gemm_tc",        "splitk_reduce", "attention_fwd", "attention_bwd",
+                                     "layernorm_fwd",  "layernorm_bwd", "reductions",    "embedding_fwd",
+                                     "embedding_bwd",  "cross_entropy", "adamw"};
+  return (c >= 0 && c < CAT_COUNT) ? n[c] : "?";
+}
+
+// Records a start/stop event pair around each profiled launch; totals are read
+// after a synchronisation. Off by default (no events are recorded).
+struct Profiler {
+  bool on = false;
+  struct Rec {
+    int cat;
+    cudaEvent_t a, b;
+    double flops, bytes;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  cudaEvent_t get() {
+    if (used == pool.size()) {
+      cudaEvent_t e;
+      cudaEventCreate(&e);
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+  void begin(cudaStream_t s, int cat, double flops, double bytes) {
+    Rec r{cat, get(), get(), flops, bytes};
+    cudaEventRecord(r.a, s);
+    recs.push_back(r);
+  }
+  void end(cudaStream_t s) { cudaEventRecord(recs.back().b, s); }
+  void reset() {
+    recs.clear();
+    used = 0;
+  }
+  ~Profiler() {
+    for (auto e : pool) cudaEventDestroy(e);
+  }
+};
+
+struct LaunchCtx {
+  Profiler* prof = nullptr;
+  cudaStream_t stream = nullptr;
+  int* d_err = nullptr;           // device error word
+  std::string* msg = nullptr;     // where failures are described
+  long long* launches = nullptr;  // launch counter (nullable)
+  float* splitk_ws = nullptr;     // split-K workspace (nullable: split-K disabled)
+  size_t splitk_cap = 0;          // floats
+  int num_sms = 148;
+};
+
+struct ProfScope {
+  const LaunchCtx& c;
+  bool on;
+  ProfScope(const LaunchCtx& ctx, int cat, double flops, double bytes) : c(ctx), on(ctx.prof && ctx.prof->on) {
+    if (on) c.prof->begin(c.stream, cat, flops, bytes);
+  }
+  ~ProfScope() {
+    if (on) c.prof->end(c.stream);
+  }
+};
+
+inline int fail(const LaunchCtx& c, int code, const std::string& m) {
+  if (c.msg) *c.msg = m;
+  return code;
+}
+
+inline int check_launch(const LaunchCtx& c, const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (c.launches) ++*c.launches;
+  if (e != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return GPT2_OK;
+}
+
+inline int device_sm_count() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors through the driver entry point (no link-time libcuda).
+// ---------------------------------------------------------------------------
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [outer][inner] with row stride ld elements; box {64, box_outer};
+// 128-byte swizzle; out-of-bounds elements read as zero.
+inline bool encode_bf16_map(CUtensorMap* map, const void* ptr, long long inner, long long outer, long long ld,
+                            int box_outer) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM
+// ---------------------------------------------------------------------------
+struct GemmDesc {
+  const void* A;
+  long long lda;
+  bool a_mn;
+  const void* B;
+  long long ldb;
+  bool b_mn;
+  int M, N, K;
+  int epi;
+  void* out;
+  long long ldo;
+  void* out2;
+  long long ldo2;
+  const float* bias;
+  const void* aux;
+  long long ld_aux;
+  int accumulate;
+  int ksplit;  // 0 = choose, 1 = none, > 1 = forced
+};
+
+template <int BN, bool AM, bool BM_, int EPI>
+int launch_tc_inst(const LaunchCtx& c, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p) {
+  auto kern = gemm_tc_kernel<BN, AM, BM_, EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM) != cudaSuccess)
+      return fail(c, GPT2_ERR_CUDA, "cudaFuncSetAttribute(gemm_tc) failed");
+    attr_set = true;
+  }
+  const int grid = p.num_units < c.num_sms ? p.num_units : c.num_sms;
+  kern<<<grid, TC_THREADS, TcCfg<BN>::SMEM, c.stream>>>(ta, tb, p);
+  return check_launch(c, "gemm_tc");
+}
+
+template <int BN, bool AM, bool BM_>
+int launch_tc_epi(const LaunchCtx& c, int epi, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p) {
+  switch (epi) {
+    case EPI_BF16: return launch_tc_inst<BN, AM, BM_, EPI_BF16>(c, ta, tb, p);
+    case EPI_BF16_GELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_GELU>(c, ta, tb, p);
+    case EPI_F32_RESID: return launch_tc_inst<BN, AM, BM_, EPI_F32_RESID>(c, ta, tb, p);
+    case EPI_BF16_DGELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_DGELU>(c, ta, tb, p);
+    case EPI_F32: return launch_tc_inst<BN, AM, BM_, EPI_F32>(c, ta, tb, p);
+  }
+  return fail(c, GPT2_ERR_CONFIG, "gemm: unknown epilogue");
+}
+
+inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
+  if (d.M <= 0 || d.N <= 0 || d.K <= 0) return fail(c, GPT2_ERR_CONFIG, "gemm: empty shape");
+  if (d.a_mn && !d.b_mn) return fail(c, GPT2_ERR_CONFIG, "gemm: MN-major A needs MN-major B");
+  if ((d.lda % 8) || (d.ldb % 8) || (reinterpret_cast<uintptr_t>(d.A) & 15) || (reinterpret_cast<uintptr_t>(d.B) & 15))
+    return fail(c, GPT2_ERR_CONFIG, "gemm: bf16 operands need 16-byte aligned rows");
+  const int BN = d.N >= 256 ? 256 : 128;
+  const int tiles_m = (d.M + TC_BM - 1) / TC_BM, tiles_n = (d.N + BN - 1) / BN;
+  const int num_kb = (d.K + TC_BK - 1) / TC_BK;
+  int ksplit = d.ksplit;
+  if (d.epi != EPI_F32 || !c.splitk_ws) {
+    if (ksplit > 1) return fail(c, GPT2_ERR_CONFIG, "gemm: split-K needs epilogue 4 and a workspace");
+    ksplit = 1;
+  } else if (ksplit == 0) {
+    const int tiles = tiles_m * tiles_n;
+    ksplit = 1;
+    if (tiles < 2 * c.num_sms) {
+      ksplit = (2 * c.num_sms + tiles - 1) / tiles;
+      if (ksplit > num_kb / 4) ksplit = num_kb / 4;
+      if (ksplit > 16) ksplit = 16;
+      if (ksplit < 1) ksplit = 1;
+    }
+  }
+  int kb_per = (num_kb + ksplit - 1) / ksplit;
+  ksplit = (num_kb + kb_per - 1) / kb_per;  // no empty slices
+  if (ksplit > 1 && (size_t)ksplit * d.M * d.N > c.splitk_cap) {
+    ksplit = 1;
+    kb_per = num_kb;
+  }
+  if (ksplit > 1 && (d.N % 4)) return fail(c, GPT2_ERR_CONFIG, "gemm: split-K needs N % 4 == 0");
+  GemmParams p{};
+  p.M = d.M;
+  p.N = d.N;
+  p.K = d.K;
+  p.tiles_m = tiles_m;
+  p.tiles_n = tiles_n;
+  p.ksplit = ksplit;
+  p.kb_per_split = kb_per;
+  p.num_kb = num_kb;
+  p.num_units = tiles_m * tiles_n * ksplit;
+  p.out = d.out;
+  p.ldo = d.ldo;
+  p.out2 = d.out2;
+  p.ldo2 = d.ldo2;
+  p.bias = d.bias;
+  p.aux = d.aux;
+  p.ld_aux = d.ld_aux;
+  p.accumulate = d.accumulate;
+  p.partial = ksplit > 1 ? c.splitk_ws : nullptr;
+  p.err = c.d_err;
+  p.timeout_ns = 4000000000ull;
+  CUtensorMap ta, tb;
+  bool ok = d.a_mn ? encode_bf16_map(&ta, d.A, d.M, d.K, d.lda, 64) : encode_bf16_map(&ta, d.A, d.K, d.M, d.lda, 128);
+  ok = ok && (d.b_mn ? encode_bf16_map(&tb, d.B, d.N, d.K, d.ldb, 64) : encode_bf16_map(&tb, d.B, d.K, d.N, d.ldb, BN));
+  if (!ok) return fail(c, GPT2_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
+  int r;
+  {
+  ProfScope ps(c, CAT_GEMM, 2.0 * d.M * d.N * d.K, 0.0);
+  if (BN == 256) {
+    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<256, false, false>(c, d.epi, ta, tb, p);
+    else if (!d.a_mn) r = launch_tc_epi<256, false, true>(c, d.epi, ta, tb, p);
+    else r = launch_tc_epi<256, true, true>(c, d.epi, ta, tb, p);
+  } else {
+    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<128, false, false>(c, d.epi, ta, tb, p);
+    else if (!d.a_mn) r = launch_tc_epi<128, false, true>(c, d.epi, ta, tb, p);
+    else r = launch_tc_epi<128, true, true>(c, d.epi, ta, tb, p);
+  }
+  }
+  if (r || ksplit == 1) return r;
+  ProfScope ps(c, CAT_SPLITK, 0.0, 4.0 * d.M * d.N * (ksplit + 1 + d.accumulate));
+  const long long n4 = (long long)d.M * (d.N / 4);
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 8LL * c.num_sms) blocks = 8LL * c.num_sms;
+  splitk_reduce_kernel<<<(int)blocks, 256, 0, c.stream>>>(c.splitk_ws, ksplit, d.M, d.N, (float*)d.out, d.ldo,
+                                                           d.accumulate);
+  return check_launch(c, "splitk_reduce");
+}
+
+inline int gemm_simt(const LaunchCtx& c, const GemmDesc& d) {
+  if (d.M <= 0 || d.N <= 0 || d.K <= 0) return fail(c, GPT2_ERR_CONFIG, "gemm: empty shape");
+  SimtGemmArgs a{};
+  a.A = (const float*)d.A;
+  a.lda = d.lda;
+  a.a_mn = d.a_mn;
+  a.B = (const float*)d.B;
+  a.ldb = d.ldb;
+  a.b_mn = d.b_mn;
+  a.M = d.M;
+  a.N = d.N;
+  a.K = d.K;
+  a.ep.out = d.out;
+  a.ep.ldo = d.ldo;
+  a.ep.out2 = d.out2;
+  a.ep.ldo2 = d.ldo2;
+  a.ep.bias = d.bias;
+  a.ep.aux = d.aux;
+  a.ep.ld_aux = d.ld_aux;
+  a.ep.accumulate = d.accumulate;
+  dim3 grid((d.N + 63) / 64, (d.M + 63) / 64);
+  ProfScope ps(c, CAT_GEMM, 2.0 * d.M * d.N * d.K, 0.0);
+  switch (d.epi) {
+    case EPI_BF16: gemm_simt_kernel<EPI_BF16><<<grid, 256, 0, c.stream>>>(a); break;
+    case EPI_BF16_GELU: gemm_simt_kernel<EPI_BF16_GELU><<<grid, 256, 0, c.stream>>>(a); break;
+    case EPI_F32_RESID: gemm_simt_kernel<EPI_F32_RESID><<<grid, 256, 0, c.stream>>>(a); break;
+    case EPI_BF16_DGELU: gemm_simt_kernel<EPI_BF16_DGELU><<<grid, 256, 0, c.stream>>>(a); break;
+    case EPI_F32: gemm_simt_kernel<EPI_F32><<<grid, 256, 0, c.stream>>>(a); break;
+    default: return fail(c, GPT2_ERR_CONFIG, "gemm: unknown epilogue");
+  }
+  return check_launch(c, "gemm_simt");
+}
+
+inline int gemm(const LaunchCtx& c, int dtype, const GemmDesc& d) {
+  return dtype == GPT2_BF16 ? gemm_tc(c, d) : gemm_simt(c, d);
+}
+
+// ---------------------------------------------------------------------------
+// LayerNorm
+// ---------------------------------------------------------------------------
+inline int ln_nv(int C) { return (C + 127) / 128; }
+
+template <class T>
+int layernorm_fwd_t(const LaunchCtx& c, const float* x, const float* g, const float* b, int N, int C, T* y, float* mean,
+                    float* rstd) {
+  const int blocks = (N + LN_WARPS - 1) / LN_WARPS;
+  const int nv = ln_nv(C);
+  ProfScope ps(c, CAT_LN_FWD, 0.0, (double)N * C * (4 + sizeof(T)) + 8.0 * N);
+#define LNF(NV) layernorm_fwd_kernel<T, NV><<<blocks, LN_WARPS * 32, 0, c.stream>>>(x, g, b, y, mean, rstd, N, C)
+  if (nv <= 1) LNF(1);
+  else if (nv <= 2) LNF(2);
+  else if (nv <= 4) LNF(4);
+  else if (nv <= 6) LNF(6);
+  else if (nv <= 8) LNF(8);
+  else if (nv <= 13) LNF(13);
+  else LNF(16);
+#undef LNF
+  return check_launch(c, "layernorm_fwd");
+}
+
+inline int ln_bwd_grid(int N) {
+  int g = (N + LN_WARPS - 1) / LN_WARPS;
+  return g < 592 ? g : 592;
+}
+
+template <class T>
+int layernorm_bwd_t(const LaunchCtx& c, const float* dy, const float* x, const float* g, const float* mean,
+                    const float* rstd, int N, int C, float* dres, T* dres_act, int accumulate, float* part /*2*grid*C*/) {
+  const int grid = ln_bwd_grid(N);
+  const int nv = ln_nv(C);
+  float* pg = part;
+  float* pb = part + (size_t)grid * C;
+  ProfScope ps(c, CAT_LN_BWD, 0.0,
+               (double)N * C * (12 + 4 * accumulate + (dres_act ? sizeof(T) : 0)) + 8.0 * N + 8.0 * grid * C);
+#define LNB(NV)                                                                                                   \
+  layernorm_bwd_kernel<T, NV><<<grid, LN_WARPS * 32, 0, c.stream>>>(dy, x, g, mean, rstd, dres, dres_act, accumulate, \
+                                                                    pg, pb, N, C)
+  if (nv <= 1) LNB(1);
+  else if (nv <= 2) LNB(2);
+  else if (nv <= 4) LNB(4);
+  else if (nv <= 6) LNB(6);
+  else if (nv <= 8) LNB(8);
+  else if (nv <= 13) LNB(13);
+  else LNB(16);
+#undef LNB
+  return check_launch(c, "layernorm_bwd");
+}
+
+inline int reduce_partials(const LaunchCtx& c, const float* part, int P, int ncols, float* out, int accumulate) {
+  ProfScope ps(c, CAT_REDUCE, 0.0, 4.0 * P * ncols + 8.0 * ncols);
+  reduce_partials_kernel<<<(ncols + 255) / 256, 256, 0, c.stream>>>(part, P, ncols, ncols, out, accumulate);
+  return check_launch(c, "reduce_partials");
+}
+
+// column sums of y [N, ncols] into out (+=), through a partial buffer of
+// colsum_rows(N, ncols) x ncols floats
+inline void colsum_shape(int N, int ncols, int& gx, int& R, int& rows_per) {
+  gx = (ncols + 511) / 512;
+  R = 1184 / gx;
+  if (R < 1) R = 1;
+  if (R > N) R = N;
+  rows_per = (N + R - 1) / R;
+  R = (N + rows_per - 1) / rows_per;
+}
+
+template <class T>
+int colsum_t(const LaunchCtx& c, const T* y, long long ld, int N, int ncols, float* part, float* out) {
+  int gx, R, rows_per;
+  colsum_shape(N, ncols, gx, R, rows_per);
+  {
+  ProfScope ps(c, CAT_REDUCE, 0.0, (double)N * ncols * sizeof(T) + 4.0 * R * ncols);
+  colsum_partial_kernel<T><<<dim3(gx, R), 256, 0, c.stream>>>(y, ld, N, ncols, rows_per, part);
+  }
+  int r = check_launch(c, "colsum_partial");
+  if (r) return r;
+  return reduce_partials(c, part, R, ncols, out, 1);
+}
+
+// ---------------------------------------------------------------------------
+// attention
+// ---------------------------------------------------------------------------
+inline int attention_fwd(const LaunchCtx& c, int dtype, const void* qkv, int B, int T, int NH, int hd, void* out,
+                         float* lse) {
+  const float scale = 1.0f / sqrtf((float)hd);
+  ProfScope ps(c, CAT_ATTN_FWD, 4.0 * B * NH * hd * (0.5 * T * (T + 1.0)), 0.0);
+  if (dtype == GPT2_BF16) {
+    if (hd != 64) return fail(c, GPT2_ERR_CONFIG, "attention (bf16): head dim must be 64");
+    dim3 grid((T + 63) / 64, B * NH);
+    attn_fwd_bf16_kernel<<<grid, 128, 0, c.stream>>>((const bf16*)qkv, (bf16*)out, lse, T, NH, scale);
+    return check_launch(c, "attn_fwd_bf16");
+  }
+  if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");
+  const long long warps = (long long)B * NH * T;
+  attn_fwd_f32_kernel<<<(int)((warps * 32 + 255) / 256), 256, 0, c.stream>>>((const float*)qkv, (float*)out, lse, B,
+                                                                             T, NH, hd, scale);
+  return check_launch(c, "attn_fwd_f32");
+}
+
+inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const void* out, const void* dout,
+                         const float* lse, int B, int T, int NH, int hd, void* dqkv, float* Dbuf) {
+  const float scale = 1.0f / sqrtf((float)hd);
+  ProfScope ps(c, CAT_ATTN_BWD, 2.5 * 4.0 * B * NH * hd * (0.5 * T * (T + 1.0)), 0.0);
+  const long long warps = (long long)B * NH * T;
+  const int dblocks = (int)((warps * 32 + 255) / 256);
+  if (dtype == GPT2_BF16) {
+    if (hd != 64) return fail(c, GPT2_ERR_CONFIG, "attention (bf16): head dim must be 64");
+    attn_bwd_dot_kernel<bf16><<<dblocks, 256, 0, c.stream>>>((const bf16*)out, (const bf16*)dout, Dbuf, B, T, NH, hd);
+    int r = check_launch(c, "attn_bwd_dot");
+    if (r) return r;
+    dim3 grid((T + 63) / 64, B * NH);
+    attn_bwd_dkdv_bf16_kernel<<<grid, 128, 0, c.stream>>>((const bf16*)qkv, (const bf16*)dout, lse, Dbuf, (bf16*)dqkv,
+                                                          T, NH, scale);
+    r = check_launch(c, "attn_bwd_dkdv");
+    if (r) return r;
+    attn_bwd_dq_bf16_kernel<<<grid, 128, 0, c.stream>>>((const bf16*)qkv, (const bf16*)dout, lse, Dbuf, (bf16*)dqkv, T,
+                                                        NH, scale);
+    return check_launch(c, "attn_bwd_dq");
+  }
+  if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");
+  attn_bwd_dot_kernel<float><<<dblocks, 256, 0, c.stream>>>((const float*)out, (const float*)dout, Dbuf, B, T, NH, hd);
+  int r = check_launch(c, "attn_bwd_dot");
+  if (r) return r;
+  attn_bwd_dq_f32_kernel<<<dblocks, 256, 0, c.stream>>>((const float*)qkv, (const float*)dout, lse, Dbuf,
+                                                        (float*)dqkv, B, T, NH, hd, scale);
+  r = check_launch(c, "attn_bwd_dq_f32");
+  if (r) return r;
+  attn_bwd_dkdv_f32_kernel<<<dblocks, 256, 0, c.stream>>>((const float*)qkv, (const float*)dout, lse, Dbuf,
+                                                          (float*)dqkv, B, T, NH, hd, scale);
+  return check_launch(c, "attn_bwd_dkdv_f32");
+}
+
+// ---------------------------------------------------------------------------
+// embedding
+// ---------------------------------------------------------------------------
+inline int embedding_fwd(const LaunchCtx& c, const int* tok, const float* wte, const float* wpe, int N, int T, int C,
+                         int V, float* x0) {
+  if (C % 4) return fail(c, GPT2_ERR_CONFIG, "embedding: C % 4 != 0");
+  ProfScope ps(c, CAT_EMB_FWD, 0.0, 12.0 * N * C + 4.0 * N);
+  embed_fwd_kernel<<<(int)(((long long)N * 32 + 255) / 256), 256, 0, c.stream>>>(tok, wte, wpe, x0, N, T, C, V, c.d_err);
+  return check_launch(c, "embed_fwd");
+}
+
+// Scratch for the embedding backward, all device memory.
+struct EmbScratch {
+  int* sorted_pos;   // [N]
+  int* chunk_start;  // [N + 1]
+  int* seg_id;       // [N]
+  int* seg_chunk0;   // [N + 1]
+  int* counts;       // [2]
+  float* partial;    // [N * C]
+};
+inline size_t emb_scratch_bytes(int N, int C) {
+  return (size_t)N * 4 * 4 + 2 * 4 + 64 + (size_t)N * C * 4 + 6 * 256;
+}
+inline EmbScratch emb_scratch_carve(void* base, int N, int C) {
+  auto al = [](uintptr_t x) { return (x + 255) & ~uintptr_t(255); };
+  uintptr_t p = al(reinterpret_cast<uintptr_t>(base));
+  EmbScratch s;
+  s.partial = reinterpret_cast<float*>(p);
+  p = al(p + (size_t)N * C * 4);
+  s.sorted_pos = reinterpret_cast<int*>(p);
+  p = al(p + (size_t)N * 4);
+  s.chunk_start = reinterpret_cast<int*>(p);
+  p = al(p + (size_t)(N + 1) * 4);
+  s.seg_id = reinterpret_cast<int*>(p);
+  p = al(p + (size_t)N * 4);
+  s.seg_chunk0 = reinterpret_cast<int*>(p);
+  p = al(p + (size_t)(N + 1) * 4);
+  s.counts = reinterpret_cast<int*>(p);
+  return s;
+}
+
+inline int token_sort(const LaunchCtx& c, const int* tok, int N, int V, const EmbScratch& s) {
+  if (N > EMB_MAX_TOKENS) return fail(c, GPT2_ERR_BATCH, "embedding backward: B*T must be <= 32768");
+  if (V > (1 << 17)) return fail(c, GPT2_ERR_CONFIG, "embedding backward: V must be <= 131072");
+  int NP = 1;
+  while (NP < N) NP <<= 1;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(token_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, EMB_MAX_TOKENS * 4);
+    attr_set = true;
+  }
+  token_sort_kernel<<<1, EMB_SORT_THREADS, NP * 4, c.stream>>>(tok, N, V, NP, s.sorted_pos, s.chunk_start, s.seg_id,
+                                                              s.seg_chunk0, s.counts, c.d_err);
+  return check_launch(c, "token_sort");
+}
+
+inline int embedding_bwd(const LaunchCtx& c, const int* tok, const float* dx0, int Bsz, int T, int C, int V,
+                         float* dwte, float* dwpe, const EmbScratch& s) {
+  const int N = Bsz * T;
+  if (C % 4) return fail(c, GPT2_ERR_CONFIG, "embedding: C % 4 != 0");
+  ProfScope ps(c, CAT_EMB_BWD, 0.0, 8.0 * N * C + 8.0 * T * C + 4.0 * N);
+  int r = token_sort(c, tok, N, V, s);
+  if (r) return r;
+  const int grid = 8 * c.num_sms;
+  embed_chunk_sum_kernel<<<grid, 128, 0, c.stream>>>(dx0, s.sorted_pos, s.chunk_start, s.counts, C, s.partial);
+  if ((r = check_launch(c, "embed_chunk_sum"))) return r;
+  embed_seg_sum_kernel<<<grid, 128, 0, c.stream>>>(s.partial, s.seg_id, s.seg_chunk0, s.counts, C, dwte);
+  if ((r = check_launch(c, "embed_seg_sum"))) return r;
+  const long long n4 = (long long)T * C / 4;
+  embed_pos_grad_kernel<<<(int)((n4 + 255) / 256), 256, 0, c.stream>>>(dx0, Bsz, T, C, dwpe);
+  return check_launch(c, "embed_pos_grad");
+}
+
+// ---------------------------------------------------------------------------
+// cross-entropy
+// ---------------------------------------------------------------------------
+inline int cross_entropy(const LaunchCtx& c, int dtype, void* logits, long long ld, int N, int V, const int* tgt,
+                         float scale, float* row_loss) {
+  if (N <= 0) return GPT2_OK;
+  ProfScope ps(c, CAT_CE, 0.0, 2.0 * N * ld * (dtype == GPT2_BF16 ? 2 : 4));
+  if (dtype == GPT2_BF16) {
+    if (ld % 8 || ld > (long long)CE_THREADS * CE_MAXVEC * 8)
+      return fail(c, GPT2_ERR_CONFIG, "cross_entropy: ld must be a multiple of 8 and <= 65536");
+    cross_entropy_bf16_kernel<<<N, CE_THREADS, 0, c.stream>>>((bf16*)logits, ld, V, tgt, scale, row_loss, c.d_err);
+  } else {
+    cross_entropy_f32_kernel<<<N, CE_THREADS, 0, c.stream>>>((float*)logits, ld, V, tgt, scale, row_loss, c.d_err);
+  }
+  return check_launch(c, "cross_entropy");
+}
+
+}  // namespace g2

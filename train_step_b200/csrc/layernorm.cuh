@@ -1,0 +1,196 @@
+// layernorm.cuh -- LayerNorm forward/backward, one warp per row, float4 loads,
+// warp-shuffle reductions ("gpt/docs/LLM.md", Transformer Blocks: layer
+// normalization before attention and before the MLP; Output Layer: final LN).
+// y = (x - mean) / sqrt(var + 1e-5) * g + b with the biased variance; mean and
+// 1/sqrt(var + eps) are kept for the backward pass.
+#pragma once
+#include "common.cuh"
+
+namespace g2 {
+
+constexpr int LN_WARPS = 8;  // rows per CTA in the forward kernel
+
+template <class T>
+__device__ __forceinline__ void store4(T* dst, float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ void store4<float>(float* dst, float a, float b, float c, float d) {
+  *reinterpret_cast<float4*>(dst) = make_float4(a, b, c, d);
+}
+template <>
+__device__ __forceinline__ void store4<bf16>(bf16* dst, float a, float b, float c, float d) {
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+}
+
+// x: fp32 [N, C]; y: T [N, C]; mean, rstd: fp32 [N]. C % 4 == 0, C <= 128 * NV.
+template <class T, int NV>
+__global__ void __launch_bounds__(LN_WARPS * 32) layernorm_fwd_kernel(const float* __restrict__ x,
+                                                                      const float* __restrict__ g,
+                                                                      const float* __restrict__ b, T* __restrict__ y,
+                                                                      float* __restrict__ mean,
+                                                                      float* __restrict__ rstd, int N, int C) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * LN_WARPS + warp;
+  if (row >= N) return;
+  const float* xr = x + row * C;
+  float4 v[NV];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (i * 32 + lane) * 4;
+    if (c < C) {
+      v[i] = *reinterpret_cast<const float4*>(xr + c);
+      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    }
+  }
+  const float mu = warp_sum(s) / (float)C;
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (i * 32 + lane) * 4;
+    if (c < C) {
+      float a = v[i].x - mu, bb = v[i].y - mu, cc = v[i].z - mu, d = v[i].w - mu;
+      ss += (a * a + bb * bb) + (cc * cc + d * d);
+    }
+  }
+  const float var = warp_sum(ss) / (float)C;
+  const float rs = 1.0f / sqrtf(var + 1e-5f);
+  T* yr = y + row * C;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (i * 32 + lane) * 4;
+    if (c < C) {
+      float4 gg = __ldg(reinterpret_cast<const float4*>(g + c));
+      float4 bb = __ldg(reinterpret_cast<const float4*>(b + c));
+      store4<T>(yr + c, (v[i].x - mu) * rs * gg.x + bb.x, (v[i].y - mu) * rs * gg.y + bb.y,
+                (v[i].z - mu) * rs * gg.z + bb.z, (v[i].w - mu) * rs * gg.w + bb.w);
+    }
+  }
+  if (lane == 0) {
+    mean[row] = mu;
+    rstd[row] = rs;
+  }
+}
+
+// Backward. With xh = (x - mean) * rstd and dxh = dy * g:
+//   dx = rstd * (dxh - mean(dxh) - xh * mean(dxh * xh))
+// dres (+)= dx (accumulate selects += vs =), dres_act (nullable) gets a copy of
+// the updated dres in the activation type. Per-CTA partial sums of dy*xh and dy
+// go to part_g / part_b [gridDim.x][C]; rows are assigned to CTAs in a fixed
+// pattern, so the reduction order never changes between runs.
+template <class T, int NV>
+__global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
+    const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
+    const float* __restrict__ mean, const float* __restrict__ rstd, float* __restrict__ dres,
+    T* __restrict__ dres_act, int accumulate, float* __restrict__ part_g, float* __restrict__ part_b, int N, int C) {
+  __shared__ float red[LN_WARPS][2][128 * 4];  // per-warp chunk partials, reused per column chunk
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4 ag[NV], ab[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) ag[i] = ab[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long row = (long long)blockIdx.x * LN_WARPS + warp; row < N; row += (long long)gridDim.x * LN_WARPS) {
+    const float mu = mean[row], rs = rstd[row];
+    const float* dyr = dy + row * C;
+    const float* xr = x + row * C;
+    float4 vd[NV], vx[NV];
+    float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = (i * 32 + lane) * 4;
+      if (c < C) {
+        vd[i] = *reinterpret_cast<const float4*>(dyr + c);
+        float4 xx = *reinterpret_cast<const float4*>(xr + c);
+        float4 gg = __ldg(reinterpret_cast<const float4*>(g + c));
+        vx[i] = make_float4((xx.x - mu) * rs, (xx.y - mu) * rs, (xx.z - mu) * rs, (xx.w - mu) * rs);
+        float a = vd[i].x * gg.x, b = vd[i].y * gg.y, cc = vd[i].z * gg.z, d = vd[i].w * gg.w;
+        m1 += (a + b) + (cc + d);
+        m2 += (a * vx[i].x + b * vx[i].y) + (cc * vx[i].z + d * vx[i].w);
+        ag[i].x += vd[i].x * vx[i].x;
+        ag[i].y += vd[i].y * vx[i].y;
+        ag[i].z += vd[i].z * vx[i].z;
+        ag[i].w += vd[i].w * vx[i].w;
+        ab[i].x += vd[i].x;
+        ab[i].y += vd[i].y;
+        ab[i].z += vd[i].z;
+        ab[i].w += vd[i].w;
+      }
+    }
+    m1 = warp_sum(m1) / (float)C;
+    m2 = warp_sum(m2) / (float)C;
+    float* dr = dres + row * C;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c = (i * 32 + lane) * 4;
+      if (c < C) {
+        float4 gg = __ldg(reinterpret_cast<const float4*>(g + c));
+        float4 o = make_float4(rs * (vd[i].x * gg.x - m1 - vx[i].x * m2), rs * (vd[i].y * gg.y - m1 - vx[i].y * m2),
+                               rs * (vd[i].z * gg.z - m1 - vx[i].z * m2), rs * (vd[i].w * gg.w - m1 - vx[i].w * m2));
+        if (accumulate) {
+          float4 r = *reinterpret_cast<const float4*>(dr + c);
+          o.x += r.x;
+          o.y += r.y;
+          o.z += r.z;
+          o.w += r.w;
+        }
+        *reinterpret_cast<float4*>(dr + c) = o;
+        if (dres_act) store4<T>(dres_act + row * C + c, o.x, o.y, o.z, o.w);
+      }
+    }
+  }
+  // reduce the warps' partials in a fixed order, 512 columns at a time
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (i * 32 + lane) * 4;
+    const int chunk = i >> 2;  // 4 vectors of 32 lanes = 512 columns per chunk
+    const int local = c - chunk * 512;
+    if ((i & 3) == 0) __syncthreads();
+    if (c < C) {
+      *reinterpret_cast<float4*>(&red[warp][0][local]) = ag[i];
+      *reinterpret_cast<float4*>(&red[warp][1][local]) = ab[i];
+    }
+    if ((i & 3) == 3 || i == NV - 1) {
+      __syncthreads();
+      for (int k = threadIdx.x; k < 512; k += blockDim.x) {
+        const int col = chunk * 512 + k;
+        if (col < C) {
+          float sg = 0.f, sb = 0.f;
+          for (int w = 0; w < LN_WARPS; ++w) {
+            sg += red[w][0][k];
+            sb += red[w][1][k];
+          }
+          part_g[(long long)blockIdx.x * C + col] = sg;
+          part_b[(long long)blockIdx.x * C + col] = sb;
+        }
+      }
+    }
+  }
+}
+
+// out[c] (+)= sum_{p < P} part[p * ld + c], in order of p (one thread per column).
+__global__ void reduce_partials_kernel(const float* __restrict__ part, int P, int ncols, long long ld,
+                                       float* __restrict__ out, int accumulate) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= ncols) return;
+  float s = 0.f;
+  for (int p = 0; p < P; ++p) s += part[(long long)p * ld + c];
+  out[c] = accumulate ? out[c] + s : s;
+}
+
+// Column sums of an activation matrix y [N, ncols] (row stride ld), stage 1:
+// CTA (bx, by) sums rows [by*rows_per, (by+1)*rows_per) of 2*blockDim.x columns.
+template <class T>
+__global__ void colsum_partial_kernel(const T* __restrict__ y, long long ld, int N, int ncols, int rows_per,
+                                      float* __restrict__ part) {
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 2;
+  if (c >= ncols) return;
+  const int r0 = blockIdx.y * rows_per, r1 = min(N, r0 + rows_per);
+  float s0 = 0.f, s1 = 0.f;
+  for (int r = r0; r < r1; ++r) {
+    const T* p = y + (long long)r * ld + c;
+    s0 += to_f32<T>(p[0]);
+    if (c + 1 < ncols) s1 += to_f32<T>(p[1]);
+  }
+  part[(long long)blockIdx.y * ncols + c] = s0;
+  if (c + 1 < ncols) part[(long long)blockIdx.y * ncols + c + 1] = s1;
+}
+
+}  // namespace g2
