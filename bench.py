@@ -210,7 +210,7 @@ def main():
 
     import torch
     import train_step_b200 as tsb
-    from train_step_b200 import synth
+    from train_step_b200 import dp, synth
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -233,12 +233,12 @@ def main():
     grads = torch.as_tensor(_CudaArray(gptr, glen), device="cuda")
 
     # inputs resident in HBM: this rank's micro-batches (weak scaling by rank)
-    mbs = [synth.micro_batch(B, T, c["V"], index=rank * accum + j) for j in range(accum)]
+    mbs = [synth.micro_batch(B, T, c["V"], index=i) for i in dp.micro_batch_indices(rank, world, accum)]
     dev_in = [(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()) for a, b in mbs]
 
     def allreduce():
         if dist is not None:
-            dist.all_reduce(grads, op=dist.ReduceOp.AVG)
+            dp.allreduce_mean_(grads)
 
     def train_step(inputs, want_outputs=False):
         loss = None
