@@ -226,6 +226,19 @@ int gpt2_op_embedding_bwd(const int32_t* tokens, const float* f32_dx0, int B, in
 int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, const int32_t* targets, float scale,
                           float* f32_row_loss, void* stream);
 
+/* Attention backward that allocates nothing (no counterpart on the pages: an
+ * interface addition for callers whose device memory is wholly owned by their
+ * own allocator or fixed budget, so they may not call cudaMalloc/cudaMallocAsync,
+ * or who cannot pay for an allocation per call). Same arguments and results as
+ * gpt2_op_attention_bwd. Its scratch (B*NH*T floats) is a fixed device array of
+ * 2^20 floats (4 MiB) that every GPU loading the library holds until exit;
+ * B*NH*T > 1,048,576 returns GPT2_ERR_CONFIG with a message. The first call on a
+ * device looks up the array's address and caches it: make that first call before
+ * any stream capture. All calls on a device share the array (each overwrites what
+ * it uses before reading it); calls whose kernels overlap on the GPU race. */
+int gpt2_op_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, const void* dout,
+                                  const float* f32_lse, int B, int T, int NH, int hd, void* dqkv, void* stream);
+
 const char* gpt2_op_last_error(void);
 
 #ifdef __cplusplus

@@ -76,6 +76,8 @@ _SYMBOLS = {
                                ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_op_cross_entropy": ([ct.c_int, ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_void_p, ct.c_float,
                                ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_attention_bwd_noalloc": ([ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int,
+                                       ct.c_int, ct.c_int, ct.c_int, ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_op_last_error": ([], ct.c_char_p),
 }
 
@@ -294,6 +296,13 @@ def attention_fwd(qkv, out, lse, B, T, NH, hd, stream=None):
 def attention_bwd(qkv, out, dout, lse, dqkv, B, T, NH, hd, stream=None):
     _op(lib().gpt2_op_attention_bwd(_dt(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), B, T, NH, hd,
                                     _ptr(dqkv), _stream(stream)))
+
+
+def attention_bwd_noalloc(qkv, out, dout, lse, dqkv, B, T, NH, hd, stream=None):
+    """Attention backward with its scratch in a fixed device array: for callers
+    that may not allocate device memory themselves (see include/gpt2.h)."""
+    _op(lib().gpt2_op_attention_bwd_noalloc(_dt(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), B, T, NH, hd,
+                                            _ptr(dqkv), _stream(stream)))
 
 
 def embedding_fwd(tokens, wte, wpe, x0, stream=None):

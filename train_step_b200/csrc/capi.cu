@@ -3,6 +3,7 @@
 // step, all enqueued on one CUDA stream.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -914,3 +915,67 @@ int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, con
 const char* gpt2_op_last_error(void) { return g_op_error.c_str(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Attention backward without any allocation. Its one scratch buffer (the
+// per-row dot products D = rowsum(dO * O), B*NH*T floats) lives in a fixed
+// file-scope device array instead of memory from cudaMallocAsync, for callers
+// whose device memory is wholly owned by their own allocator or budget and who
+// therefore may not allocate, or who cannot pay for an allocation per call.
+// Every GPU that loads this library holds the array (4 MiB) until the process
+// exits. All calls on a device share it and each call overwrites all of it that
+// it uses before reading it, so nothing has to be cleared; calls whose kernels
+// overlap on the GPU (different streams, no ordering between them) race on it.
+// The first call on each device looks up the array's device address (with that
+// device current) and caches it; make that first call before any stream capture.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr long long kNoAllocAttnRows = 1LL << 20;  // max B*NH*T
+static __device__ __align__(256) float g_noalloc_attn_D[kNoAllocAttnRows];
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 64;
+float* g_noalloc_attn_ptr[kMaxDevices] = {};
+
+int noalloc_attn_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    g_op_error = std::string("cudaGetDevice: ") + cudaGetErrorString(e);
+    return GPT2_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    g_op_error = "attention_bwd_noalloc: device ordinal beyond 63";
+    return GPT2_ERR_CONFIG;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_attn_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_attn_D);
+    if (e != cudaSuccess || !p) {
+      g_op_error = std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e);
+      return GPT2_ERR_CUDA;
+    }
+    g_noalloc_attn_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_attn_ptr[dev];
+  return GPT2_OK;
+}
+}  // namespace
+
+extern "C" int gpt2_op_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, const void* dout,
+                                             const float* lse, int B, int T, int NH, int hd, void* dqkv,
+                                             void* stream) {
+  OpCtx o(stream);
+  if (B <= 0 || T <= 0 || NH <= 0) {
+    g_op_error = "attention: empty shape";
+    return GPT2_ERR_CONFIG;
+  }
+  if ((long long)B * NH * T > kNoAllocAttnRows) {
+    g_op_error = "attention_bwd_noalloc: B*NH*T = " + std::to_string((long long)B * NH * T) +
+                 " exceeds the fixed scratch of " + std::to_string(kNoAllocAttnRows) + " rows";
+    return GPT2_ERR_CONFIG;
+  }
+  float* D = nullptr;
+  RK(noalloc_attn_scratch(&D));
+  return attention_bwd(o.c, dtype, qkv, out, dout, lse, B, T, NH, hd, dqkv, D);
+}
