@@ -220,8 +220,9 @@ int gpt2_op_token_buckets(const int32_t* tokens, int N, int V, int32_t* sorted_p
 int gpt2_op_embedding_bwd(const int32_t* tokens, const float* f32_dx0, int B, int T, int C, int V, float* f32_dwte,
                           float* f32_dwpe, void* stream);
 
-/* Cross-entropy over rows of logits(act) [N, ld] (first V columns; ld % 8 == 0,
- * ld <= 65536): f32_row_loss[n] = logsumexp - z[target]; logits overwritten by
+/* Cross-entropy over rows of logits(act) [N, ld] (first V columns; bf16 needs
+ * ld % 8 == 0 and ld <= 56320, two rows fit in one SM's shared memory):
+ * f32_row_loss[n] = logsumexp - z[target]; logits overwritten by
  * (softmax - onehot) * scale (padding columns set to 0). */
 int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, const int32_t* targets, float scale,
                           float* f32_row_loss, void* stream);

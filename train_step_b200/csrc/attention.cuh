@@ -253,6 +253,31 @@ __global__ void attn_bwd_dot_kernel(const T* __restrict__ out, const T* __restri
   }
 }
 
+// bf16, hd = 64: one thread per (row, head), 128-byte vector loads of O and dO.
+__global__ void attn_bwd_dot64_bf16_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
+                                           float* __restrict__ D, int Bsz, int Tn, int NH) {
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= (long long)Bsz * Tn * NH) return;
+  const int h = (int)(i % NH);
+  const long long row = i / NH;
+  const long long off = row * NH * 64 + h * 64;
+  const uint4* o = reinterpret_cast<const uint4*>(out + off);
+  const uint4* d = reinterpret_cast<const uint4*>(dout + off);
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint4 a = o[k], b = d[k];
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 fa = unpack_bf16x2(wa[q]), fb = unpack_bf16x2(wb[q]);
+      s += fa.x * fb.x + fa.y * fb.y;
+    }
+  }
+  const int b = (int)(row / Tn), t = (int)(row % Tn);
+  D[((long long)b * NH + h) * Tn + t] = s;
+}
+
 // dK, dV for one block of 64 keys; loops over query blocks qb >= kb.
 __global__ void __launch_bounds__(128) attn_bwd_dkdv_bf16_kernel(const bf16* __restrict__ qkv,
                                                                  const bf16* __restrict__ dout,

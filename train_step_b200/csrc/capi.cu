@@ -303,23 +303,20 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
 
   // ---------------- backward ----------------
   void* dres_act = dt == GPT2_BF16 ? (void*)m->dres_act : (void*)m->dres;
+  // LN backward; its column sums of the new dres are the bias gradient of the
+  // linear layer that produced this residual (dbias_next, nullable)
   auto LN_B = [&](const float* dy, const float* x, const float* gg, float* mu, float* rs, int accumulate, float* dg,
-                  float* db) -> int {
-    const int grid = ln_bwd_grid(N);
-    int r = dt == GPT2_BF16 ? layernorm_bwd_t<bf16>(c, dy, x, gg, mu, rs, N, C, m->dres, (bf16*)m->dres_act,
-                                                    accumulate, m->part)
-                            : layernorm_bwd_t<float>(c, dy, x, gg, mu, rs, N, C, m->dres, (float*)nullptr, accumulate,
-                                                     m->part);
-    if (r) return r;
-    r = reduce_partials(c, m->part, grid, C, dg, 1);
-    if (r) return r;
-    return reduce_partials(c, m->part + (size_t)grid * C, grid, C, db, 1);
+                  float* db, float* dbias_next) -> int {
+    return dt == GPT2_BF16 ? layernorm_bwd_t<bf16>(c, dy, x, gg, mu, rs, N, C, m->dres, (bf16*)m->dres_act,
+                                                   accumulate, m->part, dg, db, dbias_next, 1)
+                           : layernorm_bwd_t<float>(c, dy, x, gg, mu, rs, N, C, m->dres, (float*)nullptr, accumulate,
+                                                    m->part, dg, db, dbias_next, 1);
   };
   auto COLSUM_ACT = [&](const void* y, int ncols, float* out) -> int {
     return dt == GPT2_BF16 ? colsum_t<bf16>(c, (const bf16*)y, ncols, N, ncols, m->part, out)
                            : colsum_t<float>(c, (const float*)y, ncols, N, ncols, m->part, out);
   };
-  RK(LN_B(m->dh, xs(2 * L), m->lnf_g, mean(2 * L), rstd(2 * L), 0, m->g_lnf_g, m->g_lnf_b));
+  RK(LN_B(m->dh, xs(2 * L), m->lnf_g, mean(2 * L), rstd(2 * L), 0, m->g_lnf_g, m->g_lnf_b, m->lg[L - 1].pj_b));
   for (int l = L - 1; l >= 0; --l) {
     const LayerP& w = m->lp[l];
     const LayerP& gw = m->lg[l];
@@ -333,7 +330,6 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     // MLP: x_out = x_mid + pj(gelu(fc(ln2(x_mid))))
     RK(gemm(c, dt, GemmDesc{dres_act, C, true, a, F, true, C, F, N, EPI_F32, gw.pj_w, F, nullptr, 0, nullptr, nullptr,
                             0, 1, 0}));
-    RK(colsum_t<float>(c, m->dres, C, N, C, m->part, gw.pj_b));
     RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.pj_w), F, true, N, F, C, EPI_BF16_DGELU, m->du, F, nullptr, 0,
                             nullptr, u, F, 0, 1}));
     RK(gemm(c, dt, GemmDesc{m->du, F, true, h2, C, true, F, C, N, EPI_F32, gw.fc_w, C, nullptr, 0, nullptr, nullptr, 0,
@@ -341,11 +337,10 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     RK(COLSUM_ACT(m->du, F, gw.fc_b));
     RK(gemm(c, dt, GemmDesc{m->du, F, false, m->W(w.fc_w), C, true, N, C, F, EPI_F32, m->dh, C, nullptr, 0, nullptr,
                             nullptr, 0, 0, 1}));
-    RK(LN_B(m->dh, xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), 1, gw.ln2_g, gw.ln2_b));
+    RK(LN_B(m->dh, xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), 1, gw.ln2_g, gw.ln2_b, gw.ao_b));
     // attention: x_mid = x_in + ao(attn(ln1(x_in)))
     RK(gemm(c, dt, GemmDesc{dres_act, C, true, att, C, true, C, C, N, EPI_F32, gw.ao_w, C, nullptr, 0, nullptr, nullptr,
                             0, 1, 0}));
-    RK(colsum_t<float>(c, m->dres, C, N, C, m->part, gw.ao_b));
     RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.ao_w), C, true, N, C, C, EPI_BF16, m->datt, C, nullptr, 0,
                             nullptr, nullptr, 0, 0, 1}));
     RK(attention_bwd(c, dt, qkv, att, m->datt, lse, B, T, NH, hd, m->dqkv, m->Dattn));
@@ -354,7 +349,8 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     if (gw.qkv_b) RK(COLSUM_ACT(m->dqkv, 3 * C, gw.qkv_b));
     RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, false, m->W(w.qkv_w), C, true, N, C, 3 * C, EPI_F32, m->dh, C, nullptr, 0,
                             nullptr, nullptr, 0, 0, 1}));
-    RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b));
+    RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b,
+            l > 0 ? m->lg[l - 1].pj_b : nullptr));
   }
   EmbScratch es = emb_scratch_carve(m->emb_scratch, N, C);
   RK(embedding_bwd(c, m->tok, m->dres, B, T, C, m->cfg.V, m->g_wte, m->g_wpe, es));
@@ -447,9 +443,9 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
   int gx, R, rp;
   colsum_shape((int)N, (int)(3 * C > F ? 3 * C : F), gx, R, rp);
   const int64_t colsum_floats = (int64_t)(R + 1) * (3 * C > F ? 3 * C : F);
-  // colsum partials never exceed 1184 row chunks x 512 columns per chunk of columns
-  m->part_floats = (size_t)std::max<int64_t>(std::max<int64_t>(2LL * ln_bwd_grid((int)N) * C, colsum_floats),
-                                             1184LL * 512 + 4096);
+  // colsum partials never exceed 1184 row chunks x 2048 columns per chunk of columns
+  m->part_floats = (size_t)std::max<int64_t>(std::max<int64_t>(3LL * ln_bwd_grid((int)N) * C, colsum_floats),
+                                             1184LL * 2048 + 4096);
   m->splitk_floats = (size_t)std::max<int64_t>(16LL * F * C, 16LL * chunk * C);
   std::vector<std::pair<void**, size_t>> plan = {
       {(void**)&m->x, (size_t)(2 * L + 1) * N * C * 4},
@@ -808,12 +804,12 @@ int gpt2_op_layernorm_bwd(int dtype, const float* dy, const float* x, const floa
   }
   const int grid = ln_bwd_grid(N);
   float* part = nullptr;
-  if (cudaMallocAsync((void**)&part, (size_t)2 * grid * C * 4, o.s) != cudaSuccess) return GPT2_ERR_OOM;
+  if (cudaMallocAsync((void**)&part, (size_t)3 * grid * C * 4, o.s) != cudaSuccess) return GPT2_ERR_OOM;
   int r = dtype == GPT2_BF16
-              ? layernorm_bwd_t<bf16>(o.c, dy, x, g, mean, rstd, N, C, dres, (bf16*)dres_act, accumulate, part)
-              : layernorm_bwd_t<float>(o.c, dy, x, g, mean, rstd, N, C, dres, (float*)dres_act, accumulate, part);
-  if (!r) r = reduce_partials(o.c, part, grid, C, dg, accumulate_params);
-  if (!r) r = reduce_partials(o.c, part + (size_t)grid * C, grid, C, db, accumulate_params);
+              ? layernorm_bwd_t<bf16>(o.c, dy, x, g, mean, rstd, N, C, dres, (bf16*)dres_act, accumulate, part, dg, db,
+                                      nullptr, accumulate_params)
+              : layernorm_bwd_t<float>(o.c, dy, x, g, mean, rstd, N, C, dres, (float*)dres_act, accumulate, part, dg,
+                                       db, nullptr, accumulate_params);
   cudaFreeAsync(part, o.s);
   return r;
 }

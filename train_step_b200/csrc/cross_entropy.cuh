@@ -5,15 +5,14 @@
 // For each row n: lse = logsumexp over the first V columns (padding columns V..ld
 // are storage only); row_loss[n] = lse - z[target]; then
 //   z[v] <- (exp(z[v] - lse) - [v == target]) * scale  for v < V,  0 for v >= V.
-// One CTA of CE_THREADS threads per row; the row stays in registers between the
-// statistics pass and the write pass, so HBM sees one read and one write.
+// HBM sees each logit once in and once out.
 #pragma once
 #include "common.cuh"
 
 namespace g2 {
 
 constexpr int CE_THREADS = 512;
-constexpr int CE_MAXVEC = 16;  // per thread: 16 x 8 bf16 -> rows up to 65536 columns
+constexpr float LOG2E_CE = 1.4426950408889634f;
 
 __device__ __forceinline__ float block_reduce_ce(float v, bool is_max, float* buf) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -26,27 +25,64 @@ __device__ __forceinline__ float block_reduce_ce(float v, bool is_max, float* bu
   return r;
 }
 
-__global__ void __launch_bounds__(CE_THREADS) cross_entropy_bf16_kernel(bf16* __restrict__ logits, long long ld, int V,
-                                                                        const int* __restrict__ tgt, float scale,
-                                                                        float* __restrict__ row_loss, int* err) {
-  __shared__ float buf[CE_THREADS / 32];
-  const long long row = blockIdx.x;
-  bf16* z = logits + row * ld;
-  int t = tgt[row];
-  if (t < 0 || t >= V) {
-    if (threadIdx.x == 0) raise_device_error(err, DEV_TOKEN_RANGE);
-    t = 0;
-  }
-  const float zt = __bfloat162float(z[t]);
+// bf16: persistent, one CTA per SM, rows r = blockIdx.x + k * gridDim.x. Two
+// shared-memory row buffers: row k+1 arrives by a 1-D bulk copy while row k is
+// processed; the result row leaves by a bulk store from the same buffer. HBM sees
+// each logit once in and once out. ld * 2 bytes per buffer (ld % 8 == 0).
+constexpr int CE_PERSIST_THREADS = 512;
+__global__ void __launch_bounds__(CE_PERSIST_THREADS, 1) cross_entropy_bf16_kernel(
+    bf16* __restrict__ logits, long long ld, int V, int rows, const int* __restrict__ tgt, float scale,
+    float* __restrict__ row_loss, int* err, unsigned long long timeout_ns) {
+  extern __shared__ __align__(128) uint8_t ce_smem[];
+  __shared__ float red[CE_PERSIST_THREADS / 32];
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ int s_abort;
+  const uint32_t row_bytes = (uint32_t)(ld * 2);
+  bf16* buf[2] = {reinterpret_cast<bf16*>(ce_smem), reinterpret_cast<bf16*>(ce_smem + row_bytes)};
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nvec = (int)(ld / 8);
-  uint4 r[CE_MAXVEC];
-  float mx = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < CE_MAXVEC; ++i) {
-    const int vi = threadIdx.x + i * CE_THREADS;
-    if (vi < nvec) {
-      r[i] = *reinterpret_cast<const uint4*>(z + (long long)vi * 8);
-      const uint32_t w[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  int row = blockIdx.x;
+  if (tid == 0 && row < rows) {
+    mbar_arrive_expect_tx(&bar[0], row_bytes);
+    bulk_load_1d(buf[0], logits + (long long)row * ld, row_bytes, &bar[0]);
+  }
+  for (int k = 0; row < rows; ++k, row += gridDim.x) {
+    const int cur = k & 1;
+    const int nxt_row = row + gridDim.x;
+    if (tid == 0 && nxt_row < rows) {
+      bulk_wait_read<0>();  // the previous store out of buf[cur ^ 1] has been read
+      mbar_arrive_expect_tx(&bar[cur ^ 1], row_bytes);
+      bulk_load_1d(buf[cur ^ 1], logits + (long long)nxt_row * ld, row_bytes, &bar[cur ^ 1]);
+    }
+    if (tid == 0) {
+      int never = 0;
+      if (!mbar_wait_bounded(&bar[cur], (k >> 1) & 1, reinterpret_cast<volatile int*>(&never), timeout_ns)) {
+        raise_device_error(err, DEV_TIMEOUT);
+        s_abort = 1;
+      }
+    }
+    __syncthreads();
+    if (s_abort) break;
+    // every thread waits on the barrier's phase too, so the async-proxy writes are visible
+    mbar_try_wait(&bar[cur], (k >> 1) & 1);
+    bf16* z = buf[cur];
+    int t = tgt[row];
+    if (t < 0 || t >= V) {
+      if (tid == 0) raise_device_error(err, DEV_TOKEN_RANGE);
+      t = 0;
+    }
+    const float zt = __bfloat162float(z[t]);
+    float mx = -INFINITY;
+    for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
+      const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 f = unpack_bf16x2(w[q]);
@@ -55,43 +91,57 @@ __global__ void __launch_bounds__(CE_THREADS) cross_entropy_bf16_kernel(bf16* __
         if (c + 1 < V) mx = fmaxf(mx, f.y);
       }
     }
-  }
-  mx = block_reduce_ce(mx, true, buf);
-  float se = 0.f;
+    mx = warp_max(mx);
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    mx = red[0];
 #pragma unroll
-  for (int i = 0; i < CE_MAXVEC; ++i) {
-    const int vi = threadIdx.x + i * CE_THREADS;
-    if (vi < nvec) {
-      const uint32_t w[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
+    for (int w = 1; w < CE_PERSIST_THREADS / 32; ++w) mx = fmaxf(mx, red[w]);
+    __syncthreads();
+    const float ml2 = mx * LOG2E_CE;
+    float se = 0.f;
+    for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
+      const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 f = unpack_bf16x2(w[q]);
         const int c = vi * 8 + 2 * q;
-        if (c < V) se += __expf(f.x - mx);
-        if (c + 1 < V) se += __expf(f.y - mx);
+        if (c < V) se += exp2f(f.x * LOG2E_CE - ml2);
+        if (c + 1 < V) se += exp2f(f.y * LOG2E_CE - ml2);
       }
     }
-  }
-  se = block_reduce_ce(se, false, buf);
-  const float lse = mx + __logf(se);
-  if (threadIdx.x == 0) row_loss[row] = lse - zt;
+    se = warp_sum(se);
+    if (lane == 0) red[warp] = se;
+    __syncthreads();
+    se = 0.f;
 #pragma unroll
-  for (int i = 0; i < CE_MAXVEC; ++i) {
-    const int vi = threadIdx.x + i * CE_THREADS;
-    if (vi < nvec) {
-      const uint32_t w[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
+    for (int w = 0; w < CE_PERSIST_THREADS / 32; ++w) se += red[w];
+    const float lse = mx + __logf(se);
+    const float ll2 = lse * LOG2E_CE;
+    if (tid == 0) row_loss[row] = lse - zt;
+    for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
+      const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
       uint32_t o[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 f = unpack_bf16x2(w[q]);
         const int c = vi * 8 + 2 * q;
-        float a = c < V ? (__expf(f.x - lse) - (c == t ? 1.f : 0.f)) * scale : 0.f;
-        float b = c + 1 < V ? (__expf(f.y - lse) - (c + 1 == t ? 1.f : 0.f)) * scale : 0.f;
+        const float a = c < V ? (exp2f(f.x * LOG2E_CE - ll2) - (c == t ? 1.f : 0.f)) * scale : 0.f;
+        const float b = c + 1 < V ? (exp2f(f.y * LOG2E_CE - ll2) - (c + 1 == t ? 1.f : 0.f)) * scale : 0.f;
         o[q] = pack_bf16x2(a, b);
       }
-      *reinterpret_cast<uint4*>(z + (long long)vi * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<uint4*>(z)[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_store_1d(logits + (long long)row * ld, z, row_bytes);
+      bulk_commit();
     }
   }
+  if (tid == 0) bulk_wait_all();
 }
 
 // fp32 parity mode: exact expf/logf, one CTA per row, strided (rows are short).

@@ -62,7 +62,8 @@ struct TcCfg {
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = (192 * 1024) / STAGE;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr int STAGING = TC_EPI_WARPS * 4096;  // one 4 KB store buffer per epilogue warp
+  static constexpr int SMEM = STAGES * STAGE + STAGING + 1024 + 256;
 };
 
 __device__ __forceinline__ float gelu_tanh_fast(float u) {
@@ -81,22 +82,37 @@ __device__ __forceinline__ float gelu_tanh_grad_fast(float u) {
   return 0.5f * (1.0f + th) + 0.5f * u * (1.0f - th * th) * dinner;
 }
 
-// Apply the epilogue to 32 consecutive columns [col0, col0+32) of one row.
+// Output tile of one epilogue warp and chunk: 32 rows (one per lane) x 32 columns,
+// staged in shared memory in the layout of the output tensor map's box:
+//   bf16: 64-byte rows, 64-byte swizzle (16-byte chunk k of row r at chunk k ^ ((r >> 1) & 3))
+//   fp32: 128-byte rows, 128-byte swizzle (chunk k of row r at chunk k ^ (r & 7))
+// Both patterns put the 8 lanes of a 16-byte store phase in distinct banks.
+__device__ __forceinline__ void stage_bf16_row(uint8_t* buf, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int j = k * 8;
+    uint4 w = make_uint4(pack_bf16x2(v[j], v[j + 1]), pack_bf16x2(v[j + 2], v[j + 3]), pack_bf16x2(v[j + 4], v[j + 5]),
+                         pack_bf16x2(v[j + 6], v[j + 7]));
+    *reinterpret_cast<uint4*>(buf + r * 64 + ((k ^ ((r >> 1) & 3)) << 4)) = w;
+  }
+}
+__device__ __forceinline__ void stage_f32_row(uint8_t* buf, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    *reinterpret_cast<float4*>(buf + r * 128 + ((k ^ (r & 7)) << 4)) =
+        make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+}
+
+// Epilogue math on 32 consecutive columns [col0, col0+32) of one row, written into
+// the staging buffer(s) (row `lane`). Columns past N hold don't-care values: the
+// tensor-map store clips them.
 template <int EPI>
-__device__ __forceinline__ void tc_epilogue_row(const GemmParams& p, int split, int row, int col0,
-                                                const uint32_t (&r)[32]) {
-  float v[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+__device__ __forceinline__ void tc_epilogue_stage(const GemmParams& p, int row, int col0, int lane, float (&v)[32],
+                                                  uint8_t* buf) {
   const bool full = (col0 + 32 <= p.N);
-  if (p.ksplit > 1) {  // split-K partial, reduced later in a fixed order
-    float* dst = p.partial + ((long long)split * p.M + row) * (long long)p.N + col0;
-    if (full) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-    } else {
-      for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst[j] = v[j];
-    }
+  const bool row_ok = row < p.M;
+  if (p.ksplit > 1 || EPI == EPI_F32) {
+    stage_f32_row(buf, lane, v);
     return;
   }
   if (EPI == EPI_BF16 || EPI == EPI_BF16_GELU || EPI == EPI_F32_RESID) {
@@ -111,85 +127,60 @@ __device__ __forceinline__ void tc_epilogue_row(const GemmParams& p, int split, 
           v[j + 3] += b.w;
         }
       } else {
-        for (int j = 0; j < 32 && col0 + j < p.N; ++j) v[j] += p.bias[col0 + j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < p.N) v[j] += p.bias[col0 + j];
       }
     }
   }
-  if (EPI == EPI_BF16 || EPI == EPI_BF16_GELU) {
-    bf16* dst = reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + col0;
-    if (full) {
+  if (EPI == EPI_BF16) {
+    stage_bf16_row(buf, lane, v);
+  } else if (EPI == EPI_BF16_GELU) {
+    stage_bf16_row(buf, lane, v);
 #pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        uint4 w = make_uint4(pack_bf16x2(v[j], v[j + 1]), pack_bf16x2(v[j + 2], v[j + 3]),
-                             pack_bf16x2(v[j + 4], v[j + 5]), pack_bf16x2(v[j + 6], v[j + 7]));
-        *reinterpret_cast<uint4*>(dst + j) = w;
+    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
+    stage_bf16_row(buf + 2048, lane, v);
+  } else if (EPI == EPI_F32_RESID) {
+    if (row_ok) {
+      const float* res = reinterpret_cast<const float*>(p.aux) + (long long)row * p.ld_aux + col0;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          float4 x = *reinterpret_cast<const float4*>(res + j);
+          v[j] += x.x;
+          v[j + 1] += x.y;
+          v[j + 2] += x.z;
+          v[j + 3] += x.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < p.N) v[j] += res[j];
       }
-    } else {
-      for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst[j] = __float2bfloat16_rn(v[j]);
     }
-    if (EPI == EPI_BF16_GELU) {
-      bf16* dst2 = reinterpret_cast<bf16*>(p.out2) + (long long)row * p.ldo2 + col0;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
+    stage_f32_row(buf, lane, v);
+  } else if (EPI == EPI_BF16_DGELU) {
+    if (row_ok) {
+      const bf16* u = reinterpret_cast<const bf16*>(p.aux) + (long long)row * p.ld_aux + col0;
       if (full) {
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
-          uint4 w = make_uint4(pack_bf16x2(v[j], v[j + 1]), pack_bf16x2(v[j + 2], v[j + 3]),
-                               pack_bf16x2(v[j + 4], v[j + 5]), pack_bf16x2(v[j + 6], v[j + 7]));
-          *reinterpret_cast<uint4*>(dst2 + j) = w;
+          uint4 uu = *reinterpret_cast<const uint4*>(u + j);
+          const uint32_t w[4] = {uu.x, uu.y, uu.z, uu.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = unpack_bf16x2(w[q]);
+            v[j + 2 * q] *= gelu_tanh_grad_fast(f.x);
+            v[j + 2 * q + 1] *= gelu_tanh_grad_fast(f.y);
+          }
         }
       } else {
-        for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst2[j] = __float2bfloat16_rn(v[j]);
-      }
-    }
-  } else if (EPI == EPI_F32_RESID) {
-    const float* res = reinterpret_cast<const float*>(p.aux) + (long long)row * p.ld_aux + col0;
-    float* dst = reinterpret_cast<float*>(p.out) + (long long)row * p.ldo + col0;
-    if (full) {
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        float4 x = *reinterpret_cast<const float4*>(res + j);
-        *reinterpret_cast<float4*>(dst + j) = make_float4(x.x + v[j], x.y + v[j + 1], x.z + v[j + 2], x.w + v[j + 3]);
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < p.N) v[j] *= gelu_tanh_grad_fast(__bfloat162float(u[j]));
       }
-    } else {
-      for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst[j] = res[j] + v[j];
     }
-  } else if (EPI == EPI_BF16_DGELU) {
-    const bf16* u = reinterpret_cast<const bf16*>(p.aux) + (long long)row * p.ld_aux + col0;
-    bf16* dst = reinterpret_cast<bf16*>(p.out) + (long long)row * p.ldo + col0;
-    if (full) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        uint4 uu = *reinterpret_cast<const uint4*>(u + j);
-        float2 u0 = unpack_bf16x2(uu.x), u1 = unpack_bf16x2(uu.y), u2 = unpack_bf16x2(uu.z), u3 = unpack_bf16x2(uu.w);
-        uint4 w = make_uint4(pack_bf16x2(v[j] * gelu_tanh_grad_fast(u0.x), v[j + 1] * gelu_tanh_grad_fast(u0.y)),
-                             pack_bf16x2(v[j + 2] * gelu_tanh_grad_fast(u1.x), v[j + 3] * gelu_tanh_grad_fast(u1.y)),
-                             pack_bf16x2(v[j + 4] * gelu_tanh_grad_fast(u2.x), v[j + 5] * gelu_tanh_grad_fast(u2.y)),
-                             pack_bf16x2(v[j + 6] * gelu_tanh_grad_fast(u3.x), v[j + 7] * gelu_tanh_grad_fast(u3.y)));
-        *reinterpret_cast<uint4*>(dst + j) = w;
-      }
-    } else {
-      for (int j = 0; j < 32 && col0 + j < p.N; ++j)
-        dst[j] = __float2bfloat16_rn(v[j] * gelu_tanh_grad_fast(__bfloat162float(u[j])));
-    }
-  } else {  // EPI_F32
-    float* dst = reinterpret_cast<float*>(p.out) + (long long)row * p.ldo + col0;
-    if (full) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        float4 o = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        if (p.accumulate) {
-          float4 x = *reinterpret_cast<const float4*>(dst + j);
-          o.x += x.x;
-          o.y += x.y;
-          o.z += x.z;
-          o.w += x.w;
-        }
-        *reinterpret_cast<float4*>(dst + j) = o;
-      }
-    } else {
-      for (int j = 0; j < 32 && col0 + j < p.N; ++j) dst[j] = p.accumulate ? dst[j] + v[j] : v[j];
-    }
+    stage_bf16_row(buf, lane, v);
   }
 }
 
@@ -204,12 +195,14 @@ __device__ __forceinline__ void tc_decode_unit(const GemmParams& p, int unit, in
 template <int BN, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                    const GemmParams p) {
   using Cfg = TcCfg<BN>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE);
+  uint8_t* staging = smem + STAGES * Cfg::STAGE;  // 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + Cfg::STAGING);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -360,8 +353,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int ew = warp - 2;         // 0..7
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int half = ew >> 2;        // which half of the BN columns
+    uint8_t* buf = staging + ew * 4096;
+    // bf16 single-output chunks take 2 KB: two buffers alternate; others take 4 KB
+    constexpr bool two_bufs = (EPI == EPI_BF16 || EPI == EPI_BF16_DGELU);
+    if (lane == 0) {
+      if (EPI == EPI_BF16_GELU || p.ksplit > 1) tma_prefetch_desc(&tmO2);
+      tma_prefetch_desc(&tmO);
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
+    int nchunk = 0;
     for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x) {
       int tm, tn, ks;
       tc_decode_unit(p, unit, tm, tn, ks);
@@ -373,21 +374,51 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int row = tm * TC_BM + q * 32 + lane;
+      const int row0 = tm * TC_BM + q * 32;
+      const int c_begin = half * (BN / 2), c_end = (half + 1) * (BN / 2);
 #pragma unroll 1
-      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+      for (int c = c_begin; c < c_end; c += 32, ++nchunk) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c), r);
         tmem_ld_wait();
+        if (c + 32 == c_end) {  // last read of this accumulator: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
         const int col0 = tn * BN + c;
-        if (row < p.M && col0 < p.N) tc_epilogue_row<EPI>(p, ks, row, col0, r);
+        uint8_t* b = (two_bufs && (nchunk & 1)) ? buf + 2048 : buf;
+        // the staging buffer must have been read out by the previous store
+        if (lane == 0) {
+          if (two_bufs) bulk_wait_read<1>();
+          else bulk_wait_read<0>();
+        }
+        __syncwarp();
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (col0 < p.N) tc_epilogue_stage<EPI>(p, row0 + lane, col0, lane, v, b);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (col0 < p.N && row0 < p.M) {
+            if (p.ksplit > 1) {
+              tma_store_3d(&tmO2, b, col0, row0, ks);
+            } else if (EPI == EPI_F32 && p.accumulate) {
+              tma_reduce_add_2d(&tmO, b, col0, row0);
+            } else {
+              tma_store_2d(&tmO, b, col0, row0);
+              if (EPI == EPI_BF16_GELU) tma_store_2d(&tmO2, b + 2048, col0, row0);
+            }
+          }
+          bulk_commit();  // one group per chunk (possibly empty) keeps the buffer accounting exact
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();

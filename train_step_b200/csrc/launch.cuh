@@ -149,6 +149,38 @@ inline bool encode_bf16_map(CUtensorMap* map, const void* ptr, long long inner, 
   return r == CUDA_SUCCESS;
 }
 
+// Epilogue store maps: rows x cols tensor (row stride ld elements), box of 32 x 32,
+// bf16 with 64-byte swizzle or fp32 with 128-byte swizzle (the staging layouts).
+inline bool encode_out_map(CUtensorMap* map, const void* ptr, long long cols, long long rows, long long ld,
+                           bool is_f32) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const int es = is_f32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
+  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, is_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   is_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Split-K partial workspace [ksplit][rows][cols] fp32 as a 3-D map, box 32 x 32 x 1.
+inline bool encode_partial_map(CUtensorMap* map, const void* ptr, long long cols, long long rows, int ksplit) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)ksplit};
+  cuuint64_t strides[2] = {(cuuint64_t)(cols * 4), (cuuint64_t)(rows * cols * 4)};
+  cuuint32_t box[3] = {32u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // GEMM
 // ---------------------------------------------------------------------------
@@ -172,8 +204,12 @@ struct GemmDesc {
   int ksplit;  // 0 = choose, 1 = none, > 1 = forced
 };
 
+struct TcMaps {
+  CUtensorMap a, b, o, o2;
+};
+
 template <int BN, bool AM, bool BM_, int EPI>
-int launch_tc_inst(const LaunchCtx& c, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p) {
+int launch_tc_inst(const LaunchCtx& c, const TcMaps& tm, const GemmParams& p) {
   auto kern = gemm_tc_kernel<BN, AM, BM_, EPI>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -182,18 +218,18 @@ int launch_tc_inst(const LaunchCtx& c, const CUtensorMap& ta, const CUtensorMap&
     attr_set = true;
   }
   const int grid = p.num_units < c.num_sms ? p.num_units : c.num_sms;
-  kern<<<grid, TC_THREADS, TcCfg<BN>::SMEM, c.stream>>>(ta, tb, p);
+  kern<<<grid, TC_THREADS, TcCfg<BN>::SMEM, c.stream>>>(tm.a, tm.b, tm.o, tm.o2, p);
   return check_launch(c, "gemm_tc");
 }
 
 template <int BN, bool AM, bool BM_>
-int launch_tc_epi(const LaunchCtx& c, int epi, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p) {
+int launch_tc_epi(const LaunchCtx& c, int epi, const TcMaps& tm, const GemmParams& p) {
   switch (epi) {
-    case EPI_BF16: return launch_tc_inst<BN, AM, BM_, EPI_BF16>(c, ta, tb, p);
-    case EPI_BF16_GELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_GELU>(c, ta, tb, p);
-    case EPI_F32_RESID: return launch_tc_inst<BN, AM, BM_, EPI_F32_RESID>(c, ta, tb, p);
-    case EPI_BF16_DGELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_DGELU>(c, ta, tb, p);
-    case EPI_F32: return launch_tc_inst<BN, AM, BM_, EPI_F32>(c, ta, tb, p);
+    case EPI_BF16: return launch_tc_inst<BN, AM, BM_, EPI_BF16>(c, tm, p);
+    case EPI_BF16_GELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_GELU>(c, tm, p);
+    case EPI_F32_RESID: return launch_tc_inst<BN, AM, BM_, EPI_F32_RESID>(c, tm, p);
+    case EPI_BF16_DGELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_DGELU>(c, tm, p);
+    case EPI_F32: return launch_tc_inst<BN, AM, BM_, EPI_F32>(c, tm, p);
   }
   return fail(c, GPT2_ERR_CONFIG, "gemm: unknown epilogue");
 }
@@ -248,21 +284,32 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
   p.partial = ksplit > 1 ? c.splitk_ws : nullptr;
   p.err = c.d_err;
   p.timeout_ns = 4000000000ull;
-  CUtensorMap ta, tb;
-  bool ok = d.a_mn ? encode_bf16_map(&ta, d.A, d.M, d.K, d.lda, 64) : encode_bf16_map(&ta, d.A, d.K, d.M, d.lda, 128);
-  ok = ok && (d.b_mn ? encode_bf16_map(&tb, d.B, d.N, d.K, d.ldb, 64) : encode_bf16_map(&tb, d.B, d.K, d.N, d.ldb, BN));
+  const bool out_f32 = (d.epi == EPI_F32 || d.epi == EPI_F32_RESID);
+  const int oes = out_f32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(d.out) & 15) || (d.ldo * oes) % 16 ||
+      (d.epi == EPI_BF16_GELU && ((reinterpret_cast<uintptr_t>(d.out2) & 15) || (d.ldo2 * 2) % 16)))
+    return fail(c, GPT2_ERR_CONFIG, "gemm: outputs need 16-byte aligned rows");
+  TcMaps tm;
+  bool ok = d.a_mn ? encode_bf16_map(&tm.a, d.A, d.M, d.K, d.lda, 64)
+                   : encode_bf16_map(&tm.a, d.A, d.K, d.M, d.lda, 128);
+  ok = ok && (d.b_mn ? encode_bf16_map(&tm.b, d.B, d.N, d.K, d.ldb, 64)
+                     : encode_bf16_map(&tm.b, d.B, d.K, d.N, d.ldb, BN));
+  ok = ok && encode_out_map(&tm.o, d.out, d.N, d.M, d.ldo, out_f32);
+  if (ksplit > 1) ok = ok && encode_partial_map(&tm.o2, c.splitk_ws, d.N, d.M, ksplit);
+  else if (d.epi == EPI_BF16_GELU) ok = ok && encode_out_map(&tm.o2, d.out2, d.N, d.M, d.ldo2, false);
+  else tm.o2 = tm.o;
   if (!ok) return fail(c, GPT2_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   int r;
   {
   ProfScope ps(c, CAT_GEMM, 2.0 * d.M * d.N * d.K, 0.0);
   if (BN == 256) {
-    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<256, false, false>(c, d.epi, ta, tb, p);
-    else if (!d.a_mn) r = launch_tc_epi<256, false, true>(c, d.epi, ta, tb, p);
-    else r = launch_tc_epi<256, true, true>(c, d.epi, ta, tb, p);
+    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<256, false, false>(c, d.epi, tm, p);
+    else if (!d.a_mn) r = launch_tc_epi<256, false, true>(c, d.epi, tm, p);
+    else r = launch_tc_epi<256, true, true>(c, d.epi, tm, p);
   } else {
-    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<128, false, false>(c, d.epi, ta, tb, p);
-    else if (!d.a_mn) r = launch_tc_epi<128, false, true>(c, d.epi, ta, tb, p);
-    else r = launch_tc_epi<128, true, true>(c, d.epi, ta, tb, p);
+    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<128, false, false>(c, d.epi, tm, p);
+    else if (!d.a_mn) r = launch_tc_epi<128, false, true>(c, d.epi, tm, p);
+    else r = launch_tc_epi<128, true, true>(c, d.epi, tm, p);
   }
   }
   if (r || ksplit == 1) return r;
@@ -340,39 +387,49 @@ inline int ln_bwd_grid(int N) {
   return g < 592 ? g : 592;
 }
 
-template <class T>
-int layernorm_bwd_t(const LaunchCtx& c, const float* dy, const float* x, const float* g, const float* mean,
-                    const float* rstd, int N, int C, float* dres, T* dres_act, int accumulate, float* part /*2*grid*C*/) {
-  const int grid = ln_bwd_grid(N);
-  const int nv = ln_nv(C);
-  float* pg = part;
-  float* pb = part + (size_t)grid * C;
-  ProfScope ps(c, CAT_LN_BWD, 0.0,
-               (double)N * C * (12 + 4 * accumulate + (dres_act ? sizeof(T) : 0)) + 8.0 * N + 8.0 * grid * C);
-#define LNB(NV)                                                                                                   \
-  layernorm_bwd_kernel<T, NV><<<grid, LN_WARPS * 32, 0, c.stream>>>(dy, x, g, mean, rstd, dres, dres_act, accumulate, \
-                                                                    pg, pb, N, C)
-  if (nv <= 1) LNB(1);
-  else if (nv <= 2) LNB(2);
-  else if (nv <= 4) LNB(4);
-  else if (nv <= 6) LNB(6);
-  else if (nv <= 8) LNB(8);
-  else if (nv <= 13) LNB(13);
-  else LNB(16);
-#undef LNB
-  return check_launch(c, "layernorm_bwd");
-}
-
-inline int reduce_partials(const LaunchCtx& c, const float* part, int P, int ncols, float* out, int accumulate) {
-  ProfScope ps(c, CAT_REDUCE, 0.0, 4.0 * P * ncols + 8.0 * ncols);
-  reduce_partials_kernel<<<(ncols + 255) / 256, 256, 0, c.stream>>>(part, P, ncols, ncols, out, accumulate);
+// out_v (+)= column sums of partial set v, for the non-null outputs out[0..nv).
+inline int reduce_partials(const LaunchCtx& c, const float* part, int P, int ncols, int nv, float* out0, float* out1,
+                           float* out2, int accumulate) {
+  ProfScope ps(c, CAT_REDUCE, 0.0, 4.0 * nv * P * ncols + 8.0 * nv * ncols);
+  ReduceOuts o{{out0, out1, out2}};
+  reduce_partials_kernel<<<dim3((ncols + 31) / 32, nv), 512, 0, c.stream>>>(part, P, ncols, o, accumulate);
   return check_launch(c, "reduce_partials");
 }
 
-// column sums of y [N, ncols] into out (+=), through a partial buffer of
-// colsum_rows(N, ncols) x ncols floats
+// LayerNorm backward plus the reduction of its parameter gradients: dg, db (+)=;
+// dbias_next (nullable) (+)= column sums of the updated dres.
+template <class T>
+int layernorm_bwd_t(const LaunchCtx& c, const float* dy, const float* x, const float* g, const float* mean,
+                    const float* rstd, int N, int C, float* dres, T* dres_act, int accumulate,
+                    float* part /*3*grid*C*/, float* dg, float* db, float* dbias_next, int accumulate_params) {
+  const int grid = ln_bwd_grid(N);
+  const int nv = ln_nv(C);
+  const int with_rsum = dbias_next != nullptr;
+  {
+    ProfScope ps(c, CAT_LN_BWD, 0.0,
+                 (double)N * C * (12 + 4 * accumulate + (dres_act ? sizeof(T) : 0)) + 8.0 * N +
+                     4.0 * (2 + with_rsum) * grid * C);
+#define LNB(NV)                                                                                                   \
+  layernorm_bwd_kernel<T, NV><<<grid, LN_WARPS * 32, 0, c.stream>>>(dy, x, g, mean, rstd, dres, dres_act, accumulate, \
+                                                                    part, with_rsum, N, C)
+    if (nv <= 1) LNB(1);
+    else if (nv <= 2) LNB(2);
+    else if (nv <= 4) LNB(4);
+    else if (nv <= 6) LNB(6);
+    else if (nv <= 8) LNB(8);
+    else if (nv <= 13) LNB(13);
+    else LNB(16);
+#undef LNB
+  }
+  int r = check_launch(c, "layernorm_bwd");
+  if (r) return r;
+  return reduce_partials(c, part, grid, C, 2 + with_rsum, dg, db, dbias_next, accumulate_params);
+}
+
+// column sums of y [N, ncols] (ncols % 8 == 0) into out (+=), through a partial
+// buffer of R x ncols floats
 inline void colsum_shape(int N, int ncols, int& gx, int& R, int& rows_per) {
-  gx = (ncols + 511) / 512;
+  gx = (ncols + 2047) / 2048;  // 256 threads x 8 columns
   R = 1184 / gx;
   if (R < 1) R = 1;
   if (R > N) R = N;
@@ -382,15 +439,16 @@ inline void colsum_shape(int N, int ncols, int& gx, int& R, int& rows_per) {
 
 template <class T>
 int colsum_t(const LaunchCtx& c, const T* y, long long ld, int N, int ncols, float* part, float* out) {
+  if (ncols % 8) return fail(c, GPT2_ERR_CONFIG, "colsum: ncols % 8 != 0");
   int gx, R, rows_per;
   colsum_shape(N, ncols, gx, R, rows_per);
   {
-  ProfScope ps(c, CAT_REDUCE, 0.0, (double)N * ncols * sizeof(T) + 4.0 * R * ncols);
-  colsum_partial_kernel<T><<<dim3(gx, R), 256, 0, c.stream>>>(y, ld, N, ncols, rows_per, part);
+    ProfScope ps(c, CAT_REDUCE, 0.0, (double)N * ncols * sizeof(T) + 4.0 * R * ncols);
+    colsum_partial_kernel<T><<<dim3(gx, R), 256, 0, c.stream>>>(y, ld, N, ncols, rows_per, part);
   }
   int r = check_launch(c, "colsum_partial");
   if (r) return r;
-  return reduce_partials(c, part, R, ncols, out, 1);
+  return reduce_partials(c, part, R, ncols, 1, out, nullptr, nullptr, 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -421,7 +479,8 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
   const int dblocks = (int)((warps * 32 + 255) / 256);
   if (dtype == GPT2_BF16) {
     if (hd != 64) return fail(c, GPT2_ERR_CONFIG, "attention (bf16): head dim must be 64");
-    attn_bwd_dot_kernel<bf16><<<dblocks, 256, 0, c.stream>>>((const bf16*)out, (const bf16*)dout, Dbuf, B, T, NH, hd);
+    attn_bwd_dot64_bf16_kernel<<<(int)((warps + 255) / 256), 256, 0, c.stream>>>((const bf16*)out, (const bf16*)dout,
+                                                                                  Dbuf, B, T, NH);
     int r = check_launch(c, "attn_bwd_dot");
     if (r) return r;
     dim3 grid((T + 63) / 64, B * NH);
@@ -527,9 +586,17 @@ inline int cross_entropy(const LaunchCtx& c, int dtype, void* logits, long long 
   if (N <= 0) return GPT2_OK;
   ProfScope ps(c, CAT_CE, 0.0, 2.0 * N * ld * (dtype == GPT2_BF16 ? 2 : 4));
   if (dtype == GPT2_BF16) {
-    if (ld % 8 || ld > (long long)CE_THREADS * CE_MAXVEC * 8)
-      return fail(c, GPT2_ERR_CONFIG, "cross_entropy: ld must be a multiple of 8 and <= 65536");
-    cross_entropy_bf16_kernel<<<N, CE_THREADS, 0, c.stream>>>((bf16*)logits, ld, V, tgt, scale, row_loss, c.d_err);
+    const long long smem = 2 * ld * 2;
+    if (ld % 8 || smem > 220 * 1024)
+      return fail(c, GPT2_ERR_CONFIG, "cross_entropy: ld must be a multiple of 8 and <= 56320");
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaFuncSetAttribute(cross_entropy_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+      attr_set = true;
+    }
+    const int grid = N < c.num_sms ? N : c.num_sms;
+    cross_entropy_bf16_kernel<<<grid, CE_PERSIST_THREADS, (size_t)smem, c.stream>>>(
+        (bf16*)logits, ld, V, N, tgt, scale, row_loss, c.d_err, 4000000000ull);
   } else {
     cross_entropy_f32_kernel<<<N, CE_THREADS, 0, c.stream>>>((float*)logits, ld, V, tgt, scale, row_loss, c.d_err);
   }

@@ -74,19 +74,21 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_fwd_kernel(const floa
 // Backward. With xh = (x - mean) * rstd and dxh = dy * g:
 //   dx = rstd * (dxh - mean(dxh) - xh * mean(dxh * xh))
 // dres (+)= dx (accumulate selects += vs =), dres_act (nullable) gets a copy of
-// the updated dres in the activation type. Per-CTA partial sums of dy*xh and dy
-// go to part_g / part_b [gridDim.x][C]; rows are assigned to CTAs in a fixed
-// pattern, so the reduction order never changes between runs.
+// the updated dres in the activation type. Per-CTA partial column sums go to
+// part [3][gridDim.x][C]: dy*xh (gain grad), dy (bias grad) and, when
+// with_rsum, the updated dres itself (the bias gradient of the linear layer whose
+// output this residual is). Rows are assigned to CTAs in a fixed pattern, so the
+// reduction order never changes between runs.
 template <class T, int NV>
-__global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
+__global__ void __launch_bounds__(LN_WARPS * 32, 2) layernorm_bwd_kernel(
     const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
     const float* __restrict__ mean, const float* __restrict__ rstd, float* __restrict__ dres,
-    T* __restrict__ dres_act, int accumulate, float* __restrict__ part_g, float* __restrict__ part_b, int N, int C) {
-  __shared__ float red[LN_WARPS][2][128 * 4];  // per-warp chunk partials, reused per column chunk
+    T* __restrict__ dres_act, int accumulate, float* __restrict__ part, int with_rsum, int N, int C) {
+  __shared__ float red[LN_WARPS][512];  // per-warp partials of one 512-column chunk
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float4 ag[NV], ab[NV];
+  float4 ag[NV], ab[NV], ar[NV];
 #pragma unroll
-  for (int i = 0; i < NV; ++i) ag[i] = ab[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < NV; ++i) ag[i] = ab[i] = ar[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (long long row = (long long)blockIdx.x * LN_WARPS + warp; row < N; row += (long long)gridDim.x * LN_WARPS) {
     const float mu = mean[row], rs = rstd[row];
     const float* dyr = dy + row * C;
@@ -133,64 +135,98 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
         }
         *reinterpret_cast<float4*>(dr + c) = o;
         if (dres_act) store4<T>(dres_act + row * C + c, o.x, o.y, o.z, o.w);
+        ar[i].x += o.x;
+        ar[i].y += o.y;
+        ar[i].z += o.z;
+        ar[i].w += o.w;
       }
     }
   }
-  // reduce the warps' partials in a fixed order, 512 columns at a time
+  // reduce the warps' partials in a fixed order, one 512-column chunk at a time
+  const int nsum = with_rsum ? 3 : 2;
+  for (int which = 0; which < nsum; ++which) {
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = (i * 32 + lane) * 4;
-    const int chunk = i >> 2;  // 4 vectors of 32 lanes = 512 columns per chunk
-    const int local = c - chunk * 512;
-    if ((i & 3) == 0) __syncthreads();
-    if (c < C) {
-      *reinterpret_cast<float4*>(&red[warp][0][local]) = ag[i];
-      *reinterpret_cast<float4*>(&red[warp][1][local]) = ab[i];
-    }
-    if ((i & 3) == 3 || i == NV - 1) {
-      __syncthreads();
-      for (int k = threadIdx.x; k < 512; k += blockDim.x) {
-        const int col = chunk * 512 + k;
-        if (col < C) {
-          float sg = 0.f, sb = 0.f;
-          for (int w = 0; w < LN_WARPS; ++w) {
-            sg += red[w][0][k];
-            sb += red[w][1][k];
+    for (int i = 0; i < NV; ++i) {
+      const int c = (i * 32 + lane) * 4;
+      const int chunk = i >> 2;  // 4 vectors of 32 lanes = 512 columns per chunk
+      const int local = c - chunk * 512;
+      if ((i & 3) == 0) __syncthreads();
+      if (c < C) *reinterpret_cast<float4*>(&red[warp][local]) = which == 0 ? ag[i] : (which == 1 ? ab[i] : ar[i]);
+      if ((i & 3) == 3 || i == NV - 1) {
+        __syncthreads();
+        for (int k = threadIdx.x; k < 512; k += blockDim.x) {
+          const int col = chunk * 512 + k;
+          if (col < C) {
+            float sacc = 0.f;
+#pragma unroll
+            for (int w = 0; w < LN_WARPS; ++w) sacc += red[w][k];
+            part[((long long)which * gridDim.x + blockIdx.x) * C + col] = sacc;
           }
-          part_g[(long long)blockIdx.x * C + col] = sg;
-          part_b[(long long)blockIdx.x * C + col] = sb;
         }
       }
     }
   }
 }
 
-// out[c] (+)= sum_{p < P} part[p * ld + c], in order of p (one thread per column).
-__global__ void reduce_partials_kernel(const float* __restrict__ part, int P, int ncols, long long ld,
-                                       float* __restrict__ out, int accumulate) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= ncols) return;
+// Deterministic column reduction of up to three partial sets at once:
+// out_v[c] (+)= sum_{p < P} part[(v*P + p)*ncols + c] for v = blockIdx.y. Each CTA
+// owns 32 columns; warp w sums rows p = w, w + 16, ... in order, then the 16
+// warp sums are added in order.
+struct ReduceOuts {
+  float* out[3];
+};
+__global__ void __launch_bounds__(512) reduce_partials_kernel(const float* __restrict__ part, int P, int ncols,
+                                                              ReduceOuts outs, int accumulate) {
+  __shared__ float sm[16][33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int v = blockIdx.y;
+  const int c = blockIdx.x * 32 + lane;
+  const float* base = part + (long long)v * P * ncols;
   float s = 0.f;
-  for (int p = 0; p < P; ++p) s += part[(long long)p * ld + c];
-  out[c] = accumulate ? out[c] + s : s;
+  if (c < ncols)
+    for (int p = warp; p < P; p += 16) s += base[(long long)p * ncols + c];
+  sm[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0 && c < ncols) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 16; ++w) t += sm[w][lane];
+    float* o = outs.out[v];
+    o[c] = accumulate ? o[c] + t : t;
+  }
 }
 
 // Column sums of an activation matrix y [N, ncols] (row stride ld), stage 1:
-// CTA (bx, by) sums rows [by*rows_per, (by+1)*rows_per) of 2*blockDim.x columns.
+// CTA (bx, by) sums rows [by*rows_per, (by+1)*rows_per) of 8 * blockDim.x
+// columns, 8 consecutive columns per thread (one 16-byte load of bf16, or two of fp32).
 template <class T>
 __global__ void colsum_partial_kernel(const T* __restrict__ y, long long ld, int N, int ncols, int rows_per,
                                       float* __restrict__ part) {
-  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 2;
+  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   if (c >= ncols) return;
   const int r0 = blockIdx.y * rows_per, r1 = min(N, r0 + rows_per);
-  float s0 = 0.f, s1 = 0.f;
+  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (int r = r0; r < r1; ++r) {
     const T* p = y + (long long)r * ld + c;
-    s0 += to_f32<T>(p[0]);
-    if (c + 1 < ncols) s1 += to_f32<T>(p[1]);
+    if (sizeof(T) == 2) {
+      const uint4 u = *reinterpret_cast<const uint4*>(p);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = unpack_bf16x2(w[q]);
+        s[2 * q] += f.x;
+        s[2 * q + 1] += f.y;
+      }
+    } else {
+      const float4 a = *reinterpret_cast<const float4*>(p);
+      const float4 b = *reinterpret_cast<const float4*>(p + 4);
+      s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
+      s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
+    }
   }
-  part[(long long)blockIdx.y * ncols + c] = s0;
-  if (c + 1 < ncols) part[(long long)blockIdx.y * ncols + c + 1] = s1;
+  float* o = part + (long long)blockIdx.y * ncols + c;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) o[q] = s[q];
 }
 
 }  // namespace g2
