@@ -13,6 +13,7 @@ namespace g2 {
 
 constexpr int CE_THREADS = 512;
 constexpr float LOG2E_CE = 1.4426950408889634f;
+constexpr float LN2_CE = 0.6931471805599453f;
 
 __device__ __forceinline__ float block_reduce_ce(float v, bool is_max, float* buf) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -25,16 +26,25 @@ __device__ __forceinline__ float block_reduce_ce(float v, bool is_max, float* bu
   return r;
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // bf16: persistent, one CTA per SM, rows r = blockIdx.x + k * gridDim.x. Two
 // shared-memory row buffers: row k+1 arrives by a 1-D bulk copy while row k is
-// processed; the result row leaves by a bulk store from the same buffer. HBM sees
-// each logit once in and once out. ld * 2 bytes per buffer (ld % 8 == 0).
+// processed. Each thread keeps a running (max, sum of exp) over its share of the
+// row (one pass), the block combines them, and a second pass writes the gradient
+// row to global memory with coalesced 16-byte stores, so the buffer is free for
+// the next-but-one row as soon as the pass ends. HBM sees each logit once in and
+// once out. ld * 2 bytes per buffer (ld % 8 == 0).
 constexpr int CE_PERSIST_THREADS = 512;
 __global__ void __launch_bounds__(CE_PERSIST_THREADS, 1) cross_entropy_bf16_kernel(
     bf16* __restrict__ logits, long long ld, int V, int rows, const int* __restrict__ tgt, float scale,
     float* __restrict__ row_loss, int* err, unsigned long long timeout_ns) {
   extern __shared__ __align__(128) uint8_t ce_smem[];
-  __shared__ float red[CE_PERSIST_THREADS / 32];
+  __shared__ float red_m[CE_PERSIST_THREADS / 32], red_s[CE_PERSIST_THREADS / 32];
   __shared__ __align__(8) uint64_t bar[2];
   __shared__ int s_abort;
   const uint32_t row_bytes = (uint32_t)(ld * 2);
@@ -56,8 +66,10 @@ __global__ void __launch_bounds__(CE_PERSIST_THREADS, 1) cross_entropy_bf16_kern
   for (int k = 0; row < rows; ++k, row += gridDim.x) {
     const int cur = k & 1;
     const int nxt_row = row + gridDim.x;
+    // buf[cur ^ 1] was last read in the previous iteration, which every thread has
+    // finished (the __syncthreads at its end)
     if (tid == 0 && nxt_row < rows) {
-      bulk_wait_read<0>();  // the previous store out of buf[cur ^ 1] has been read
+      fence_proxy_async_smem();  // order the generic reads of that buffer before the async write
       mbar_arrive_expect_tx(&bar[cur ^ 1], row_bytes);
       bulk_load_1d(buf[cur ^ 1], logits + (long long)nxt_row * ld, row_bytes, &bar[cur ^ 1]);
     }
@@ -70,56 +82,59 @@ __global__ void __launch_bounds__(CE_PERSIST_THREADS, 1) cross_entropy_bf16_kern
     }
     __syncthreads();
     if (s_abort) break;
-    // every thread waits on the barrier's phase too, so the async-proxy writes are visible
-    mbar_try_wait(&bar[cur], (k >> 1) & 1);
-    bf16* z = buf[cur];
+    mbar_try_wait(&bar[cur], (k >> 1) & 1);  // every thread observes the completed phase
+    const bf16* z = buf[cur];
     int t = tgt[row];
     if (t < 0 || t >= V) {
       if (tid == 0) raise_device_error(err, DEV_TOKEN_RANGE);
       t = 0;
     }
-    const float zt = __bfloat162float(z[t]);
-    float mx = -INFINITY;
+    // one pass: running max m and sum s of 2^(x*log2e - m) over this thread's columns
+    float m = -INFINITY, sacc = 0.f;
     for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
       const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      float x[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 f = unpack_bf16x2(w[q]);
-        const int c = vi * 8 + 2 * q;
-        if (c < V) mx = fmaxf(mx, f.x);
-        if (c + 1 < V) mx = fmaxf(mx, f.y);
+        x[2 * q] = vi * 8 + 2 * q < V ? f.x * LOG2E_CE : -INFINITY;
+        x[2 * q + 1] = vi * 8 + 2 * q + 1 < V ? f.y * LOG2E_CE : -INFINITY;
       }
-    }
-    mx = warp_max(mx);
-    if (lane == 0) red[warp] = mx;
-    __syncthreads();
-    mx = red[0];
+      float bm = x[0];
 #pragma unroll
-    for (int w = 1; w < CE_PERSIST_THREADS / 32; ++w) mx = fmaxf(mx, red[w]);
-    __syncthreads();
-    const float ml2 = mx * LOG2E_CE;
-    float se = 0.f;
-    for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
-      const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = unpack_bf16x2(w[q]);
-        const int c = vi * 8 + 2 * q;
-        if (c < V) se += exp2f(f.x * LOG2E_CE - ml2);
-        if (c + 1 < V) se += exp2f(f.y * LOG2E_CE - ml2);
+      for (int q = 1; q < 8; ++q) bm = fmaxf(bm, x[q]);
+      if (bm == -INFINITY) continue;  // all eight columns are padding
+      if (bm > m) {
+        sacc *= ex2_approx(m - bm);
+        m = bm;
       }
-    }
-    se = warp_sum(se);
-    if (lane == 0) red[warp] = se;
-    __syncthreads();
-    se = 0.f;
 #pragma unroll
-    for (int w = 0; w < CE_PERSIST_THREADS / 32; ++w) se += red[w];
-    const float lse = mx + __logf(se);
-    const float ll2 = lse * LOG2E_CE;
-    if (tid == 0) row_loss[row] = lse - zt;
+      for (int q = 0; q < 8; ++q) sacc += ex2_approx(x[q] - m);
+    }
+    // combine (m, s) pairs: warp, then block
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sacc, o);
+      const float mm = fmaxf(m, m2);
+      sacc = (m == -INFINITY ? 0.f : sacc * ex2_approx(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * ex2_approx(m2 - mm));
+      m = mm;
+    }
+    if (lane == 0) {
+      red_m[warp] = m;
+      red_s[warp] = sacc;
+    }
+    __syncthreads();
+    float M = red_m[0];
+#pragma unroll
+    for (int w = 1; w < CE_PERSIST_THREADS / 32; ++w) M = fmaxf(M, red_m[w]);
+    float S = 0.f;
+#pragma unroll
+    for (int w = 0; w < CE_PERSIST_THREADS / 32; ++w)
+      S += red_m[w] == -INFINITY ? 0.f : red_s[w] * ex2_approx(red_m[w] - M);
+    const float ll2 = M + __log2f(S);  // lse in the log2 domain
+    if (tid == 0) row_loss[row] = (ll2 - __bfloat162float(z[t]) * LOG2E_CE) * LN2_CE;
+    bf16* dst = logits + (long long)row * ld;
     for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
       const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -128,20 +143,14 @@ __global__ void __launch_bounds__(CE_PERSIST_THREADS, 1) cross_entropy_bf16_kern
       for (int q = 0; q < 4; ++q) {
         const float2 f = unpack_bf16x2(w[q]);
         const int c = vi * 8 + 2 * q;
-        const float a = c < V ? (exp2f(f.x * LOG2E_CE - ll2) - (c == t ? 1.f : 0.f)) * scale : 0.f;
-        const float b = c + 1 < V ? (exp2f(f.y * LOG2E_CE - ll2) - (c + 1 == t ? 1.f : 0.f)) * scale : 0.f;
+        const float a = c < V ? (ex2_approx(f.x * LOG2E_CE - ll2) - (c == t ? 1.f : 0.f)) * scale : 0.f;
+        const float b = c + 1 < V ? (ex2_approx(f.y * LOG2E_CE - ll2) - (c + 1 == t ? 1.f : 0.f)) * scale : 0.f;
         o[q] = pack_bf16x2(a, b);
       }
-      reinterpret_cast<uint4*>(z)[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<uint4*>(dst)[vi] = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      bulk_store_1d(logits + (long long)row * ld, z, row_bytes);
-      bulk_commit();
-    }
+    __syncthreads();  // everyone is done with buf[cur] and red_* before they are reused
   }
-  if (tid == 0) bulk_wait_all();
 }
 
 // fp32 parity mode: exact expf/logf, one CTA per row, strided (rows are short).

@@ -396,6 +396,19 @@ inline int reduce_partials(const LaunchCtx& c, const float* part, int P, int nco
   return check_launch(c, "reduce_partials");
 }
 
+template <class T, int NV>
+void launch_ln_bwd(const LaunchCtx& c, int grid, size_t smem, const float* dy, const float* x, const float* g,
+                   const float* mean, const float* rstd, float* dres, T* dres_act, int accumulate, float* part,
+                   int with_rsum, int N, int C) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(layernorm_bwd_kernel<T, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    attr = true;
+  }
+  layernorm_bwd_kernel<T, NV><<<grid, LN_WARPS * 32, smem, c.stream>>>(dy, x, g, mean, rstd, dres, dres_act,
+                                                                       accumulate, part, with_rsum, N, C);
+}
+
 // LayerNorm backward plus the reduction of its parameter gradients: dg, db (+)=;
 // dbias_next (nullable) (+)= column sums of the updated dres.
 template <class T>
@@ -409,17 +422,14 @@ int layernorm_bwd_t(const LaunchCtx& c, const float* dy, const float* x, const f
     ProfScope ps(c, CAT_LN_BWD, 0.0,
                  (double)N * C * (12 + 4 * accumulate + (dres_act ? sizeof(T) : 0)) + 8.0 * N +
                      4.0 * (2 + with_rsum) * grid * C);
-#define LNB(NV)                                                                                                   \
-  layernorm_bwd_kernel<T, NV><<<grid, LN_WARPS * 32, 0, c.stream>>>(dy, x, g, mean, rstd, dres, dres_act, accumulate, \
-                                                                    part, with_rsum, N, C)
-    if (nv <= 1) LNB(1);
-    else if (nv <= 2) LNB(2);
-    else if (nv <= 4) LNB(4);
-    else if (nv <= 6) LNB(6);
-    else if (nv <= 8) LNB(8);
-    else if (nv <= 13) LNB(13);
-    else LNB(16);
-#undef LNB
+    const size_t smem = (size_t)LN_WARPS * 3 * C * 4;
+    if (nv <= 1) launch_ln_bwd<T, 1>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 2) launch_ln_bwd<T, 2>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 4) launch_ln_bwd<T, 4>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 6) launch_ln_bwd<T, 6>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 8) launch_ln_bwd<T, 8>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 13) launch_ln_bwd<T, 13>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else launch_ln_bwd<T, 16>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
   }
   int r = check_launch(c, "layernorm_bwd");
   if (r) return r;

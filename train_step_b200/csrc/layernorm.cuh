@@ -80,15 +80,21 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_fwd_kernel(const floa
 // output this residual is). Rows are assigned to CTAs in a fixed pattern, so the
 // reduction order never changes between runs.
 template <class T, int NV>
-__global__ void __launch_bounds__(LN_WARPS * 32, 2) layernorm_bwd_kernel(
+__global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
     const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
     const float* __restrict__ mean, const float* __restrict__ rstd, float* __restrict__ dres,
     T* __restrict__ dres_act, int accumulate, float* __restrict__ part, int with_rsum, int N, int C) {
-  __shared__ float red[LN_WARPS][512];  // per-warp partials of one 512-column chunk
+  // per-warp column accumulators [warp][3][C] in dynamic shared memory; lane l owns
+  // the float4 slots (i*32 + l), so there are no bank conflicts and no atomics
+  extern __shared__ float4 ln_acc[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float4 ag[NV], ab[NV], ar[NV];
+  const int C4 = C / 4;
+  float4* accw = ln_acc + (size_t)warp * 3 * C4;
 #pragma unroll
-  for (int i = 0; i < NV; ++i) ag[i] = ab[i] = ar[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < NV; ++i) {
+    const int c4 = i * 32 + lane;
+    if (c4 < C4) accw[c4] = accw[C4 + c4] = accw[2 * C4 + c4] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   for (long long row = (long long)blockIdx.x * LN_WARPS + warp; row < N; row += (long long)gridDim.x * LN_WARPS) {
     const float mu = mean[row], rs = rstd[row];
     const float* dyr = dy + row * C;
@@ -106,14 +112,17 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 2) layernorm_bwd_kernel(
         float a = vd[i].x * gg.x, b = vd[i].y * gg.y, cc = vd[i].z * gg.z, d = vd[i].w * gg.w;
         m1 += (a + b) + (cc + d);
         m2 += (a * vx[i].x + b * vx[i].y) + (cc * vx[i].z + d * vx[i].w);
-        ag[i].x += vd[i].x * vx[i].x;
-        ag[i].y += vd[i].y * vx[i].y;
-        ag[i].z += vd[i].z * vx[i].z;
-        ag[i].w += vd[i].w * vx[i].w;
-        ab[i].x += vd[i].x;
-        ab[i].y += vd[i].y;
-        ab[i].z += vd[i].z;
-        ab[i].w += vd[i].w;
+        float4 ag = accw[i * 32 + lane], ab = accw[C4 + i * 32 + lane];
+        ag.x += vd[i].x * vx[i].x;
+        ag.y += vd[i].y * vx[i].y;
+        ag.z += vd[i].z * vx[i].z;
+        ag.w += vd[i].w * vx[i].w;
+        ab.x += vd[i].x;
+        ab.y += vd[i].y;
+        ab.z += vd[i].z;
+        ab.w += vd[i].w;
+        accw[i * 32 + lane] = ag;
+        accw[C4 + i * 32 + lane] = ab;
       }
     }
     m1 = warp_sum(m1) / (float)C;
@@ -135,36 +144,27 @@ __global__ void __launch_bounds__(LN_WARPS * 32, 2) layernorm_bwd_kernel(
         }
         *reinterpret_cast<float4*>(dr + c) = o;
         if (dres_act) store4<T>(dres_act + row * C + c, o.x, o.y, o.z, o.w);
-        ar[i].x += o.x;
-        ar[i].y += o.y;
-        ar[i].z += o.z;
-        ar[i].w += o.w;
-      }
-    }
-  }
-  // reduce the warps' partials in a fixed order, one 512-column chunk at a time
-  const int nsum = with_rsum ? 3 : 2;
-  for (int which = 0; which < nsum; ++which) {
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int c = (i * 32 + lane) * 4;
-      const int chunk = i >> 2;  // 4 vectors of 32 lanes = 512 columns per chunk
-      const int local = c - chunk * 512;
-      if ((i & 3) == 0) __syncthreads();
-      if (c < C) *reinterpret_cast<float4*>(&red[warp][local]) = which == 0 ? ag[i] : (which == 1 ? ab[i] : ar[i]);
-      if ((i & 3) == 3 || i == NV - 1) {
-        __syncthreads();
-        for (int k = threadIdx.x; k < 512; k += blockDim.x) {
-          const int col = chunk * 512 + k;
-          if (col < C) {
-            float sacc = 0.f;
-#pragma unroll
-            for (int w = 0; w < LN_WARPS; ++w) sacc += red[w][k];
-            part[((long long)which * gridDim.x + blockIdx.x) * C + col] = sacc;
-          }
+        if (with_rsum) {
+          float4 ar = accw[2 * C4 + i * 32 + lane];
+          ar.x += o.x;
+          ar.y += o.y;
+          ar.z += o.z;
+          ar.w += o.w;
+          accw[2 * C4 + i * 32 + lane] = ar;
         }
       }
     }
+  }
+  __syncthreads();
+  // CTA partials: sum the warps' accumulators in a fixed order
+  const int nsum = with_rsum ? 3 : 2;
+  const float* accf = reinterpret_cast<const float*>(ln_acc);
+  for (int idx = threadIdx.x; idx < nsum * C; idx += blockDim.x) {
+    const int which = idx / C, col = idx - which * C;
+    float sacc = 0.f;
+#pragma unroll
+    for (int w = 0; w < LN_WARPS; ++w) sacc += accf[((size_t)w * 3 + which) * C + col];
+    part[((long long)which * gridDim.x + blockIdx.x) * C + col] = sacc;
   }
 }
 
