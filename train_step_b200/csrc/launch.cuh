@@ -11,6 +11,7 @@
 #include "../../include/gpt2.h"
 #include "adamw.cuh"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 #include "cross_entropy.cuh"
 #include "embedding.cuh"
@@ -163,6 +164,21 @@ inline bool encode_out_map(CUtensorMap* map, const void* ptr, long long cols, lo
   CUresult r = enc(map, is_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    is_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// qkv [B][T][3C] bf16 as a 3-D map {3C, T, B}; box {64, 128, 1} (one head's 64
+// columns of 128 positions), 128-byte swizzle; positions past T read as zero.
+inline bool encode_qkv_map(CUtensorMap* map, const void* ptr, long long cols, long long T, long long B) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), (cuuint64_t)(T * cols * 2)};
+  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -470,9 +486,18 @@ inline int attention_fwd(const LaunchCtx& c, int dtype, const void* qkv, int B, 
   ProfScope ps(c, CAT_ATTN_FWD, 4.0 * B * NH * hd * (0.5 * T * (T + 1.0)), 0.0);
   if (dtype == GPT2_BF16) {
     if (hd != 64) return fail(c, GPT2_ERR_CONFIG, "attention (bf16): head dim must be 64");
-    dim3 grid((T + 63) / 64, B * NH);
-    attn_fwd_bf16_kernel<<<grid, 128, 0, c.stream>>>((const bf16*)qkv, (bf16*)out, lse, T, NH, scale);
-    return check_launch(c, "attn_fwd_bf16");
+    if (reinterpret_cast<uintptr_t>(qkv) & 15) return fail(c, GPT2_ERR_CONFIG, "attention: qkv must be 16-byte aligned");
+    CUtensorMap tm;
+    if (!encode_qkv_map(&tm, qkv, 3LL * NH * 64, T, B)) return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
+      attr_set = true;
+    }
+    dim3 grid((T + FA_BM - 1) / FA_BM, B * NH);
+    attn_fwd_tc_kernel<<<grid, FA_THREADS, FA_SMEM, c.stream>>>(tm, (bf16*)out, lse, T, NH, scale, c.d_err,
+                                                                4000000000ull);
+    return check_launch(c, "attn_fwd_tc");
   }
   if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");
   const long long warps = (long long)B * NH * T;
@@ -489,18 +514,29 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
   const int dblocks = (int)((warps * 32 + 255) / 256);
   if (dtype == GPT2_BF16) {
     if (hd != 64) return fail(c, GPT2_ERR_CONFIG, "attention (bf16): head dim must be 64");
+    if ((reinterpret_cast<uintptr_t>(qkv) & 15) || (reinterpret_cast<uintptr_t>(dout) & 15))
+      return fail(c, GPT2_ERR_CONFIG, "attention: qkv and dout must be 16-byte aligned");
     attn_bwd_dot64_bf16_kernel<<<(int)((warps + 255) / 256), 256, 0, c.stream>>>((const bf16*)out, (const bf16*)dout,
                                                                                   Dbuf, B, T, NH);
     int r = check_launch(c, "attn_bwd_dot");
     if (r) return r;
-    dim3 grid((T + 63) / 64, B * NH);
-    attn_bwd_dkdv_bf16_kernel<<<grid, 128, 0, c.stream>>>((const bf16*)qkv, (const bf16*)dout, lse, Dbuf, (bf16*)dqkv,
-                                                          T, NH, scale);
-    r = check_launch(c, "attn_bwd_dkdv");
+    CUtensorMap tq, td;
+    if (!encode_qkv_map(&tq, qkv, 3LL * NH * 64, T, B) || !encode_qkv_map(&td, dout, (long long)NH * 64, T, B))
+      return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FBK_SMEM);
+      cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FBQ_SMEM);
+      attr_set = true;
+    }
+    dim3 grid((T + FA_BM - 1) / FA_BM, B * NH);
+    attn_bwd_dkdv_tc_kernel<<<grid, FB_THREADS, FBK_SMEM, c.stream>>>(tq, td, lse, Dbuf, (bf16*)dqkv, T, NH, scale,
+                                                                      c.d_err, 4000000000ull);
+    r = check_launch(c, "attn_bwd_dkdv_tc");
     if (r) return r;
-    attn_bwd_dq_bf16_kernel<<<grid, 128, 0, c.stream>>>((const bf16*)qkv, (const bf16*)dout, lse, Dbuf, (bf16*)dqkv, T,
-                                                        NH, scale);
-    return check_launch(c, "attn_bwd_dq");
+    attn_bwd_dq_tc_kernel<<<grid, FB_THREADS, FBQ_SMEM, c.stream>>>(tq, td, lse, Dbuf, (bf16*)dqkv, T, NH, scale,
+                                                                    c.d_err, 4000000000ull);
+    return check_launch(c, "attn_bwd_dq_tc");
   }
   if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");
   attn_bwd_dot_kernel<float><<<dblocks, 256, 0, c.stream>>>((const float*)out, (const float*)dout, Dbuf, B, T, NH, hd);
