@@ -176,6 +176,16 @@ int gpt2_op_gemm(int dtype, const void* A, int64_t lda, int a_mn, const void* B,
                  int K, int epilogue, void* out, int64_t ldo, void* out2, int64_t ldo2, const float* bias,
                  const void* aux, int64_t ld_aux, int accumulate, int ksplit, void* stream);
 
+/* Time the bf16 tensor-core GEMM of gpt2_op_gemm (same arguments) over `iters`
+ * back-to-back launches after one warm-up launch, with CUDA events on `stream`;
+ * *ms_out = average milliseconds per call (split-K reduction included).
+ * ksplit 0 lets the library choose the split as inside the training step; bn is
+ * the tile width (0 = the library's choice, or 128 / 256). Synchronises. */
+int gpt2_op_gemm_bench(const void* A, int64_t lda, int a_mn, const void* B, int64_t ldb, int b_mn, int M, int N, int K,
+                       int epilogue, void* out, int64_t ldo, void* out2, int64_t ldo2, const float* bias,
+                       const void* aux, int64_t ld_aux, int accumulate, int ksplit, int bn, int iters,
+                       float* ms_out, void* stream);
+
 /* LayerNorm forward over rows of f32_x [N, C]: y(act) [N, C], f32 mean and rstd
  * [N]. eps 1e-5, biased variance. C % 4 == 0, C <= 2048. */
 int gpt2_op_layernorm_fwd(int dtype, const float* f32_x, const float* f32_g, const float* f32_b, int N, int C, void* y,

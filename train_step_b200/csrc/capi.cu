@@ -287,14 +287,14 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     const int rows = (N - r0) < chunk ? (N - r0) : chunk;
     char* xf_c = m->xf + (int64_t)r0 * C * ab;
     RK(gemm(c, dt, GemmDesc{xf_c, C, false, m->W(headw), C, false, rows, Vp, C, EPI_BF16, m->logits, Vp, nullptr, 0,
-                            nullptr, nullptr, 0, 0, 1}));
+                            nullptr, nullptr, 0, 0, 1, CAT_GEMM_HEAD}));
     RK(cross_entropy(c, dt, m->logits, Vp, rows, m->cfg.V, m->tgt + r0, 1.0f / (float)N, m->row_loss + r0));
     if (backward) {
       // dxf = dlogits W ; dW += dlogits^T xf
       RK(gemm(c, dt, GemmDesc{m->logits, Vp, false, m->W(headw), C, true, rows, C, Vp, EPI_F32, m->dh + (int64_t)r0 * C,
-                              C, nullptr, 0, nullptr, nullptr, 0, 0, 0}));
+                              C, nullptr, 0, nullptr, nullptr, 0, 0, 0, CAT_GEMM_HEAD}));
       RK(gemm(c, dt, GemmDesc{m->logits, Vp, true, xf_c, C, true, Vp, C, rows, EPI_F32, g_head, C, nullptr, 0, nullptr,
-                              nullptr, 0, 1, 0}));
+                              nullptr, 0, 1, 0, CAT_GEMM_HEAD}));
     }
   }
   sum_rows_kernel<<<1, 1024, 0, m->stream>>>(m->row_loss, N, 1.0f / (float)N, m->d_loss, 0);
@@ -329,26 +329,26 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     float* lse = m->lse + l * NLSE;
     // MLP: x_out = x_mid + pj(gelu(fc(ln2(x_mid))))
     RK(gemm(c, dt, GemmDesc{dres_act, C, true, a, F, true, C, F, N, EPI_F32, gw.pj_w, F, nullptr, 0, nullptr, nullptr,
-                            0, 1, 0}));
+                            0, 1, 0, CAT_GEMM_DW}));
     RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.pj_w), F, true, N, F, C, EPI_BF16_DGELU, m->du, F, nullptr, 0,
-                            nullptr, u, F, 0, 1}));
+                            nullptr, u, F, 0, 1, CAT_GEMM_DX}));
     RK(gemm(c, dt, GemmDesc{m->du, F, true, h2, C, true, F, C, N, EPI_F32, gw.fc_w, C, nullptr, 0, nullptr, nullptr, 0,
-                            1, 0}));
+                            1, 0, CAT_GEMM_DW}));
     RK(COLSUM_ACT(m->du, F, gw.fc_b));
     RK(gemm(c, dt, GemmDesc{m->du, F, false, m->W(w.fc_w), C, true, N, C, F, EPI_F32, m->dh, C, nullptr, 0, nullptr,
-                            nullptr, 0, 0, 1}));
+                            nullptr, 0, 0, 1, CAT_GEMM_DX}));
     RK(LN_B(m->dh, xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), 1, gw.ln2_g, gw.ln2_b, gw.ao_b));
     // attention: x_mid = x_in + ao(attn(ln1(x_in)))
     RK(gemm(c, dt, GemmDesc{dres_act, C, true, att, C, true, C, C, N, EPI_F32, gw.ao_w, C, nullptr, 0, nullptr, nullptr,
-                            0, 1, 0}));
+                            0, 1, 0, CAT_GEMM_DW}));
     RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.ao_w), C, true, N, C, C, EPI_BF16, m->datt, C, nullptr, 0,
-                            nullptr, nullptr, 0, 0, 1}));
+                            nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
     RK(attention_bwd(c, dt, qkv, att, m->datt, lse, B, T, NH, hd, m->dqkv, m->Dattn));
     RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, true, h1, C, true, 3 * C, C, N, EPI_F32, gw.qkv_w, C, nullptr, 0, nullptr,
-                            nullptr, 0, 1, 0}));
+                            nullptr, 0, 1, 0, CAT_GEMM_DW}));
     if (gw.qkv_b) RK(COLSUM_ACT(m->dqkv, 3 * C, gw.qkv_b));
     RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, false, m->W(w.qkv_w), C, true, N, C, 3 * C, EPI_F32, m->dh, C, nullptr, 0,
-                            nullptr, nullptr, 0, 0, 1}));
+                            nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
     RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b,
             l > 0 ? m->lg[l - 1].pj_b : nullptr));
   }
@@ -780,6 +780,43 @@ int gpt2_op_gemm(int dtype, const void* A, int64_t lda, int a_mn, const void* B,
                         ld_aux, accumulate, ksplit <= 0 ? 1 : ksplit});
   if (ws) cudaFreeAsync(ws, o.s);
   int r2 = o.finish();
+  return r ? r : r2;
+}
+
+int gpt2_op_gemm_bench(const void* A, int64_t lda, int a_mn, const void* B, int64_t ldb, int b_mn, int M, int N, int K,
+                       int epilogue, void* out, int64_t ldo, void* out2, int64_t ldo2, const float* bias,
+                       const void* aux, int64_t ld_aux, int accumulate, int ksplit, int bn, int iters,
+                       float* ms_out, void* stream) {
+  if (iters <= 0 || !ms_out) {
+    g_op_error = "gemm_bench: iters > 0 and ms_out required";
+    return GPT2_ERR_CONFIG;
+  }
+  OpCtx o(stream);
+  RK(o.alloc_err());
+  float* ws = nullptr;
+  if (epilogue == EPI_F32 && ksplit != 1) {
+    const size_t n = (size_t)(ksplit > 1 ? ksplit : 16) * M * N;
+    if (cudaMallocAsync((void**)&ws, n * 4, o.s) != cudaSuccess) return GPT2_ERR_OOM;
+    o.c.splitk_ws = ws;
+    o.c.splitk_cap = n;
+  }
+  GemmDesc d{A, lda, a_mn != 0, B, ldb, b_mn != 0, M, N, K, epilogue, out, ldo, out2, ldo2, bias, aux, ld_aux,
+             accumulate, ksplit < 0 ? 1 : ksplit};
+  d.bn = bn;
+  int r = gemm_tc(o.c, d);  // warm-up (also sets kernel attributes)
+  cudaEvent_t e0, e1;
+  cudaEventCreate(&e0);
+  cudaEventCreate(&e1);
+  cudaEventRecord(e0, o.s);
+  for (int i = 0; i < iters && !r; ++i) r = gemm_tc(o.c, d);
+  cudaEventRecord(e1, o.s);
+  if (ws) cudaFreeAsync(ws, o.s);
+  int r2 = o.finish();
+  float ms = 0.f;
+  cudaEventElapsedTime(&ms, e0, e1);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  *ms_out = ms / iters;
   return r ? r : r2;
 }
 

@@ -23,7 +23,10 @@ namespace g2 {
 
 // Kernel categories for the per-launch CUDA-event profiler.
 enum ProfCat : int {
-  CAT_GEMM = 0,
+  CAT_GEMM = 0,   // forward linears (qkv, attention-out, fc, proj)
+  CAT_GEMM_HEAD,  // lm_head logits, dxf, dW
+  CAT_GEMM_DX,    // backward input gradients
+  CAT_GEMM_DW,    // backward weight gradients
   CAT_SPLITK,
   CAT_ATTN_FWD,
   CAT_ATTN_BWD,
@@ -37,9 +40,10 @@ enum ProfCat : int {
   CAT_COUNT
 };
 inline const char* prof_cat_name(int c) {
-  static const char* n[CAT_COUNT] = {"gemm_tc",        "splitk_reduce", "attention_fwd", "attention_bwd",
-                                     "layernorm_fwd",  "layernorm_bwd", "reductions",    "embedding_fwd",
-                                     "embedding_bwd",  "cross_entropy", "adamw"};
+  static const char* n[CAT_COUNT] = {"gemm_tc_fwd",   "gemm_tc_head",  "gemm_tc_dx",    "gemm_tc_dw",
+                                     "splitk_reduce", "attention_fwd", "attention_bwd", "layernorm_fwd",
+                                     "layernorm_bwd", "reductions",    "embedding_fwd", "embedding_bwd",
+                                     "cross_entropy", "adamw"};
   return (c >= 0 && c < CAT_COUNT) ? n[c] : "?";
 }
 
@@ -218,6 +222,8 @@ struct GemmDesc {
   long long ld_aux;
   int accumulate;
   int ksplit;  // 0 = choose, 1 = none, > 1 = forced
+  int role = CAT_GEMM;  // profiler category
+  int bn = 0;           // tile width: 0 = choose (256 when N >= 256), else 128 or 256
 };
 
 struct TcMaps {
@@ -255,7 +261,7 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
   if (d.a_mn && !d.b_mn) return fail(c, GPT2_ERR_CONFIG, "gemm: MN-major A needs MN-major B");
   if ((d.lda % 8) || (d.ldb % 8) || (reinterpret_cast<uintptr_t>(d.A) & 15) || (reinterpret_cast<uintptr_t>(d.B) & 15))
     return fail(c, GPT2_ERR_CONFIG, "gemm: bf16 operands need 16-byte aligned rows");
-  const int BN = d.N >= 256 ? 256 : 128;
+  const int BN = d.bn == 128 || d.bn == 256 ? d.bn : (d.N >= 256 ? 256 : 128);
   const int tiles_m = (d.M + TC_BM - 1) / TC_BM, tiles_n = (d.N + BN - 1) / BN;
   const int num_kb = (d.K + TC_BK - 1) / TC_BK;
   int ksplit = d.ksplit;
@@ -317,7 +323,7 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
   if (!ok) return fail(c, GPT2_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   int r;
   {
-  ProfScope ps(c, CAT_GEMM, 2.0 * d.M * d.N * d.K, 0.0);
+  ProfScope ps(c, d.role, 2.0 * d.M * d.N * d.K, 0.0);
   if (BN == 256) {
     if (!d.a_mn && !d.b_mn) r = launch_tc_epi<256, false, false>(c, d.epi, tm, p);
     else if (!d.a_mn) r = launch_tc_epi<256, false, true>(c, d.epi, tm, p);
@@ -359,7 +365,7 @@ inline int gemm_simt(const LaunchCtx& c, const GemmDesc& d) {
   a.ep.ld_aux = d.ld_aux;
   a.ep.accumulate = d.accumulate;
   dim3 grid((d.N + 63) / 64, (d.M + 63) / 64);
-  ProfScope ps(c, CAT_GEMM, 2.0 * d.M * d.N * d.K, 0.0);
+  ProfScope ps(c, d.role, 2.0 * d.M * d.N * d.K, 0.0);
   switch (d.epi) {
     case EPI_BF16: gemm_simt_kernel<EPI_BF16><<<grid, 256, 0, c.stream>>>(a); break;
     case EPI_BF16_GELU: gemm_simt_kernel<EPI_BF16_GELU><<<grid, 256, 0, c.stream>>>(a); break;
