@@ -180,10 +180,13 @@ int gpt2_op_gemm(int dtype, const void* A, int64_t lda, int a_mn, const void* B,
  * back-to-back launches after one warm-up launch, with CUDA events on `stream`;
  * *ms_out = average milliseconds per call (split-K reduction included).
  * ksplit 0 lets the library choose the split as inside the training step; bn is
- * the tile width (0 = the library's choice, or 128 / 256). Synchronises. */
+ * the tile width (0 = the library's choice, or 128 / 256); pair selects 256-row
+ * tiles computed by a cluster of two CTAs whose MMAs span both SMs (-1 = the
+ * library's choice, 0 = one CTA per 128-row tile, 1 = pairs; needs tile width
+ * 256). Returns GPT2_ERR_CONFIG for iters <= 0 or a NULL ms_out. Synchronises. */
 int gpt2_op_gemm_bench(const void* A, int64_t lda, int a_mn, const void* B, int64_t ldb, int b_mn, int M, int N, int K,
                        int epilogue, void* out, int64_t ldo, void* out2, int64_t ldo2, const float* bias,
-                       const void* aux, int64_t ld_aux, int accumulate, int ksplit, int bn, int iters,
+                       const void* aux, int64_t ld_aux, int accumulate, int ksplit, int bn, int pair, int iters,
                        float* ms_out, void* stream);
 
 /* LayerNorm forward over rows of f32_x [N, C]: y(act) [N, C], f32 mean and rstd

@@ -108,6 +108,48 @@ def test_gemm_bf16_epilogues(M, N, K):
     assert rel_l2(g64(o3), oracle.gelu_bwd(g64(ua), D)) < 5e-3
 
 
+@pytest.mark.parametrize("M,N,K", [(300, 520, 200), (130, 256, 72), (1000, 768, 768), (512, 2304, 1024)])
+@pytest.mark.parametrize("a_mn,b_mn", MAJORS)
+def test_gemm_bf16_pair_tiles(M, N, K, a_mn, b_mn):
+    """256 x 256 tiles computed by a 2-CTA cluster (M = 256 MMAs across both SMs), forced
+    through the timing entry point: every epilogue, ragged M / N tails (the second CTA's
+    rows partly or wholly past M), and a split-K fp32 store."""
+    if a_mn and M % 8:
+        M += 8 - M % 8
+    A, As, lda = operand(M, K, a_mn, 11, torch.bfloat16)
+    B, Bs, ldb = operand(N, K, b_mn, 12, torch.bfloat16)
+    D = oracle.linear_fwd(g64(A), g64(B))
+    bias = randn((N,), 13, torch.float32)
+    kw = dict(M=M, N=N, K=K, lda=lda, ldb=ldb, ldo=N, a_mn=a_mn, b_mn=b_mn, bn=256, pair=1, iters=1)
+    out = torch.zeros(M, N, dtype=torch.float32, device=DEV)
+    tsb.gemm_bench(As, Bs, out, epilogue=tsb.EPI_F32, **kw)
+    torch.cuda.synchronize()
+    assert rel_l2(g64(out), D) < 1e-5
+    if K >= 192:
+        out.zero_()
+        tsb.gemm_bench(As, Bs, out, epilogue=tsb.EPI_F32, ksplit=3, **kw)
+        torch.cuda.synchronize()
+        assert rel_l2(g64(out), D) < 1e-5
+    ref = D + g64(bias)
+    o0 = torch.zeros(M, N, dtype=torch.bfloat16, device=DEV)
+    tsb.gemm_bench(As, Bs, o0, epilogue=tsb.EPI_BIAS, bias=bias, **kw)
+    u = torch.zeros(M, N, dtype=torch.bfloat16, device=DEV)
+    a = torch.zeros_like(u)
+    tsb.gemm_bench(As, Bs, u, epilogue=tsb.EPI_BIAS_GELU, out2=a, ldo2=N, bias=bias, **kw)
+    res = randn((M, N), 14, torch.float32)
+    o2 = torch.zeros(M, N, dtype=torch.float32, device=DEV)
+    tsb.gemm_bench(As, Bs, o2, epilogue=tsb.EPI_RESID, bias=bias, aux=res, ld_aux=N, **kw)
+    ua = randn((M, N), 15, torch.bfloat16)
+    o3 = torch.zeros(M, N, dtype=torch.bfloat16, device=DEV)
+    tsb.gemm_bench(As, Bs, o3, epilogue=tsb.EPI_DGELU, aux=ua, ld_aux=N, **kw)
+    torch.cuda.synchronize()
+    assert rel_l2(g64(o0), ref) < 4e-3
+    assert rel_l2(g64(u), ref) < 4e-3
+    assert rel_l2(g64(a), oracle.gelu_fwd(ref)) < 5e-3
+    assert rel_l2(g64(o2), ref + g64(res)) < 1e-5
+    assert rel_l2(g64(o3), oracle.gelu_bwd(g64(ua), D)) < 5e-3
+
+
 @pytest.mark.parametrize("a_mn,b_mn", MAJORS)
 @pytest.mark.parametrize("epi", [0, 1, 2, 3, 4])
 def test_gemm_fp32_simt(a_mn, b_mn, epi):

@@ -61,8 +61,8 @@ _SYMBOLS = {
                       ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_void_p], ct.c_int),
     "gpt2_op_gemm_bench": ([ct.c_void_p, ct.c_int64, ct.c_int, ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_int,
                             ct.c_int, ct.c_int, ct.c_void_p, ct.c_int64, ct.c_void_p, ct.c_int64, ct.c_void_p,
-                            ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_int, ct.c_int, ct.POINTER(ct.c_float),
-                            ct.c_void_p], ct.c_int),
+                            ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_int, ct.c_int, ct.c_int,
+                            ct.POINTER(ct.c_float), ct.c_void_p], ct.c_int),
     "gpt2_op_layernorm_fwd": ([ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_void_p,
                                ct.c_void_p, ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_op_layernorm_bwd": ([ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int,
@@ -279,12 +279,14 @@ def gemm(A, B, out, *, M, N, K, lda, ldb, ldo, a_mn=False, b_mn=False, epilogue=
 
 
 def gemm_bench(A, B, out, *, M, N, K, lda, ldb, ldo, a_mn=False, b_mn=False, epilogue=EPI_F32, out2=None, ldo2=0,
-               bias=None, aux=None, ld_aux=0, accumulate=False, ksplit=1, bn=0, iters=20, stream=None) -> float:
-    """Average milliseconds of the bf16 tensor-core GEMM over `iters` back-to-back launches."""
+               bias=None, aux=None, ld_aux=0, accumulate=False, ksplit=1, bn=0, pair=-1, iters=20,
+               stream=None) -> float:
+    """Average milliseconds of the bf16 tensor-core GEMM over `iters` back-to-back launches
+    (pair: -1 library choice, 0 one CTA per tile, 1 two-CTA 256 x 256 tiles)."""
     ms = ct.c_float()
     _op(lib().gpt2_op_gemm_bench(_ptr(A), lda, int(a_mn), _ptr(B), ldb, int(b_mn), M, N, K, epilogue, _ptr(out), ldo,
-                                 _ptr(out2), ldo2, _ptr(bias), _ptr(aux), ld_aux, int(accumulate), ksplit, bn, iters,
-                                 ct.byref(ms), _stream(stream)))
+                                 _ptr(out2), ldo2, _ptr(bias), _ptr(aux), ld_aux, int(accumulate), ksplit, bn, pair,
+                                 iters, ct.byref(ms), _stream(stream)))
     return ms.value
 
 

@@ -785,7 +785,7 @@ int gpt2_op_gemm(int dtype, const void* A, int64_t lda, int a_mn, const void* B,
 
 int gpt2_op_gemm_bench(const void* A, int64_t lda, int a_mn, const void* B, int64_t ldb, int b_mn, int M, int N, int K,
                        int epilogue, void* out, int64_t ldo, void* out2, int64_t ldo2, const float* bias,
-                       const void* aux, int64_t ld_aux, int accumulate, int ksplit, int bn, int iters,
+                       const void* aux, int64_t ld_aux, int accumulate, int ksplit, int bn, int pair, int iters,
                        float* ms_out, void* stream) {
   if (iters <= 0 || !ms_out) {
     g_op_error = "gemm_bench: iters > 0 and ms_out required";
@@ -803,6 +803,7 @@ int gpt2_op_gemm_bench(const void* A, int64_t lda, int a_mn, const void* B, int6
   GemmDesc d{A, lda, a_mn != 0, B, ldb, b_mn != 0, M, N, K, epilogue, out, ldo, out2, ldo2, bias, aux, ld_aux,
              accumulate, ksplit < 0 ? 1 : ksplit};
   d.bn = bn;
+  d.pair = pair;
   int r = gemm_tc(o.c, d);  // warm-up (also sets kernel attributes)
   cudaEvent_t e0, e1;
   cudaEventCreate(&e0);

@@ -55,15 +55,22 @@ constexpr int TC_BK = 64;
 constexpr int TC_THREADS = 320;
 constexpr int TC_EPI_WARPS = 8;
 
-template <int BN>
+// PAIR: a 2-CTA cluster computes one (2 * TC_BM) x BN tile with M = 256 MMAs that
+// span both SMs' tensor cores. Each CTA stages its own 128 rows of A and its own
+// BN / 2 rows of B, so a CTA moves 2/3 of the shared-memory and L2 bytes per FLOP
+// that the single-CTA form (128 rows of A, BN rows of B) does.
+template <int BN, bool PAIR = false>
 struct TcCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
-  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows staged by one CTA
+  static constexpr int B_BYTES = B_ROWS * TC_BK * 2;
+  static constexpr int UNIT_M = PAIR ? 2 * TC_BM : TC_BM;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = (192 * 1024) / STAGE;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  static constexpr int STAGING = TC_EPI_WARPS * 4096;  // one 4 KB store buffer per epilogue warp
-  static constexpr int SMEM = STAGES * STAGE + STAGING + 1024 + 256;
+  static constexpr int STAGING = TC_EPI_WARPS * 4096;  // two 2 KB chunk buffers per epilogue warp
+  static constexpr int BARS = 512;                      // mbarriers, TMEM slot, abort flag
+  static constexpr int SMEM = STAGES * STAGE + STAGING + 1024 + BARS;
 };
 
 __device__ __forceinline__ float gelu_tanh_fast(float u) {
@@ -82,44 +89,45 @@ __device__ __forceinline__ float gelu_tanh_grad_fast(float u) {
   return 0.5f * (1.0f + th) + 0.5f * u * (1.0f - th * th) * dinner;
 }
 
-// Output tile of one epilogue warp and chunk: 32 rows (one per lane) x 32 columns,
-// staged in shared memory in the layout of the output tensor map's box:
-//   bf16: 64-byte rows, 64-byte swizzle (16-byte chunk k of row r at chunk k ^ ((r >> 1) & 3))
-//   fp32: 128-byte rows, 128-byte swizzle (chunk k of row r at chunk k ^ (r & 7))
-// Both patterns put the 8 lanes of a 16-byte store phase in distinct banks.
-__device__ __forceinline__ void stage_bf16_row(uint8_t* buf, int r, const float (&v)[32]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int j = k * 8;
-    uint4 w = make_uint4(pack_bf16x2(v[j], v[j + 1]), pack_bf16x2(v[j + 2], v[j + 3]), pack_bf16x2(v[j + 4], v[j + 5]),
-                         pack_bf16x2(v[j + 6], v[j + 7]));
-    *reinterpret_cast<uint4*>(buf + r * 64 + ((k ^ ((r >> 1) & 3)) << 4)) = w;
-  }
-}
-__device__ __forceinline__ void stage_f32_row(uint8_t* buf, int r, const float (&v)[32]) {
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    *reinterpret_cast<float4*>(buf + r * 128 + ((k ^ (r & 7)) << 4)) =
-        make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-}
-
-// Epilogue math on 32 consecutive columns [col0, col0+32) of one row, written into
-// the staging buffer(s) (row `lane`). Columns past N hold don't-care values: the
-// tensor-map store clips them.
+// Epilogue chunks: each epilogue warp turns 32 accumulator rows (one per lane) into
+// one 2 KB output tile at a time, staged in shared memory in exactly the layout
+// of the output tensor map's box:
+//   "row64": 64-byte rows (16 fp32 or 32 bf16 columns), 64-byte swizzle: 16-byte
+//            piece k of row r sits at piece k ^ ((r >> 1) & 3)
+// It puts the 8 lanes of a 16-byte access phase in distinct banks. When the
+// epilogue reads an auxiliary tile (the residual, or the pre-GELU input), TMA
+// loads it into the same buffer beforehand and the result overwrites it in place.
 template <int EPI>
-__device__ __forceinline__ void tc_epilogue_stage(const GemmParams& p, int row, int col0, int lane, float (&v)[32],
+__host__ __device__ constexpr int tc_chunk_cols() {
+  return (EPI == EPI_BF16 || EPI == EPI_BF16_DGELU || EPI == EPI_BF16_GELU) ? 32 : 16;
+}
+// GELU writes two 2 KB outputs per chunk: one 4 KB buffer per warp, no alternation
+template <int EPI>
+__host__ __device__ constexpr bool tc_single_buffer() {
+  return EPI == EPI_BF16_GELU;
+}
+template <int EPI>
+__host__ __device__ constexpr bool tc_has_aux() {
+  return EPI == EPI_F32_RESID || EPI == EPI_BF16_DGELU;
+}
+__device__ __forceinline__ uint8_t* row64_at(uint8_t* buf, int r, int k) {
+  return buf + r * 64 + ((k ^ ((r >> 1) & 3)) << 4);
+}
+template <int EPI, int CW>
+__device__ __forceinline__ void tc_epilogue_chunk(const GemmParams& p, int col0, int lane, float (&v)[CW],
                                                   uint8_t* buf) {
-  const bool full = (col0 + 32 <= p.N);
-  const bool row_ok = row < p.M;
-  if (p.ksplit > 1 || EPI == EPI_F32) {
-    stage_f32_row(buf, lane, v);
+  const bool full = (col0 + CW <= p.N);
+  if (p.ksplit > 1 || EPI == EPI_F32) {  // fp32, 16 columns, row64
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      *reinterpret_cast<float4*>(row64_at(buf, lane, k)) = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
     return;
   }
   if (EPI == EPI_BF16 || EPI == EPI_BF16_GELU || EPI == EPI_F32_RESID) {
     if (p.bias) {
       if (full) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
+        for (int j = 0; j < CW; j += 4) {
           float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + col0 + j));
           v[j] += b.x;
           v[j + 1] += b.y;
@@ -128,59 +136,53 @@ __device__ __forceinline__ void tc_epilogue_stage(const GemmParams& p, int row, 
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < CW; ++j)
           if (col0 + j < p.N) v[j] += p.bias[col0 + j];
       }
     }
   }
-  if (EPI == EPI_BF16) {
-    stage_bf16_row(buf, lane, v);
-  } else if (EPI == EPI_BF16_GELU) {
-    stage_bf16_row(buf, lane, v);
+  if (EPI == EPI_F32_RESID) {  // fp32, 16 columns: out = residual (staged by TMA) + acc + bias
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_fast(v[j]);
-    stage_bf16_row(buf + 2048, lane, v);
-  } else if (EPI == EPI_F32_RESID) {
-    if (row_ok) {
-      const float* res = reinterpret_cast<const float*>(p.aux) + (long long)row * p.ld_aux + col0;
-      if (full) {
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          float4 x = *reinterpret_cast<const float4*>(res + j);
-          v[j] += x.x;
-          v[j + 1] += x.y;
-          v[j + 2] += x.z;
-          v[j + 3] += x.w;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (col0 + j < p.N) v[j] += res[j];
-      }
+    for (int k = 0; k < 4; ++k) {
+      float4* q = reinterpret_cast<float4*>(row64_at(buf, lane, k));
+      const float4 x = *q;
+      *q = make_float4(x.x + v[4 * k], x.y + v[4 * k + 1], x.z + v[4 * k + 2], x.w + v[4 * k + 3]);
     }
-    stage_f32_row(buf, lane, v);
-  } else if (EPI == EPI_BF16_DGELU) {
-    if (row_ok) {
-      const bf16* u = reinterpret_cast<const bf16*>(p.aux) + (long long)row * p.ld_aux + col0;
-      if (full) {
+  } else if (EPI == EPI_BF16) {  // bf16, 32 columns, row64
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
-          uint4 uu = *reinterpret_cast<const uint4*>(u + j);
-          const uint32_t w[4] = {uu.x, uu.y, uu.z, uu.w};
+    for (int k = 0; k < 4; ++k)
+      *reinterpret_cast<uint4*>(row64_at(buf, lane, k)) =
+          make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                     pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+  } else if (EPI == EPI_BF16_DGELU) {  // bf16, 32 columns: out = acc * gelu'(u), u staged by TMA
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f = unpack_bf16x2(w[q]);
-            v[j + 2 * q] *= gelu_tanh_grad_fast(f.x);
-            v[j + 2 * q + 1] *= gelu_tanh_grad_fast(f.y);
-          }
-        }
-      } else {
+    for (int k = 0; k < 4; ++k) {
+      uint4* q = reinterpret_cast<uint4*>(row64_at(buf, lane, k));
+      const uint4 uu = *q;
+      const uint32_t w[4] = {uu.x, uu.y, uu.z, uu.w};
+      uint32_t o[4];
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (col0 + j < p.N) v[j] *= gelu_tanh_grad_fast(__bfloat162float(u[j]));
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = unpack_bf16x2(w[t]);
+        o[t] = pack_bf16x2(v[8 * k + 2 * t] * gelu_tanh_grad_fast(f.x), v[8 * k + 2 * t + 1] * gelu_tanh_grad_fast(f.y));
       }
+      *q = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    stage_bf16_row(buf, lane, v);
+  } else if (EPI == EPI_BF16_GELU) {  // bf16, 32 columns: u at buf, gelu(u) at buf + 2 KB, row64
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      *reinterpret_cast<uint4*>(row64_at(buf, lane, k)) =
+          make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                     pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+    }
+#pragma unroll
+    for (int j = 0; j < CW; ++j) v[j] = gelu_tanh_fast(v[j]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      *reinterpret_cast<uint4*>(row64_at(buf + 2048, lane, k)) =
+          make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                     pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+    }
   }
 }
 
@@ -192,13 +194,22 @@ __device__ __forceinline__ void tc_decode_unit(const GemmParams& p, int unit, in
   tn = t - tm * p.tiles_n;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+// PAIR = true runs as clusters of two CTAs (launch attribute cluster dim 2 x 1 x 1):
+// rank 0 (the leader) issues the M = 256 MMAs for both; both ranks load their halves
+// of each stage, completing on the leader's `full` barrier; the leader's commits
+// arrive on both ranks' `empty` / `tfull` barriers; both ranks' epilogue warps
+// arrive on the leader's `tempty`. No load is multicast.
+template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                    const GemmParams p) {
-  using Cfg = TcCfg<BN>;
+  using Cfg = TcCfg<BN, PAIR>;
   constexpr int STAGES = Cfg::STAGES;
+  constexpr int UNIT_M = Cfg::UNIT_M;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int cid = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // cluster (or CTA) index
+  const int ncl = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + STAGES * Cfg::STAGE;  // 1024-aligned
@@ -209,6 +220,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* auxbar = drain + 2;  // [TC_EPI_WARPS][2]: auxiliary tile landed in chunk buffer 0 / 1
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -220,9 +232,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], TC_EPI_WARPS);
+      mbar_init(&tempty[a], PAIR ? 2 * TC_EPI_WARPS : TC_EPI_WARPS);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 2 * TC_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -231,11 +244,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync();  // the peer's barriers are initialised before anything arrives on them
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t lim = p.timeout_ns;
@@ -247,31 +268,50 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, last_par = 0;  // bit s: stage s has a copy issued / its parity
       bool ok = true;
-      for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x) {
+      for (int unit = cid; unit < p.num_units && ok; unit += ncl) {
         int tm, tn, ks;
         tc_decode_unit(p, unit, tm, tn, ks);
         const int kb0 = ks * p.kb_per_split;
         const int kb1 = min(kb0 + p.kb_per_split, p.num_kb);
+        const int arow = tm * UNIT_M + (int)rank * TC_BM;        // this CTA's rows of A
+        const int brow = tn * BN + (int)rank * Cfg::B_ROWS;      // this CTA's rows of B
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, lim)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE);
+          // the leader expects both CTAs' bytes; the peer's copies complete on the leader's barrier
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], PAIR ? 2 * Cfg::STAGE : Cfg::STAGE);
           uint8_t* sa = smem + stage * Cfg::STAGE;
           uint8_t* sb = sa + Cfg::A_BYTES;
           const int kx = kb * TC_BK;
-          if (!A_MN) {
-            tma_load_2d(sa, &tmA, &full[stage], kx, tm * TC_BM);
-          } else {
-            tma_load_2d(sa, &tmA, &full[stage], tm * TC_BM, kx);
-            tma_load_2d(sa + 8192, &tmA, &full[stage], tm * TC_BM + 64, kx);
-          }
-          if (!B_MN) {
-            tma_load_2d(sb, &tmB, &full[stage], kx, tn * BN);
-          } else {
+          if (PAIR) {
+            const uint32_t fb = cluster_addr(&full[stage], 0);
+            if (!A_MN) {
+              tma_load_2d_pair(sa, &tmA, fb, kx, arow);
+            } else {
+              tma_load_2d_pair(sa, &tmA, fb, arow, kx);
+              tma_load_2d_pair(sa + 8192, &tmA, fb, arow + 64, kx);
+            }
+            if (!B_MN) {
+              tma_load_2d_pair(sb, &tmB, fb, kx, brow);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, &full[stage], tn * BN + j * 64, kx);
+              for (int j = 0; j < Cfg::B_ROWS / 64; ++j) tma_load_2d_pair(sb + j * 8192, &tmB, fb, brow + j * 64, kx);
+            }
+          } else {
+            if (!A_MN) {
+              tma_load_2d(sa, &tmA, &full[stage], kx, arow);
+            } else {
+              tma_load_2d(sa, &tmA, &full[stage], arow, kx);
+              tma_load_2d(sa + 8192, &tmA, &full[stage], arow + 64, kx);
+            }
+            if (!B_MN) {
+              tma_load_2d(sb, &tmB, &full[stage], kx, brow);
+            } else {
+#pragma unroll
+              for (int j = 0; j < Cfg::B_ROWS / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, &full[stage], brow + j * 64, kx);
+            }
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -286,20 +326,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         *abort_flag = 1;
         // let every copy already issued land before the CTA's shared memory goes away
         int never = 0;
-        for (int s = 0; s < STAGES; ++s)
-          if ((issued >> s) & 1u) mbar_wait_bounded(&full[s], (last_par >> s) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+        if (rank == 0) {
+          for (int s = 0; s < STAGES; ++s)
+            if ((issued >> s) & 1u)
+              mbar_wait_bounded(&full[s], (last_par >> s) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+        } else if (issued) {
+          // the peer's copies complete on the leader's barriers, which it cannot wait on:
+          // give them a fixed grace period (a tile copy lands in microseconds)
+          spin_for_ns(2000000ull);
+        }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = make_idesc_bf16(TC_BM, BN, A_MN, B_MN);
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (the leader alone, for a pair) ----------------
+      constexpr uint32_t idesc = make_idesc_bf16(UNIT_M, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true, any = false;
-      for (int unit = blockIdx.x; unit < p.num_units && ok; unit += gridDim.x) {
+      for (int unit = cid; unit < p.num_units && ok; unit += ncl) {
         int tm, tn, ks;
         tc_decode_unit(p, unit, tm, tn, ks);
         const int kb0 = ks * p.kb_per_split;
@@ -324,17 +371,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                      : make_sw128_desc(a_addr + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? make_sw128_desc(b_addr + k * 2048, 8192, 1024)
                                      : make_sw128_desc(b_addr + k * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            if (PAIR)
+              umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           }
           any = true;
-          umma_commit(&empty[stage]);
+          if (PAIR)
+            umma_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
+          else
+            umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if (PAIR)
+          umma_commit_pair_mc(&tfull[acc], 0x3);
+        else
+          umma_commit(&tfull[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
@@ -343,27 +399,44 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         *abort_flag = 1;
         if (any) {  // wait for the MMAs already issued before the TMEM is freed
           int never = 0;
-          umma_commit(drain);
+          if (PAIR)
+            umma_commit_pair(drain);
+          else
+            umma_commit(drain);
           mbar_wait_bounded(drain, 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
   } else {
     // ---------------- epilogue warps ----------------
+    constexpr int CW = tc_chunk_cols<EPI>();
+    constexpr bool HAS_AUX = tc_has_aux<EPI>();
     const int ew = warp - 2;         // 0..7
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int half = ew >> 2;        // which half of the BN columns
-    uint8_t* buf = staging + ew * 4096;
-    // bf16 single-output chunks take 2 KB: two buffers alternate; others take 4 KB
-    constexpr bool two_bufs = (EPI == EPI_BF16 || EPI == EPI_BF16_DGELU);
+    const int c_begin = half * (BN / 2), c_end = (half + 1) * (BN / 2);
+    uint8_t* wbuf = staging + ew * 4096;  // chunk buffers: wbuf, wbuf + 2048
+    uint64_t* abar = auxbar + 2 * ew;
     if (lane == 0) {
-      if (EPI == EPI_BF16_GELU || p.ksplit > 1) tma_prefetch_desc(&tmO2);
+      if (EPI == EPI_BF16_GELU || p.ksplit > 1 || HAS_AUX) tma_prefetch_desc(&tmO2);
       tma_prefetch_desc(&tmO);
+    }
+    // auxiliary tile of the first chunk (tmO2 is the auxiliary map for these epilogues);
+    // lane 0 tracks the loads in flight (bit b: buffer b) for the abort path
+    uint32_t aux_pending = 0, aux_par = 0;
+    const int rbase = (int)rank * TC_BM + q * 32;  // this warp's first row within a unit
+    if (HAS_AUX && lane == 0 && cid < p.num_units) {
+      int tm0, tn0, ks0;
+      tc_decode_unit(p, cid, tm0, tn0, ks0);
+      mbar_arrive_expect_tx(&abar[0], 2048);
+      tma_load_2d(wbuf, &tmO2, &abar[0], tn0 * BN + c_begin, tm0 * UNIT_M + rbase);
+      aux_pending = 1u;
     }
     int acc = 0;
     uint32_t acc_phase = 0;
-    int nchunk = 0;
-    for (int unit = blockIdx.x; unit < p.num_units; unit += gridDim.x) {
+    int n = 0;  // chunks processed by this warp
+    bool ok = true;
+    for (int unit = cid; unit < p.num_units && ok; unit += ncl) {
       int tm, tn, ks;
       tc_decode_unit(p, unit, tm, tn, ks);
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, lim)) {
@@ -374,41 +447,91 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int row0 = tm * TC_BM + q * 32;
-      const int c_begin = half * (BN / 2), c_end = (half + 1) * (BN / 2);
+      const int row0 = tm * UNIT_M + rbase;
 #pragma unroll 1
-      for (int c = c_begin; c < c_end; c += 32, ++nchunk) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c), r);
-        tmem_ld_wait();
-        if (c + 32 == c_end) {  // last read of this accumulator: hand it back to the MMA warp
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
-        }
-        const int col0 = tn * BN + c;
-        uint8_t* b = (two_bufs && (nchunk & 1)) ? buf + 2048 : buf;
-        // the staging buffer must have been read out by the previous store
+      for (int c = c_begin; c < c_end; c += CW, ++n) {
+        const int b = tc_single_buffer<EPI>() ? 0 : (n & 1);
+        uint8_t* cur = wbuf + b * 2048;
         if (lane == 0) {
-          if (two_bufs) bulk_wait_read<1>();
-          else bulk_wait_read<0>();
+          if (HAS_AUX) {
+            // the other buffer's store has been read out: fetch the next chunk's auxiliary tile into it
+            bulk_wait_read<0>();
+            int nrow = -1, ncol = 0;
+            if (c + CW < c_end) {
+              nrow = row0;
+              ncol = tn * BN + c + CW;
+            } else if (unit + ncl < p.num_units) {
+              int tm2, tn2, ks2;
+              tc_decode_unit(p, unit + ncl, tm2, tn2, ks2);
+              nrow = tm2 * UNIT_M + rbase;
+              ncol = tn2 * BN + c_begin;
+            }
+            if (nrow >= 0) {
+              mbar_arrive_expect_tx(&abar[b ^ 1], 2048);
+              tma_load_2d(wbuf + (b ^ 1) * 2048, &tmO2, &abar[b ^ 1], ncol, nrow);
+              aux_pending |= 1u << (b ^ 1);
+              aux_par = (aux_par & ~(1u << (b ^ 1))) | ((uint32_t)(((n + 1) >> 1) & 1) << (b ^ 1));
+            }
+          } else if (tc_single_buffer<EPI>()) {
+            bulk_wait_read<0>();  // the previous chunk's stores have been read out
+          } else {
+            bulk_wait_read<1>();  // this buffer's previous store (two chunks ago) has been read out
+          }
         }
         __syncwarp();
-        float v[32];
+        float v[CW];
+        {
+          uint32_t r[CW];
+          if (CW == 32)
+            tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c),
+                               *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          else
+            tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c),
+                               *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (col0 < p.N) tc_epilogue_stage<EPI>(p, row0 + lane, col0, lane, v, b);
+          for (int j = 0; j < CW; ++j) v[j] = __uint_as_float(r[j]);
+        }
+        if (c + CW == c_end) {  // last read of this accumulator: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (PAIR)
+              mbar_arrive_cluster(cluster_addr(&tempty[acc], 0));
+            else
+              mbar_arrive(&tempty[acc]);
+          }
+        }
+        if (HAS_AUX) {
+          int got = 1;
+          if (lane == 0) {
+            got = mbar_wait_bounded(&abar[b], (n >> 1) & 1, abort_flag, lim) ? 1 : 0;
+            if (got) aux_pending &= ~(1u << b);
+          }
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (!got) {
+            if (lane == 0) {
+              raise_device_error(p.err, DEV_TIMEOUT);
+              *abort_flag = 1;
+            }
+            ok = false;
+            break;
+          }
+          mbar_try_wait(&abar[b], (n >> 1) & 1);  // every lane observes the completed phase
+        }
+        const int col0 = tn * BN + c;
+        if (col0 < p.N) tc_epilogue_chunk<EPI, CW>(p, col0, lane, v, cur);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           if (col0 < p.N && row0 < p.M) {
             if (p.ksplit > 1) {
-              tma_store_3d(&tmO2, b, col0, row0, ks);
+              tma_store_3d(&tmO2, cur, col0, row0, ks);
             } else if (EPI == EPI_F32 && p.accumulate) {
-              tma_reduce_add_2d(&tmO, b, col0, row0);
+              tma_reduce_add_2d(&tmO, cur, col0, row0);
             } else {
-              tma_store_2d(&tmO, b, col0, row0);
-              if (EPI == EPI_BF16_GELU) tma_store_2d(&tmO2, b + 2048, col0, row0);
+              tma_store_2d(&tmO, cur, col0, row0);
+              if (EPI == EPI_BF16_GELU) tma_store_2d(&tmO2, cur + 2048, col0, row0);
             }
           }
           bulk_commit();  // one group per chunk (possibly empty) keeps the buffer accounting exact
@@ -417,15 +540,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
-    if (lane == 0) bulk_wait_all();
+    if (lane == 0) {
+      bulk_wait_all();
+      int never = 0;  // auxiliary loads still in flight (abort path only) land before the CTA exits
+      for (int bb = 0; bb < 2; ++bb)
+        if ((aux_pending >> bb) & 1u)
+          mbar_wait_bounded(&abar[bb], (aux_par >> bb) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+    }
     __syncwarp();
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (PAIR)
+    cluster_sync();  // the leader's MMAs into the peer's TMEM, and remote arrivals, are done
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    if (PAIR)
+      tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
 }
 

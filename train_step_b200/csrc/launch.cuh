@@ -154,20 +154,36 @@ inline bool encode_bf16_map(CUtensorMap* map, const void* ptr, long long inner, 
   return r == CUDA_SUCCESS;
 }
 
-// Epilogue store maps: rows x cols tensor (row stride ld elements), box of 32 x 32,
-// bf16 with 64-byte swizzle or fp32 with 128-byte swizzle (the staging layouts).
+// Epilogue maps: rows x cols tensor (row stride ld elements), box of box_cols x 32
+// rows, matching the epilogue's 2 KB chunk layout: 64-byte rows (16 fp32 or 32 bf16
+// columns) with 64-byte swizzle.
 inline bool encode_out_map(CUtensorMap* map, const void* ptr, long long cols, long long rows, long long ld,
-                           bool is_f32) {
+                           bool is_f32, int box_cols) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const int es = is_f32 ? 4 : 2;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
-  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, 32u};
   cuuint32_t estr[2] = {1u, 1u};
+  const int row_bytes = box_cols * es;
   CUresult r = enc(map, is_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   is_f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Split-K partial workspace [ksplit][rows][cols] fp32 as a 3-D map, box 16 x 32 x 1.
+inline bool encode_partial_map(CUtensorMap* map, const void* ptr, long long cols, long long rows, int ksplit) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)ksplit};
+  cuuint64_t strides[2] = {(cuuint64_t)(cols * 4), (cuuint64_t)(rows * cols * 4)};
+  cuuint32_t box[3] = {16u, 32u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -183,20 +199,6 @@ inline bool encode_qkv_map(CUtensorMap* map, const void* ptr, long long cols, lo
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// Split-K partial workspace [ksplit][rows][cols] fp32 as a 3-D map, box 32 x 32 x 1.
-inline bool encode_partial_map(CUtensorMap* map, const void* ptr, long long cols, long long rows, int ksplit) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)ksplit};
-  cuuint64_t strides[2] = {(cuuint64_t)(cols * 4), (cuuint64_t)(rows * cols * 4)};
-  cuuint32_t box[3] = {32u, 32u, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -224,34 +226,70 @@ struct GemmDesc {
   int ksplit;  // 0 = choose, 1 = none, > 1 = forced
   int role = CAT_GEMM;  // profiler category
   int bn = 0;           // tile width: 0 = choose (256 when N >= 256), else 128 or 256
+  int pair = -1;        // 2-CTA tiles (256 x 256): -1 = choose, 0 = off, 1 = on (needs BN 256)
 };
 
 struct TcMaps {
   CUtensorMap a, b, o, o2;
 };
 
-template <int BN, bool AM, bool BM_, int EPI>
+template <int BN, bool AM, bool BM_, int EPI, bool PAIR>
 int launch_tc_inst(const LaunchCtx& c, const TcMaps& tm, const GemmParams& p) {
-  auto kern = gemm_tc_kernel<BN, AM, BM_, EPI>;
+  auto kern = gemm_tc_kernel<BN, AM, BM_, EPI, PAIR>;
+  constexpr int smem = TcCfg<BN, PAIR>::SMEM;
+  static int max_clusters = 0;  // co-resident clusters (PAIR), once per instantiation
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return fail(c, GPT2_ERR_CUDA, "cudaFuncSetAttribute(gemm_tc) failed");
+    if (PAIR) {
+      cudaLaunchConfig_t q{};
+      q.gridDim = dim3(2 * (c.num_sms / 2));
+      q.blockDim = dim3(TC_THREADS);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = 2;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &q) != cudaSuccess || max_clusters < 1)
+        return fail(c, GPT2_ERR_CUDA, "gemm_tc: no 2-CTA cluster fits");
+    }
     attr_set = true;
   }
-  const int grid = p.num_units < c.num_sms ? p.num_units : c.num_sms;
-  kern<<<grid, TC_THREADS, TcCfg<BN>::SMEM, c.stream>>>(tm.a, tm.b, tm.o, tm.o2, p);
-  return check_launch(c, "gemm_tc");
+  if (!PAIR) {
+    const int grid = p.num_units < c.num_sms ? p.num_units : c.num_sms;
+    kern<<<grid, TC_THREADS, smem, c.stream>>>(tm.a, tm.b, tm.o, tm.o2, p);
+    return check_launch(c, "gemm_tc");
+  }
+  const int clusters = p.num_units < max_clusters ? p.num_units : max_clusters;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tm.a, tm.b, tm.o, tm.o2, p) != cudaSuccess)
+    return fail(c, GPT2_ERR_CUDA, "gemm_tc: cluster launch failed");
+  return check_launch(c, "gemm_tc_pair");
 }
 
-template <int BN, bool AM, bool BM_>
+template <int BN, bool AM, bool BM_, bool PAIR>
 int launch_tc_epi(const LaunchCtx& c, int epi, const TcMaps& tm, const GemmParams& p) {
   switch (epi) {
-    case EPI_BF16: return launch_tc_inst<BN, AM, BM_, EPI_BF16>(c, tm, p);
-    case EPI_BF16_GELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_GELU>(c, tm, p);
-    case EPI_F32_RESID: return launch_tc_inst<BN, AM, BM_, EPI_F32_RESID>(c, tm, p);
-    case EPI_BF16_DGELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_DGELU>(c, tm, p);
-    case EPI_F32: return launch_tc_inst<BN, AM, BM_, EPI_F32>(c, tm, p);
+    case EPI_BF16: return launch_tc_inst<BN, AM, BM_, EPI_BF16, PAIR>(c, tm, p);
+    case EPI_BF16_GELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_GELU, PAIR>(c, tm, p);
+    case EPI_F32_RESID: return launch_tc_inst<BN, AM, BM_, EPI_F32_RESID, PAIR>(c, tm, p);
+    case EPI_BF16_DGELU: return launch_tc_inst<BN, AM, BM_, EPI_BF16_DGELU, PAIR>(c, tm, p);
+    case EPI_F32: return launch_tc_inst<BN, AM, BM_, EPI_F32, PAIR>(c, tm, p);
   }
   return fail(c, GPT2_ERR_CONFIG, "gemm: unknown epilogue");
 }
@@ -262,7 +300,15 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
   if ((d.lda % 8) || (d.ldb % 8) || (reinterpret_cast<uintptr_t>(d.A) & 15) || (reinterpret_cast<uintptr_t>(d.B) & 15))
     return fail(c, GPT2_ERR_CONFIG, "gemm: bf16 operands need 16-byte aligned rows");
   const int BN = d.bn == 128 || d.bn == 256 ? d.bn : (d.N >= 256 ? 256 : 128);
-  const int tiles_m = (d.M + TC_BM - 1) / TC_BM, tiles_n = (d.N + BN - 1) / BN;
+  if (d.pair == 1 && BN != 256) return fail(c, GPT2_ERR_CONFIG, "gemm: 2-CTA tiles need tile width 256");
+  // 2-CTA tiles halve each SM's B-operand traffic; measured on B200 they lose where a short
+  // main loop (K < 1536) meets an epilogue that reads an auxiliary tile (residual / GELU
+  // input), and where the output is too small to keep 74 pairs busy
+  const bool aux_epi = d.epi == EPI_F32_RESID || d.epi == EPI_BF16_DGELU;
+  const bool pair = BN == 256 && (d.pair == 1 || (d.pair < 0 && d.M >= 2 * TC_BM && (!aux_epi || d.K >= 1536) &&
+                                                  (long long)d.M * d.N >= (1LL << 20)));
+  const int unit_m = pair ? 2 * TC_BM : TC_BM;
+  const int tiles_m = (d.M + unit_m - 1) / unit_m, tiles_n = (d.N + BN - 1) / BN;
   const int num_kb = (d.K + TC_BK - 1) / TC_BK;
   int ksplit = d.ksplit;
   if (d.epi != EPI_F32 || !c.splitk_ws) {
@@ -270,9 +316,10 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
     ksplit = 1;
   } else if (ksplit == 0) {
     const int tiles = tiles_m * tiles_n;
+    const int slots = pair ? c.num_sms / 2 : c.num_sms;  // tiles in flight at once
     ksplit = 1;
-    if (tiles < 2 * c.num_sms) {
-      ksplit = (2 * c.num_sms + tiles - 1) / tiles;
+    if (tiles < 2 * slots) {
+      ksplit = (2 * slots + tiles - 1) / tiles;
       if (ksplit > num_kb / 4) ksplit = num_kb / 4;
       if (ksplit > 16) ksplit = 16;
       if (ksplit < 1) ksplit = 1;
@@ -315,23 +362,36 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
   bool ok = d.a_mn ? encode_bf16_map(&tm.a, d.A, d.M, d.K, d.lda, 64)
                    : encode_bf16_map(&tm.a, d.A, d.K, d.M, d.lda, 128);
   ok = ok && (d.b_mn ? encode_bf16_map(&tm.b, d.B, d.N, d.K, d.ldb, 64)
-                     : encode_bf16_map(&tm.b, d.B, d.K, d.N, d.ldb, BN));
-  ok = ok && encode_out_map(&tm.o, d.out, d.N, d.M, d.ldo, out_f32);
-  if (ksplit > 1) ok = ok && encode_partial_map(&tm.o2, c.splitk_ws, d.N, d.M, ksplit);
-  else if (d.epi == EPI_BF16_GELU) ok = ok && encode_out_map(&tm.o2, d.out2, d.N, d.M, d.ldo2, false);
-  else tm.o2 = tm.o;
+                     : encode_bf16_map(&tm.b, d.B, d.K, d.N, d.ldb, pair ? BN / 2 : BN));
+  const int cw = (d.epi == EPI_F32 || d.epi == EPI_F32_RESID) ? 16 : 32;  // epilogue chunk columns
+  ok = ok && encode_out_map(&tm.o, d.out, d.N, d.M, d.ldo, out_f32, cw);
+  if (ksplit > 1) {
+    ok = ok && encode_partial_map(&tm.o2, c.splitk_ws, d.N, d.M, ksplit);
+  } else if (d.epi == EPI_BF16_GELU) {
+    ok = ok && encode_out_map(&tm.o2, d.out2, d.N, d.M, d.ldo2, false, 32);
+  } else if (d.epi == EPI_F32_RESID || d.epi == EPI_BF16_DGELU) {  // the auxiliary input, read by TMA
+    if ((reinterpret_cast<uintptr_t>(d.aux) & 15) || (d.ld_aux * (d.epi == EPI_F32_RESID ? 4 : 2)) % 16)
+      return fail(c, GPT2_ERR_CONFIG, "gemm: the auxiliary input needs 16-byte aligned rows");
+    ok = ok && encode_out_map(&tm.o2, d.aux, d.N, d.M, d.ld_aux, d.epi == EPI_F32_RESID, cw);
+  } else {
+    tm.o2 = tm.o;
+  }
   if (!ok) return fail(c, GPT2_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
   int r;
   {
   ProfScope ps(c, d.role, 2.0 * d.M * d.N * d.K, 0.0);
-  if (BN == 256) {
-    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<256, false, false>(c, d.epi, tm, p);
-    else if (!d.a_mn) r = launch_tc_epi<256, false, true>(c, d.epi, tm, p);
-    else r = launch_tc_epi<256, true, true>(c, d.epi, tm, p);
+  if (pair) {
+    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<256, false, false, true>(c, d.epi, tm, p);
+    else if (!d.a_mn) r = launch_tc_epi<256, false, true, true>(c, d.epi, tm, p);
+    else r = launch_tc_epi<256, true, true, true>(c, d.epi, tm, p);
+  } else if (BN == 256) {
+    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<256, false, false, false>(c, d.epi, tm, p);
+    else if (!d.a_mn) r = launch_tc_epi<256, false, true, false>(c, d.epi, tm, p);
+    else r = launch_tc_epi<256, true, true, false>(c, d.epi, tm, p);
   } else {
-    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<128, false, false>(c, d.epi, tm, p);
-    else if (!d.a_mn) r = launch_tc_epi<128, false, true>(c, d.epi, tm, p);
-    else r = launch_tc_epi<128, true, true>(c, d.epi, tm, p);
+    if (!d.a_mn && !d.b_mn) r = launch_tc_epi<128, false, false, false>(c, d.epi, tm, p);
+    else if (!d.a_mn) r = launch_tc_epi<128, false, true, false>(c, d.epi, tm, p);
+    else r = launch_tc_epi<128, true, true, false>(c, d.epi, tm, p);
   }
   }
   if (r || ksplit == 1) return r;
