@@ -310,83 +310,171 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Backward on tcgen05. Two deterministic kernels (no atomics):
-//   dK/dV: one CTA per (128-key block, batch*head), looping over query blocks i:
-//     S^T = K Q_i^T, dP^T = V dO_i^T                  (M=128, N=128, K=64)
-//     P^T = 2^(S^T*scale*log2e - lse_q*log2e), dS^T = P^T (dP^T - D_q)   (softmax warps)
-//     dV += P^T dO_i, dK += dS^T Q_i                    (M=128, N=64, K=128)
-//   dQ: one CTA per (128-query block, batch*head), looping over key blocks j:
-//     S = Q K_j^T, dP = dO V_j^T; P, dS as above; dQ += dS K_j
-// Warp roles as in the forward (producer, MMA issuer, 8 element-wise warps that
-// split the 128 columns in halves). D_q = rowsum(dO * O) comes precomputed.
+// Backward on tcgen05. Two deterministic kernels (no atomics). Both are
+// persistent (one CTA per SM looping over work items, so an item's loads overlap
+// the previous item's tail) and work in 64-wide units:
+//
+//   dK/dV: item = (128-key block kb, batch*head); units = 64-query halves of the
+//     query blocks kb .. nqb-1, in key-row orientation:
+//       S^T = K Q_u^T, dP^T = V dO_u^T                 (M=128 keys, N=64 queries, K=64)
+//       P^T = 2^(S^T*scale*log2e - lse*log2e), dS^T = P^T (dP^T - D)   (element-wise)
+//       dV += P^T dO_u, dK += dS^T Q_u                 (M=128 keys, N=64, K=64 queries)
+//     lse*log2e and D of a unit's queries are staged in shared memory by the producer warp.
+//   dQ: item = (128-query block qb, batch*head); units = 64-key halves of the key
+//     blocks 0 .. qb, in query-row orientation (lse and D are registers):
+//       S = Q K_u^T, dP = dO V_u^T                     (M=128 queries, N=64 keys, K=64)
+//       dQ += dS K_u                                   (M=128 queries, N=64, K=64 keys)
+//
+// Operands. With both MMA operands in shared memory these small products are
+// bound by shared-memory bandwidth (a 128 x 64 x 16 MMA re-reads a 4 KB A tile
+// for 2 KB of B). So every A operand lives in TMEM: the item's fixed 128-row tiles
+// (Q and dO, or K and V) are copied there once per item by the element-wise warps,
+// which also write P^T / dS^T (dS) there directly; only the 64-row B tiles of each
+// unit are read from shared memory.
+// Pipelining. Every unit streams its own 16 KB stage (two 64-row tiles) through a
+// 7- or 8-deep ring, released as soon as that unit's accumulation MMAs complete,
+// so a stage's copy is issued several units before it is needed (tile loads take
+// 1-3 us under load). The score tiles are double-buffered in TMEM.
+// MMA issue. One thread can issue a 1-SM tcgen05.mma only every ~96 cycles whatever
+// its N (measured on B200), while the tensor pipe overlaps the streams of several
+// threads. So each product has its own issuing thread (lane 0 of its own warp):
+// dK/dV: S^T, dP^T, dV, dK; dQ: S, dP, dQ. The score threads never wait behind the
+// accumulation threads, which wait for the element-wise warps.
+// Warps: 0 TMA producer (lane 0 issues the copies), then the MMA warps (warp 1 owns
+// the TMEM allocation), then 16 element-wise warps: warp w reads TMEM lane quarter
+// w % 4 (32 rows) and column group (w - first) / 4 (16 of the 64 unit columns).
+// D = rowsum(dO * O) comes precomputed. Every wait is bounded (device error word,
+// no trap).
 // ---------------------------------------------------------------------------
-constexpr int FB_STAGES = 3;
-constexpr int FB_THREADS = 320;
-// dK/dV kernel shared memory: K | V | stages (Q_i, dO_i) | P^T | dS^T | L/D [2][2][128] | barriers
-constexpr int FBK_OFF_K = 0;
-constexpr int FBK_OFF_V = FA_TILE;
-constexpr int FBK_OFF_ST = 2 * FA_TILE;
-constexpr int FBK_OFF_P = FBK_OFF_ST + FB_STAGES * 2 * FA_TILE;
-constexpr int FBK_OFF_DS = FBK_OFF_P + FA_P;
-constexpr int FBK_OFF_LD = FBK_OFF_DS + FA_P;
-constexpr int FBK_OFF_BAR = FBK_OFF_LD + 2 * 2 * 128 * 4;
-constexpr int FBK_SMEM = FBK_OFF_BAR + 256 + 1024;
-// dQ kernel shared memory: Q | dO | stages (K_j, V_j) | dS | barriers
-constexpr int FBQ_OFF_Q = 0;
-constexpr int FBQ_OFF_DO = FA_TILE;
-constexpr int FBQ_OFF_ST = 2 * FA_TILE;
-constexpr int FBQ_OFF_DS = FBQ_OFF_ST + FB_STAGES * 2 * FA_TILE;
-constexpr int FBQ_OFF_BAR = FBQ_OFF_DS + FA_P;
-constexpr int FBQ_SMEM = FBQ_OFF_BAR + 256 + 1024;
-// TMEM columns: S (or S^T) 0..127, dP (or dP^T) 128..255, accumulators from 256
+constexpr int FB_EW_WARPS = 16;
+constexpr int FBK_EW0 = 5;  // dK/dV: producer, S^T, dP^T, dV, dK issuers, then element-wise warps
+constexpr int FBQ_EW0 = 4;  // dQ: producer, S, dP, dQ issuers, then element-wise warps
+constexpr int FBK_THREADS = 32 * (FBK_EW0 + FB_EW_WARPS);  // 672
+constexpr int FBQ_THREADS = 32 * (FBQ_EW0 + FB_EW_WARPS);  // 640
+constexpr int FB_HALF = 64 * 128;                  // 8 KB: 64 rows x 64 bf16 (128-byte rows)
+constexpr int FB_UNIT = 2 * FB_HALF;               // 16 KB: a stage (two half tiles) or a 128 x 64 tile
+constexpr int FB_BARS = 512;
+// dK/dV kernel shared memory: K/V [2 items] | stages (Q_u, dO_u) | lse/D per stage | barriers
+constexpr int FBK_NST = 8;
+constexpr int FBK_OFF_KV = 0;
+constexpr int FBK_OFF_ST = 4 * FA_TILE;
+constexpr int FBK_OFF_LD = FBK_OFF_ST + FBK_NST * FB_UNIT;
+constexpr int FBK_OFF_BAR = FBK_OFF_LD + 4096;  // FBK_NST x 512 bytes
+constexpr int FBK_SMEM = FBK_OFF_BAR + FB_BARS + 1024;
+// dQ kernel shared memory: Q/dO [2 items] | stages (K_u, V_u) | barriers
+constexpr int FBQ_NST = 8;
+constexpr int FBQ_OFF_QD = 0;
+constexpr int FBQ_OFF_ST = 4 * FA_TILE;
+constexpr int FBQ_OFF_BAR = FBQ_OFF_ST + FBQ_NST * FB_UNIT;
+constexpr int FBQ_SMEM = FBQ_OFF_BAR + FB_BARS + 1024;
+static_assert(FBK_NST * 512 <= 4096, "lse/D staging");
+static_assert(FBQ_SMEM <= 232448 && FBK_SMEM <= 232448, "shared memory per CTA");
+// TMEM columns (512): score tiles [2 units] x (S 64 | dP 64) at 0 and 128, then
+//   dK/dV: K | V A operands (32 + 32) at 256, P^T at 320, dS^T at 352 (32 each), dV | dK at 384
+//   dQ:    Q | dO A operands (32 + 32) at 256, dS [2 units] at 320 (32 each), dQ [2 items] at 384
+constexpr int FB_SBUF = 2;
+constexpr uint32_t FBK_TM_KV = 256, FBK_TM_P = 320, FBK_TM_DS = 352, FBK_TM_ACC = 384;
+constexpr uint32_t FBQ_TM_Q = 256, FBQ_TM_DS = 320, FBQ_TM_ACC = 384;
 constexpr uint32_t FB_TMEM_COLS = 512;
 
-// 8 consecutive columns (chunk k of half hf) of row r of an element-wise tile.
-__device__ __forceinline__ void fb_store_chunk(uint8_t* buf, int r, int hf, int k, const float (&v)[8]) {
-  uint4 w = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                       pack_bf16x2(v[6], v[7]));
-  *reinterpret_cast<uint4*>(buf + fa_p_off(r, hf * 8 + k)) = w;
+// 16 bf16 values (two 16-byte chunks, chunk index c16 and c16 + 1 of a 64-column row)
+// into row r of a 128-byte-swizzled tile with 128-byte rows.
+__device__ __forceinline__ void fb_store16(uint8_t* tile, int r, int c16, const float (&v)[16]) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = 8 * k;
+    uint4 w = make_uint4(pack_bf16x2(v[e], v[e + 1]), pack_bf16x2(v[e + 2], v[e + 3]),
+                         pack_bf16x2(v[e + 4], v[e + 5]), pack_bf16x2(v[e + 6], v[e + 7]));
+    *reinterpret_cast<uint4*>(tile + r * 128 + (((c16 + k) ^ (r & 7)) << 4)) = w;
+  }
 }
 
-__global__ void __launch_bounds__(FB_THREADS, 1)
-    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                            const float* __restrict__ lse, const float* __restrict__ Dg, bf16* __restrict__ dqkv, int T,
-                            int NH, float scale, int* err, unsigned long long timeout_ns) {
+// 16 bf16 values of one output row (two 16-byte stores)
+__device__ __forceinline__ void fb_store_row16(bf16* dst, const uint32_t (&v)[16], float mul) {
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int e = 8 * k;
+    *reinterpret_cast<uint4*>(dst + e) =
+        make_uint4(pack_bf16x2(__uint_as_float(v[e]) * mul, __uint_as_float(v[e + 1]) * mul),
+                   pack_bf16x2(__uint_as_float(v[e + 2]) * mul, __uint_as_float(v[e + 3]) * mul),
+                   pack_bf16x2(__uint_as_float(v[e + 4]) * mul, __uint_as_float(v[e + 5]) * mul),
+                   pack_bf16x2(__uint_as_float(v[e + 6]) * mul, __uint_as_float(v[e + 7]) * mul));
+  }
+}
+
+// Bounded wait whose result is the same for every lane of the warp (lane 0 waits).
+__device__ __forceinline__ bool fb_warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t lim,
+                                             int lane) {
+  int ok = 1;
+  if (lane == 0) ok = mbar_wait_bounded(bar, parity, abort, lim) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Copy 16 bf16 (columns [cg*16, cg*16 + 16)) of row r of a 128-byte-swizzled tile
+// with 128-byte rows into 8 TMEM columns of the thread's lane, as an MMA A operand.
+__device__ __forceinline__ void fb_row_to_tmem(const uint8_t* tile, int r, int cg, uint32_t taddr) {
+  const uint4 a = *reinterpret_cast<const uint4*>(tile + r * 128 + (((cg * 2) ^ (r & 7)) << 4));
+  const uint4 b = *reinterpret_cast<const uint4*>(tile + r * 128 + (((cg * 2 + 1) ^ (r & 7)) << 4));
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  tmem_st_32x32b_x8(taddr, w);
+}
+// 16 values as 8 packed bf16 pairs into 8 TMEM columns of the thread's lane
+__device__ __forceinline__ void fb_vals_to_tmem(const float (&v)[16], uint32_t taddr) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  tmem_st_32x32b_x8(taddr, w);
+}
+
+
+__global__ void __launch_bounds__(FBK_THREADS, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q64,
+                            const __grid_constant__ CUtensorMap tm_do64, const float* __restrict__ lse,
+                            const float* __restrict__ Dg, bf16* __restrict__ dqkv, int T, int NH, int BH, float scale,
+                            int* err, unsigned long long timeout_ns) {
   extern __shared__ uint8_t fb_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FBK_OFF_BAR);
-  uint64_t* kv_full = bar + 0;
-  uint64_t* st_full = bar + 1;   // [3]
-  uint64_t* st_empty = bar + 4;  // [3]
-  uint64_t* s_full = bar + 7;
-  uint64_t* s_empty = bar + 8;
-  uint64_t* p_full = bar + 9;
-  uint64_t* p_free = bar + 10;
-  uint64_t* acc_full = bar + 11;
-  uint64_t* drain = bar + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 13);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 14);
+  uint64_t* kv_full = bar;                    // [2] K/V tiles landed in shared memory
+  uint64_t* kv_empty = kv_full + 2;           // [2] copied into TMEM by the element-wise warps
+  uint64_t* kva_full = kv_empty + 2;          // K/V A operands written to TMEM (once per item)
+  uint64_t* st_full = kva_full + 1;           // [FBK_NST]
+  uint64_t* st_empty = st_full + FBK_NST;     // [FBK_NST]
+  uint64_t* s_full = st_empty + FBK_NST;      // [FB_SBUF]
+  uint64_t* s_empty = s_full + FB_SBUF;       // [FB_SBUF]
+  uint64_t* p_full = s_empty + FB_SBUF;
+  uint64_t* p_free = p_full + 1;
+  uint64_t* acc_full = p_free + 1;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;            // [4]: one per MMA thread (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 5);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = blockIdx.x;
-  const int bh = blockIdx.y, b = bh / NH, h = bh % NH;
   const int C = NH * 64;
   const int nqb = (T + FA_BM - 1) / FA_BM;
-  const int n = nqb - kb;  // query blocks kb .. nqb-1
+  const int nitems = nqb * BH;  // item = kb * BH + bh: the longest rows (kb = 0) come first
   const uint64_t lim = timeout_ns;
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
-    for (int i = 0; i < FB_STAGES; ++i) {
-      mbar_init(&st_full[i], 1);
-      mbar_init(&st_empty[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], FB_EW_WARPS);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_empty, 8);
-    mbar_init(p_full, 8);
-    mbar_init(p_free, 1);
-    mbar_init(acc_full, 1);
-    mbar_init(drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&drain[i], 1);
+    mbar_init(kva_full, FB_EW_WARPS);
+    for (int i = 0; i < FBK_NST; ++i) {
+      mbar_init(&st_full[i], 32);  // the producer warp's lanes (lane 0 with the copy bytes)
+      mbar_init(&st_empty[i], 2);  // the dV and dK threads
+    }
+    for (int i = 0; i < FB_SBUF; ++i) {
+      mbar_init(&s_full[i], 2);  // the S^T and dP^T threads
+      mbar_init(&s_empty[i], FB_EW_WARPS);
+    }
+    mbar_init(p_full, FB_EW_WARPS);
+    mbar_init(p_free, 2);  // the dV and dK threads
+    mbar_init(acc_full, 2);
+    mbar_init(acc_empty, FB_EW_WARPS);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -400,191 +488,256 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
+    // ---------------- producer: K/V per item; (Q_u, dO_u, lse, D) per unit ----------------
     if (lane == 0) {
-      tma_prefetch_desc(&tm_qkv);
-      tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(kv_full, 2 * FA_TILE);
-      tma_load_3d(sm + FBK_OFF_K, &tm_qkv, kv_full, C + h * 64, kb * FA_BN, b);
-      tma_load_3d(sm + FBK_OFF_V, &tm_qkv, kv_full, 2 * C + h * 64, kb * FA_BN, b);
-      bool ok = true;
-      uint32_t issued = 0, par = 0;
-      for (int t = 0; t < n; ++t) {
-        const int qi = kb + t, st = t % FB_STAGES;
-        const uint32_t ph = (uint32_t)((t / FB_STAGES) & 1);
-        if (!mbar_wait_bounded(&st_empty[st], ph ^ 1, abort_flag, lim)) {
+      tma_prefetch_desc(&tm_kv);
+      tma_prefetch_desc(&tm_q64);
+      tma_prefetch_desc(&tm_do64);
+    }
+    bool ok = true;
+    uint32_t kv_iss = 0, kv_par = 0, st_iss = 0, st_par = 0;  // lane 0: copies in flight, for the abort path
+    int U = 0;                                                 // unit (= stage use) counter over all items
+    for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+      const int kb = item / BH, bh = item - kb * BH, b = bh / NH, h = bh - b * NH;
+      const int kvb = it & 1;
+      if (!(ok = fb_warp_wait(&kv_empty[kvb], ((it >> 1) & 1) ^ 1, abort_flag, lim, lane))) break;
+      if (lane == 0) {
+        uint8_t* kd = sm + FBK_OFF_KV + kvb * 2 * FA_TILE;
+        mbar_arrive_expect_tx(&kv_full[kvb], 2 * FA_TILE);
+        tma_load_3d(kd, &tm_kv, &kv_full[kvb], C + h * 64, kb * FA_BN, b);
+        tma_load_3d(kd + FA_TILE, &tm_kv, &kv_full[kvb], 2 * C + h * 64, kb * FA_BN, b);
+        kv_iss |= 1u << kvb;
+        kv_par = (kv_par & ~(1u << kvb)) | ((uint32_t)((it >> 1) & 1) << kvb);
+      }
+      const float* lse_bh = lse + (long long)bh * T;
+      const float* D_bh = Dg + (long long)bh * T;
+      for (int q0 = kb * FA_BM; q0 < nqb * FA_BM; q0 += 64, ++U) {
+        const int s = U % FBK_NST;
+        const uint32_t ph = (uint32_t)((U / FBK_NST) & 1);
+        if (!(ok = fb_warp_wait(&st_empty[s], ph ^ 1, abort_flag, lim, lane))) break;
+        float* ld = reinterpret_cast<float*>(sm + FBK_OFF_LD + s * 512);  // [lse*log2e 64][D 64]
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int c = lane * 2 + k, q = q0 + c;
+          ld[c] = q < T ? lse_bh[q] * LOG2E : INFINITY;  // P = 0 for queries past the end
+          ld[64 + c] = q < T ? D_bh[q] : 0.f;
+        }
+        if (lane == 0) {
+          uint8_t* d = sm + FBK_OFF_ST + s * FB_UNIT;
+          mbar_arrive_expect_tx(&st_full[s], FB_UNIT);
+          tma_load_3d(d, &tm_q64, &st_full[s], h * 64, q0, b);
+          tma_load_3d(d + FB_HALF, &tm_do64, &st_full[s], h * 64, q0, b);
+          st_iss |= 1u << s;
+          st_par = (st_par & ~(1u << s)) | (ph << s);
+        } else {
+          mbar_arrive(&st_full[s]);
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      raise_device_error(err, DEV_TIMEOUT);
+      *abort_flag = 1;
+      int never = 0;  // let the copies in flight land before the CTA's shared memory goes away
+      for (int i = 0; i < 2; ++i)
+        if ((kv_iss >> i) & 1u)
+          mbar_wait_bounded(&kv_full[i], (kv_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+      for (int i = 0; i < FBK_NST; ++i)
+        if ((st_iss >> i) & 1u)
+          mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+    }
+  } else if (warp == 1 || warp == 2) {
+    if (lane == 0) {
+      // ---------------- score MMAs: S^T = K Q_u^T (warp 1), dP^T = V dO_u^T (warp 2); A from TMEM ----------------
+      const int part = warp - 1;
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64, false, false);
+      bool ok = true, any = false;
+      int U = 0;
+      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+        const int nu = 2 * (nqb - item / BH);
+        if (!mbar_wait_bounded(kva_full, it & 1, abort_flag, lim)) {
           ok = false;
           break;
         }
-        uint8_t* d = sm + FBK_OFF_ST + st * 2 * FA_TILE;
-        mbar_arrive_expect_tx(&st_full[st], 2 * FA_TILE);
-        tma_load_3d(d, &tm_qkv, &st_full[st], h * 64, qi * FA_BM, b);
-        tma_load_3d(d + FA_TILE, &tm_do, &st_full[st], h * 64, qi * FA_BM, b);
-        issued |= 1u << st;
-        par = (par & ~(1u << st)) | (ph << st);
+        for (int u = 0; u < nu; ++u, ++U) {
+          const int s = U % FBK_NST, sb = U % FB_SBUF;
+          if (!mbar_wait_bounded(&st_full[s], (U / FBK_NST) & 1, abort_flag, lim) ||
+              !mbar_wait_bounded(&s_empty[sb], ((U / FB_SBUF) & 1) ^ 1, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // B = Q_u (part 0) or dO_u (part 1): 64 rows, K-major
+          const uint32_t b_addr = smem_u32(sm + FBK_OFF_ST + s * FB_UNIT) + part * FB_HALF;
+          const uint32_t d = tmem + (uint32_t)(sb * 128 + part * 64);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_ts(d, tmem + FBK_TM_KV + part * 32 + k * 8, make_sw128_desc(b_addr + k * 32, 16, 1024), idesc_s,
+                         k > 0 ? 1u : 0u);
+          umma_commit(&s_full[sb]);
+          any = true;
+        }
       }
       if (!ok) {
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
-        int never = 0;
-        mbar_wait_bounded(kv_full, 0, reinterpret_cast<volatile int*>(&never), lim);
-        for (int s2 = 0; s2 < FB_STAGES; ++s2)
-          if ((issued >> s2) & 1u)
-            mbar_wait_bounded(&st_full[s2], (par >> s2) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+        if (any) {  // wait for the MMAs already issued before the TMEM is freed
+          int never = 0;
+          umma_commit(&drain[part]);
+          mbar_wait_bounded(&drain[part], 0, reinterpret_cast<volatile int*>(&never), lim);
+        }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 3 || warp == 4) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_o = make_idesc_bf16(128, 64, false, true);
-      const uint32_t k_addr = smem_u32(sm + FBK_OFF_K), v_addr = smem_u32(sm + FBK_OFF_V);
-      const uint32_t p_addr = smem_u32(sm + FBK_OFF_P), ds_addr = smem_u32(sm + FBK_OFF_DS);
-      bool ok = mbar_wait_bounded(kv_full, 0, abort_flag, lim);
-      bool any = false;
-      for (int t = 0; t <= n && ok; ++t) {
-        if (t < n) {  // S^T = K Q_t^T, dP^T = V dO_t^T
-          const int st = t % FB_STAGES;
-          if (!mbar_wait_bounded(&st_full[st], (t / FB_STAGES) & 1, abort_flag, lim) ||
-              !mbar_wait_bounded(s_empty, (t & 1) ^ 1, abort_flag, lim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t q_addr = smem_u32(sm + FBK_OFF_ST + st * 2 * FA_TILE), do_addr = q_addr + FA_TILE;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem, make_sw128_desc(k_addr + k * 32, 16, 1024), make_sw128_desc(q_addr + k * 32, 16, 1024),
-                      idesc_s, k > 0 ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem + 128, make_sw128_desc(v_addr + k * 32, 16, 1024),
-                      make_sw128_desc(do_addr + k * 32, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
-          umma_commit(s_full);
-          any = true;
+      // ---------------- accumulation MMAs: dV += P^T dO_u (warp 3), dK += dS^T Q_u (warp 4); A from TMEM ----------------
+      const int part = warp - 3;
+      constexpr uint32_t idesc_a = make_idesc_bf16(128, 64, false, true);  // B = dO_u / Q_u, MN-major
+      bool ok = true, any = false;
+      int U = 0;
+      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+        const int nu = 2 * (nqb - item / BH);
+        // the element-wise warps have read the previous item's dV / dK
+        if (!mbar_wait_bounded(acc_empty, (it & 1) ^ 1, abort_flag, lim)) {
+          ok = false;
+          break;
         }
-        if (t >= 1) {  // dV += P^T dO, dK += dS^T Q for the previous query block
-          const int i = t - 1, st = i % FB_STAGES;
-          if (!mbar_wait_bounded(p_full, i & 1, abort_flag, lim)) {
+        for (int u = 0; u < nu; ++u, ++U) {
+          const int s = U % FBK_NST;
+          if (!mbar_wait_bounded(&st_full[s], (U / FBK_NST) & 1, abort_flag, lim) ||
+              !mbar_wait_bounded(p_full, U & 1, abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t q_addr = smem_u32(sm + FBK_OFF_ST + st * 2 * FA_TILE), do_addr = q_addr + FA_TILE;
+          // K = 64 queries: A = P^T (part 0) or dS^T (part 1); B = 16 query rows of dO_u (part 0)
+          // or Q_u (part 1) per step (MN-major)
+          const uint32_t b_addr = smem_u32(sm + FBK_OFF_ST + s * FB_UNIT) + (1 - part) * FB_HALF;
+          const uint32_t a_tm = tmem + (part == 0 ? FBK_TM_P : FBK_TM_DS);
+          const uint32_t acc = tmem + FBK_TM_ACC + part * 64;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tmem + 256, make_sw128_desc(p_addr + (kk >> 2) * (FA_BM * 128) + (kk & 3) * 32, 16, 1024),
-                      make_sw128_desc(do_addr + kk * 2048, 8192, 1024), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tmem + 320, make_sw128_desc(ds_addr + (kk >> 2) * (FA_BM * 128) + (kk & 3) * 32, 16, 1024),
-                      make_sw128_desc(q_addr + kk * 2048, 8192, 1024), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_ts(acc, a_tm + k * 8, make_sw128_desc(b_addr + k * 2048, 8192, 1024), idesc_a,
+                         (u > 0 || k > 0) ? 1u : 0u);
+          any = true;
           umma_commit(p_free);
-          umma_commit(&st_empty[st]);
+          // the unit's scores were consumed before P^T was written: its score MMAs are complete
+          umma_commit(&st_empty[s]);
+          if (u == nu - 1) umma_commit(acc_full);
         }
       }
-      if (ok) umma_commit(acc_full);
       if (!ok) {
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
         if (any) {
           int never = 0;
-          umma_commit(drain);
-          mbar_wait_bounded(drain, 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[2 + part]);
+          mbar_wait_bounded(&drain[2 + part], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
   } else {
-    // element-wise warps: thread = key row r, queries [hf*64, hf*64 + 64) of the block
-    const int hf = (warp - 2) >> 2, q4 = warp & 3;
+    // ---------------- element-wise warps: key row r, query columns [cg*16, cg*16 + 16) of each unit ----------------
+    const int q4 = warp & 3, cg = (warp - FBK_EW0) >> 2;
     const int r = q4 * 32 + lane;
-    const int key = kb * FA_BN + r;
-    const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-    float* ldb = reinterpret_cast<float*>(sm + FBK_OFF_LD);  // [2][L or D][128]
-    const float* lse_bh = lse + (long long)bh * T;
-    const float* D_bh = Dg + (long long)bh * T;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * LOG2E;
-    const int tid8 = threadIdx.x - 64;  // 0..255
     bool fail = false;
-    for (int t = 0; t < n; ++t) {
-      const int qi = kb + t, buf = t & 1;
-      {  // stage this query block's lse (log2 units) and D in shared memory
-        const int idx = tid8 & 127, which = tid8 >> 7;
-        const int q = qi * FA_BM + idx;
-        float v = 0.f;
-        if (q < T) v = which == 0 ? lse_bh[q] * LOG2E : D_bh[q];
-        ldb[(buf * 2 + which) * 128 + idx] = v;
-      }
-      if (!fail && !mbar_wait_bounded(s_full, t & 1, abort_flag, lim)) fail = true;
-      uint32_t sv[64], dv[64];
-      if (!fail) {
-        tc_fence_after();
-        tmem_ld_32x32b_x32(lane_base + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld_32x32b_x32(lane_base + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_32x32b_x32(lane_base + 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
-        tmem_ld_32x32b_x32(lane_base + 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) sv[e] = dv[e] = 0u;
-      }
+    int U = 0;
+    // K and V rows of item `it` into the TMEM A operands (after the previous item's score
+    // MMAs, whose results this warp has all seen)
+    auto load_operands = [&](int it) -> bool {
+      const int kvb = it & 1;
+      if (!mbar_wait_bounded(&kv_full[kvb], (it >> 1) & 1, abort_flag, lim)) return false;
+      const uint8_t* kd = sm + FBK_OFF_KV + kvb * 2 * FA_TILE;
+      fb_row_to_tmem(kd, r, cg, tmem + lane_off + FBK_TM_KV + cg * 8);
+      fb_row_to_tmem(kd + FA_TILE, r, cg, tmem + lane_off + FBK_TM_KV + 32 + cg * 8);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty);
-      if (named_barrier_or(1, 256, fail || *abort_flag)) {  // also publishes the L/D stage
+      if (lane == 0) {
+        mbar_arrive(kva_full);
+        mbar_arrive(&kv_empty[kvb]);
+      }
+      return true;
+    };
+    if ((int)blockIdx.x < nitems) fail = !load_operands(0);
+    for (int it = 0, item = blockIdx.x; item < nitems && !fail; ++it, item += gridDim.x) {
+      const int kb = item / BH, bh = item - kb * BH, b = bh / NH, h = bh - b * NH;
+      const int nu = 2 * (nqb - kb);
+      for (int u = 0; u < nu; ++u, ++U) {
+        const int sb = U % FB_SBUF, s = U % FBK_NST;
+        // the producer's lse / D of this unit (acquired directly from its lanes), then the scores
+        if (!mbar_wait_bounded(&st_full[s], (U / FBK_NST) & 1, abort_flag, lim) ||
+            !mbar_wait_bounded(&s_full[sb], (U / FB_SBUF) & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[16], dv[16];
+        tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(sb * 128 + cg * 16), sv);
+        tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(sb * 128 + 64 + cg * 16), dv);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[sb]);
+        const float* ld = reinterpret_cast<const float*>(sm + FBK_OFF_LD + s * 512) + cg * 16;
+        float p[16], ds[16];
+        const int qcol0 = (u & 1) * 64 + cg * 16;  // query index within the block of column 0
+        const bool diag = u < 2;                    // the query block kb itself
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const float4 L4 = *reinterpret_cast<const float4*>(ld + 4 * e4);
+          const float4 D4 = *reinterpret_cast<const float4*>(ld + 64 + 4 * e4);
+          const float Lv[4] = {L4.x, L4.y, L4.z, L4.w}, Dv[4] = {D4.x, D4.y, D4.z, D4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int e = 4 * e4 + i;
+            float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -Lv[i]));
+            if (diag && r > qcol0 + e) pe = 0.f;  // key after query
+            p[e] = pe;
+            ds[e] = pe * (__uint_as_float(dv[e]) - Dv[i]);
+          }
+        }
+        // the previous unit's dV / dK MMAs have finished reading P^T and dS^T
+        if (!mbar_wait_bounded(p_free, (U & 1) ^ 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        fb_vals_to_tmem(p, tmem + lane_off + FBK_TM_P + cg * 8);
+        fb_vals_to_tmem(ds, tmem + lane_off + FBK_TM_DS + cg * 8);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      if (fail) break;
+      // the next item's K / V first (lets its score MMAs start), then this item's dV / dK
+      if (item + (int)gridDim.x < nitems && !load_operands(it + 1)) {
         fail = true;
         break;
       }
-      const float* Lq = ldb + (buf * 2 + 0) * 128 + hf * 64;
-      const float* Dq = ldb + (buf * 2 + 1) * 128 + hf * 64;
-      const bool diag = (t == 0);  // queries qi*128 + c with qi == kb
-      if (!fail && !mbar_wait_bounded(p_free, (t & 1) ^ 1, abort_flag, lim)) fail = true;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float pv[8], dsv[8];
-#pragma unroll
-        for (int e8 = 0; e8 < 8; ++e8) {
-          const int e = 8 * k + e8;
-          float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -Lq[e]));
-          if (diag && hf * 64 + e < r) pe = 0.f;  // query before key
-          pv[e8] = pe;
-          dsv[e8] = pe * (__uint_as_float(dv[e]) - Dq[e]);
-        }
-        fb_store_chunk(sm + FBK_OFF_P, r, hf, k, pv);
-        fb_store_chunk(sm + FBK_OFF_DS, r, hf, k, dsv);
+      if (!mbar_wait_bounded(acc_full, it & 1, abort_flag, lim)) {
+        fail = true;
+        break;
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    if (!fail && !mbar_wait_bounded(acc_full, 0, abort_flag, lim)) fail = true;
-    if (named_barrier_or(1, 256, fail || *abort_flag)) {
-      if (lane == 0) {
-        raise_device_error(err, DEV_TIMEOUT);
-        *abort_flag = 1;
-      }
-    } else {
       tc_fence_after();
-      uint32_t v[32], k[32];
-      tmem_ld_32x32b_x32(lane_base + 256 + hf * 32, v);
-      tmem_ld_32x32b_x32(lane_base + 320 + hf * 32, k);
+      uint32_t v[16], k[16];
+      tmem_ld_32x32b_x16(tmem + lane_off + FBK_TM_ACC + (uint32_t)(cg * 16), v);
+      tmem_ld_32x32b_x16(tmem + lane_off + FBK_TM_ACC + (uint32_t)(64 + cg * 16), k);
       tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      const int key = kb * FA_BN + r;
       if (key < T) {
-        bf16* dk = dqkv + ((long long)b * T + key) * 3 * C + C + h * 64 + hf * 32;
-        bf16* dvp = dk + C;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int e = 8 * q;
-          *reinterpret_cast<uint4*>(dvp + e) =
-              make_uint4(pack_bf16x2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
-                         pack_bf16x2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
-                         pack_bf16x2(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5])),
-                         pack_bf16x2(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7])));
-          *reinterpret_cast<uint4*>(dk + e) =
-              make_uint4(pack_bf16x2(__uint_as_float(k[e]) * scale, __uint_as_float(k[e + 1]) * scale),
-                         pack_bf16x2(__uint_as_float(k[e + 2]) * scale, __uint_as_float(k[e + 3]) * scale),
-                         pack_bf16x2(__uint_as_float(k[e + 4]) * scale, __uint_as_float(k[e + 5]) * scale),
-                         pack_bf16x2(__uint_as_float(k[e + 6]) * scale, __uint_as_float(k[e + 7]) * scale));
-        }
+        bf16* dk = dqkv + ((long long)b * T + key) * 3 * C + C + h * 64 + cg * 16;
+        fb_store_row16(dk + C, v, 1.0f);
+        fb_store_row16(dk, k, scale);
       }
+    }
+    if (fail && lane == 0) {
+      raise_device_error(err, DEV_TIMEOUT);
+      *abort_flag = 1;
     }
   }
 
@@ -596,44 +749,54 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
   }
 }
 
-__global__ void __launch_bounds__(FB_THREADS, 1)
-    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                          const float* __restrict__ lse, const float* __restrict__ Dg, bf16* __restrict__ dqkv, int T,
-                          int NH, float scale, int* err, unsigned long long timeout_ns) {
+__global__ void __launch_bounds__(FBQ_THREADS, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ CUtensorMap tm_kv64, const float* __restrict__ lse,
+                          const float* __restrict__ Dg, bf16* __restrict__ dqkv, int T, int NH, int BH, float scale,
+                          int* err, unsigned long long timeout_ns) {
   extern __shared__ uint8_t fb_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FBQ_OFF_BAR);
-  uint64_t* q_full = bar + 0;
-  uint64_t* st_full = bar + 1;   // [3]
-  uint64_t* st_empty = bar + 4;  // [3]
-  uint64_t* s_full = bar + 7;
-  uint64_t* s_empty = bar + 8;
-  uint64_t* ds_full = bar + 9;
-  uint64_t* ds_free = bar + 10;
-  uint64_t* acc_full = bar + 11;
-  uint64_t* drain = bar + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 13);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 14);
+  uint64_t* qd_full = bar;                    // [2] Q/dO tiles landed in shared memory
+  uint64_t* qd_empty = qd_full + 2;           // [2] copied into TMEM by the element-wise warps
+  uint64_t* qa_full = qd_empty + 2;           // Q/dO A operands written to TMEM (once per item)
+  uint64_t* st_full = qa_full + 1;            // [FBQ_NST]
+  uint64_t* st_empty = st_full + FBQ_NST;     // [FBQ_NST]
+  uint64_t* s_full = st_empty + FBQ_NST;      // [FB_SBUF]
+  uint64_t* s_empty = s_full + FB_SBUF;       // [FB_SBUF]
+  uint64_t* ds_full = s_empty + FB_SBUF;      // [2]
+  uint64_t* ds_free = ds_full + 2;            // [2]
+  uint64_t* acc_full = ds_free + 2;           // [2]
+  uint64_t* acc_empty = acc_full + 2;         // [2]
+  uint64_t* drain = acc_empty + 2;            // [3]: one per MMA thread (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  const int bh = blockIdx.y, b = bh / NH, h = bh % NH;
   const int C = NH * 64;
-  const int nkb = qb + 1;
+  const int nqb = (T + FA_BM - 1) / FA_BM;
+  const int nitems = nqb * BH;  // item w: query block nqb - 1 - w / BH (longest rows first), bh = w % BH
   const uint64_t lim = timeout_ns;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int i = 0; i < FB_STAGES; ++i) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&qd_full[i], 1);
+      mbar_init(&qd_empty[i], FB_EW_WARPS);
+      mbar_init(&ds_full[i], FB_EW_WARPS);
+      mbar_init(&ds_free[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], FB_EW_WARPS);
+    }
+    for (int i = 0; i < 3; ++i) mbar_init(&drain[i], 1);
+    mbar_init(qa_full, FB_EW_WARPS);
+    for (int i = 0; i < FBQ_NST; ++i) {
       mbar_init(&st_full[i], 1);
       mbar_init(&st_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_empty, 8);
-    mbar_init(ds_full, 8);
-    mbar_init(ds_free, 1);
-    mbar_init(acc_full, 1);
-    mbar_init(drain, 1);
+    for (int i = 0; i < FB_SBUF; ++i) {
+      mbar_init(&s_full[i], 2);  // the S and dP threads
+      mbar_init(&s_empty[i], FB_EW_WARPS);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -648,162 +811,247 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tm_qkv);
+      // ---------------- producer: Q/dO per item, (K_u, V_u) per unit ----------------
+      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(q_full, 2 * FA_TILE);
-      tma_load_3d(sm + FBQ_OFF_Q, &tm_qkv, q_full, h * 64, qb * FA_BM, b);
-      tma_load_3d(sm + FBQ_OFF_DO, &tm_do, q_full, h * 64, qb * FA_BM, b);
+      tma_prefetch_desc(&tm_kv64);
       bool ok = true;
-      uint32_t issued = 0, par = 0;
-      for (int j = 0; j < nkb; ++j) {
-        const int st = j % FB_STAGES;
-        const uint32_t ph = (uint32_t)((j / FB_STAGES) & 1);
-        if (!mbar_wait_bounded(&st_empty[st], ph ^ 1, abort_flag, lim)) {
+      uint32_t qd_iss = 0, qd_par = 0, st_iss = 0, st_par = 0;
+      int U = 0;
+      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+        const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
+        const int qdb = it & 1;
+        if (!mbar_wait_bounded(&qd_empty[qdb], ((it >> 1) & 1) ^ 1, abort_flag, lim)) {
           ok = false;
           break;
         }
-        uint8_t* d = sm + FBQ_OFF_ST + st * 2 * FA_TILE;
-        mbar_arrive_expect_tx(&st_full[st], 2 * FA_TILE);
-        tma_load_3d(d, &tm_qkv, &st_full[st], C + h * 64, j * FA_BN, b);
-        tma_load_3d(d + FA_TILE, &tm_qkv, &st_full[st], 2 * C + h * 64, j * FA_BN, b);
-        issued |= 1u << st;
-        par = (par & ~(1u << st)) | (ph << st);
+        uint8_t* qd = sm + FBQ_OFF_QD + qdb * 2 * FA_TILE;
+        mbar_arrive_expect_tx(&qd_full[qdb], 2 * FA_TILE);
+        tma_load_3d(qd, &tm_q, &qd_full[qdb], h * 64, qb * FA_BM, b);
+        tma_load_3d(qd + FA_TILE, &tm_do, &qd_full[qdb], h * 64, qb * FA_BM, b);
+        qd_iss |= 1u << qdb;
+        qd_par = (qd_par & ~(1u << qdb)) | ((uint32_t)((it >> 1) & 1) << qdb);
+        for (int k0 = 0; k0 < (qb + 1) * FA_BN; k0 += 64, ++U) {
+          const int s = U % FBQ_NST;
+          const uint32_t ph = (uint32_t)((U / FBQ_NST) & 1);
+          if (!mbar_wait_bounded(&st_empty[s], ph ^ 1, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          uint8_t* d = sm + FBQ_OFF_ST + s * FB_UNIT;
+          mbar_arrive_expect_tx(&st_full[s], FB_UNIT);
+          tma_load_3d(d, &tm_kv64, &st_full[s], C + h * 64, k0, b);
+          tma_load_3d(d + FB_HALF, &tm_kv64, &st_full[s], 2 * C + h * 64, k0, b);
+          st_iss |= 1u << s;
+          st_par = (st_par & ~(1u << s)) | (ph << s);
+        }
       }
       if (!ok) {
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
         int never = 0;
-        mbar_wait_bounded(q_full, 0, reinterpret_cast<volatile int*>(&never), lim);
-        for (int s2 = 0; s2 < FB_STAGES; ++s2)
-          if ((issued >> s2) & 1u)
-            mbar_wait_bounded(&st_full[s2], (par >> s2) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+        for (int i = 0; i < 2; ++i)
+          if ((qd_iss >> i) & 1u)
+            mbar_wait_bounded(&qd_full[i], (qd_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+        for (int i = 0; i < FBQ_NST; ++i)
+          if ((st_iss >> i) & 1u)
+            mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_o = make_idesc_bf16(128, 64, false, true);
-      const uint32_t q_addr = smem_u32(sm + FBQ_OFF_Q), do_addr = smem_u32(sm + FBQ_OFF_DO);
-      const uint32_t ds_addr = smem_u32(sm + FBQ_OFF_DS);
-      bool ok = mbar_wait_bounded(q_full, 0, abort_flag, lim);
-      bool any = false;
-      for (int j = 0; j <= nkb && ok; ++j) {
-        if (j < nkb) {  // S = Q K_j^T, dP = dO V_j^T
-          const int st = j % FB_STAGES;
-          if (!mbar_wait_bounded(&st_full[st], (j / FB_STAGES) & 1, abort_flag, lim) ||
-              !mbar_wait_bounded(s_empty, (j & 1) ^ 1, abort_flag, lim)) {
+      // ---------------- score MMAs: S = Q K_u^T (warp 1), dP = dO V_u^T (warp 2); A from TMEM ----------------
+      const int part = warp - 1;
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64, false, false);
+      bool ok = true, any = false;
+      int U = 0;
+      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+        const int nu = 2 * (nqb - item / BH);
+        if (!mbar_wait_bounded(qa_full, it & 1, abort_flag, lim)) {
+          ok = false;
+          break;
+        }
+        for (int u = 0; u < nu; ++u, ++U) {
+          const int s = U % FBQ_NST, sb = U % FB_SBUF;
+          if (!mbar_wait_bounded(&st_full[s], (U / FBQ_NST) & 1, abort_flag, lim) ||
+              !mbar_wait_bounded(&s_empty[sb], ((U / FB_SBUF) & 1) ^ 1, abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm + FBQ_OFF_ST + st * 2 * FA_TILE), v_addr = k_addr + FA_TILE;
+          // B = K_u (part 0) or V_u (part 1): 64 rows, K-major
+          const uint32_t b_addr = smem_u32(sm + FBQ_OFF_ST + s * FB_UNIT) + part * FB_HALF;
+          const uint32_t d = tmem + (uint32_t)(sb * 128 + part * 64);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem, make_sw128_desc(q_addr + k * 32, 16, 1024), make_sw128_desc(k_addr + k * 32, 16, 1024),
-                      idesc_s, k > 0 ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem + 128, make_sw128_desc(do_addr + k * 32, 16, 1024),
-                      make_sw128_desc(v_addr + k * 32, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
-          umma_commit(s_full);
+            umma_bf16_ts(d, tmem + FBQ_TM_Q + part * 32 + k * 8, make_sw128_desc(b_addr + k * 32, 16, 1024), idesc_s,
+                         k > 0 ? 1u : 0u);
+          umma_commit(&s_full[sb]);
           any = true;
         }
-        if (j >= 1) {  // dQ += dS K for the previous key block
-          const int i = j - 1, st = i % FB_STAGES;
-          if (!mbar_wait_bounded(ds_full, i & 1, abort_flag, lim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm + FBQ_OFF_ST + st * 2 * FA_TILE);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tmem + 256, make_sw128_desc(ds_addr + (kk >> 2) * (FA_BM * 128) + (kk & 3) * 32, 16, 1024),
-                      make_sw128_desc(k_addr + kk * 2048, 8192, 1024), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(ds_free);
-          umma_commit(&st_empty[st]);
-        }
       }
-      if (ok) umma_commit(acc_full);
       if (!ok) {
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
         if (any) {
           int never = 0;
-          umma_commit(drain);
-          mbar_wait_bounded(drain, 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[part]);
+          mbar_wait_bounded(&drain[part], 0, reinterpret_cast<volatile int*>(&never), lim);
+        }
+      }
+    }
+  } else if (warp == 3) {
+    if (lane == 0) {
+      // ---------------- accumulation MMAs: dQ += dS K_u (A = dS from TMEM) ----------------
+      constexpr uint32_t idesc_q = make_idesc_bf16(128, 64, false, true);  // B = K_u, MN-major
+      bool ok = true, any = false;
+      int U = 0;
+      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+        const int ab = it & 1, nu = 2 * (nqb - item / BH);
+        if (!mbar_wait_bounded(&acc_empty[ab], ((it >> 1) & 1) ^ 1, abort_flag, lim)) {
+          ok = false;
+          break;
+        }
+        for (int u = 0; u < nu; ++u, ++U) {
+          const int s = U % FBQ_NST, dsb = U & 1;
+          if (!mbar_wait_bounded(&st_full[s], (U / FBQ_NST) & 1, abort_flag, lim) ||
+              !mbar_wait_bounded(&ds_full[dsb], (U >> 1) & 1, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sm + FBQ_OFF_ST + s * FB_UNIT);
+          const uint32_t acc = tmem + FBQ_TM_ACC + (uint32_t)(ab * 64);
+          // K = 64 keys: B = 16 key rows of K_u per step (MN-major)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_ts(acc, tmem + FBQ_TM_DS + dsb * 32 + k * 8, make_sw128_desc(k_addr + k * 2048, 8192, 1024),
+                         idesc_q, (u > 0 || k > 0) ? 1u : 0u);
+          any = true;
+          umma_commit(&ds_free[dsb]);
+          umma_commit(&st_empty[s]);  // the unit's score MMAs completed before dS was written
+          if (u == nu - 1) umma_commit(&acc_full[ab]);
+        }
+      }
+      if (!ok) {
+        raise_device_error(err, DEV_TIMEOUT);
+        *abort_flag = 1;
+        if (any) {
+          int never = 0;
+          umma_commit(&drain[2]);
+          mbar_wait_bounded(&drain[2], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
   } else {
-    // element-wise warps: thread = query row r, keys [hf*64, hf*64 + 64) of the block
-    const int hf = (warp - 2) >> 2, q4 = warp & 3;
+    // ---------------- element-wise warps: query row r, key columns [cg*16, cg*16 + 16) of each unit ----------------
+    const int q4 = warp & 3, cg = (warp - FBQ_EW0) >> 2;
     const int r = q4 * 32 + lane;
-    const int qrow = qb * FA_BM + r;
-    const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * LOG2E;
-    const float L2 = qrow < T ? lse[(long long)bh * T + qrow] * LOG2E : 0.f;
-    const float Dr = qrow < T ? Dg[(long long)bh * T + qrow] : 0.f;
     bool fail = false;
-    for (int j = 0; j < nkb; ++j) {
-      if (!fail && !mbar_wait_bounded(s_full, j & 1, abort_flag, lim)) fail = true;
-      uint32_t sv[64], dv[64];
-      if (!fail) {
-        tc_fence_after();
-        tmem_ld_32x32b_x32(lane_base + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld_32x32b_x32(lane_base + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_32x32b_x32(lane_base + 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
-        tmem_ld_32x32b_x32(lane_base + 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
-        tmem_ld_wait();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) sv[e] = dv[e] = 0u;
-      }
+    int U = 0;
+    // Q and dO rows of item `it` (in shared memory) into the TMEM A operands. The score
+    // MMAs of the previous item, the only readers of that TMEM, are complete: this warp
+    // has seen all of their results.
+    auto load_operands = [&](int it) -> bool {
+      const int qdb = it & 1;
+      if (!mbar_wait_bounded(&qd_full[qdb], (it >> 1) & 1, abort_flag, lim)) return false;
+      const uint8_t* qd = sm + FBQ_OFF_QD + qdb * 2 * FA_TILE;
+      fb_row_to_tmem(qd, r, cg, tmem + lane_off + FBQ_TM_Q + cg * 8);
+      fb_row_to_tmem(qd + FA_TILE, r, cg, tmem + lane_off + FBQ_TM_Q + 32 + cg * 8);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty);
-      const bool diag = (j == qb);
-      const int kbase = j * FA_BN + hf * 64;
-      if (!fail && !mbar_wait_bounded(ds_free, (j & 1) ^ 1, abort_flag, lim)) fail = true;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float dsv[8];
-#pragma unroll
-        for (int e8 = 0; e8 < 8; ++e8) {
-          const int e = 8 * k + e8;
-          float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -L2));
-          if (diag && kbase + e > qrow) pe = 0.f;
-          dsv[e8] = pe * (__uint_as_float(dv[e]) - Dr);
-        }
-        fb_store_chunk(sm + FBQ_OFF_DS, r, hf, k, dsv);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_full);
-    }
-    if (!fail && !mbar_wait_bounded(acc_full, 0, abort_flag, lim)) fail = true;
-    if (named_barrier_or(1, 256, fail || *abort_flag)) {
       if (lane == 0) {
-        raise_device_error(err, DEV_TIMEOUT);
-        *abort_flag = 1;
+        mbar_arrive(qa_full);
+        mbar_arrive(&qd_empty[qdb]);
       }
-    } else {
-      tc_fence_after();
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(lane_base + 256 + hf * 32, v);
-      tmem_ld_wait();
+      return true;
+    };
+    // lse (log2 units) and D of this thread's query row, one item ahead
+    float lse2 = INFINITY, Dr = 0.f;
+    if ((int)blockIdx.x < nitems) {
+      const int item = blockIdx.x, qrow = (nqb - 1 - item / BH) * FA_BM + r;
+      const long long o = (long long)(item % BH) * T + qrow;
       if (qrow < T) {
-        bf16* dq = dqkv + ((long long)b * T + qrow) * 3 * C + h * 64 + hf * 32;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int e = 8 * q;
-          *reinterpret_cast<uint4*>(dq + e) =
-              make_uint4(pack_bf16x2(__uint_as_float(v[e]) * scale, __uint_as_float(v[e + 1]) * scale),
-                         pack_bf16x2(__uint_as_float(v[e + 2]) * scale, __uint_as_float(v[e + 3]) * scale),
-                         pack_bf16x2(__uint_as_float(v[e + 4]) * scale, __uint_as_float(v[e + 5]) * scale),
-                         pack_bf16x2(__uint_as_float(v[e + 6]) * scale, __uint_as_float(v[e + 7]) * scale));
+        lse2 = lse[o] * LOG2E;
+        Dr = Dg[o];
+      }
+      fail = !load_operands(0);
+    }
+    for (int it = 0, item = blockIdx.x; item < nitems && !fail; ++it, item += gridDim.x) {
+      const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
+      const int nu = 2 * (qb + 1);
+      const int qrow = qb * FA_BM + r;
+      float lse2_n = INFINITY, Dr_n = 0.f;
+      if (item + (int)gridDim.x < nitems) {
+        const int item2 = item + gridDim.x, qrow2 = (nqb - 1 - item2 / BH) * FA_BM + r;
+        const long long o = (long long)(item2 % BH) * T + qrow2;
+        if (qrow2 < T) {
+          lse2_n = lse[o] * LOG2E;
+          Dr_n = Dg[o];
         }
       }
+      for (int u = 0; u < nu; ++u, ++U) {
+        const int sb = U % FB_SBUF, dsb = U & 1;
+        if (!mbar_wait_bounded(&s_full[sb], (U / FB_SBUF) & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[16], dv[16];
+        tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(sb * 128 + cg * 16), sv);
+        tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(sb * 128 + 64 + cg * 16), dv);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[sb]);
+        float ds[16];
+        const int kcol0 = (u & 1) * 64 + cg * 16;  // key index within the block of column 0
+        const bool diag = u >= nu - 2;             // the key block qb itself
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -lse2));
+          if (diag && kcol0 + e > r) pe = 0.f;  // key after query
+          ds[e] = pe * (__uint_as_float(dv[e]) - Dr);
+        }
+        // the dQ MMAs of unit U - 2 have finished reading this dS buffer
+        if (!mbar_wait_bounded(&ds_free[dsb], ((U >> 1) & 1) ^ 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        fb_vals_to_tmem(ds, tmem + lane_off + FBQ_TM_DS + dsb * 32 + cg * 8);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_full[dsb]);
+      }
+      if (fail) break;
+      // the next item's operands first (lets its score MMAs start), then this item's dQ
+      if (item + (int)gridDim.x < nitems && !load_operands(it + 1)) {
+        fail = true;
+        break;
+      }
+      const int ab = it & 1;
+      if (!mbar_wait_bounded(&acc_full[ab], (it >> 1) & 1, abort_flag, lim)) {
+        fail = true;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(tmem + lane_off + FBQ_TM_ACC + (uint32_t)(ab * 64 + cg * 16), v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (qrow < T) fb_store_row16(dqkv + ((long long)b * T + qrow) * 3 * C + h * 64 + cg * 16, v, scale);
+      lse2 = lse2_n;
+      Dr = Dr_n;
+    }
+    if (fail && lane == 0) {
+      raise_device_error(err, DEV_TIMEOUT);
+      *abort_flag = 1;
     }
   }
 

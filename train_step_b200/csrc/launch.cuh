@@ -188,14 +188,15 @@ inline bool encode_partial_map(CUtensorMap* map, const void* ptr, long long cols
   return r == CUDA_SUCCESS;
 }
 
-// qkv [B][T][3C] bf16 as a 3-D map {3C, T, B}; box {64, 128, 1} (one head's 64
-// columns of 128 positions), 128-byte swizzle; positions past T read as zero.
-inline bool encode_qkv_map(CUtensorMap* map, const void* ptr, long long cols, long long T, long long B) {
+// qkv [B][T][3C] bf16 as a 3-D map {3C, T, B}; box {64, rows, 1} (one head's 64
+// columns of `rows` positions), 128-byte swizzle; positions past T read as zero.
+inline bool encode_qkv_map(CUtensorMap* map, const void* ptr, long long cols, long long T, long long B,
+                           unsigned rows = 128) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), (cuuint64_t)(T * cols * 2)};
-  cuuint32_t box[3] = {64u, 128u, 1u};
+  cuuint32_t box[3] = {64u, rows, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -586,8 +587,10 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
                                                                                   Dbuf, B, T, NH);
     int r = check_launch(c, "attn_bwd_dot");
     if (r) return r;
-    CUtensorMap tq, td;
-    if (!encode_qkv_map(&tq, qkv, 3LL * NH * 64, T, B) || !encode_qkv_map(&td, dout, (long long)NH * 64, T, B))
+    CUtensorMap tq, td, tq64, td64;  // 128-row tiles per item, 64-row tiles per streamed unit
+    if (!encode_qkv_map(&tq, qkv, 3LL * NH * 64, T, B) || !encode_qkv_map(&td, dout, (long long)NH * 64, T, B) ||
+        !encode_qkv_map(&tq64, qkv, 3LL * NH * 64, T, B, 64) ||
+        !encode_qkv_map(&td64, dout, (long long)NH * 64, T, B, 64))
       return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
     static bool attr_set = false;
     if (!attr_set) {
@@ -595,13 +598,15 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
       cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FBQ_SMEM);
       attr_set = true;
     }
-    dim3 grid((T + FA_BM - 1) / FA_BM, B * NH);
-    attn_bwd_dkdv_tc_kernel<<<grid, FB_THREADS, FBK_SMEM, c.stream>>>(tq, td, lse, Dbuf, (bf16*)dqkv, T, NH, scale,
-                                                                      c.d_err, 4000000000ull);
+    // persistent: one CTA per SM loops over (block, batch*head) items
+    const long long items = (long long)((T + FA_BM - 1) / FA_BM) * B * NH;
+    const int grid = items < c.num_sms ? (int)items : c.num_sms;
+    attn_bwd_dkdv_tc_kernel<<<grid, FBK_THREADS, FBK_SMEM, c.stream>>>(tq, tq64, td64, lse, Dbuf, (bf16*)dqkv, T, NH,
+                                                                      B * NH, scale, c.d_err, 4000000000ull);
     r = check_launch(c, "attn_bwd_dkdv_tc");
     if (r) return r;
-    attn_bwd_dq_tc_kernel<<<grid, FB_THREADS, FBQ_SMEM, c.stream>>>(tq, td, lse, Dbuf, (bf16*)dqkv, T, NH, scale,
-                                                                    c.d_err, 4000000000ull);
+    attn_bwd_dq_tc_kernel<<<grid, FBQ_THREADS, FBQ_SMEM, c.stream>>>(tq, td, tq64, lse, Dbuf, (bf16*)dqkv, T, NH,
+                                                                    B * NH, scale, c.d_err, 4000000000ull);
     return check_launch(c, "attn_bwd_dq_tc");
   }
   if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");
