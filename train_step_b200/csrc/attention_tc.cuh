@@ -354,18 +354,21 @@ constexpr int FBQ_THREADS = 32 * (FBQ_EW0 + FB_EW_WARPS);  // 640
 constexpr int FB_HALF = 64 * 128;                  // 8 KB: 64 rows x 64 bf16 (128-byte rows)
 constexpr int FB_UNIT = 2 * FB_HALF;               // 16 KB: a stage (two half tiles) or a 128 x 64 tile
 constexpr int FB_BARS = 512;
-// dK/dV kernel shared memory: K/V [2 items] | stages (Q_u, dO_u) | lse/D per stage | barriers
-constexpr int FBK_NST = 8;
+// dK/dV kernel shared memory: K/V [2 items] | stages (Q_u, dO_u) | lse/D per stage |
+// output staging (dK, dV tiles for one TMA store each) | barriers
+constexpr int FBK_NST = 6;
 constexpr int FBK_OFF_KV = 0;
 constexpr int FBK_OFF_ST = 4 * FA_TILE;
 constexpr int FBK_OFF_LD = FBK_OFF_ST + FBK_NST * FB_UNIT;
-constexpr int FBK_OFF_BAR = FBK_OFF_LD + 4096;  // FBK_NST x 512 bytes
+constexpr int FBK_OFF_OUT = FBK_OFF_LD + 4096;  // FBK_NST x 512 bytes, rounded up
+constexpr int FBK_OFF_BAR = FBK_OFF_OUT + 2 * FA_TILE;
 constexpr int FBK_SMEM = FBK_OFF_BAR + FB_BARS + 1024;
-// dQ kernel shared memory: Q/dO [2 items] | stages (K_u, V_u) | barriers
+// dQ kernel shared memory: Q/dO [2 items] | stages (K_u, V_u) | output staging (dQ) | barriers
 constexpr int FBQ_NST = 8;
 constexpr int FBQ_OFF_QD = 0;
 constexpr int FBQ_OFF_ST = 4 * FA_TILE;
-constexpr int FBQ_OFF_BAR = FBQ_OFF_ST + FBQ_NST * FB_UNIT;
+constexpr int FBQ_OFF_OUT = FBQ_OFF_ST + FBQ_NST * FB_UNIT;
+constexpr int FBQ_OFF_BAR = FBQ_OFF_OUT + FA_TILE;
 constexpr int FBQ_SMEM = FBQ_OFF_BAR + FB_BARS + 1024;
 static_assert(FBK_NST * 512 <= 4096, "lse/D staging");
 static_assert(FBQ_SMEM <= 232448 && FBK_SMEM <= 232448, "shared memory per CTA");
@@ -389,17 +392,13 @@ __device__ __forceinline__ void fb_store16(uint8_t* tile, int r, int c16, const 
   }
 }
 
-// 16 bf16 values of one output row (two 16-byte stores)
-__device__ __forceinline__ void fb_store_row16(bf16* dst, const uint32_t (&v)[16], float mul) {
+// 16 accumulator values (x mul) of row r into a 128-row output staging tile laid out
+// as the 128-byte-swizzled box of a TMA store
+__device__ __forceinline__ void fb_stage_row16(uint8_t* tile, int r, int cg, const uint32_t (&v)[16], float mul) {
+  float f[16];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int e = 8 * k;
-    *reinterpret_cast<uint4*>(dst + e) =
-        make_uint4(pack_bf16x2(__uint_as_float(v[e]) * mul, __uint_as_float(v[e + 1]) * mul),
-                   pack_bf16x2(__uint_as_float(v[e + 2]) * mul, __uint_as_float(v[e + 3]) * mul),
-                   pack_bf16x2(__uint_as_float(v[e + 4]) * mul, __uint_as_float(v[e + 5]) * mul),
-                   pack_bf16x2(__uint_as_float(v[e + 6]) * mul, __uint_as_float(v[e + 7]) * mul));
-  }
+  for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(v[e]) * mul;
+  fb_store16(tile, r, cg * 2, f);
 }
 
 // Bounded wait whose result is the same for every lane of the warp (lane 0 waits).
@@ -429,9 +428,9 @@ __device__ __forceinline__ void fb_vals_to_tmem(const float (&v)[16], uint32_t t
 
 __global__ void __launch_bounds__(FBK_THREADS, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q64,
-                            const __grid_constant__ CUtensorMap tm_do64, const float* __restrict__ lse,
-                            const float* __restrict__ Dg, bf16* __restrict__ dqkv, int T, int NH, int BH, float scale,
-                            int* err, unsigned long long timeout_ns) {
+                            const __grid_constant__ CUtensorMap tm_do64, const __grid_constant__ CUtensorMap tm_out,
+                            const float* __restrict__ lse, const float* __restrict__ Dg, int T, int NH, int BH,
+                            float scale, int* err, unsigned long long timeout_ns) {
   extern __shared__ uint8_t fb_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FBK_OFF_BAR);
@@ -446,7 +445,9 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
   uint64_t* p_free = p_full + 1;
   uint64_t* acc_full = p_free + 1;
   uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;            // [4]: one per MMA thread (abort path)
+  uint64_t* out_full = acc_empty + 1;         // output tiles staged (element-wise warps)
+  uint64_t* out_free = out_full + 1;          // the previous item's TMA stores have read the staging
+  uint64_t* drain = out_free + 1;             // [4]: one per MMA thread (abort path)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 5);
 
@@ -475,6 +476,8 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
     mbar_init(p_free, 2);  // the dV and dK threads
     mbar_init(acc_full, 2);
     mbar_init(acc_empty, FB_EW_WARPS);
+    mbar_init(out_full, FB_EW_WARPS);
+    mbar_init(out_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -639,6 +642,7 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
     // ---------------- element-wise warps: key row r, query columns [cg*16, cg*16 + 16) of each unit ----------------
     const int q4 = warp & 3, cg = (warp - FBK_EW0) >> 2;
     const int r = q4 * 32 + lane;
+    const bool issuer = (warp == FBK_EW0 && lane == 0);  // issues the output tiles' TMA stores
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * LOG2E;
     bool fail = false;
@@ -728,13 +732,31 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
-      const int key = kb * FA_BN + r;
-      if (key < T) {
-        bf16* dk = dqkv + ((long long)b * T + key) * 3 * C + C + h * 64 + cg * 16;
-        fb_store_row16(dk + C, v, 1.0f);
-        fb_store_row16(dk, k, scale);
+      // dK (scaled) and dV through shared memory, one TMA store per tile (rows past T are clipped)
+      if (issuer && it > 0) {
+        bulk_wait_read<0>();
+        mbar_arrive(out_free);
+      }
+      if (!mbar_wait_bounded(out_free, (it & 1) ^ 1, abort_flag, lim)) {
+        fail = true;
+        break;
+      }
+      fb_stage_row16(sm + FBK_OFF_OUT, r, cg, k, scale);
+      fb_stage_row16(sm + FBK_OFF_OUT + FA_TILE, r, cg, v, 1.0f);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(out_full);
+      if (issuer) {
+        if (!mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        tma_store_3d(&tm_out, sm + FBK_OFF_OUT, C + h * 64, kb * FA_BN, b);
+        tma_store_3d(&tm_out, sm + FBK_OFF_OUT + FA_TILE, 2 * C + h * 64, kb * FA_BN, b);
+        bulk_commit();
       }
     }
+    if (issuer) bulk_wait_all();  // the staging must outlive the stores' reads
     if (fail && lane == 0) {
       raise_device_error(err, DEV_TIMEOUT);
       *abort_flag = 1;
@@ -751,9 +773,9 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
 
 __global__ void __launch_bounds__(FBQ_THREADS, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                          const __grid_constant__ CUtensorMap tm_kv64, const float* __restrict__ lse,
-                          const float* __restrict__ Dg, bf16* __restrict__ dqkv, int T, int NH, int BH, float scale,
-                          int* err, unsigned long long timeout_ns) {
+                          const __grid_constant__ CUtensorMap tm_kv64, const __grid_constant__ CUtensorMap tm_out,
+                          const float* __restrict__ lse, const float* __restrict__ Dg, int T, int NH, int BH,
+                          float scale, int* err, unsigned long long timeout_ns) {
   extern __shared__ uint8_t fb_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FBQ_OFF_BAR);
@@ -768,7 +790,9 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
   uint64_t* ds_free = ds_full + 2;            // [2]
   uint64_t* acc_full = ds_free + 2;           // [2]
   uint64_t* acc_empty = acc_full + 2;         // [2]
-  uint64_t* drain = acc_empty + 2;            // [3]: one per MMA thread (abort path)
+  uint64_t* out_full = acc_empty + 2;         // output tile staged (element-wise warps)
+  uint64_t* out_free = out_full + 1;          // the previous item's TMA store has read the staging
+  uint64_t* drain = out_free + 1;             // [3]: one per MMA thread (abort path)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 4);
 
@@ -788,6 +812,8 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
       mbar_init(&acc_empty[i], FB_EW_WARPS);
     }
     for (int i = 0; i < 3; ++i) mbar_init(&drain[i], 1);
+    mbar_init(out_full, FB_EW_WARPS);
+    mbar_init(out_free, 1);
     mbar_init(qa_full, FB_EW_WARPS);
     for (int i = 0; i < FBQ_NST; ++i) {
       mbar_init(&st_full[i], 1);
@@ -947,6 +973,7 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
     // ---------------- element-wise warps: query row r, key columns [cg*16, cg*16 + 16) of each unit ----------------
     const int q4 = warp & 3, cg = (warp - FBQ_EW0) >> 2;
     const int r = q4 * 32 + lane;
+    const bool issuer = (warp == FBQ_EW0 && lane == 0);  // issues the output tile's TMA store
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * LOG2E;
     bool fail = false;
@@ -983,14 +1010,14 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
     for (int it = 0, item = blockIdx.x; item < nitems && !fail; ++it, item += gridDim.x) {
       const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
       const int nu = 2 * (qb + 1);
-      const int qrow = qb * FA_BM + r;
-      float lse2_n = INFINITY, Dr_n = 0.f;
+      // the next item's lse / D: loads issued now, first used at the item switch
+      float lse_n = INFINITY, Dr_n = 0.f;
       if (item + (int)gridDim.x < nitems) {
         const int item2 = item + gridDim.x, qrow2 = (nqb - 1 - item2 / BH) * FA_BM + r;
         const long long o = (long long)(item2 % BH) * T + qrow2;
         if (qrow2 < T) {
-          lse2_n = lse[o] * LOG2E;
-          Dr_n = Dg[o];
+          lse_n = __ldg(lse + o);
+          Dr_n = __ldg(Dg + o);
         }
       }
       for (int u = 0; u < nu; ++u, ++U) {
@@ -1045,10 +1072,31 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
-      if (qrow < T) fb_store_row16(dqkv + ((long long)b * T + qrow) * 3 * C + h * 64 + cg * 16, v, scale);
-      lse2 = lse2_n;
+      // dQ (scaled) through shared memory, one TMA store (rows past T are clipped)
+      if (issuer && it > 0) {
+        bulk_wait_read<0>();
+        mbar_arrive(out_free);
+      }
+      if (!mbar_wait_bounded(out_free, (it & 1) ^ 1, abort_flag, lim)) {
+        fail = true;
+        break;
+      }
+      fb_stage_row16(sm + FBQ_OFF_OUT, r, cg, v, scale);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(out_full);
+      if (issuer) {
+        if (!mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        tma_store_3d(&tm_out, sm + FBQ_OFF_OUT, h * 64, qb * FA_BM, b);
+        bulk_commit();
+      }
+      lse2 = lse_n * LOG2E;
       Dr = Dr_n;
     }
+    if (issuer) bulk_wait_all();  // the staging must outlive the store's read
     if (fail && lane == 0) {
       raise_device_error(err, DEV_TIMEOUT);
       *abort_flag = 1;

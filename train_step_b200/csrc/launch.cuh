@@ -587,11 +587,13 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
                                                                                   Dbuf, B, T, NH);
     int r = check_launch(c, "attn_bwd_dot");
     if (r) return r;
-    CUtensorMap tq, td, tq64, td64;  // 128-row tiles per item, 64-row tiles per streamed unit
+    CUtensorMap tq, td, tq64, td64, tout;  // 128-row tiles per item, 64-row tiles per streamed unit
     if (!encode_qkv_map(&tq, qkv, 3LL * NH * 64, T, B) || !encode_qkv_map(&td, dout, (long long)NH * 64, T, B) ||
         !encode_qkv_map(&tq64, qkv, 3LL * NH * 64, T, B, 64) ||
-        !encode_qkv_map(&td64, dout, (long long)NH * 64, T, B, 64))
+        !encode_qkv_map(&td64, dout, (long long)NH * 64, T, B, 64) ||
+        !encode_qkv_map(&tout, dqkv, 3LL * NH * 64, T, B))
       return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
+    if (reinterpret_cast<uintptr_t>(dqkv) & 15) return fail(c, GPT2_ERR_CONFIG, "attention: dqkv must be 16-byte aligned");
     static bool attr_set = false;
     if (!attr_set) {
       cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FBK_SMEM);
@@ -601,12 +603,12 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
     // persistent: one CTA per SM loops over (block, batch*head) items
     const long long items = (long long)((T + FA_BM - 1) / FA_BM) * B * NH;
     const int grid = items < c.num_sms ? (int)items : c.num_sms;
-    attn_bwd_dkdv_tc_kernel<<<grid, FBK_THREADS, FBK_SMEM, c.stream>>>(tq, tq64, td64, lse, Dbuf, (bf16*)dqkv, T, NH,
-                                                                      B * NH, scale, c.d_err, 4000000000ull);
+    attn_bwd_dkdv_tc_kernel<<<grid, FBK_THREADS, FBK_SMEM, c.stream>>>(tq, tq64, td64, tout, lse, Dbuf, T, NH, B * NH,
+                                                                       scale, c.d_err, 4000000000ull);
     r = check_launch(c, "attn_bwd_dkdv_tc");
     if (r) return r;
-    attn_bwd_dq_tc_kernel<<<grid, FBQ_THREADS, FBQ_SMEM, c.stream>>>(tq, td, tq64, lse, Dbuf, (bf16*)dqkv, T, NH,
-                                                                    B * NH, scale, c.d_err, 4000000000ull);
+    attn_bwd_dq_tc_kernel<<<grid, FBQ_THREADS, FBQ_SMEM, c.stream>>>(tq, td, tq64, tout, lse, Dbuf, T, NH, B * NH,
+                                                                     scale, c.d_err, 4000000000ull);
     return check_launch(c, "attn_bwd_dq_tc");
   }
   if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");
