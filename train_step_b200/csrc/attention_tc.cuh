@@ -1,24 +1,24 @@
 // attention_tc.cuh -- causal flash attention on the 5th-generation tensor cores
-// (tcgen05, accumulators in TMEM, tiles by TMA), head dim 64, bf16 operands.
+// (tcgen05, accumulators and A operands in TMEM, tiles by TMA), head dim 64, bf16.
 //
 // Same mathematics as attention.cuh ("AxonLM", Key Features: Flash Attention;
-// "GPT From Scratch", Key decisions): per (batch, head) and per 128-query block,
-// online softmax over 128-key blocks; lse = logsumexp of the scaled scores.
+// "GPT From Scratch", Key decisions): per (batch, head), online softmax over key
+// blocks; lse = logsumexp of the scaled scores; the backward recomputes P from lse.
 //
-// Forward, one CTA per (query block, batch*head), 320 threads:
-//   warp 0     TMA producer: Q once, then K_j and V_j into a 3-stage ring
-//   warp 1     one thread issues tcgen05.mma:
-//                S_j  = Q K_j^T  (M=128, N=128, K=64)  into TMEM S[j % 2]
-//                PV_j = P_j V_j  (M=128, N=64,  K=128) into TMEM PV[j % 2]
-//   warps 2-9  softmax: each query row is shared by two threads (TMEM lane, one
-//              per half of the 128 key columns; the halves swap row maxima
-//              through shared memory). P_j = 2^(S_j*scale*log2e - m_j) goes to
-//              shared memory as bf16 (128-byte swizzled, K-major); row sums and
-//              the running output O = O * 2^(m_{j-1} - m_j) + PV_j (each thread
-//              keeps 32 of the 64 output columns) stay in registers.
-// S, P and PV are double-buffered so the tensor cores compute S_{j+1} and PV_j
-// while the softmax warps work on block j.
-// Every mbarrier wait is bounded (device error word + early exit, no trap).
+// Three persistent kernels (one CTA per SM looping over (block, batch*head) items,
+// longest first): the forward, and a deterministic backward split into a dK/dV
+// kernel (per key block) and a dQ kernel (per query block). They share one design,
+// set by what B200 measurements showed:
+//  * a thread can issue a 1-SM tcgen05.mma only every ~96 cycles whatever its N,
+//    but the tensor pipe overlaps the streams of several threads, so every product
+//    has its own issuing thread;
+//  * A operands live in TMEM (the item's fixed 128-row tile, and the P / dS tiles
+//    written there by the element-wise warps), so only 64-row B tiles are read from
+//    shared memory;
+//  * each 64-wide unit streams its own 16 KB stage through a deep TMA ring, so a
+//    tile is requested several units before it is needed;
+//  * outputs leave through a shared-memory tile and one TMA store per tile.
+// Every mbarrier wait is bounded (device error word, early exit, no trap).
 #pragma once
 #include "attention.cuh"
 #include "common.cuh"
@@ -27,287 +27,7 @@ namespace g2 {
 
 constexpr int FA_BM = 128;  // queries per CTA
 constexpr int FA_BN = 128;  // keys per block
-constexpr int FA_THREADS = 320;
 constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
-constexpr int FA_P = FA_BM * FA_BN * 2;  // 32 KB: P tile
-constexpr int FA_KV_STAGES = 3;
-// shared memory: Q | K0 V0 | K1 V1 | K2 V2 | P0 | P1 | barriers | exchange
-constexpr int FA_OFF_Q = 0;
-constexpr int FA_OFF_KV = FA_TILE;
-constexpr int FA_OFF_P = FA_OFF_KV + 2 * FA_KV_STAGES * FA_TILE;
-constexpr int FA_OFF_BAR = FA_OFF_P + 2 * FA_P;
-constexpr int FA_OFF_RED = FA_OFF_BAR + 256;  // row-max / row-sum exchange, 3 x 2 x 128 floats
-constexpr int FA_SMEM = FA_OFF_RED + 3 * 2 * 128 * 4 + 1024;
-constexpr uint32_t FA_TMEM_COLS = 512;  // S0 0..127, S1 128..255, PV0 256..319, PV1 320..383
-
-// P row r, key column c (0..127): 128-byte-swizzled K-major tile in two 64-key halves.
-__device__ __forceinline__ uint32_t fa_p_off(int r, int chunk16 /*0..15*/) {
-  const int half = chunk16 >> 3, c8 = chunk16 & 7;
-  return (uint32_t)(half * (FA_BM * 128) + r * 128 + ((c8 ^ (r & 7)) << 4));
-}
-
-__global__ void __launch_bounds__(FA_THREADS, 1)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
-                       int T, int NH, float scale, int* err, unsigned long long timeout_ns) {
-  extern __shared__ uint8_t fa_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FA_OFF_BAR);
-  uint64_t* q_full = bar + 0;
-  uint64_t* kv_full = bar + 1;   // [3]
-  uint64_t* kv_empty = bar + 4;  // [3]
-  uint64_t* s_full = bar + 7;    // [2]
-  uint64_t* s_empty = bar + 9;   // [2]
-  uint64_t* p_full = bar + 11;   // [2]
-  uint64_t* pv_full = bar + 13;  // [2]
-  uint64_t* drain = bar + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 16);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 17);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  const int bh = blockIdx.y, b = bh / NH, h = bh % NH;
-  const int C = NH * 64;
-  const int nkb = qb + 1;
-  const uint64_t lim = timeout_ns;
-
-  if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int i = 0; i < FA_KV_STAGES; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 8);
-      mbar_init(&p_full[i], 8);
-      mbar_init(&pv_full[i], 1);
-    }
-    mbar_init(drain, 1);  // for the abort path
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, FA_TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer ----------------
-      tma_prefetch_desc(&tm_qkv);
-      bool ok = true;
-      mbar_arrive_expect_tx(q_full, FA_TILE);
-      tma_load_3d(sm + FA_OFF_Q, &tm_qkv, q_full, h * 64, qb * FA_BM, b);
-      uint32_t issued = 0, par = 0;  // bit s: stage s has a load issued / parity of its last load
-      for (int j = 0; j < nkb && ok; ++j) {
-        const int st = j % FA_KV_STAGES;
-        const uint32_t ph = (uint32_t)((j / FA_KV_STAGES) & 1);
-        if (!mbar_wait_bounded(&kv_empty[st], ph ^ 1, abort_flag, lim)) {
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&kv_full[st], 2 * FA_TILE);
-        uint8_t* kd = sm + FA_OFF_KV + st * 2 * FA_TILE;  // stage st: K then V
-        tma_load_3d(kd, &tm_qkv, &kv_full[st], C + h * 64, j * FA_BN, b);
-        tma_load_3d(kd + FA_TILE, &tm_qkv, &kv_full[st], 2 * C + h * 64, j * FA_BN, b);
-        issued |= 1u << st;
-        par = (par & ~(1u << st)) | (ph << st);
-      }
-      if (!ok) {
-        raise_device_error(err, DEV_TIMEOUT);
-        *abort_flag = 1;
-        int never = 0;
-        mbar_wait_bounded(q_full, 0, reinterpret_cast<volatile int*>(&never), lim);
-        for (int s = 0; s < FA_KV_STAGES; ++s)
-          if ((issued >> s) & 1u)
-            mbar_wait_bounded(&kv_full[s], (par >> s) & 1u, reinterpret_cast<volatile int*>(&never), lim);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_o = make_idesc_bf16(128, 64, false, true);
-      const uint32_t q_addr = smem_u32(sm + FA_OFF_Q);
-      bool ok = mbar_wait_bounded(q_full, 0, abort_flag, lim);
-      bool any = false;
-      for (int j = 0; j <= nkb && ok; ++j) {
-        if (j < nkb) {  // S_j = Q K_j^T
-          const int st = j & 1, ks = j % FA_KV_STAGES;
-          if (!mbar_wait_bounded(&kv_full[ks], (j / FA_KV_STAGES) & 1, abort_flag, lim) ||
-              !mbar_wait_bounded(&s_empty[st], ((j >> 1) & 1) ^ 1, abort_flag, lim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm + FA_OFF_KV + ks * 2 * FA_TILE);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem + st * 128, make_sw128_desc(q_addr + k * 32, 16, 1024),
-                      make_sw128_desc(k_addr + k * 32, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
-          umma_commit(&s_full[st]);
-          any = true;
-        }
-        if (j >= 1) {  // PV_{j-1} = P_{j-1} V_{j-1}
-          const int i = j - 1, st = i & 1, ks = i % FA_KV_STAGES;
-          if (!mbar_wait_bounded(&p_full[st], (i >> 1) & 1, abort_flag, lim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t p_addr = smem_u32(sm + FA_OFF_P + st * FA_P);
-          const uint32_t v_addr = smem_u32(sm + FA_OFF_KV + ks * 2 * FA_TILE + FA_TILE);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tmem + 256 + st * 64,
-                      make_sw128_desc(p_addr + (kk >> 2) * (FA_BM * 128) + (kk & 3) * 32, 16, 1024),
-                      make_sw128_desc(v_addr + kk * 2048, 8192, 1024), idesc_o, kk > 0 ? 1u : 0u);
-          umma_commit(&pv_full[st]);
-          umma_commit(&kv_empty[ks]);
-        }
-      }
-      if (!ok) {
-        raise_device_error(err, DEV_TIMEOUT);
-        *abort_flag = 1;
-        if (any) {
-          int never = 0;
-          umma_commit(drain);
-          mbar_wait_bounded(drain, 0, reinterpret_cast<volatile int*>(&never), lim);
-        }
-      }
-    }
-  } else {
-    // ---------------- softmax warps ----------------
-    // warps 2-5 take S columns 0-63, warps 6-9 columns 64-127 of the same rows; the
-    // two halves exchange their row maxima through shared memory once per block
-    const int hf = (warp - 2) >> 2;       // column half
-    const int q4 = warp & 3;              // TMEM lane quarter
-    const int r = q4 * 32 + lane;         // row within the query block
-    const int qrow = qb * FA_BM + r;      // query position
-    const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
-    float* red = reinterpret_cast<float*>(sm + FA_OFF_RED);  // [3 buffers][2 halves][128 rows]
-    const float sl2 = scale * LOG2E;
-    float o[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) o[i] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f, c_prev = 0.f, c_cur = 0.f;
-    // A failed (timed-out) wait never makes a warp leave on its own: every softmax
-    // warp reaches each named barrier, and the barrier's OR decides for all.
-    bool fail = false;
-    for (int j = 0; j <= nkb; ++j) {
-      if (j < nkb) {
-        const int st = j & 1;
-        if (!fail && !mbar_wait_bounded(&s_full[st], (j >> 1) & 1, abort_flag, lim)) fail = true;
-        uint32_t sv[64];
-        if (!fail) {
-          tc_fence_after();
-          tmem_ld_32x32b_x32(lane_base + st * 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-          tmem_ld_32x32b_x32(lane_base + st * 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) sv[e] = 0u;
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[st]);  // S[st] is free for S_{j+2}
-        const bool diag = (j == qb);
-        const int kbase = j * FA_BN + hf * 64;
-        if (diag) {  // causal mask: keys after the query get -inf (only on the diagonal block)
-#pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (kbase + e > qrow) sv[e] = __float_as_uint(-INFINITY);
-        }
-        float mx;
-        {
-          float m8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sv[e]);
-#pragma unroll
-          for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sv[e]));
-          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        }
-        red[(st * 2 + hf) * FA_BM + r] = mx;
-        if (named_barrier_or(1, 256, fail || *abort_flag)) {
-          fail = true;
-          break;
-        }
-        mx = fmaxf(mx, red[(st * 2 + (hf ^ 1)) * FA_BM + r]);
-        const float m_new = fmaxf(m_run, mx * sl2);
-        const float corr = (m_run == -INFINITY) ? 0.f : ex2_fast(m_run - m_new);
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        uint8_t* pbuf = sm + FA_OFF_P + st * FA_P;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float p[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = ex2_fast(fmaf(__uint_as_float(sv[8 * k + e]), sl2, -m_new));  // 2^-inf = 0 for masked keys
-            rs8[e] += p[e];
-          }
-          uint4 w = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
-                               pack_bf16x2(p[6], p[7]));
-          *reinterpret_cast<uint4*>(pbuf + fa_p_off(r, hf * 8 + k)) = w;
-        }
-        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[st]);
-        l_run = l_run * corr + rs;
-        m_run = m_new;
-        c_cur = corr;
-      }
-      // fold PV_{j-1} into O with the correction of block j-1
-      if (j >= 1) {
-        const int i = j - 1, sp = i & 1;
-        if (!fail && !mbar_wait_bounded(&pv_full[sp], (i >> 1) & 1, abort_flag, lim)) fail = true;
-        if (!fail) {
-          tc_fence_after();
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(lane_base + 256 + sp * 64 + hf * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = fmaf(o[e], c_prev, __uint_as_float(v[e]));
-        }
-      }
-      c_prev = c_cur;
-    }
-    // combine the two halves' row sums; the barrier also decides success for all
-    red[(4 + hf) * FA_BM + r] = l_run;
-    if (named_barrier_or(1, 256, fail || *abort_flag)) {
-      if (lane == 0) {
-        raise_device_error(err, DEV_TIMEOUT);
-        *abort_flag = 1;
-      }
-    } else {
-      const float l = l_run + red[(4 + (hf ^ 1)) * FA_BM + r];
-      if (qrow < T) {
-        const float inv = 1.0f / l;
-        bf16* orow = out + ((long long)b * T + qrow) * C + h * 64 + hf * 32;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint4 w = make_uint4(pack_bf16x2(o[8 * k] * inv, o[8 * k + 1] * inv),
-                               pack_bf16x2(o[8 * k + 2] * inv, o[8 * k + 3] * inv),
-                               pack_bf16x2(o[8 * k + 4] * inv, o[8 * k + 5] * inv),
-                               pack_bf16x2(o[8 * k + 6] * inv, o[8 * k + 7] * inv));
-          *reinterpret_cast<uint4*>(orow + 8 * k) = w;
-        }
-        if (hf == 0) lse[((long long)b * NH + h) * T + qrow] = (m_run + __log2f(l)) * LN2;
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, FA_TMEM_COLS);
-  }
-}
 
 // ---------------------------------------------------------------------------
 // Backward on tcgen05. Two deterministic kernels (no atomics). Both are
@@ -1108,6 +828,415 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, FB_TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Forward on tcgen05, persistent (one CTA per SM looping over items). Item =
+// (128-query block qb, batch*head), longest rows first; units = 64-key halves of
+// the key blocks 0 .. qb, each streamed through the same 16 KB stage ring as the
+// backward kernels.
+//   S_u  = Q K_u^T     (M=128 queries, N=64 keys, K=64; A = Q in TMEM, B = K_u)
+//   O_g += P_u V_u     (M=128, N=64, K=64 keys;     A = P_u in TMEM, B = V_u)
+// Two softmax groups (4 warps each) take alternate units. Each thread owns one
+// query row of its group's units, so a unit needs no exchange between threads;
+// each group keeps its own running max m, row sum l and output accumulator O_g,
+// and the two are merged when the item ends:
+//   m = max(m_0, m_1), O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)).
+// A group re-bases its running max only when the new block maximum exceeds it by
+// more than 8 (log2 units); otherwise its probabilities are taken against the
+// stale max (at most 2^8, exact in fp32 and representable in bf16) and O_g and l
+// stay consistent because both use the same reference. A re-base rescales the
+// thread's row of O_g in TMEM once the previous P V product has completed.
+// Warps: 0 TMA producer, 1 S MMAs, 2 P V MMAs, 3-6 softmax group 0, 7-10 group 1.
+// Every wait is bounded (device error word, no trap).
+// ---------------------------------------------------------------------------
+constexpr int FF_THREADS = 352;
+constexpr int FF_NST = 8;
+constexpr int FF_OFF_Q = 0;                                  // Q tiles [2 items]
+constexpr int FF_OFF_ST = 2 * FA_TILE;                       // stages (K_u | V_u)
+constexpr int FF_OFF_OUT = FF_OFF_ST + FF_NST * FB_UNIT;     // output staging tile
+constexpr int FF_OFF_X = FF_OFF_OUT + FA_TILE;               // (m, l) exchange [2 items][2 groups][128]
+constexpr int FF_OFF_BAR = FF_OFF_X + 2 * 2 * 128 * 8;
+constexpr int FF_SMEM = FF_OFF_BAR + FB_BARS + 1024;
+static_assert(FF_SMEM <= 232448, "shared memory per CTA");
+// TMEM: S [group][2] x 64 at 0..255, O [group] x 64 at 256, Q (32) at 384, P [group] x 32 at 416
+constexpr uint32_t FF_TM_O = 256, FF_TM_Q = 384, FF_TM_P = 416, FF_TMEM_COLS = 512;
+constexpr float FF_REBASE = 8.0f;
+
+__global__ void __launch_bounds__(FF_THREADS, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv64,
+                       const __grid_constant__ CUtensorMap tm_out, float* __restrict__ lse, int T, int NH, int BH,
+                       float scale, int* err, unsigned long long timeout_ns) {
+  extern __shared__ uint8_t ff_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ff_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FF_OFF_BAR);
+  uint64_t* q_full = bar;                  // [2] Q tile landed
+  uint64_t* q_empty = q_full + 2;          // [2] Q copied into TMEM (8 softmax warps)
+  uint64_t* qa_full = q_empty + 2;         // the TMEM Q operand is written (8 softmax warps)
+  uint64_t* st_full = qa_full + 1;         // [FF_NST]
+  uint64_t* st_empty = st_full + FF_NST;   // [FF_NST]
+  uint64_t* s_full = st_empty + FF_NST;    // [group][2]
+  uint64_t* s_empty = s_full + 4;          // [group][2] (the group's 4 warps)
+  uint64_t* p_full = s_empty + 4;          // [group] (4 warps)
+  uint64_t* o_done = p_full + 2;           // [group] P V product complete
+  uint64_t* x_full = o_done + 2;           // (m, l) of both groups written (8 warps), once per item
+  uint64_t* o_read = x_full + 1;           // both groups have read O_0 and O_1 (8 warps), once per item
+  uint64_t* out_full = o_read + 1;         // output tile staged (8 warps)
+  uint64_t* out_free = out_full + 1;       // the previous item's TMA store has read the staging
+  uint64_t* drain = out_free + 1;          // [2]: one per MMA thread (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 3);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = NH * 64;
+  const int nqb = (T + FA_BM - 1) / FA_BM;
+  const int nitems = nqb * BH;  // item w: query block nqb - 1 - w / BH, bh = w % BH
+  const uint64_t lim = timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 8);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_done[i], 1);
+      mbar_init(&drain[i], 1);
+    }
+    mbar_init(qa_full, 8);
+    for (int i = 0; i < FF_NST; ++i) {
+      mbar_init(&st_full[i], 1);
+      mbar_init(&st_empty[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
+    }
+    mbar_init(x_full, 8);
+    mbar_init(o_read, 8);
+    mbar_init(out_full, 8);
+    mbar_init(out_free, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, FF_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- producer: Q per item, (K_u, V_u) per unit ----------------
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_kv64);
+      bool ok = true;
+      uint32_t q_iss = 0, q_par = 0, st_iss = 0, st_par = 0;
+      int U = 0;
+      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+        const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
+        const int qbuf = it & 1;
+        if (!mbar_wait_bounded(&q_empty[qbuf], ((it >> 1) & 1) ^ 1, abort_flag, lim)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&q_full[qbuf], FA_TILE);
+        tma_load_3d(sm + FF_OFF_Q + qbuf * FA_TILE, &tm_q, &q_full[qbuf], h * 64, qb * FA_BM, b);
+        q_iss |= 1u << qbuf;
+        q_par = (q_par & ~(1u << qbuf)) | ((uint32_t)((it >> 1) & 1) << qbuf);
+        for (int k0 = 0; k0 < (qb + 1) * FA_BN; k0 += 64, ++U) {
+          const int s = U % FF_NST;
+          const uint32_t ph = (uint32_t)((U / FF_NST) & 1);
+          if (!mbar_wait_bounded(&st_empty[s], ph ^ 1, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          uint8_t* d = sm + FF_OFF_ST + s * FB_UNIT;
+          mbar_arrive_expect_tx(&st_full[s], FB_UNIT);
+          tma_load_3d(d, &tm_kv64, &st_full[s], C + h * 64, k0, b);
+          tma_load_3d(d + FB_HALF, &tm_kv64, &st_full[s], 2 * C + h * 64, k0, b);
+          st_iss |= 1u << s;
+          st_par = (st_par & ~(1u << s)) | (ph << s);
+        }
+      }
+      if (!ok) {
+        raise_device_error(err, DEV_TIMEOUT);
+        *abort_flag = 1;
+        int never = 0;
+        for (int i = 0; i < 2; ++i)
+          if ((q_iss >> i) & 1u)
+            mbar_wait_bounded(&q_full[i], (q_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+        for (int i = 0; i < FF_NST; ++i)
+          if ((st_iss >> i) & 1u)
+            mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+      }
+    }
+  } else if (warp == 1 || warp == 2) {
+    if (lane == 0) {
+      // ---------------- MMAs: S_u = Q K_u^T (warp 1); O_g += P_u V_u (warp 2) ----------------
+      const bool is_s = warp == 1;
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, 64, false, true);  // B = V_u, MN-major
+      bool ok = true, any = false;
+      int U = 0;  // unit counter over all items; unit U belongs to group U % 2 (items have even unit counts)
+      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+        const int nu = 2 * (nqb - item / BH);
+        if (is_s && !mbar_wait_bounded(qa_full, it & 1, abort_flag, lim)) {
+          ok = false;
+          break;
+        }
+        for (int u = 0; u < nu; ++u, ++U) {
+          const int s = U % FF_NST, g = U & 1, Ug = U >> 1;  // Ug: the unit's index within its group
+          if (!mbar_wait_bounded(&st_full[s], (U / FF_NST) & 1, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          const uint32_t k_addr = smem_u32(sm + FF_OFF_ST + s * FB_UNIT), v_addr = k_addr + FB_HALF;
+          if (is_s) {
+            const int sg = g * 2 + (Ug & 1);
+            if (!mbar_wait_bounded(&s_empty[sg], ((Ug >> 1) & 1) ^ 1, abort_flag, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_ts(tmem + sg * 64, tmem + FF_TM_Q + k * 8, make_sw128_desc(k_addr + k * 32, 16, 1024), idesc_s,
+                           k > 0 ? 1u : 0u);
+            umma_commit(&s_full[sg]);
+          } else {
+            if (!mbar_wait_bounded(&p_full[g], Ug & 1, abort_flag, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // K = 64 keys: B = 16 key rows of V_u per step (MN-major); each group's first unit
+            // of an item starts its accumulator
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_ts(tmem + FF_TM_O + g * 64, tmem + FF_TM_P + g * 32 + k * 8,
+                           make_sw128_desc(v_addr + k * 2048, 8192, 1024), idesc_o, (u >= 2 || k > 0) ? 1u : 0u);
+            umma_commit(&o_done[g]);
+            umma_commit(&st_empty[s]);  // the unit's S MMAs completed before its P was written
+          }
+          any = true;
+        }
+      }
+      if (!ok) {
+        raise_device_error(err, DEV_TIMEOUT);
+        *abort_flag = 1;
+        if (any) {
+          int never = 0;
+          umma_commit(&drain[warp - 1]);
+          mbar_wait_bounded(&drain[warp - 1], 0, reinterpret_cast<volatile int*>(&never), lim);
+        }
+      }
+    }
+  } else {
+    // ---------------- softmax: group g, query row r ----------------
+    const int g = (warp - 3) >> 2, q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const float sl2 = scale * LOG2E;
+    const bool issuer = (warp == 3 && lane == 0);  // issues the output tile's TMA store
+    float* xb = reinterpret_cast<float*>(sm + FF_OFF_X);  // [item parity][group][row] x (m, l)
+    bool fail = false;
+    // the Q rows of item `it` into the TMEM A operand: this group copies head dims [g*32, g*32 + 32)
+    auto load_q = [&](int it) -> bool {
+      const int qbuf = it & 1;
+      if (!mbar_wait_bounded(&q_full[qbuf], (it >> 1) & 1, abort_flag, lim)) return false;
+      const uint8_t* qt = sm + FF_OFF_Q + qbuf * FA_TILE;
+      fb_row_to_tmem(qt, r, 2 * g, tmem + lane_off + FF_TM_Q + (2 * g) * 8);
+      fb_row_to_tmem(qt, r, 2 * g + 1, tmem + lane_off + FF_TM_Q + (2 * g + 1) * 8);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(qa_full);
+        mbar_arrive(&q_empty[qbuf]);
+      }
+      return true;
+    };
+    if ((int)blockIdx.x < nitems) fail = !load_q(0);
+    int U0 = 0;  // first global unit of the current item
+    for (int it = 0, item = blockIdx.x; item < nitems && !fail; ++it, item += gridDim.x) {
+      const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
+      const int nu = 2 * (qb + 1);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int u = g; u < nu; u += 2) {
+        const int U = U0 + u, Ug = U >> 1, sg = g * 2 + (Ug & 1);
+        if (!mbar_wait_bounded(&s_full[sg], (Ug >> 1) & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[64];
+        tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(sg * 64), *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(sg * 64 + 32), *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[sg]);
+        if (u >= nu - 2) {  // the diagonal key block: keys after the query get -inf
+          const int kbase = (u & 1) * 64;
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (kbase + e > r) sv[e] = __float_as_uint(-INFINITY);
+        }
+        float mx;
+        {
+          float m8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sv[e]);
+#pragma unroll
+          for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sv[e]));
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        }
+        const float m_blk = mx * sl2;
+        // re-base only when the block maximum exceeds the reference by more than FF_REBASE
+        const bool rebase = m_blk > m_run + FF_REBASE;
+        const float m_use = rebase ? m_blk : m_run;
+        const float m_ref = m_use == -INFINITY ? 0.f : m_use;  // fully masked so far: P = 0
+        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint32_t pw[32];
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) {
+          const float p0 = ex2_fast(fmaf(__uint_as_float(sv[2 * e2]), sl2, -m_ref));
+          const float p1 = ex2_fast(fmaf(__uint_as_float(sv[2 * e2 + 1]), sl2, -m_ref));
+          rs8[(2 * e2) & 7] += p0;
+          rs8[(2 * e2 + 1) & 7] += p1;
+          pw[e2] = pack_bf16x2(p0, p1);
+        }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        // the group's previous P V product has finished reading P_g (and updating O_g)
+        if (Ug > 0 && !mbar_wait_bounded(&o_done[g], (Ug - 1) & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        tc_fence_after();
+        if (rebase && m_run != -INFINITY) {  // rescale this row of O_g to the new reference
+          const float corr = ex2_fast(m_run - m_use);
+          uint32_t ov[32];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            tmem_ld_32x32b_x32(tmem + lane_off + FF_TM_O + g * 64 + hh * 32, ov);
+            tmem_ld_wait();
+            uint32_t a[16], c[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              a[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
+              c[e] = __float_as_uint(__uint_as_float(ov[16 + e]) * corr);
+            }
+            tmem_st_32x32b_x16(tmem + lane_off + FF_TM_O + g * 64 + hh * 32, a);
+            tmem_st_32x32b_x16(tmem + lane_off + FF_TM_O + g * 64 + hh * 32 + 16, c);
+          }
+          l_run *= corr;
+        }
+        l_run += rs;
+        m_run = m_use;
+        // the first unit of an item (after the first item) starts a fresh O_g: both groups
+        // must have read the previous item's accumulators
+        if (u < 2 && it > 0 && !mbar_wait_bounded(o_read, (it - 1) & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        tmem_st_32x32b_x16(tmem + lane_off + FF_TM_P + g * 32, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
+        tmem_st_32x32b_x16(tmem + lane_off + FF_TM_P + g * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pw[16]));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[g]);
+      }
+      if (fail) break;
+      // the other group's last S product of this item is complete too: then no MMA
+      // still reads the TMEM Q operand, and the next item's Q can be written
+      {
+        const int uo = nu - 1 - g, Uo = U0 + uo, Ugo = Uo >> 1;
+        if (!mbar_wait_bounded(&s_full[(1 - g) * 2 + (Ugo & 1)], (Ugo >> 1) & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+      }
+      if (item + (int)gridDim.x < nitems && !load_q(it + 1)) {
+        fail = true;
+        break;
+      }
+      // merge the two groups' rows
+      float* xm = xb + ((it & 1) * 2 + g) * 256;
+      xm[r] = m_run;
+      xm[128 + r] = l_run;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(x_full);
+      // both groups' last P V products complete
+      const int Ug_last = (U0 + nu - 2 + g) >> 1, Ugo_last = (U0 + nu - 1 - g) >> 1;
+      if (!mbar_wait_bounded(x_full, it & 1, abort_flag, lim) ||
+          !mbar_wait_bounded(&o_done[g], Ug_last & 1, abort_flag, lim) ||
+          !mbar_wait_bounded(&o_done[1 - g], Ugo_last & 1, abort_flag, lim)) {
+        fail = true;
+        break;
+      }
+      const float* xo = xb + ((it & 1) * 2 + (1 - g)) * 256;
+      const float m_o = xo[r], l_o = xo[128 + r];
+      const float m = fmaxf(m_run, m_o);
+      const float a_s = m_run == -INFINITY ? 0.f : ex2_fast(m_run - m);
+      const float a_o = m_o == -INFINITY ? 0.f : ex2_fast(m_o - m);
+      const float l = l_run * a_s + l_o * a_o;
+      const float inv = 1.0f / l;
+      const float a0 = (g == 0 ? a_s : a_o) * inv, a1 = (g == 0 ? a_o : a_s) * inv;
+      // this thread's output columns [g*32, g*32 + 32) from O_0 and O_1
+      tc_fence_after();
+      uint32_t o0[32], o1[32];
+      tmem_ld_32x32b_x32(tmem + lane_off + FF_TM_O + g * 32, o0);
+      tmem_ld_32x32b_x32(tmem + lane_off + FF_TM_O + 64 + g * 32, o1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_read);
+      const int qrow = qb * FA_BM + r;
+      if (g == 0 && qrow < T) lse[(long long)bh * T + qrow] = (m + __log2f(l)) * LN2;
+      if (issuer && it > 0) {
+        bulk_wait_read<0>();
+        mbar_arrive(out_free);
+      }
+      if (!mbar_wait_bounded(out_free, (it & 1) ^ 1, abort_flag, lim)) {
+        fail = true;
+        break;
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float f[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          f[e] = __uint_as_float(o0[hh * 16 + e]) * a0 + __uint_as_float(o1[hh * 16 + e]) * a1;
+        fb_store16(sm + FF_OFF_OUT, r, g * 4 + hh * 2, f);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(out_full);
+      if (issuer) {
+        if (!mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+          fail = true;
+          break;
+        }
+        tma_store_3d(&tm_out, sm + FF_OFF_OUT, h * 64, qb * FA_BM, b);
+        bulk_commit();
+      }
+      U0 += nu;
+    }
+    if (issuer) bulk_wait_all();
+    if (fail && lane == 0) {
+      raise_device_error(err, DEV_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, FF_TMEM_COLS);
   }
 }
 

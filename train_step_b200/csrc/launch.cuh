@@ -553,16 +553,21 @@ inline int attention_fwd(const LaunchCtx& c, int dtype, const void* qkv, int B, 
   ProfScope ps(c, CAT_ATTN_FWD, 4.0 * B * NH * hd * (0.5 * T * (T + 1.0)), 0.0);
   if (dtype == GPT2_BF16) {
     if (hd != 64) return fail(c, GPT2_ERR_CONFIG, "attention (bf16): head dim must be 64");
-    if (reinterpret_cast<uintptr_t>(qkv) & 15) return fail(c, GPT2_ERR_CONFIG, "attention: qkv must be 16-byte aligned");
-    CUtensorMap tm;
-    if (!encode_qkv_map(&tm, qkv, 3LL * NH * 64, T, B)) return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
+    if ((reinterpret_cast<uintptr_t>(qkv) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
+      return fail(c, GPT2_ERR_CONFIG, "attention: qkv and out must be 16-byte aligned");
+    CUtensorMap tq, tkv64, tout;  // Q: 128-row tiles per item; K / V: 64-row tiles per unit
+    if (!encode_qkv_map(&tq, qkv, 3LL * NH * 64, T, B) || !encode_qkv_map(&tkv64, qkv, 3LL * NH * 64, T, B, 64) ||
+        !encode_qkv_map(&tout, out, (long long)NH * 64, T, B))
+      return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
     static bool attr_set = false;
     if (!attr_set) {
-      cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
+      cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FF_SMEM);
       attr_set = true;
     }
-    dim3 grid((T + FA_BM - 1) / FA_BM, B * NH);
-    attn_fwd_tc_kernel<<<grid, FA_THREADS, FA_SMEM, c.stream>>>(tm, (bf16*)out, lse, T, NH, scale, c.d_err,
+    // persistent: one CTA per SM loops over (query block, batch*head) items
+    const long long items = (long long)((T + FA_BM - 1) / FA_BM) * B * NH;
+    const int grid = items < c.num_sms ? (int)items : c.num_sms;
+    attn_fwd_tc_kernel<<<grid, FF_THREADS, FF_SMEM, c.stream>>>(tq, tkv64, tout, lse, T, NH, B * NH, scale, c.d_err,
                                                                 4000000000ull);
     return check_launch(c, "attn_fwd_tc");
   }
