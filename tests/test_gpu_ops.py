@@ -236,6 +236,38 @@ def test_attention_bf16(B, T, NH):
         assert rel_l2(got[:, sl], rd[:, sl]) < 2e-2, part
 
 
+def test_attention_bf16_running_max_rebase():
+    """Scores that grow by ~12 (log2 units) per 64 keys on odd query rows and stay flat
+    on even rows: the odd rows re-base their running maximum (rescaling their output
+    accumulator row) on every unit while their even neighbours in the same warp do not."""
+    B, T, NH, hd = 1, 512, 2, 64
+    C = NH * hd
+    gen = torch.Generator().manual_seed(40)
+    qkv = torch.zeros(B * T, 3 * C)
+    t = torch.arange(T, dtype=torch.float32)
+    for h in range(NH):
+        qkv[:, h * hd] = torch.where(t % 2 == 1, 32.0, 0.0)    # q_t = a_t e0
+        qkv[:, C + h * hd] = 33.0 * t / T                       # k_j = 33 j / T e0
+        qkv[:, 2 * C + h * hd:2 * C + (h + 1) * hd] = torch.randn(T, hd, generator=gen)
+    qkv = qkv.to(torch.bfloat16).to(DEV)
+    out = torch.zeros(B * T, C, dtype=torch.bfloat16, device=DEV)
+    lse = torch.zeros(B, NH, T, device=DEV)
+    tsb.attention_fwd(qkv, out, lse, B, T, NH, hd)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attention_fwd(g64(qkv), B, T, NH, hd, mode=1)
+    assert rel_l2(g64(out), ro) < 1e-2
+    assert np.max(np.abs(g64(lse) - rl) / np.maximum(1.0, np.abs(rl))) < 1e-3
+    dout = randn((B * T, C), 41, torch.bfloat16)
+    dqkv = torch.zeros_like(qkv)
+    tsb.attention_bwd(qkv, out, dout, lse, dqkv, B, T, NH, hd)
+    torch.cuda.synchronize()
+    rd = oracle.attention_bwd(g64(qkv), g64(dout), B, T, NH, hd)
+    got = g64(dqkv)
+    for part in range(3):
+        sl = slice(part * C, (part + 1) * C)
+        assert rel_l2(got[:, sl], rd[:, sl]) < 2e-2, part
+
+
 @pytest.mark.parametrize("B,T,NH,hd", [(2, 70, 2, 32), (1, 64, 4, 64), (2, 33, 1, 128)])
 def test_attention_fp32(B, T, NH, hd):
     C = NH * hd

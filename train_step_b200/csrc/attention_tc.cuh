@@ -121,12 +121,17 @@ __device__ __forceinline__ void fb_stage_row16(uint8_t* tile, int r, int cg, con
   fb_store16(tile, r, cg * 2, f);
 }
 
-// Bounded wait whose result is the same for every lane of the warp (lane 0 waits).
+// Bounded wait whose result is the same for every lane of the warp: lane 0 waits,
+// broadcasts the outcome, and on success every lane observes the completed phase
+// (its own acquire). Warps that go on to warp-collective tcgen05 instructions must
+// never split on a wait's outcome.
 __device__ __forceinline__ bool fb_warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t lim,
                                              int lane) {
   int ok = 1;
   if (lane == 0) ok = mbar_wait_bounded(bar, parity, abort, lim) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_try_wait(bar, parity);
+  return ok != 0;
 }
 
 // Copy 16 bf16 (columns [cg*16, cg*16 + 16)) of row r of a 128-byte-swizzled tile
@@ -371,7 +376,7 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
     // MMAs, whose results this warp has all seen)
     auto load_operands = [&](int it) -> bool {
       const int kvb = it & 1;
-      if (!mbar_wait_bounded(&kv_full[kvb], (it >> 1) & 1, abort_flag, lim)) return false;
+      if (!fb_warp_wait(&kv_full[kvb], (it >> 1) & 1, abort_flag, lim, lane)) return false;
       const uint8_t* kd = sm + FBK_OFF_KV + kvb * 2 * FA_TILE;
       fb_row_to_tmem(kd, r, cg, tmem + lane_off + FBK_TM_KV + cg * 8);
       fb_row_to_tmem(kd + FA_TILE, r, cg, tmem + lane_off + FBK_TM_KV + 32 + cg * 8);
@@ -391,8 +396,8 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
       for (int u = 0; u < nu; ++u, ++U) {
         const int sb = U % FB_SBUF, s = U % FBK_NST;
         // the producer's lse / D of this unit (acquired directly from its lanes), then the scores
-        if (!mbar_wait_bounded(&st_full[s], (U / FBK_NST) & 1, abort_flag, lim) ||
-            !mbar_wait_bounded(&s_full[sb], (U / FB_SBUF) & 1, abort_flag, lim)) {
+        if (!fb_warp_wait(&st_full[s], (U / FBK_NST) & 1, abort_flag, lim, lane) ||
+            !fb_warp_wait(&s_full[sb], (U / FB_SBUF) & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
@@ -423,7 +428,7 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
           }
         }
         // the previous unit's dV / dK MMAs have finished reading P^T and dS^T
-        if (!mbar_wait_bounded(p_free, (U & 1) ^ 1, abort_flag, lim)) {
+        if (!fb_warp_wait(p_free, (U & 1) ^ 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
@@ -440,7 +445,7 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
         fail = true;
         break;
       }
-      if (!mbar_wait_bounded(acc_full, it & 1, abort_flag, lim)) {
+      if (!fb_warp_wait(acc_full, it & 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
         bulk_wait_read<0>();
         mbar_arrive(out_free);
       }
-      if (!mbar_wait_bounded(out_free, (it & 1) ^ 1, abort_flag, lim)) {
+      if (!fb_warp_wait(out_free, (it & 1) ^ 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
@@ -467,13 +472,17 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(out_full);
       if (issuer) {
-        if (!mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+        if (mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+          tma_store_3d(&tm_out, sm + FBK_OFF_OUT, C + h * 64, kb * FA_BN, b);
+          tma_store_3d(&tm_out, sm + FBK_OFF_OUT + FA_TILE, 2 * C + h * 64, kb * FA_BN, b);
+          bulk_commit();
+        } else {
           fail = true;
-          break;
         }
-        tma_store_3d(&tm_out, sm + FBK_OFF_OUT, C + h * 64, kb * FA_BN, b);
-        tma_store_3d(&tm_out, sm + FBK_OFF_OUT + FA_TILE, 2 * C + h * 64, kb * FA_BN, b);
-        bulk_commit();
+      }
+      if (__shfl_sync(0xffffffffu, fail ? 1 : 0, 0)) {  // the issuer's warp leaves together
+        fail = true;
+        break;
       }
     }
     if (issuer) bulk_wait_all();  // the staging must outlive the stores' reads
@@ -703,7 +712,7 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
     // has seen all of their results.
     auto load_operands = [&](int it) -> bool {
       const int qdb = it & 1;
-      if (!mbar_wait_bounded(&qd_full[qdb], (it >> 1) & 1, abort_flag, lim)) return false;
+      if (!fb_warp_wait(&qd_full[qdb], (it >> 1) & 1, abort_flag, lim, lane)) return false;
       const uint8_t* qd = sm + FBQ_OFF_QD + qdb * 2 * FA_TILE;
       fb_row_to_tmem(qd, r, cg, tmem + lane_off + FBQ_TM_Q + cg * 8);
       fb_row_to_tmem(qd + FA_TILE, r, cg, tmem + lane_off + FBQ_TM_Q + 32 + cg * 8);
@@ -742,7 +751,7 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
       }
       for (int u = 0; u < nu; ++u, ++U) {
         const int sb = U % FB_SBUF, dsb = U & 1;
-        if (!mbar_wait_bounded(&s_full[sb], (U / FB_SBUF) & 1, abort_flag, lim)) {
+        if (!fb_warp_wait(&s_full[sb], (U / FB_SBUF) & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
@@ -764,7 +773,7 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
           ds[e] = pe * (__uint_as_float(dv[e]) - Dr);
         }
         // the dQ MMAs of unit U - 2 have finished reading this dS buffer
-        if (!mbar_wait_bounded(&ds_free[dsb], ((U >> 1) & 1) ^ 1, abort_flag, lim)) {
+        if (!fb_warp_wait(&ds_free[dsb], ((U >> 1) & 1) ^ 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
@@ -781,7 +790,7 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
         break;
       }
       const int ab = it & 1;
-      if (!mbar_wait_bounded(&acc_full[ab], (it >> 1) & 1, abort_flag, lim)) {
+      if (!fb_warp_wait(&acc_full[ab], (it >> 1) & 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
@@ -797,7 +806,7 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
         bulk_wait_read<0>();
         mbar_arrive(out_free);
       }
-      if (!mbar_wait_bounded(out_free, (it & 1) ^ 1, abort_flag, lim)) {
+      if (!fb_warp_wait(out_free, (it & 1) ^ 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
@@ -806,12 +815,16 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(out_full);
       if (issuer) {
-        if (!mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+        if (mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+          tma_store_3d(&tm_out, sm + FBQ_OFF_OUT, h * 64, qb * FA_BM, b);
+          bulk_commit();
+        } else {
           fail = true;
-          break;
         }
-        tma_store_3d(&tm_out, sm + FBQ_OFF_OUT, h * 64, qb * FA_BM, b);
-        bulk_commit();
+      }
+      if (__shfl_sync(0xffffffffu, fail ? 1 : 0, 0)) {  // the issuer's warp leaves together
+        fail = true;
+        break;
       }
       lse2 = lse_n * LOG2E;
       Dr = Dr_n;
@@ -1046,7 +1059,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
     // the Q rows of item `it` into the TMEM A operand: this group copies head dims [g*32, g*32 + 32)
     auto load_q = [&](int it) -> bool {
       const int qbuf = it & 1;
-      if (!mbar_wait_bounded(&q_full[qbuf], (it >> 1) & 1, abort_flag, lim)) return false;
+      if (!fb_warp_wait(&q_full[qbuf], (it >> 1) & 1, abort_flag, lim, lane)) return false;
       const uint8_t* qt = sm + FF_OFF_Q + qbuf * FA_TILE;
       fb_row_to_tmem(qt, r, 2 * g, tmem + lane_off + FF_TM_Q + (2 * g) * 8);
       fb_row_to_tmem(qt, r, 2 * g + 1, tmem + lane_off + FF_TM_Q + (2 * g + 1) * 8);
@@ -1067,7 +1080,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
       float m_run = -INFINITY, l_run = 0.f;
       for (int u = g; u < nu; u += 2) {
         const int U = U0 + u, Ug = U >> 1, sg = g * 2 + (Ug & 1);
-        if (!mbar_wait_bounded(&s_full[sg], (Ug >> 1) & 1, abort_flag, lim)) {
+        if (!fb_warp_wait(&s_full[sg], (Ug >> 1) & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
@@ -1111,13 +1124,17 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         }
         const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         // the group's previous P V product has finished reading P_g (and updating O_g)
-        if (Ug > 0 && !mbar_wait_bounded(&o_done[g], (Ug - 1) & 1, abort_flag, lim)) {
+        if (Ug > 0 && !fb_warp_wait(&o_done[g], (Ug - 1) & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
         tc_fence_after();
-        if (rebase && m_run != -INFINITY) {  // rescale this row of O_g to the new reference
-          const float corr = ex2_fast(m_run - m_use);
+        // rescale rows of O_g to their new reference. tcgen05.ld / st are warp-collective
+        // (.sync.aligned), so the whole warp takes this path when any of its rows re-bases;
+        // the other rows use the factor 1.
+        const bool my_rescale = rebase && m_run != -INFINITY;
+        if (__any_sync(0xffffffffu, my_rescale)) {
+          const float corr = my_rescale ? ex2_fast(m_run - m_use) : 1.0f;
           uint32_t ov[32];
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
@@ -1138,7 +1155,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         m_run = m_use;
         // the first unit of an item (after the first item) starts a fresh O_g: both groups
         // must have read the previous item's accumulators
-        if (u < 2 && it > 0 && !mbar_wait_bounded(o_read, (it - 1) & 1, abort_flag, lim)) {
+        if (u < 2 && it > 0 && !fb_warp_wait(o_read, (it - 1) & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
@@ -1154,7 +1171,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
       // still reads the TMEM Q operand, and the next item's Q can be written
       {
         const int uo = nu - 1 - g, Uo = U0 + uo, Ugo = Uo >> 1;
-        if (!mbar_wait_bounded(&s_full[(1 - g) * 2 + (Ugo & 1)], (Ugo >> 1) & 1, abort_flag, lim)) {
+        if (!fb_warp_wait(&s_full[(1 - g) * 2 + (Ugo & 1)], (Ugo >> 1) & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
@@ -1171,9 +1188,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
       if (lane == 0) mbar_arrive(x_full);
       // both groups' last P V products complete
       const int Ug_last = (U0 + nu - 2 + g) >> 1, Ugo_last = (U0 + nu - 1 - g) >> 1;
-      if (!mbar_wait_bounded(x_full, it & 1, abort_flag, lim) ||
-          !mbar_wait_bounded(&o_done[g], Ug_last & 1, abort_flag, lim) ||
-          !mbar_wait_bounded(&o_done[1 - g], Ugo_last & 1, abort_flag, lim)) {
+      if (!fb_warp_wait(x_full, it & 1, abort_flag, lim, lane) ||
+          !fb_warp_wait(&o_done[g], Ug_last & 1, abort_flag, lim, lane) ||
+          !fb_warp_wait(&o_done[1 - g], Ugo_last & 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
@@ -1200,7 +1217,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         bulk_wait_read<0>();
         mbar_arrive(out_free);
       }
-      if (!mbar_wait_bounded(out_free, (it & 1) ^ 1, abort_flag, lim)) {
+      if (!fb_warp_wait(out_free, (it & 1) ^ 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
@@ -1216,12 +1233,16 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(out_full);
       if (issuer) {
-        if (!mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+        if (mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
+          tma_store_3d(&tm_out, sm + FF_OFF_OUT, h * 64, qb * FA_BM, b);
+          bulk_commit();
+        } else {
           fail = true;
-          break;
         }
-        tma_store_3d(&tm_out, sm + FF_OFF_OUT, h * 64, qb * FA_BM, b);
-        bulk_commit();
+      }
+      if (__shfl_sync(0xffffffffu, fail ? 1 : 0, 0)) {  // the issuer's warp leaves together
+        fail = true;
+        break;
       }
       U0 += nu;
     }

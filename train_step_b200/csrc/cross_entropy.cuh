@@ -89,52 +89,33 @@ __global__ void __launch_bounds__(CE_PERSIST_THREADS, 1) cross_entropy_bf16_kern
       if (tid == 0) raise_device_error(err, DEV_TOKEN_RANGE);
       t = 0;
     }
-    // one pass: running max m and sum s of 2^(x*log2e - m) over this thread's columns
-    float m = -INFINITY, sacc = 0.f;
+    // Three passes over the row in shared memory, one exponential per logit:
+    //   1. the row maximum M (log2 units);
+    //   2. p = 2^(x*log2e - M) and its sum S; p (<= 1) replaces the logit in place as bf16;
+    //   3. dlogits = (p / S - onehot(t)) * scale. The target column is recomputed in fp32,
+    //      since p / S - 1 cancels there.
+    const float xt = __bfloat162float(z[t]) * LOG2E_CE;  // read before pass 2 overwrites it
+    bf16* zw = buf[cur];
+    float m = -INFINITY;
     for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
       const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-      float x[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const float2 f = unpack_bf16x2(w[q]);
-        x[2 * q] = vi * 8 + 2 * q < V ? f.x * LOG2E_CE : -INFINITY;
-        x[2 * q + 1] = vi * 8 + 2 * q + 1 < V ? f.y * LOG2E_CE : -INFINITY;
+        if (vi * 8 + 2 * q < V) m = fmaxf(m, f.x);
+        if (vi * 8 + 2 * q + 1 < V) m = fmaxf(m, f.y);
       }
-      float bm = x[0];
-#pragma unroll
-      for (int q = 1; q < 8; ++q) bm = fmaxf(bm, x[q]);
-      if (bm == -INFINITY) continue;  // all eight columns are padding
-      if (bm > m) {
-        sacc *= ex2_approx(m - bm);
-        m = bm;
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) sacc += ex2_approx(x[q] - m);
     }
-    // combine (m, s) pairs: warp, then block
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sacc, o);
-      const float mm = fmaxf(m, m2);
-      sacc = (m == -INFINITY ? 0.f : sacc * ex2_approx(m - mm)) + (m2 == -INFINITY ? 0.f : s2 * ex2_approx(m2 - mm));
-      m = mm;
-    }
-    if (lane == 0) {
-      red_m[warp] = m;
-      red_s[warp] = sacc;
-    }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red_m[warp] = m;
     __syncthreads();
     float M = red_m[0];
 #pragma unroll
     for (int w = 1; w < CE_PERSIST_THREADS / 32; ++w) M = fmaxf(M, red_m[w]);
-    float S = 0.f;
-#pragma unroll
-    for (int w = 0; w < CE_PERSIST_THREADS / 32; ++w)
-      S += red_m[w] == -INFINITY ? 0.f : red_s[w] * ex2_approx(red_m[w] - M);
-    const float ll2 = M + __log2f(S);  // lse in the log2 domain
-    if (tid == 0) row_loss[row] = (ll2 - __bfloat162float(z[t]) * LOG2E_CE) * LN2_CE;
-    bf16* dst = logits + (long long)row * ld;
+    M *= LOG2E_CE;
+    float sacc = 0.f;
     for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
       const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -143,8 +124,35 @@ __global__ void __launch_bounds__(CE_PERSIST_THREADS, 1) cross_entropy_bf16_kern
       for (int q = 0; q < 4; ++q) {
         const float2 f = unpack_bf16x2(w[q]);
         const int c = vi * 8 + 2 * q;
-        const float a = c < V ? (ex2_approx(f.x * LOG2E_CE - ll2) - (c == t ? 1.f : 0.f)) * scale : 0.f;
-        const float b = c + 1 < V ? (ex2_approx(f.y * LOG2E_CE - ll2) - (c + 1 == t ? 1.f : 0.f)) * scale : 0.f;
+        const float a = c < V ? ex2_approx(fmaf(f.x, LOG2E_CE, -M)) : 0.f;
+        const float b = c + 1 < V ? ex2_approx(fmaf(f.y, LOG2E_CE, -M)) : 0.f;
+        sacc += a + b;
+        o[q] = pack_bf16x2(a, b);
+      }
+      reinterpret_cast<uint4*>(zw)[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
+    if (lane == 0) red_s[warp] = sacc;
+    __syncthreads();
+    float S = 0.f;
+#pragma unroll
+    for (int w = 0; w < CE_PERSIST_THREADS / 32; ++w) S += red_s[w];
+    const float ll2 = M + __log2f(S);  // lse in the log2 domain
+    if (tid == 0) row_loss[row] = (ll2 - xt) * LN2_CE;
+    const float ps = scale / S;
+    const float dt_val = (ex2_approx(xt - M) / S - 1.f) * scale;
+    bf16* dst = logits + (long long)row * ld;
+    for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
+      const uint4 u = reinterpret_cast<const uint4*>(zw)[vi];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = unpack_bf16x2(w[q]);  // p, zero on padding columns
+        const int c = vi * 8 + 2 * q;
+        const float a = c == t ? dt_val : f.x * ps;
+        const float b = c + 1 == t ? dt_val : f.y * ps;
         o[q] = pack_bf16x2(a, b);
       }
       reinterpret_cast<uint4*>(dst)[vi] = make_uint4(o[0], o[1], o[2], o[3]);

@@ -475,7 +475,7 @@ inline int reduce_partials(const LaunchCtx& c, const float* part, int P, int nco
                            float* out2, int accumulate) {
   ProfScope ps(c, CAT_REDUCE, 0.0, 4.0 * nv * P * ncols + 8.0 * nv * ncols);
   ReduceOuts o{{out0, out1, out2}};
-  reduce_partials_kernel<<<dim3((ncols + 31) / 32, nv), 512, 0, c.stream>>>(part, P, ncols, o, accumulate);
+  reduce_partials_kernel<<<dim3((ncols + 7) / 8, nv), 256, 0, c.stream>>>(part, P, ncols, o, accumulate);
   return check_launch(c, "reduce_partials");
 }
 

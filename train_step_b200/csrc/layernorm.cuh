@@ -99,8 +99,16 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
     const float mu = mean[row], rs = rstd[row];
     const float* dyr = dy + row * C;
     const float* xr = x + row * C;
-    float4 vd[NV], vx[NV];
+    float4 vd[NV], vx[NV], vr[NV];
     float m1 = 0.f, m2 = 0.f;
+    float* dr = dres + row * C;
+    if (accumulate) {  // issued now, so its latency overlaps the row statistics
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int c = (i * 32 + lane) * 4;
+        if (c < C) vr[i] = *reinterpret_cast<const float4*>(dr + c);
+      }
+    }
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c = (i * 32 + lane) * 4;
@@ -127,7 +135,6 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
     }
     m1 = warp_sum(m1) / (float)C;
     m2 = warp_sum(m2) / (float)C;
-    float* dr = dres + row * C;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c = (i * 32 + lane) * 4;
@@ -136,11 +143,10 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
         float4 o = make_float4(rs * (vd[i].x * gg.x - m1 - vx[i].x * m2), rs * (vd[i].y * gg.y - m1 - vx[i].y * m2),
                                rs * (vd[i].z * gg.z - m1 - vx[i].z * m2), rs * (vd[i].w * gg.w - m1 - vx[i].w * m2));
         if (accumulate) {
-          float4 r = *reinterpret_cast<const float4*>(dr + c);
-          o.x += r.x;
-          o.y += r.y;
-          o.z += r.z;
-          o.w += r.w;
+          o.x += vr[i].x;
+          o.y += vr[i].y;
+          o.z += vr[i].z;
+          o.w += vr[i].w;
         }
         *reinterpret_cast<float4*>(dr + c) = o;
         if (dres_act) store4<T>(dres_act + row * C + c, o.x, o.y, o.z, o.w);
@@ -170,27 +176,37 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
 
 // Deterministic column reduction of up to three partial sets at once:
 // out_v[c] (+)= sum_{p < P} part[(v*P + p)*ncols + c] for v = blockIdx.y. Each CTA
-// owns 32 columns; warp w sums rows p = w, w + 16, ... in order, then the 16
-// warp sums are added in order.
+// owns 8 columns: thread t sums column t % 8 over rows p = t / 8, t / 8 + 32, ...
+// (four loads in flight), then the 32 row-group sums are added in order.
 struct ReduceOuts {
   float* out[3];
 };
-__global__ void __launch_bounds__(512) reduce_partials_kernel(const float* __restrict__ part, int P, int ncols,
+__global__ void __launch_bounds__(256) reduce_partials_kernel(const float* __restrict__ part, int P, int ncols,
                                                               ReduceOuts outs, int accumulate) {
-  __shared__ float sm[16][33];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float sm[32][9];
   const int v = blockIdx.y;
-  const int c = blockIdx.x * 32 + lane;
-  const float* base = part + (long long)v * P * ncols;
+  const int cl = threadIdx.x & 7, rg = threadIdx.x >> 3;
+  const int c = blockIdx.x * 8 + cl;
+  const float* base = part + (long long)v * P * ncols + c;
   float s = 0.f;
-  if (c < ncols)
-    for (int p = warp; p < P; p += 16) s += base[(long long)p * ncols + c];
-  sm[warp][lane] = s;
+  if (c < ncols) {
+    int p = rg;
+    for (; p + 96 < P; p += 128) {
+      const float a0 = base[(long long)p * ncols], a1 = base[(long long)(p + 32) * ncols];
+      const float a2 = base[(long long)(p + 64) * ncols], a3 = base[(long long)(p + 96) * ncols];
+      s += a0;
+      s += a1;
+      s += a2;
+      s += a3;
+    }
+    for (; p < P; p += 32) s += base[(long long)p * ncols];
+  }
+  sm[rg][cl] = s;
   __syncthreads();
-  if (warp == 0 && c < ncols) {
+  if (threadIdx.x < 8 && c < ncols) {
     float t = 0.f;
 #pragma unroll
-    for (int w = 0; w < 16; ++w) t += sm[w][lane];
+    for (int w = 0; w < 32; ++w) t += sm[w][cl];
     float* o = outs.out[v];
     o[c] = accumulate ? o[c] + t : t;
   }
@@ -206,7 +222,25 @@ __global__ void colsum_partial_kernel(const T* __restrict__ y, long long ld, int
   if (c >= ncols) return;
   const int r0 = blockIdx.y * rows_per, r1 = min(N, r0 + rows_per);
   float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int r = r0; r < r1; ++r) {
+  int r = r0;
+  if (sizeof(T) == 2) {  // four rows in flight per iteration; same summation order as one at a time
+    for (; r + 4 <= r1; r += 4) {
+      uint4 u[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) u[j] = *reinterpret_cast<const uint4*>(y + (long long)(r + j) * ld + c);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = unpack_bf16x2(w[q]);
+          s[2 * q] += f.x;
+          s[2 * q + 1] += f.y;
+        }
+      }
+    }
+  }
+  for (; r < r1; ++r) {
     const T* p = y + (long long)r * ld + c;
     if (sizeof(T) == 2) {
       const uint4 u = *reinterpret_cast<const uint4*>(p);
