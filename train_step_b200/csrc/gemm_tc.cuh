@@ -572,7 +572,8 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int kspl
     const long long row = i / (N / 4);
     const int c = (int)(i - row * (N / 4)) * 4;
     float4 s = *reinterpret_cast<const float4*>(partial + row * N + c);
-    for (int k = 1; k < ksplit; ++k) {
+#pragma unroll 4
+    for (int k = 1; k < ksplit; ++k) {  // loads of several slices in flight; sums still in slice order
       float4 t = *reinterpret_cast<const float4*>(partial + ((long long)k * M + row) * N + c);
       s.x += t.x;
       s.y += t.y;

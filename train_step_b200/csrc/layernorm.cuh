@@ -223,13 +223,13 @@ __global__ void colsum_partial_kernel(const T* __restrict__ y, long long ld, int
   const int r0 = blockIdx.y * rows_per, r1 = min(N, r0 + rows_per);
   float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   int r = r0;
-  if (sizeof(T) == 2) {  // four rows in flight per iteration; same summation order as one at a time
-    for (; r + 4 <= r1; r += 4) {
-      uint4 u[4];
+  if (sizeof(T) == 2) {  // eight rows in flight per iteration; same summation order as one at a time
+    for (; r + 8 <= r1; r += 8) {
+      uint4 u[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) u[j] = *reinterpret_cast<const uint4*>(y + (long long)(r + j) * ld + c);
+      for (int j = 0; j < 8; ++j) u[j] = *reinterpret_cast<const uint4*>(y + (long long)(r + j) * ld + c);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
