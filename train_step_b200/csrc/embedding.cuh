@@ -74,6 +74,74 @@ struct OpAdd {
   __device__ int operator()(int a, int b) const { return a + b; }
 };
 
+// Bitonic sort of NP = 1024 * E keys (ascending) with the keys in registers: key
+// i = (warp * E + e) * 32 + lane sits in register e of that lane. Partners i ^ j with
+// j < 32 are in another lane (shuffle), with 32 <= j < 32 E in another register of the
+// same thread, and only j >= 32 E crosses warps (one shared-memory pass). The sequence of
+// compare-exchanges is the textbook network, so the result is the same sorted array.
+template <int JE, int E>
+__device__ __forceinline__ void bitonic_reg_stage(uint32_t (&v)[E], int k, int base, int lane) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    if ((e & JE) == 0) {
+      const int e2 = e | JE;
+      const bool up = (((base + e) * 32 + lane) & k) == 0;
+      const uint32_t a = v[e], b = v[e2];
+      if ((a > b) == up) {
+        v[e] = b;
+        v[e2] = a;
+      }
+    }
+  }
+}
+template <int E>
+__device__ void bitonic_sort_regs(uint32_t* keys, int tid) {
+  constexpr int NP = 1024 * E;
+  const int lane = tid & 31, base = (tid >> 5) * E;
+  uint32_t v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] = keys[(base + e) * 32 + lane];
+  for (int k = 2; k <= NP; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 32 * E) {  // across warps, through shared memory
+#pragma unroll
+        for (int e = 0; e < E; ++e) keys[(base + e) * 32 + lane] = v[e];
+        __syncthreads();
+        for (int t = tid; t < NP / 2; t += 1024) {
+          const int i = ((t & ~(j - 1)) << 1) | (t & (j - 1)), ixj = i | j;
+          const uint32_t a = keys[i], b = keys[ixj];
+          if ((a > b) == ((i & k) == 0)) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = keys[(base + e) * 32 + lane];
+      } else if (j >= 32) {  // another register of this thread
+        switch (j >> 5) {
+          case 1: bitonic_reg_stage<1, E>(v, k, base, lane); break;
+          case 2: bitonic_reg_stage<2, E>(v, k, base, lane); break;
+          case 4: bitonic_reg_stage<4, E>(v, k, base, lane); break;
+          case 8: bitonic_reg_stage<8, E>(v, k, base, lane); break;
+          case 16: bitonic_reg_stage<16, E>(v, k, base, lane); break;
+        }
+      } else {  // another lane of this warp
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, v[e], j);
+          const bool up = ((((base + e) * 32) + lane) & k) == 0;
+          const bool lower = (lane & j) == 0;  // this lane holds the smaller index of the pair
+          v[e] = (lower == up) ? min(v[e], other) : max(v[e], other);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) keys[(base + e) * 32 + lane] = v[e];
+  __syncthreads();
+}
+
 // One CTA. Outputs:
 //   sorted_pos[i]        position of the i-th entry in (id, position) order
 //   chunk_start[c]       first sorted index of chunk c (chunks never straddle ids)
@@ -103,20 +171,26 @@ __global__ void __launch_bounds__(EMB_SORT_THREADS) token_sort_kernel(const int*
   }
   __syncthreads();
   // bitonic sort, ascending
-  for (int k = 2; k <= NP; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < NP; i += EMB_SORT_THREADS) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint32_t a = keys[i], b = keys[ixj];
-          const bool up = (i & k) == 0;
-          if ((a > b) == up) {
-            keys[i] = b;
-            keys[ixj] = a;
+  if (NP == 1024 * 16) {
+    bitonic_sort_regs<16>(keys, tid);
+  } else if (NP == 1024 * 32) {
+    bitonic_sort_regs<32>(keys, tid);
+  } else {
+    for (int k = 2; k <= NP; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < NP; i += EMB_SORT_THREADS) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const uint32_t a = keys[i], b = keys[ixj];
+            const bool up = (i & k) == 0;
+            if ((a > b) == up) {
+              keys[i] = b;
+              keys[ixj] = a;
+            }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
   // each thread owns E consecutive sorted entries

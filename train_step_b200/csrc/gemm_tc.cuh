@@ -473,7 +473,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               aux_par = (aux_par & ~(1u << (b ^ 1))) | ((uint32_t)(((n + 1) >> 1) & 1) << (b ^ 1));
             }
           } else if (tc_single_buffer<EPI>()) {
-            bulk_wait_read<0>();  // the previous chunk's stores have been read out
+            // GELU: u and gelu(u) go out as two bulk groups; the u half is free once the
+            // previous chunk's u store has been read (its gelu store may still be reading)
+            bulk_wait_read<1>();
           } else {
             bulk_wait_read<1>();  // this buffer's previous store (two chunks ago) has been read out
           }
@@ -520,6 +522,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           mbar_try_wait(&abar[b], (n >> 1) & 1);  // every lane observes the completed phase
         }
         const int col0 = tn * BN + c;
+        if (EPI == EPI_BF16_GELU) {
+          // u = acc + bias into the first half, stored as its own group; gelu(u) into the
+          // second half once the previous chunk's gelu store has read it
+          if (col0 < p.N) tc_epilogue_chunk<EPI_BF16, CW>(p, col0, lane, v, cur);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (col0 < p.N && row0 < p.M) tma_store_2d(&tmO, cur, col0, row0);
+            bulk_commit();
+            bulk_wait_read<1>();
+          }
+          __syncwarp();
+          if (col0 < p.N) {
+#pragma unroll
+            for (int j = 0; j < CW; ++j) v[j] = gelu_tanh_fast(v[j]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              *reinterpret_cast<uint4*>(row64_at(cur + 2048, lane, k)) =
+                  make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                             pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (col0 < p.N && row0 < p.M) tma_store_2d(&tmO2, cur + 2048, col0, row0);
+            bulk_commit();
+          }
+          continue;
+        }
         if (col0 < p.N) tc_epilogue_chunk<EPI, CW>(p, col0, lane, v, cur);
         fence_proxy_async_smem();
         __syncwarp();
