@@ -125,6 +125,10 @@ int gpt2_get_params(gpt2* m, float* host, int64_t n);
 int gpt2_set_params(gpt2* m, const float* host, int64_t n); /* also refreshes the bf16 shadow */
 int gpt2_get_grads(gpt2* m, float* host, int64_t n);
 int gpt2_get_adam(gpt2* m, float* m_host, float* v_host, int64_t n, int64_t* t_out);
+/* Restore the Adam moments and step count t (>= 0) from HOST memory, canonical order, for
+ * resuming from a checkpoint (with gpt2_set_params). Returns GPT2_ERR_CONFIG on a NULL
+ * pointer, n != gpt2_num_params or t < 0. Synchronises. */
+int gpt2_set_adam(gpt2* m, const float* m_host, const float* v_host, int64_t n, int64_t t);
 
 /* Device address and length (floats) of the flat fp32 gradient storage (the
  * library's internal, padded layout), e.g. for a data-parallel all-reduce of the

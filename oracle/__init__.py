@@ -6,6 +6,7 @@ may import this package. The product library never loads it.
 from __future__ import annotations
 
 import ctypes as ct
+import math
 import os
 import subprocess
 from dataclasses import dataclass
@@ -291,3 +292,22 @@ def set_threads(n: int) -> None:
 
 def get_threads() -> int:
     return int(lib().orc_get_threads())
+
+
+def lr_schedule(step: int, max_lr: float = 6e-4, min_lr: float = 6e-5, warmup: int = 715,
+                total: int = 19073) -> float:
+    """Learning rate at optimizer step `step` (0-based), in float64.
+
+    "GPT From Scratch", Training Recipe table: peak 6e-4, minimum 6e-5 (peak / 10), 715
+    warmup steps, 19,073 total steps; repository tour, "Cosine LR Schedule": linear warmup,
+    then cosine decay. Reading (the pages leave the indexing open): warmup step s takes
+    peak * (s + 1) / warmup; from s = warmup the rate is
+    min + (peak - min) * (1 + cos(pi * (s - warmup) / (total - warmup))) / 2, reaching the
+    minimum at s = total and staying there.
+    """
+    if step < warmup:
+        return max_lr * float(step + 1) / float(warmup)
+    if step >= total:
+        return min_lr
+    x = math.pi * float(step - warmup) / float(total - warmup)
+    return min_lr + (max_lr - min_lr) * (1.0 + math.cos(x)) / 2.0

@@ -49,6 +49,7 @@ _SYMBOLS = {
     "gpt2_set_params": ([ct.c_void_p, ct.c_void_p, ct.c_int64], ct.c_int),
     "gpt2_get_grads": ([ct.c_void_p, ct.c_void_p, ct.c_int64], ct.c_int),
     "gpt2_get_adam": ([ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int64, ct.POINTER(ct.c_int64)], ct.c_int),
+    "gpt2_set_adam": ([ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int64, ct.c_int64], ct.c_int),
     "gpt2_launch_count": ([ct.c_void_p, ct.POINTER(ct.c_int64)], ct.c_int),
     "gpt2_grad_buffer": ([ct.c_void_p, ct.POINTER(ct.c_void_p), ct.POINTER(ct.c_int64)], ct.c_int),
     "gpt2_profile": ([ct.c_void_p, ct.c_int], ct.c_int),
@@ -234,6 +235,14 @@ class GPT2:
         t = ct.c_int64()
         self._check(lib().gpt2_get_adam(self.h, m.ctypes.data, v.ctypes.data, m.size, ct.byref(t)))
         return m, v, t.value
+
+    def set_adam(self, m: np.ndarray, v: np.ndarray, t: int) -> None:
+        """Restore the Adam moments (canonical order) and step count."""
+        m = np.ascontiguousarray(m, dtype=np.float32)
+        v = np.ascontiguousarray(v, dtype=np.float32)
+        if m.size != self.num_params or v.size != self.num_params:
+            raise ValueError("Adam moments must have num_params entries")
+        self._check(lib().gpt2_set_adam(self.h, m.ctypes.data, v.ctypes.data, m.size, int(t)))
 
     def grad_buffer(self):
         """(device address, length in floats) of the flat gradient storage."""

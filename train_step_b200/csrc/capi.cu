@@ -660,6 +660,14 @@ int gpt2_get_adam(gpt2* m, float* m_host, float* v_host, int64_t n, int64_t* t_o
   return check_device_error(m);
 }
 
+int gpt2_set_adam(gpt2* m, const float* m_host, const float* v_host, int64_t n, int64_t t) {
+  if (!m || !m_host || !v_host || t < 0) return GPT2_ERR_CONFIG;
+  RK(xfer(m, m->m, nullptr, m_host, n, false, 1.0f));
+  RK(xfer(m, m->v, nullptr, v_host, n, false, 1.0f));
+  m->t = t;
+  return check_device_error(m);
+}
+
 int gpt2_grad_buffer(gpt2* m, float** dev, int64_t* n) {
   if (!m || !dev || !n) return GPT2_ERR_CONFIG;
   *dev = m->g;

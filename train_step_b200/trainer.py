@@ -1,0 +1,44 @@
+"""Training driver around the C-ABI model: gradient accumulation, optional data-parallel
+gradient averaging, the warmup + cosine learning-rate schedule, AdamW, evaluation loss
+and checkpoints ("GPT From Scratch", Training Recipe; recipe pieces: warmup plus cosine
+decay, clipping at 1.0, gradient accumulation).
+"""
+from __future__ import annotations
+
+from typing import Callable, Iterable
+
+from . import checkpoint
+from .schedule import CosineSchedule
+
+
+class Trainer:
+    def __init__(self, model, schedule: Callable[[int], float] | None = None, weight_decay: float = 0.1,
+                 beta1: float = 0.9, beta2: float = 0.95, allreduce: Callable[[], None] | None = None):
+        self.model = model
+        self.schedule = schedule or CosineSchedule()
+        self.weight_decay = weight_decay
+        self.beta1 = beta1
+        self.beta2 = beta2
+        self.allreduce = allreduce
+        self.step = 0
+
+    def train_step(self, micro_batches: Iterable) -> dict:
+        """One optimizer step over the (tokens, targets) micro-batches: returns the mean
+        micro-batch loss, the pre-clip gradient norm and the learning rate used."""
+        losses = [self.model.forward_backward(tok, tgt) for tok, tgt in micro_batches]
+        if self.allreduce is not None:
+            self.allreduce()
+        lr = self.schedule(self.step)
+        gnorm = self.model.step(lr, self.weight_decay, self.beta1, self.beta2)
+        self.step += 1
+        return {"loss": sum(losses) / len(losses), "grad_norm": gnorm, "lr": lr, "step": self.step}
+
+    def eval_loss(self, batches: Iterable) -> float:
+        losses = [self.model.forward(tok, tgt) for tok, tgt in batches]
+        return sum(losses) / len(losses)
+
+    def save(self, path: str) -> None:
+        checkpoint.save(self.model, path, step=self.step)
+
+    def load(self, path: str) -> None:
+        self.step, _ = checkpoint.load(self.model, path)
