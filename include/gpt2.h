@@ -152,6 +152,47 @@ int gpt2_profile_read(gpt2* m, int cat, char* name, int name_len, double* ms, in
 /* Number of kernel launches the handle has issued since creation (for reports). */
 int gpt2_launch_count(const gpt2* m, int64_t* out);
 
+/* ------------------------------------------------------------------------
+ * Generation with a key/value cache. "GPT From Scratch" (Architecture diagram)
+ * samples with temperature and top-k; "Genesis" (Project Structure; What I built
+ * from scratch) adds top-p, and lists a key/value cache under Roadmap; the cache is
+ * the incremental form of causal attention: keys and values of earlier positions do
+ * not change when a token is appended. bf16 models with head size
+ * 64 only (others: GPT2_ERR_CONFIG); 1 <= B <= min(B_max, 16) sequences of equal
+ * length. The cache ([L][B_max][T][2C] bf16, keys then values per row) is
+ * allocated by the first prefill and lives with the handle. Generation calls reuse
+ * the training activation memory: make them between optimizer steps, not between
+ * the micro-batches of one accumulation. Asynchronous on the handle's stream
+ * unless stated otherwise.
+ *
+ * gpt2_prefill: forward of B prompts of T0 tokens (tokens: host or device int32
+ * [B][T0], 1 <= T0 <= T), keys and values of every layer into cache positions
+ * 0..T0-1, and the fp32 logits of each prompt's last position into logits_out
+ * (DEVICE, caller-owned, row b at logits_out + b*ld, ld >= V). Synchronises and
+ * reports token-range errors.
+ * gpt2_decode_step: feed one token per sequence (tokens: host or device int32 [B],
+ * B equal to the prefill's) at the next position p = gpt2_kv_length; appends its
+ * keys and values at p and writes the fp32 logits of position p to logits_out.
+ * GPT2_ERR_SEQ_TOO_LONG once the cache holds T positions. A token id outside
+ * [0, V) raises the device error word (reported by the next synchronising call).
+ * gpt2_sample_topk: one index per row of fp32 logits [rows][ld] on the DEVICE:
+ * order the V logits by value descending, ties by lower index; keep the first k
+ * (1 <= k <= min(V, 1024)); weights w_j = exp((z_j - z_max)/temperature) in
+ * float64 (temperature > 0); running sums c_j taken in that order; with top_p < 1
+ * keep only the prefix up to the first j with c_j >= top_p * c_{k-1} (0 < top_p
+ * <= 1); return the index at the first kept j with c_j > u[row] * c_last, else the
+ * last kept one. u: DEVICE float64 [rows] in [0, 1), the caller's random draws.
+ * idx_out: DEVICE int32 [rows]. Logits must not be NaN. */
+int gpt2_prefill(gpt2* m, const int32_t* tokens, int B, int T0, float* logits_out, int64_t ld);
+int gpt2_decode_step(gpt2* m, const int32_t* tokens, int B, float* logits_out, int64_t ld);
+int gpt2_sample_topk(gpt2* m, const float* logits, int64_t ld, int rows, int k, float temperature, float top_p,
+                     const double* u, int32_t* idx_out);
+/* Wait for the handle's stream and report the device error word (e.g. a token id
+ * outside [0, V) fed to gpt2_decode_step). */
+int gpt2_synchronize(gpt2* m);
+/* Positions held in the key/value cache (0 before the first prefill). */
+int gpt2_kv_length(const gpt2* m, int* out);
+
 const char* gpt2_last_error(const gpt2* m);
 void gpt2_destroy(gpt2* m);
 
@@ -256,6 +297,11 @@ int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, con
  * it uses before reading it); calls whose kernels overlap on the GPU race. */
 int gpt2_op_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, const void* dout,
                                   const float* f32_lse, int B, int T, int NH, int hd, void* dqkv, void* stream);
+
+/* gpt2_sample_topk without a handle, for V given explicitly (same rules and
+ * arguments, all DEVICE pointers). Synchronises. */
+int gpt2_op_sample_topk(const float* logits, int64_t ld, int rows, int V, int k, float temperature, float top_p,
+                        const double* u, int32_t* idx_out, void* stream);
 
 const char* gpt2_op_last_error(void);
 

@@ -311,3 +311,44 @@ def lr_schedule(step: int, max_lr: float = 6e-4, min_lr: float = 6e-5, warmup: i
         return min_lr
     x = math.pi * float(step - warmup) / float(total - warmup)
     return min_lr + (max_lr - min_lr) * (1.0 + math.cos(x)) / 2.0
+
+
+def sample_topk(z, k: int, temperature: float, top_p: float, u: float) -> int:
+    """Index drawn from one logits row by temperature / top-k / top-p sampling.
+
+    "GPT From Scratch", Architecture diagram: generation samples with temperature and
+    top-k; "Genesis", Project Structure and What I built from scratch: temperature, top-k
+    and top-p (nucleus) sampling. The pages give no tie or precision rule; the reading:
+    rank the logits by value, larger first, equal values by lower index (-0.0 equals
+    +0.0); keep the first k; weight each kept logit by exp((z - z_max) / temperature) in
+    float64; form running sums c_0, c_1, ... of the weights in rank order; with top_p < 1
+    keep only ranks up to the first one whose running sum reaches top_p * c_{k-1}; return
+    the first kept rank whose running sum exceeds u * (running sum of the last kept rank),
+    or the last kept rank. temperature and top_p are taken at float32 precision (the
+    library's argument type), u in float64.
+    """
+    z = [float(x) for x in np.asarray(z, dtype=np.float32).reshape(-1)]
+    V = len(z)
+    if not (1 <= k <= V):
+        raise ValueError("1 <= k <= V")
+    temperature = float(np.float32(temperature))
+    top_p = float(np.float32(top_p))
+    ranked = sorted(range(V), key=lambda i: (-z[i], i))[:k]
+    zmax = z[ranked[0]]
+    weights = [math.exp((z[i] - zmax) / temperature) for i in ranked]
+    running = []
+    acc = 0.0
+    for w in weights:
+        acc += w
+        running.append(acc)
+    last = k - 1
+    if top_p < 1.0:
+        for j in range(k):
+            if running[j] >= top_p * running[k - 1]:
+                last = j
+                break
+    target = u * running[last]
+    for j in range(last + 1):
+        if running[j] > target:
+            return ranked[j]
+    return ranked[last]

@@ -50,7 +50,7 @@ def operand(rows, cols, mn, seed, dtype):
     return logical, stored, ld
 
 
-GEMM_SHAPES = [(300, 384, 200), (256, 128, 64), (128, 520, 136), (1000, 768, 768), (296, 2304, 1024)]
+GEMM_SHAPES = [(300, 384, 200), (256, 128, 64), (128, 520, 136), (1000, 768, 768), (296, 2304, 1024), (15, 256, 136)]
 MAJORS = [(False, False), (False, True), (True, True)]
 
 

@@ -83,6 +83,14 @@ _SYMBOLS = {
                                ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_op_attention_bwd_noalloc": ([ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int,
                                        ct.c_int, ct.c_int, ct.c_int, ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_prefill": ([ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_void_p, ct.c_int64], ct.c_int),
+    "gpt2_decode_step": ([ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_void_p, ct.c_int64], ct.c_int),
+    "gpt2_sample_topk": ([ct.c_void_p, ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_float, ct.c_float,
+                          ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_kv_length": ([ct.c_void_p, ct.POINTER(ct.c_int)], ct.c_int),
+    "gpt2_synchronize": ([ct.c_void_p], ct.c_int),
+    "gpt2_op_sample_topk": ([ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_int, ct.c_float, ct.c_float,
+                             ct.c_void_p, ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_op_last_error": ([], ct.c_char_p),
 }
 
@@ -271,6 +279,90 @@ class GPT2:
         self._check(lib().gpt2_launch_count(self.h, ct.byref(n)))
         return n.value
 
+    # ---- generation (bf16 models) ----
+    # The library runs on the handle's stream (its own unless one was given). With
+    # sync=True (the default) a call first waits for torch's current stream (so inputs made
+    # there are ready) and returns after its own kernels have finished, so its outputs can
+    # be used from any stream; sync=False does neither: inputs must come from the handle's
+    # stream and outputs stay in flight there (call synchronize() before using them
+    # elsewhere).
+    def synchronize(self) -> None:
+        self._check(lib().gpt2_synchronize(self.h))
+
+    def _logits_buffer(self, B: int, out=None):
+        import torch
+        if out is None:
+            out = torch.empty(B, self.cfg.V, device="cuda", dtype=torch.float32)
+        return out
+
+    def prefill(self, tokens, logits_out=None):
+        """Forward of B prompts (int32 [B, T0], host or CUDA), fill the key/value cache,
+        return the fp32 logits [B, V] of each prompt's last position (a CUDA tensor).
+        Always synchronises (before and after, as sync=True does)."""
+        import torch
+        B, T0 = tokens.shape
+        out = self._logits_buffer(B, logits_out)
+        torch.cuda.current_stream().synchronize()
+        self._check(lib().gpt2_prefill(self.h, _ptr(tokens), B, T0, _ptr(out), out.stride(0)))
+        return out
+
+    def decode_step(self, tokens, logits_out=None, sync: bool = True):
+        """Append one token per sequence (int32 [B]) at the next cache position; return
+        the fp32 logits [B, V] of that position."""
+        import torch
+        B = tokens.shape[0]
+        out = self._logits_buffer(B, logits_out)
+        if sync:
+            torch.cuda.current_stream().synchronize()
+        self._check(lib().gpt2_decode_step(self.h, _ptr(tokens), B, _ptr(out), out.stride(0)))
+        if sync:
+            self.synchronize()
+        return out
+
+    def sample_topk(self, logits, k: int, temperature: float, top_p: float, u, out=None, sync: bool = True):
+        """One index per logits row (int32 CUDA tensor); u: float64 CUDA tensor [rows] in [0, 1)."""
+        import torch
+        rows = logits.shape[0]
+        if out is None:
+            out = torch.empty(rows, device="cuda", dtype=torch.int32)
+        if sync:
+            torch.cuda.current_stream().synchronize()
+        self._check(lib().gpt2_sample_topk(self.h, _ptr(logits), logits.stride(0), rows, k, temperature, top_p,
+                                           _ptr(u), _ptr(out)))
+        if sync:
+            self.synchronize()
+        return out
+
+    @property
+    def kv_length(self) -> int:
+        n = ct.c_int()
+        self._check(lib().gpt2_kv_length(self.h, ct.byref(n)))
+        return n.value
+
+    def generate(self, prompt, max_new_tokens: int, k: int = 50, temperature: float = 1.0, top_p: float = 1.0,
+                 seed: int = 0):
+        """Sample max_new_tokens tokens after each prompt row (int32 [B, T0]); returns the
+        int32 CUDA tensor [B, T0 + max_new_tokens]. The uniform draws u come from numpy's
+        PCG64 seeded with `seed`, shape [max_new_tokens, B], and are passed to the sampler;
+        the loop stays on the handle's stream and synchronises once at the end."""
+        import torch
+        B, T0 = prompt.shape
+        if T0 + max_new_tokens > self.cfg.T + 1:
+            raise ValueError("prompt plus new tokens exceed the block size + 1")
+        prompt = torch.as_tensor(prompt, dtype=torch.int32).cuda().contiguous()
+        if max_new_tokens == 0:
+            return prompt
+        u = torch.from_numpy(np.random.default_rng(seed).random((max_new_tokens, B))).cuda()
+        new = torch.empty(max_new_tokens, B, device="cuda", dtype=torch.int32)
+        torch.cuda.current_stream().synchronize()  # inputs made on torch's stream are ready
+        logits = self.prefill(prompt)
+        for s in range(max_new_tokens):
+            self.sample_topk(logits, k, temperature, top_p, u[s], out=new[s], sync=False)
+            if s + 1 < max_new_tokens:
+                self.decode_step(new[s], logits_out=logits, sync=False)
+        self.synchronize()
+        return torch.cat([prompt, new.t()], dim=1)
+
 
 # ---------------------------------------------------------------------------
 # op-level wrappers (torch CUDA tensors in, results written in place)
@@ -312,6 +404,12 @@ def layernorm_bwd(dy, x, g, mean, rstd, dres, dres_act, dg, db, accumulate=False
     _op(lib().gpt2_op_layernorm_bwd(dt, _ptr(dy), _ptr(x), _ptr(g), _ptr(mean), _ptr(rstd), N, C, _ptr(dres),
                                     _ptr(dres_act), int(accumulate), _ptr(dg), _ptr(db), int(accumulate_params),
                                     _stream(stream)))
+
+
+def sample_topk(logits, V, k, temperature, top_p, u, out, stream=None):
+    """Op-level sampler: logits fp32 [rows, ld] (ld = stride), u float64 [rows], out int32 [rows]."""
+    _op(lib().gpt2_op_sample_topk(_ptr(logits), logits.stride(0), logits.shape[0], V, k, temperature, top_p,
+                                  _ptr(u), _ptr(out), _stream(stream)))
 
 
 def attention_fwd(qkv, out, lse, B, T, NH, hd, stream=None):

@@ -63,6 +63,16 @@ struct gpt2 {
   size_t part_floats = 0, splitk_floats = 0;
   int *tok = nullptr, *tgt = nullptr;
   void* emb_scratch = nullptr;
+  // generation: key/value cache [L][B_max][T][2C] bf16 (allocated by the first prefill)
+  bf16* kv = nullptr;
+  int kv_B = 0, kv_len = 0;
+  int* d_pos = nullptr;        // device copy of the next cache position (read by captured steps)
+  float* dec_part = nullptr;   // split-key partial attention results
+  cudaGraphExec_t dec_graph = nullptr;  // captured decode step, for (dec_B, dec_logits, dec_ld)
+  int dec_B = 0;
+  float* dec_logits = nullptr;
+  int64_t dec_ld = 0;
+  long long dec_graph_launches = 0;
   // scalars
   int* d_err = nullptr;
   float* d_loss = nullptr;
@@ -236,12 +246,13 @@ int copy_tokens(gpt2* m, int* dst, const int32_t* src, size_t n) {
   return GPT2_OK;
 }
 
-// Forward of one micro-batch; with `backward`, also the backward pass that adds
-// the gradients of this micro-batch's mean loss into m->g.
-int run_micro_batch(gpt2* m, int B, int T, bool backward) {
+// Forward of the embedding, the L blocks and the final LayerNorm for B sequences of T
+// tokens already in m->tok: leaves every activation the backward pass reads, the keys and
+// values of each layer in its qkv activation, and ln_f's output in m->xf.
+int forward_layers(gpt2* m, int B, int T) {
   LaunchCtx c = m->ctx();
   const int dt = m->cfg.dtype;
-  const int N = B * T, C = m->C, F = m->F, L = m->L, NH = m->NH, hd = m->hd, Vp = m->Vp;
+  const int N = B * T, C = m->C, F = m->F, L = m->L, NH = m->NH, hd = m->hd;
   const int64_t NC = (int64_t)m->Nmax * C, NF = (int64_t)m->Nmax * F, N3C = 3 * NC;
   const int64_t NLSE = (int64_t)m->cfg.B_max * NH * m->T;
   const int ab = m->act_bytes;
@@ -254,7 +265,6 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
                            : layernorm_fwd_t<float>(c, x, gg, bb, N, C, (float*)y, mu, rs);
   };
 
-  // ---------------- forward ----------------
   RK(embedding_fwd(c, m->tok, m->wte, m->wpe, N, T, C, m->cfg.V, xs(0)));
   for (int l = 0; l < L; ++l) {
     const LayerP& w = m->lp[l];
@@ -278,6 +288,26 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
                             w.pj_b, xs(2 * l + 1), C, 0, 1}));
   }
   RK(LN_F(xs(2 * L), m->lnf_g, m->lnf_b, m->xf, mean(2 * L), rstd(2 * L)));
+
+  return GPT2_OK;
+}
+
+// Forward of one micro-batch; with `backward`, also the backward pass that adds
+// the gradients of this micro-batch's mean loss into m->g.
+int run_micro_batch(gpt2* m, int B, int T, bool backward) {
+  LaunchCtx c = m->ctx();
+  const int dt = m->cfg.dtype;
+  const int N = B * T, C = m->C, F = m->F, L = m->L, NH = m->NH, hd = m->hd, Vp = m->Vp;
+  const int64_t NC = (int64_t)m->Nmax * C, NF = (int64_t)m->Nmax * F, N3C = 3 * NC;
+  const int64_t NLSE = (int64_t)m->cfg.B_max * NH * m->T;
+  const int ab = m->act_bytes;
+  auto xs = [&](int i) { return m->x + (int64_t)i * NC; };
+  auto mean = [&](int i) { return m->stat_mean + (int64_t)i * m->Nmax; };
+  auto rstd = [&](int i) { return m->stat_rstd + (int64_t)i * m->Nmax; };
+  auto ACT = [&](char* base, int l, int64_t per) -> void* { return base + (int64_t)l * per * ab; };
+
+  // ---------------- forward ----------------
+  RK(forward_layers(m, B, T));
 
   // ---------------- head + cross-entropy, chunk by chunk ----------------
   const float* headw = m->cfg.tied ? m->wte : m->head;
@@ -668,6 +698,167 @@ int gpt2_set_adam(gpt2* m, const float* m_host, const float* v_host, int64_t n, 
   return check_device_error(m);
 }
 
+// ---------------- generation ----------------
+namespace {
+int64_t kv_seq_elems(const gpt2* m) { return (int64_t)m->T * 2 * m->C; }
+bf16* kv_layer(gpt2* m, int l) { return m->kv + (int64_t)l * m->cfg.B_max * kv_seq_elems(m); }
+
+// fp32 logits of B rows of ln_f output (bf16, row stride ldx) against the head weight.
+int head_logits(gpt2* m, const bf16* xf_rows, int64_t ldx, int B, float* logits_out, int64_t ld) {
+  const float* headw = m->cfg.tied ? m->wte : m->head;
+  return gemv_bf16(m->ctx(), EPI_F32, xf_rows, ldx, B, (const bf16*)m->W(headw), m->cfg.V, m->C, nullptr, logits_out,
+                   ld, nullptr, 0);
+}
+
+int check_generation(gpt2* m, float* logits_out, int64_t ld, int B) {
+  if (!m) return GPT2_ERR_CONFIG;
+  if (m->cfg.dtype != GPT2_BF16) return set_err(m, GPT2_ERR_CONFIG, "generation needs a bf16 model");
+  if (m->hd != DEC_HD) return set_err(m, GPT2_ERR_CONFIG, "generation needs head size 64");
+  if (!logits_out || ld < m->cfg.V) return set_err(m, GPT2_ERR_CONFIG, "logits_out with ld >= V required");
+  if (B < 1 || B > m->cfg.B_max || B > DEC_MAX_B) return set_err(m, GPT2_ERR_BATCH, "1 <= B <= min(B_max, 16)");
+  return GPT2_OK;
+}
+}  // namespace
+
+int gpt2_prefill(gpt2* m, const int32_t* tokens, int B, int T0, float* logits_out, int64_t ld) {
+  RK(check_generation(m, logits_out, ld, B));
+  if (!tokens) return set_err(m, GPT2_ERR_CONFIG, "tokens required");
+  if (T0 < 1 || T0 > m->T) return set_err(m, GPT2_ERR_SEQ_TOO_LONG, "1 <= T0 <= block size");
+  if (m->k > 0) return set_err(m, GPT2_ERR_BATCH, "prefill between micro-batches of an accumulation");
+  if (!m->kv) {
+    const size_t bytes = (size_t)m->L * m->cfg.B_max * kv_seq_elems(m) * sizeof(bf16);
+    const size_t part = (size_t)m->cfg.B_max * m->NH * DEC_MAX_SPLIT * DEC_PART * sizeof(float);
+    if (cudaMalloc(&m->kv, bytes) != cudaSuccess || cudaMalloc(&m->d_pos, 256) != cudaSuccess ||
+        cudaMalloc(&m->dec_part, part) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(m->kv);
+      cudaFree(m->d_pos);
+      m->kv = nullptr;
+      m->d_pos = nullptr;
+      m->dec_part = nullptr;
+      return set_err(m, GPT2_ERR_OOM, "key/value cache");
+    }
+  }
+  RK(copy_tokens(m, m->tok, tokens, (size_t)B * T0));
+  RK(forward_layers(m, B, T0));
+  LaunchCtx c = m->ctx();
+  const int64_t N3C = 3 * (int64_t)m->Nmax * m->C;
+  for (int l = 0; l < m->L; ++l)
+    RK(kv_fill(c, (const bf16*)(m->qkv + (int64_t)l * N3C * m->act_bytes), B, T0, m->C, kv_layer(m, l),
+               kv_seq_elems(m)));
+  // the last position of each prompt: rows b*T0 + T0-1 of ln_f's output
+  RK(head_logits(m, (const bf16*)m->xf + (int64_t)(T0 - 1) * m->C, (int64_t)T0 * m->C, B, logits_out, ld));
+  set_pos_kernel<<<1, 1, 0, m->stream>>>(m->d_pos, T0);
+  RK(check_launch(c, "set_pos"));
+  m->kv_B = B;
+  m->kv_len = T0;
+  return check_device_error(m);
+}
+
+namespace {
+// Enqueue one decode step for the B tokens in m->tok at the position in m->d_pos (which
+// the step then advances): no synchronisation, so that it can be captured.
+int decode_body(gpt2* m, int B, float* logits_out, int64_t ld) {
+  LaunchCtx c = m->ctx();
+  const int C = m->C, F = m->F;
+  float* x0 = m->x;
+  float* x1 = m->x + (int64_t)B * C;
+  bf16* h = (bf16*)m->h1;
+  bf16* qkv = (bf16*)m->qkv;
+  bf16* att = (bf16*)m->att;
+  bf16* a = (bf16*)m->a;
+  const int S = decode_splits(B, m->NH, m->num_sms);
+  {
+    ProfScope ps(c, CAT_EMB_FWD, 0.0, 12.0 * B * C);
+    embed_decode_kernel<<<(B * 32 + 255) / 256, 256, 0, m->stream>>>(m->tok, m->wte, m->wpe, m->d_pos, x0, B, C,
+                                                                    m->cfg.V, m->d_err);
+    RK(check_launch(c, "embed_decode"));
+  }
+  for (int l = 0; l < m->L; ++l) {
+    const LayerP& w = m->lp[l];
+    RK(layernorm_fwd_t<bf16>(c, x0, w.ln1_g, w.ln1_b, B, C, h, m->stat_mean, m->stat_rstd));
+    RK(gemv_bf16(c, EPI_BF16, h, C, B, (const bf16*)m->W(w.qkv_w), 3 * C, C, w.qkv_b, qkv, 3 * C, nullptr, 0));
+    RK(decode_attention(c, qkv, kv_layer(m, l), kv_seq_elems(m), m->T, B, C, m->NH, m->d_pos, S, att, m->dec_part,
+                        (double)m->kv_len + 1.0));
+    RK(gemv_bf16(c, EPI_F32_RESID, att, C, B, (const bf16*)m->W(w.ao_w), C, C, w.ao_b, x1, C, x0, C));
+    RK(layernorm_fwd_t<bf16>(c, x1, w.ln2_g, w.ln2_b, B, C, h, m->stat_mean, m->stat_rstd));
+    RK(gemv_bf16(c, EPI_BF16_GELU, h, C, B, (const bf16*)m->W(w.fc_w), F, C, w.fc_b, a, F, nullptr, 0));
+    RK(gemv_bf16(c, EPI_F32_RESID, a, F, B, (const bf16*)m->W(w.pj_w), C, F, w.pj_b, x0, C, x1, C));
+  }
+  RK(layernorm_fwd_t<bf16>(c, x0, m->lnf_g, m->lnf_b, B, C, h, m->stat_mean, m->stat_rstd));
+  RK(head_logits(m, h, C, B, logits_out, ld));
+  set_pos_kernel<<<1, 1, 0, m->stream>>>(m->d_pos, -1);
+  return check_launch(c, "set_pos");
+}
+
+// Capture decode_body into a CUDA graph for (B, logits_out, ld).
+int capture_decode(gpt2* m, int B, float* logits_out, int64_t ld) {
+  if (m->dec_graph) {
+    cudaGraphExecDestroy(m->dec_graph);
+    m->dec_graph = nullptr;
+  }
+  const long long before = m->launches;
+  CK(m, cudaStreamBeginCapture(m->stream, cudaStreamCaptureModeThreadLocal));
+  const int r = decode_body(m, B, logits_out, ld);
+  cudaGraph_t g = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(m->stream, &g);
+  if (r || e != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return r ? r : cuda_err(m, e, "decode step capture");
+  }
+  const cudaError_t ei = cudaGraphInstantiate(&m->dec_graph, g, 0);
+  cudaGraphDestroy(g);
+  if (ei != cudaSuccess) {
+    m->dec_graph = nullptr;
+    return cuda_err(m, ei, "decode step graph");
+  }
+  m->dec_graph_launches = m->launches - before;
+  m->launches = before;
+  m->dec_B = B;
+  m->dec_logits = logits_out;
+  m->dec_ld = ld;
+  return GPT2_OK;
+}
+}  // namespace
+
+int gpt2_decode_step(gpt2* m, const int32_t* tokens, int B, float* logits_out, int64_t ld) {
+  RK(check_generation(m, logits_out, ld, B));
+  if (!tokens) return set_err(m, GPT2_ERR_CONFIG, "tokens required");
+  if (!m->kv || m->kv_len == 0) return set_err(m, GPT2_ERR_CONFIG, "decode step before a prefill");
+  if (B != m->kv_B) return set_err(m, GPT2_ERR_BATCH, "B must equal the prefill's B");
+  if (m->kv_len >= m->T) return set_err(m, GPT2_ERR_SEQ_TOO_LONG, "the cache holds block-size positions");
+  RK(copy_tokens(m, m->tok, tokens, (size_t)B));
+  if (m->prof.on) {
+    RK(decode_body(m, B, logits_out, ld));  // launch by launch, so that each kernel is timed
+  } else {
+    if (!m->dec_graph || m->dec_B != B || m->dec_logits != logits_out || m->dec_ld != ld)
+      RK(capture_decode(m, B, logits_out, ld));
+    CK(m, cudaGraphLaunch(m->dec_graph, m->stream));
+    m->launches += m->dec_graph_launches;
+  }
+  m->kv_len += 1;
+  return GPT2_OK;
+}
+
+int gpt2_sample_topk(gpt2* m, const float* logits, int64_t ld, int rows, int k, float temperature, float top_p,
+                     const double* u, int32_t* idx_out) {
+  if (!m) return GPT2_ERR_CONFIG;
+  if (!logits || !u || !idx_out) return set_err(m, GPT2_ERR_CONFIG, "logits, u and idx_out are required");
+  return sample_topk(m->ctx(), logits, ld, rows, m->cfg.V, k, temperature, top_p, u, idx_out);
+}
+
+int gpt2_synchronize(gpt2* m) {
+  if (!m) return GPT2_ERR_CONFIG;
+  return check_device_error(m);
+}
+
+int gpt2_kv_length(const gpt2* m, int* out) {
+  if (!m || !out) return GPT2_ERR_CONFIG;
+  *out = m->kv_len;
+  return GPT2_OK;
+}
+
 int gpt2_grad_buffer(gpt2* m, float** dev, int64_t* n) {
   if (!m || !dev || !n) return GPT2_ERR_CONFIG;
   *dev = m->g;
@@ -717,6 +908,10 @@ void gpt2_destroy(gpt2* m) {
   if (!m) return;
   if (m->stream) cudaStreamSynchronize(m->stream);
   cudaFree(m->arena);
+  cudaFree(m->kv);
+  cudaFree(m->d_pos);
+  cudaFree(m->dec_part);
+  if (m->dec_graph) cudaGraphExecDestroy(m->dec_graph);
   cudaFree(m->p);
   cudaFree(m->g);
   cudaFree(m->m);
@@ -950,6 +1145,19 @@ int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, con
   OpCtx o(stream);
   RK(o.alloc_err());
   int r = cross_entropy(o.c, dtype, logits, ld, N, V, targets, scale, row_loss);
+  int r2 = o.finish();
+  return r ? r : r2;
+}
+
+int gpt2_op_sample_topk(const float* logits, int64_t ld, int rows, int V, int k, float temperature, float top_p,
+                        const double* u, int32_t* idx_out, void* stream) {
+  if (!logits || !u || !idx_out) {
+    g_op_error = "sample_topk: logits, u and idx_out are required";
+    return GPT2_ERR_CONFIG;
+  }
+  OpCtx o(stream);
+  RK(o.alloc_err());
+  int r = sample_topk(o.c, logits, ld, rows, V, k, temperature, top_p, u, idx_out);
   int r2 = o.finish();
   return r ? r : r2;
 }

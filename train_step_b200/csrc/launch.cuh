@@ -4,6 +4,7 @@
 #pragma once
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdio>
 #include <string>
 #include <vector>
@@ -14,10 +15,12 @@
 #include "attention_tc.cuh"
 #include "common.cuh"
 #include "cross_entropy.cuh"
+#include "decode.cuh"
 #include "embedding.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "layernorm.cuh"
+#include "sample.cuh"
 
 namespace g2 {
 
@@ -37,13 +40,17 @@ enum ProfCat : int {
   CAT_EMB_BWD,
   CAT_CE,
   CAT_ADAMW,
+  CAT_DEC_GEMV,
+  CAT_DEC_ATTN,
+  CAT_SAMPLE,
   CAT_COUNT
 };
 inline const char* prof_cat_name(int c) {
   static const char* n[CAT_COUNT] = {"gemm_tc_fwd",   "gemm_tc_head",  "gemm_tc_dx",    "gemm_tc_dw",
                                      "splitk_reduce", "attention_fwd", "attention_bwd", "layernorm_fwd",
                                      "layernorm_bwd", "reductions",    "embedding_fwd", "embedding_bwd",
-                                     "cross_entropy", "adamw"};
+                                     "cross_entropy", "adamw",         "decode_gemv",   "decode_attention",
+                                     "sample_topk"};
   return (c >= 0 && c < CAT_COUNT) ? n[c] : "?";
 }
 
@@ -725,6 +732,110 @@ inline int cross_entropy(const LaunchCtx& c, int dtype, void* logits, long long 
     cross_entropy_f32_kernel<<<N, CE_THREADS, 0, c.stream>>>((float*)logits, ld, V, tgt, scale, row_loss, c.d_err);
   }
   return check_launch(c, "cross_entropy");
+}
+
+// ---------------------------------------------------------------------------
+// generation: skinny GEMMs, single-query attention, key/value cache, sampling
+// ---------------------------------------------------------------------------
+template <int KW>
+int gemv_inst(const LaunchCtx& c, int epi, int grid, const bf16* x, int64_t ldx, int B, const bf16* W, int N, int K,
+              const float* bias, void* out, int64_t ldo, const float* resid, int64_t ldr) {
+  switch (epi) {
+    case EPI_BF16:
+      gemv_bf16_kernel<EPI_BF16, KW><<<grid, DEC_WARPS * 32, 0, c.stream>>>(x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+      break;
+    case EPI_BF16_GELU:
+      gemv_bf16_kernel<EPI_BF16_GELU, KW>
+          <<<grid, DEC_WARPS * 32, 0, c.stream>>>(x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+      break;
+    case EPI_F32_RESID:
+      gemv_bf16_kernel<EPI_F32_RESID, KW>
+          <<<grid, DEC_WARPS * 32, 0, c.stream>>>(x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+      break;
+    case EPI_F32:
+      gemv_bf16_kernel<EPI_F32, KW><<<grid, DEC_WARPS * 32, 0, c.stream>>>(x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+      break;
+    default: return fail(c, GPT2_ERR_CONFIG, "gemv: epilogue must be 0, 1, 2 or 4");
+  }
+  return check_launch(c, "gemv_bf16");
+}
+
+// out[b][n] = epilogue(x[b] . W[n]) for B <= 16 rows (see gemv_bf16_kernel).
+inline int gemv_bf16(const LaunchCtx& c, int epi, const bf16* x, int64_t ldx, int B, const bf16* W, int N, int K,
+                     const float* bias, void* out, int64_t ldo, const float* resid, int64_t ldr) {
+  if (B < 1 || B > DEC_MAX_B) return fail(c, GPT2_ERR_BATCH, "gemv: 1 <= B <= 16 rows");
+  if (N <= 0 || K <= 0 || (K % 8) || (ldx % 8) || (reinterpret_cast<uintptr_t>(x) & 15) ||
+      (reinterpret_cast<uintptr_t>(W) & 15))
+    return fail(c, GPT2_ERR_CONFIG, "gemv: K and ldx multiples of 8, 16-byte aligned x and W");
+  if (epi == EPI_F32_RESID && !resid) return fail(c, GPT2_ERR_CONFIG, "gemv: residual epilogue needs resid");
+  // wide outputs: one warp per 4 columns; narrow ones: split K across the block's warps
+  int kw = 1;
+  if (N < 4096)
+    while (kw < DEC_WARPS && kw * 256 < K) kw *= 2;
+  const int cols = DEC_COLS * (DEC_WARPS / kw);
+  const int grid = (N + cols - 1) / cols;
+  const bool f32o = epi == EPI_F32_RESID || epi == EPI_F32;
+  ProfScope ps(c, CAT_DEC_GEMV, 2.0 * B * N * K,
+               2.0 * N * K + 2.0 * B * K + (double)B * N * (f32o ? 4 : 2) + (epi == EPI_F32_RESID ? 4.0 * B * N : 0.0));
+  switch (kw) {
+    case 1: return gemv_inst<1>(c, epi, grid, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+    case 2: return gemv_inst<2>(c, epi, grid, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+    case 4: return gemv_inst<4>(c, epi, grid, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+    default: return gemv_inst<8>(c, epi, grid, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+  }
+}
+
+// Key splits per (sequence, head) for a generation step: enough blocks for two per SM.
+inline int decode_splits(int B, int NH, int num_sms) {
+  const int bh = B * NH;
+  int S = (2 * num_sms + bh - 1) / bh;
+  return S < 1 ? 1 : (S > DEC_MAX_SPLIT ? DEC_MAX_SPLIT : S);
+}
+
+// Single-query attention of one generation step (head size 64) at the position held in
+// device memory (*pos_ptr < Tc); part: B*NH*S*DEC_PART floats when S > 1.
+inline int decode_attention(const LaunchCtx& c, const bf16* qkv, bf16* cache, int64_t cache_seq, int Tc, int B, int C,
+                            int NH, const int* pos_ptr, int S, bf16* att, float* part, double mean_keys) {
+  if (B < 1 || NH < 1 || C != NH * DEC_HD) return fail(c, GPT2_ERR_CONFIG, "decode attention: head size must be 64");
+  if (S < 1 || S > DEC_MAX_SPLIT || (S > 1 && !part)) return fail(c, GPT2_ERR_CONFIG, "decode attention: splits");
+  const size_t smem = (size_t)Tc * 4;
+  if (smem > 200 * 1024) return fail(c, GPT2_ERR_SEQ_TOO_LONG, "decode attention: more than 51200 positions");
+  if (smem > 48 * 1024) {
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+      attr_set = true;
+    }
+  }
+  ProfScope ps(c, CAT_DEC_ATTN, 4.0 * B * C * mean_keys, 4.0 * B * C * mean_keys + 10.0 * B * C);
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)DEC_HD);
+  decode_attn_kernel<<<B * NH * S, DEC_ATT_THREADS, smem, c.stream>>>(qkv, cache, cache_seq, C, NH, pos_ptr, S,
+                                                                       scale_log2, att, part);
+  int r = check_launch(c, "decode_attention");
+  if (r || S == 1) return r;
+  decode_attn_combine_kernel<<<B * NH, DEC_HD, 0, c.stream>>>(part, S, C, NH, att);
+  return check_launch(c, "decode_attention_combine");
+}
+
+// Keys and values of a prompt's forward pass (qkv rows b*T0 + t) into cache rows t.
+inline int kv_fill(const LaunchCtx& c, const bf16* qkv, int B, int T0, int C, bf16* cache, int64_t cache_seq) {
+  if (C % 4) return fail(c, GPT2_ERR_CONFIG, "kv_fill: C % 4 != 0");
+  const long long vec = (long long)B * T0 * (2 * C / 8);
+  const int grid = (int)std::min<long long>((vec + 255) / 256, 8LL * c.num_sms);
+  ProfScope ps(c, CAT_DEC_ATTN, 0.0, 8.0 * B * T0 * C);
+  kv_fill_kernel<<<grid, 256, 0, c.stream>>>(qkv, B, T0, C, cache, cache_seq);
+  return check_launch(c, "kv_fill");
+}
+
+// One sampled index per logits row (see sample_topk_kernel); u: [rows] doubles in [0, 1).
+inline int sample_topk(const LaunchCtx& c, const float* logits, int64_t ld, int rows, int V, int k, float temperature,
+                       float top_p, const double* u, int* out) {
+  if (rows < 1 || V < 1 || ld < V || k < 1 || k > V || k > TOPK_MAX_K || !(temperature > 0.f) || !(top_p > 0.f) ||
+      top_p > 1.f)
+    return fail(c, GPT2_ERR_CONFIG, "sample_topk: 1 <= k <= min(V, 1024), temperature > 0, 0 < top_p <= 1");
+  ProfScope ps(c, CAT_SAMPLE, 0.0, 5.0 * 4 * rows * V);
+  sample_topk_kernel<<<rows, TOPK_THREADS, 0, c.stream>>>(logits, ld, V, k, temperature, top_p, u, out);
+  return check_launch(c, "sample_topk");
 }
 
 }  // namespace g2

@@ -3,6 +3,7 @@
     python -m train_step_b200.kernel_bench gemm --M 16384 --N 3072 --K 768 --epi 1
     python -m train_step_b200.kernel_bench attn --B 16 --T 1024 --H 12
     python -m train_step_b200.kernel_bench ln --N 16384 --C 768
+    python -m train_step_b200.kernel_bench decode --B 16 --T0 512 --steps 64
 
 Used for focused profiler captures of one kernel on a small case. Inputs are
 seeded random tensors; nothing is checked here (the tests check numerics).
@@ -31,9 +32,75 @@ def timeit(fn, iters: int, warmup: int = 3) -> float:
     return a.elapsed_time(b) / iters
 
 
+def hbm_peak():
+    """(GB/s, 'measured' | 'fallback'): the copy bandwidth measured on this GPU type."""
+    import os
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def decode_bench(a) -> dict:
+    """Generation with the key/value cache on GPT-2 124M (random weights): B prompts of T0
+    tokens, then `steps` decode steps, each one forward step for all B sequences followed
+    by the sampler. Reports milliseconds per decode step (forward + sampling), generated
+    tokens per second, and the step's algorithmic HBM bytes over its time against the
+    measured copy bandwidth: every bf16 weight once, the fp32 LayerNorm parameters and
+    biases, the cache rows read (positions 0..p of every layer and sequence) and written."""
+    import numpy as np
+    cfg = tsb.Config(L=12, H=a.H, C=a.C, T=1024, V=a.V, tied=1, qkv_bias=1, dtype=tsb.BF16, B_max=a.B)
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    m = tsb.GPT2(cfg, seed=1, stream=stream.cuda_stream)
+    B, T0, steps = a.B, a.T0, a.steps
+    if T0 + steps > cfg.T:
+        raise SystemExit("T0 + steps must not exceed 1024")
+    prompt = torch.randint(0, cfg.V, (B, T0), dtype=torch.int32, device="cuda")
+    u = torch.from_numpy(np.random.default_rng(0).random((steps, B))).cuda()
+    idx = torch.empty(B, dtype=torch.int32, device="cuda")
+    logits = torch.empty(B, cfg.V, dtype=torch.float32, device="cuda")
+
+    def run(n):
+        m.prefill(prompt, logits_out=logits)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for s in range(n):
+            m.sample_topk(logits, a.topk, 1.0, 1.0, u[s], out=idx, sync=False)
+            m.decode_step(idx, logits_out=logits, sync=False)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n
+
+    run(min(steps, 8))
+    ms = run(steps)
+    n0 = m.launch_count()
+    run(steps)
+    launches = (m.launch_count() - n0) / steps  # includes the prefill's launches, spread over the steps
+    m.profile(True)
+    run(steps)
+    prof = {k: dict(ms_per_step=v[0] / steps, launches_per_step=v[1] / steps, gbs=v[3] / (v[0] * 1e-3) / 1e9)
+            for k, v in m.profile_read().items() if v[1] > 0 and k.startswith(("decode", "sample", "layernorm_fwd",
+                                                                               "embedding_fwd"))}
+    m.profile(False)
+    L, C, V = cfg.L, cfg.C, cfg.V
+    F = 4 * C
+    w_bytes = 2.0 * (L * (3 * C * C + C * C + 2 * F * C) + V * C)
+    p_bytes = 4.0 * (L * (3 * C + C + F + C + 4 * C) + 2 * C)
+    mean_pos = T0 + (steps - 1) / 2.0
+    kv_bytes = 2.0 * L * B * 2 * C * (mean_pos + 1) + 2.0 * L * B * 2 * C
+    step_bytes = w_bytes + p_bytes + kv_bytes
+    gbs = step_bytes / (ms * 1e-3) / 1e9
+    return dict(shape=[B, T0, steps], ms_per_step=ms, tokens_per_s=B / (ms * 1e-3), bytes_per_step=step_bytes,
+                gbs=gbs, hbm_frac=gbs / hbm_peak()[0], peak_kind=hbm_peak()[1], launches_per_step=launches,
+                kernels=prof)
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["gemm", "attn", "attn_bwd", "ln", "ce"])
+    ap.add_argument("kernel", choices=["gemm", "attn", "attn_bwd", "ln", "ce", "decode"])
     ap.add_argument("--M", type=int, default=16384)
     ap.add_argument("--N", type=int, default=3072)
     ap.add_argument("--K", type=int, default=768)
@@ -48,6 +115,9 @@ def main() -> None:
     ap.add_argument("--C", type=int, default=768)
     ap.add_argument("--V", type=int, default=50257)
     ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--T0", type=int, default=512, help="decode: prompt length")
+    ap.add_argument("--steps", type=int, default=64, help="decode: generated tokens per sequence")
+    ap.add_argument("--topk", type=int, default=50, help="decode: k of the sampler")
     a = ap.parse_args()
     g = torch.Generator(device="cuda").manual_seed(0)
     dev = "cuda"
@@ -96,6 +166,8 @@ def main() -> None:
         rstd = torch.zeros(N, device=dev)
         ms = timeit(lambda: tsb.layernorm_fwd(x, w, bb, y, mean, rstd), a.iters)
         res.update(shape=[N, C], ms=ms, gbs=N * C * 6 / (ms * 1e-3) / 1e9)
+    elif a.kernel == "decode":
+        res.update(decode_bench(a))
     else:
         N, V = a.M, a.V
         ld = (V + 63) // 64 * 64
