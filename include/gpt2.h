@@ -298,6 +298,18 @@ int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, con
 int gpt2_op_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, const void* dout,
                                   const float* f32_lse, int B, int T, int NH, int hd, void* dqkv, void* stream);
 
+/* Skinny product of a generation step, all DEVICE pointers: out[b][n] = epilogue(sum_k
+ * x[b][k] W[n][k]) for b < B <= 16, n < N; W bf16 [N][K] row-major; epilogue 0 (bf16 out,
+ * + bias), 1 (bf16 gelu_tanh(acc + bias)), 2 (fp32 out = resid + acc + bias) or 4 (fp32
+ * out = acc). x is bf16 rows of stride ldx, or, when ln_g and ln_b are given, fp32 rows that
+ * are layer-normalised first (eps 1e-5, result rounded to bf16). K and ldx multiples of 8,
+ * 16-byte aligned x, W, ln_g, ln_b; B*K*2 <= 200 KB. With iters > 1 the product is then
+ * launched iters more times back to back (as programmatic dependents when pdl != 0) and
+ * *ms_out receives the mean milliseconds per launch. Synchronises. */
+int gpt2_op_gemv(const void* x, int64_t ldx, int B, const void* W, int N, int K, int epilogue, const float* bias,
+                 void* out, int64_t ldo, const float* resid, int64_t ldr, const float* ln_g, const float* ln_b,
+                 int iters, int pdl, float* ms_out, void* stream);
+
 /* gpt2_sample_topk without a handle, for V given explicitly (same rules and
  * arguments, all DEVICE pointers). Synchronises. */
 int gpt2_op_sample_topk(const float* logits, int64_t ld, int rows, int V, int k, float temperature, float top_p,

@@ -298,9 +298,9 @@ def lr_schedule(step: int, max_lr: float = 6e-4, min_lr: float = 6e-5, warmup: i
                 total: int = 19073) -> float:
     """Learning rate at optimizer step `step` (0-based), in float64.
 
-    "GPT From Scratch", Training Recipe table: peak 6e-4, minimum 6e-5 (peak / 10), 715
-    warmup steps, 19,073 total steps; repository tour, "Cosine LR Schedule": linear warmup,
-    then cosine decay. Reading (the pages leave the indexing open): warmup step s takes
+    "AxonLM", Training Recipe table: peak 6e-4, minimum 6e-5 (peak / 10), 715 warmup steps,
+    19,073 total steps; "AxonLM", Key Features, and "Genesis", Training Features: linear
+    warmup, then cosine decay. Reading (the pages leave the indexing open): warmup step s takes
     peak * (s + 1) / warmup; from s = warmup the rate is
     min + (peak - min) * (1 + cos(pi * (s - warmup) / (total - warmup))) / 2, reaching the
     minimum at s = total and staying there.

@@ -193,3 +193,42 @@ def test_split_key_attention_many_splits():
     ref = _oracle_last_logits(cfg, p, seq)
     assert rel_l2(z[0], ref[0]) <= 2e-2
     m.close()
+
+
+def _dev(a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dtype).cuda()
+
+
+def _g64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("B,N,K", [(1, 2304, 768), (5, 770, 256), (16, 3072, 768), (16, 768, 3072), (3, 1001, 128),
+                                   (16, 50257, 768)])
+def test_gemv_epilogues_match_oracle(B, N, K):
+    rng = np.random.default_rng(N + K + B)
+    x = _dev(rng.standard_normal((B, K)), torch.bfloat16)
+    W = _dev(rng.standard_normal((N, K)) * 0.05, torch.bfloat16)
+    bias = _dev(rng.standard_normal(N), torch.float32)
+    resid = _dev(rng.standard_normal((B, N)), torch.float32)
+    D = oracle.linear_fwd(_g64(x), _g64(W))
+    kw = dict(B=B, N=N, K=K)
+    o0 = torch.empty(B, N, dtype=torch.bfloat16, device="cuda")
+    tsb.gemv(x, W, o0, epilogue=tsb.EPI_BIAS, bias=bias, **kw)
+    assert rel_l2(_g64(o0), D + _g64(bias)) < 4e-3
+    o1 = torch.empty_like(o0)
+    tsb.gemv(x, W, o1, epilogue=tsb.EPI_BIAS_GELU, bias=bias, **kw)
+    assert rel_l2(_g64(o1), oracle.gelu_fwd(D + _g64(bias))) < 5e-3
+    o2 = torch.empty(B, N, dtype=torch.float32, device="cuda")
+    tsb.gemv(x, W, o2, epilogue=tsb.EPI_RESID, bias=bias, resid=resid, ldr=N, **kw)
+    assert rel_l2(_g64(o2), D + _g64(bias) + _g64(resid)) < 1e-5
+    o4 = torch.empty(B, N, dtype=torch.float32, device="cuda")
+    tsb.gemv(x, W, o4, epilogue=tsb.EPI_F32, **kw)
+    assert rel_l2(_g64(o4), D) < 1e-5
+    # LayerNorm applied on the fly to fp32 rows (the kernel rounds the normalised rows to bf16)
+    xf = _dev(rng.standard_normal((B, K)) * 3 + 1, torch.float32)
+    g = _dev(1 + 0.1 * rng.standard_normal(K), torch.float32)
+    b = _dev(0.1 * rng.standard_normal(K), torch.float32)
+    y, _, _ = oracle.layernorm_fwd(_g64(xf), _g64(g), _g64(b))
+    tsb.gemv(xf, W, o4, epilogue=tsb.EPI_F32, ln_g=g, ln_b=b, **kw)
+    assert rel_l2(_g64(o4), oracle.linear_fwd(y, _g64(W))) < 4e-3

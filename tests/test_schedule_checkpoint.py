@@ -1,7 +1,7 @@
 """Learning-rate schedule and checkpoint file format (CPU).
 
-The oracle's schedule is pinned to values the recipe fixes ("GPT From Scratch", Training
-Recipe table: peak 6e-4, minimum 6e-5, 715 warmup steps, 19,073 total) and to closed-form
+The oracle's schedule is pinned to values the recipe fixes ("AxonLM", Training Recipe
+table: peak 6e-4, minimum 6e-5, 715 warmup steps, 19,073 total) and to closed-form
 properties of a linear warmup and a half-cosine; the library's schedule must agree with it.
 """
 import numpy as np

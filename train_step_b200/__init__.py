@@ -89,6 +89,9 @@ _SYMBOLS = {
                           ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_kv_length": ([ct.c_void_p, ct.POINTER(ct.c_int)], ct.c_int),
     "gpt2_synchronize": ([ct.c_void_p], ct.c_int),
+    "gpt2_op_gemv": ([ct.c_void_p, ct.c_int64, ct.c_int, ct.c_void_p, ct.c_int, ct.c_int, ct.c_int, ct.c_void_p,
+                      ct.c_void_p, ct.c_int64, ct.c_void_p, ct.c_int64, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int,
+                      ct.POINTER(ct.c_float), ct.c_void_p], ct.c_int),
     "gpt2_op_sample_topk": ([ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_int, ct.c_float, ct.c_float,
                              ct.c_void_p, ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_op_last_error": ([], ct.c_char_p),
@@ -404,6 +407,17 @@ def layernorm_bwd(dy, x, g, mean, rstd, dres, dres_act, dg, db, accumulate=False
     _op(lib().gpt2_op_layernorm_bwd(dt, _ptr(dy), _ptr(x), _ptr(g), _ptr(mean), _ptr(rstd), N, C, _ptr(dres),
                                     _ptr(dres_act), int(accumulate), _ptr(dg), _ptr(db), int(accumulate_params),
                                     _stream(stream)))
+
+
+def gemv(x, W, out, *, B, N, K, epilogue, ldx=None, ldo=None, bias=None, resid=None, ldr=0, ln_g=None, ln_b=None,
+         iters=1, pdl=False, stream=None):
+    """Skinny product of a generation step (see gpt2_op_gemv); returns ms per launch when
+    iters > 1."""
+    ms = ct.c_float()
+    _op(lib().gpt2_op_gemv(_ptr(x), x.stride(0) if ldx is None else ldx, B, _ptr(W), N, K, epilogue, _ptr(bias),
+                           _ptr(out), out.stride(0) if ldo is None else ldo, _ptr(resid), ldr, _ptr(ln_g),
+                           _ptr(ln_b), iters, int(pdl), ct.byref(ms), _stream(stream)))
+    return ms.value if iters > 1 else None
 
 
 def sample_topk(logits, V, k, temperature, top_p, u, out, stream=None):

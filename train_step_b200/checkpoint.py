@@ -3,7 +3,8 @@
 A checkpoint is taken between optimizer steps (no gradients are pending): it holds the
 fp32 parameters and the Adam moments m, v in canonical order (12 bytes per parameter,
 1.49 GB at 124M), the Adam step count t, the caller's step counter and the model
-configuration, which `load` checks against the target model.
+configuration, which `load` checks against the target model ("AxonLM", Key Features:
+checkpoint resume; "gpt/docs/LLM.md", Memory Footprint: about 1.49 GB with optimizer states).
 """
 from __future__ import annotations
 

@@ -703,11 +703,13 @@ namespace {
 int64_t kv_seq_elems(const gpt2* m) { return (int64_t)m->T * 2 * m->C; }
 bf16* kv_layer(gpt2* m, int l) { return m->kv + (int64_t)l * m->cfg.B_max * kv_seq_elems(m); }
 
-// fp32 logits of B rows of ln_f output (bf16, row stride ldx) against the head weight.
-int head_logits(gpt2* m, const bf16* xf_rows, int64_t ldx, int B, float* logits_out, int64_t ld) {
+// fp32 logits of B rows against the head weight: rows of ln_f output (bf16, row stride
+// ldx), or with ln, fp32 residual rows that ln_f is applied to on the fly.
+int head_logits(gpt2* m, const LaunchCtx& c, const void* rows, int64_t ldx, int B, float* logits_out, int64_t ld,
+                bool ln = false) {
   const float* headw = m->cfg.tied ? m->wte : m->head;
-  return gemv_bf16(m->ctx(), EPI_F32, xf_rows, ldx, B, (const bf16*)m->W(headw), m->cfg.V, m->C, nullptr, logits_out,
-                   ld, nullptr, 0);
+  return gemv_bf16(c, EPI_F32, rows, ldx, B, (const bf16*)m->W(headw), m->cfg.V, m->C, nullptr, logits_out, ld,
+                   nullptr, 0, ln ? m->lnf_g : nullptr, ln ? m->lnf_b : nullptr);
 }
 
 int check_generation(gpt2* m, float* logits_out, int64_t ld, int B) {
@@ -747,7 +749,7 @@ int gpt2_prefill(gpt2* m, const int32_t* tokens, int B, int T0, float* logits_ou
     RK(kv_fill(c, (const bf16*)(m->qkv + (int64_t)l * N3C * m->act_bytes), B, T0, m->C, kv_layer(m, l),
                kv_seq_elems(m)));
   // the last position of each prompt: rows b*T0 + T0-1 of ln_f's output
-  RK(head_logits(m, (const bf16*)m->xf + (int64_t)(T0 - 1) * m->C, (int64_t)T0 * m->C, B, logits_out, ld));
+  RK(head_logits(m, c, (const bf16*)m->xf + (int64_t)(T0 - 1) * m->C, (int64_t)T0 * m->C, B, logits_out, ld));
   set_pos_kernel<<<1, 1, 0, m->stream>>>(m->d_pos, T0);
   RK(check_launch(c, "set_pos"));
   m->kv_B = B;
@@ -763,7 +765,6 @@ int decode_body(gpt2* m, int B, float* logits_out, int64_t ld) {
   const int C = m->C, F = m->F;
   float* x0 = m->x;
   float* x1 = m->x + (int64_t)B * C;
-  bf16* h = (bf16*)m->h1;
   bf16* qkv = (bf16*)m->qkv;
   bf16* att = (bf16*)m->att;
   bf16* a = (bf16*)m->a;
@@ -774,19 +775,23 @@ int decode_body(gpt2* m, int B, float* logits_out, int64_t ld) {
                                                                     m->cfg.V, m->d_err);
     RK(check_launch(c, "embed_decode"));
   }
+  // every later kernel of the step starts as a programmatic dependent of the one before:
+  // it fetches its weights while that one finishes and waits for it before reading
+  // activations or writing anything
+  c.pdl = true;
+  // each LayerNorm is applied inside the product that consumes it
   for (int l = 0; l < m->L; ++l) {
     const LayerP& w = m->lp[l];
-    RK(layernorm_fwd_t<bf16>(c, x0, w.ln1_g, w.ln1_b, B, C, h, m->stat_mean, m->stat_rstd));
-    RK(gemv_bf16(c, EPI_BF16, h, C, B, (const bf16*)m->W(w.qkv_w), 3 * C, C, w.qkv_b, qkv, 3 * C, nullptr, 0));
+    RK(gemv_bf16(c, EPI_BF16, x0, C, B, (const bf16*)m->W(w.qkv_w), 3 * C, C, w.qkv_b, qkv, 3 * C, nullptr, 0,
+                 w.ln1_g, w.ln1_b));
     RK(decode_attention(c, qkv, kv_layer(m, l), kv_seq_elems(m), m->T, B, C, m->NH, m->d_pos, S, att, m->dec_part,
                         (double)m->kv_len + 1.0));
     RK(gemv_bf16(c, EPI_F32_RESID, att, C, B, (const bf16*)m->W(w.ao_w), C, C, w.ao_b, x1, C, x0, C));
-    RK(layernorm_fwd_t<bf16>(c, x1, w.ln2_g, w.ln2_b, B, C, h, m->stat_mean, m->stat_rstd));
-    RK(gemv_bf16(c, EPI_BF16_GELU, h, C, B, (const bf16*)m->W(w.fc_w), F, C, w.fc_b, a, F, nullptr, 0));
+    RK(gemv_bf16(c, EPI_BF16_GELU, x1, C, B, (const bf16*)m->W(w.fc_w), F, C, w.fc_b, a, F, nullptr, 0, w.ln2_g,
+                 w.ln2_b));
     RK(gemv_bf16(c, EPI_F32_RESID, a, F, B, (const bf16*)m->W(w.pj_w), C, F, w.pj_b, x0, C, x1, C));
   }
-  RK(layernorm_fwd_t<bf16>(c, x0, m->lnf_g, m->lnf_b, B, C, h, m->stat_mean, m->stat_rstd));
-  RK(head_logits(m, h, C, B, logits_out, ld));
+  RK(head_logits(m, c, x0, C, B, logits_out, ld, true));
   set_pos_kernel<<<1, 1, 0, m->stream>>>(m->d_pos, -1);
   return check_launch(c, "set_pos");
 }
@@ -798,6 +803,7 @@ int capture_decode(gpt2* m, int B, float* logits_out, int64_t ld) {
     m->dec_graph = nullptr;
   }
   const long long before = m->launches;
+  gemv_prepare();  // function attributes are set outside the capture
   CK(m, cudaStreamBeginCapture(m->stream, cudaStreamCaptureModeThreadLocal));
   const int r = decode_body(m, B, logits_out, ld);
   cudaGraph_t g = nullptr;
@@ -1021,6 +1027,38 @@ int gpt2_op_gemm_bench(const void* A, int64_t lda, int a_mn, const void* B, int6
   cudaEventDestroy(e0);
   cudaEventDestroy(e1);
   *ms_out = ms / iters;
+  return r ? r : r2;
+}
+
+int gpt2_op_gemv(const void* x, int64_t ldx, int B, const void* W, int N, int K, int epilogue, const float* bias,
+                 void* out, int64_t ldo, const float* resid, int64_t ldr, const float* ln_g, const float* ln_b,
+                 int iters, int pdl, float* ms_out, void* stream) {
+  if (!x || !W || !out || iters < 1 || (iters > 1 && !ms_out)) {
+    g_op_error = "gemv: x, W, out required; iters >= 1 (ms_out with iters > 1)";
+    return GPT2_ERR_CONFIG;
+  }
+  OpCtx o(stream);
+  RK(o.alloc_err());
+  auto one = [&]() {
+    return gemv_bf16(o.c, epilogue, x, ldx, B, (const bf16*)W, N, K, bias, out, ldo, resid, ldr, ln_g, ln_b);
+  };
+  int r = one();  // warm-up (sets kernel attributes)
+  if (!r && iters > 1) {
+    o.c.pdl = pdl != 0;
+    cudaEvent_t e0, e1;
+    cudaEventCreate(&e0);
+    cudaEventCreate(&e1);
+    cudaEventRecord(e0, o.s);
+    for (int i = 0; i < iters && !r; ++i) r = one();
+    cudaEventRecord(e1, o.s);
+    cudaEventSynchronize(e1);
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, e0, e1);
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    *ms_out = ms / iters;
+  }
+  int r2 = o.finish();
   return r ? r : r2;
 }
 

@@ -33,82 +33,163 @@ __device__ __forceinline__ uint4 dec_ld_stream(const void* p) {
 }
 
 // out[b][n] = epilogue(sum_k x[b][k] * W[n][k] (+ bias[n])) for b < B, n < N.
-// x: bf16 rows of stride ldx; W: bf16 [N][K] row-major (the K-major layout the training
-// GEMMs read). The 8 warps of a block form KW groups along K and 8/KW groups of 4 output
-// columns; each lane accumulates 4 columns x 16 rows in fp32 over 8-element K chunks,
-// then a butterfly reduce-scatter leaves lane L with entries 2L and 2L+1 of that 4x16
-// block (column L/8, rows 2L mod 16 and the next one).
+// W: bf16 [N][K] row-major (the K-major layout the training GEMMs read). x: bf16 rows of
+// stride ldx; or, with LN, fp32 rows of the residual stream that the kernel layer-
+// normalises itself (y = (x - mean) * rstd * ln_g + ln_b with the biased variance and
+// eps 1e-5, rounded to bf16 as the LayerNorm kernel stores it), so that no LayerNorm
+// launch sits between two products.
+// Each block first stages all B rows of x in shared memory as bf16 (one burst of loads,
+// one wait) and then walks groups of output columns (group g = blockIdx.x, + gridDim.x,
+// ...). Its 8 warps form KW groups along K and 8/KW groups of 4 columns; a lane
+// accumulates 4 columns x 16 rows in fp32 over 8-element K chunks, and a butterfly
+// reduce-scatter leaves lane L with entries 2L and 2L+1 of that 4x16 block (column L/8,
+// rows 2L mod 16 and the next). Dynamic shared memory: B*K bf16.
 // Epilogues: EPI_BF16 (bf16 out), EPI_BF16_GELU (bf16 gelu_tanh(acc + bias)), EPI_F32_RESID
 // (fp32 out = resid + acc + bias), EPI_F32 (fp32 out = acc).
-template <int EPI, int KW>
-__global__ void __launch_bounds__(DEC_WARPS * 32)
-    gemv_bf16_kernel(const bf16* __restrict__ x, int64_t ldx, int B, const bf16* __restrict__ W, int N, int K,
+template <int EPI, int KW, bool LN>
+__global__ void __launch_bounds__(DEC_WARPS * 32, 2)
+    gemv_bf16_kernel(const void* __restrict__ xin, int64_t ldx, int B, const bf16* __restrict__ W, int N, int K,
                      const float* __restrict__ bias, void* __restrict__ out, int64_t ldo,
-                     const float* __restrict__ resid, int64_t ldr) {
+                     const float* __restrict__ resid, int64_t ldr, const float* __restrict__ ln_g,
+                     const float* __restrict__ ln_b) {
   constexpr int NW = DEC_WARPS / KW;
   constexpr int NA = DEC_COLS * DEC_MAX_B;  // 64 accumulators per lane
+  extern __shared__ __align__(16) unsigned char dec_smem[];
+  bf16* xs = reinterpret_cast<bf16*>(dec_smem);  // [B][K]
   __shared__ float red[DEC_WARPS][NA];
+  __shared__ float stat[DEC_MAX_B][2];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int kw = warp % KW, nw = warp / KW;
-  const int n0 = (blockIdx.x * NW + nw) * DEC_COLS;
-  float acc[NA];
-#pragma unroll
-  for (int i = 0; i < NA; ++i) acc[i] = 0.f;
-  for (int k = (kw * 32 + lane) * 8; k < K; k += KW * 256) {
-    float wv[DEC_COLS][8];
+  const int groups = (N + NW * DEC_COLS - 1) / (NW * DEC_COLS);
+  const int k_first = (kw * 32 + lane) * 8;
+  // weights do not depend on the previous kernel: the first chunk is fetched before
+  // waiting for it, and each later chunk while the one before is in use
+  uint4 wraw[DEC_COLS];
+  {
+    const int n0 = (blockIdx.x * NW + nw) * DEC_COLS;
 #pragma unroll
     for (int r = 0; r < DEC_COLS; ++r) {
-      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (n0 + r < N) raw = dec_ld_stream(W + (int64_t)(n0 + r) * K + k);
-      dec_unpack8(raw, wv[r]);
+      wraw[r] = make_uint4(0u, 0u, 0u, 0u);
+      if (k_first < K && n0 + r < N) wraw[r] = dec_ld_stream(W + (int64_t)(n0 + r) * K + k_first);
     }
-#pragma unroll
-    for (int b = 0; b < DEC_MAX_B; ++b) {
-      if (b < B) {
-        float xv[8];
-        dec_unpack8(__ldg(reinterpret_cast<const uint4*>(x + (int64_t)b * ldx + k)), xv);
-#pragma unroll
-        for (int r = 0; r < DEC_COLS; ++r)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[r * DEC_MAX_B + b] = fmaf(wv[r][e], xv[e], acc[r * DEC_MAX_B + b]);
+  }
+  pdl_launch_dependents();
+  pdl_wait();
+  // stage x
+  if (LN) {
+    const float* xf = static_cast<const float*>(xin);
+    for (int b = warp; b < B; b += DEC_WARPS) {  // row statistics, K % 4 == 0
+      const float* xr = xf + (int64_t)b * ldx;
+      float s = 0.f;
+      for (int c = lane * 4; c < K; c += 128) {
+        const float4 v = *reinterpret_cast<const float4*>(xr + c);
+        s += (v.x + v.y) + (v.z + v.w);
+      }
+      const float mu = warp_sum(s) / (float)K;
+      float ss = 0.f;
+      for (int c = lane * 4; c < K; c += 128) {
+        const float4 v = *reinterpret_cast<const float4*>(xr + c);
+        const float e0 = v.x - mu, e1 = v.y - mu, e2 = v.z - mu, e3 = v.w - mu;
+        ss += (e0 * e0 + e1 * e1) + (e2 * e2 + e3 * e3);
+      }
+      const float var = warp_sum(ss) / (float)K;
+      if (lane == 0) {
+        stat[b][0] = mu;
+        stat[b][1] = 1.0f / sqrtf(var + 1e-5f);
       }
     }
-  }
-  // reduce-scatter across the warp: each step keeps half of the entries, adding the
-  // partner lane's copy of them
-#pragma unroll
-  for (int o = 16, half = NA / 2; o >= 1; o >>= 1, half >>= 1) {
-    const bool hi = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = hi ? acc[i] : acc[i + half];
-      const float keep = hi ? acc[i + half] : acc[i];
-      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  if (KW > 1) {
-    red[warp][2 * lane] = acc[0];
-    red[warp][2 * lane + 1] = acc[1];
     __syncthreads();
-    if (kw != 0) return;
-#pragma unroll
-    for (int q = 1; q < KW; ++q) {
-      acc[0] += red[warp + q][2 * lane];
-      acc[1] += red[warp + q][2 * lane + 1];
+    const int per_row = K / 4;
+    for (int i = threadIdx.x; i < B * per_row; i += DEC_WARPS * 32) {
+      const int b = i / per_row, c = (i % per_row) * 4;
+      const float4 v = *reinterpret_cast<const float4*>(xf + (int64_t)b * ldx + c);
+      const float4 g = __ldg(reinterpret_cast<const float4*>(ln_g + c));
+      const float4 bb = __ldg(reinterpret_cast<const float4*>(ln_b + c));
+      const float mu = stat[b][0], rs = stat[b][1];
+      *reinterpret_cast<uint2*>(xs + (int64_t)b * K + c) =
+          make_uint2(pack_bf16x2((v.x - mu) * rs * g.x + bb.x, (v.y - mu) * rs * g.y + bb.y),
+                     pack_bf16x2((v.z - mu) * rs * g.z + bb.z, (v.w - mu) * rs * g.w + bb.w));
+    }
+  } else {
+    const bf16* x = static_cast<const bf16*>(xin);
+    const int per_row = K / 8;
+    for (int i = threadIdx.x; i < B * per_row; i += DEC_WARPS * 32) {
+      const int b = i / per_row, c = (i % per_row) * 8;
+      *reinterpret_cast<uint4*>(xs + (int64_t)b * K + c) = *reinterpret_cast<const uint4*>(x + (int64_t)b * ldx + c);
     }
   }
-  const int n = n0 + (lane >> 3);
-  if (n >= N) return;
-  const float bn = (EPI != EPI_F32 && bias) ? bias[n] : 0.f;
+  __syncthreads();
+  for (int grp = blockIdx.x; grp < groups; grp += gridDim.x) {
+    const int n0 = (grp * NW + nw) * DEC_COLS;
+    if (grp != (int)blockIdx.x) {
 #pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int b = ((2 * lane) & (DEC_MAX_B - 1)) + e;
-    if (b >= B) continue;
-    const float v = acc[e] + bn;
-    if (EPI == EPI_BF16) static_cast<bf16*>(out)[(int64_t)b * ldo + n] = __float2bfloat16_rn(v);
-    if (EPI == EPI_BF16_GELU) static_cast<bf16*>(out)[(int64_t)b * ldo + n] = __float2bfloat16_rn(gelu_tanh(v));
-    if (EPI == EPI_F32_RESID) static_cast<float*>(out)[(int64_t)b * ldo + n] = resid[(int64_t)b * ldr + n] + v;
-    if (EPI == EPI_F32) static_cast<float*>(out)[(int64_t)b * ldo + n] = v;
+      for (int r = 0; r < DEC_COLS; ++r) {
+        wraw[r] = make_uint4(0u, 0u, 0u, 0u);
+        if (k_first < K && n0 + r < N) wraw[r] = dec_ld_stream(W + (int64_t)(n0 + r) * K + k_first);
+      }
+    }
+    float acc[NA];
+#pragma unroll
+    for (int i = 0; i < NA; ++i) acc[i] = 0.f;
+    for (int k = k_first; k < K; k += KW * 256) {
+      float wv[DEC_COLS][8];
+#pragma unroll
+      for (int r = 0; r < DEC_COLS; ++r) dec_unpack8(wraw[r], wv[r]);
+      const int kn = k + KW * 256;
+#pragma unroll
+      for (int r = 0; r < DEC_COLS; ++r)
+        if (kn < K && n0 + r < N) wraw[r] = dec_ld_stream(W + (int64_t)(n0 + r) * K + kn);
+#pragma unroll
+      for (int b = 0; b < DEC_MAX_B; ++b) {
+        if (b < B) {
+          float xv[8];
+          dec_unpack8(*reinterpret_cast<const uint4*>(xs + b * K + k), xv);
+#pragma unroll
+          for (int r = 0; r < DEC_COLS; ++r)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[r * DEC_MAX_B + b] = fmaf(wv[r][e], xv[e], acc[r * DEC_MAX_B + b]);
+        }
+      }
+    }
+    // reduce-scatter across the warp: each step keeps half of the entries, adding the
+    // partner lane's copy of them
+#pragma unroll
+    for (int o = 16, half = NA / 2; o >= 1; o >>= 1, half >>= 1) {
+      const bool hi = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = hi ? acc[i] : acc[i + half];
+        const float keep = hi ? acc[i + half] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    if (KW > 1) {
+      red[warp][2 * lane] = acc[0];
+      red[warp][2 * lane + 1] = acc[1];
+      __syncthreads();
+      if (kw == 0) {
+#pragma unroll
+        for (int q = 1; q < KW; ++q) {
+          acc[0] += red[warp + q][2 * lane];
+          acc[1] += red[warp + q][2 * lane + 1];
+        }
+      }
+      __syncthreads();  // red is rewritten by the next group
+    }
+    const int n = n0 + (lane >> 3);
+    if (kw == 0 && n < N) {
+      const float bn = (EPI != EPI_F32 && bias) ? bias[n] : 0.f;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int b = ((2 * lane) & (DEC_MAX_B - 1)) + e;
+        if (b >= B) continue;
+        const float v = acc[e] + bn;
+        if (EPI == EPI_BF16) static_cast<bf16*>(out)[(int64_t)b * ldo + n] = __float2bfloat16_rn(v);
+        if (EPI == EPI_BF16_GELU) static_cast<bf16*>(out)[(int64_t)b * ldo + n] = __float2bfloat16_rn(gelu_tanh(v));
+        if (EPI == EPI_F32_RESID) static_cast<float*>(out)[(int64_t)b * ldo + n] = resid[(int64_t)b * ldr + n] + v;
+        if (EPI == EPI_F32) static_cast<float*>(out)[(int64_t)b * ldo + n] = v;
+      }
+    }
   }
 }
 
@@ -144,6 +225,8 @@ __global__ void __launch_bounds__(DEC_ATT_THREADS)
   __shared__ float red[DEC_ATT_THREADS / 32][DEC_HD];
   __shared__ float wred[DEC_ATT_THREADS / 32];
   constexpr int NWARP = DEC_ATT_THREADS / 32;
+  pdl_launch_dependents();
+  pdl_wait();
   const int bh = blockIdx.x / S, split = blockIdx.x % S;
   const int b = bh / NH, h = bh % NH;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -256,6 +339,8 @@ __global__ void __launch_bounds__(DEC_ATT_THREADS)
 // att[b][h*64 + d] from the S partial results of (b, h): rescale each to the largest m.
 __global__ void decode_attn_combine_kernel(const float* __restrict__ part, int S, int C, int NH,
                                            bf16* __restrict__ att) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int bh = blockIdx.x, d = threadIdx.x;
   const float* pp = part + (int64_t)bh * S * DEC_PART;
   float M = -INFINITY;

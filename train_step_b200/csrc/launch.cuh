@@ -98,7 +98,27 @@ struct LaunchCtx {
   float* splitk_ws = nullptr;     // split-K workspace (nullable: split-K disabled)
   size_t splitk_cap = 0;          // floats
   int num_sms = 148;
+  bool pdl = false;  // launch as programmatic dependents of the previous kernel (kernels that support it)
 };
+
+// Launch `kern` on c.stream; with c.pdl as a programmatic dependent of the stream's
+// previous kernel (the kernel must call pdl_wait before reading that kernel's results and
+// before any write).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(const LaunchCtx& c, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = c.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 
 struct ProfScope {
   const LaunchCtx& c;
@@ -460,7 +480,12 @@ int layernorm_fwd_t(const LaunchCtx& c, const float* x, const float* g, const fl
   const int blocks = (N + LN_WARPS - 1) / LN_WARPS;
   const int nv = ln_nv(C);
   ProfScope ps(c, CAT_LN_FWD, 0.0, (double)N * C * (4 + sizeof(T)) + 8.0 * N);
-#define LNF(NV) layernorm_fwd_kernel<T, NV><<<blocks, LN_WARPS * 32, 0, c.stream>>>(x, g, b, y, mean, rstd, N, C)
+  cudaError_t e = cudaSuccess;
+#define LNF(NV)                                                                                           \
+  e = c.pdl ? launch_k(c, layernorm_fwd_kernel<T, NV, true>, dim3(blocks), dim3(LN_WARPS * 32), 0, x, g, b, y, \
+                       mean, rstd, N, C)                                                                  \
+            : (layernorm_fwd_kernel<T, NV><<<blocks, LN_WARPS * 32, 0, c.stream>>>(x, g, b, y, mean, rstd, N, C), \
+               cudaSuccess)
   if (nv <= 1) LNF(1);
   else if (nv <= 2) LNF(2);
   else if (nv <= 4) LNF(4);
@@ -469,6 +494,7 @@ int layernorm_fwd_t(const LaunchCtx& c, const float* x, const float* g, const fl
   else if (nv <= 13) LNF(13);
   else LNF(16);
 #undef LNF
+  if (e != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("layernorm_fwd: ") + cudaGetErrorString(e));
   return check_launch(c, "layernorm_fwd");
 }
 
@@ -737,57 +763,109 @@ inline int cross_entropy(const LaunchCtx& c, int dtype, void* logits, long long 
 // ---------------------------------------------------------------------------
 // generation: skinny GEMMs, single-query attention, key/value cache, sampling
 // ---------------------------------------------------------------------------
-template <int KW>
-int gemv_inst(const LaunchCtx& c, int epi, int grid, const bf16* x, int64_t ldx, int B, const bf16* W, int N, int K,
-              const float* bias, void* out, int64_t ldo, const float* resid, int64_t ldr) {
+constexpr int DEC_GEMV_MAX_SMEM = 200 * 1024;  // staged x: B * K bf16
+
+template <int KW, bool LN>
+void gemv_attrs() {
+  cudaFuncSetAttribute(gemv_bf16_kernel<EPI_BF16, KW, LN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       DEC_GEMV_MAX_SMEM);
+  cudaFuncSetAttribute(gemv_bf16_kernel<EPI_BF16_GELU, KW, LN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       DEC_GEMV_MAX_SMEM);
+  cudaFuncSetAttribute(gemv_bf16_kernel<EPI_F32_RESID, KW, LN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       DEC_GEMV_MAX_SMEM);
+  cudaFuncSetAttribute(gemv_bf16_kernel<EPI_F32, KW, LN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       DEC_GEMV_MAX_SMEM);
+}
+
+// Shared-memory limits of every GEMV variant, set once per process before any launch
+// (and so before a decode step is captured).
+inline void gemv_prepare() {
+  static bool done = false;
+  if (done) return;
+  gemv_attrs<1, false>();
+  gemv_attrs<2, false>();
+  gemv_attrs<4, false>();
+  gemv_attrs<8, false>();
+  gemv_attrs<1, true>();
+  gemv_attrs<2, true>();
+  gemv_attrs<4, true>();
+  gemv_attrs<8, true>();
+  done = true;
+}
+
+template <int KW, bool LN>
+int gemv_inst(const LaunchCtx& c, int epi, int grid, size_t smem, const void* x, int64_t ldx, int B, const bf16* W,
+              int N, int K, const float* bias, void* out, int64_t ldo, const float* resid, int64_t ldr,
+              const float* ln_g, const float* ln_b) {
+  cudaError_t e = cudaSuccess;
+  const dim3 g(grid), blk(DEC_WARPS * 32);
   switch (epi) {
     case EPI_BF16:
-      gemv_bf16_kernel<EPI_BF16, KW><<<grid, DEC_WARPS * 32, 0, c.stream>>>(x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+      e = launch_k(c, gemv_bf16_kernel<EPI_BF16, KW, LN>, g, blk, smem, x, ldx, B, W, N, K, bias, out, ldo, resid,
+                   ldr, ln_g, ln_b);
       break;
     case EPI_BF16_GELU:
-      gemv_bf16_kernel<EPI_BF16_GELU, KW>
-          <<<grid, DEC_WARPS * 32, 0, c.stream>>>(x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+      e = launch_k(c, gemv_bf16_kernel<EPI_BF16_GELU, KW, LN>, g, blk, smem, x, ldx, B, W, N, K, bias, out, ldo,
+                   resid, ldr, ln_g, ln_b);
       break;
     case EPI_F32_RESID:
-      gemv_bf16_kernel<EPI_F32_RESID, KW>
-          <<<grid, DEC_WARPS * 32, 0, c.stream>>>(x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+      e = launch_k(c, gemv_bf16_kernel<EPI_F32_RESID, KW, LN>, g, blk, smem, x, ldx, B, W, N, K, bias, out, ldo,
+                   resid, ldr, ln_g, ln_b);
       break;
     case EPI_F32:
-      gemv_bf16_kernel<EPI_F32, KW><<<grid, DEC_WARPS * 32, 0, c.stream>>>(x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+      e = launch_k(c, gemv_bf16_kernel<EPI_F32, KW, LN>, g, blk, smem, x, ldx, B, W, N, K, bias, out, ldo, resid,
+                   ldr, ln_g, ln_b);
       break;
     default: return fail(c, GPT2_ERR_CONFIG, "gemv: epilogue must be 0, 1, 2 or 4");
   }
+  if (e != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("gemv_bf16: ") + cudaGetErrorString(e));
   return check_launch(c, "gemv_bf16");
 }
 
-// out[b][n] = epilogue(x[b] . W[n]) for B <= 16 rows (see gemv_bf16_kernel).
-inline int gemv_bf16(const LaunchCtx& c, int epi, const bf16* x, int64_t ldx, int B, const bf16* W, int N, int K,
-                     const float* bias, void* out, int64_t ldo, const float* resid, int64_t ldr) {
+// out[b][n] = epilogue(x[b] . W[n]) for B <= 16 rows (see gemv_bf16_kernel). With ln_g and
+// ln_b set, x is the fp32 residual stream and is layer-normalised on the fly (ldx in
+// floats); otherwise x is bf16.
+inline int gemv_bf16(const LaunchCtx& c, int epi, const void* x, int64_t ldx, int B, const bf16* W, int N, int K,
+                     const float* bias, void* out, int64_t ldo, const float* resid, int64_t ldr,
+                     const float* ln_g = nullptr, const float* ln_b = nullptr) {
+  const bool ln = ln_g != nullptr;
   if (B < 1 || B > DEC_MAX_B) return fail(c, GPT2_ERR_BATCH, "gemv: 1 <= B <= 16 rows");
   if (N <= 0 || K <= 0 || (K % 8) || (ldx % 8) || (reinterpret_cast<uintptr_t>(x) & 15) ||
-      (reinterpret_cast<uintptr_t>(W) & 15))
-    return fail(c, GPT2_ERR_CONFIG, "gemv: K and ldx multiples of 8, 16-byte aligned x and W");
+      (reinterpret_cast<uintptr_t>(W) & 15) || (ln && (!ln_b || (reinterpret_cast<uintptr_t>(ln_g) & 15) ||
+                                                      (reinterpret_cast<uintptr_t>(ln_b) & 15))))
+    return fail(c, GPT2_ERR_CONFIG, "gemv: K and ldx multiples of 8, 16-byte aligned x, W and LayerNorm vectors");
   if (epi == EPI_F32_RESID && !resid) return fail(c, GPT2_ERR_CONFIG, "gemv: residual epilogue needs resid");
+  const size_t smem = (size_t)B * K * sizeof(bf16);
+  if (smem > (size_t)DEC_GEMV_MAX_SMEM) return fail(c, GPT2_ERR_CONFIG, "gemv: B * K * 2 bytes exceed 200 KB");
+  gemv_prepare();
   // wide outputs: one warp per 4 columns; narrow ones: split K across the block's warps
   int kw = 1;
   if (N < 4096)
     while (kw < DEC_WARPS && kw * 256 < K) kw *= 2;
   const int cols = DEC_COLS * (DEC_WARPS / kw);
-  const int grid = (N + cols - 1) / cols;
+  const int groups = (N + cols - 1) / cols;
+  const int grid = groups < 2 * c.num_sms ? groups : 2 * c.num_sms;  // one wave; blocks loop over groups
   const bool f32o = epi == EPI_F32_RESID || epi == EPI_F32;
   ProfScope ps(c, CAT_DEC_GEMV, 2.0 * B * N * K,
-               2.0 * N * K + 2.0 * B * K + (double)B * N * (f32o ? 4 : 2) + (epi == EPI_F32_RESID ? 4.0 * B * N : 0.0));
+               2.0 * N * K + (ln ? 4.0 : 2.0) * B * K + (double)B * N * (f32o ? 4 : 2) +
+                   (epi == EPI_F32_RESID ? 4.0 * B * N : 0.0));
+#define GEMV_KW(KWV)                                                                                          \
+  return ln ? gemv_inst<KWV, true>(c, epi, grid, smem, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr, ln_g, ln_b) \
+            : gemv_inst<KWV, false>(c, epi, grid, smem, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr, ln_g, ln_b)
   switch (kw) {
-    case 1: return gemv_inst<1>(c, epi, grid, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
-    case 2: return gemv_inst<2>(c, epi, grid, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
-    case 4: return gemv_inst<4>(c, epi, grid, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
-    default: return gemv_inst<8>(c, epi, grid, x, ldx, B, W, N, K, bias, out, ldo, resid, ldr);
+    case 1: GEMV_KW(1);
+    case 2: GEMV_KW(2);
+    case 4: GEMV_KW(4);
+    default: GEMV_KW(8);
   }
+#undef GEMV_KW
 }
 
-// Key splits per (sequence, head) for a generation step: enough blocks for two per SM.
+// Key splits per (sequence, head) for a generation step: none once every SM has a
+// (sequence, head); else enough splits for two blocks per SM.
 inline int decode_splits(int B, int NH, int num_sms) {
   const int bh = B * NH;
+  if (bh >= num_sms) return 1;
   int S = (2 * num_sms + bh - 1) / bh;
   return S < 1 ? 1 : (S > DEC_MAX_SPLIT ? DEC_MAX_SPLIT : S);
 }
@@ -809,11 +887,13 @@ inline int decode_attention(const LaunchCtx& c, const bf16* qkv, bf16* cache, in
   }
   ProfScope ps(c, CAT_DEC_ATTN, 4.0 * B * C * mean_keys, 4.0 * B * C * mean_keys + 10.0 * B * C);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DEC_HD);
-  decode_attn_kernel<<<B * NH * S, DEC_ATT_THREADS, smem, c.stream>>>(qkv, cache, cache_seq, C, NH, pos_ptr, S,
-                                                                       scale_log2, att, part);
+  cudaError_t e = launch_k(c, decode_attn_kernel, dim3(B * NH * S), dim3(DEC_ATT_THREADS), smem, qkv, cache,
+                           cache_seq, C, NH, pos_ptr, S, scale_log2, att, part);
+  if (e != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("decode_attention: ") + cudaGetErrorString(e));
   int r = check_launch(c, "decode_attention");
   if (r || S == 1) return r;
-  decode_attn_combine_kernel<<<B * NH, DEC_HD, 0, c.stream>>>(part, S, C, NH, att);
+  e = launch_k(c, decode_attn_combine_kernel, dim3(B * NH), dim3(DEC_HD), 0, (const float*)part, S, C, NH, att);
+  if (e != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("decode_combine: ") + cudaGetErrorString(e));
   return check_launch(c, "decode_attention_combine");
 }
 

@@ -22,13 +22,19 @@ __device__ __forceinline__ void store4<bf16>(bf16* dst, float a, float b, float 
 }
 
 // x: fp32 [N, C]; y: T [N, C]; mean, rstd: fp32 [N]. C % 4 == 0, C <= 128 * NV.
-template <class T, int NV>
+// PDL: launched as a programmatic dependent (generation steps), it waits for the
+// previous kernel before reading x.
+template <class T, int NV, bool PDL = false>
 __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_fwd_kernel(const float* __restrict__ x,
                                                                       const float* __restrict__ g,
                                                                       const float* __restrict__ b, T* __restrict__ y,
                                                                       float* __restrict__ mean,
                                                                       float* __restrict__ rstd, int N, int C) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (PDL) {
+    pdl_launch_dependents();
+    pdl_wait();
+  }
   const long long row = (long long)blockIdx.x * LN_WARPS + warp;
   if (row >= N) return;
   const float* xr = x + row * C;

@@ -8,10 +8,11 @@
 // c_j > u * c_last, else the last kept one. -0.0 ranks equal to +0.0. Logits must not be NaN.
 //
 // One CTA of 1024 threads per row. The k-th largest value comes from a most-significant-
-// digit radix select over order-preserving 32-bit keys (four 8-bit passes over the row);
-// the k candidates are gathered (equal keys taken in index order), sorted by (value desc,
-// index asc) with a bitonic sort in shared memory, weighted in parallel, and one thread
-// forms the running sums in order.
+// digit radix select over order-preserving 32-bit keys (four 8-bit passes over the row,
+// each digit found by one warp's scan of the 256-bin histogram); the k candidates are
+// gathered (equal keys taken in index order), sorted by (value desc, index asc) with a
+// bitonic sort in shared memory, weighted in parallel, and one thread forms the running
+// sums in order.
 #pragma once
 #include "common.cuh"
 
@@ -39,7 +40,7 @@ __global__ void __launch_bounds__(TOPK_THREADS)
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long cand[TOPK_MAX_K];  // (~key << 32 | index): ascending = value desc, index asc
   __shared__ double w[TOPK_MAX_K];
-  __shared__ uint32_t s_prefix, s_need, s_count, s_eq_base;
+  __shared__ uint32_t s_prefix, s_need, s_count;
   __shared__ int warp_cnt[TOPK_THREADS / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* z = logits + (int64_t)blockIdx.x * ld;
@@ -60,53 +61,71 @@ __global__ void __launch_bounds__(TOPK_THREADS)
       if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      const uint32_t need = s_need;
-      uint32_t acc = 0u;
-      int digit = 255;
-      for (; digit > 0; --digit) {  // largest digit first, until `need` keys are covered
-        if (acc + hist[digit] >= need) break;
-        acc += hist[digit];
+    if (warp == 0) {
+      // lane l holds digits 255-8l .. 248-8l (descending); an inclusive scan over lanes
+      // finds the digit at which the running count of larger keys reaches `need`
+      uint32_t cnt[8], tot = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cnt[i] = hist[255 - (lane * 8 + i)];
+        tot += cnt[i];
       }
-      s_prefix = prefix | ((uint32_t)digit << shift);
-      s_need = need - acc;  // keys wanted among those that share the new prefix
+      uint32_t incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const uint32_t need = s_need, excl = incl - tot;
+      if (excl < need && need <= incl) {  // exactly one lane: need <= keys under the prefix
+        uint32_t acc = excl;
+        int i = 0;
+        for (; i < 7; ++i) {
+          if (acc + cnt[i] >= need) break;
+          acc += cnt[i];
+        }
+        s_prefix = prefix | ((uint32_t)(255 - (lane * 8 + i)) << shift);
+        s_need = need - acc;  // keys wanted among those that share the new prefix
+      }
     }
     __syncthreads();
   }
-  // every key above the k-th, and the first s_need keys equal to it in index order
+  // every key above the k-th, and the first s_need keys equal to it in index order: each
+  // warp owns a contiguous range of the row, counts its equal keys, and after one scan of
+  // those counts walks its range again placing candidates
   const uint32_t kth = s_prefix, n_eq = s_need;
-  if (tid == 0) {
-    s_count = 0u;
-    s_eq_base = 0u;
+  constexpr int NWARP = TOPK_THREADS / 32;
+  const int seg = ((V + NWARP - 1) / NWARP + 31) & ~31;
+  const int r0 = min(V, warp * seg), r1 = min(V, r0 + seg);
+  if (tid == 0) s_count = 0u;
+  uint32_t n_mine = 0u;
+  for (int i0 = r0; i0 < r1; i0 += 32) {
+    const int i = i0 + lane;
+    const bool eq = i < r1 && topk_key(z[i]) == kth;
+    n_mine += (uint32_t)__popc(__ballot_sync(0xffffffffu, eq));
   }
+  if (lane == 0) warp_cnt[warp] = (int)n_mine;
   __syncthreads();
-  for (int base = 0; base < V; base += TOPK_THREADS) {
-    const int i = base + tid;
+  uint32_t before = 0u;  // equal keys at lower indices than this warp's range
+  for (int q = 0; q < warp; ++q) before += (uint32_t)warp_cnt[q];
+  for (int i0 = r0; i0 < r1; i0 += 32) {
+    const int i = i0 + lane;
     uint32_t key = 0u;
     bool gt = false, eq = false;
-    if (i < V) {
+    if (i < r1) {
       key = topk_key(z[i]);
       gt = key > kth;
       eq = key == kth;
     }
     const unsigned ballot = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) warp_cnt[warp] = __popc(ballot);
-    __syncthreads();
-    uint32_t before = s_eq_base;  // equal keys at lower indices
-    for (int q = 0; q < warp; ++q) before += (uint32_t)warp_cnt[q];
-    before += (uint32_t)__popc(ballot & ((1u << lane) - 1u));
-    if (gt || (eq && before < n_eq)) {
+    const uint32_t rank = before + (uint32_t)__popc(ballot & ((1u << lane) - 1u));
+    if (gt || (eq && rank < n_eq)) {
       const uint32_t slot = atomicAdd(&s_count, 1u);
       if (slot < (uint32_t)TOPK_MAX_K) cand[slot] = ((unsigned long long)(~key) << 32) | (unsigned)i;
     }
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t tot = 0u;
-      for (int q = 0; q < TOPK_THREADS / 32; ++q) tot += (uint32_t)warp_cnt[q];
-      s_eq_base += tot;
-    }
-    __syncthreads();
+    before += (uint32_t)__popc(ballot);
   }
+  __syncthreads();
   // bitonic sort of the candidates, padded to a power of two with the largest code
   int np = 1;
   while (np < k) np <<= 1;

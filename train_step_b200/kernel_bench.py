@@ -42,6 +42,33 @@ def hbm_peak():
     return 6650.0, "fallback"
 
 
+def gemv_bench(a) -> dict:
+    """The generation step's skinny products (GPT-2 124M shapes) timed alone: `iters`
+    back-to-back launches, plain and as programmatic dependents. One weight matrix is
+    reused, so after the first launch it is served from L2: this is each kernel's latency
+    floor, not its HBM-bound time."""
+    C, V = a.C, a.V
+    shapes = {"qkv+ln": (3 * C, C, 0, True), "attn_out": (C, C, 2, False), "fc+ln": (4 * C, C, 1, True),
+              "proj": (C, 4 * C, 2, False), "head+ln": (V, C, 4, True)}
+    out = {}
+    for name, (N, K, epi, ln) in shapes.items():
+        B = a.B
+        x = torch.randn(B, K, device="cuda", dtype=torch.float32 if ln else torch.bfloat16)
+        W = torch.randn(N, K, device="cuda").to(torch.bfloat16)
+        bias = torch.zeros(N, device="cuda")
+        g = torch.ones(K, device="cuda") if ln else None
+        b = torch.zeros(K, device="cuda") if ln else None
+        resid = torch.zeros(B, N, device="cuda") if epi == 2 else None
+        o = torch.empty(B, N, device="cuda", dtype=torch.float32 if epi in (2, 4) else torch.bfloat16)
+        row = {}
+        for pdl in (False, True):
+            ms = tsb.gemv(x, W, o, B=B, N=N, K=K, epilogue=epi, bias=bias, resid=resid, ldr=N, ln_g=g, ln_b=b,
+                          iters=a.iters, pdl=pdl)
+            row["pdl" if pdl else "plain"] = dict(us=ms * 1e3, gbs=2.0 * N * K / (ms * 1e-3) / 1e9)
+        out[name] = row
+    return dict(B=a.B, gemv=out)
+
+
 def decode_bench(a) -> dict:
     """Generation with the key/value cache on GPT-2 124M (random weights): B prompts of T0
     tokens, then `steps` decode steps, each one forward step for all B sequences followed
@@ -100,7 +127,7 @@ def decode_bench(a) -> dict:
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["gemm", "attn", "attn_bwd", "ln", "ce", "decode"])
+    ap.add_argument("kernel", choices=["gemm", "attn", "attn_bwd", "ln", "ce", "decode", "gemv"])
     ap.add_argument("--M", type=int, default=16384)
     ap.add_argument("--N", type=int, default=3072)
     ap.add_argument("--K", type=int, default=768)
@@ -168,6 +195,8 @@ def main() -> None:
         res.update(shape=[N, C], ms=ms, gbs=N * C * 6 / (ms * 1e-3) / 1e9)
     elif a.kernel == "decode":
         res.update(decode_bench(a))
+    elif a.kernel == "gemv":
+        res.update(gemv_bench(a))
     else:
         N, V = a.M, a.V
         ld = (V + 63) // 64 * 64

@@ -1,9 +1,9 @@
 """Learning-rate schedule of the training recipe: linear warmup, then cosine decay.
 
-The recipe ("GPT From Scratch", Training Recipe table; "Cosine LR Schedule" in the
-repository tour) fixes the peak rate 6e-4, the floor 6e-5 (peak / 10), 715 warmup
-steps and 19,073 total steps, and names the shape: linear warmup, then cosine decay
-to the floor. It does not fix the step indexing; here step s (0-based) of the warmup
+The recipe ("AxonLM", Training Recipe table) fixes the peak rate 6e-4, the floor 6e-5
+(peak / 10), 715 warmup steps and 19,073 total steps; "AxonLM", Key Features, and
+"Genesis", Training Features, name the shape: linear warmup, then cosine decay to the
+floor. It does not fix the step indexing; here step s (0-based) of the warmup
 uses peak * (s + 1) / warmup, so the first update is not wasted at rate 0, the
 cosine runs from the peak at s = warmup to the floor at s = total, and the rate
 stays at the floor afterwards.

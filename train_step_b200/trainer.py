@@ -1,7 +1,8 @@
 """Training driver around the C-ABI model: gradient accumulation, optional data-parallel
 gradient averaging, the warmup + cosine learning-rate schedule, AdamW, evaluation loss
-and checkpoints ("GPT From Scratch", Training Recipe; recipe pieces: warmup plus cosine
-decay, clipping at 1.0, gradient accumulation).
+and checkpoints ("AxonLM", Training Recipe and Key Features: cosine schedule with warmup,
+checkpoint resume; "GPT From Scratch", Key decisions: warmup plus cosine decay, clipping at
+1.0, gradient accumulation).
 """
 from __future__ import annotations
 
