@@ -232,3 +232,18 @@ def test_gemv_epilogues_match_oracle(B, N, K):
     y, _, _ = oracle.layernorm_fwd(_g64(xf), _g64(g), _g64(b))
     tsb.gemv(xf, W, o4, epilogue=tsb.EPI_F32, ln_g=g, ln_b=b, **kw)
     assert rel_l2(_g64(o4), oracle.linear_fwd(y, _g64(W))) < 4e-3
+
+
+def test_generation_token_range_errors():
+    m = tsb.GPT2(SMALL, seed=2)
+    bad = torch.full((2, 4), SMALL.V, dtype=torch.int32)
+    with pytest.raises(tsb.Gpt2Error):
+        m.prefill(bad)
+    good = torch.randint(0, SMALL.V, (2, 4), dtype=torch.int32)
+    m.prefill(good)
+    with pytest.raises(tsb.Gpt2Error):
+        m.decode_step(torch.tensor([0, -1], dtype=torch.int32))  # reported by the synchronisation
+    m.decode_step(torch.tensor([1, 2], dtype=torch.int32))       # the handle stays usable
+    with pytest.raises(tsb.Gpt2Error):
+        m.decode_step(torch.tensor([1, 2, 3], dtype=torch.int32))  # B differs from the prefill's
+    m.close()
