@@ -1,10 +1,12 @@
 // decode.cuh -- kernels of one generation step with a key/value cache.
 //
 // A step advances B <= 16 sequences by one token. Its linear layers are skinny
-// products (B rows against a [N, K] weight): bound by reading each weight once from
-// HBM, so they run on CUDA cores with 16-byte weight loads spread over every SM rather
-// than on 128-row tensor-core tiles that would sit 7/8 empty. Attention is one query
-// row per (sequence, head) against the cached keys and values of positions 0..pos.
+// products (B rows against a [N, K] weight), bound by reading each weight once and by
+// the latency of a chain of small kernels: they use register-level m16n8k16 tensor-core
+// products with the batch rows as the 16-row operand and 16-byte weight loads spread over
+// every SM, not 128-row tcgen05 tiles that would sit at least 7/8 empty behind a TMEM and
+// barrier set-up. Attention is one query row per (sequence, head) against the cached keys
+// and values of positions 0..pos.
 #pragma once
 #include "common.cuh"
 #include "gemm_tc.cuh"
@@ -12,8 +14,8 @@
 namespace g2 {
 
 constexpr int DEC_MAX_B = 16;  // sequences advanced by one step
-constexpr int DEC_COLS = 4;    // output columns per warp
 constexpr int DEC_WARPS = 8;
+constexpr int DEC_PF = 8;  // weight slices in flight per warp in the skinny product
 constexpr int DEC_ATT_THREADS = 256;
 constexpr int DEC_HD = 64;  // head size the attention kernel is written for
 
@@ -32,50 +34,65 @@ __device__ __forceinline__ uint4 dec_ld_stream(const void* p) {
   return r;
 }
 
-// out[b][n] = epilogue(sum_k x[b][k] * W[n][k] (+ bias[n])) for b < B, n < N.
-// W: bf16 [N][K] row-major (the K-major layout the training GEMMs read). x: bf16 rows of
-// stride ldx; or, with LN, fp32 rows of the residual stream that the kernel layer-
-// normalises itself (y = (x - mean) * rstd * ln_g + ln_b with the biased variance and
-// eps 1e-5, rounded to bf16 as the LayerNorm kernel stores it), so that no LayerNorm
-// launch sits between two products.
-// Each block first stages all B rows of x in shared memory as bf16 (one burst of loads,
-// one wait) and then walks groups of output columns (group g = blockIdx.x, + gridDim.x,
-// ...). Its 8 warps form KW groups along K and 8/KW groups of 4 columns; a lane
-// accumulates 4 columns x 16 rows in fp32 over 8-element K chunks, and a butterfly
-// reduce-scatter leaves lane L with entries 2L and 2L+1 of that 4x16 block (column L/8,
-// rows 2L mod 16 and the next). Dynamic shared memory: B*K bf16.
+// One m16n8k16 bf16 tensor-core product with fp32 accumulation (D += A B): A is 16 x 16
+// (rows x k), B is 16 x 8 (k x columns), fragments as the PTX ISA lays them out.
+__device__ __forceinline__ void dec_mma(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                        uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// out[b][n] = epilogue(sum_k x[b][k] * W[n][k] (+ bias[n])) for b < B <= 16, n < N.
+// W: bf16 [N][K] row-major (the K-major layout the training GEMMs read), K % 32 == 0.
+// x: bf16 rows of stride ldx; or, with LN, fp32 rows of the residual stream that the kernel
+// layer-normalises itself (y = (x - mean) * rstd * ln_g + ln_b with the biased variance and
+// eps 1e-5, rounded to bf16 as the LayerNorm kernel stores it), so that no LayerNorm launch
+// sits between two products.
+// The batch rows are the 16-row operand of m16n8k16 tensor-core products: each block stages
+// the B rows of x in shared memory as bf16 rows of K + 8 (the 16-byte pad spreads the
+// fragment loads over all banks; rows B..15 enter the products as zero registers), and each
+// warp accumulates one 16 x 8 output tile (8 weight rows) over its share of K, with up to 8
+// weight slices in flight; KW warps split K and their tiles are summed through shared
+// memory. For a 32-wide slice of K a lane loads 16 bytes of one weight row (row n0 + lane/4,
+// k = 8 (lane % 4) ... + 7) and 16 bytes of x rows lane/4 and lane/4 + 8 at the same k; the
+// slice's k positions are assigned to the two k16 products so that these registers are
+// exactly the A and B fragments (any one-to-one assignment of k gives the same sum).
 // Epilogues: EPI_BF16 (bf16 out), EPI_BF16_GELU (bf16 gelu_tanh(acc + bias)), EPI_F32_RESID
 // (fp32 out = resid + acc + bias), EPI_F32 (fp32 out = acc).
 template <int EPI, int KW, bool LN>
-__global__ void __launch_bounds__(DEC_WARPS * 32, 2)
+__global__ void __launch_bounds__(DEC_WARPS * 32)
     gemv_bf16_kernel(const void* __restrict__ xin, int64_t ldx, int B, const bf16* __restrict__ W, int N, int K,
                      const float* __restrict__ bias, void* __restrict__ out, int64_t ldo,
                      const float* __restrict__ resid, int64_t ldr, const float* __restrict__ ln_g,
                      const float* __restrict__ ln_b) {
-  constexpr int NW = DEC_WARPS / KW;
-  constexpr int NA = DEC_COLS * DEC_MAX_B;  // 64 accumulators per lane
+  constexpr int NW = DEC_WARPS / KW;  // 8-column tiles per block
   extern __shared__ __align__(16) unsigned char dec_smem[];
-  bf16* xs = reinterpret_cast<bf16*>(dec_smem);  // [B][K]
-  __shared__ float red[DEC_WARPS][NA];
+  bf16* xs = reinterpret_cast<bf16*>(dec_smem);  // [16][K + 8]
+  __shared__ float red[DEC_WARPS][4][32];
   __shared__ float stat[DEC_MAX_B][2];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int kw = warp % KW, nw = warp / KW;
-  const int groups = (N + NW * DEC_COLS - 1) / (NW * DEC_COLS);
-  const int k_first = (kw * 32 + lane) * 8;
-  // weights do not depend on the previous kernel: the first chunk is fetched before
-  // waiting for it, and each later chunk while the one before is in use
-  uint4 wraw[DEC_COLS];
-  {
-    const int n0 = (blockIdx.x * NW + nw) * DEC_COLS;
+  const int g = lane >> 2, q = lane & 3;
+  const int n0 = (blockIdx.x * NW + nw) * 8;
+  const int xstride = K + 8;  // rows 0..B-1 staged; the 16-byte pad spreads fragment loads over the banks
+  const bf16* wrow = W + (int64_t)(n0 + g) * K + q * 8;
+  const bool wok = n0 + g < N;
+  // this warp's 32-wide slices of K are kw, kw + KW, ...; weights do not depend on the
+  // previous kernel, so the first DEC_PF slices are fetched before waiting for it, and
+  // each slot is refilled DEC_PF slices ahead as it is consumed
+  const int nslices = (K / 32 - kw + KW - 1) / KW;
+  uint4 wbuf[DEC_PF];
 #pragma unroll
-    for (int r = 0; r < DEC_COLS; ++r) {
-      wraw[r] = make_uint4(0u, 0u, 0u, 0u);
-      if (k_first < K && n0 + r < N) wraw[r] = dec_ld_stream(W + (int64_t)(n0 + r) * K + k_first);
-    }
+  for (int j = 0; j < DEC_PF; ++j) {
+    wbuf[j] = make_uint4(0u, 0u, 0u, 0u);
+    if (wok && j < nslices) wbuf[j] = dec_ld_stream(wrow + (kw + j * KW) * 32);
   }
   pdl_launch_dependents();
   pdl_wait();
-  // stage x
+  // stage the B rows of x as bf16
   if (LN) {
     const float* xf = static_cast<const float*>(xin);
     for (int b = warp; b < B; b += DEC_WARPS) {  // row statistics, K % 4 == 0
@@ -103,93 +120,63 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 2)
     for (int i = threadIdx.x; i < B * per_row; i += DEC_WARPS * 32) {
       const int b = i / per_row, c = (i % per_row) * 4;
       const float4 v = *reinterpret_cast<const float4*>(xf + (int64_t)b * ldx + c);
-      const float4 g = __ldg(reinterpret_cast<const float4*>(ln_g + c));
+      const float4 gg = __ldg(reinterpret_cast<const float4*>(ln_g + c));
       const float4 bb = __ldg(reinterpret_cast<const float4*>(ln_b + c));
       const float mu = stat[b][0], rs = stat[b][1];
-      *reinterpret_cast<uint2*>(xs + (int64_t)b * K + c) =
-          make_uint2(pack_bf16x2((v.x - mu) * rs * g.x + bb.x, (v.y - mu) * rs * g.y + bb.y),
-                     pack_bf16x2((v.z - mu) * rs * g.z + bb.z, (v.w - mu) * rs * g.w + bb.w));
+      *reinterpret_cast<uint2*>(xs + b * xstride + c) =
+          make_uint2(pack_bf16x2((v.x - mu) * rs * gg.x + bb.x, (v.y - mu) * rs * gg.y + bb.y),
+                     pack_bf16x2((v.z - mu) * rs * gg.z + bb.z, (v.w - mu) * rs * gg.w + bb.w));
     }
   } else {
     const bf16* x = static_cast<const bf16*>(xin);
     const int per_row = K / 8;
     for (int i = threadIdx.x; i < B * per_row; i += DEC_WARPS * 32) {
       const int b = i / per_row, c = (i % per_row) * 8;
-      *reinterpret_cast<uint4*>(xs + (int64_t)b * K + c) = *reinterpret_cast<const uint4*>(x + (int64_t)b * ldx + c);
+      *reinterpret_cast<uint4*>(xs + b * xstride + c) = *reinterpret_cast<const uint4*>(x + (int64_t)b * ldx + c);
     }
   }
   __syncthreads();
-  for (int grp = blockIdx.x; grp < groups; grp += gridDim.x) {
-    const int n0 = (grp * NW + nw) * DEC_COLS;
-    if (grp != (int)blockIdx.x) {
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  const bool rlo = g < B, rhi = g + 8 < B;  // rows g and g + 8 exist (others enter as zeros)
+  const bf16* xa = xs + g * xstride + q * 8;
+  const bf16* xb = xa + 8 * xstride;
+  for (int base = 0; base < nslices; base += DEC_PF) {
 #pragma unroll
-      for (int r = 0; r < DEC_COLS; ++r) {
-        wraw[r] = make_uint4(0u, 0u, 0u, 0u);
-        if (k_first < K && n0 + r < N) wraw[r] = dec_ld_stream(W + (int64_t)(n0 + r) * K + k_first);
+    for (int j = 0; j < DEC_PF; ++j) {
+      const int sl = base + j;
+      if (sl < nslices) {
+        const uint4 w = wbuf[j];
+        const int sn = sl + DEC_PF;
+        if (wok && sn < nslices) wbuf[j] = dec_ld_stream(wrow + (kw + sn * KW) * 32);
+        const int kb = (kw + sl * KW) * 32;
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 a = rlo ? *reinterpret_cast<const uint4*>(xa + kb) : z;
+        const uint4 c = rhi ? *reinterpret_cast<const uint4*>(xb + kb) : z;
+        dec_mma(d, a.x, c.x, a.y, c.y, w.x, w.y);  // k = 8q + {0,1} and 8q + {2,3} of the slice
+        dec_mma(d, a.z, c.z, a.w, c.w, w.z, w.w);  // k = 8q + {4,5} and 8q + {6,7}
       }
     }
-    float acc[NA];
+  }
+  if (KW > 1) {
 #pragma unroll
-    for (int i = 0; i < NA; ++i) acc[i] = 0.f;
-    for (int k = k_first; k < K; k += KW * 256) {
-      float wv[DEC_COLS][8];
+    for (int i = 0; i < 4; ++i) red[warp][i][lane] = d[i];
+    __syncthreads();
+    if (kw != 0) return;
 #pragma unroll
-      for (int r = 0; r < DEC_COLS; ++r) dec_unpack8(wraw[r], wv[r]);
-      const int kn = k + KW * 256;
+    for (int j = 1; j < KW; ++j)
 #pragma unroll
-      for (int r = 0; r < DEC_COLS; ++r)
-        if (kn < K && n0 + r < N) wraw[r] = dec_ld_stream(W + (int64_t)(n0 + r) * K + kn);
+      for (int i = 0; i < 4; ++i) d[i] += red[warp + j][i][lane];
+  }
+  // d[0], d[1]: row g, columns 2q, 2q+1; d[2], d[3]: row g + 8, the same columns
 #pragma unroll
-      for (int b = 0; b < DEC_MAX_B; ++b) {
-        if (b < B) {
-          float xv[8];
-          dec_unpack8(*reinterpret_cast<const uint4*>(xs + b * K + k), xv);
-#pragma unroll
-          for (int r = 0; r < DEC_COLS; ++r)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[r * DEC_MAX_B + b] = fmaf(wv[r][e], xv[e], acc[r * DEC_MAX_B + b]);
-        }
-      }
-    }
-    // reduce-scatter across the warp: each step keeps half of the entries, adding the
-    // partner lane's copy of them
-#pragma unroll
-    for (int o = 16, half = NA / 2; o >= 1; o >>= 1, half >>= 1) {
-      const bool hi = (lane & o) != 0;
-#pragma unroll
-      for (int i = 0; i < half; ++i) {
-        const float send = hi ? acc[i] : acc[i + half];
-        const float keep = hi ? acc[i + half] : acc[i];
-        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-    }
-    if (KW > 1) {
-      red[warp][2 * lane] = acc[0];
-      red[warp][2 * lane + 1] = acc[1];
-      __syncthreads();
-      if (kw == 0) {
-#pragma unroll
-        for (int q = 1; q < KW; ++q) {
-          acc[0] += red[warp + q][2 * lane];
-          acc[1] += red[warp + q][2 * lane + 1];
-        }
-      }
-      __syncthreads();  // red is rewritten by the next group
-    }
-    const int n = n0 + (lane >> 3);
-    if (kw == 0 && n < N) {
-      const float bn = (EPI != EPI_F32 && bias) ? bias[n] : 0.f;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int b = ((2 * lane) & (DEC_MAX_B - 1)) + e;
-        if (b >= B) continue;
-        const float v = acc[e] + bn;
-        if (EPI == EPI_BF16) static_cast<bf16*>(out)[(int64_t)b * ldo + n] = __float2bfloat16_rn(v);
-        if (EPI == EPI_BF16_GELU) static_cast<bf16*>(out)[(int64_t)b * ldo + n] = __float2bfloat16_rn(gelu_tanh(v));
-        if (EPI == EPI_F32_RESID) static_cast<float*>(out)[(int64_t)b * ldo + n] = resid[(int64_t)b * ldr + n] + v;
-        if (EPI == EPI_F32) static_cast<float*>(out)[(int64_t)b * ldo + n] = v;
-      }
-    }
+  for (int i = 0; i < 4; ++i) {
+    const int b = g + (i >> 1) * 8, n = n0 + 2 * q + (i & 1);
+    if (b >= B || n >= N) continue;
+    const float v = d[i] + ((EPI != EPI_F32 && bias) ? bias[n] : 0.f);
+    if (EPI == EPI_BF16) static_cast<bf16*>(out)[(int64_t)b * ldo + n] = __float2bfloat16_rn(v);
+    if (EPI == EPI_BF16_GELU) static_cast<bf16*>(out)[(int64_t)b * ldo + n] = __float2bfloat16_rn(gelu_tanh(v));
+    if (EPI == EPI_F32_RESID) static_cast<float*>(out)[(int64_t)b * ldo + n] = resid[(int64_t)b * ldr + n] + v;
+    if (EPI == EPI_F32) static_cast<float*>(out)[(int64_t)b * ldo + n] = v;
   }
 }
 

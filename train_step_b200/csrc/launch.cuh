@@ -763,7 +763,7 @@ inline int cross_entropy(const LaunchCtx& c, int dtype, void* logits, long long 
 // ---------------------------------------------------------------------------
 // generation: skinny GEMMs, single-query attention, key/value cache, sampling
 // ---------------------------------------------------------------------------
-constexpr int DEC_GEMV_MAX_SMEM = 200 * 1024;  // staged x: B * K bf16
+constexpr int DEC_GEMV_MAX_SMEM = 200 * 1024;  // staged x: 16 * (K + 8) bf16
 
 template <int KW, bool LN>
 void gemv_attrs() {
@@ -830,21 +830,20 @@ inline int gemv_bf16(const LaunchCtx& c, int epi, const void* x, int64_t ldx, in
                      const float* ln_g = nullptr, const float* ln_b = nullptr) {
   const bool ln = ln_g != nullptr;
   if (B < 1 || B > DEC_MAX_B) return fail(c, GPT2_ERR_BATCH, "gemv: 1 <= B <= 16 rows");
-  if (N <= 0 || K <= 0 || (K % 8) || (ldx % 8) || (reinterpret_cast<uintptr_t>(x) & 15) ||
+  if (N <= 0 || K <= 0 || (K % 32) || (ldx % 8) || (reinterpret_cast<uintptr_t>(x) & 15) ||
       (reinterpret_cast<uintptr_t>(W) & 15) || (ln && (!ln_b || (reinterpret_cast<uintptr_t>(ln_g) & 15) ||
                                                       (reinterpret_cast<uintptr_t>(ln_b) & 15))))
-    return fail(c, GPT2_ERR_CONFIG, "gemv: K and ldx multiples of 8, 16-byte aligned x, W and LayerNorm vectors");
+    return fail(c, GPT2_ERR_CONFIG, "gemv: K % 32 == 0, ldx % 8 == 0, 16-byte aligned x, W and LayerNorm vectors");
   if (epi == EPI_F32_RESID && !resid) return fail(c, GPT2_ERR_CONFIG, "gemv: residual epilogue needs resid");
-  const size_t smem = (size_t)B * K * sizeof(bf16);
-  if (smem > (size_t)DEC_GEMV_MAX_SMEM) return fail(c, GPT2_ERR_CONFIG, "gemv: B * K * 2 bytes exceed 200 KB");
+  const size_t smem = (size_t)DEC_MAX_B * (K + 8) * sizeof(bf16);
+  if (smem > (size_t)DEC_GEMV_MAX_SMEM) return fail(c, GPT2_ERR_CONFIG, "gemv: K too large for the staged rows");
   gemv_prepare();
-  // wide outputs: one warp per 4 columns; narrow ones: split K across the block's warps
+  // 8-column tiles; split K over up to 8 warps until there are about 8 warps per SM
+  const int tiles = (N + 7) / 8;
   int kw = 1;
-  if (N < 4096)
-    while (kw < DEC_WARPS && kw * 256 < K) kw *= 2;
-  const int cols = DEC_COLS * (DEC_WARPS / kw);
-  const int groups = (N + cols - 1) / cols;
-  const int grid = groups < 2 * c.num_sms ? groups : 2 * c.num_sms;  // one wave; blocks loop over groups
+  while (kw < DEC_WARPS && (long long)tiles * kw < 8LL * c.num_sms && K / 32 >= 2 * kw) kw *= 2;
+  const int nw = DEC_WARPS / kw;
+  const int grid = (tiles + nw - 1) / nw;
   const bool f32o = epi == EPI_F32_RESID || epi == EPI_F32;
   ProfScope ps(c, CAT_DEC_GEMV, 2.0 * B * N * K,
                2.0 * N * K + (ln ? 4.0 : 2.0) * B * K + (double)B * N * (f32o ? 4 : 2) +
