@@ -302,8 +302,10 @@ int gpt2_op_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, c
  * x[b][k] W[n][k]) for b < B <= 16, n < N; W bf16 [N][K] row-major; epilogue 0 (bf16 out,
  * + bias), 1 (bf16 gelu_tanh(acc + bias)), 2 (fp32 out = resid + acc + bias) or 4 (fp32
  * out = acc). x is bf16 rows of stride ldx, or, when ln_g and ln_b are given, fp32 rows that
- * are layer-normalised first (eps 1e-5, result rounded to bf16). K and ldx multiples of 8,
- * 16-byte aligned x, W, ln_g, ln_b; B*K*2 <= 200 KB. With iters > 1 the product is then
+ * are layer-normalised first (eps 1e-5, result rounded to bf16). K a multiple of 32 with
+ * 16 * (K + 8) * 2 bytes <= 200 KB (K <= 6392), ldx a multiple of 8, 16-byte aligned x, W,
+ * ln_g, ln_b; GPT2_ERR_BATCH for B outside [1, 16], GPT2_ERR_CONFIG for the rest. Runs on
+ * the tensor cores (m16n8k16 products, fp32 accumulation). With iters > 1 the product is then
  * launched iters more times back to back (as programmatic dependents when pdl != 0) and
  * *ms_out receives the mean milliseconds per launch. Synchronises. */
 int gpt2_op_gemv(const void* x, int64_t ldx, int B, const void* W, int N, int K, int epilogue, const float* bias,
