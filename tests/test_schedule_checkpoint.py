@@ -77,3 +77,19 @@ def test_checkpoint_round_trip(tmp_path):
     c = _FakeModel(Config(L=2, H=2, C=8, T=4, V=11), 1000, 3)
     with pytest.raises(ValueError):
         checkpoint.load(c, path)
+
+
+def test_checkpoint_payload_and_atomic_name(tmp_path):
+    # 12 bytes per parameter (fp32 p, m, v): 1.49 GB at 124,439,808 parameters, the figure
+    # "gpt/docs/LLM.md" (Memory Footprint) gives for a checkpoint with optimizer state
+    from train_step_b200 import Config
+    cfg = Config(L=1, H=2, C=8, T=4, V=11)
+    a = _FakeModel(cfg, 5000, 4)
+    path = str(tmp_path / "ckpt")  # no extension: the file is written under exactly this name
+    checkpoint.save(a, path, step=3)
+    assert sorted(p.name for p in tmp_path.iterdir()) == ["ckpt"]
+    with np.load(path) as d:
+        payload = sum(d[k].nbytes for k in ("params", "adam_m", "adam_v"))
+        assert all(d[k].dtype == np.float32 for k in ("params", "adam_m", "adam_v"))
+    assert payload == 12 * 5000
+    assert abs(12 * 124_439_808 / 1e9 - 1.49) < 0.01

@@ -262,6 +262,20 @@ class GPT2:
         self._check(lib().gpt2_grad_buffer(self.h, ct.byref(p), ct.byref(n)))
         return p.value, n.value
 
+    def grad_tensor(self):
+        """Zero-copy fp32 CUDA tensor over the flat gradient storage (the library's padded
+        layout), e.g. for a data-parallel all-reduce between micro-batch accumulation and
+        the optimizer step."""
+        import torch
+
+        class _View:
+            pass
+
+        ptr, n = self.grad_buffer()
+        v = _View()
+        v.__cuda_array_interface__ = {"shape": (n,), "typestr": "<f4", "data": (ptr, False), "version": 3}
+        return torch.as_tensor(v, device="cuda")
+
     def profile(self, enable: bool) -> None:
         self._check(lib().gpt2_profile(self.h, int(enable)))
 

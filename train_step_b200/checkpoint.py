@@ -9,16 +9,23 @@ checkpoint resume; "gpt/docs/LLM.md", Memory Footprint: about 1.49 GB with optim
 from __future__ import annotations
 
 import json
+import os
 from dataclasses import asdict
 
 import numpy as np
 
 
 def save(model, path: str, step: int = 0, extra: dict | None = None) -> None:
+    """Write the checkpoint to `path` (exactly that name) through a temporary file in the
+    same directory and an atomic rename, so that an interrupted save never leaves a
+    truncated file under `path`."""
     params = model.get_params()
     m, v, t = model.get_adam()
-    np.savez(path, params=params, adam_m=m, adam_v=v, adam_t=np.int64(t), step=np.int64(step),
-             config=json.dumps(asdict(model.cfg), sort_keys=True), extra=json.dumps(extra or {}))
+    tmp = f"{path}.tmp.{os.getpid()}"
+    with open(tmp, "wb") as f:
+        np.savez(f, params=params, adam_m=m, adam_v=v, adam_t=np.int64(t), step=np.int64(step),
+                 config=json.dumps(asdict(model.cfg), sort_keys=True), extra=json.dumps(extra or {}))
+    os.replace(tmp, path)
 
 
 def load(model, path: str) -> tuple[int, dict]:
