@@ -12,6 +12,15 @@ from . import checkpoint
 from .schedule import CosineSchedule
 
 
+def _sync_torch_stream() -> None:
+    try:
+        import torch
+    except ImportError:
+        return
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        torch.cuda.current_stream().synchronize()
+
+
 class Trainer:
     def __init__(self, model, schedule: Callable[[int], float] | None = None, weight_decay: float = 0.1,
                  beta1: float = 0.9, beta2: float = 0.95, allreduce: Callable[[], None] | None = None):
@@ -28,7 +37,11 @@ class Trainer:
         micro-batch loss, the pre-clip gradient norm and the learning rate used."""
         losses = [self.model.forward_backward(tok, tgt) for tok, tgt in micro_batches]
         if self.allreduce is not None:
+            # the gradients are complete (each forward_backward returned its loss); the
+            # collective runs on torch's current stream, which the optimizer step on the
+            # model's own stream must not overtake
             self.allreduce()
+            _sync_torch_stream()
         lr = self.schedule(self.step)
         gnorm = self.model.step(lr, self.weight_decay, self.beta1, self.beta2)
         self.step += 1
