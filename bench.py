@@ -146,9 +146,33 @@ def cpu_baseline(c, seconds_hint=True):
     _, g = oracle.forward_backward(oc, p, tok, tgt)
     oracle.adamw_step(oc, p, g, np.zeros_like(p), np.zeros_like(p), 1, LR, WD, B1, B2)
     dt = time.perf_counter() - t0
-    return {"value": Ts / dt, "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
-            "sample": f"1 sequence x {Ts} tokens of the {c['L']}-layer C={c['C']} model: float64 forward+backward "
-                      f"and one AdamW step ({dt:.1f} s)"}
+    out = {"value": Ts / dt, "unit": "tokens/s", "cores": oracle.get_threads(), "kind": "oracle",
+           "sample": f"1 sequence x {Ts} tokens of the {c['L']}-layer C={c['C']} model: float64 forward+backward "
+                     f"and one AdamW step ({dt:.1f} s)"}
+    # the same on one thread (a shorter sample), and the tiny character-level config's full step
+    threads = oracle.get_threads()
+    T1 = 32
+    tok1, tgt1 = synth.micro_batch(1, T1, c["V"], index=1)
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        _, g = oracle.forward_backward(oc, p, tok1, tgt1)
+        oracle.adamw_step(oc, p, g, np.zeros_like(p), np.zeros_like(p), 1, LR, WD, B1, B2)
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(threads)
+    out["single_thread"] = {"value": T1 / dt1, "unit": "tokens/s", "cores": 1,
+                            "sample": f"1 sequence x {T1} tokens, same model and work ({dt1:.1f} s)"}
+    tc = oracle.Config(4, 4, 128, 64, 65, 1, 1)
+    tp = oracle.init_params(tc, 42).astype(np.float64)
+    ttok, ttgt = synth.micro_batch(8, 64, 65, dist="uniform")
+    t0 = time.perf_counter()
+    _, g = oracle.forward_backward(tc, tp, ttok, ttgt)
+    oracle.adamw_step(tc, tp, g, np.zeros_like(tp), np.zeros_like(tp), 1, LR, WD, B1, B2)
+    dtt = time.perf_counter() - t0
+    out["tiny_step"] = {"value": 8 * 64 / dtt, "unit": "tokens/s", "cores": threads,
+                        "sample": f"tiny config (L4 H4 C128 T64 V65), B=8: one full step ({dtt * 1e3:.1f} ms)"}
+    return out
 
 
 def run_reference(args, c):
