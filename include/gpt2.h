@@ -5,7 +5,9 @@
  * residual connections), final LayerNorm, a bias-free head tied to the token
  * embedding (or a separate head), mean next-token cross-entropy, the backward
  * pass, gradient accumulation over micro-batches, global-norm clipping at 1.0 and
- * AdamW with weight decay on >= 2-D tensors only.
+ * AdamW with weight decay on >= 2-D tensors only; and, for generation, the
+ * forward of the last position with a key/value cache and temperature / top-k /
+ * top-p sampling.
  * Sources (page titles and sections): "gpt/docs/LLM.md" Architecture Details
  * (Embedding Layer, Transformer Blocks, Output Layer); "GPT From Scratch" Key
  * decisions (pre-norm blocks, tanh-GELU, tying, padding 50,257 -> 50,304, decay
@@ -71,7 +73,7 @@ typedef struct gpt2 gpt2; /* opaque; the library owns all device memory it uses 
 /* Create a model on the current CUDA device. Weights: N(0, 0.02), attention-out
  * and MLP-projection weights N(0, 0.02 / sqrt(2L)), biases 0, LayerNorm gains 1
  * and biases 0 ("AxonLM", Key Features: 1/sqrt(2L) for residual projections).
- * The draws follow the init stream of the design notes: element j of tensor i
+ * The draws: element j of tensor i
  * (canonical order) takes two splitmix64 outputs of seed ^ (i << 40) ^ 2j and
  * ^ (2j + 1), maps them to u1 in (0, 1] and u2 in [0, 1), and uses the cos branch
  * of Box-Muller, computed on the host in double and rounded to fp32.

@@ -20,9 +20,10 @@
 //    1.0: "AxonLM", Training Recipe; "GPT From Scratch", Key decisions.
 //  * Init N(0, 0.02), residual projections scaled by 1/sqrt(2L): "AxonLM", Key
 //    Features; "GPT From Scratch", Key decisions.
-// Readings where the pages are silent (LN eps 1e-5 with biased variance, Adam eps
-// 1e-8, clip eps 1e-6, padded vocabulary rows excluded from the softmax, the init
-// random stream) are listed in the repository's design notes.
+// Readings where the pages are silent, taken here: LN eps 1e-5 with the biased
+// variance; Adam eps 1e-8 with bias correction; clip coefficient 1 / (norm + 1e-6)
+// capped at 1; padded vocabulary rows excluded from the softmax; the init random
+// stream of init_params below.
 //
 // Parity pins: parity of this file is pinned by tests/test_oracle_*.py against
 // numbers the pages print (parameter counts, ln 65 initial loss), closed forms,
@@ -97,7 +98,7 @@ int64_t total_params(const std::vector<Tensor>& t) {
 
 // ---------------------------------------------------------------------------
 // splitmix64 (S. Vigna): state advance by the golden-ratio increment, then the
-// published finaliser. Used only for the init stream (design notes, "Init").
+// published finaliser. Used only for the init stream (init_params).
 // ---------------------------------------------------------------------------
 uint64_t splitmix64_at(uint64_t x) {
   uint64_t z = x + 0x9E3779B97F4A7C15ull;
