@@ -10,8 +10,9 @@
 //  * Pre-LN block x += Attn(LN1(x)); x += MLP(LN2(x)), 4x tanh-GELU MLP:
 //    "gpt/docs/LLM.md", Transformer Blocks; "GPT From Scratch", Key decisions
 //    (pre-norm, tanh-GELU, 4x); "Genesis", Model Specs (GELU tanh, Pre-LayerNorm).
-//  * Causal multi-head attention, two formulations (explicit masked softmax and
-//    blocked online softmax) that must agree: "GPT From Scratch", Key decisions.
+//  * Causal multi-head attention as the explicit masked softmax; a second, blocked
+//    online-softmax formulation is kept only for the check that the two agree:
+//    "GPT From Scratch", Key decisions.
 //  * Final LN and a bias-free head tied to wte (or a separate head):
 //    "gpt/docs/LLM.md", Output Layer; "AxonLM", Key Features (weight tying);
 //    "Genesis", Model Specs (untied, 163,009,536 parameters).
@@ -395,6 +396,16 @@ void token_buckets(const int32_t* tok, int64_t N, int V, int64_t* counts, int64_
   for (int64_t n = 0; n < N; ++n) positions[cursor[tok[n]]++] = (int32_t)n;
 }
 
+// x0[b*T + t] = wte[tok[b*T + t]] + wpe[t]: the token row plus the row of its
+// position within its own sequence.
+void embedding_fwd(const int32_t* tok, const double* wte, const double* wpe, int B, int T, int C, double* x0) {
+  for (int b = 0; b < B; ++b)
+    for (int t = 0; t < T; ++t) {
+      const int64_t n = (int64_t)b * T + t;
+      for (int i = 0; i < C; ++i) x0[n * C + i] = wte[(int64_t)tok[n] * C + i] + wpe[(int64_t)t * C + i];
+    }
+}
+
 // dwte[v] += sum over positions n with tok[n] == v of dx0[n];  dwpe[t] += sum_b dx0[b, t]
 void embedding_bwd(const int32_t* tok, const double* dx0, int B, int T, int C, double* dwte, double* dwpe) {
   for (int64_t n = 0; n < (int64_t)B * T; ++n) {
@@ -450,10 +461,7 @@ double forward_impl(const Model& M, const double* p, const int32_t* tok, const i
   const double* wte = M.at(p, "wte");
   const double* wpe = M.at(p, "wpe");
   K.x0.assign(N * C, 0.0);
-  for (int64_t n = 0; n < N; ++n) {
-    int t = (int)(n % T);
-    for (int i = 0; i < C; ++i) K.x0[n * C + i] = wte[(int64_t)tok[n] * C + i] + wpe[(int64_t)t * C + i];
-  }
+  embedding_fwd(tok, wte, wpe, B, T, C, K.x0.data());
   std::vector<double> x = K.x0;
   auto L = c.L;
   K.xin.assign(L, {});
@@ -612,6 +620,8 @@ void orc_init_params(const int* cfg, uint64_t seed, float* out) {
 }
 
 // Mean cross-entropy of one batch; logits [B*T, V] written when non-null.
+// attn_mode 0 is the explicit masked softmax (the default of the Python wrapper);
+// mode 1, the blocked online softmax, exists for the equivalence check of the two.
 double orc_forward(const int* cfg, const double* params, const int32_t* tok, const int32_t* tgt, int B, int T,
                    int attn_mode, double* logits) {
   Model M(to_cfg(cfg));
@@ -624,7 +634,8 @@ double orc_forward_backward(const int* cfg, const double* params, const int32_t*
                             int T, double* grads) {
   Model M(to_cfg(cfg));
   Cache K;
-  double loss = forward_impl(M, params, tok, tgt, B, T, 1, K, nullptr, nullptr);
+  // the explicit masked softmax (mode 0): the plain definition of causal attention
+  double loss = forward_impl(M, params, tok, tgt, B, T, 0, K, nullptr, nullptr);
   backward_impl(M, params, tok, tgt, K, grads);
   return loss;
 }
@@ -696,9 +707,9 @@ void orc_token_buckets(const int32_t* tok, int64_t N, int V, int64_t* counts, in
 void orc_embedding_bwd(const int32_t* tok, const double* dx0, int B, int T, int C, double* dwte, double* dwpe) {
   embedding_bwd(tok, dx0, B, T, C, dwte, dwpe);
 }
+// the model's own embedding step (the one forward_impl runs)
 void orc_embedding_fwd(const int32_t* tok, const double* wte, const double* wpe, int B, int T, int C, double* x0) {
-  for (int64_t n = 0; n < (int64_t)B * T; ++n)
-    for (int i = 0; i < C; ++i) x0[n * C + i] = wte[(int64_t)tok[n] * C + i] + wpe[(int64_t)(n % T) * C + i];
+  embedding_fwd(tok, wte, wpe, B, T, C, x0);
 }
 
 }  // extern "C"

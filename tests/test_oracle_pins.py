@@ -226,6 +226,40 @@ def test_token_buckets_are_a_stable_counting_sort():
     assert np.array_equal(pos, np.argsort(flat, kind="stable"))
 
 
+def test_embedding_fwd_is_a_gather_plus_position_rows():
+    # "gpt/docs/LLM.md", Embedding Layer: token embedding plus learned position
+    # embedding; position t is the index within its own sequence. B = 3 and a
+    # position table longer than T make any other position index (n / B, n without
+    # the modulus, a transposed [T, B] order) pick different rows.
+    rng = np.random.default_rng(5)
+    B, T, Tmax, C, V = 3, 7, 11, 6, 23
+    tok, _ = synth.micro_batch(B, T, V, dist="uniform")
+    wte = rng.standard_normal((V, C))
+    wpe = rng.standard_normal((Tmax, C))
+    x0 = oracle.embedding_fwd(tok, wte, wpe)
+    ref = (wte[tok] + wpe[np.arange(T)][None, :, :]).reshape(B * T, C)
+    assert np.array_equal(x0, ref)
+
+
+def test_model_embedding_step_is_the_exported_one():
+    # The model's forward adds position row t to position t of EVERY sequence of the
+    # batch: perturbing wpe row t leaves every earlier position of every sequence
+    # unchanged (causality) and changes position t of every sequence.
+    cfg = oracle.Config(L=1, H=2, C=8, T=6, V=13, tied=1, qkv_bias=1)
+    p = rand_params(cfg, 9)
+    tok, tgt = synth.micro_batch(3, cfg.T, cfg.V, dist="uniform")
+    _, z0 = oracle.forward(cfg, p, tok, tgt, want_logits=True)
+    wpe = next(t for t in oracle.tensors(cfg) if t.name == "wpe")
+    t = 4
+    p2 = p.copy()
+    p2[wpe.offset + t * cfg.C:wpe.offset + (t + 1) * cfg.C] += 0.5
+    _, z1 = oracle.forward(cfg, p2, tok, tgt, want_logits=True)
+    d = np.abs(z1 - z0).reshape(3, cfg.T, cfg.V).max(axis=2)
+    # causal: positions before t unchanged in every sequence; position t changed in every sequence
+    assert np.all(d[:, :t] == 0.0)
+    assert np.all(d[:, t] > 0.0)
+
+
 def test_embedding_bwd_matches_scatter_add():
     rng = np.random.default_rng(6)
     tok, _ = synth.micro_batch(3, 20, 97, dist="zipf")
