@@ -21,7 +21,9 @@
  *    have no handle; their last message is in gpt2_op_last_error().
  *  - Pointers are plain host or device addresses; sizes are element counts. No
  *    call keeps a caller pointer after it returns.
- *  - A handle is not thread-safe: one thread at a time per handle.
+ *  - A handle is not thread-safe: one thread at a time per handle. Handles on
+ *    different devices may be used from one process; kernel attributes are set
+ *    once per device, under a lock.
  *  - All GPU work of a handle is enqueued on its stream (gpt2_set_stream); calls
  *    that return data to host memory synchronise that stream.
  *  - Kernels never trap. Bad token ids are caught on the device (recorded in a
@@ -86,6 +88,14 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out);
 int gpt2_set_stream(gpt2* m, void* stream);
 
 /* Forward + backward of one micro-batch of B sequences of length T (T <= cfg.T).
+ * The forward is the pre-LN stack of "gpt/docs/LLM.md", Architecture Details
+ * (embedding, blocks x += attn(ln_1(x)); x += mlp(ln_2(x)), final LayerNorm, head);
+ * the loss is the mean next-token cross-entropy over all B*T positions ("GPT From
+ * Scratch", Architecture diagram: the train loop and estimate_loss use the model's
+ * loss); gradients are accumulated over micro-batches ("GPT From Scratch", Key
+ * decisions: accumulation equals one large batch; "AxonLM", Key Features: gradient
+ * accumulation set by the total and micro batch sizes, and Training Recipe: an
+ * effective batch of 524,288 tokens).
  * tokens, targets: int32 [B, T], host or device memory (detected), copied in
  * before the call returns. Gradients of the micro-batch's mean cross-entropy
  * are ADDED to the accumulated gradients; the micro-batch count k grows by 1.
@@ -94,10 +104,15 @@ int gpt2_set_stream(gpt2* m, void* stream);
  * given, the call synchronises the stream. */
 int gpt2_forward_backward(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T, float* loss_out);
 
-/* Forward only (no gradients, no change to k). loss_out as above (nullable). */
+/* Forward only (no gradients, no change to k): the same forward and loss as
+ * gpt2_forward_backward, for evaluation ("GPT From Scratch", Architecture diagram:
+ * estimate_loss on held-out batches). loss_out as above (nullable). */
 int gpt2_forward(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T, float* loss_out);
 
-/* Optimizer step on the accumulated gradients: G = (sum of micro-batch
+/* Optimizer step ("AxonLM", Training Recipe: betas (0.9, 0.95), weight decay 0.1
+ * on 2-D tensors only, gradient clip 1.0; "GPT From Scratch", Key decisions: AdamW
+ * decays only parameters of two or more dimensions, clipping at 1.0) on the
+ * accumulated gradients: G = (sum of micro-batch
  * gradients) / k; global-norm clip to 1.0 (coefficient 1 / (||G|| + 1e-6) when
  * below 1); AdamW with eps 1e-8, bias correction, decoupled decay
  * p <- p (1 - lr wd) on >= 2-D tensors only; t += 1; gradients zeroed; k = 0.
@@ -107,6 +122,36 @@ int gpt2_step(gpt2* m, float lr, float wd, float beta1, float beta2, float* grad
 
 /* Zero the accumulated gradients; k = 0. */
 int gpt2_zero_grad(gpt2* m);
+
+/* ------------------------------------------------------------------------
+ * Sharded optimizer step for data parallelism (ZeRO stage 1: each of W ranks keeps
+ * the full parameters, updates only its shard of parameters and optimizer state, and
+ * the ranks exchange the updated shards). It computes exactly gpt2_step's update
+ * ("AxonLM", Key Features: DDP multi-GPU; Training Recipe: clip 1.0, AdamW 0.9 /
+ * 0.95, decay 0.1 on 2-D tensors), split by storage range. Ranges index the library's
+ * flat storage (gpt2_grad_buffer, gpt2_param_buffer), whose length is a multiple of
+ * 4096 floats; lo and hi must be multiples of 64 with 0 <= lo <= hi <= that length
+ * (GPT2_ERR_CONFIG otherwise). Sequence per step: reduce-scatter the gradient buffer,
+ * gpt2_grad_sumsq on the shard, sum the scalars over the ranks, gpt2_step_range on the
+ * shard, all-gather the parameter shards, gpt2_refresh_shadow, gpt2_zero_grad.
+ *
+ * gpt2_grad_sumsq: *dev_out (DEVICE double) = sum over [lo, hi) of g^2, g the
+ * accumulated gradient SUM over the k micro-batches (not divided by k). Asynchronous.
+ * gpt2_step_range: gpt2_step restricted to [lo, hi), with the squared norm of the
+ * whole accumulated gradient read from *dev_sumsq (DEVICE double: the sum of every
+ * shard's gpt2_grad_sumsq): ||G|| = sqrt(sumsq) / k, the same clip, AdamW on [lo, hi)
+ * (decay where the range overlaps the >= 2-D tensors), the bf16 shadow of [lo, hi)
+ * refreshed; t += 1; k = 0. The gradient buffer is left unchanged (zero it with
+ * gpt2_zero_grad). grad_norm_out as in gpt2_step; GPT2_ERR_NO_GRAD when k == 0.
+ * gpt2_param_buffer: device address and length of the flat fp32 parameter storage
+ * (owned by the handle, valid until gpt2_destroy).
+ * gpt2_refresh_shadow: recast the whole bf16 weight shadow from the fp32 parameters
+ * (after the parameter shards were exchanged). Asynchronous. */
+int gpt2_grad_sumsq(gpt2* m, int64_t lo, int64_t hi, double* dev_out);
+int gpt2_step_range(gpt2* m, float lr, float wd, float beta1, float beta2, int64_t lo, int64_t hi,
+                    const double* dev_sumsq, float* grad_norm_out);
+int gpt2_param_buffer(gpt2* m, float** dev, int64_t* n);
+int gpt2_refresh_shadow(gpt2* m);
 
 /* Logical parameter count (V rows, not the padded rows). */
 int gpt2_num_params(const gpt2* m, int64_t* out);
@@ -250,12 +295,14 @@ int gpt2_op_layernorm_bwd(int dtype, const float* f32_dy, const float* f32_x, co
 
 /* Causal attention forward: qkv(act) [B*T, 3*NH*hd] -> out(act) [B*T, NH*hd],
  * f32_lse [B, NH, T] (natural log). bf16 requires hd == 64; fp32 requires hd a
- * multiple of 32, at most 128. */
+ * multiple of 32, at most 128. Synchronises the stream and reports a bounded wait
+ * that gave up as GPT2_ERR_TIMEOUT. */
 int gpt2_op_attention_fwd(int dtype, const void* qkv, int B, int T, int NH, int hd, void* out, float* f32_lse,
                           void* stream);
 
 /* Causal attention backward: dqkv(act) [B*T, 3*NH*hd] from qkv, out, dout(act)
- * and f32_lse. Deterministic (no atomics). */
+ * and f32_lse. Deterministic (no atomics). Synchronises the stream and reports a
+ * bounded wait that gave up as GPT2_ERR_TIMEOUT. */
 int gpt2_op_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* f32_lse, int B,
                           int T, int NH, int hd, void* dqkv, void* stream);
 
@@ -281,9 +328,10 @@ int gpt2_op_embedding_bwd(const int32_t* tokens, const float* f32_dx0, int B, in
                           float* f32_dwpe, void* stream);
 
 /* Cross-entropy over rows of logits(act) [N, ld] (first V columns; bf16 needs
- * ld % 8 == 0 and ld <= 56320, two rows fit in one SM's shared memory):
- * f32_row_loss[n] = logsumexp - z[target]; logits overwritten by
- * (softmax - onehot) * scale (padding columns set to 0). */
+ * ld % 8 == 0): f32_row_loss[n] = logsumexp - z[target]; logits overwritten by
+ * (softmax - onehot) * scale (padding columns set to 0). bf16 runs the training
+ * step's path: per-row softmax partials (here computed from the logits; in the step
+ * the head GEMM's epilogue leaves them), then one streaming pass. Synchronises. */
 int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, const int32_t* targets, float scale,
                           float* f32_row_loss, void* stream);
 
@@ -293,10 +341,13 @@ int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, con
  * or who cannot pay for an allocation per call). Same arguments and results as
  * gpt2_op_attention_bwd. Its scratch (B*NH*T floats) is a fixed device array of
  * 2^20 floats (4 MiB) that every GPU loading the library holds until exit;
- * B*NH*T > 1,048,576 returns GPT2_ERR_CONFIG with a message. The first call on a
- * device looks up the array's address and caches it: make that first call before
- * any stream capture. All calls on a device share the array (each overwrites what
- * it uses before reading it); calls whose kernels overlap on the GPU race. */
+ * B*NH*T > 1,048,576 returns GPT2_ERR_CONFIG with a message. A second fixed word
+ * holds the kernels' error flag: the call clears it, runs the kernels, reads it
+ * back (so the call synchronises the stream) and reports a bounded wait that gave
+ * up as GPT2_ERR_TIMEOUT. The first call on a device looks up both addresses and
+ * caches them: make that first call before any stream capture. All calls on a
+ * device share the array and the word (each overwrites what it uses before reading
+ * it); calls whose kernels overlap on the GPU race. */
 int gpt2_op_attention_bwd_noalloc(int dtype, const void* qkv, const void* out, const void* dout,
                                   const float* f32_lse, int B, int T, int NH, int hd, void* dqkv, void* stream);
 
@@ -318,6 +369,14 @@ int gpt2_op_gemv(const void* x, int64_t ldx, int B, const void* W, int N, int K,
  * arguments, all DEVICE pointers). Synchronises. */
 int gpt2_op_sample_topk(const float* logits, int64_t ld, int rows, int V, int k, float temperature, float top_p,
                         const double* u, int32_t* idx_out, void* stream);
+
+/* Check of the device-side timeout path (no counterpart on the pages: it tests the
+ * library's error reporting). One thread initialises an mbarrier of count 1,
+ * completes it when arrive != 0, then waits for it with the same bounded wait as every
+ * kernel of the library, giving up after limit_ns nanoseconds (at most 1e9). Returns
+ * GPT2_OK when the barrier completed and GPT2_ERR_TIMEOUT when the wait gave up (always
+ * the case for arrive == 0). Nothing else is in flight during the wait. Synchronises. */
+int gpt2_op_bounded_wait_check(int arrive, unsigned long long limit_ns, void* stream);
 
 const char* gpt2_op_last_error(void);
 

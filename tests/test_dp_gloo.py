@@ -150,3 +150,123 @@ def test_trainer_two_rank_gloo_matches_single_process(tmp_path):
     assert np.max(np.abs(p_r[0] - model.p)) < 1e-12
     lrs = np.load(tmp_path / "lr0.npy")
     assert np.allclose(lrs, [oracle.lr_schedule(s, 1e-3, 1e-4, 1, 4) for s in range(3)], rtol=0, atol=1e-18)
+
+
+class _ShardedFlatModel:
+    """Float64 CPU stand-in for the library's sharded-step interface (ZeRO stage 1), to
+    test the host logic of dp.zero1_step: flat storage in canonical order padded to a
+    multiple of 4096, gradients accumulated as a sum over k micro-batches, and the
+    documented range update (norm sqrt(sumsq) / k, clip 1/(norm + 1e-6) capped at 1,
+    AdamW with decay on the >= 2-D tensors)."""
+
+    def __init__(self, seed):
+        import oracle
+        self.oc = oracle.Config(**CFG)
+        p0 = oracle.init_params(self.oc, seed).astype(np.float64)
+        self.P = p0.size
+        n = (self.P + 4095) // 4096 * 4096
+        self.p = np.zeros(n)
+        self.p[:self.P] = p0
+        self.m = np.zeros(n)
+        self.v = np.zeros(n)
+        self.decay = np.zeros(n, dtype=bool)
+        for t in oracle.tensors(self.oc):
+            self.decay[t.offset:t.offset + t.size] = t.decay
+        self.g = torch.zeros(n, dtype=torch.float64)
+        self.k = 0
+        self.t = 0
+
+    def forward_backward(self, tok, tgt):
+        import oracle
+        loss, g = oracle.forward_backward(self.oc, self.p[:self.P], tok, tgt)
+        self.g[:self.P] += torch.from_numpy(g)
+        self.k += 1
+        return loss
+
+    def grad_tensor(self):
+        return self.g
+
+    def param_tensor(self):
+        return torch.from_numpy(self.p)
+
+    def grad_sumsq(self, lo, hi, out):
+        out[0] = float((self.g[lo:hi] ** 2).sum())
+
+    def step_range(self, lr, wd, b1, b2, lo, hi, sumsq):
+        self.t += 1
+        norm = np.sqrt(float(sumsq[0])) / self.k
+        coef = min(1.0, 1.0 / (norm + 1e-6))
+        gg = self.g[lo:hi].numpy() * (coef / self.k)
+        p, m, v, d = self.p[lo:hi], self.m[lo:hi], self.v[lo:hi], self.decay[lo:hi]
+        p[d] *= 1.0 - lr * wd
+        m[:] = b1 * m + (1.0 - b1) * gg
+        v[:] = b2 * v + (1.0 - b2) * gg * gg
+        p -= lr * (m / (1.0 - b1 ** self.t)) / (np.sqrt(v / (1.0 - b2 ** self.t)) + 1e-8)
+        self.k = 0
+
+    def refresh_shadow(self):
+        pass
+
+    def zero_grad(self):
+        self.g.zero_()
+        self.k = 0
+
+
+def _zero1_rank(rank, world, port, out_dir):
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from train_step_b200 import dp, synth
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    model = _ShardedFlatModel(11)
+    for step in range(2):
+        for i in dp.micro_batch_indices(rank, world, ACCUM, step=step):
+            model.forward_backward(*synth.micro_batch(2, CFG["T"], CFG["V"], index=i, dist="uniform"))
+        dp.zero1_step(model, 6e-4, 0.1)
+    np.save(os.path.join(out_dir, f"z{rank}.npy"), model.p[:model.P])
+    np.save(os.path.join(out_dir, f"zm{rank}.npy"), model.m)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_shard_bounds_partition():
+    from train_step_b200 import dp
+    n = 4096 * 3
+    for world in (1, 2, 4, 8, 64):
+        cuts = [dp.shard_bounds(n, world, r) for r in range(world)]
+        assert cuts[0][0] == 0 and cuts[-1][1] == n
+        assert all(a[1] == b[0] for a, b in zip(cuts, cuts[1:]))
+        assert all(lo % 64 == 0 and (hi - lo) == n // world for lo, hi in cuts)
+    with pytest.raises(ValueError):
+        dp.shard_bounds(4096 + 64, 2, 0)
+
+
+def test_zero1_two_rank_gloo_matches_single_process(tmp_path):
+    """Two optimizer steps with the optimizer sharded over two gloo ranks (reduce-scatter,
+    the norm from the shards' sums of squares, AdamW on each rank's half, all-gather)
+    give the parameters of one process taking the full step on all micro-batches, and
+    each rank's moments are non-zero only on its own half."""
+    import oracle
+    from train_step_b200 import dp, synth
+    world = 2
+    mp.start_processes(_zero1_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, start_method="spawn")
+    p_r = [np.load(tmp_path / f"z{r}.npy") for r in range(world)]
+    assert np.array_equal(p_r[0], p_r[1])
+    oc = oracle.Config(**CFG)
+    p = oracle.init_params(oc, 11).astype(np.float64)
+    m = np.zeros_like(p)
+    v = np.zeros_like(p)
+    for step in range(2):
+        idx = [i for r in range(world) for i in dp.micro_batch_indices(r, world, ACCUM, step=step)]
+        g = np.zeros_like(p)
+        for i in idx:
+            g += oracle.forward_backward(oc, p, *synth.micro_batch(2, CFG["T"], CFG["V"], index=i, dist="uniform"))[1]
+        p, m, v, _ = oracle.adamw_step(oc, p, g / len(idx), m, v, step + 1, 6e-4, 0.1)
+    assert np.max(np.abs(p_r[0] - p)) < 1e-12
+    n = np.load(tmp_path / "zm0.npy").size
+    for r in range(world):
+        mr = np.load(tmp_path / f"zm{r}.npy")
+        lo, hi = dp.shard_bounds(n, world, r)
+        assert np.all(mr[:lo] == 0) and np.all(mr[hi:] == 0) and np.any(mr[lo:hi] != 0)

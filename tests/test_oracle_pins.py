@@ -119,14 +119,15 @@ def test_attention_first_row_is_v0():
     rng = np.random.default_rng(1)
     B, T, NH, hd = 1, 9, 2, 8
     qkv = rng.standard_normal((B * T, 3 * NH * hd))
-    o, lse = oracle.attention_fwd(qkv, B, T, NH, hd, mode=1)
     C = NH * hd
-    assert np.array_equal(o[0], qkv[0, 2 * C:3 * C])
-    # lse of row 0 is the single scaled score
-    for h in range(NH):
-        q = qkv[0, h * hd:(h + 1) * hd]
-        k = qkv[0, C + h * hd:C + (h + 1) * hd]
-        assert abs(lse[0, h, 0] - q @ k / math.sqrt(hd)) < 1e-14
+    for mode in (0, 1):
+        o, lse = oracle.attention_fwd(qkv, B, T, NH, hd, mode=mode)
+        assert np.array_equal(o[0], qkv[0, 2 * C:3 * C])
+        # lse of row 0 is the single scaled score
+        for h in range(NH):
+            q = qkv[0, h * hd:(h + 1) * hd]
+            k = qkv[0, C + h * hd:C + (h + 1) * hd]
+            assert abs(lse[0, h, 0] - q @ k / math.sqrt(hd)) < 1e-14
 
 
 def test_attention_matches_torch_sdpa():

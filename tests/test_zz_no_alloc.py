@@ -5,19 +5,12 @@ fixed budget owns it all); this entry point keeps its scratch in a fixed device
 array instead. It must give the same gradients as gpt2_op_attention_bwd, call
 after call, through the C ABI. This file is collected last on purpose.
 """
-import numpy as np
 import pytest
 import torch
 
 import train_step_b200 as tsb
 
 pytestmark = pytest.mark.gpu
-
-
-def rel_l2(a, b):
-    a = a.double().cpu().numpy()
-    b = b.double().cpu().numpy()
-    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
 
 
 def _inputs(B, T, NH, hd, dtype, seed):
@@ -31,8 +24,10 @@ def _inputs(B, T, NH, hd, dtype, seed):
     return qkv, out, dout, lse
 
 
-@pytest.mark.parametrize("dtype,hd,tol", [(torch.bfloat16, 64, 2e-2), (torch.float32, 32, 1e-5)])
-def test_noalloc_matches_allocating_entry_point_twice(dtype, hd, tol):
+@pytest.mark.parametrize("dtype,hd", [(torch.bfloat16, 64), (torch.float32, 32)])
+def test_noalloc_matches_allocating_entry_point_twice(dtype, hd):
+    # The two entry points run the same deterministic kernels on the same inputs, so
+    # the gradients must be bitwise equal; any stale or aliased scratch would show.
     for call, (B, T, NH) in enumerate([(2, 200, 3), (1, 96, 2)]):  # two calls in a row, new shapes
         qkv, out, dout, lse = _inputs(B, T, NH, hd, dtype, seed=10 + call)
         ref = torch.zeros_like(qkv)
@@ -41,7 +36,20 @@ def test_noalloc_matches_allocating_entry_point_twice(dtype, hd, tol):
         tsb.attention_bwd_noalloc(qkv, out, dout, lse, got, B, T, NH, hd)
         torch.cuda.synchronize()
         assert torch.isfinite(got.float()).all()
-        assert rel_l2(got, ref) <= tol
+        assert torch.equal(got, ref)
+
+
+def test_noalloc_at_the_full_scratch_size():
+    # B*NH*T == 2^20 rows: exactly the fixed scratch array.
+    B, T, NH, hd = 16, 1024, 64, 64
+    assert B * NH * T == 1 << 20
+    qkv, out, dout, lse = _inputs(B, T, NH, hd, torch.bfloat16, seed=21)
+    ref = torch.zeros_like(qkv)
+    tsb.attention_bwd(qkv, out, dout, lse, ref, B, T, NH, hd)
+    got = torch.full_like(qkv, float("nan"))
+    tsb.attention_bwd_noalloc(qkv, out, dout, lse, got, B, T, NH, hd)
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():

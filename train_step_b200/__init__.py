@@ -94,6 +94,12 @@ _SYMBOLS = {
                       ct.POINTER(ct.c_float), ct.c_void_p], ct.c_int),
     "gpt2_op_sample_topk": ([ct.c_void_p, ct.c_int64, ct.c_int, ct.c_int, ct.c_int, ct.c_float, ct.c_float,
                              ct.c_void_p, ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_bounded_wait_check": ([ct.c_int, ct.c_ulonglong, ct.c_void_p], ct.c_int),
+    "gpt2_grad_sumsq": ([ct.c_void_p, ct.c_int64, ct.c_int64, ct.c_void_p], ct.c_int),
+    "gpt2_step_range": ([ct.c_void_p, ct.c_float, ct.c_float, ct.c_float, ct.c_float, ct.c_int64, ct.c_int64,
+                         ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_param_buffer": ([ct.c_void_p, ct.POINTER(ct.c_void_p), ct.POINTER(ct.c_int64)], ct.c_int),
+    "gpt2_refresh_shadow": ([ct.c_void_p], ct.c_int),
     "gpt2_op_last_error": ([], ct.c_char_p),
 }
 
@@ -262,19 +268,50 @@ class GPT2:
         self._check(lib().gpt2_grad_buffer(self.h, ct.byref(p), ct.byref(n)))
         return p.value, n.value
 
-    def grad_tensor(self):
-        """Zero-copy fp32 CUDA tensor over the flat gradient storage (the library's padded
-        layout), e.g. for a data-parallel all-reduce between micro-batch accumulation and
-        the optimizer step."""
+    @staticmethod
+    def _device_view(ptr: int, n: int):
         import torch
 
         class _View:
             pass
 
-        ptr, n = self.grad_buffer()
         v = _View()
         v.__cuda_array_interface__ = {"shape": (n,), "typestr": "<f4", "data": (ptr, False), "version": 3}
         return torch.as_tensor(v, device="cuda")
+
+    def grad_tensor(self):
+        """Zero-copy fp32 CUDA tensor over the flat gradient storage (the library's padded
+        layout), e.g. for a data-parallel all-reduce between micro-batch accumulation and
+        the optimizer step."""
+        return self._device_view(*self.grad_buffer())
+
+    def param_buffer(self):
+        """(device address, length in floats) of the flat fp32 parameter storage."""
+        p = ct.c_void_p()
+        n = ct.c_int64()
+        self._check(lib().gpt2_param_buffer(self.h, ct.byref(p), ct.byref(n)))
+        return p.value, n.value
+
+    def param_tensor(self):
+        """Zero-copy fp32 CUDA tensor over the flat parameter storage (padded layout)."""
+        return self._device_view(*self.param_buffer())
+
+    def grad_sumsq(self, lo: int, hi: int, out) -> None:
+        """out (a CUDA float64 tensor of one element) = sum of squares of the accumulated
+        gradient sum over storage [lo, hi); asynchronous."""
+        self._check(lib().gpt2_grad_sumsq(self.h, int(lo), int(hi), _ptr(out)))
+
+    def step_range(self, lr: float, wd: float, beta1: float, beta2: float, lo: int, hi: int, sumsq,
+                   want_norm: bool = False):
+        """The optimizer step on storage [lo, hi) with the whole gradient's squared norm in
+        sumsq (a CUDA float64 tensor of one element); returns the pre-clip norm if asked."""
+        n = ct.c_float()
+        self._check(lib().gpt2_step_range(self.h, lr, wd, beta1, beta2, int(lo), int(hi), _ptr(sumsq),
+                                          ct.byref(n) if want_norm else None))
+        return n.value if want_norm else None
+
+    def refresh_shadow(self) -> None:
+        self._check(lib().gpt2_refresh_shadow(self.h))
 
     def profile(self, enable: bool) -> None:
         self._check(lib().gpt2_profile(self.h, int(enable)))
@@ -479,3 +516,9 @@ def cross_entropy(logits, V, targets, scale, row_loss, stream=None):
     N, ld = logits.shape
     _op(lib().gpt2_op_cross_entropy(_dt(logits), _ptr(logits), ld, N, V, _ptr(targets), scale, _ptr(row_loss),
                                     _stream(stream)))
+
+
+def bounded_wait_check(arrive: bool, limit_ns: int, stream=None) -> None:
+    """The library's bounded device-side wait on a barrier that is completed (arrive) or
+    never completed; raises Gpt2Error(GPT2_ERR_TIMEOUT) when the wait gives up."""
+    _op(lib().gpt2_op_bounded_wait_check(int(arrive), int(limit_ns), _stream(stream)))

@@ -52,13 +52,18 @@ struct AdamArgs {
   float step_size;     // lr / (1 - b1^t)
   float inv_sqrt_bc2;  // 1 / sqrt(1 - b2^t)
   float* gnorm_out;    // device scalar: pre-clip ||G||
+  const double* sumsq_total;  // nullable: the global sum of raw squared gradients, in place of the partials
+  int zero_grad;              // zero the gradients that were read
 };
 
 __global__ void __launch_bounds__(ADAM_THREADS) adamw_kernel(const AdamArgs a) {
   __shared__ float s_coef;
   if (threadIdx.x == 0) {
     double ss = 0.0;
-    for (int i = 0; i < a.nparts; ++i) ss += a.partial[i];
+    if (a.sumsq_total)
+      ss = *a.sumsq_total;
+    else
+      for (int i = 0; i < a.nparts; ++i) ss += a.partial[i];
     const double norm = sqrt(ss) * (double)a.inv_k;
     double coef = 1.0 / (norm + 1e-6);
     if (coef > 1.0) coef = 1.0;
@@ -92,9 +97,18 @@ __global__ void __launch_bounds__(ADAM_THREADS) adamw_kernel(const AdamArgs a) {
     *reinterpret_cast<float4*>(a.p + e) = p;
     *reinterpret_cast<float4*>(a.m + e) = m;
     *reinterpret_cast<float4*>(a.v + e) = v;
-    *reinterpret_cast<float4*>(a.g + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (a.zero_grad) *reinterpret_cast<float4*>(a.g + e) = make_float4(0.f, 0.f, 0.f, 0.f);
     if (a.shadow && dec)
       *reinterpret_cast<uint2*>(a.shadow + e) = make_uint2(pack_bf16x2(p.x, p.y), pack_bf16x2(p.z, p.w));
+  }
+}
+
+// out[0] = sum of the partials in index order (the sum of squares of a storage range).
+__global__ void sum_partials_kernel(const double* __restrict__ partial, int nparts, double* __restrict__ out) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    double s = 0.0;
+    for (int i = 0; i < nparts; ++i) s += partial[i];
+    out[0] = s;
   }
 }
 

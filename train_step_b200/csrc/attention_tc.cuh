@@ -30,75 +30,64 @@ constexpr int FA_BN = 128;  // keys per block
 constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 
 // ---------------------------------------------------------------------------
-// Backward on tcgen05. Two deterministic kernels (no atomics). Both are
-// persistent (one CTA per SM looping over work items, so an item's loads overlap
-// the previous item's tail) and work in 64-wide units:
+// Backward on tcgen05. Two deterministic kernels (no atomics), both persistent (one
+// CTA per SM looping over work items, longest first, dealt to the CTAs in a zigzag so
+// that the causal lengths even out), in 128 x 128 units:
 //
-//   dK/dV: item = (128-key block kb, batch*head); units = 64-query halves of the
-//     query blocks kb .. nqb-1, in key-row orientation:
-//       S^T = K Q_u^T, dP^T = V dO_u^T                 (M=128 keys, N=64 queries, K=64)
+//   dK/dV: item = (128-key block kb, batch*head); units = the query blocks kb .. nqb-1,
+//     in key-row orientation:
+//       S^T = K Q_i^T, dP^T = V dO_i^T        (M=128 keys, N=128 queries, K=64;
+//                                              A = K / V and B = Q_i / dO_i from shared memory)
 //       P^T = 2^(S^T*scale*log2e - lse*log2e), dS^T = P^T (dP^T - D)   (element-wise)
-//       dV += P^T dO_u, dK += dS^T Q_u                 (M=128 keys, N=64, K=64 queries)
+//       dV += P^T dO_i, dK += dS^T Q_i        (M=128 keys, N=64, K=128 queries; A = P^T /
+//                                              dS^T in TMEM, B = dO_i / Q_i MN-major)
 //     lse*log2e and D of a unit's queries are staged in shared memory by the producer warp.
-//   dQ: item = (128-query block qb, batch*head); units = 64-key halves of the key
-//     blocks 0 .. qb, in query-row orientation (lse and D are registers):
-//       S = Q K_u^T, dP = dO V_u^T                     (M=128 queries, N=64 keys, K=64)
-//       dQ += dS K_u                                   (M=128 queries, N=64, K=64 keys)
+//   dQ: item = (128-query block qb, batch*head); units = the key blocks 0 .. qb, in
+//     query-row orientation (lse and D of the thread's row are registers):
+//       S = Q K_j^T, dP = dO V_j^T            (M=128 queries, N=128 keys, K=64; A = Q / dO
+//                                              copied into TMEM once per item)
+//       dQ += dS K_j                          (M=128 queries, N=64, K=128 keys; A = dS in TMEM)
 //
-// Operands. With both MMA operands in shared memory these small products are
-// bound by shared-memory bandwidth (a 128 x 64 x 16 MMA re-reads a 4 KB A tile
-// for 2 KB of B). So every A operand lives in TMEM: the item's fixed 128-row tiles
-// (Q and dO, or K and V) are copied there once per item by the element-wise warps,
-// which also write P^T / dS^T (dS) there directly; only the 64-row B tiles of each
-// unit are read from shared memory.
-// Pipelining. Every unit streams its own 16 KB stage (two 64-row tiles) through a
-// 7- or 8-deep ring, released as soon as that unit's accumulation MMAs complete,
-// so a stage's copy is issued several units before it is needed (tile loads take
-// 1-3 us under load). The score tiles are double-buffered in TMEM.
-// MMA issue. One thread can issue a 1-SM tcgen05.mma only every ~96 cycles whatever
-// its N (measured on B200), while the tensor pipe overlaps the streams of several
-// threads. So each product has its own issuing thread (lane 0 of its own warp):
-// dK/dV: S^T, dP^T, dV, dK; dQ: S, dP, dQ. The score threads never wait behind the
-// accumulation threads, which wait for the element-wise warps.
-// Warps: 0 TMA producer (lane 0 issues the copies), then the MMA warps (warp 1 owns
-// the TMEM allocation), then 16 element-wise warps: warp w reads TMEM lane quarter
-// w % 4 (32 rows) and column group (w - first) / 4 (16 of the 64 unit columns).
-// D = rowsum(dO * O) comes precomputed. Every wait is bounded (device error word,
-// no trap).
+// TMEM (512 columns). dK/dV: S^T | dP^T (128 + 128), P^T | dS^T (64 + 64, bf16 pairs),
+// dV | dK (64 + 64). dQ: S | dP (128 + 128), Q | dO operands (32 + 32), dS (64), dQ for two
+// items (64 + 64). The score tiles are single-buffered: the element-wise warps load them
+// into registers first thing, and the next unit's score products run while they compute.
+// MMA issue: the two score products of a unit come from one thread, and each
+// accumulation product from a thread of its own (lane 0 of its warp).
+// Warps: 0 TMA producer, then the MMA issuers, then 16 element-wise warps: warp w reads
+// TMEM lane quarter w % 4 (32 rows) and column group (w - first) / 4 (32 of the 128
+// unit columns). D = rowsum(dO * O) comes precomputed. Every wait is bounded (device
+// error word, early exit, no trap).
 // ---------------------------------------------------------------------------
 constexpr int FB_EW_WARPS = 16;
-constexpr int FBK_EW0 = 5;  // dK/dV: producer, S^T, dP^T, dV, dK issuers, then element-wise warps
-constexpr int FBQ_EW0 = 4;  // dQ: producer, S, dP, dQ issuers, then element-wise warps
-constexpr int FBK_THREADS = 32 * (FBK_EW0 + FB_EW_WARPS);  // 672
-constexpr int FBQ_THREADS = 32 * (FBQ_EW0 + FB_EW_WARPS);  // 640
-constexpr int FB_HALF = 64 * 128;                  // 8 KB: 64 rows x 64 bf16 (128-byte rows)
-constexpr int FB_UNIT = 2 * FB_HALF;               // 16 KB: a stage (two half tiles) or a 128 x 64 tile
 constexpr int FB_BARS = 512;
-// dK/dV kernel shared memory: K/V [2 items] | stages (Q_u, dO_u) | lse/D per stage |
-// output staging (dK, dV tiles for one TMA store each) | barriers
-constexpr int FBK_NST = 6;
-constexpr int FBK_OFF_KV = 0;
-constexpr int FBK_OFF_ST = 4 * FA_TILE;
-constexpr int FBK_OFF_LD = FBK_OFF_ST + FBK_NST * FB_UNIT;
-constexpr int FBK_OFF_OUT = FBK_OFF_LD + 4096;  // FBK_NST x 512 bytes, rounded up
-constexpr int FBK_OFF_BAR = FBK_OFF_OUT + 2 * FA_TILE;
-constexpr int FBK_SMEM = FBK_OFF_BAR + FB_BARS + 1024;
-// dQ kernel shared memory: Q/dO [2 items] | stages (K_u, V_u) | output staging (dQ) | barriers
-constexpr int FBQ_NST = 8;
-constexpr int FBQ_OFF_QD = 0;
-constexpr int FBQ_OFF_ST = 4 * FA_TILE;
-constexpr int FBQ_OFF_OUT = FBQ_OFF_ST + FBQ_NST * FB_UNIT;
-constexpr int FBQ_OFF_BAR = FBQ_OFF_OUT + FA_TILE;
-constexpr int FBQ_SMEM = FBQ_OFF_BAR + FB_BARS + 1024;
-static_assert(FBK_NST * 512 <= 4096, "lse/D staging");
-static_assert(FBQ_SMEM <= 232448 && FBK_SMEM <= 232448, "shared memory per CTA");
-// TMEM columns (512): score tiles [2 units] x (S 64 | dP 64) at 0 and 128, then
-//   dK/dV: K | V A operands (32 + 32) at 256, P^T at 320, dS^T at 352 (32 each), dV | dK at 384
-//   dQ:    Q | dO A operands (32 + 32) at 256, dS [2 units] at 320 (32 each), dQ [2 items] at 384
-constexpr int FB_SBUF = 2;
-constexpr uint32_t FBK_TM_KV = 256, FBK_TM_P = 320, FBK_TM_DS = 352, FBK_TM_ACC = 384;
-constexpr uint32_t FBQ_TM_Q = 256, FBQ_TM_DS = 320, FBQ_TM_ACC = 384;
+constexpr int FB_STAGE = 2 * FA_TILE;  // two 128-row tiles: 32 KB
 constexpr uint32_t FB_TMEM_COLS = 512;
+// dK/dV kernel
+constexpr int BK_EW0 = 4;  // producer, score (S^T and dP^T), dV, dK issuers, then element-wise warps
+constexpr int BK_THREADS = 32 * (BK_EW0 + FB_EW_WARPS);  // 640
+constexpr int BK_NST = 3;
+constexpr int BK_OFF_KV = 0;                            // K | V [2 items]
+constexpr int BK_OFF_ST = 4 * FA_TILE;                  // stages: Q_i | dO_i
+constexpr int BK_OFF_LD = BK_OFF_ST + BK_NST * FB_STAGE;  // per stage: lse*log2e [128] | D [128]
+constexpr int BK_OFF_OUT = BK_OFF_LD + BK_NST * 1024;   // dK | dV staging for the TMA stores
+constexpr int BK_OFF_BAR = BK_OFF_OUT + 2 * FA_TILE;
+constexpr int BK_SMEM = BK_OFF_BAR + FB_BARS + 1024;
+constexpr uint32_t BK_TM_DP = 128, BK_TM_P = 256, BK_TM_DS = 320, BK_TM_DV = 384, BK_TM_DK = 448;
+// dQ kernel
+constexpr int BQ_EW0 = 3;  // producer, score (S and dP), dQ issuers, then element-wise warps
+constexpr int BQ_THREADS = 32 * (BQ_EW0 + FB_EW_WARPS);  // 608
+constexpr int BQ_NST = 4;
+constexpr int BQ_OFF_QD = 0;                            // Q | dO [2 items]
+constexpr int BQ_OFF_ST = 4 * FA_TILE;                  // stages: K_j | V_j
+constexpr int BQ_OFF_OUT = BQ_OFF_ST + BQ_NST * FB_STAGE;
+constexpr int BQ_OFF_BAR = BQ_OFF_OUT + FA_TILE;
+constexpr int BQ_SMEM = BQ_OFF_BAR + FB_BARS + 1024;
+constexpr uint32_t BQ_TM_DP = 128, BQ_TM_Q = 256, BQ_TM_DS = 320, BQ_TM_ACC = 384;
+static_assert(BK_SMEM <= 232448 && BQ_SMEM <= 232448, "shared memory per CTA");
+
+// Item of CTA `cta` in round k over G CTAs: zigzag over the longest-first order.
+__device__ __forceinline__ int fx_item(int k, int cta, int G) { return k * G + ((k & 1) ? (G - 1 - cta) : cta); }
 
 // 16 bf16 values (two 16-byte chunks, chunk index c16 and c16 + 1 of a 64-column row)
 // into row r of a 128-byte-swizzled tile with 128-byte rows.
@@ -134,6 +123,24 @@ __device__ __forceinline__ bool fb_warp_wait(uint64_t* bar, uint32_t parity, vol
   return ok != 0;
 }
 
+// Column sums over the warp's 32 rows of 16 columns held one row per lane: afterwards
+// lane j < 16 holds the sum of column j (a fixed summation order, the same every run).
+__device__ __forceinline__ float warp_colsum16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] += __shfl_xor_sync(0xffffffffu, v[j], 16);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int j = 0; j < w; ++j) {
+      const float send = upper ? v[j] : v[j + w];
+      const float keep = upper ? v[j + w] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
+}
+
 // Copy 16 bf16 (columns [cg*16, cg*16 + 16)) of row r of a 128-byte-swizzled tile
 // with 128-byte rows into 8 TMEM columns of the thread's lane, as an MMA A operand.
 __device__ __forceinline__ void fb_row_to_tmem(const uint8_t* tile, int r, int cg, uint32_t taddr) {
@@ -151,58 +158,55 @@ __device__ __forceinline__ void fb_vals_to_tmem(const float (&v)[16], uint32_t t
 }
 
 
-__global__ void __launch_bounds__(FBK_THREADS, 1)
-    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_q64,
-                            const __grid_constant__ CUtensorMap tm_do64, const __grid_constant__ CUtensorMap tm_out,
-                            const float* __restrict__ lse, const float* __restrict__ Dg, int T, int NH, int BH,
+__global__ void __launch_bounds__(BK_THREADS, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
+                            const __grid_constant__ CUtensorMap tm_out, const float* __restrict__ lse,
+                            const float* __restrict__ Dg, float* __restrict__ colsum, int T, int NH, int BH,
                             float scale, int* err, unsigned long long timeout_ns) {
   extern __shared__ uint8_t fb_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FBK_OFF_BAR);
-  uint64_t* kv_full = bar;                    // [2] K/V tiles landed in shared memory
-  uint64_t* kv_empty = kv_full + 2;           // [2] copied into TMEM by the element-wise warps
-  uint64_t* kva_full = kv_empty + 2;          // K/V A operands written to TMEM (once per item)
-  uint64_t* st_full = kva_full + 1;           // [FBK_NST]
-  uint64_t* st_empty = st_full + FBK_NST;     // [FBK_NST]
-  uint64_t* s_full = st_empty + FBK_NST;      // [FB_SBUF]
-  uint64_t* s_empty = s_full + FB_SBUF;       // [FB_SBUF]
-  uint64_t* p_full = s_empty + FB_SBUF;
-  uint64_t* p_free = p_full + 1;
-  uint64_t* acc_full = p_free + 1;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* out_full = acc_empty + 1;         // output tiles staged (element-wise warps)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BK_OFF_BAR);
+  uint64_t* kv_full = bar;                    // [2] K / V tiles landed
+  uint64_t* kv_empty = kv_full + 2;           // [2] the item's S^T / dP^T products are complete
+  uint64_t* st_full = kv_empty + 2;           // [BK_NST] Q_i / dO_i landed, lse / D staged (32 producer lanes)
+  uint64_t* st_empty = st_full + BK_NST;      // [BK_NST] the unit's dV and dK products are complete
+  uint64_t* s_full = st_empty + BK_NST;       // S^T and dP^T complete
+  uint64_t* s_empty = s_full + 1;             // both read into registers (16 warps)
+  uint64_t* p_full = s_empty + 1;             // P^T and dS^T written (16 warps)
+  uint64_t* p_free = p_full + 1;              // the dV and dK products have read them (2 commits)
+  uint64_t* acc_full = p_free + 1;            // the item's dV and dK complete (2 commits)
+  uint64_t* acc_empty = acc_full + 1;         // dV and dK read by the epilogue (16 warps)
+  uint64_t* out_full = acc_empty + 1;         // output tiles staged (16 warps)
   uint64_t* out_free = out_full + 1;          // the previous item's TMA stores have read the staging
-  uint64_t* drain = out_free + 1;             // [4]: one per MMA thread (abort path)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 5);
+  uint64_t* drain = out_free + 1;             // [3]: one per MMA thread (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = NH * 64;
   const int nqb = (T + FA_BM - 1) / FA_BM;
-  const int nitems = nqb * BH;  // item = kb * BH + bh: the longest rows (kb = 0) come first
+  const int nitems = nqb * BH;  // item w: key block w / BH (the longest rows first), bh = w % BH
+  const int G = gridDim.x, cta = blockIdx.x;
   const uint64_t lim = timeout_ns;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], FB_EW_WARPS);
+      mbar_init(&kv_empty[i], 1);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&drain[i], 1);
-    mbar_init(kva_full, FB_EW_WARPS);
-    for (int i = 0; i < FBK_NST; ++i) {
-      mbar_init(&st_full[i], 32);  // the producer warp's lanes (lane 0 with the copy bytes)
-      mbar_init(&st_empty[i], 2);  // the dV and dK threads
+    for (int i = 0; i < BK_NST; ++i) {
+      mbar_init(&st_full[i], 32);
+      mbar_init(&st_empty[i], 2);
     }
-    for (int i = 0; i < FB_SBUF; ++i) {
-      mbar_init(&s_full[i], 2);  // the S^T and dP^T threads
-      mbar_init(&s_empty[i], FB_EW_WARPS);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, FB_EW_WARPS);
     mbar_init(p_full, FB_EW_WARPS);
-    mbar_init(p_free, 2);  // the dV and dK threads
+    mbar_init(p_free, 2);
     mbar_init(acc_full, 2);
     mbar_init(acc_empty, FB_EW_WARPS);
     mbar_init(out_full, FB_EW_WARPS);
     mbar_init(out_free, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&drain[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -216,45 +220,46 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- producer: K/V per item; (Q_u, dO_u, lse, D) per unit ----------------
+    // ---------------- producer: K/V per item; (Q_i, dO_i, lse, D) per unit ----------------
     if (lane == 0) {
-      tma_prefetch_desc(&tm_kv);
-      tma_prefetch_desc(&tm_q64);
-      tma_prefetch_desc(&tm_do64);
+      tma_prefetch_desc(&tm_qkv);
+      tma_prefetch_desc(&tm_do);
     }
     bool ok = true;
     uint32_t kv_iss = 0, kv_par = 0, st_iss = 0, st_par = 0;  // lane 0: copies in flight, for the abort path
-    int U = 0;                                                 // unit (= stage use) counter over all items
-    for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+    int U = 0;
+    for (int k = 0; ok; ++k) {
+      const int item = fx_item(k, cta, G);
+      if (item >= nitems) break;
       const int kb = item / BH, bh = item - kb * BH, b = bh / NH, h = bh - b * NH;
-      const int kvb = it & 1;
-      if (!(ok = fb_warp_wait(&kv_empty[kvb], ((it >> 1) & 1) ^ 1, abort_flag, lim, lane))) break;
+      const int kvb = k & 1;
+      if (!(ok = fb_warp_wait(&kv_empty[kvb], ((k >> 1) & 1) ^ 1, abort_flag, lim, lane))) break;
       if (lane == 0) {
-        uint8_t* kd = sm + FBK_OFF_KV + kvb * 2 * FA_TILE;
+        uint8_t* kd = sm + BK_OFF_KV + kvb * 2 * FA_TILE;
         mbar_arrive_expect_tx(&kv_full[kvb], 2 * FA_TILE);
-        tma_load_3d(kd, &tm_kv, &kv_full[kvb], C + h * 64, kb * FA_BN, b);
-        tma_load_3d(kd + FA_TILE, &tm_kv, &kv_full[kvb], 2 * C + h * 64, kb * FA_BN, b);
+        tma_load_3d(kd, &tm_qkv, &kv_full[kvb], C + h * 64, kb * FA_BN, b);
+        tma_load_3d(kd + FA_TILE, &tm_qkv, &kv_full[kvb], 2 * C + h * 64, kb * FA_BN, b);
         kv_iss |= 1u << kvb;
-        kv_par = (kv_par & ~(1u << kvb)) | ((uint32_t)((it >> 1) & 1) << kvb);
+        kv_par = (kv_par & ~(1u << kvb)) | ((uint32_t)((k >> 1) & 1) << kvb);
       }
       const float* lse_bh = lse + (long long)bh * T;
       const float* D_bh = Dg + (long long)bh * T;
-      for (int q0 = kb * FA_BM; q0 < nqb * FA_BM; q0 += 64, ++U) {
-        const int s = U % FBK_NST;
-        const uint32_t ph = (uint32_t)((U / FBK_NST) & 1);
+      for (int i = kb; i < nqb; ++i, ++U) {
+        const int s = U % BK_NST;
+        const uint32_t ph = (uint32_t)((U / BK_NST) & 1);
         if (!(ok = fb_warp_wait(&st_empty[s], ph ^ 1, abort_flag, lim, lane))) break;
-        float* ld = reinterpret_cast<float*>(sm + FBK_OFF_LD + s * 512);  // [lse*log2e 64][D 64]
+        float* ld = reinterpret_cast<float*>(sm + BK_OFF_LD + s * 1024);  // [lse*log2e 128][D 128]
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int c = lane * 2 + k, q = q0 + c;
+        for (int e = 0; e < 4; ++e) {
+          const int c = lane * 4 + e, q = i * FA_BM + c;
           ld[c] = q < T ? lse_bh[q] * LOG2E : INFINITY;  // P = 0 for queries past the end
-          ld[64 + c] = q < T ? D_bh[q] : 0.f;
+          ld[128 + c] = q < T ? D_bh[q] : 0.f;
         }
         if (lane == 0) {
-          uint8_t* d = sm + FBK_OFF_ST + s * FB_UNIT;
-          mbar_arrive_expect_tx(&st_full[s], FB_UNIT);
-          tma_load_3d(d, &tm_q64, &st_full[s], h * 64, q0, b);
-          tma_load_3d(d + FB_HALF, &tm_do64, &st_full[s], h * 64, q0, b);
+          uint8_t* d = sm + BK_OFF_ST + s * FB_STAGE;
+          mbar_arrive_expect_tx(&st_full[s], FB_STAGE);
+          tma_load_3d(d, &tm_qkv, &st_full[s], h * 64, i * FA_BM, b);
+          tma_load_3d(d + FA_TILE, &tm_do, &st_full[s], h * 64, i * FA_BM, b);
           st_iss |= 1u << s;
           st_par = (st_par & ~(1u << s)) | (ph << s);
         } else {
@@ -269,87 +274,92 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
       for (int i = 0; i < 2; ++i)
         if ((kv_iss >> i) & 1u)
           mbar_wait_bounded(&kv_full[i], (kv_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
-      for (int i = 0; i < FBK_NST; ++i)
+      for (int i = 0; i < BK_NST; ++i)
         if ((st_iss >> i) & 1u)
           mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
     }
-  } else if (warp == 1 || warp == 2) {
+  } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- score MMAs: S^T = K Q_u^T (warp 1), dP^T = V dO_u^T (warp 2); A from TMEM ----------------
-      const int part = warp - 1;
-      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64, false, false);
+      // ---------------- score MMAs: S^T = K Q_i^T, then dP^T = V dO_i^T ----------------
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
       bool ok = true, any = false;
       int U = 0;
-      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
-        const int nu = 2 * (nqb - item / BH);
-        if (!mbar_wait_bounded(kva_full, it & 1, abort_flag, lim)) {
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
+        const int nu = nqb - item / BH, kvb = k & 1;
+        if (!mbar_wait_bounded(&kv_full[kvb], (k >> 1) & 1, abort_flag, lim)) {
           ok = false;
           break;
         }
+        const uint32_t kv_addr = smem_u32(sm + BK_OFF_KV + kvb * 2 * FA_TILE);
         for (int u = 0; u < nu; ++u, ++U) {
-          const int s = U % FBK_NST, sb = U % FB_SBUF;
-          if (!mbar_wait_bounded(&st_full[s], (U / FBK_NST) & 1, abort_flag, lim) ||
-              !mbar_wait_bounded(&s_empty[sb], ((U / FB_SBUF) & 1) ^ 1, abort_flag, lim)) {
+          const int s = U % BK_NST;
+          if (!mbar_wait_bounded(&st_full[s], (U / BK_NST) & 1, abort_flag, lim) ||
+              !mbar_wait_bounded(s_empty, (U & 1) ^ 1, abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // B = Q_u (part 0) or dO_u (part 1): 64 rows, K-major
-          const uint32_t b_addr = smem_u32(sm + FBK_OFF_ST + s * FB_UNIT) + part * FB_HALF;
-          const uint32_t d = tmem + (uint32_t)(sb * 128 + part * 64);
+          const uint32_t st_addr = smem_u32(sm + BK_OFF_ST + s * FB_STAGE);
+          // part 0: A = K, B = Q_i -> S^T; part 1: A = V, B = dO_i -> dP^T
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16_ts(d, tmem + FBK_TM_KV + part * 32 + k * 8, make_sw128_desc(b_addr + k * 32, 16, 1024), idesc_s,
-                         k > 0 ? 1u : 0u);
-          umma_commit(&s_full[sb]);
+          for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(tmem + part * BK_TM_DP, make_sw128_desc(kv_addr + part * FA_TILE + kk * 32, 16, 1024),
+                        make_sw128_desc(st_addr + part * FA_TILE + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          umma_commit(s_full);
           any = true;
         }
+        if (ok) umma_commit(&kv_empty[kvb]);  // the item's K / V tile is no longer read
       }
       if (!ok) {
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
         if (any) {  // wait for the MMAs already issued before the TMEM is freed
           int never = 0;
-          umma_commit(&drain[part]);
-          mbar_wait_bounded(&drain[part], 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[0]);
+          mbar_wait_bounded(&drain[0], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
-  } else if (warp == 3 || warp == 4) {
+  } else if (warp == 2 || warp == 3) {
     if (lane == 0) {
-      // ---------------- accumulation MMAs: dV += P^T dO_u (warp 3), dK += dS^T Q_u (warp 4); A from TMEM ----------------
-      const int part = warp - 3;
-      constexpr uint32_t idesc_a = make_idesc_bf16(128, 64, false, true);  // B = dO_u / Q_u, MN-major
+      // ---------------- accumulation MMAs: dV += P^T dO_i (warp 2), dK += dS^T Q_i (warp 3) ----------------
+      const int part = warp - 2;
+      constexpr uint32_t idesc_a = make_idesc_bf16(128, 64, false, true);  // B = dO_i / Q_i, MN-major
       bool ok = true, any = false;
       int U = 0;
-      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
-        const int nu = 2 * (nqb - item / BH);
-        // the element-wise warps have read the previous item's dV / dK
-        if (!mbar_wait_bounded(acc_empty, (it & 1) ^ 1, abort_flag, lim)) {
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
+        const int nu = nqb - item / BH;
+        // the epilogue has read the previous item's dV / dK
+        if (!mbar_wait_bounded(acc_empty, (k & 1) ^ 1, abort_flag, lim)) {
           ok = false;
           break;
         }
         for (int u = 0; u < nu; ++u, ++U) {
-          const int s = U % FBK_NST;
-          if (!mbar_wait_bounded(&st_full[s], (U / FBK_NST) & 1, abort_flag, lim) ||
+          const int s = U % BK_NST;
+          if (!mbar_wait_bounded(&st_full[s], (U / BK_NST) & 1, abort_flag, lim) ||
               !mbar_wait_bounded(p_full, U & 1, abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // K = 64 queries: A = P^T (part 0) or dS^T (part 1); B = 16 query rows of dO_u (part 0)
-          // or Q_u (part 1) per step (MN-major)
-          const uint32_t b_addr = smem_u32(sm + FBK_OFF_ST + s * FB_UNIT) + (1 - part) * FB_HALF;
-          const uint32_t a_tm = tmem + (part == 0 ? FBK_TM_P : FBK_TM_DS);
-          const uint32_t acc = tmem + FBK_TM_ACC + part * 64;
+          // K = 128 queries: A = P^T (part 0) or dS^T (part 1), 8 TMEM columns per 16 queries;
+          // B = 16 query rows of dO_i (part 0) or Q_i (part 1) per step
+          const uint32_t b_addr = smem_u32(sm + BK_OFF_ST + s * FB_STAGE + (1 - part) * FA_TILE);
+          const uint32_t a_tm = tmem + (part == 0 ? BK_TM_P : BK_TM_DS);
+          const uint32_t acc = tmem + (part == 0 ? BK_TM_DV : BK_TM_DK);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16_ts(acc, a_tm + k * 8, make_sw128_desc(b_addr + k * 2048, 8192, 1024), idesc_a,
-                         (u > 0 || k > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16_ts(acc, a_tm + kk * 8, make_sw128_desc(b_addr + kk * 2048, 8192, 1024), idesc_a,
+                         (u > 0 || kk > 0) ? 1u : 0u);
           any = true;
           umma_commit(p_free);
-          // the unit's scores were consumed before P^T was written: its score MMAs are complete
-          umma_commit(&st_empty[s]);
+          umma_commit(&st_empty[s]);  // the unit's score products completed before P^T was written
           if (u == nu - 1) umma_commit(acc_full);
         }
       }
@@ -358,123 +368,123 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
         *abort_flag = 1;
         if (any) {
           int never = 0;
-          umma_commit(&drain[2 + part]);
-          mbar_wait_bounded(&drain[2 + part], 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[1 + part]);
+          mbar_wait_bounded(&drain[1 + part], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
   } else {
-    // ---------------- element-wise warps: key row r, query columns [cg*16, cg*16 + 16) of each unit ----------------
-    const int q4 = warp & 3, cg = (warp - FBK_EW0) >> 2;
+    // ---------------- element-wise warps: key row r, query columns [cg*32, cg*32 + 32) of each unit ----------------
+    const int q4 = warp & 3, cg = (warp - BK_EW0) >> 2;
     const int r = q4 * 32 + lane;
-    const bool issuer = (warp == FBK_EW0 && lane == 0);  // issues the output tiles' TMA stores
+    const bool issuer = (warp == BK_EW0 && lane == 0);  // issues the output tiles' TMA stores
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * LOG2E;
     bool fail = false;
     int U = 0;
-    // K and V rows of item `it` into the TMEM A operands (after the previous item's score
-    // MMAs, whose results this warp has all seen)
-    auto load_operands = [&](int it) -> bool {
-      const int kvb = it & 1;
-      if (!fb_warp_wait(&kv_full[kvb], (it >> 1) & 1, abort_flag, lim, lane)) return false;
-      const uint8_t* kd = sm + FBK_OFF_KV + kvb * 2 * FA_TILE;
-      fb_row_to_tmem(kd, r, cg, tmem + lane_off + FBK_TM_KV + cg * 8);
-      fb_row_to_tmem(kd + FA_TILE, r, cg, tmem + lane_off + FBK_TM_KV + 32 + cg * 8);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(kva_full);
-        mbar_arrive(&kv_empty[kvb]);
-      }
-      return true;
-    };
-    if ((int)blockIdx.x < nitems) fail = !load_operands(0);
-    for (int it = 0, item = blockIdx.x; item < nitems && !fail; ++it, item += gridDim.x) {
+    for (int k = 0; !fail; ++k) {
+      const int item = fx_item(k, cta, G);
+      if (item >= nitems) break;
       const int kb = item / BH, bh = item - kb * BH, b = bh / NH, h = bh - b * NH;
-      const int nu = 2 * (nqb - kb);
+      const int nu = nqb - kb;
       for (int u = 0; u < nu; ++u, ++U) {
-        const int sb = U % FB_SBUF, s = U % FBK_NST;
+        const int s = U % BK_NST;
         // the producer's lse / D of this unit (acquired directly from its lanes), then the scores
-        if (!fb_warp_wait(&st_full[s], (U / FBK_NST) & 1, abort_flag, lim, lane) ||
-            !fb_warp_wait(&s_full[sb], (U / FB_SBUF) & 1, abort_flag, lim, lane)) {
+        if (!fb_warp_wait(&st_full[s], (U / BK_NST) & 1, abort_flag, lim, lane) ||
+            !fb_warp_wait(s_full, U & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
         tc_fence_after();
-        uint32_t sv[16], dv[16];
-        tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(sb * 128 + cg * 16), sv);
-        tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(sb * 128 + 64 + cg * 16), dv);
+        uint32_t sv[32], dv[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(cg * 32), sv);
+        tmem_ld_32x32b_x32(tmem + lane_off + BK_TM_DP + (uint32_t)(cg * 32), dv);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[sb]);
-        const float* ld = reinterpret_cast<const float*>(sm + FBK_OFF_LD + s * 512) + cg * 16;
-        float p[16], ds[16];
-        const int qcol0 = (u & 1) * 64 + cg * 16;  // query index within the block of column 0
-        const bool diag = u < 2;                    // the query block kb itself
+        if (lane == 0) mbar_arrive(s_empty);
+        const float* ld = reinterpret_cast<const float*>(sm + BK_OFF_LD + s * 1024) + cg * 32;
+        uint32_t pw[16], dw[16];
+        const bool diag = u == 0;  // the query block kb itself: queries before the key get P = 0
 #pragma unroll
-        for (int e4 = 0; e4 < 4; ++e4) {
+        for (int e4 = 0; e4 < 8; ++e4) {
           const float4 L4 = *reinterpret_cast<const float4*>(ld + 4 * e4);
-          const float4 D4 = *reinterpret_cast<const float4*>(ld + 64 + 4 * e4);
+          const float4 D4 = *reinterpret_cast<const float4*>(ld + 128 + 4 * e4);
           const float Lv[4] = {L4.x, L4.y, L4.z, L4.w}, Dv[4] = {D4.x, D4.y, D4.z, D4.w};
+          float p[4], ds[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int e = 4 * e4 + i;
             float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -Lv[i]));
-            if (diag && r > qcol0 + e) pe = 0.f;  // key after query
-            p[e] = pe;
-            ds[e] = pe * (__uint_as_float(dv[e]) - Dv[i]);
+            if (diag && cg * 32 + e < r) pe = 0.f;
+            p[i] = pe;
+            ds[i] = pe * (__uint_as_float(dv[e]) - Dv[i]);
           }
+          pw[2 * e4] = pack_bf16x2(p[0], p[1]);
+          pw[2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
+          dw[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+          dw[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        // the previous unit's dV / dK MMAs have finished reading P^T and dS^T
+        // the previous unit's dV / dK products have finished reading P^T and dS^T
         if (!fb_warp_wait(p_free, (U & 1) ^ 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
-        fb_vals_to_tmem(p, tmem + lane_off + FBK_TM_P + cg * 8);
-        fb_vals_to_tmem(ds, tmem + lane_off + FBK_TM_DS + cg * 8);
+        tmem_st_32x32b_x16(tmem + lane_off + BK_TM_P + (uint32_t)(cg * 16), pw);
+        tmem_st_32x32b_x16(tmem + lane_off + BK_TM_DS + (uint32_t)(cg * 16), dw);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
       }
       if (fail) break;
-      // the next item's K / V first (lets its score MMAs start), then this item's dV / dK
-      if (item + (int)gridDim.x < nitems && !load_operands(it + 1)) {
-        fail = true;
-        break;
-      }
-      if (!fb_warp_wait(acc_full, it & 1, abort_flag, lim, lane)) {
+      if (!fb_warp_wait(acc_full, k & 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
       tc_fence_after();
-      uint32_t v[16], k[16];
-      tmem_ld_32x32b_x16(tmem + lane_off + FBK_TM_ACC + (uint32_t)(cg * 16), v);
-      tmem_ld_32x32b_x16(tmem + lane_off + FBK_TM_ACC + (uint32_t)(64 + cg * 16), k);
+      uint32_t v[16], kg[16];
+      tmem_ld_32x32b_x16(tmem + lane_off + BK_TM_DV + (uint32_t)(cg * 16), v);
+      tmem_ld_32x32b_x16(tmem + lane_off + BK_TM_DK + (uint32_t)(cg * 16), kg);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
+      if (colsum) {
+        // column sums of dK and dV over this warp's 32 key rows (rows past T left out): the
+        // key and value thirds of the qkv bias gradient, one partial per 32-row block
+        const bool row_ok = kb * FA_BN + r < T;
+        float ck[16], cv[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          ck[e] = row_ok ? __uint_as_float(kg[e]) * scale : 0.f;
+          cv[e] = row_ok ? __uint_as_float(v[e]) : 0.f;
+        }
+        const float sk = warp_colsum16(ck, lane), sv2 = warp_colsum16(cv, lane);
+        if (lane < 16) {
+          float* row = colsum + (long long)((b * nqb + kb) * 4 + q4) * (3 * C) + h * 64 + cg * 16 + lane;
+          row[C] = sk;
+          row[2 * C] = sv2;
+        }
+      }
       // dK (scaled) and dV through shared memory, one TMA store per tile (rows past T are clipped)
-      if (issuer && it > 0) {
+      if (issuer && k > 0) {
         bulk_wait_read<0>();
         mbar_arrive(out_free);
       }
-      if (!fb_warp_wait(out_free, (it & 1) ^ 1, abort_flag, lim, lane)) {
+      if (!fb_warp_wait(out_free, (k & 1) ^ 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
-      fb_stage_row16(sm + FBK_OFF_OUT, r, cg, k, scale);
-      fb_stage_row16(sm + FBK_OFF_OUT + FA_TILE, r, cg, v, 1.0f);
+      fb_stage_row16(sm + BK_OFF_OUT, r, cg, kg, scale);
+      fb_stage_row16(sm + BK_OFF_OUT + FA_TILE, r, cg, v, 1.0f);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(out_full);
       if (issuer) {
-        if (mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
-          tma_store_3d(&tm_out, sm + FBK_OFF_OUT, C + h * 64, kb * FA_BN, b);
-          tma_store_3d(&tm_out, sm + FBK_OFF_OUT + FA_TILE, 2 * C + h * 64, kb * FA_BN, b);
+        if (mbar_wait_bounded(out_full, k & 1, abort_flag, lim)) {
+          tma_store_3d(&tm_out, sm + BK_OFF_OUT, C + h * 64, kb * FA_BN, b);
+          tma_store_3d(&tm_out, sm + BK_OFF_OUT + FA_TILE, 2 * C + h * 64, kb * FA_BN, b);
           bulk_commit();
         } else {
           fail = true;
@@ -500,58 +510,57 @@ __global__ void __launch_bounds__(FBK_THREADS, 1)
   }
 }
 
-__global__ void __launch_bounds__(FBQ_THREADS, 1)
-    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                          const __grid_constant__ CUtensorMap tm_kv64, const __grid_constant__ CUtensorMap tm_out,
-                          const float* __restrict__ lse, const float* __restrict__ Dg, int T, int NH, int BH,
+__global__ void __launch_bounds__(BQ_THREADS, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ CUtensorMap tm_out, const float* __restrict__ lse,
+                          const float* __restrict__ Dg, float* __restrict__ colsum, int T, int NH, int BH,
                           float scale, int* err, unsigned long long timeout_ns) {
   extern __shared__ uint8_t fb_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FBQ_OFF_BAR);
-  uint64_t* qd_full = bar;                    // [2] Q/dO tiles landed in shared memory
-  uint64_t* qd_empty = qd_full + 2;           // [2] copied into TMEM by the element-wise warps
-  uint64_t* qa_full = qd_empty + 2;           // Q/dO A operands written to TMEM (once per item)
-  uint64_t* st_full = qa_full + 1;            // [FBQ_NST]
-  uint64_t* st_empty = st_full + FBQ_NST;     // [FBQ_NST]
-  uint64_t* s_full = st_empty + FBQ_NST;      // [FB_SBUF]
-  uint64_t* s_empty = s_full + FB_SBUF;       // [FB_SBUF]
-  uint64_t* ds_full = s_empty + FB_SBUF;      // [2]
-  uint64_t* ds_free = ds_full + 2;            // [2]
-  uint64_t* acc_full = ds_free + 2;           // [2]
-  uint64_t* acc_empty = acc_full + 2;         // [2]
-  uint64_t* out_full = acc_empty + 2;         // output tile staged (element-wise warps)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BQ_OFF_BAR);
+  uint64_t* qd_full = bar;                    // [2] Q / dO tiles landed in shared memory
+  uint64_t* qd_empty = qd_full + 2;           // [2] copied into TMEM (16 warps)
+  uint64_t* qa_full = qd_empty + 2;           // the Q / dO A operands are written to TMEM (16 warps)
+  uint64_t* st_full = qa_full + 1;            // [BQ_NST]
+  uint64_t* st_empty = st_full + BQ_NST;      // [BQ_NST]
+  uint64_t* s_full = st_empty + BQ_NST;       // S and dP complete
+  uint64_t* s_empty = s_full + 1;             // both read into registers (16 warps)
+  uint64_t* ds_full = s_empty + 1;            // dS written (16 warps)
+  uint64_t* ds_free = ds_full + 1;            // the dQ product has read it
+  uint64_t* acc_full = ds_free + 1;           // [2] the item's dQ complete
+  uint64_t* acc_empty = acc_full + 2;         // [2] read by the epilogue (16 warps)
+  uint64_t* out_full = acc_empty + 2;         // output tile staged (16 warps)
   uint64_t* out_free = out_full + 1;          // the previous item's TMA store has read the staging
-  uint64_t* drain = out_free + 1;             // [3]: one per MMA thread (abort path)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 4);
+  uint64_t* drain = out_free + 1;             // [2]: one per MMA thread (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 3);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = NH * 64;
   const int nqb = (T + FA_BM - 1) / FA_BM;
   const int nitems = nqb * BH;  // item w: query block nqb - 1 - w / BH (longest rows first), bh = w % BH
+  const int G = gridDim.x, cta = blockIdx.x;
   const uint64_t lim = timeout_ns;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&qd_full[i], 1);
       mbar_init(&qd_empty[i], FB_EW_WARPS);
-      mbar_init(&ds_full[i], FB_EW_WARPS);
-      mbar_init(&ds_free[i], 1);
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], FB_EW_WARPS);
     }
-    for (int i = 0; i < 3; ++i) mbar_init(&drain[i], 1);
-    mbar_init(out_full, FB_EW_WARPS);
-    mbar_init(out_free, 1);
     mbar_init(qa_full, FB_EW_WARPS);
-    for (int i = 0; i < FBQ_NST; ++i) {
+    for (int i = 0; i < BQ_NST; ++i) {
       mbar_init(&st_full[i], 1);
       mbar_init(&st_empty[i], 1);
     }
-    for (int i = 0; i < FB_SBUF; ++i) {
-      mbar_init(&s_full[i], 2);  // the S and dP threads
-      mbar_init(&s_empty[i], FB_EW_WARPS);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, FB_EW_WARPS);
+    mbar_init(ds_full, FB_EW_WARPS);
+    mbar_init(ds_free, 1);
+    mbar_init(out_full, FB_EW_WARPS);
+    mbar_init(out_free, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&drain[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -566,37 +575,38 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- producer: Q/dO per item, (K_u, V_u) per unit ----------------
-      tma_prefetch_desc(&tm_q);
+      // ---------------- producer: Q/dO per item, (K_j, V_j) per unit ----------------
+      tma_prefetch_desc(&tm_qkv);
       tma_prefetch_desc(&tm_do);
-      tma_prefetch_desc(&tm_kv64);
       bool ok = true;
       uint32_t qd_iss = 0, qd_par = 0, st_iss = 0, st_par = 0;
       int U = 0;
-      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
         const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
-        const int qdb = it & 1;
-        if (!mbar_wait_bounded(&qd_empty[qdb], ((it >> 1) & 1) ^ 1, abort_flag, lim)) {
+        const int qdb = k & 1;
+        if (!mbar_wait_bounded(&qd_empty[qdb], ((k >> 1) & 1) ^ 1, abort_flag, lim)) {
           ok = false;
           break;
         }
-        uint8_t* qd = sm + FBQ_OFF_QD + qdb * 2 * FA_TILE;
+        uint8_t* qd = sm + BQ_OFF_QD + qdb * 2 * FA_TILE;
         mbar_arrive_expect_tx(&qd_full[qdb], 2 * FA_TILE);
-        tma_load_3d(qd, &tm_q, &qd_full[qdb], h * 64, qb * FA_BM, b);
+        tma_load_3d(qd, &tm_qkv, &qd_full[qdb], h * 64, qb * FA_BM, b);
         tma_load_3d(qd + FA_TILE, &tm_do, &qd_full[qdb], h * 64, qb * FA_BM, b);
         qd_iss |= 1u << qdb;
-        qd_par = (qd_par & ~(1u << qdb)) | ((uint32_t)((it >> 1) & 1) << qdb);
-        for (int k0 = 0; k0 < (qb + 1) * FA_BN; k0 += 64, ++U) {
-          const int s = U % FBQ_NST;
-          const uint32_t ph = (uint32_t)((U / FBQ_NST) & 1);
+        qd_par = (qd_par & ~(1u << qdb)) | ((uint32_t)((k >> 1) & 1) << qdb);
+        for (int j = 0; j <= qb; ++j, ++U) {
+          const int s = U % BQ_NST;
+          const uint32_t ph = (uint32_t)((U / BQ_NST) & 1);
           if (!mbar_wait_bounded(&st_empty[s], ph ^ 1, abort_flag, lim)) {
             ok = false;
             break;
           }
-          uint8_t* d = sm + FBQ_OFF_ST + s * FB_UNIT;
-          mbar_arrive_expect_tx(&st_full[s], FB_UNIT);
-          tma_load_3d(d, &tm_kv64, &st_full[s], C + h * 64, k0, b);
-          tma_load_3d(d + FB_HALF, &tm_kv64, &st_full[s], 2 * C + h * 64, k0, b);
+          uint8_t* d = sm + BQ_OFF_ST + s * FB_STAGE;
+          mbar_arrive_expect_tx(&st_full[s], FB_STAGE);
+          tma_load_3d(d, &tm_qkv, &st_full[s], C + h * 64, j * FA_BN, b);
+          tma_load_3d(d + FA_TILE, &tm_qkv, &st_full[s], 2 * C + h * 64, j * FA_BN, b);
           st_iss |= 1u << s;
           st_par = (st_par & ~(1u << s)) | (ph << s);
         }
@@ -608,40 +618,42 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
         for (int i = 0; i < 2; ++i)
           if ((qd_iss >> i) & 1u)
             mbar_wait_bounded(&qd_full[i], (qd_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
-        for (int i = 0; i < FBQ_NST; ++i)
+        for (int i = 0; i < BQ_NST; ++i)
           if ((st_iss >> i) & 1u)
             mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
       }
     }
-  } else if (warp == 1 || warp == 2) {
+  } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- score MMAs: S = Q K_u^T (warp 1), dP = dO V_u^T (warp 2); A from TMEM ----------------
-      const int part = warp - 1;
-      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64, false, false);
+      // ---------------- score MMAs: S = Q K_j^T, then dP = dO V_j^T; A from TMEM ----------------
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
       bool ok = true, any = false;
       int U = 0;
-      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
-        const int nu = 2 * (nqb - item / BH);
-        if (!mbar_wait_bounded(qa_full, it & 1, abort_flag, lim)) {
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
+        const int nu = nqb - item / BH;
+        if (!mbar_wait_bounded(qa_full, k & 1, abort_flag, lim)) {
           ok = false;
           break;
         }
         for (int u = 0; u < nu; ++u, ++U) {
-          const int s = U % FBQ_NST, sb = U % FB_SBUF;
-          if (!mbar_wait_bounded(&st_full[s], (U / FBQ_NST) & 1, abort_flag, lim) ||
-              !mbar_wait_bounded(&s_empty[sb], ((U / FB_SBUF) & 1) ^ 1, abort_flag, lim)) {
+          const int s = U % BQ_NST;
+          if (!mbar_wait_bounded(&st_full[s], (U / BQ_NST) & 1, abort_flag, lim) ||
+              !mbar_wait_bounded(s_empty, (U & 1) ^ 1, abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          // B = K_u (part 0) or V_u (part 1): 64 rows, K-major
-          const uint32_t b_addr = smem_u32(sm + FBQ_OFF_ST + s * FB_UNIT) + part * FB_HALF;
-          const uint32_t d = tmem + (uint32_t)(sb * 128 + part * 64);
+          // part 0: A = Q, B = K_j -> S; part 1: A = dO, B = V_j -> dP (B: 128 rows, K-major)
+          const uint32_t st_addr = smem_u32(sm + BQ_OFF_ST + s * FB_STAGE);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16_ts(d, tmem + FBQ_TM_Q + part * 32 + k * 8, make_sw128_desc(b_addr + k * 32, 16, 1024), idesc_s,
-                         k > 0 ? 1u : 0u);
-          umma_commit(&s_full[sb]);
+          for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ts(tmem + part * BQ_TM_DP, tmem + BQ_TM_Q + part * 32 + kk * 8,
+                           make_sw128_desc(st_addr + part * FA_TILE + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          umma_commit(s_full);
           any = true;
         }
       }
@@ -650,41 +662,43 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
         *abort_flag = 1;
         if (any) {
           int never = 0;
-          umma_commit(&drain[part]);
-          mbar_wait_bounded(&drain[part], 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[0]);
+          mbar_wait_bounded(&drain[0], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
-  } else if (warp == 3) {
+  } else if (warp == 2) {
     if (lane == 0) {
-      // ---------------- accumulation MMAs: dQ += dS K_u (A = dS from TMEM) ----------------
-      constexpr uint32_t idesc_q = make_idesc_bf16(128, 64, false, true);  // B = K_u, MN-major
+      // ---------------- accumulation MMAs: dQ += dS K_j (A = dS from TMEM) ----------------
+      constexpr uint32_t idesc_q = make_idesc_bf16(128, 64, false, true);  // B = K_j, MN-major
       bool ok = true, any = false;
       int U = 0;
-      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
-        const int ab = it & 1, nu = 2 * (nqb - item / BH);
-        if (!mbar_wait_bounded(&acc_empty[ab], ((it >> 1) & 1) ^ 1, abort_flag, lim)) {
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
+        const int ab = k & 1, nu = nqb - item / BH;
+        if (!mbar_wait_bounded(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag, lim)) {
           ok = false;
           break;
         }
         for (int u = 0; u < nu; ++u, ++U) {
-          const int s = U % FBQ_NST, dsb = U & 1;
-          if (!mbar_wait_bounded(&st_full[s], (U / FBQ_NST) & 1, abort_flag, lim) ||
-              !mbar_wait_bounded(&ds_full[dsb], (U >> 1) & 1, abort_flag, lim)) {
+          const int s = U % BQ_NST;
+          if (!mbar_wait_bounded(&st_full[s], (U / BQ_NST) & 1, abort_flag, lim) ||
+              !mbar_wait_bounded(ds_full, U & 1, abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm + FBQ_OFF_ST + s * FB_UNIT);
-          const uint32_t acc = tmem + FBQ_TM_ACC + (uint32_t)(ab * 64);
-          // K = 64 keys: B = 16 key rows of K_u per step (MN-major)
+          const uint32_t k_addr = smem_u32(sm + BQ_OFF_ST + s * FB_STAGE);
+          const uint32_t acc = tmem + BQ_TM_ACC + (uint32_t)(ab * 64);
+          // K = 128 keys: A = dS (8 TMEM columns per 16 keys), B = 16 key rows of K_j per step
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16_ts(acc, tmem + FBQ_TM_DS + dsb * 32 + k * 8, make_sw128_desc(k_addr + k * 2048, 8192, 1024),
-                         idesc_q, (u > 0 || k > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16_ts(acc, tmem + BQ_TM_DS + kk * 8, make_sw128_desc(k_addr + kk * 2048, 8192, 1024), idesc_q,
+                         (u > 0 || kk > 0) ? 1u : 0u);
           any = true;
-          umma_commit(&ds_free[dsb]);
-          umma_commit(&st_empty[s]);  // the unit's score MMAs completed before dS was written
+          umma_commit(ds_free);
+          umma_commit(&st_empty[s]);  // the unit's score products completed before dS was written
           if (u == nu - 1) umma_commit(&acc_full[ab]);
         }
       }
@@ -693,29 +707,29 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
         *abort_flag = 1;
         if (any) {
           int never = 0;
-          umma_commit(&drain[2]);
-          mbar_wait_bounded(&drain[2], 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[1]);
+          mbar_wait_bounded(&drain[1], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
   } else {
-    // ---------------- element-wise warps: query row r, key columns [cg*16, cg*16 + 16) of each unit ----------------
-    const int q4 = warp & 3, cg = (warp - FBQ_EW0) >> 2;
+    // ---------------- element-wise warps: query row r, key columns [cg*32, cg*32 + 32) of each unit ----------------
+    const int q4 = warp & 3, cg = (warp - BQ_EW0) >> 2;
     const int r = q4 * 32 + lane;
-    const bool issuer = (warp == FBQ_EW0 && lane == 0);  // issues the output tile's TMA store
+    const bool issuer = (warp == BQ_EW0 && lane == 0);  // issues the output tile's TMA store
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * LOG2E;
     bool fail = false;
     int U = 0;
-    // Q and dO rows of item `it` (in shared memory) into the TMEM A operands. The score
-    // MMAs of the previous item, the only readers of that TMEM, are complete: this warp
+    // Q and dO rows of item round k (in shared memory) into the TMEM A operands. The score
+    // products of the previous item, the only readers of that TMEM, are complete: this warp
     // has seen all of their results.
-    auto load_operands = [&](int it) -> bool {
-      const int qdb = it & 1;
-      if (!fb_warp_wait(&qd_full[qdb], (it >> 1) & 1, abort_flag, lim, lane)) return false;
-      const uint8_t* qd = sm + FBQ_OFF_QD + qdb * 2 * FA_TILE;
-      fb_row_to_tmem(qd, r, cg, tmem + lane_off + FBQ_TM_Q + cg * 8);
-      fb_row_to_tmem(qd + FA_TILE, r, cg, tmem + lane_off + FBQ_TM_Q + 32 + cg * 8);
+    auto load_operands = [&](int k) -> bool {
+      const int qdb = k & 1;
+      if (!fb_warp_wait(&qd_full[qdb], (k >> 1) & 1, abort_flag, lim, lane)) return false;
+      const uint8_t* qd = sm + BQ_OFF_QD + qdb * 2 * FA_TILE;
+      fb_row_to_tmem(qd, r, cg, tmem + lane_off + BQ_TM_Q + cg * 8);
+      fb_row_to_tmem(qd + FA_TILE, r, cg, tmem + lane_off + BQ_TM_Q + 32 + cg * 8);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -726,97 +740,109 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
       return true;
     };
     // lse (log2 units) and D of this thread's query row, one item ahead
-    float lse2 = INFINITY, Dr = 0.f;
-    if ((int)blockIdx.x < nitems) {
-      const int item = blockIdx.x, qrow = (nqb - 1 - item / BH) * FA_BM + r;
-      const long long o = (long long)(item % BH) * T + qrow;
+    auto row_stats = [&](int item, float& l2, float& d) {
+      l2 = INFINITY;
+      d = 0.f;
+      if (item >= nitems) return;
+      const int qrow = (nqb - 1 - item / BH) * FA_BM + r;
       if (qrow < T) {
-        lse2 = lse[o] * LOG2E;
-        Dr = Dg[o];
+        const long long o = (long long)(item % BH) * T + qrow;
+        l2 = __ldg(lse + o) * LOG2E;
+        d = __ldg(Dg + o);
       }
-      fail = !load_operands(0);
-    }
-    for (int it = 0, item = blockIdx.x; item < nitems && !fail; ++it, item += gridDim.x) {
+    };
+    float lse2, Dr;
+    row_stats(fx_item(0, cta, G), lse2, Dr);
+    if (fx_item(0, cta, G) < nitems) fail = !load_operands(0);
+    for (int k = 0; !fail; ++k) {
+      const int item = fx_item(k, cta, G);
+      if (item >= nitems) break;
       const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
-      const int nu = 2 * (qb + 1);
-      // the next item's lse / D: loads issued now, first used at the item switch
-      float lse_n = INFINITY, Dr_n = 0.f;
-      if (item + (int)gridDim.x < nitems) {
-        const int item2 = item + gridDim.x, qrow2 = (nqb - 1 - item2 / BH) * FA_BM + r;
-        const long long o = (long long)(item2 % BH) * T + qrow2;
-        if (qrow2 < T) {
-          lse_n = __ldg(lse + o);
-          Dr_n = __ldg(Dg + o);
-        }
-      }
+      const int nu = qb + 1;
+      const int next = fx_item(k + 1, cta, G);
+      float lse_n, Dr_n;
+      row_stats(next, lse_n, Dr_n);
       for (int u = 0; u < nu; ++u, ++U) {
-        const int sb = U % FB_SBUF, dsb = U & 1;
-        if (!fb_warp_wait(&s_full[sb], (U / FB_SBUF) & 1, abort_flag, lim, lane)) {
+        if (!fb_warp_wait(s_full, U & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
         tc_fence_after();
-        uint32_t sv[16], dv[16];
-        tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(sb * 128 + cg * 16), sv);
-        tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(sb * 128 + 64 + cg * 16), dv);
+        uint32_t sv[32], dv[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(cg * 32), sv);
+        tmem_ld_32x32b_x32(tmem + lane_off + BQ_TM_DP + (uint32_t)(cg * 32), dv);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[sb]);
-        float ds[16];
-        const int kcol0 = (u & 1) * 64 + cg * 16;  // key index within the block of column 0
-        const bool diag = u >= nu - 2;             // the key block qb itself
+        if (lane == 0) mbar_arrive(s_empty);
+        uint32_t dw[16];
+        const bool diag = u == nu - 1;  // the key block qb itself: keys after the query get P = 0
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -lse2));
-          if (diag && kcol0 + e > r) pe = 0.f;  // key after query
-          ds[e] = pe * (__uint_as_float(dv[e]) - Dr);
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float ds[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int e = 2 * e2 + i;
+            float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -lse2));
+            if (diag && cg * 32 + e > r) pe = 0.f;
+            ds[i] = pe * (__uint_as_float(dv[e]) - Dr);
+          }
+          dw[e2] = pack_bf16x2(ds[0], ds[1]);
         }
-        // the dQ MMAs of unit U - 2 have finished reading this dS buffer
-        if (!fb_warp_wait(&ds_free[dsb], ((U >> 1) & 1) ^ 1, abort_flag, lim, lane)) {
+        // the previous unit's dQ product has finished reading dS
+        if (!fb_warp_wait(ds_free, (U & 1) ^ 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
-        fb_vals_to_tmem(ds, tmem + lane_off + FBQ_TM_DS + dsb * 32 + cg * 8);
+        tmem_st_32x32b_x16(tmem + lane_off + BQ_TM_DS + (uint32_t)(cg * 16), dw);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ds_full[dsb]);
+        if (lane == 0) mbar_arrive(ds_full);
       }
       if (fail) break;
-      // the next item's operands first (lets its score MMAs start), then this item's dQ
-      if (item + (int)gridDim.x < nitems && !load_operands(it + 1)) {
+      // the next item's operands first (lets its score products start), then this item's dQ
+      if (next < nitems && !load_operands(k + 1)) {
         fail = true;
         break;
       }
-      const int ab = it & 1;
-      if (!fb_warp_wait(&acc_full[ab], (it >> 1) & 1, abort_flag, lim, lane)) {
+      const int ab = k & 1;
+      if (!fb_warp_wait(&acc_full[ab], (k >> 1) & 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
       tc_fence_after();
       uint32_t v[16];
-      tmem_ld_32x32b_x16(tmem + lane_off + FBQ_TM_ACC + (uint32_t)(ab * 64 + cg * 16), v);
+      tmem_ld_32x32b_x16(tmem + lane_off + BQ_TM_ACC + (uint32_t)(ab * 64 + cg * 16), v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (colsum) {
+        // column sums of dQ over this warp's 32 query rows (rows past T are zero here): the
+        // query third of the qkv bias gradient, one partial per 32-row block
+        float cq[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) cq[e] = __uint_as_float(v[e]) * scale;
+        const float sq = warp_colsum16(cq, lane);
+        if (lane < 16) colsum[(long long)((b * nqb + qb) * 4 + q4) * (3 * C) + h * 64 + cg * 16 + lane] = sq;
+      }
       // dQ (scaled) through shared memory, one TMA store (rows past T are clipped)
-      if (issuer && it > 0) {
+      if (issuer && k > 0) {
         bulk_wait_read<0>();
         mbar_arrive(out_free);
       }
-      if (!fb_warp_wait(out_free, (it & 1) ^ 1, abort_flag, lim, lane)) {
+      if (!fb_warp_wait(out_free, (k & 1) ^ 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
-      fb_stage_row16(sm + FBQ_OFF_OUT, r, cg, v, scale);
+      fb_stage_row16(sm + BQ_OFF_OUT, r, cg, v, scale);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(out_full);
       if (issuer) {
-        if (mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
-          tma_store_3d(&tm_out, sm + FBQ_OFF_OUT, h * 64, qb * FA_BM, b);
+        if (mbar_wait_bounded(out_full, k & 1, abort_flag, lim)) {
+          tma_store_3d(&tm_out, sm + BQ_OFF_OUT, h * 64, qb * FA_BM, b);
           bulk_commit();
         } else {
           fail = true;
@@ -826,7 +852,7 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
         fail = true;
         break;
       }
-      lse2 = lse_n * LOG2E;
+      lse2 = lse_n;
       Dr = Dr_n;
     }
     if (issuer) bulk_wait_all();  // the staging must outlive the store's read
@@ -845,94 +871,90 @@ __global__ void __launch_bounds__(FBQ_THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Forward on tcgen05, persistent (one CTA per SM looping over items). Item =
-// (128-query block qb, batch*head), longest rows first; units = 64-key halves of
-// the key blocks 0 .. qb, each streamed through the same 16 KB stage ring as the
-// backward kernels.
-//   S_u  = Q K_u^T     (M=128 queries, N=64 keys, K=64; A = Q in TMEM, B = K_u)
-//   O_g += P_u V_u     (M=128, N=64, K=64 keys;     A = P_u in TMEM, B = V_u)
-// Two softmax groups (4 warps each) take alternate units. Each thread owns one
-// query row of its group's units, so a unit needs no exchange between threads;
-// each group keeps its own running max m, row sum l and output accumulator O_g,
-// and the two are merged when the item ends:
-//   m = max(m_0, m_1), O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)).
-// A group re-bases its running max only when the new block maximum exceeds it by
-// more than 8 (log2 units); otherwise its probabilities are taken against the
-// stale max (at most 2^8, exact in fp32 and representable in bf16) and O_g and l
-// stay consistent because both use the same reference. A re-base rescales the
-// thread's row of O_g in TMEM once the previous P V product has completed.
-// Warps: 0 TMA producer, 1 S MMAs, 2 P V MMAs, 3-6 softmax group 0, 7-10 group 1.
-// Every wait is bounded (device error word, no trap).
+// Forward on tcgen05, persistent (one CTA per SM looping over items). Item = (pair of
+// 128-query tiles, batch*head): query rows [256 qp, 256 qp + 256), tile t holding rows
+// 256 qp + 128 t. Items are ordered longest first and dealt to the CTAs in a zigzag
+// (round k runs over the CTAs forward for even k, backward for odd k), which evens out
+// the causal lengths. Keys come in blocks of 128: tile t needs blocks 0 .. 2 qp + t,
+// the last being its diagonal; each block's K and V are loaded once per item for both
+// tiles.
+//   S_t  = Q_t K_j^T   (M=128 queries, N=128 keys, K=64;     A = Q_t in TMEM, B = K_j)
+//   O_t += P_t V_j     (M=128 queries, N=64,       K=128 keys; A = P_t in TMEM, B = V_j)
+// One softmax warpgroup per tile, one query row per thread: running max with a lazy
+// re-base (only when a block maximum exceeds it by more than 8 in log2 units: the
+// probabilities against the stale maximum stay <= 2^8, exact in fp32 and bf16, and O
+// and the row sum keep one reference), row sum, and P written as bf16 over the first
+// half of S_t's own TMEM columns; so S_t of the next block is issued once P_t V_j has
+// completed. The two tiles interleave: while one warpgroup exponentiates, the tensor
+// core computes the other tile's products.
+// Warps: 0 TMA producer, 1 S MMAs (and the TMEM allocation), 2 P V MMAs, 3-6 softmax
+// of tile 0, 7-10 softmax of tile 1. Every wait is bounded (device error word, no trap).
 // ---------------------------------------------------------------------------
-constexpr int FF_THREADS = 352;
-constexpr int FF_NST = 8;
-constexpr int FF_OFF_Q = 0;                                  // Q tiles [2 items]
-constexpr int FF_OFF_ST = 2 * FA_TILE;                       // stages (K_u | V_u)
-constexpr int FF_OFF_OUT = FF_OFF_ST + FF_NST * FB_UNIT;     // output staging tile
-constexpr int FF_OFF_X = FF_OFF_OUT + FA_TILE;               // (m, l) exchange [2 items][2 groups][128]
-constexpr int FF_OFF_BAR = FF_OFF_X + 2 * 2 * 128 * 8;
-constexpr int FF_SMEM = FF_OFF_BAR + FB_BARS + 1024;
-static_assert(FF_SMEM <= 232448, "shared memory per CTA");
-// TMEM: S [group][2] x 64 at 0..255, O [group] x 64 at 256, Q (32) at 384, P [group] x 32 at 416
-constexpr uint32_t FF_TM_O = 256, FF_TM_Q = 384, FF_TM_P = 416, FF_TMEM_COLS = 512;
-constexpr float FF_REBASE = 8.0f;
+constexpr int FX_THREADS = 352;
+constexpr int FX_NST = 4;                                 // K/V stages
+constexpr int FX_STAGE = 2 * FA_TILE;                     // K_j | V_j: 32 KB
+constexpr int FX_OFF_Q = 0;                               // the item's two Q tiles
+constexpr int FX_OFF_ST = 2 * FA_TILE;
+constexpr int FX_OFF_OUT = FX_OFF_ST + FX_NST * FX_STAGE;  // output staging, one tile per warpgroup
+constexpr int FX_OFF_BAR = FX_OFF_OUT + 2 * FA_TILE;
+constexpr int FX_SMEM = FX_OFF_BAR + FB_BARS + 1024;
+static_assert(FX_SMEM <= 232448, "shared memory per CTA");
+// TMEM: S_t (P_t over its first 64 columns) at 128 t, O_t at 256 + 64 t, Q_t at 384 + 32 t
+constexpr uint32_t FX_TM_O = 256, FX_TM_Q = 384, FX_TMEM_COLS = 512;
+constexpr float FX_REBASE = 8.0f;
 
-__global__ void __launch_bounds__(FF_THREADS, 1)
-    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv64,
-                       const __grid_constant__ CUtensorMap tm_out, float* __restrict__ lse, int T, int NH, int BH,
-                       float scale, int* err, unsigned long long timeout_ns) {
-  extern __shared__ uint8_t ff_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ff_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FF_OFF_BAR);
-  uint64_t* q_full = bar;                  // [2] Q tile landed
-  uint64_t* q_empty = q_full + 2;          // [2] Q copied into TMEM (8 softmax warps)
-  uint64_t* qa_full = q_empty + 2;         // the TMEM Q operand is written (8 softmax warps)
-  uint64_t* st_full = qa_full + 1;         // [FF_NST]
-  uint64_t* st_empty = st_full + FF_NST;   // [FF_NST]
-  uint64_t* s_full = st_empty + FF_NST;    // [group][2]
-  uint64_t* s_empty = s_full + 4;          // [group][2] (the group's 4 warps)
-  uint64_t* p_full = s_empty + 4;          // [group] (4 warps)
-  uint64_t* o_done = p_full + 2;           // [group] P V product complete
-  uint64_t* x_full = o_done + 2;           // (m, l) of both groups written (8 warps), once per item
-  uint64_t* o_read = x_full + 1;           // both groups have read O_0 and O_1 (8 warps), once per item
-  uint64_t* out_full = o_read + 1;         // output tile staged (8 warps)
-  uint64_t* out_free = out_full + 1;       // the previous item's TMA store has read the staging
-  uint64_t* drain = out_free + 1;          // [2]: one per MMA thread (abort path)
+__global__ void __launch_bounds__(FX_THREADS, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_out,
+                       float* __restrict__ lse, int T, int NH, int BH, float scale, int* err,
+                       unsigned long long timeout_ns) {
+  extern __shared__ uint8_t fx_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fx_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FX_OFF_BAR);
+  uint64_t* q_full = bar;                  // the item's Q tiles landed
+  uint64_t* q_empty = q_full + 1;          // both warpgroups copied them (8 warps)
+  uint64_t* qa_full = q_empty + 1;         // [tile] Q_t written to TMEM (4 warps)
+  uint64_t* st_full = qa_full + 2;         // [FX_NST]
+  uint64_t* st_empty = st_full + FX_NST;   // [FX_NST]
+  uint64_t* s_full = st_empty + FX_NST;    // [tile] S_t complete
+  uint64_t* p_full = s_full + 2;           // [tile] P_t written (4 warps)
+  uint64_t* pv_done = p_full + 2;          // [tile] P_t V_j complete
+  uint64_t* o_read = pv_done + 2;          // [tile] O_t read by the epilogue (4 warps)
+  uint64_t* out_full = o_read + 2;         // [tile] output tile staged (4 warps)
+  uint64_t* out_free = out_full + 2;       // [tile] the previous TMA store has read the staging
+  uint64_t* drain = out_free + 2;          // [2]: one per MMA thread (abort path)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 3);
+  static_assert((2 + 2 + 2 * FX_NST + 2 * 7 + 3) * 8 <= FB_BARS, "barrier space");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = NH * 64;
-  const int nqb = (T + FA_BM - 1) / FA_BM;
-  const int nitems = nqb * BH;  // item w: query block nqb - 1 - w / BH, bh = w % BH
+  const int nqp = (T + 255) / 256;
+  const int nitems = nqp * BH;  // item w: query pair nqp - 1 - w / BH, bh = w % BH
+  const int G = gridDim.x, cta = blockIdx.x;
   const uint64_t lim = timeout_ns;
 
   if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 8);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 8);
+      mbar_init(&qa_full[i], 4);
+      mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);
-      mbar_init(&o_done[i], 1);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&o_read[i], 4);
+      mbar_init(&out_full[i], 4);
+      mbar_init(&out_free[i], 1);
       mbar_init(&drain[i], 1);
     }
-    mbar_init(qa_full, 8);
-    for (int i = 0; i < FF_NST; ++i) {
+    for (int i = 0; i < FX_NST; ++i) {
       mbar_init(&st_full[i], 1);
       mbar_init(&st_empty[i], 1);
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
-    }
-    mbar_init(x_full, 8);
-    mbar_init(o_read, 8);
-    mbar_init(out_full, 8);
-    mbar_init(out_free, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, FF_TMEM_COLS);
+    tmem_alloc(tmem_slot, FX_TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -942,34 +964,37 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- producer: Q per item, (K_u, V_u) per unit ----------------
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_kv64);
-      bool ok = true;
-      uint32_t q_iss = 0, q_par = 0, st_iss = 0, st_par = 0;
-      int U = 0;
-      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
-        const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
-        const int qbuf = it & 1;
-        if (!mbar_wait_bounded(&q_empty[qbuf], ((it >> 1) & 1) ^ 1, abort_flag, lim)) {
+      // ---------------- producer: Q tiles per item, (K_j, V_j) per block ----------------
+      tma_prefetch_desc(&tm_qkv);
+      bool ok = true, q_iss = false;
+      uint32_t q_par = 0, st_iss = 0, st_par = 0;
+      int J = 0;  // block loads over all items (stage uses)
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
+        const int qp = nqp - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
+        const int nb = qp * 256 + 128 < T ? 2 * qp + 2 : 2 * qp + 1;
+        // one Q buffer: free once both warpgroups copied the previous item's tiles to TMEM
+        if (k > 0 && !mbar_wait_bounded(q_empty, (k - 1) & 1, abort_flag, lim)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&q_full[qbuf], FA_TILE);
-        tma_load_3d(sm + FF_OFF_Q + qbuf * FA_TILE, &tm_q, &q_full[qbuf], h * 64, qb * FA_BM, b);
-        q_iss |= 1u << qbuf;
-        q_par = (q_par & ~(1u << qbuf)) | ((uint32_t)((it >> 1) & 1) << qbuf);
-        for (int k0 = 0; k0 < (qb + 1) * FA_BN; k0 += 64, ++U) {
-          const int s = U % FF_NST;
-          const uint32_t ph = (uint32_t)((U / FF_NST) & 1);
+        mbar_arrive_expect_tx(q_full, 2 * FA_TILE);
+        tma_load_3d(sm + FX_OFF_Q, &tm_qkv, q_full, h * 64, qp * 256, b);
+        tma_load_3d(sm + FX_OFF_Q + FA_TILE, &tm_qkv, q_full, h * 64, qp * 256 + 128, b);
+        q_iss = true;
+        q_par = k & 1;
+        for (int j = 0; j < nb; ++j, ++J) {
+          const int s = J % FX_NST;
+          const uint32_t ph = (uint32_t)((J / FX_NST) & 1);
           if (!mbar_wait_bounded(&st_empty[s], ph ^ 1, abort_flag, lim)) {
             ok = false;
             break;
           }
-          uint8_t* d = sm + FF_OFF_ST + s * FB_UNIT;
-          mbar_arrive_expect_tx(&st_full[s], FB_UNIT);
-          tma_load_3d(d, &tm_kv64, &st_full[s], C + h * 64, k0, b);
-          tma_load_3d(d + FB_HALF, &tm_kv64, &st_full[s], 2 * C + h * 64, k0, b);
+          uint8_t* d = sm + FX_OFF_ST + s * FX_STAGE;
+          mbar_arrive_expect_tx(&st_full[s], FX_STAGE);
+          tma_load_3d(d, &tm_qkv, &st_full[s], C + h * 64, j * 128, b);
+          tma_load_3d(d + FA_TILE, &tm_qkv, &st_full[s], 2 * C + h * 64, j * 128, b);
           st_iss |= 1u << s;
           st_par = (st_par & ~(1u << s)) | (ph << s);
         }
@@ -977,70 +1002,79 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
       if (!ok) {
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
-        int never = 0;
-        for (int i = 0; i < 2; ++i)
-          if ((q_iss >> i) & 1u)
-            mbar_wait_bounded(&q_full[i], (q_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
-        for (int i = 0; i < FF_NST; ++i)
+        int never = 0;  // let the copies in flight land before the CTA's shared memory goes away
+        if (q_iss) mbar_wait_bounded(q_full, q_par, reinterpret_cast<volatile int*>(&never), lim);
+        for (int i = 0; i < FX_NST; ++i)
           if ((st_iss >> i) & 1u)
             mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
       }
     }
   } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
-      // ---------------- MMAs: S_u = Q K_u^T (warp 1); O_g += P_u V_u (warp 2) ----------------
+      // ---------------- MMAs: S_t = Q_t K_j^T (warp 1); O_t += P_t V_j (warp 2) ----------------
       const bool is_s = warp == 1;
-      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64, false, false);
-      constexpr uint32_t idesc_o = make_idesc_bf16(128, 64, false, true);  // B = V_u, MN-major
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, 64, false, true);  // B = V_j, MN-major
       bool ok = true, any = false;
-      int U = 0;  // unit counter over all items; unit U belongs to group U % 2 (items have even unit counts)
-      for (int it = 0, item = blockIdx.x; item < nitems && ok; ++it, item += gridDim.x) {
-        const int nu = 2 * (nqb - item / BH);
-        if (is_s && !mbar_wait_bounded(qa_full, it & 1, abort_flag, lim)) {
-          ok = false;
-          break;
-        }
-        for (int u = 0; u < nu; ++u, ++U) {
-          const int s = U % FF_NST, g = U & 1, Ug = U >> 1;  // Ug: the unit's index within its group
-          if (!mbar_wait_bounded(&st_full[s], (U / FF_NST) & 1, abort_flag, lim)) {
+      int J = 0, n[2] = {0, 0}, ni[2] = {0, 0};  // blocks, products per tile, valid items per tile
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
+        const int qp = nqp - 1 - item / BH;
+        const bool v1 = qp * 256 + 128 < T;
+        const int nbt[2] = {2 * qp + 1, v1 ? 2 * qp + 2 : 0};
+        const int nb = v1 ? nbt[1] : nbt[0];
+        for (int j = 0; j < nb && ok; ++j, ++J) {
+          const int s = J % FX_NST;
+          if (!mbar_wait_bounded(&st_full[s], (J / FX_NST) & 1, abort_flag, lim)) {
             ok = false;
             break;
           }
-          const uint32_t k_addr = smem_u32(sm + FF_OFF_ST + s * FB_UNIT), v_addr = k_addr + FB_HALF;
-          if (is_s) {
-            const int sg = g * 2 + (Ug & 1);
-            if (!mbar_wait_bounded(&s_empty[sg], ((Ug >> 1) & 1) ^ 1, abort_flag, lim)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
+          const uint32_t k_addr = smem_u32(sm + FX_OFF_ST + s * FX_STAGE), v_addr = k_addr + FA_TILE;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= nbt[t]) continue;
+            if (is_s) {
+              // Q_t of this item is in TMEM; the previous P_t V product (the last reader of
+              // S_t's columns) is complete
+              if ((j == 0 && !mbar_wait_bounded(&qa_full[t], ni[t] & 1, abort_flag, lim)) ||
+                  (n[t] > 0 && !mbar_wait_bounded(&pv_done[t], (n[t] - 1) & 1, abort_flag, lim))) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_bf16_ts(tmem + sg * 64, tmem + FF_TM_Q + k * 8, make_sw128_desc(k_addr + k * 32, 16, 1024), idesc_s,
-                           k > 0 ? 1u : 0u);
-            umma_commit(&s_full[sg]);
-          } else {
-            if (!mbar_wait_bounded(&p_full[g], Ug & 1, abort_flag, lim)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            // K = 64 keys: B = 16 key rows of V_u per step (MN-major); each group's first unit
-            // of an item starts its accumulator
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16_ts(tmem + t * 128, tmem + FX_TM_Q + t * 32 + kk * 8,
+                             make_sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+              umma_commit(&s_full[t]);
+            } else {
+              // the epilogue has read O_t of the tile's previous item; P_t is written
+              if ((j == 0 && ni[t] > 0 && !mbar_wait_bounded(&o_read[t], (ni[t] - 1) & 1, abort_flag, lim)) ||
+                  !mbar_wait_bounded(&p_full[t], n[t] & 1, abort_flag, lim)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              // K = 128 keys: A = P_t (8 TMEM columns per 16 keys), B = 16 key rows of V_j per step
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_bf16_ts(tmem + FF_TM_O + g * 64, tmem + FF_TM_P + g * 32 + k * 8,
-                           make_sw128_desc(v_addr + k * 2048, 8192, 1024), idesc_o, (u >= 2 || k > 0) ? 1u : 0u);
-            umma_commit(&o_done[g]);
-            umma_commit(&st_empty[s]);  // the unit's S MMAs completed before its P was written
+              for (int kk = 0; kk < 8; ++kk)
+                umma_bf16_ts(tmem + FX_TM_O + t * 64, tmem + t * 128 + kk * 8,
+                             make_sw128_desc(v_addr + kk * 2048, 8192, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+              umma_commit(&pv_done[t]);
+            }
+            ++n[t];
+            any = true;
           }
-          any = true;
+          // the block's stage is free once its last P V product completes
+          if (ok && !is_s) umma_commit(&st_empty[s]);
         }
+        if (v1) ++ni[1];
+        ++ni[0];
       }
       if (!ok) {
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
-        if (any) {
+        if (any) {  // wait for the MMAs already issued before the TMEM is freed
           int never = 0;
           umma_commit(&drain[warp - 1]);
           mbar_wait_bounded(&drain[warp - 1], 0, reinterpret_cast<volatile int*>(&never), lim);
@@ -1048,55 +1082,61 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
       }
     }
   } else {
-    // ---------------- softmax: group g, query row r ----------------
-    const int g = (warp - 3) >> 2, q4 = warp & 3;
+    // ---------------- softmax warpgroup of tile t: query row r ----------------
+    const int t = (warp - 3) >> 2, q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tm_s = tmem + lane_off + (uint32_t)(t * 128);
+    const uint32_t tm_o = tmem + lane_off + FX_TM_O + (uint32_t)(t * 64);
     const float sl2 = scale * LOG2E;
-    const bool issuer = (warp == 3 && lane == 0);  // issues the output tile's TMA store
-    float* xb = reinterpret_cast<float*>(sm + FF_OFF_X);  // [item parity][group][row] x (m, l)
+    const bool issuer = (warp == 3 + 4 * t && lane == 0);  // issues the tile's TMA stores
+    uint8_t* stage_out = sm + FX_OFF_OUT + t * FA_TILE;
     bool fail = false;
-    // the Q rows of item `it` into the TMEM A operand: this group copies head dims [g*32, g*32 + 32)
-    auto load_q = [&](int it) -> bool {
-      const int qbuf = it & 1;
-      if (!fb_warp_wait(&q_full[qbuf], (it >> 1) & 1, abort_flag, lim, lane)) return false;
-      const uint8_t* qt = sm + FF_OFF_Q + qbuf * FA_TILE;
-      fb_row_to_tmem(qt, r, 2 * g, tmem + lane_off + FF_TM_Q + (2 * g) * 8);
-      fb_row_to_tmem(qt, r, 2 * g + 1, tmem + lane_off + FF_TM_Q + (2 * g + 1) * 8);
-      tmem_st_wait();
+    // Q_t of item round k into the TMEM A operand (both warpgroups release the smem tiles)
+    auto copy_q = [&](int k, bool valid) -> bool {
+      if (!fb_warp_wait(q_full, k & 1, abort_flag, lim, lane)) return false;
+      if (valid) {
+        const uint8_t* qt = sm + FX_OFF_Q + t * FA_TILE;
+#pragma unroll
+        for (int cg = 0; cg < 4; ++cg) fb_row_to_tmem(qt, r, cg, tmem + lane_off + FX_TM_Q + t * 32 + cg * 8);
+        tmem_st_wait();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(qa_full);
-        mbar_arrive(&q_empty[qbuf]);
+        if (valid) mbar_arrive(&qa_full[t]);
+        mbar_arrive(q_empty);
       }
       return true;
     };
-    if ((int)blockIdx.x < nitems) fail = !load_q(0);
-    int U0 = 0;  // first global unit of the current item
-    for (int it = 0, item = blockIdx.x; item < nitems && !fail; ++it, item += gridDim.x) {
-      const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
-      const int nu = 2 * (qb + 1);
+    auto valid_of = [&](int item) { return t == 0 || (nqp - 1 - item / BH) * 256 + 128 < T; };
+    int n = 0, ni = 0;  // products of this tile; valid items of this tile
+    {
+      const int item0 = fx_item(0, cta, G);
+      if (item0 < nitems) fail = !copy_q(0, valid_of(item0));
+    }
+    for (int k = 0; !fail; ++k) {
+      const int item = fx_item(k, cta, G);
+      if (item >= nitems) break;
+      const int qp = nqp - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
+      const bool valid = valid_of(item);
+      const int nb = valid ? 2 * qp + t + 1 : 0;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int u = g; u < nu; u += 2) {
-        const int U = U0 + u, Ug = U >> 1, sg = g * 2 + (Ug & 1);
-        if (!fb_warp_wait(&s_full[sg], (Ug >> 1) & 1, abort_flag, lim, lane)) {
+      for (int j = 0; j < nb; ++j, ++n) {
+        if (!fb_warp_wait(&s_full[t], n & 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
         tc_fence_after();
-        uint32_t sv[64];
-        tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(sg * 64), *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(sg * 64 + 32), *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[sg]);
-        if (u >= nu - 2) {  // the diagonal key block: keys after the query get -inf
-          const int kbase = (u & 1) * 64;
+        uint32_t sv[128];
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (kbase + e > r) sv[e] = __float_as_uint(-INFINITY);
+        for (int i = 0; i < 4; ++i)
+          tmem_ld_32x32b_x32(tm_s + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * i]));
+        tmem_ld_wait();
+        if (j == nb - 1) {  // the diagonal block: keys after the query get -inf
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > r) sv[c] = __float_as_uint(-INFINITY);
         }
         float mx;
         {
@@ -1104,137 +1144,106 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sv[e]);
 #pragma unroll
-          for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sv[e]));
+          for (int e = 8; e < 128; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sv[e]));
           mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
         const float m_blk = mx * sl2;
-        // re-base only when the block maximum exceeds the reference by more than FF_REBASE
-        const bool rebase = m_blk > m_run + FF_REBASE;
+        const bool rebase = m_blk > m_run + FX_REBASE;
         const float m_use = rebase ? m_blk : m_run;
-        const float m_ref = m_use == -INFINITY ? 0.f : m_use;  // fully masked so far: P = 0
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        uint32_t pw[32];
-#pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) {
-          const float p0 = ex2_fast(fmaf(__uint_as_float(sv[2 * e2]), sl2, -m_ref));
-          const float p1 = ex2_fast(fmaf(__uint_as_float(sv[2 * e2 + 1]), sl2, -m_ref));
-          rs8[(2 * e2) & 7] += p0;
-          rs8[(2 * e2 + 1) & 7] += p1;
-          pw[e2] = pack_bf16x2(p0, p1);
-        }
-        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-        // the group's previous P V product has finished reading P_g (and updating O_g)
-        if (Ug > 0 && !fb_warp_wait(&o_done[g], (Ug - 1) & 1, abort_flag, lim, lane)) {
-          fail = true;
-          break;
-        }
-        tc_fence_after();
-        // rescale rows of O_g to their new reference. tcgen05.ld / st are warp-collective
-        // (.sync.aligned), so the whole warp takes this path when any of its rows re-bases;
-        // the other rows use the factor 1.
+        const float m_ref = m_use == -INFINITY ? 0.f : m_use;
+        // rows that re-base rescale their O_t row (complete: S_t of this block was issued
+        // after the previous P_t V product finished); tcgen05.ld / st are warp-collective,
+        // so the whole warp takes this path when any of its rows needs it
         const bool my_rescale = rebase && m_run != -INFINITY;
+        const float corr = my_rescale ? ex2_fast(m_run - m_use) : 1.0f;
         if (__any_sync(0xffffffffu, my_rescale)) {
-          const float corr = my_rescale ? ex2_fast(m_run - m_use) : 1.0f;
-          uint32_t ov[32];
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            tmem_ld_32x32b_x32(tmem + lane_off + FF_TM_O + g * 64 + hh * 32, ov);
+            uint32_t ov[32];
+            tmem_ld_32x32b_x32(tm_o + hh * 32, ov);
             tmem_ld_wait();
-            uint32_t a[16], c[16];
+            uint32_t a[16], c2[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               a[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-              c[e] = __float_as_uint(__uint_as_float(ov[16 + e]) * corr);
+              c2[e] = __float_as_uint(__uint_as_float(ov[16 + e]) * corr);
             }
-            tmem_st_32x32b_x16(tmem + lane_off + FF_TM_O + g * 64 + hh * 32, a);
-            tmem_st_32x32b_x16(tmem + lane_off + FF_TM_O + g * 64 + hh * 32 + 16, c);
+            tmem_st_32x32b_x16(tm_o + hh * 32, a);
+            tmem_st_32x32b_x16(tm_o + hh * 32 + 16, c2);
           }
-          l_run *= corr;
         }
-        l_run += rs;
+        // P = 2^(s * scale * log2e - m_ref), row sum, bf16 pairs over S_t's first 64 columns
+        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t pw[16];
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const int c = ch * 32 + 2 * e2;
+            const float p0 = ex2_fast(fmaf(__uint_as_float(sv[c]), sl2, -m_ref));
+            const float p1 = ex2_fast(fmaf(__uint_as_float(sv[c + 1]), sl2, -m_ref));
+            rs8[c & 7] += p0;
+            rs8[(c + 1) & 7] += p1;
+            pw[e2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_32x32b_x16(tm_s + ch * 16, pw);
+        }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        l_run = l_run * corr + rs;
         m_run = m_use;
-        // the first unit of an item (after the first item) starts a fresh O_g: both groups
-        // must have read the previous item's accumulators
-        if (u < 2 && it > 0 && !fb_warp_wait(o_read, (it - 1) & 1, abort_flag, lim, lane)) {
-          fail = true;
-          break;
-        }
-        tmem_st_32x32b_x16(tmem + lane_off + FF_TM_P + g * 32, *reinterpret_cast<uint32_t(*)[16]>(&pw[0]));
-        tmem_st_32x32b_x16(tmem + lane_off + FF_TM_P + g * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pw[16]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[g]);
+        if (lane == 0) mbar_arrive(&p_full[t]);
       }
       if (fail) break;
-      // the other group's last S product of this item is complete too: then no MMA
-      // still reads the TMEM Q operand, and the next item's Q can be written
+      // the next item's Q: every S_t product of this item is complete (all seen), so the
+      // TMEM Q_t operand may be overwritten
       {
-        const int uo = nu - 1 - g, Uo = U0 + uo, Ugo = Uo >> 1;
-        if (!fb_warp_wait(&s_full[(1 - g) * 2 + (Ugo & 1)], (Ugo >> 1) & 1, abort_flag, lim, lane)) {
+        const int next = fx_item(k + 1, cta, G);
+        if (next < nitems && !copy_q(k + 1, valid_of(next))) {
           fail = true;
           break;
         }
       }
-      if (item + (int)gridDim.x < nitems && !load_q(it + 1)) {
+      if (!valid) continue;
+      // ---- epilogue: O_t / l to bf16 through the staging tile and one TMA store; lse ----
+      if (!fb_warp_wait(&pv_done[t], (n - 1) & 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
-      // merge the two groups' rows
-      float* xm = xb + ((it & 1) * 2 + g) * 256;
-      xm[r] = m_run;
-      xm[128 + r] = l_run;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(x_full);
-      // both groups' last P V products complete
-      const int Ug_last = (U0 + nu - 2 + g) >> 1, Ugo_last = (U0 + nu - 1 - g) >> 1;
-      if (!fb_warp_wait(x_full, it & 1, abort_flag, lim, lane) ||
-          !fb_warp_wait(&o_done[g], Ug_last & 1, abort_flag, lim, lane) ||
-          !fb_warp_wait(&o_done[1 - g], Ugo_last & 1, abort_flag, lim, lane)) {
-        fail = true;
-        break;
-      }
-      const float* xo = xb + ((it & 1) * 2 + (1 - g)) * 256;
-      const float m_o = xo[r], l_o = xo[128 + r];
-      const float m = fmaxf(m_run, m_o);
-      const float a_s = m_run == -INFINITY ? 0.f : ex2_fast(m_run - m);
-      const float a_o = m_o == -INFINITY ? 0.f : ex2_fast(m_o - m);
-      const float l = l_run * a_s + l_o * a_o;
-      const float inv = 1.0f / l;
-      const float a0 = (g == 0 ? a_s : a_o) * inv, a1 = (g == 0 ? a_o : a_s) * inv;
-      // this thread's output columns [g*32, g*32 + 32) from O_0 and O_1
       tc_fence_after();
-      uint32_t o0[32], o1[32];
-      tmem_ld_32x32b_x32(tmem + lane_off + FF_TM_O + g * 32, o0);
-      tmem_ld_32x32b_x32(tmem + lane_off + FF_TM_O + 64 + g * 32, o1);
+      uint32_t o[64];
+      tmem_ld_32x32b_x32(tm_o, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+      tmem_ld_32x32b_x32(tm_o + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(o_read);
-      const int qrow = qb * FA_BM + r;
-      if (g == 0 && qrow < T) lse[(long long)bh * T + qrow] = (m + __log2f(l)) * LN2;
-      if (issuer && it > 0) {
+      if (lane == 0) mbar_arrive(&o_read[t]);
+      const float inv = 1.0f / l_run;
+      const int qrow = qp * 256 + t * 128 + r;
+      if (qrow < T) lse[(long long)bh * T + qrow] = (m_run + __log2f(l_run)) * LN2;
+      if (issuer && ni > 0) {
         bulk_wait_read<0>();
-        mbar_arrive(out_free);
+        mbar_arrive(&out_free[t]);
       }
-      if (!fb_warp_wait(out_free, (it & 1) ^ 1, abort_flag, lim, lane)) {
+      if (!fb_warp_wait(&out_free[t], (ni & 1) ^ 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int cg = 0; cg < 4; ++cg) {
         float f[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          f[e] = __uint_as_float(o0[hh * 16 + e]) * a0 + __uint_as_float(o1[hh * 16 + e]) * a1;
-        fb_store16(sm + FF_OFF_OUT, r, g * 4 + hh * 2, f);
+        for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(o[cg * 16 + e]) * inv;
+        fb_store16(stage_out, r, cg * 2, f);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(out_full);
+      if (lane == 0) mbar_arrive(&out_full[t]);
       if (issuer) {
-        if (mbar_wait_bounded(out_full, it & 1, abort_flag, lim)) {
-          tma_store_3d(&tm_out, sm + FF_OFF_OUT, h * 64, qb * FA_BM, b);
+        if (mbar_wait_bounded(&out_full[t], ni & 1, abort_flag, lim)) {
+          tma_store_3d(&tm_out, stage_out, h * 64, qp * 256 + t * 128, b);
           bulk_commit();
         } else {
           fail = true;
@@ -1244,9 +1253,9 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
         fail = true;
         break;
       }
-      U0 += nu;
+      ++ni;
     }
-    if (issuer) bulk_wait_all();
+    if (issuer) bulk_wait_all();  // the staging must outlive the stores' reads
     if (fail && lane == 0) {
       raise_device_error(err, DEV_TIMEOUT);
       *abort_flag = 1;
@@ -1257,7 +1266,7 @@ __global__ void __launch_bounds__(FF_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, FF_TMEM_COLS);
+    tmem_dealloc(tmem, FX_TMEM_COLS);
   }
 }
 

@@ -60,6 +60,7 @@ struct gpt2 {
   char *h1 = nullptr, *qkv = nullptr, *att = nullptr, *h2 = nullptr, *u = nullptr, *a = nullptr, *xf = nullptr;
   char *logits = nullptr, *dres_act = nullptr, *du = nullptr, *datt = nullptr, *dqkv = nullptr;
   float *dres = nullptr, *dh = nullptr, *Dattn = nullptr, *row_loss = nullptr, *part = nullptr, *splitk = nullptr;
+  float2* ce_stats = nullptr;  // softmax partials of one head chunk, [chunk rows][2 * ceil(Vp / 128)]
   size_t part_floats = 0, splitk_floats = 0;
   int *tok = nullptr, *tgt = nullptr;
   void* emb_scratch = nullptr;
@@ -197,7 +198,9 @@ void build_tensors(gpt2* m) {
       x.dev_off = d;
       d = align64(d + x.dev_rows * x.cols);
     }
-  m->n_store = d;
+  // a multiple of 4096 floats, so that the storage splits into equal 64-aligned shards for
+  // up to 64 data-parallel ranks (the tail is zero and stays zero under AdamW)
+  m->n_store = (d + 4095) / 4096 * 4096;
 }
 
 void host_init(const gpt2* m, uint64_t seed, std::vector<float>& out) {
@@ -316,9 +319,19 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
   for (int r0 = 0; r0 < N; r0 += chunk) {
     const int rows = (N - r0) < chunk ? (N - r0) : chunk;
     char* xf_c = m->xf + (int64_t)r0 * C * ab;
-    RK(gemm(c, dt, GemmDesc{xf_c, C, false, m->W(headw), C, false, rows, Vp, C, EPI_BF16, m->logits, Vp, nullptr, 0,
-                            nullptr, nullptr, 0, 0, 1, CAT_GEMM_HEAD}));
-    RK(cross_entropy(c, dt, m->logits, Vp, rows, m->cfg.V, m->tgt + r0, 1.0f / (float)N, m->row_loss + r0));
+    GemmDesc hd{xf_c, C, false, m->W(headw), C, false, rows, Vp, C, EPI_BF16, m->logits, Vp, nullptr, 0,
+                nullptr, nullptr, 0, 0, 1, CAT_GEMM_HEAD};
+    if (dt == GPT2_BF16) {
+      // the head GEMM's epilogue leaves each row's softmax partials for the cross-entropy
+      hd.rowstats = m->ce_stats;
+      hd.stats_ncols = m->cfg.V;
+    }
+    RK(gemm(c, dt, hd));
+    if (dt == GPT2_BF16)
+      RK(cross_entropy_stats(c, (bf16*)m->logits, Vp, rows, m->cfg.V, m->tgt + r0, 1.0f / (float)N,
+                             m->row_loss + r0, m->ce_stats, gemm_rowstats_count(hd), nullptr));
+    else
+      RK(cross_entropy(c, dt, m->logits, Vp, rows, m->cfg.V, m->tgt + r0, 1.0f / (float)N, m->row_loss + r0));
     if (backward) {
       // dxf = dlogits W ; dW += dlogits^T xf
       RK(gemm(c, dt, GemmDesc{m->logits, Vp, false, m->W(headw), C, true, rows, C, Vp, EPI_F32, m->dh + (int64_t)r0 * C,
@@ -360,11 +373,20 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     // MLP: x_out = x_mid + pj(gelu(fc(ln2(x_mid))))
     RK(gemm(c, dt, GemmDesc{dres_act, C, true, a, F, true, C, F, N, EPI_F32, gw.pj_w, F, nullptr, 0, nullptr, nullptr,
                             0, 1, 0, CAT_GEMM_DW}));
-    RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.pj_w), F, true, N, F, C, EPI_BF16_DGELU, m->du, F, nullptr, 0,
-                            nullptr, u, F, 0, 1, CAT_GEMM_DX}));
+    {
+      // bf16: the GELU-backward epilogue leaves the column sums of du (fc's bias gradient)
+      // per 32-row block in m->part
+      GemmDesc d{dres_act, C, false, m->W(w.pj_w), F, true, N, F, C, EPI_BF16_DGELU, m->du, F, nullptr, 0,
+                 nullptr, u, F, 0, 1, CAT_GEMM_DX};
+      if (dt == GPT2_BF16) d.colsum = m->part;
+      RK(gemm(c, dt, d));
+    }
     RK(gemm(c, dt, GemmDesc{m->du, F, true, h2, C, true, F, C, N, EPI_F32, gw.fc_w, C, nullptr, 0, nullptr, nullptr, 0,
                             1, 0, CAT_GEMM_DW}));
-    RK(COLSUM_ACT(m->du, F, gw.fc_b));
+    if (dt == GPT2_BF16)
+      RK(reduce_partials(c, m->part, (N + 31) / 32, F, 1, gw.fc_b, nullptr, nullptr, 1));
+    else
+      RK(COLSUM_ACT(m->du, F, gw.fc_b));
     RK(gemm(c, dt, GemmDesc{m->du, F, false, m->W(w.fc_w), C, true, N, C, F, EPI_F32, m->dh, C, nullptr, 0, nullptr,
                             nullptr, 0, 0, 1, CAT_GEMM_DX}));
     RK(LN_B(m->dh, xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), 1, gw.ln2_g, gw.ln2_b, gw.ao_b));
@@ -373,10 +395,16 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
                             0, 1, 0, CAT_GEMM_DW}));
     RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.ao_w), C, true, N, C, C, EPI_BF16, m->datt, C, nullptr, 0,
                             nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
-    RK(attention_bwd(c, dt, qkv, att, m->datt, lse, B, T, NH, hd, m->dqkv, m->Dattn));
+    // bf16: the attention backward leaves the column sums of dqkv (the qkv bias gradient)
+    // per 32-row block in m->part
+    const bool qkvb_fused = gw.qkv_b && dt == GPT2_BF16;
+    RK(attention_bwd(c, dt, qkv, att, m->datt, lse, B, T, NH, hd, m->dqkv, m->Dattn, qkvb_fused ? m->part : nullptr));
     RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, true, h1, C, true, 3 * C, C, N, EPI_F32, gw.qkv_w, C, nullptr, 0, nullptr,
                             nullptr, 0, 1, 0, CAT_GEMM_DW}));
-    if (gw.qkv_b) RK(COLSUM_ACT(m->dqkv, 3 * C, gw.qkv_b));
+    if (qkvb_fused)
+      RK(reduce_partials(c, m->part, attn_colsum_blocks(B, T), 3 * C, 1, gw.qkv_b, nullptr, nullptr, 1));
+    else if (gw.qkv_b)
+      RK(COLSUM_ACT(m->dqkv, 3 * C, gw.qkv_b));
     RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, false, m->W(w.qkv_w), C, true, N, C, 3 * C, EPI_F32, m->dh, C, nullptr, 0,
                             nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
     RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b,
@@ -426,9 +454,11 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
   m->num_sms = device_sm_count();
   build_tensors(m);
   auto bail = [&](int code, const char* what) {
-    std::string msg = what;
+    (void)what;
     gpt2_destroy(m);
-    (void)msg;
+    // a failed cudaMalloc leaves its error as the runtime's last error: clear it so that
+    // it is not reported by the next launch check of another handle
+    cudaGetLastError();
     return code;
   };
   if (cudaStreamCreateWithFlags(&m->stream, cudaStreamNonBlocking) != cudaSuccess) return bail(GPT2_ERR_CUDA, "stream");
@@ -474,8 +504,11 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
   colsum_shape((int)N, (int)(3 * C > F ? 3 * C : F), gx, R, rp);
   const int64_t colsum_floats = (int64_t)(R + 1) * (3 * C > F ? 3 * C : F);
   // colsum partials never exceed 1184 row chunks x 2048 columns per chunk of columns
-  m->part_floats = (size_t)std::max<int64_t>(std::max<int64_t>(3LL * ln_bwd_grid((int)N) * C, colsum_floats),
-                                             1184LL * 2048 + 4096);
+  m->part_floats = (size_t)std::max<int64_t>(
+      std::max<int64_t>(std::max<int64_t>(3LL * ln_bwd_grid((int)N, (int)C, m->num_sms) * C, colsum_floats),
+                        1184LL * 2048 + 4096),
+      std::max<int64_t>((N + 31) / 32 * F,                         // the GELU-backward epilogue's column sums
+                        (int64_t)(c.B_max * ((c.T + 127) / 128) * 4) * 3 * C));  // the attention backward's
   m->splitk_floats = (size_t)std::max<int64_t>(16LL * F * C, 16LL * chunk * C);
   std::vector<std::pair<void**, size_t>> plan = {
       {(void**)&m->x, (size_t)(2 * L + 1) * N * C * 4},
@@ -490,6 +523,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
       {(void**)&m->a, (size_t)L * N * F * ab},
       {(void**)&m->xf, (size_t)N * C * ab},
       {(void**)&m->logits, (size_t)chunk * m->Vp * ab},
+      {(void**)&m->ce_stats, (size_t)chunk * 2 * ((m->Vp + 127) / 128) * sizeof(float2)},
       {(void**)&m->dres_act, (size_t)N * C * ab},
       {(void**)&m->du, (size_t)N * F * ab},
       {(void**)&m->datt, (size_t)N * C * ab},
@@ -604,6 +638,8 @@ int gpt2_step(gpt2* m, float lr, float wd, float beta1, float beta2, float* grad
   a.step_size = (float)(lr / (1.0 - std::pow((double)beta1, (double)m->t)));
   a.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(1.0 - std::pow((double)beta2, (double)m->t)));
   a.gnorm_out = m->d_gnorm;
+  a.sumsq_total = nullptr;
+  a.zero_grad = 1;
   adamw_kernel<<<8 * m->num_sms, ADAM_THREADS, 0, m->stream>>>(a);
   RK(check_launch(c, "adamw"));
   m->k = 0;
@@ -612,6 +648,77 @@ int gpt2_step(gpt2* m, float lr, float wd, float beta1, float beta2, float* grad
     RK(check_device_error(m));
   }
   return GPT2_OK;
+}
+
+int gpt2_grad_sumsq(gpt2* m, int64_t lo, int64_t hi, double* dev_out) {
+  if (!m || !dev_out) return GPT2_ERR_CONFIG;
+  if (lo < 0 || hi < lo || hi > m->n_store || lo % 64 || hi % 64)
+    return set_err(m, GPT2_ERR_CONFIG, "0 <= lo <= hi <= storage length, both multiples of 64");
+  LaunchCtx c = m->ctx();
+  ProfScope ps(c, CAT_ADAMW, 0.0, 4.0 * (double)(hi - lo));
+  sumsq_partial_kernel<<<m->norm_parts, ADAM_THREADS, 0, m->stream>>>(m->g + lo, hi - lo, m->d_norm_part);
+  RK(check_launch(c, "sumsq_partial"));
+  sum_partials_kernel<<<1, 32, 0, m->stream>>>(m->d_norm_part, m->norm_parts, dev_out);
+  return check_launch(c, "sum_partials");
+}
+
+int gpt2_step_range(gpt2* m, float lr, float wd, float beta1, float beta2, int64_t lo, int64_t hi,
+                    const double* dev_sumsq, float* grad_norm_out) {
+  if (!m || !dev_sumsq) return GPT2_ERR_CONFIG;
+  if (lo < 0 || hi < lo || hi > m->n_store || lo % 64 || hi % 64)
+    return set_err(m, GPT2_ERR_CONFIG, "0 <= lo <= hi <= storage length, both multiples of 64");
+  if (m->k == 0) return set_err(m, GPT2_ERR_NO_GRAD, "step without an accumulated micro-batch");
+  LaunchCtx c = m->ctx();
+  m->t += 1;
+  const int64_t n = hi - lo;
+  const int64_t nd = std::min<int64_t>(std::max<int64_t>(m->n_decay - lo, 0), n);
+  {
+    ProfScope ps(c, CAT_ADAMW, 0.0, (double)n * 32 + (m->cfg.dtype == GPT2_BF16 ? 2.0 * nd : 0.0));
+    AdamArgs a{};
+    a.p = m->p + lo;
+    a.g = m->g + lo;
+    a.m = m->m + lo;
+    a.v = m->v + lo;
+    a.shadow = m->cfg.dtype == GPT2_BF16 ? m->shadow + lo : nullptr;
+    a.n = n;
+    a.n_decay = nd;
+    a.partial = nullptr;
+    a.nparts = 0;
+    a.inv_k = 1.0f / (float)m->k;
+    a.lr = lr;
+    a.wd = wd;
+    a.b1 = beta1;
+    a.b2 = beta2;
+    a.step_size = (float)(lr / (1.0 - std::pow((double)beta1, (double)m->t)));
+    a.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(1.0 - std::pow((double)beta2, (double)m->t)));
+    a.gnorm_out = m->d_gnorm;
+    a.sumsq_total = dev_sumsq;
+    a.zero_grad = 0;
+    adamw_kernel<<<8 * m->num_sms, ADAM_THREADS, 0, m->stream>>>(a);
+    RK(check_launch(c, "adamw_range"));
+  }
+  m->k = 0;
+  if (grad_norm_out) {
+    CK(m, cudaMemcpyAsync(grad_norm_out, m->d_gnorm, 4, cudaMemcpyDeviceToHost, m->stream));
+    RK(check_device_error(m));
+  }
+  return GPT2_OK;
+}
+
+int gpt2_param_buffer(gpt2* m, float** dev, int64_t* n) {
+  if (!m || !dev || !n) return GPT2_ERR_CONFIG;
+  *dev = m->p;
+  *n = m->n_store;
+  return GPT2_OK;
+}
+
+int gpt2_refresh_shadow(gpt2* m) {
+  if (!m) return GPT2_ERR_CONFIG;
+  if (m->cfg.dtype != GPT2_BF16) return GPT2_OK;
+  LaunchCtx c = m->ctx();
+  ProfScope ps(c, CAT_ADAMW, 0.0, 6.0 * (double)m->n_decay);
+  cast_shadow_kernel<<<8 * m->num_sms, 256, 0, m->stream>>>(m->p, m->shadow, m->n_decay);
+  return check_launch(c, "cast_shadow");
 }
 
 int gpt2_zero_grad(gpt2* m) {
@@ -954,6 +1061,10 @@ struct OpCtx {
       cudaFreeAsync(d_err, s);
       d_err = nullptr;
     }
+    return sync_and_translate(s, h);
+  }
+  // after a device-to-host copy of the error word into h was enqueued on s
+  static int sync_and_translate(cudaStream_t s, const int& h) {
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) {
       g_op_error = cudaGetErrorString(e);
@@ -966,6 +1077,10 @@ struct OpCtx {
     if (h == DEV_TIMEOUT) {
       g_op_error = "a bounded device-side wait gave up";
       return GPT2_ERR_TIMEOUT;
+    }
+    if (h) {
+      g_op_error = "device error word set";
+      return GPT2_ERR_CUDA;
     }
     return GPT2_OK;
   }
@@ -1081,7 +1196,7 @@ int gpt2_op_layernorm_bwd(int dtype, const float* dy, const float* x, const floa
     g_op_error = "layernorm: C % 4 == 0, C <= 2048, N > 0 required";
     return GPT2_ERR_CONFIG;
   }
-  const int grid = ln_bwd_grid(N);
+  const int grid = ln_bwd_grid(N, C, o.c.num_sms);
   float* part = nullptr;
   if (cudaMallocAsync((void**)&part, (size_t)3 * grid * C * 4, o.s) != cudaSuccess) return GPT2_ERR_OOM;
   int r = dtype == GPT2_BF16
@@ -1100,7 +1215,10 @@ int gpt2_op_attention_fwd(int dtype, const void* qkv, int B, int T, int NH, int 
     g_op_error = "attention: empty shape";
     return GPT2_ERR_CONFIG;
   }
-  return attention_fwd(o.c, dtype, qkv, B, T, NH, hd, out, lse);
+  RK(o.alloc_err());
+  int r = attention_fwd(o.c, dtype, qkv, B, T, NH, hd, out, lse);
+  int r2 = o.finish();
+  return r ? r : r2;
 }
 
 int gpt2_op_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* lse, int B,
@@ -1110,11 +1228,16 @@ int gpt2_op_attention_bwd(int dtype, const void* qkv, const void* out, const voi
     g_op_error = "attention: empty shape";
     return GPT2_ERR_CONFIG;
   }
+  RK(o.alloc_err());
   float* D = nullptr;
-  if (cudaMallocAsync((void**)&D, (size_t)B * NH * T * 4, o.s) != cudaSuccess) return GPT2_ERR_OOM;
+  if (cudaMallocAsync((void**)&D, (size_t)B * NH * T * 4, o.s) != cudaSuccess) {
+    o.finish();
+    return GPT2_ERR_OOM;
+  }
   int r = attention_bwd(o.c, dtype, qkv, out, dout, lse, B, T, NH, hd, dqkv, D);
   cudaFreeAsync(D, o.s);
-  return r;
+  int r2 = o.finish();
+  return r ? r : r2;
 }
 
 int gpt2_op_embedding_fwd(const int32_t* tokens, const float* wte, const float* wpe, int B, int T, int C, int V,
@@ -1182,7 +1305,20 @@ int gpt2_op_cross_entropy(int dtype, void* logits, int64_t ld, int N, int V, con
                           float* row_loss, void* stream) {
   OpCtx o(stream);
   RK(o.alloc_err());
-  int r = cross_entropy(o.c, dtype, logits, ld, N, V, targets, scale, row_loss);
+  int r;
+  if (dtype == GPT2_BF16 && N > 0) {
+    // the training step's bf16 path: per-row softmax partials (here from the logits
+    // themselves), then the one-pass gradient
+    float2* stats = nullptr;
+    if (cudaMallocAsync((void**)&stats, (size_t)N * sizeof(float2), o.s) != cudaSuccess) {
+      o.finish();
+      return GPT2_ERR_OOM;
+    }
+    r = cross_entropy_stats(o.c, (bf16*)logits, ld, N, V, targets, scale, row_loss, nullptr, 0, stats);
+    cudaFreeAsync(stats, o.s);
+  } else {
+    r = cross_entropy(o.c, dtype, logits, ld, N, V, targets, scale, row_loss);
+  }
   int r2 = o.finish();
   return r ? r : r2;
 }
@@ -1200,6 +1336,19 @@ int gpt2_op_sample_topk(const float* logits, int64_t ld, int rows, int V, int k,
   return r ? r : r2;
 }
 
+int gpt2_op_bounded_wait_check(int arrive, unsigned long long limit_ns, void* stream) {
+  if (limit_ns > 1000000000ull) {
+    g_op_error = "bounded_wait_check: limit_ns must be at most 1e9";
+    return GPT2_ERR_CONFIG;
+  }
+  OpCtx o(stream);
+  RK(o.alloc_err());
+  bounded_wait_check_kernel<<<1, 32, 0, o.s>>>(arrive, limit_ns, o.d_err);
+  int r = check_launch(o.c, "bounded_wait_check");
+  int r2 = o.finish();
+  return r ? r : r2;
+}
+
 const char* gpt2_op_last_error(void) { return g_op_error.c_str(); }
 
 }  // extern "C"
@@ -1212,19 +1361,24 @@ const char* gpt2_op_last_error(void) { return g_op_error.c_str(); }
 // therefore may not allocate, or who cannot pay for an allocation per call.
 // Every GPU that loads this library holds the array (4 MiB) until the process
 // exits. All calls on a device share it and each call overwrites all of it that
-// it uses before reading it, so nothing has to be cleared; calls whose kernels
-// overlap on the GPU (different streams, no ordering between them) race on it.
-// The first call on each device looks up the array's device address (with that
-// device current) and caches it; make that first call before any stream capture.
+// it uses before reading it; calls whose kernels overlap on the GPU (different
+// streams or threads, no ordering between them) race on it. A second fixed word
+// carries the kernels' error flag (a bounded wait that gave up): each call clears
+// it before its kernels and reads it back after them, so the call synchronises
+// its stream and reports a timeout like every other entry point.
+// The first call on each device looks up both addresses (with that device
+// current) and caches them; make that first call before any stream capture.
 // ---------------------------------------------------------------------------
 namespace {
 constexpr long long kNoAllocAttnRows = 1LL << 20;  // max B*NH*T
 static __device__ __align__(256) float g_noalloc_attn_D[kNoAllocAttnRows];
+static __device__ __align__(256) int g_noalloc_attn_err;
 std::mutex g_noalloc_mu;
 constexpr int kMaxDevices = 64;
 float* g_noalloc_attn_ptr[kMaxDevices] = {};
+int* g_noalloc_err_ptr[kMaxDevices] = {};
 
-int noalloc_attn_scratch(float** out) {
+int noalloc_attn_scratch(float** out, int** err_out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -1238,14 +1392,18 @@ int noalloc_attn_scratch(float** out) {
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (!g_noalloc_attn_ptr[dev]) {
     void* p = nullptr;
+    void* q = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_attn_D);
-    if (e != cudaSuccess || !p) {
+    if (e == cudaSuccess) e = cudaGetSymbolAddress(&q, g_noalloc_attn_err);
+    if (e != cudaSuccess || !p || !q) {
       g_op_error = std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e);
       return GPT2_ERR_CUDA;
     }
+    g_noalloc_err_ptr[dev] = static_cast<int*>(q);
     g_noalloc_attn_ptr[dev] = static_cast<float*>(p);
   }
   *out = g_noalloc_attn_ptr[dev];
+  *err_out = g_noalloc_err_ptr[dev];
   return GPT2_OK;
 }
 }  // namespace
@@ -1264,6 +1422,22 @@ extern "C" int gpt2_op_attention_bwd_noalloc(int dtype, const void* qkv, const v
     return GPT2_ERR_CONFIG;
   }
   float* D = nullptr;
-  RK(noalloc_attn_scratch(&D));
-  return attention_bwd(o.c, dtype, qkv, out, dout, lse, B, T, NH, hd, dqkv, D);
+  int* err = nullptr;
+  RK(noalloc_attn_scratch(&D, &err));
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), o.s);
+  if (e != cudaSuccess) {
+    g_op_error = std::string("attention_bwd_noalloc: clearing the error word: ") + cudaGetErrorString(e);
+    return GPT2_ERR_CUDA;
+  }
+  o.c.d_err = err;
+  const int r = attention_bwd(o.c, dtype, qkv, out, dout, lse, B, T, NH, hd, dqkv, D);
+  int h = 0;
+  e = cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, o.s);
+  const int r2 = OpCtx::sync_and_translate(o.s, h);
+  if (r) return r;
+  if (e != cudaSuccess) {
+    g_op_error = std::string("attention_bwd_noalloc: reading the error word: ") + cudaGetErrorString(e);
+    return GPT2_ERR_CUDA;
+  }
+  return r2;
 }

@@ -68,20 +68,48 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: while the phase is incomplete the thread may be
+// suspended (it resumes when the phase completes, or after at most about `hint_ns`),
+// so a waiting warp does not take issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity. Gives up after `limit_ns`
-// of wall time (checked every 1024 polls) or as soon as *abort becomes nonzero;
-// returns false in both cases. Never traps.
+// of wall time or as soon as *abort becomes nonzero (both checked after every
+// suspended try of at most ~20 us); returns false in both cases. Never traps.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                   uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 1023u) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > limit_ns) return false;
-    }
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
+}
+
+// One thread: an mbarrier of count 1 that is completed (arrive != 0) or left
+// pending, then the same bounded wait every kernel of the library uses; a wait that
+// gives up raises DEV_TIMEOUT in the error word. Nothing else is in flight, so the
+// check exercises the timeout path without any copy or tensor-core product pending.
+__global__ void bounded_wait_check_kernel(int arrive, unsigned long long limit_ns, int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int no_abort;
+  if (threadIdx.x != 0) return;
+  no_abort = 0;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  if (arrive) mbar_arrive(&bar);
+  if (!mbar_wait_bounded(&bar, 0, &no_abort, limit_ns)) raise_device_error(err, DEV_TIMEOUT);
 }
 
 // ---------------------------------------------------------------------------

@@ -5,7 +5,8 @@
 // For each row n: lse = logsumexp over the first V columns (padding columns V..ld
 // are storage only); row_loss[n] = lse - z[target]; then
 //   z[v] <- (exp(z[v] - lse) - [v == target]) * scale  for v < V,  0 for v >= V.
-// HBM sees each logit once in and once out.
+// HBM sees each logit once in and once out: in bf16 the row statistics come from the
+// producer of the logits (softmax partials), so one streaming pass remains.
 #pragma once
 #include "common.cuh"
 
@@ -32,133 +33,88 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// bf16: persistent, one CTA per SM, rows r = blockIdx.x + k * gridDim.x. Two
-// shared-memory row buffers: row k+1 arrives by a 1-D bulk copy while row k is
-// processed. Each thread keeps a running (max, sum of exp) over its share of the
-// row (one pass), the block combines them, and a second pass writes the gradient
-// row to global memory with coalesced 16-byte stores, so the buffer is free for
-// the next-but-one row as soon as the pass ends. HBM sees each logit once in and
-// once out. ld * 2 bytes per buffer (ld % 8 == 0).
-constexpr int CE_PERSIST_THREADS = 512;
-__global__ void __launch_bounds__(CE_PERSIST_THREADS, 1) cross_entropy_bf16_kernel(
+// bf16, from per-row softmax partials. The producer of the logits leaves, per row, pairs
+// (m_i, s_i) over disjoint column ranges with s_i = sum of exp(z - m_i) over the range's
+// columns < V (the head GEMM's epilogue, or ce_row_stats_kernel). Then
+//   lse = M + ln(sum_i s_i exp(m_i - M)), M = max_i m_i;  row_loss = lse - z[target];
+//   z[v] <- (exp(z[v] - lse) - [v == target]) * scale for v < V, 0 for V <= v < ld,
+// one pass over the row: each logit is read once and written once, with 16-byte
+// accesses, and nothing waits for a row to be staged.
+constexpr int CE_SROWS = 4;       // rows per CTA
+constexpr int CE_STHREADS = 512;
+__global__ void __launch_bounds__(CE_STHREADS) cross_entropy_stats_kernel(
     bf16* __restrict__ logits, long long ld, int V, int rows, const int* __restrict__ tgt, float scale,
-    float* __restrict__ row_loss, int* err, unsigned long long timeout_ns) {
-  extern __shared__ __align__(128) uint8_t ce_smem[];
-  __shared__ float red_m[CE_PERSIST_THREADS / 32], red_s[CE_PERSIST_THREADS / 32];
-  __shared__ __align__(8) uint64_t bar[2];
-  __shared__ int s_abort;
-  const uint32_t row_bytes = (uint32_t)(ld * 2);
-  bf16* buf[2] = {reinterpret_cast<bf16*>(ce_smem), reinterpret_cast<bf16*>(ce_smem + row_bytes)};
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nvec = (int)(ld / 8);
-  if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    s_abort = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-  int row = blockIdx.x;
-  if (tid == 0 && row < rows) {
-    mbar_arrive_expect_tx(&bar[0], row_bytes);
-    bulk_load_1d(buf[0], logits + (long long)row * ld, row_bytes, &bar[0]);
-  }
-  for (int k = 0; row < rows; ++k, row += gridDim.x) {
-    const int cur = k & 1;
-    const int nxt_row = row + gridDim.x;
-    // buf[cur ^ 1] was last read in the previous iteration, which every thread has
-    // finished (the __syncthreads at its end)
-    if (tid == 0 && nxt_row < rows) {
-      fence_proxy_async_smem();  // order the generic reads of that buffer before the async write
-      mbar_arrive_expect_tx(&bar[cur ^ 1], row_bytes);
-      bulk_load_1d(buf[cur ^ 1], logits + (long long)nxt_row * ld, row_bytes, &bar[cur ^ 1]);
+    const float2* __restrict__ stats, int nstats, float* __restrict__ row_loss, int* err) {
+  __shared__ float s_lse2[CE_SROWS];
+  __shared__ int s_tgt[CE_SROWS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long r0 = (long long)blockIdx.x * CE_SROWS;
+  if (warp < CE_SROWS && r0 + warp < rows) {
+    const long long row = r0 + warp;
+    const float2* st = stats + row * nstats;
+    float m = -INFINITY;
+    for (int i = lane; i < nstats; i += 32) m = fmaxf(m, st[i].x);
+    m = warp_max(m);
+    const float m2 = m * LOG2E_CE;
+    float ssum = 0.f;
+    for (int i = lane; i < nstats; i += 32) {
+      const float2 x = st[i];
+      if (x.x != -INFINITY) ssum += x.y * ex2_approx(fmaf(x.x, LOG2E_CE, -m2));
     }
-    if (tid == 0) {
-      int never = 0;
-      if (!mbar_wait_bounded(&bar[cur], (k >> 1) & 1, reinterpret_cast<volatile int*>(&never), timeout_ns)) {
-        raise_device_error(err, DEV_TIMEOUT);
-        s_abort = 1;
-      }
-    }
-    __syncthreads();
-    if (s_abort) break;
-    mbar_try_wait(&bar[cur], (k >> 1) & 1);  // every thread observes the completed phase
-    const bf16* z = buf[cur];
+    ssum = warp_sum(ssum);
     int t = tgt[row];
     if (t < 0 || t >= V) {
-      if (tid == 0) raise_device_error(err, DEV_TOKEN_RANGE);
+      if (lane == 0) raise_device_error(err, DEV_TOKEN_RANGE);
       t = 0;
     }
-    // Three passes over the row in shared memory, one exponential per logit:
-    //   1. the row maximum M (log2 units);
-    //   2. p = 2^(x*log2e - M) and its sum S; p (<= 1) replaces the logit in place as bf16;
-    //   3. dlogits = (p / S - onehot(t)) * scale. The target column is recomputed in fp32,
-    //      since p / S - 1 cancels there.
-    const float xt = __bfloat162float(z[t]) * LOG2E_CE;  // read before pass 2 overwrites it
-    bf16* zw = buf[cur];
-    float m = -INFINITY;
-    for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
-      const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = unpack_bf16x2(w[q]);
-        if (vi * 8 + 2 * q < V) m = fmaxf(m, f.x);
-        if (vi * 8 + 2 * q + 1 < V) m = fmaxf(m, f.y);
-      }
+    const float lse2 = m2 + __log2f(ssum);  // log2 units
+    if (lane == 0) {
+      const float zt = __bfloat162float(logits[row * ld + t]);  // read before the row is overwritten
+      row_loss[row] = (lse2 - zt * LOG2E_CE) * LN2_CE;
+      s_lse2[warp] = lse2;
+      s_tgt[warp] = t;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) red_m[warp] = m;
-    __syncthreads();
-    float M = red_m[0];
-#pragma unroll
-    for (int w = 1; w < CE_PERSIST_THREADS / 32; ++w) M = fmaxf(M, red_m[w]);
-    M *= LOG2E_CE;
-    float sacc = 0.f;
-    for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
-      const uint4 u = reinterpret_cast<const uint4*>(z)[vi];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-      uint32_t o[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = unpack_bf16x2(w[q]);
-        const int c = vi * 8 + 2 * q;
-        const float a = c < V ? ex2_approx(fmaf(f.x, LOG2E_CE, -M)) : 0.f;
-        const float b = c + 1 < V ? ex2_approx(fmaf(f.y, LOG2E_CE, -M)) : 0.f;
-        sacc += a + b;
-        o[q] = pack_bf16x2(a, b);
-      }
-      reinterpret_cast<uint4*>(zw)[vi] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
-    if (lane == 0) red_s[warp] = sacc;
-    __syncthreads();
-    float S = 0.f;
-#pragma unroll
-    for (int w = 0; w < CE_PERSIST_THREADS / 32; ++w) S += red_s[w];
-    const float ll2 = M + __log2f(S);  // lse in the log2 domain
-    if (tid == 0) row_loss[row] = (ll2 - xt) * LN2_CE;
-    const float ps = scale / S;
-    const float dt_val = (ex2_approx(xt - M) / S - 1.f) * scale;
-    bf16* dst = logits + (long long)row * ld;
-    for (int vi = tid; vi < nvec; vi += CE_PERSIST_THREADS) {
-      const uint4 u = reinterpret_cast<const uint4*>(zw)[vi];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-      uint32_t o[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = unpack_bf16x2(w[q]);  // p, zero on padding columns
-        const int c = vi * 8 + 2 * q;
-        const float a = c == t ? dt_val : f.x * ps;
-        const float b = c + 1 == t ? dt_val : f.y * ps;
-        o[q] = pack_bf16x2(a, b);
-      }
-      reinterpret_cast<uint4*>(dst)[vi] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-    __syncthreads();  // everyone is done with buf[cur] and red_* before they are reused
   }
+  __syncthreads();
+  const int nvec = (int)(ld / 8);
+  const int nrows = (int)min((long long)CE_SROWS, (long long)rows - r0);
+  for (int i = threadIdx.x; i < nrows * nvec; i += CE_STHREADS) {
+    const int rr = i / nvec, vi = i - rr * nvec;
+    uint4* ptr = reinterpret_cast<uint4*>(logits + (r0 + rr) * ld) + vi;
+    const uint4 u = *ptr;
+    const float lse2 = s_lse2[rr];
+    const int t = s_tgt[rr];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = unpack_bf16x2(w[q]);
+      const int c = vi * 8 + 2 * q;
+      float a = 0.f, b = 0.f;
+      if (c < V) a = (ex2_approx(fmaf(f.x, LOG2E_CE, -lse2)) - (c == t ? 1.f : 0.f)) * scale;
+      if (c + 1 < V) b = (ex2_approx(fmaf(f.y, LOG2E_CE, -lse2)) - (c + 1 == t ? 1.f : 0.f)) * scale;
+      o[q] = pack_bf16x2(a, b);
+    }
+    *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Softmax partials of whole bf16 rows (one pair per row), for rows whose producer left
+// none: one warp per row, the maximum first, then the sum of exp(z - max) over v < V.
+__global__ void __launch_bounds__(256) ce_row_stats_kernel(const bf16* __restrict__ logits, long long ld, int V,
+                                                           int rows, float2* __restrict__ stats) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const bf16* z = logits + row * ld;
+  float m = -INFINITY;
+  for (int c = lane; c < V; c += 32) m = fmaxf(m, __bfloat162float(z[c]));
+  m = warp_max(m);
+  const float m2 = m * LOG2E_CE;
+  float ssum = 0.f;
+  for (int c = lane; c < V; c += 32) ssum += ex2_approx(fmaf(__bfloat162float(z[c]), LOG2E_CE, -m2));
+  ssum = warp_sum(ssum);
+  if (lane == 0) stats[row] = make_float2(m, ssum);
 }
 
 // fp32 parity mode: exact expf/logf, one CTA per row, strided (rows are short).

@@ -46,6 +46,10 @@ struct GemmParams {
   long long ld_aux;
   int accumulate;
   float* partial;  // split-K workspace [ksplit][M][N] fp32, used when ksplit > 1
+  float* colsum;   // EPI_BF16_DGELU (nullable): column sums of the output per 32-row block, [ceil(M/32)][N]
+  float2* rowstats;  // EPI_BF16 (nullable): per row and half tile, (max, sum of exp(z - max)) of the bf16
+                     // outputs in columns < stats_ncols, [M][2 * tiles_n]
+  int stats_ncols;
   int* err;
   unsigned long long timeout_ns;
 };
@@ -164,7 +168,9 @@ __device__ __forceinline__ void tc_epilogue_chunk(const GemmParams& p, int col0,
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const float2 f = unpack_bf16x2(w[t]);
-        o[t] = pack_bf16x2(v[8 * k + 2 * t] * gelu_tanh_grad_fast(f.x), v[8 * k + 2 * t + 1] * gelu_tanh_grad_fast(f.y));
+        v[8 * k + 2 * t] *= gelu_tanh_grad_fast(f.x);  // kept in v for the column sums
+        v[8 * k + 2 * t + 1] *= gelu_tanh_grad_fast(f.y);
+        o[t] = pack_bf16x2(v[8 * k + 2 * t], v[8 * k + 2 * t + 1]);
       }
       *q = make_uint4(o[0], o[1], o[2], o[3]);
     }
@@ -184,6 +190,24 @@ __device__ __forceinline__ void tc_epilogue_chunk(const GemmParams& p, int col0,
                      pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
     }
   }
+}
+
+// Column sums of a 32 x 32 block held one row per lane (v[j] = column j of the lane's
+// row): after the exchange lane j holds the sum of column j over the 32 rows. Each
+// stage halves the columns a lane keeps and adds its partner's half; the summation
+// order is fixed, so the result is the same on every run.
+__device__ __forceinline__ float warp_colsum32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int j = 0; j < w; ++j) {
+      const float send = upper ? v[j] : v[j + w];
+      const float keep = upper ? v[j + w] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
 }
 
 __device__ __forceinline__ void tc_decode_unit(const GemmParams& p, int unit, int& tm, int& tn, int& ks) {
@@ -436,9 +460,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint32_t acc_phase = 0;
     int n = 0;  // chunks processed by this warp
     bool ok = true;
+    const bool stats = EPI == EPI_BF16 && p.rowstats != nullptr;
     for (int unit = cid; unit < p.num_units && ok; unit += ncl) {
       int tm, tn, ks;
       tc_decode_unit(p, unit, tm, tn, ks);
+      float st_m = -INFINITY, st_s = 0.f;  // this lane's row over this warp's half of the tile
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, lim)) {
         if (lane == 0) {
           raise_device_error(p.err, DEV_TIMEOUT);
@@ -552,6 +578,36 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           continue;
         }
         if (col0 < p.N) tc_epilogue_chunk<EPI, CW>(p, col0, lane, v, cur);
+        if (EPI == EPI_BF16 && stats) {
+          // softmax statistics of the stored (bf16-rounded) values, for the cross-entropy
+          // that reads them: running max and sum of exp(z - max) over columns < stats_ncols
+          float cm = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < CW; ++j) {
+            v[j] = col0 + j < p.stats_ncols ? __bfloat162float(__float2bfloat16_rn(v[j])) : -INFINITY;
+            cm = fmaxf(cm, v[j]);
+          }
+          const float nm = fmaxf(st_m, cm);
+          if (nm != -INFINITY) {
+            const float nm2 = nm * 1.4426950408889634f;
+            float cs = 0.f;
+#pragma unroll
+            for (int j = 0; j < CW; ++j) cs += ex2_fast(fmaf(v[j], 1.4426950408889634f, -nm2));
+            st_s = st_s * ex2_fast((st_m - nm) * 1.4426950408889634f) + cs;
+            st_m = nm;
+          }
+          if (c + CW == c_end && row0 + lane < p.M)
+            p.rowstats[(long long)(row0 + lane) * (2 * p.tiles_n) + tn * 2 + half] = make_float2(st_m, st_s);
+        }
+        if (EPI == EPI_BF16_DGELU && CW == 32 && p.colsum != nullptr && col0 < p.N && row0 < p.M) {
+          // the bias gradient of the layer that produced the GELU input: column sums of this
+          // chunk's 32 rows (rows past M hold zeros), one partial per 32-row block
+          float vv[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) vv[j] = v[j % CW];
+          const float cs = warp_colsum32(vv, lane);
+          if (col0 + lane < p.N) p.colsum[(long long)(row0 >> 5) * p.N + col0 + lane] = cs;
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

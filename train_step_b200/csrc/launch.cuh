@@ -6,7 +6,10 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <map>
+#include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/gpt2.h"
@@ -143,6 +146,40 @@ inline int check_launch(const LaunchCtx& c, const char* what) {
   return GPT2_OK;
 }
 
+// One-time set-up per (device, key), thread-safe. Function attributes such as the
+// dynamic shared-memory opt-in (cudaFuncSetAttribute) apply only on the device that is
+// current when they are set, so each device that launches a kernel needs its own. The
+// value `setup` returns (>= 0) is kept and returned on later calls for that device and
+// key; a negative value is returned without being kept, so the set-up is tried again.
+struct DeviceOnce {
+  std::mutex mu;
+  std::map<std::pair<int, const void*>, int> val;
+};
+inline DeviceOnce& device_once_registry() {
+  static DeviceOnce r;
+  return r;
+}
+template <class F>
+inline int per_device_once(const void* key, F&& setup) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  DeviceOnce& r = device_once_registry();
+  std::lock_guard<std::mutex> lk(r.mu);
+  auto it = r.val.find({dev, key});
+  if (it != r.val.end()) return it->second;
+  const int v = setup();
+  if (v >= 0) r.val[{dev, key}] = v;
+  return v;
+}
+// The dynamic shared-memory opt-in of `kern` on the current device (once per device).
+template <class K>
+inline bool smem_optin(K kern, int bytes) {
+  return per_device_once(reinterpret_cast<const void*>(kern), [&]() -> int {
+           return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess ? 0
+                                                                                                                : -1;
+         }) >= 0;
+}
+
 inline int device_sm_count() {
   int dev = 0, n = 148;
   cudaGetDevice(&dev);
@@ -255,7 +292,15 @@ struct GemmDesc {
   int role = CAT_GEMM;  // profiler category
   int bn = 0;           // tile width: 0 = choose (256 when N >= 256), else 128 or 256
   int pair = -1;        // 2-CTA tiles (256 x 256): -1 = choose, 0 = off, 1 = on (needs BN 256)
+  float* colsum = nullptr;  // EPI_BF16_DGELU: per-32-row-block column sums [ceil(M/32)][N] (nullable)
+  float2* rowstats = nullptr;  // EPI_BF16: softmax partials per row and half tile (nullable)
+  int stats_ncols = 0;         // columns counted by rowstats
 };
+
+// Tile width of a tensor-core GEMM: 256 when N >= 256 unless forced.
+inline int gemm_bn(const GemmDesc& d) { return d.bn == 128 || d.bn == 256 ? d.bn : (d.N >= 256 ? 256 : 128); }
+// Softmax partials per row that a GEMM with rowstats writes.
+inline int gemm_rowstats_count(const GemmDesc& d) { return 2 * ((d.N + gemm_bn(d) - 1) / gemm_bn(d)); }
 
 struct TcMaps {
   CUtensorMap a, b, o, o2;
@@ -265,28 +310,27 @@ template <int BN, bool AM, bool BM_, int EPI, bool PAIR>
 int launch_tc_inst(const LaunchCtx& c, const TcMaps& tm, const GemmParams& p) {
   auto kern = gemm_tc_kernel<BN, AM, BM_, EPI, PAIR>;
   constexpr int smem = TcCfg<BN, PAIR>::SMEM;
-  static int max_clusters = 0;  // co-resident clusters (PAIR), once per instantiation
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return fail(c, GPT2_ERR_CUDA, "cudaFuncSetAttribute(gemm_tc) failed");
-    if (PAIR) {
-      cudaLaunchConfig_t q{};
-      q.gridDim = dim3(2 * (c.num_sms / 2));
-      q.blockDim = dim3(TC_THREADS);
-      q.dynamicSmemBytes = smem;
-      cudaLaunchAttribute qa[1];
-      qa[0].id = cudaLaunchAttributeClusterDimension;
-      qa[0].val.clusterDim.x = 2;
-      qa[0].val.clusterDim.y = 1;
-      qa[0].val.clusterDim.z = 1;
-      q.attrs = qa;
-      q.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &q) != cudaSuccess || max_clusters < 1)
-        return fail(c, GPT2_ERR_CUDA, "gemm_tc: no 2-CTA cluster fits");
-    }
-    attr_set = true;
-  }
+  // shared-memory opt-in and, for pairs, the co-resident clusters: once per device
+  const int max_clusters = per_device_once(reinterpret_cast<const void*>(kern), [&]() -> int {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -1;
+    if (!PAIR) return 0;
+    cudaLaunchConfig_t q{};
+    q.gridDim = dim3(2 * (c.num_sms / 2));
+    q.blockDim = dim3(TC_THREADS);
+    q.dynamicSmemBytes = smem;
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n < 1) return -2;
+    return n;
+  });
+  if (max_clusters == -1) return fail(c, GPT2_ERR_CUDA, "cudaFuncSetAttribute(gemm_tc) failed");
+  if (max_clusters < 0) return fail(c, GPT2_ERR_CUDA, "gemm_tc: no 2-CTA cluster fits");
   if (!PAIR) {
     const int grid = p.num_units < c.num_sms ? p.num_units : c.num_sms;
     kern<<<grid, TC_THREADS, smem, c.stream>>>(tm.a, tm.b, tm.o, tm.o2, p);
@@ -327,7 +371,7 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
   if (d.a_mn && !d.b_mn) return fail(c, GPT2_ERR_CONFIG, "gemm: MN-major A needs MN-major B");
   if ((d.lda % 8) || (d.ldb % 8) || (reinterpret_cast<uintptr_t>(d.A) & 15) || (reinterpret_cast<uintptr_t>(d.B) & 15))
     return fail(c, GPT2_ERR_CONFIG, "gemm: bf16 operands need 16-byte aligned rows");
-  const int BN = d.bn == 128 || d.bn == 256 ? d.bn : (d.N >= 256 ? 256 : 128);
+  const int BN = gemm_bn(d);
   if (d.pair == 1 && BN != 256) return fail(c, GPT2_ERR_CONFIG, "gemm: 2-CTA tiles need tile width 256");
   // 2-CTA tiles halve each SM's B-operand traffic; measured on B200 they lose where a short
   // main loop (K < 1536) meets an epilogue that reads an auxiliary tile (residual / GELU
@@ -379,6 +423,9 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
   p.ld_aux = d.ld_aux;
   p.accumulate = d.accumulate;
   p.partial = ksplit > 1 ? c.splitk_ws : nullptr;
+  p.colsum = d.epi == EPI_BF16_DGELU ? d.colsum : nullptr;
+  p.rowstats = d.epi == EPI_BF16 ? d.rowstats : nullptr;
+  p.stats_ncols = d.stats_ncols;
   p.err = c.d_err;
   p.timeout_ns = 4000000000ull;
   const bool out_f32 = (d.epi == EPI_F32 || d.epi == EPI_F32_RESID);
@@ -498,9 +545,17 @@ int layernorm_fwd_t(const LaunchCtx& c, const float* x, const float* g, const fl
   return check_launch(c, "layernorm_fwd");
 }
 
-inline int ln_bwd_grid(int N) {
-  int g = (N + LN_WARPS - 1) / LN_WARPS;
-  return g < 592 ? g : 592;
+// LayerNorm backward grid: at most the CTAs that are resident at once (each holds
+// LN_WARPS x 3 x C fp32 column accumulators in shared memory), so that no CTA waits
+// for a second wave.
+inline int ln_bwd_grid(int N, int C, int num_sms) {
+  const long long per_cta = (long long)LN_WARPS * 3 * C * 4 + 1024;
+  long long resident = 233472 / per_cta;
+  if (resident > 8) resident = 8;
+  if (resident < 1) resident = 1;
+  const long long cap = resident * num_sms;
+  const long long g = (N + LN_WARPS - 1) / LN_WARPS;
+  return (int)(g < cap ? g : cap);
 }
 
 // out_v (+)= column sums of partial set v, for the non-null outputs out[0..nv).
@@ -516,11 +571,7 @@ template <class T, int NV>
 void launch_ln_bwd(const LaunchCtx& c, int grid, size_t smem, const float* dy, const float* x, const float* g,
                    const float* mean, const float* rstd, float* dres, T* dres_act, int accumulate, float* part,
                    int with_rsum, int N, int C) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(layernorm_bwd_kernel<T, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr = true;
-  }
+  smem_optin(layernorm_bwd_kernel<T, NV>, 200 * 1024);
   layernorm_bwd_kernel<T, NV><<<grid, LN_WARPS * 32, smem, c.stream>>>(dy, x, g, mean, rstd, dres, dres_act,
                                                                        accumulate, part, with_rsum, N, C);
 }
@@ -531,7 +582,7 @@ template <class T>
 int layernorm_bwd_t(const LaunchCtx& c, const float* dy, const float* x, const float* g, const float* mean,
                     const float* rstd, int N, int C, float* dres, T* dres_act, int accumulate,
                     float* part /*3*grid*C*/, float* dg, float* db, float* dbias_next, int accumulate_params) {
-  const int grid = ln_bwd_grid(N);
+  const int grid = ln_bwd_grid(N, C, c.num_sms);
   const int nv = ln_nv(C);
   const int with_rsum = dbias_next != nullptr;
   {
@@ -588,19 +639,14 @@ inline int attention_fwd(const LaunchCtx& c, int dtype, const void* qkv, int B, 
     if (hd != 64) return fail(c, GPT2_ERR_CONFIG, "attention (bf16): head dim must be 64");
     if ((reinterpret_cast<uintptr_t>(qkv) & 15) || (reinterpret_cast<uintptr_t>(out) & 15))
       return fail(c, GPT2_ERR_CONFIG, "attention: qkv and out must be 16-byte aligned");
-    CUtensorMap tq, tkv64, tout;  // Q: 128-row tiles per item; K / V: 64-row tiles per unit
-    if (!encode_qkv_map(&tq, qkv, 3LL * NH * 64, T, B) || !encode_qkv_map(&tkv64, qkv, 3LL * NH * 64, T, B, 64) ||
-        !encode_qkv_map(&tout, out, (long long)NH * 64, T, B))
+    CUtensorMap tqkv, tout;  // 128-row tiles of Q, K and V; 128-row output tiles
+    if (!encode_qkv_map(&tqkv, qkv, 3LL * NH * 64, T, B) || !encode_qkv_map(&tout, out, (long long)NH * 64, T, B))
       return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FF_SMEM);
-      attr_set = true;
-    }
-    // persistent: one CTA per SM loops over (query block, batch*head) items
-    const long long items = (long long)((T + FA_BM - 1) / FA_BM) * B * NH;
+    if (!smem_optin(attn_fwd_tc_kernel, FX_SMEM)) return fail(c, GPT2_ERR_CUDA, "attention: shared-memory opt-in");
+    // persistent: one CTA per SM loops over (pair of query tiles, batch*head) items
+    const long long items = (long long)((T + 255) / 256) * B * NH;
     const int grid = items < c.num_sms ? (int)items : c.num_sms;
-    attn_fwd_tc_kernel<<<grid, FF_THREADS, FF_SMEM, c.stream>>>(tq, tkv64, tout, lse, T, NH, B * NH, scale, c.d_err,
+    attn_fwd_tc_kernel<<<grid, FX_THREADS, FX_SMEM, c.stream>>>(tqkv, tout, lse, T, NH, B * NH, scale, c.d_err,
                                                                 4000000000ull);
     return check_launch(c, "attn_fwd_tc");
   }
@@ -611,8 +657,12 @@ inline int attention_fwd(const LaunchCtx& c, int dtype, const void* qkv, int B, 
   return check_launch(c, "attn_fwd_f32");
 }
 
+// colsum (nullable, bf16 only): the kernels also leave the column sums of dqkv per 32-row
+// block, [B * ceil(T / 128) * 4][3 * NH * hd] (the qkv bias gradient after a reduction).
+inline int attn_colsum_blocks(int B, int T) { return B * ((T + FA_BM - 1) / FA_BM) * 4; }
 inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const void* out, const void* dout,
-                         const float* lse, int B, int T, int NH, int hd, void* dqkv, float* Dbuf) {
+                         const float* lse, int B, int T, int NH, int hd, void* dqkv, float* Dbuf,
+                         float* colsum = nullptr) {
   const float scale = 1.0f / sqrtf((float)hd);
   ProfScope ps(c, CAT_ATTN_BWD, 2.5 * 4.0 * B * NH * hd * (0.5 * T * (T + 1.0)), 0.0);
   const long long warps = (long long)B * NH * T;
@@ -625,28 +675,22 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
                                                                                   Dbuf, B, T, NH);
     int r = check_launch(c, "attn_bwd_dot");
     if (r) return r;
-    CUtensorMap tq, td, tq64, td64, tout;  // 128-row tiles per item, 64-row tiles per streamed unit
+    CUtensorMap tq, td, tout;  // 128-row tiles of qkv, dout and dqkv
     if (!encode_qkv_map(&tq, qkv, 3LL * NH * 64, T, B) || !encode_qkv_map(&td, dout, (long long)NH * 64, T, B) ||
-        !encode_qkv_map(&tq64, qkv, 3LL * NH * 64, T, B, 64) ||
-        !encode_qkv_map(&td64, dout, (long long)NH * 64, T, B, 64) ||
         !encode_qkv_map(&tout, dqkv, 3LL * NH * 64, T, B))
       return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
     if (reinterpret_cast<uintptr_t>(dqkv) & 15) return fail(c, GPT2_ERR_CONFIG, "attention: dqkv must be 16-byte aligned");
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FBK_SMEM);
-      cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FBQ_SMEM);
-      attr_set = true;
-    }
+    if (!smem_optin(attn_bwd_dkdv_tc_kernel, BK_SMEM) || !smem_optin(attn_bwd_dq_tc_kernel, BQ_SMEM))
+      return fail(c, GPT2_ERR_CUDA, "attention: shared-memory opt-in");
     // persistent: one CTA per SM loops over (block, batch*head) items
     const long long items = (long long)((T + FA_BM - 1) / FA_BM) * B * NH;
     const int grid = items < c.num_sms ? (int)items : c.num_sms;
-    attn_bwd_dkdv_tc_kernel<<<grid, FBK_THREADS, FBK_SMEM, c.stream>>>(tq, tq64, td64, tout, lse, Dbuf, T, NH, B * NH,
-                                                                       scale, c.d_err, 4000000000ull);
+    attn_bwd_dkdv_tc_kernel<<<grid, BK_THREADS, BK_SMEM, c.stream>>>(tq, td, tout, lse, Dbuf, colsum, T, NH, B * NH,
+                                                                     scale, c.d_err, 4000000000ull);
     r = check_launch(c, "attn_bwd_dkdv_tc");
     if (r) return r;
-    attn_bwd_dq_tc_kernel<<<grid, FBQ_THREADS, FBQ_SMEM, c.stream>>>(tq, td, tq64, tout, lse, Dbuf, T, NH, B * NH,
-                                                                     scale, c.d_err, 4000000000ull);
+    attn_bwd_dq_tc_kernel<<<grid, BQ_THREADS, BQ_SMEM, c.stream>>>(tq, td, tout, lse, Dbuf, colsum, T, NH, B * NH,
+                                                                   scale, c.d_err, 4000000000ull);
     return check_launch(c, "attn_bwd_dq_tc");
   }
   if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");
@@ -708,11 +752,7 @@ inline int token_sort(const LaunchCtx& c, const int* tok, int N, int V, const Em
   if (V > (1 << 17)) return fail(c, GPT2_ERR_CONFIG, "embedding backward: V must be <= 131072");
   int NP = 1;
   while (NP < N) NP <<= 1;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(token_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, EMB_MAX_TOKENS * 4);
-    attr_set = true;
-  }
+  smem_optin(token_sort_kernel, EMB_MAX_TOKENS * 4);
   token_sort_kernel<<<1, EMB_SORT_THREADS, NP * 4, c.stream>>>(tok, N, V, NP, s.sorted_pos, s.chunk_start, s.seg_id,
                                                               s.seg_chunk0, s.counts, c.d_err);
   return check_launch(c, "token_sort");
@@ -738,26 +778,39 @@ inline int embedding_bwd(const LaunchCtx& c, const int* tok, const float* dx0, i
 // ---------------------------------------------------------------------------
 // cross-entropy
 // ---------------------------------------------------------------------------
+// fp32 parity path (one CTA per row, exact expf / logf); bf16 goes through
+// cross_entropy_stats below.
 inline int cross_entropy(const LaunchCtx& c, int dtype, void* logits, long long ld, int N, int V, const int* tgt,
                          float scale, float* row_loss) {
   if (N <= 0) return GPT2_OK;
-  ProfScope ps(c, CAT_CE, 0.0, 2.0 * N * ld * (dtype == GPT2_BF16 ? 2 : 4));
-  if (dtype == GPT2_BF16) {
-    const long long smem = 2 * ld * 2;
-    if (ld % 8 || smem > 220 * 1024)
-      return fail(c, GPT2_ERR_CONFIG, "cross_entropy: ld must be a multiple of 8 and <= 56320");
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaFuncSetAttribute(cross_entropy_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-      attr_set = true;
-    }
-    const int grid = N < c.num_sms ? N : c.num_sms;
-    cross_entropy_bf16_kernel<<<grid, CE_PERSIST_THREADS, (size_t)smem, c.stream>>>(
-        (bf16*)logits, ld, V, N, tgt, scale, row_loss, c.d_err, 4000000000ull);
-  } else {
-    cross_entropy_f32_kernel<<<N, CE_THREADS, 0, c.stream>>>((float*)logits, ld, V, tgt, scale, row_loss, c.d_err);
-  }
+  if (dtype != GPT2_FP32) return fail(c, GPT2_ERR_CONFIG, "cross_entropy: the bf16 path needs softmax partials");
+  ProfScope ps(c, CAT_CE, 0.0, 2.0 * N * ld * 4);
+  cross_entropy_f32_kernel<<<N, CE_THREADS, 0, c.stream>>>((float*)logits, ld, V, tgt, scale, row_loss, c.d_err);
   return check_launch(c, "cross_entropy");
+}
+
+// bf16 cross-entropy from softmax partials (nstats per row). With stats == nullptr the
+// partials are computed first from the logits themselves (one per row) into `scratch`
+// (rows float2).
+inline int cross_entropy_stats(const LaunchCtx& c, bf16* logits, long long ld, int N, int V, const int* tgt,
+                               float scale, float* row_loss, const float2* stats, int nstats, float2* scratch) {
+  if (N <= 0) return GPT2_OK;
+  if (ld % 8) return fail(c, GPT2_ERR_CONFIG, "cross_entropy: ld must be a multiple of 8");
+  if (!stats) {
+    if (!scratch) return fail(c, GPT2_ERR_CONFIG, "cross_entropy: no softmax partials");
+    {
+      ProfScope ps(c, CAT_CE, 0.0, 2.0 * N * V + 8.0 * N);
+      ce_row_stats_kernel<<<(N + 7) / 8, 256, 0, c.stream>>>(logits, ld, V, N, scratch);
+    }
+    int r = check_launch(c, "ce_row_stats");
+    if (r) return r;
+    stats = scratch;
+    nstats = 1;
+  }
+  ProfScope ps(c, CAT_CE, 0.0, 2.0 * N * ld * 2 + 8.0 * N * nstats);
+  cross_entropy_stats_kernel<<<(N + CE_SROWS - 1) / CE_SROWS, CE_STHREADS, 0, c.stream>>>(
+      logits, ld, V, N, tgt, scale, stats, nstats, row_loss, c.d_err);
+  return check_launch(c, "cross_entropy_stats");
 }
 
 // ---------------------------------------------------------------------------
@@ -777,20 +830,20 @@ void gemv_attrs() {
                        DEC_GEMV_MAX_SMEM);
 }
 
-// Shared-memory limits of every GEMV variant, set once per process before any launch
+// Shared-memory limits of every GEMV variant, set once per device before any launch
 // (and so before a decode step is captured).
 inline void gemv_prepare() {
-  static bool done = false;
-  if (done) return;
-  gemv_attrs<1, false>();
-  gemv_attrs<2, false>();
-  gemv_attrs<4, false>();
-  gemv_attrs<8, false>();
-  gemv_attrs<1, true>();
-  gemv_attrs<2, true>();
-  gemv_attrs<4, true>();
-  gemv_attrs<8, true>();
-  done = true;
+  per_device_once(reinterpret_cast<const void*>(&gemv_prepare), []() -> int {
+    gemv_attrs<1, false>();
+    gemv_attrs<2, false>();
+    gemv_attrs<4, false>();
+    gemv_attrs<8, false>();
+    gemv_attrs<1, true>();
+    gemv_attrs<2, true>();
+    gemv_attrs<4, true>();
+    gemv_attrs<8, true>();
+    return 0;
+  });
 }
 
 template <int KW, bool LN>
@@ -877,13 +930,7 @@ inline int decode_attention(const LaunchCtx& c, const bf16* qkv, bf16* cache, in
   if (S < 1 || S > DEC_MAX_SPLIT || (S > 1 && !part)) return fail(c, GPT2_ERR_CONFIG, "decode attention: splits");
   const size_t smem = (size_t)Tc * 4;
   if (smem > 200 * 1024) return fail(c, GPT2_ERR_SEQ_TOO_LONG, "decode attention: more than 51200 positions");
-  if (smem > 48 * 1024) {
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-      attr_set = true;
-    }
-  }
+  if (smem > 48 * 1024) smem_optin(decode_attn_kernel, 200 * 1024);
   ProfScope ps(c, CAT_DEC_ATTN, 4.0 * B * C * mean_keys, 4.0 * B * C * mean_keys + 10.0 * B * C);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)DEC_HD);
   cudaError_t e = launch_k(c, decode_attn_kernel, dim3(B * NH * S), dim3(DEC_ATT_THREADS), smem, qkv, cache,

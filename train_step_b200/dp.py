@@ -27,3 +27,68 @@ def allreduce_mean_(tensor, group=None) -> None:
     else:
         dist.all_reduce(tensor, op=dist.ReduceOp.SUM, group=group)
         tensor.div_(world)
+
+
+def shard_bounds(n: int, world: int, rank: int) -> tuple[int, int]:
+    """Storage range [lo, hi) of rank `rank`'s shard: W equal pieces, each a multiple of 64
+    floats (the library's storage length is a multiple of 4096)."""
+    if n % (64 * world):
+        raise ValueError(f"storage length {n} does not split into {world} shards of 64-float multiples")
+    shard = n // world
+    return rank * shard, (rank + 1) * shard
+
+
+def reduce_scatter_mean_(tensor, lo: int, hi: int, group=None) -> None:
+    """tensor[lo:hi] <- the average over the ranks of their tensor[lo:hi] (this rank's
+    shard of an equal split). NCCL reduces in place into the shard; gloo, which has no
+    reduce-scatter, all-reduces the whole tensor (the same values in the shard)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    if world == 1:
+        return
+    if dist.get_backend(group) == "nccl":
+        out = torch.empty_like(tensor[lo:hi])
+        dist.reduce_scatter_tensor(out, tensor, op=dist.ReduceOp.AVG, group=group)
+        tensor[lo:hi].copy_(out)
+    else:
+        dist.all_reduce(tensor, op=dist.ReduceOp.SUM, group=group)
+        tensor.div_(world)
+
+
+def all_gather_shards_(tensor, lo: int, hi: int, group=None) -> None:
+    """Every rank's shard tensor[lo_r:hi_r] into every rank's tensor (in place)."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    if world == 1:
+        return
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(tensor, tensor[lo:hi].clone(), group=group)
+    else:
+        parts = [torch.empty_like(tensor[lo:hi]) for _ in range(world)]
+        dist.all_gather(parts, tensor[lo:hi].contiguous(), group=group)
+        torch.cat(parts, out=tensor)
+
+
+def zero1_step(model, lr: float, wd: float, beta1: float = 0.9, beta2: float = 0.95, group=None) -> None:
+    """One optimizer step with the optimizer sharded over the ranks (ZeRO stage 1):
+    reduce-scatter of the accumulated gradients, the global norm from every shard's sum
+    of squares, AdamW on this rank's shard of parameters and moments, all-gather of the
+    updated parameter shards, refresh of the bf16 weight shadow, gradients zeroed. Gives
+    the update of an all-reduce followed by the full step (same clip, same AdamW). All
+    work runs on torch's current stream, which must be the model's stream."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    g = model.grad_tensor()
+    lo, hi = shard_bounds(g.numel(), world, rank)
+    reduce_scatter_mean_(g, lo, hi, group)
+    ss = torch.zeros(1, dtype=torch.float64, device=g.device)
+    model.grad_sumsq(lo, hi, ss)
+    if world > 1:
+        dist.all_reduce(ss, op=dist.ReduceOp.SUM, group=group)
+    model.step_range(lr, wd, beta1, beta2, lo, hi, ss)
+    all_gather_shards_(model.param_tensor(), lo, hi, group)
+    model.refresh_shadow()
+    model.zero_grad()

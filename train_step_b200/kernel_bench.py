@@ -136,6 +136,7 @@ def main() -> None:
     ap.add_argument("--b-mn", action="store_true")
     ap.add_argument("--ksplit", type=int, default=1, help="0 = the library's choice")
     ap.add_argument("--bn", type=int, default=0, help="GEMM tile width: 0 = the library's choice, 128 or 256")
+    ap.add_argument("--pair", type=int, default=-1, help="GEMM 2-CTA tiles: -1 = the library's choice, 0 off, 1 on")
     ap.add_argument("--B", type=int, default=16)
     ap.add_argument("--T", type=int, default=1024)
     ap.add_argument("--H", type=int, default=12)
@@ -165,7 +166,7 @@ def main() -> None:
 
         ms = tsb.gemm_bench(A, B, out, M=M, N=N, K=K, lda=M if a.a_mn else K, ldb=N if a.b_mn else K, ldo=N,
                             a_mn=a.a_mn, b_mn=a.b_mn, epilogue=a.epi, out2=out2, ldo2=N, bias=bias, aux=aux,
-                            ld_aux=N, ksplit=a.ksplit, bn=a.bn, iters=a.iters)
+                            ld_aux=N, ksplit=a.ksplit, bn=a.bn, pair=a.pair, iters=a.iters)
         res.update(shape=[M, N, K], ms=ms, tflops=2.0 * M * N * K / (ms * 1e-3) / 1e12)
     elif a.kernel in ("attn", "attn_bwd"):
         B, T, H, hd = a.B, a.T, a.H, 64
