@@ -288,7 +288,9 @@ int gpt2_op_layernorm_fwd(int dtype, const float* f32_x, const float* f32_g, con
 
 /* LayerNorm backward: f32_dres (+)= dx (accumulate = 1 adds), dres_act (nullable)
  * = copy of the new f32_dres in the activation type, f32_dg and f32_db (+)= the
- * parameter gradients (accumulate_params = 1 adds). */
+ * parameter gradients (accumulate_params = 1 adds). C % 4 == 0, C <= 2048, and the
+ * row arrays (dy, x, g, dres, dres_act) start on 16-byte boundaries; otherwise
+ * GPT2_ERR_CONFIG. */
 int gpt2_op_layernorm_bwd(int dtype, const float* f32_dy, const float* f32_x, const float* f32_g,
                           const float* f32_mean, const float* f32_rstd, int N, int C, float* f32_dres, void* dres_act,
                           int accumulate, float* f32_dg, float* f32_db, int accumulate_params, void* stream);

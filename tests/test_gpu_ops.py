@@ -179,7 +179,8 @@ def test_gemm_fp32_simt(a_mn, b_mn, epi):
 # ---------------------------------------------------------------------------
 # LayerNorm
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("N,C", [(1000, 768), (77, 1600), (512, 128), (16384, 768)])
+@pytest.mark.parametrize("N,C", [(1000, 768), (77, 1600), (512, 128), (16384, 768), (3001, 1024), (5, 768),
+                                 (2371, 256)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_layernorm_fwd_bwd(N, C, dtype):
     x = randn((N, C), 20, torch.float32, scale=2.0) + 0.5
@@ -208,6 +209,30 @@ def test_layernorm_fwd_bwd(N, C, dtype):
     if dres_act is not None:
         assert rel_l2(g64(dres_act), rdx + g64(dres0)) < 4e-3
     assert rel_l2(g64(dg), rdg + 1) < 1e-5 and rel_l2(g64(db), rdb + 1) < 1e-5
+
+
+@pytest.mark.parametrize("N,C", [(1000, 768), (3001, 1024), (77, 1600)])
+def test_layernorm_bwd_overwrite(N, C):
+    """accumulate = 0: dres is overwritten (never read), the parameter grads too."""
+    x = randn((N, C), 25, torch.float32, scale=2.0) - 0.25
+    g = randn((C,), 26, torch.float32) * 0.3 + 1.0
+    b = torch.zeros(C, device=DEV)
+    y = torch.zeros(N, C, dtype=torch.bfloat16, device=DEV)
+    mean = torch.zeros(N, device=DEV)
+    rstd = torch.zeros(N, device=DEV)
+    tsb.layernorm_fwd(x, g, b, y, mean, rstd)
+    dy = randn((N, C), 27, torch.float32)
+    dres = torch.full((N, C), float("nan"), device=DEV)
+    dres_act = torch.zeros(N, C, dtype=torch.bfloat16, device=DEV)
+    dg = torch.full((C,), float("nan"), device=DEV)
+    db = torch.full((C,), float("nan"), device=DEV)
+    tsb.layernorm_bwd(dy, x, g, mean, rstd, dres, dres_act, dg, db, accumulate=False, accumulate_params=False,
+                      dtype=tsb.BF16)
+    torch.cuda.synchronize()
+    rdx, rdg, rdb = oracle.layernorm_bwd(g64(dy), g64(x), g64(g), g64(mean), g64(rstd))
+    assert rel_l2(g64(dres), rdx) < 1e-5
+    assert rel_l2(g64(dres_act), rdx) < 4e-3
+    assert rel_l2(g64(dg), rdg) < 1e-5 and rel_l2(g64(db), rdb) < 1e-5
 
 
 # ---------------------------------------------------------------------------
@@ -378,3 +403,4 @@ def test_cross_entropy(N, V, ld, dtype):
     assert np.max(np.abs(g64(rl) - rrow)) < tol * max(1.0, np.max(np.abs(rrow)))
     assert rel_l2(g64(z), rdl) < (1e-2 if dtype == torch.bfloat16 else 1e-6)
     assert np.all(g64(z)[:, V:] == 0)
+

@@ -89,7 +89,12 @@ def test_step_gemm_at_full_size(name, M, N, K, a_mn, b_mn):
     ref = oracle.linear_fwd(g64(A_rows), g64(B_log))
     got = g64(out[torch.from_numpy(rows).to(DEV)])
     assert np.all(np.isfinite(got))
-    assert rel_l2(got, ref) < 1e-5, name
+    # fp32 accumulation of K exact bf16 products: the rounding error of a length-K sum grows
+    # like sqrt(K) units of 2^-24 (random-walk bound; a factor 4 covers the tensor core's
+    # accumulation order, measured 1.9e-5 at K = 50,304). The per-op bar of 1e-5 stays the
+    # floor for short sums.
+    tol = max(1e-5, 4.0 * (K ** 0.5) * 2.0 ** -24)
+    assert rel_l2(got, ref) < tol, (name, rel_l2(got, ref), tol)
 
 
 # ---------------------------------------------------------------------------

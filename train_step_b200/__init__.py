@@ -522,3 +522,4 @@ def bounded_wait_check(arrive: bool, limit_ns: int, stream=None) -> None:
     """The library's bounded device-side wait on a barrier that is completed (arrive) or
     never completed; raises Gpt2Error(GPT2_ERR_TIMEOUT) when the wait gives up."""
     _op(lib().gpt2_op_bounded_wait_check(int(arrive), int(limit_ns), _stream(stream)))
+

@@ -9,15 +9,15 @@
 // longest first): the forward, and a deterministic backward split into a dK/dV
 // kernel (per key block) and a dQ kernel (per query block). They share one design,
 // set by what B200 measurements showed:
-//  * a thread can issue a 1-SM tcgen05.mma only every ~96 cycles whatever its N,
-//    but the tensor pipe overlaps the streams of several threads, so every product
-//    has its own issuing thread;
-//  * A operands live in TMEM (the item's fixed 128-row tile, and the P / dS tiles
-//    written there by the element-wise warps), so only 64-row B tiles are read from
-//    shared memory;
-//  * each 64-wide unit streams its own 16 KB stage through a deep TMA ring, so a
-//    tile is requested several units before it is needed;
-//  * outputs leave through a shared-memory tile and one TMA store per tile.
+//  * a thread can issue a 1-SM tcgen05.mma only every ~80-150 cycles, while the
+//    tensor pipe overlaps the streams of several threads, so each product (or pair of
+//    products that always run together) has its own issuing thread;
+//  * units are 128 x 128 (128 queries against 128 keys), so every score product runs
+//    at N = 128; the accumulations (P V, dS K and their transposes) run at N = 64;
+//  * P and dS are written to TMEM by the element-wise warps and used there as the A
+//    operand of the following product; tiles are streamed through a TMA ring several
+//    units deep;
+//  * outputs leave through a swizzled shared-memory tile and one TMA store per tile.
 // Every mbarrier wait is bounded (device error word, early exit, no trap).
 #pragma once
 #include "attention.cuh"
@@ -52,8 +52,10 @@ constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 // dV | dK (64 + 64). dQ: S | dP (128 + 128), Q | dO operands (32 + 32), dS (64), dQ for two
 // items (64 + 64). The score tiles are single-buffered: the element-wise warps load them
 // into registers first thing, and the next unit's score products run while they compute.
-// MMA issue: the two score products of a unit come from one thread, and each
-// accumulation product from a thread of its own (lane 0 of its warp).
+// MMA issue: a thread issues one tcgen05.mma every ~80-150 cycles (measured), so each
+// score product has its own issuing thread (lane 0 of its warp); dK/dV's two
+// accumulation products share one thread (a thread each measured slower: 21 warps
+// leave 80 registers per thread and the element-wise code spills).
 // Warps: 0 TMA producer, then the MMA issuers, then 16 element-wise warps: warp w reads
 // TMEM lane quarter w % 4 (32 rows) and column group (w - first) / 4 (32 of the 128
 // unit columns). D = rowsum(dO * O) comes precomputed. Every wait is bounded (device
@@ -64,7 +66,7 @@ constexpr int FB_BARS = 512;
 constexpr int FB_STAGE = 2 * FA_TILE;  // two 128-row tiles: 32 KB
 constexpr uint32_t FB_TMEM_COLS = 512;
 // dK/dV kernel
-constexpr int BK_EW0 = 4;  // producer, score (S^T and dP^T), dV, dK issuers, then element-wise warps
+constexpr int BK_EW0 = 4;  // producer, S^T, dP^T, (dV and dK) issuers, then element-wise warps
 constexpr int BK_THREADS = 32 * (BK_EW0 + FB_EW_WARPS);  // 640
 constexpr int BK_NST = 3;
 constexpr int BK_OFF_KV = 0;                            // K | V [2 items]
@@ -75,8 +77,8 @@ constexpr int BK_OFF_BAR = BK_OFF_OUT + 2 * FA_TILE;
 constexpr int BK_SMEM = BK_OFF_BAR + FB_BARS + 1024;
 constexpr uint32_t BK_TM_DP = 128, BK_TM_P = 256, BK_TM_DS = 320, BK_TM_DV = 384, BK_TM_DK = 448;
 // dQ kernel
-constexpr int BQ_EW0 = 3;  // producer, score (S and dP), dQ issuers, then element-wise warps
-constexpr int BQ_THREADS = 32 * (BQ_EW0 + FB_EW_WARPS);  // 608
+constexpr int BQ_EW0 = 4;  // producer, S, dP, dQ issuers, then element-wise warps
+constexpr int BQ_THREADS = 32 * (BQ_EW0 + FB_EW_WARPS);  // 640
 constexpr int BQ_NST = 4;
 constexpr int BQ_OFF_QD = 0;                            // Q | dO [2 items]
 constexpr int BQ_OFF_ST = 4 * FA_TILE;                  // stages: K_j | V_j
@@ -167,14 +169,14 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BK_OFF_BAR);
   uint64_t* kv_full = bar;                    // [2] K / V tiles landed
-  uint64_t* kv_empty = kv_full + 2;           // [2] the item's S^T / dP^T products are complete
+  uint64_t* kv_empty = kv_full + 2;           // [2] the item's S^T / dP^T products are complete (2 commits)
   uint64_t* st_full = kv_empty + 2;           // [BK_NST] Q_i / dO_i landed, lse / D staged (32 producer lanes)
   uint64_t* st_empty = st_full + BK_NST;      // [BK_NST] the unit's dV and dK products are complete
-  uint64_t* s_full = st_empty + BK_NST;       // S^T and dP^T complete
+  uint64_t* s_full = st_empty + BK_NST;       // S^T and dP^T complete (2 commits)
   uint64_t* s_empty = s_full + 1;             // both read into registers (16 warps)
   uint64_t* p_full = s_empty + 1;             // P^T and dS^T written (16 warps)
-  uint64_t* p_free = p_full + 1;              // the dV and dK products have read them (2 commits)
-  uint64_t* acc_full = p_free + 1;            // the item's dV and dK complete (2 commits)
+  uint64_t* p_free = p_full + 1;              // the dV and dK products have read them
+  uint64_t* acc_full = p_free + 1;            // the item's dV and dK complete
   uint64_t* acc_empty = acc_full + 1;         // dV and dK read by the epilogue (16 warps)
   uint64_t* out_full = acc_empty + 1;         // output tiles staged (16 warps)
   uint64_t* out_free = out_full + 1;          // the previous item's TMA stores have read the staging
@@ -192,17 +194,17 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&kv_empty[i], 2);
     }
     for (int i = 0; i < BK_NST; ++i) {
       mbar_init(&st_full[i], 32);
-      mbar_init(&st_empty[i], 2);
+      mbar_init(&st_empty[i], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(s_full, 2);
     mbar_init(s_empty, FB_EW_WARPS);
     mbar_init(p_full, FB_EW_WARPS);
-    mbar_init(p_free, 2);
-    mbar_init(acc_full, 2);
+    mbar_init(p_free, 1);
+    mbar_init(acc_full, 1);
     mbar_init(acc_empty, FB_EW_WARPS);
     mbar_init(out_full, FB_EW_WARPS);
     mbar_init(out_free, 1);
@@ -278,9 +280,10 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
         if ((st_iss >> i) & 1u)
           mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
-      // ---------------- score MMAs: S^T = K Q_i^T, then dP^T = V dO_i^T ----------------
+      // ---------------- score MMAs: S^T = K Q_i^T (warp 1), dP^T = V dO_i^T (warp 2) ----------------
+      const int part = warp - 1;
       constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
       bool ok = true, any = false;
       int U = 0;
@@ -292,7 +295,8 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
           ok = false;
           break;
         }
-        const uint32_t kv_addr = smem_u32(sm + BK_OFF_KV + kvb * 2 * FA_TILE);
+        // A = K (part 0) or V (part 1): descriptor of k-step kk = base + 2 kk (32 bytes)
+        const uint64_t a_desc = make_sw128_desc(smem_u32(sm + BK_OFF_KV + kvb * 2 * FA_TILE + part * FA_TILE), 16, 1024);
         for (int u = 0; u < nu; ++u, ++U) {
           const int s = U % BK_NST;
           if (!mbar_wait_bounded(&st_full[s], (U / BK_NST) & 1, abort_flag, lim) ||
@@ -301,14 +305,11 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t st_addr = smem_u32(sm + BK_OFF_ST + s * FB_STAGE);
-          // part 0: A = K, B = Q_i -> S^T; part 1: A = V, B = dO_i -> dP^T
+          // B = Q_i (part 0) or dO_i (part 1)
+          const uint64_t b_desc = make_sw128_desc(smem_u32(sm + BK_OFF_ST + s * FB_STAGE + part * FA_TILE), 16, 1024);
 #pragma unroll
-          for (int part = 0; part < 2; ++part)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(tmem + part * BK_TM_DP, make_sw128_desc(kv_addr + part * FA_TILE + kk * 32, 16, 1024),
-                        make_sw128_desc(st_addr + part * FA_TILE + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem + part * BK_TM_DP, a_desc + 2 * kk, b_desc + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
           umma_commit(s_full);
           any = true;
         }
@@ -319,15 +320,14 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
         *abort_flag = 1;
         if (any) {  // wait for the MMAs already issued before the TMEM is freed
           int never = 0;
-          umma_commit(&drain[0]);
-          mbar_wait_bounded(&drain[0], 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[part]);
+          mbar_wait_bounded(&drain[part], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp == 3) {
     if (lane == 0) {
-      // ---------------- accumulation MMAs: dV += P^T dO_i (warp 2), dK += dS^T Q_i (warp 3) ----------------
-      const int part = warp - 2;
+      // ---------------- accumulation MMAs: dV += P^T dO_i, then dK += dS^T Q_i ----------------
       constexpr uint32_t idesc_a = make_idesc_bf16(128, 64, false, true);  // B = dO_i / Q_i, MN-major
       bool ok = true, any = false;
       int U = 0;
@@ -348,15 +348,18 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
             break;
           }
           tc_fence_after();
-          // K = 128 queries: A = P^T (part 0) or dS^T (part 1), 8 TMEM columns per 16 queries;
-          // B = 16 query rows of dO_i (part 0) or Q_i (part 1) per step
-          const uint32_t b_addr = smem_u32(sm + BK_OFF_ST + s * FB_STAGE + (1 - part) * FA_TILE);
-          const uint32_t a_tm = tmem + (part == 0 ? BK_TM_P : BK_TM_DS);
-          const uint32_t acc = tmem + (part == 0 ? BK_TM_DV : BK_TM_DK);
+          // K = 128 queries: A = P^T (dV) or dS^T (dK), 8 TMEM columns per 16 queries; B = 16
+          // query rows of dO_i (dV) or Q_i (dK) per step, descriptor base + 128 kk (2 KB)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16_ts(acc, a_tm + kk * 8, make_sw128_desc(b_addr + kk * 2048, 8192, 1024), idesc_a,
-                         (u > 0 || kk > 0) ? 1u : 0u);
+          for (int part = 0; part < 2; ++part) {
+            const uint64_t b_desc =
+                make_sw128_desc(smem_u32(sm + BK_OFF_ST + s * FB_STAGE + (1 - part) * FA_TILE), 8192, 1024);
+            const uint32_t a_tm = tmem + (part == 0 ? BK_TM_P : BK_TM_DS);
+            const uint32_t acc = tmem + (part == 0 ? BK_TM_DV : BK_TM_DK);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_bf16_ts(acc, a_tm + kk * 8, b_desc + 128 * kk, idesc_a, (u > 0 || kk > 0) ? 1u : 0u);
+          }
           any = true;
           umma_commit(p_free);
           umma_commit(&st_empty[s]);  // the unit's score products completed before P^T was written
@@ -368,8 +371,8 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
         *abort_flag = 1;
         if (any) {
           int never = 0;
-          umma_commit(&drain[1 + part]);
-          mbar_wait_bounded(&drain[1 + part], 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[2]);
+          mbar_wait_bounded(&drain[2], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
@@ -523,7 +526,7 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
   uint64_t* qa_full = qd_empty + 2;           // the Q / dO A operands are written to TMEM (16 warps)
   uint64_t* st_full = qa_full + 1;            // [BQ_NST]
   uint64_t* st_empty = st_full + BQ_NST;      // [BQ_NST]
-  uint64_t* s_full = st_empty + BQ_NST;       // S and dP complete
+  uint64_t* s_full = st_empty + BQ_NST;       // S and dP complete (2 commits)
   uint64_t* s_empty = s_full + 1;             // both read into registers (16 warps)
   uint64_t* ds_full = s_empty + 1;            // dS written (16 warps)
   uint64_t* ds_free = ds_full + 1;            // the dQ product has read it
@@ -531,9 +534,9 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
   uint64_t* acc_empty = acc_full + 2;         // [2] read by the epilogue (16 warps)
   uint64_t* out_full = acc_empty + 2;         // output tile staged (16 warps)
   uint64_t* out_free = out_full + 1;          // the previous item's TMA store has read the staging
-  uint64_t* drain = out_free + 1;             // [2]: one per MMA thread (abort path)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 3);
+  uint64_t* drain = out_free + 1;             // [3]: one per MMA thread (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = NH * 64;
@@ -554,13 +557,13 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
       mbar_init(&st_full[i], 1);
       mbar_init(&st_empty[i], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(s_full, 2);
     mbar_init(s_empty, FB_EW_WARPS);
     mbar_init(ds_full, FB_EW_WARPS);
     mbar_init(ds_free, 1);
     mbar_init(out_full, FB_EW_WARPS);
     mbar_init(out_free, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&drain[i], 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&drain[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -623,9 +626,10 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
             mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
-      // ---------------- score MMAs: S = Q K_j^T, then dP = dO V_j^T; A from TMEM ----------------
+      // ---------------- score MMAs: S = Q K_j^T (warp 1), dP = dO V_j^T (warp 2); A from TMEM ----------------
+      const int part = warp - 1;
       constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
       bool ok = true, any = false;
       int U = 0;
@@ -645,14 +649,12 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
             break;
           }
           tc_fence_after();
-          // part 0: A = Q, B = K_j -> S; part 1: A = dO, B = V_j -> dP (B: 128 rows, K-major)
-          const uint32_t st_addr = smem_u32(sm + BQ_OFF_ST + s * FB_STAGE);
+          // B = K_j (part 0) or V_j (part 1): 128 rows, K-major
+          const uint64_t b_desc = make_sw128_desc(smem_u32(sm + BQ_OFF_ST + s * FB_STAGE + part * FA_TILE), 16, 1024);
 #pragma unroll
-          for (int part = 0; part < 2; ++part)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16_ts(tmem + part * BQ_TM_DP, tmem + BQ_TM_Q + part * 32 + kk * 8,
-                           make_sw128_desc(st_addr + part * FA_TILE + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ts(tmem + part * BQ_TM_DP, tmem + BQ_TM_Q + part * 32 + kk * 8, b_desc + 2 * kk, idesc_s,
+                         kk > 0 ? 1u : 0u);
           umma_commit(s_full);
           any = true;
         }
@@ -662,12 +664,12 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
         *abort_flag = 1;
         if (any) {
           int never = 0;
-          umma_commit(&drain[0]);
-          mbar_wait_bounded(&drain[0], 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[part]);
+          mbar_wait_bounded(&drain[part], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
-  } else if (warp == 2) {
+  } else if (warp == 3) {
     if (lane == 0) {
       // ---------------- accumulation MMAs: dQ += dS K_j (A = dS from TMEM) ----------------
       constexpr uint32_t idesc_q = make_idesc_bf16(128, 64, false, true);  // B = K_j, MN-major
@@ -689,13 +691,12 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm + BQ_OFF_ST + s * FB_STAGE);
+          const uint64_t k_desc = make_sw128_desc(smem_u32(sm + BQ_OFF_ST + s * FB_STAGE), 8192, 1024);
           const uint32_t acc = tmem + BQ_TM_ACC + (uint32_t)(ab * 64);
           // K = 128 keys: A = dS (8 TMEM columns per 16 keys), B = 16 key rows of K_j per step
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_bf16_ts(acc, tmem + BQ_TM_DS + kk * 8, make_sw128_desc(k_addr + kk * 2048, 8192, 1024), idesc_q,
-                         (u > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_ts(acc, tmem + BQ_TM_DS + kk * 8, k_desc + 128 * kk, idesc_q, (u > 0 || kk > 0) ? 1u : 0u);
           any = true;
           umma_commit(ds_free);
           umma_commit(&st_empty[s]);  // the unit's score products completed before dS was written
@@ -707,8 +708,8 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
         *abort_flag = 1;
         if (any) {
           int never = 0;
-          umma_commit(&drain[1]);
-          mbar_wait_bounded(&drain[1], 0, reinterpret_cast<volatile int*>(&never), lim);
+          umma_commit(&drain[2]);
+          mbar_wait_bounded(&drain[2], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
@@ -878,29 +879,30 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
 // the causal lengths. Keys come in blocks of 128: tile t needs blocks 0 .. 2 qp + t,
 // the last being its diagonal; each block's K and V are loaded once per item for both
 // tiles.
-//   S_t  = Q_t K_j^T   (M=128 queries, N=128 keys, K=64;     A = Q_t in TMEM, B = K_j)
+//   S_t  = Q_t K_j^T   (M=128 queries, N=128 keys, K=64;     A = Q_t, B = K_j from shared memory)
 //   O_t += P_t V_j     (M=128 queries, N=64,       K=128 keys; A = P_t in TMEM, B = V_j)
 // One softmax warpgroup per tile, one query row per thread: running max with a lazy
 // re-base (only when a block maximum exceeds it by more than 8 in log2 units: the
 // probabilities against the stale maximum stay <= 2^8, exact in fp32 and bf16, and O
-// and the row sum keep one reference), row sum, and P written as bf16 over the first
-// half of S_t's own TMEM columns; so S_t of the next block is issued once P_t V_j has
-// completed. The two tiles interleave: while one warpgroup exponentiates, the tensor
-// core computes the other tile's products.
+// and the row sum keep one reference), row sum, P as bf16 pairs in the tile's own TMEM
+// columns. S_t has its own columns too, so S_t of the next block is computed while the
+// warpgroup exponentiates this one, and P_t V of this block runs while the warpgroup
+// exponentiates the next; the warpgroup waits for P_t V only before it writes P_t again
+// (and rescales O_t). The two tiles interleave on the tensor core.
 // Warps: 0 TMA producer, 1 S MMAs (and the TMEM allocation), 2 P V MMAs, 3-6 softmax
 // of tile 0, 7-10 softmax of tile 1. Every wait is bounded (device error word, no trap).
 // ---------------------------------------------------------------------------
 constexpr int FX_THREADS = 352;
 constexpr int FX_NST = 4;                                 // K/V stages
 constexpr int FX_STAGE = 2 * FA_TILE;                     // K_j | V_j: 32 KB
-constexpr int FX_OFF_Q = 0;                               // the item's two Q tiles
-constexpr int FX_OFF_ST = 2 * FA_TILE;
+constexpr int FX_OFF_Q = 0;                               // [2 items] the item's two Q tiles
+constexpr int FX_OFF_ST = 4 * FA_TILE;
 constexpr int FX_OFF_OUT = FX_OFF_ST + FX_NST * FX_STAGE;  // output staging, one tile per warpgroup
 constexpr int FX_OFF_BAR = FX_OFF_OUT + 2 * FA_TILE;
 constexpr int FX_SMEM = FX_OFF_BAR + FB_BARS + 1024;
 static_assert(FX_SMEM <= 232448, "shared memory per CTA");
-// TMEM: S_t (P_t over its first 64 columns) at 128 t, O_t at 256 + 64 t, Q_t at 384 + 32 t
-constexpr uint32_t FX_TM_O = 256, FX_TM_Q = 384, FX_TMEM_COLS = 512;
+// TMEM: S_t at 128 t, P_t (bf16 pairs) at 256 + 64 t, O_t at 384 + 64 t
+constexpr uint32_t FX_TM_P = 256, FX_TM_O = 384, FX_TMEM_COLS = 512;
 constexpr float FX_REBASE = 8.0f;
 
 __global__ void __launch_bounds__(FX_THREADS, 1)
@@ -910,13 +912,13 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
   extern __shared__ uint8_t fx_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fx_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + FX_OFF_BAR);
-  uint64_t* q_full = bar;                  // the item's Q tiles landed
-  uint64_t* q_empty = q_full + 1;          // both warpgroups copied them (8 warps)
-  uint64_t* qa_full = q_empty + 1;         // [tile] Q_t written to TMEM (4 warps)
-  uint64_t* st_full = qa_full + 2;         // [FX_NST]
+  uint64_t* q_full = bar;                  // [2 items] the item's Q tiles landed
+  uint64_t* q_empty = q_full + 2;          // [2 items] the item's S products are complete
+  uint64_t* st_full = q_empty + 2;         // [FX_NST]
   uint64_t* st_empty = st_full + FX_NST;   // [FX_NST]
   uint64_t* s_full = st_empty + FX_NST;    // [tile] S_t complete
-  uint64_t* p_full = s_full + 2;           // [tile] P_t written (4 warps)
+  uint64_t* s_empty = s_full + 2;          // [tile] S_t read into registers (4 warps)
+  uint64_t* p_full = s_empty + 2;          // [tile] P_t written (4 warps)
   uint64_t* pv_done = p_full + 2;          // [tile] P_t V_j complete
   uint64_t* o_read = pv_done + 2;          // [tile] O_t read by the epilogue (4 warps)
   uint64_t* out_full = o_read + 2;         // [tile] output tile staged (4 warps)
@@ -924,7 +926,7 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
   uint64_t* drain = out_free + 2;          // [2]: one per MMA thread (abort path)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 3);
-  static_assert((2 + 2 + 2 * FX_NST + 2 * 7 + 3) * 8 <= FB_BARS, "barrier space");
+  static_assert((4 + 2 * FX_NST + 2 * 8 + 3) * 8 <= FB_BARS, "barrier space");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = NH * 64;
@@ -934,11 +936,11 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
   const uint64_t lim = timeout_ns;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 8);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&qa_full[i], 4);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 4);
       mbar_init(&p_full[i], 4);
       mbar_init(&pv_done[i], 1);
       mbar_init(&o_read[i], 4);
@@ -966,24 +968,26 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
     if (lane == 0) {
       // ---------------- producer: Q tiles per item, (K_j, V_j) per block ----------------
       tma_prefetch_desc(&tm_qkv);
-      bool ok = true, q_iss = false;
-      uint32_t q_par = 0, st_iss = 0, st_par = 0;
+      bool ok = true;
+      uint32_t q_iss = 0, q_par = 0, st_iss = 0, st_par = 0;
       int J = 0;  // block loads over all items (stage uses)
       for (int k = 0; ok; ++k) {
         const int item = fx_item(k, cta, G);
         if (item >= nitems) break;
         const int qp = nqp - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
         const int nb = qp * 256 + 128 < T ? 2 * qp + 2 : 2 * qp + 1;
-        // one Q buffer: free once both warpgroups copied the previous item's tiles to TMEM
-        if (k > 0 && !mbar_wait_bounded(q_empty, (k - 1) & 1, abort_flag, lim)) {
+        const int qb = k & 1;
+        // the Q buffer is free once the S products of the item two rounds back completed
+        if (!mbar_wait_bounded(&q_empty[qb], ((k >> 1) & 1) ^ 1, abort_flag, lim)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(q_full, 2 * FA_TILE);
-        tma_load_3d(sm + FX_OFF_Q, &tm_qkv, q_full, h * 64, qp * 256, b);
-        tma_load_3d(sm + FX_OFF_Q + FA_TILE, &tm_qkv, q_full, h * 64, qp * 256 + 128, b);
-        q_iss = true;
-        q_par = k & 1;
+        uint8_t* qd = sm + FX_OFF_Q + qb * 2 * FA_TILE;
+        mbar_arrive_expect_tx(&q_full[qb], 2 * FA_TILE);
+        tma_load_3d(qd, &tm_qkv, &q_full[qb], h * 64, qp * 256, b);
+        tma_load_3d(qd + FA_TILE, &tm_qkv, &q_full[qb], h * 64, qp * 256 + 128, b);
+        q_iss |= 1u << qb;
+        q_par = (q_par & ~(1u << qb)) | ((uint32_t)((k >> 1) & 1) << qb);
         for (int j = 0; j < nb; ++j, ++J) {
           const int s = J % FX_NST;
           const uint32_t ph = (uint32_t)((J / FX_NST) & 1);
@@ -1003,7 +1007,9 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
         int never = 0;  // let the copies in flight land before the CTA's shared memory goes away
-        if (q_iss) mbar_wait_bounded(q_full, q_par, reinterpret_cast<volatile int*>(&never), lim);
+        for (int i = 0; i < 2; ++i)
+          if ((q_iss >> i) & 1u)
+            mbar_wait_bounded(&q_full[i], (q_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
         for (int i = 0; i < FX_NST; ++i)
           if ((st_iss >> i) & 1u)
             mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
@@ -1024,6 +1030,12 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
         const bool v1 = qp * 256 + 128 < T;
         const int nbt[2] = {2 * qp + 1, v1 ? 2 * qp + 2 : 0};
         const int nb = v1 ? nbt[1] : nbt[0];
+        const int qb = k & 1;
+        if (is_s && !mbar_wait_bounded(&q_full[qb], (k >> 1) & 1, abort_flag, lim)) {
+          ok = false;
+          break;
+        }
+        const uint32_t q_addr = smem_u32(sm + FX_OFF_Q + qb * 2 * FA_TILE);
         for (int j = 0; j < nb && ok; ++j, ++J) {
           const int s = J % FX_NST;
           if (!mbar_wait_bounded(&st_full[s], (J / FX_NST) & 1, abort_flag, lim)) {
@@ -1034,18 +1046,16 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
           for (int t = 0; t < 2; ++t) {
             if (j >= nbt[t]) continue;
             if (is_s) {
-              // Q_t of this item is in TMEM; the previous P_t V product (the last reader of
-              // S_t's columns) is complete
-              if ((j == 0 && !mbar_wait_bounded(&qa_full[t], ni[t] & 1, abort_flag, lim)) ||
-                  (n[t] > 0 && !mbar_wait_bounded(&pv_done[t], (n[t] - 1) & 1, abort_flag, lim))) {
+              // the softmax warpgroup has read the previous S_t into registers
+              if (n[t] > 0 && !mbar_wait_bounded(&s_empty[t], (n[t] - 1) & 1, abort_flag, lim)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
+              const uint64_t qd = make_sw128_desc(q_addr + t * FA_TILE, 16, 1024), kd = make_sw128_desc(k_addr, 16, 1024);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                umma_bf16_ts(tmem + t * 128, tmem + FX_TM_Q + t * 32 + kk * 8,
-                             make_sw128_desc(k_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                umma_bf16(tmem + t * 128, qd + 2 * kk, kd + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
               umma_commit(&s_full[t]);
             } else {
               // the epilogue has read O_t of the tile's previous item; P_t is written
@@ -1056,10 +1066,11 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
               }
               tc_fence_after();
               // K = 128 keys: A = P_t (8 TMEM columns per 16 keys), B = 16 key rows of V_j per step
+              const uint64_t vd = make_sw128_desc(v_addr, 8192, 1024);
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                umma_bf16_ts(tmem + FX_TM_O + t * 64, tmem + t * 128 + kk * 8,
-                             make_sw128_desc(v_addr + kk * 2048, 8192, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                umma_bf16_ts(tmem + FX_TM_O + t * 64, tmem + FX_TM_P + t * 64 + kk * 8, vd + 128 * kk, idesc_o,
+                             (j > 0 || kk > 0) ? 1u : 0u);
               umma_commit(&pv_done[t]);
             }
             ++n[t];
@@ -1068,6 +1079,8 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
           // the block's stage is free once its last P V product completes
           if (ok && !is_s) umma_commit(&st_empty[s]);
         }
+        // the item's Q buffer is free once its last S product completes
+        if (ok && is_s) umma_commit(&q_empty[qb]);
         if (v1) ++ni[1];
         ++ni[0];
       }
@@ -1087,40 +1100,20 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t tm_s = tmem + lane_off + (uint32_t)(t * 128);
+    const uint32_t tm_p = tmem + lane_off + FX_TM_P + (uint32_t)(t * 64);
     const uint32_t tm_o = tmem + lane_off + FX_TM_O + (uint32_t)(t * 64);
     const float sl2 = scale * LOG2E;
     const bool issuer = (warp == 3 + 4 * t && lane == 0);  // issues the tile's TMA stores
     uint8_t* stage_out = sm + FX_OFF_OUT + t * FA_TILE;
     bool fail = false;
-    // Q_t of item round k into the TMEM A operand (both warpgroups release the smem tiles)
-    auto copy_q = [&](int k, bool valid) -> bool {
-      if (!fb_warp_wait(q_full, k & 1, abort_flag, lim, lane)) return false;
-      if (valid) {
-        const uint8_t* qt = sm + FX_OFF_Q + t * FA_TILE;
-#pragma unroll
-        for (int cg = 0; cg < 4; ++cg) fb_row_to_tmem(qt, r, cg, tmem + lane_off + FX_TM_Q + t * 32 + cg * 8);
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (valid) mbar_arrive(&qa_full[t]);
-        mbar_arrive(q_empty);
-      }
-      return true;
-    };
-    auto valid_of = [&](int item) { return t == 0 || (nqp - 1 - item / BH) * 256 + 128 < T; };
     int n = 0, ni = 0;  // products of this tile; valid items of this tile
-    {
-      const int item0 = fx_item(0, cta, G);
-      if (item0 < nitems) fail = !copy_q(0, valid_of(item0));
-    }
     for (int k = 0; !fail; ++k) {
       const int item = fx_item(k, cta, G);
       if (item >= nitems) break;
       const int qp = nqp - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
-      const bool valid = valid_of(item);
-      const int nb = valid ? 2 * qp + t + 1 : 0;
+      const bool valid = t == 0 || qp * 256 + 128 < T;
+      if (!valid) continue;
+      const int nb = 2 * qp + t + 1;
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < nb; ++j, ++n) {
         if (!fb_warp_wait(&s_full[t], n & 1, abort_flag, lim, lane)) {
@@ -1133,6 +1126,9 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
         for (int i = 0; i < 4; ++i)
           tmem_ld_32x32b_x32(tm_s + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * i]));
         tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[t]);  // the next S_t may be computed
         if (j == nb - 1) {  // the diagonal block: keys after the query get -inf
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -1151,9 +1147,27 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
         const bool rebase = m_blk > m_run + FX_REBASE;
         const float m_use = rebase ? m_blk : m_run;
         const float m_ref = m_use == -INFINITY ? 0.f : m_use;
-        // rows that re-base rescale their O_t row (complete: S_t of this block was issued
-        // after the previous P_t V product finished); tcgen05.ld / st are warp-collective,
-        // so the whole warp takes this path when any of its rows needs it
+        // P = 2^(s * scale * log2e - m_ref) and the row sum, in registers as bf16 pairs
+        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint32_t pw[64];
+#pragma unroll
+        for (int e2 = 0; e2 < 64; ++e2) {
+          const float p0 = ex2_fast(fmaf(__uint_as_float(sv[2 * e2]), sl2, -m_ref));
+          const float p1 = ex2_fast(fmaf(__uint_as_float(sv[2 * e2 + 1]), sl2, -m_ref));
+          rs8[(2 * e2) & 7] += p0;
+          rs8[(2 * e2 + 1) & 7] += p1;
+          pw[e2] = pack_bf16x2(p0, p1);
+        }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        // the previous P_t V product has completed: P_t may be overwritten and O_t is final
+        // for the previous block
+        if (j > 0 && !fb_warp_wait(&pv_done[t], (n - 1) & 1, abort_flag, lim, lane)) {
+          fail = true;
+          break;
+        }
+        tc_fence_after();
+        // rows that re-base rescale their O_t row; tcgen05.ld / st are warp-collective, so
+        // the whole warp takes this path when any of its rows needs it
         const bool my_rescale = rebase && m_run != -INFINITY;
         const float corr = my_rescale ? ex2_fast(m_run - m_use) : 1.0f;
         if (__any_sync(0xffffffffu, my_rescale)) {
@@ -1172,23 +1186,8 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
             tmem_st_32x32b_x16(tm_o + hh * 32 + 16, c2);
           }
         }
-        // P = 2^(s * scale * log2e - m_ref), row sum, bf16 pairs over S_t's first 64 columns
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t pw[16];
-#pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            const int c = ch * 32 + 2 * e2;
-            const float p0 = ex2_fast(fmaf(__uint_as_float(sv[c]), sl2, -m_ref));
-            const float p1 = ex2_fast(fmaf(__uint_as_float(sv[c + 1]), sl2, -m_ref));
-            rs8[c & 7] += p0;
-            rs8[(c + 1) & 7] += p1;
-            pw[e2] = pack_bf16x2(p0, p1);
-          }
-          tmem_st_32x32b_x16(tm_s + ch * 16, pw);
-        }
-        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        for (int ch = 0; ch < 4; ++ch) tmem_st_32x32b_x16(tm_p + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&pw[16 * ch]));
         l_run = l_run * corr + rs;
         m_run = m_use;
         tmem_st_wait();
@@ -1197,16 +1196,6 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[t]);
       }
       if (fail) break;
-      // the next item's Q: every S_t product of this item is complete (all seen), so the
-      // TMEM Q_t operand may be overwritten
-      {
-        const int next = fx_item(k + 1, cta, G);
-        if (next < nitems && !copy_q(k + 1, valid_of(next))) {
-          fail = true;
-          break;
-        }
-      }
-      if (!valid) continue;
       // ---- epilogue: O_t / l to bf16 through the staging tile and one TMA store; lse ----
       if (!fb_warp_wait(&pv_done[t], (n - 1) & 1, abort_flag, lim, lane)) {
         fail = true;

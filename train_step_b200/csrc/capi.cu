@@ -61,6 +61,10 @@ struct gpt2 {
   char *logits = nullptr, *dres_act = nullptr, *du = nullptr, *datt = nullptr, *dqkv = nullptr;
   float *dres = nullptr, *dh = nullptr, *Dattn = nullptr, *row_loss = nullptr, *part = nullptr, *splitk = nullptr;
   float2* ce_stats = nullptr;  // softmax partials of one head chunk, [chunk rows][2 * ceil(Vp / 128)]
+  float* splitk2 = nullptr;    // second split-K workspace (dW reductions alternate on the side stream)
+  float* part_bias = nullptr;  // bias-gradient column-sum partials (GELU-backward epilogue, attention backward)
+  size_t part_bias_floats = 0;
+  SideStream side;             // reductions of gradient partials overlapping the backward pass
   size_t part_floats = 0, splitk_floats = 0;
   int *tok = nullptr, *tgt = nullptr;
   void* emb_scratch = nullptr;
@@ -99,6 +103,7 @@ struct gpt2 {
     c.launches = &launches;
     c.splitk_ws = splitk;
     c.splitk_cap = splitk_floats;
+    c.ws_buf = SIDE_WS0;
     c.num_sms = num_sms;
     return c;
   }
@@ -313,6 +318,9 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
   RK(forward_layers(m, B, T));
 
   // ---------------- head + cross-entropy, chunk by chunk ----------------
+  // bf16 backward: reductions of gradient partials run on the side stream (cb)
+  LaunchCtx cb = c;
+  if (backward && dt == GPT2_BF16) cb.side = &m->side;
   const float* headw = m->cfg.tied ? m->wte : m->head;
   float* g_head = m->cfg.tied ? m->g_wte : m->g_head;
   const int chunk = N < HEAD_CHUNK_ROWS ? N : HEAD_CHUNK_ROWS;
@@ -334,10 +342,10 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
       RK(cross_entropy(c, dt, m->logits, Vp, rows, m->cfg.V, m->tgt + r0, 1.0f / (float)N, m->row_loss + r0));
     if (backward) {
       // dxf = dlogits W ; dW += dlogits^T xf
-      RK(gemm(c, dt, GemmDesc{m->logits, Vp, false, m->W(headw), C, true, rows, C, Vp, EPI_F32, m->dh + (int64_t)r0 * C,
-                              C, nullptr, 0, nullptr, nullptr, 0, 0, 0, CAT_GEMM_HEAD}));
-      RK(gemm(c, dt, GemmDesc{m->logits, Vp, true, xf_c, C, true, Vp, C, rows, EPI_F32, g_head, C, nullptr, 0, nullptr,
-                              nullptr, 0, 1, 0, CAT_GEMM_HEAD}));
+      RK(gemm(cb, dt, GemmDesc{m->logits, Vp, false, m->W(headw), C, true, rows, C, Vp, EPI_F32, m->dh + (int64_t)r0 * C,
+                               C, nullptr, 0, nullptr, nullptr, 0, 0, 0, CAT_GEMM_HEAD}));
+      RK(gemm(cb, dt, GemmDesc{m->logits, Vp, true, xf_c, C, true, Vp, C, rows, EPI_F32, g_head, C, nullptr, 0, nullptr,
+                               nullptr, 0, 1, 0, CAT_GEMM_HEAD}));
     }
   }
   sum_rows_kernel<<<1, 1024, 0, m->stream>>>(m->row_loss, N, 1.0f / (float)N, m->d_loss, 0);
@@ -350,14 +358,34 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
   // linear layer that produced this residual (dbias_next, nullable)
   auto LN_B = [&](const float* dy, const float* x, const float* gg, float* mu, float* rs, int accumulate, float* dg,
                   float* db, float* dbias_next) -> int {
-    return dt == GPT2_BF16 ? layernorm_bwd_t<bf16>(c, dy, x, gg, mu, rs, N, C, m->dres, (bf16*)m->dres_act,
-                                                   accumulate, m->part, dg, db, dbias_next, 1)
+    return dt == GPT2_BF16 ? layernorm_bwd_t<bf16>(cb, dy, x, gg, mu, rs, N, C, m->dres, (bf16*)m->dres_act,
+                                                   accumulate, m->part, dg, db, dbias_next, 1, SIDE_LN)
                            : layernorm_bwd_t<float>(c, dy, x, gg, mu, rs, N, C, m->dres, (float*)nullptr, accumulate,
                                                     m->part, dg, db, dbias_next, 1);
   };
   auto COLSUM_ACT = [&](const void* y, int ncols, float* out) -> int {
     return dt == GPT2_BF16 ? colsum_t<bf16>(c, (const bf16*)y, ncols, N, ncols, m->part, out)
                            : colsum_t<float>(c, (const float*)y, ncols, N, ncols, m->part, out);
+  };
+  // weight-gradient GEMMs alternate between two split-K workspaces, each reduced on the
+  // side stream while the next GEMMs run
+  int dw_i = 0;
+  auto DW = [&](const GemmDesc& d) -> int {
+    LaunchCtx cw = cb;
+    if (cb.side) {
+      cw.splitk_ws = (dw_i & 1) ? m->splitk2 : m->splitk;
+      cw.ws_buf = (dw_i & 1) ? SIDE_WS1 : SIDE_WS0;
+      cw.reduce_on_side = true;
+      ++dw_i;
+    }
+    return gemm(cw, dt, d);
+  };
+  // a bias-gradient reduction of m->part_bias on the side stream (in order when there is none)
+  auto BIAS_RED = [&](int P, int ncols, float* out) -> int {
+    if (!cb.side) return reduce_partials(cb, m->part_bias, P, ncols, 1, out, nullptr, nullptr, 1);
+    const int r = reduce_partials(side_ctx(cb), m->part_bias, P, ncols, 1, out, nullptr, nullptr, 1);
+    side_mark_free(cb, SIDE_BIAS);
+    return r;
   };
   RK(LN_B(m->dh, xs(2 * L), m->lnf_g, mean(2 * L), rstd(2 * L), 0, m->g_lnf_g, m->g_lnf_b, m->lg[L - 1].pj_b));
   for (int l = L - 1; l >= 0; --l) {
@@ -371,40 +399,41 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     void* a = ACT(m->a, l, NF);
     float* lse = m->lse + l * NLSE;
     // MLP: x_out = x_mid + pj(gelu(fc(ln2(x_mid))))
-    RK(gemm(c, dt, GemmDesc{dres_act, C, true, a, F, true, C, F, N, EPI_F32, gw.pj_w, F, nullptr, 0, nullptr, nullptr,
-                            0, 1, 0, CAT_GEMM_DW}));
+    RK(DW(GemmDesc{dres_act, C, true, a, F, true, C, F, N, EPI_F32, gw.pj_w, F, nullptr, 0, nullptr, nullptr,
+                   0, 1, 0, CAT_GEMM_DW}));
     {
       // bf16: the GELU-backward epilogue leaves the column sums of du (fc's bias gradient)
-      // per 32-row block in m->part
+      // per 32-row block in m->part_bias
       GemmDesc d{dres_act, C, false, m->W(w.pj_w), F, true, N, F, C, EPI_BF16_DGELU, m->du, F, nullptr, 0,
                  nullptr, u, F, 0, 1, CAT_GEMM_DX};
-      if (dt == GPT2_BF16) d.colsum = m->part;
-      RK(gemm(c, dt, d));
+      if (dt == GPT2_BF16) {
+        d.colsum = m->part_bias;
+        RK(side_wait_free(cb, SIDE_BIAS));
+      }
+      RK(gemm(cb, dt, d));
     }
-    RK(gemm(c, dt, GemmDesc{m->du, F, true, h2, C, true, F, C, N, EPI_F32, gw.fc_w, C, nullptr, 0, nullptr, nullptr, 0,
-                            1, 0, CAT_GEMM_DW}));
-    if (dt == GPT2_BF16)
-      RK(reduce_partials(c, m->part, (N + 31) / 32, F, 1, gw.fc_b, nullptr, nullptr, 1));
-    else
-      RK(COLSUM_ACT(m->du, F, gw.fc_b));
+    if (dt == GPT2_BF16) RK(BIAS_RED((N + 31) / 32, F, gw.fc_b));
+    RK(DW(GemmDesc{m->du, F, true, h2, C, true, F, C, N, EPI_F32, gw.fc_w, C, nullptr, 0, nullptr, nullptr, 0,
+                   1, 0, CAT_GEMM_DW}));
+    if (dt != GPT2_BF16) RK(COLSUM_ACT(m->du, F, gw.fc_b));
     RK(gemm(c, dt, GemmDesc{m->du, F, false, m->W(w.fc_w), C, true, N, C, F, EPI_F32, m->dh, C, nullptr, 0, nullptr,
                             nullptr, 0, 0, 1, CAT_GEMM_DX}));
     RK(LN_B(m->dh, xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), 1, gw.ln2_g, gw.ln2_b, gw.ao_b));
     // attention: x_mid = x_in + ao(attn(ln1(x_in)))
-    RK(gemm(c, dt, GemmDesc{dres_act, C, true, att, C, true, C, C, N, EPI_F32, gw.ao_w, C, nullptr, 0, nullptr, nullptr,
-                            0, 1, 0, CAT_GEMM_DW}));
+    RK(DW(GemmDesc{dres_act, C, true, att, C, true, C, C, N, EPI_F32, gw.ao_w, C, nullptr, 0, nullptr, nullptr,
+                   0, 1, 0, CAT_GEMM_DW}));
     RK(gemm(c, dt, GemmDesc{dres_act, C, false, m->W(w.ao_w), C, true, N, C, C, EPI_BF16, m->datt, C, nullptr, 0,
                             nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
     // bf16: the attention backward leaves the column sums of dqkv (the qkv bias gradient)
-    // per 32-row block in m->part
+    // per 32-row block in m->part_bias
     const bool qkvb_fused = gw.qkv_b && dt == GPT2_BF16;
-    RK(attention_bwd(c, dt, qkv, att, m->datt, lse, B, T, NH, hd, m->dqkv, m->Dattn, qkvb_fused ? m->part : nullptr));
-    RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, true, h1, C, true, 3 * C, C, N, EPI_F32, gw.qkv_w, C, nullptr, 0, nullptr,
-                            nullptr, 0, 1, 0, CAT_GEMM_DW}));
-    if (qkvb_fused)
-      RK(reduce_partials(c, m->part, attn_colsum_blocks(B, T), 3 * C, 1, gw.qkv_b, nullptr, nullptr, 1));
-    else if (gw.qkv_b)
-      RK(COLSUM_ACT(m->dqkv, 3 * C, gw.qkv_b));
+    if (qkvb_fused) RK(side_wait_free(cb, SIDE_BIAS));
+    RK(attention_bwd(c, dt, qkv, att, m->datt, lse, B, T, NH, hd, m->dqkv, m->Dattn,
+                     qkvb_fused ? m->part_bias : nullptr));
+    if (qkvb_fused) RK(BIAS_RED(attn_colsum_blocks(B, T), 3 * C, gw.qkv_b));
+    RK(DW(GemmDesc{m->dqkv, 3 * C, true, h1, C, true, 3 * C, C, N, EPI_F32, gw.qkv_w, C, nullptr, 0, nullptr,
+                   nullptr, 0, 1, 0, CAT_GEMM_DW}));
+    if (gw.qkv_b && !qkvb_fused) RK(COLSUM_ACT(m->dqkv, 3 * C, gw.qkv_b));
     RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, false, m->W(w.qkv_w), C, true, N, C, 3 * C, EPI_F32, m->dh, C, nullptr, 0,
                             nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
     RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b,
@@ -412,7 +441,7 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
   }
   EmbScratch es = emb_scratch_carve(m->emb_scratch, N, C);
   RK(embedding_bwd(c, m->tok, m->dres, B, T, C, m->cfg.V, m->g_wte, m->g_wpe, es));
-  return GPT2_OK;
+  return side_join(cb);  // every gradient is complete on the main stream from here on
 }
 
 int validate_batch(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T) {
@@ -463,6 +492,12 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
   };
   if (cudaStreamCreateWithFlags(&m->stream, cudaStreamNonBlocking) != cudaSuccess) return bail(GPT2_ERR_CUDA, "stream");
   m->own_stream = true;
+  if (cudaStreamCreateWithFlags(&m->side.s, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&m->side.ready, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&m->side.joined, cudaEventDisableTiming) != cudaSuccess)
+    return bail(GPT2_ERR_CUDA, "side stream");
+  for (auto& e : m->side.freed)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return bail(GPT2_ERR_CUDA, "side events");
   const size_t S = (size_t)m->n_store;
   if (cudaMalloc(&m->p, S * 4) || cudaMalloc(&m->g, S * 4) || cudaMalloc(&m->m, S * 4) || cudaMalloc(&m->v, S * 4))
     return bail(GPT2_ERR_OOM, "state");
@@ -510,6 +545,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
       std::max<int64_t>((N + 31) / 32 * F,                         // the GELU-backward epilogue's column sums
                         (int64_t)(c.B_max * ((c.T + 127) / 128) * 4) * 3 * C));  // the attention backward's
   m->splitk_floats = (size_t)std::max<int64_t>(16LL * F * C, 16LL * chunk * C);
+  m->part_bias_floats = (size_t)std::max<int64_t>((N + 31) / 32 * F, (int64_t)c.B_max * ((c.T + 127) / 128) * 4 * 3 * C);
   std::vector<std::pair<void**, size_t>> plan = {
       {(void**)&m->x, (size_t)(2 * L + 1) * N * C * 4},
       {(void**)&m->stat_mean, (size_t)(2 * L + 1) * N * 4},
@@ -534,6 +570,8 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
       {(void**)&m->row_loss, (size_t)N * 4},
       {(void**)&m->part, m->part_floats * 4},
       {(void**)&m->splitk, m->splitk_floats * 4},
+      {(void**)&m->splitk2, m->splitk_floats * 4},
+      {(void**)&m->part_bias, m->part_bias_floats * 4},
       {(void**)&m->tok, (size_t)N * 4},
       {(void**)&m->tgt, (size_t)N * 4},
       {(void**)&m->emb_scratch, emb_scratch_bytes((int)N, (int)C)},
@@ -1031,6 +1069,14 @@ void gpt2_destroy(gpt2* m) {
   cudaFree(m->v);
   cudaFree(m->shadow);
   if (m->own_stream && m->stream) cudaStreamDestroy(m->stream);
+  if (m->side.s) {
+    cudaStreamSynchronize(m->side.s);
+    cudaStreamDestroy(m->side.s);
+  }
+  if (m->side.ready) cudaEventDestroy(m->side.ready);
+  if (m->side.joined) cudaEventDestroy(m->side.joined);
+  for (auto& e : m->side.freed)
+    if (e) cudaEventDestroy(e);
   delete m;
 }
 
@@ -1195,6 +1241,13 @@ int gpt2_op_layernorm_bwd(int dtype, const float* dy, const float* x, const floa
   if (C % 4 || C > 2048 || N <= 0) {
     g_op_error = "layernorm: C % 4 == 0, C <= 2048, N > 0 required";
     return GPT2_ERR_CONFIG;
+  }
+  {
+    const uintptr_t any = (uintptr_t)dy | (uintptr_t)x | (uintptr_t)g | (uintptr_t)dres | (uintptr_t)dres_act;
+    if (any & 15) {
+      g_op_error = "layernorm: dy, x, g, dres and dres_act must start on 16-byte boundaries";
+      return GPT2_ERR_CONFIG;
+    }
   }
   const int grid = ln_bwd_grid(N, C, o.c.num_sms);
   float* part = nullptr;

@@ -63,17 +63,22 @@ constexpr int TC_EPI_WARPS = 8;
 // span both SMs' tensor cores. Each CTA stages its own 128 rows of A and its own
 // BN / 2 rows of B, so a CTA moves 2/3 of the shared-memory and L2 bytes per FLOP
 // that the single-CTA form (128 rows of A, BN rows of B) does.
-template <int BN, bool PAIR = false>
+// AUX: the epilogue reads an auxiliary tile (residual or GELU input) per chunk; it gets
+// four 2 KB chunk buffers per epilogue warp so that the auxiliary tile of chunk n + 3 is
+// in flight while chunk n is computed (one chunk of lookahead left the epilogue waiting
+// on every load), at the price of one main-loop stage.
+template <int BN, bool PAIR = false, bool AUX = false>
 struct TcCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows staged by one CTA
   static constexpr int B_BYTES = B_ROWS * TC_BK * 2;
   static constexpr int UNIT_M = PAIR ? 2 * TC_BM : TC_BM;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (192 * 1024) / STAGE;
+  static constexpr int NBUF = AUX ? 4 : 2;                   // 2 KB chunk buffers per epilogue warp
+  static constexpr int STAGING = TC_EPI_WARPS * NBUF * 2048;
+  static constexpr int BARS = 512;                           // mbarriers, TMEM slot, abort flag
+  static constexpr int STAGES = (232448 - 1024 - BARS - STAGING) / STAGE;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  static constexpr int STAGING = TC_EPI_WARPS * 4096;  // two 2 KB chunk buffers per epilogue warp
-  static constexpr int BARS = 512;                      // mbarriers, TMEM slot, abort flag
   static constexpr int SMEM = STAGES * STAGE + STAGING + 1024 + BARS;
 };
 
@@ -228,7 +233,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                    const GemmParams p) {
-  using Cfg = TcCfg<BN, PAIR>;
+  using Cfg = TcCfg<BN, PAIR, tc_has_aux<EPI>()>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int UNIT_M = Cfg::UNIT_M;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint64_t* auxbar = drain + 2;  // [TC_EPI_WARPS][2]: auxiliary tile landed in chunk buffer 0 / 1
+  uint64_t* auxbar = drain + 2;  // [TC_EPI_WARPS][NBUF]: auxiliary tile landed in chunk buffer b
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -259,7 +264,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&tempty[a], PAIR ? 2 * TC_EPI_WARPS : TC_EPI_WARPS);
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < 2 * TC_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
+    for (int i = 0; i < Cfg::NBUF * TC_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -439,23 +444,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int q = warp & 3;          // TMEM lane quarter this warp may access
     const int half = ew >> 2;        // which half of the BN columns
     const int c_begin = half * (BN / 2), c_end = (half + 1) * (BN / 2);
-    uint8_t* wbuf = staging + ew * 4096;  // chunk buffers: wbuf, wbuf + 2048
-    uint64_t* abar = auxbar + 2 * ew;
+    constexpr int NBUF = Cfg::NBUF;
+    uint8_t* wbuf = staging + ew * (NBUF * 2048);  // chunk buffers: wbuf + b * 2048
+    uint64_t* abar = auxbar + NBUF * ew;
     if (lane == 0) {
       if (EPI == EPI_BF16_GELU || p.ksplit > 1 || HAS_AUX) tma_prefetch_desc(&tmO2);
       tma_prefetch_desc(&tmO);
     }
-    // auxiliary tile of the first chunk (tmO2 is the auxiliary map for these epilogues);
+    // auxiliary tiles (tmO2 is the auxiliary map for these epilogues): chunk g of this
+    // warp's sequence goes to buffer g % NBUF, NBUF - 1 chunks ahead of the one computed;
     // lane 0 tracks the loads in flight (bit b: buffer b) for the abort path
     uint32_t aux_pending = 0, aux_par = 0;
     const int rbase = (int)rank * TC_BM + q * 32;  // this warp's first row within a unit
-    if (HAS_AUX && lane == 0 && cid < p.num_units) {
-      int tm0, tn0, ks0;
-      tc_decode_unit(p, cid, tm0, tn0, ks0);
-      mbar_arrive_expect_tx(&abar[0], 2048);
-      tma_load_2d(wbuf, &tmO2, &abar[0], tn0 * BN + c_begin, tm0 * UNIT_M + rbase);
-      aux_pending = 1u;
-    }
+    constexpr int CPU_ = (BN / 2) / CW;             // chunks per unit for this warp
+    // issue the auxiliary load of this warp's chunk g (g counted over all its units)
+    auto aux_load = [&](int g) {
+      const int unit_g = cid + (g / CPU_) * ncl;
+      if (unit_g >= p.num_units) return;
+      int tmg, tng, ksg;
+      tc_decode_unit(p, unit_g, tmg, tng, ksg);
+      const int b = g % NBUF;
+      mbar_arrive_expect_tx(&abar[b], 2048);
+      tma_load_2d(wbuf + b * 2048, &tmO2, &abar[b], tng * BN + c_begin + (g % CPU_) * CW, tmg * UNIT_M + rbase);
+      aux_pending |= 1u << b;
+      aux_par = (aux_par & ~(1u << b)) | ((uint32_t)((g / NBUF) & 1) << b);
+    };
+    if (HAS_AUX && lane == 0)
+      for (int g = 0; g < NBUF - 1; ++g) aux_load(g);
     int acc = 0;
     uint32_t acc_phase = 0;
     int n = 0;  // chunks processed by this warp
@@ -476,28 +491,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int row0 = tm * UNIT_M + rbase;
 #pragma unroll 1
       for (int c = c_begin; c < c_end; c += CW, ++n) {
-        const int b = tc_single_buffer<EPI>() ? 0 : (n & 1);
+        const int b = tc_single_buffer<EPI>() ? 0 : (n % NBUF);
         uint8_t* cur = wbuf + b * 2048;
         if (lane == 0) {
           if (HAS_AUX) {
-            // the other buffer's store has been read out: fetch the next chunk's auxiliary tile into it
-            bulk_wait_read<0>();
-            int nrow = -1, ncol = 0;
-            if (c + CW < c_end) {
-              nrow = row0;
-              ncol = tn * BN + c + CW;
-            } else if (unit + ncl < p.num_units) {
-              int tm2, tn2, ks2;
-              tc_decode_unit(p, unit + ncl, tm2, tn2, ks2);
-              nrow = tm2 * UNIT_M + rbase;
-              ncol = tn2 * BN + c_begin;
-            }
-            if (nrow >= 0) {
-              mbar_arrive_expect_tx(&abar[b ^ 1], 2048);
-              tma_load_2d(wbuf + (b ^ 1) * 2048, &tmO2, &abar[b ^ 1], ncol, nrow);
-              aux_pending |= 1u << (b ^ 1);
-              aux_par = (aux_par & ~(1u << (b ^ 1))) | ((uint32_t)(((n + 1) >> 1) & 1) << (b ^ 1));
-            }
+            // nothing to wait for: the auxiliary tile of this chunk was requested NBUF - 1
+            // chunks ago, into the buffer it is computed and stored from
           } else if (tc_single_buffer<EPI>()) {
             // GELU: u and gelu(u) go out as two bulk groups; the u half is free once the
             // previous chunk's u store has been read (its gelu store may still be reading)
@@ -533,7 +532,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (HAS_AUX) {
           int got = 1;
           if (lane == 0) {
-            got = mbar_wait_bounded(&abar[b], (n >> 1) & 1, abort_flag, lim) ? 1 : 0;
+            got = mbar_wait_bounded(&abar[b], (n / NBUF) & 1, abort_flag, lim) ? 1 : 0;
             if (got) aux_pending &= ~(1u << b);
           }
           got = __shfl_sync(0xffffffffu, got, 0);
@@ -545,7 +544,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             ok = false;
             break;
           }
-          mbar_try_wait(&abar[b], (n >> 1) & 1);  // every lane observes the completed phase
+          mbar_try_wait(&abar[b], (n / NBUF) & 1);  // every lane observes the completed phase
         }
         const int col0 = tn * BN + c;
         if (EPI == EPI_BF16_GELU) {
@@ -622,6 +621,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
           bulk_commit();  // one group per chunk (possibly empty) keeps the buffer accounting exact
+          if (HAS_AUX) {
+            // the store of chunk n - 1 (committed a chunk ago) has read its buffer out: fetch
+            // the auxiliary tile of chunk n + NBUF - 1, which uses that buffer next; the store
+            // just committed may still be reading
+            bulk_wait_read<1>();
+            aux_load(n + NBUF - 1);
+          }
         }
       }
       acc ^= 1;
@@ -630,7 +636,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (lane == 0) {
       bulk_wait_all();
       int never = 0;  // auxiliary loads still in flight (abort path only) land before the CTA exits
-      for (int bb = 0; bb < 2; ++bb)
+      for (int bb = 0; bb < NBUF; ++bb)
         if ((aux_pending >> bb) & 1u)
           mbar_wait_bounded(&abar[bb], (aux_par >> bb) & 1u, reinterpret_cast<volatile int*>(&never), lim);
     }

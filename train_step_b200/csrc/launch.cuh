@@ -92,6 +92,20 @@ struct Profiler {
   }
 };
 
+// A second stream for work that nothing on the main stream needs before a later join:
+// the reductions of gradient partials into parameter gradients, which then overlap the
+// next GEMM (they fit beside a GEMM's CTA on each SM). A partial buffer is written again
+// only after the reduction that reads it has finished (its `freed` event); the main
+// stream joins the side stream at the end of a micro-batch's backward pass.
+enum SideBuf : int { SIDE_LN = 0, SIDE_BIAS = 1, SIDE_WS0 = 2, SIDE_WS1 = 3, SIDE_NBUF = 4 };
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t ready = nullptr;  // recorded on the main stream before side work is enqueued
+  cudaEvent_t joined = nullptr;
+  cudaEvent_t freed[SIDE_NBUF] = {};
+  bool used[SIDE_NBUF] = {};
+};
+
 struct LaunchCtx {
   Profiler* prof = nullptr;
   cudaStream_t stream = nullptr;
@@ -102,7 +116,44 @@ struct LaunchCtx {
   size_t splitk_cap = 0;          // floats
   int num_sms = 148;
   bool pdl = false;  // launch as programmatic dependents of the previous kernel (kernels that support it)
+  SideStream* side = nullptr;     // nullable: every reduction on `stream`
+  int ws_buf = -1;                // the side buffer id of splitk_ws (-1: none)
+  bool reduce_on_side = false;    // a split-K reduction goes to the side stream
 };
+
+// The main stream waits until the last reduction that read side buffer b has finished.
+inline int side_wait_free(const LaunchCtx& c, int b) {
+  if (!c.side || b < 0 || !c.side->used[b]) return GPT2_OK;
+  if (cudaStreamWaitEvent(c.stream, c.side->freed[b], 0) != cudaSuccess) {
+    if (c.msg) *c.msg = "cudaStreamWaitEvent failed";
+    return GPT2_ERR_CUDA;
+  }
+  return GPT2_OK;
+}
+// A context that launches on the side stream, after everything enqueued on c.stream so far.
+inline LaunchCtx side_ctx(const LaunchCtx& c) {
+  LaunchCtx r = c;
+  cudaEventRecord(c.side->ready, c.stream);
+  cudaStreamWaitEvent(c.side->s, c.side->ready, 0);
+  r.stream = c.side->s;
+  r.side = nullptr;
+  return r;
+}
+// After the side-stream launches that read side buffer b.
+inline void side_mark_free(const LaunchCtx& c, int b) {
+  cudaEventRecord(c.side->freed[b], c.side->s);
+  c.side->used[b] = true;
+}
+// The main stream waits for all side-stream work enqueued so far.
+inline int side_join(const LaunchCtx& c) {
+  if (!c.side) return GPT2_OK;
+  if (cudaEventRecord(c.side->joined, c.side->s) != cudaSuccess ||
+      cudaStreamWaitEvent(c.stream, c.side->joined, 0) != cudaSuccess) {
+    if (c.msg) *c.msg = "side stream join failed";
+    return GPT2_ERR_CUDA;
+  }
+  return GPT2_OK;
+}
 
 // Launch `kern` on c.stream; with c.pdl as a programmatic dependent of the stream's
 // previous kernel (the kernel must call pdl_wait before reading that kernel's results and
@@ -309,7 +360,7 @@ struct TcMaps {
 template <int BN, bool AM, bool BM_, int EPI, bool PAIR>
 int launch_tc_inst(const LaunchCtx& c, const TcMaps& tm, const GemmParams& p) {
   auto kern = gemm_tc_kernel<BN, AM, BM_, EPI, PAIR>;
-  constexpr int smem = TcCfg<BN, PAIR>::SMEM;
+  constexpr int smem = TcCfg<BN, PAIR, tc_has_aux<EPI>()>::SMEM;
   // shared-memory opt-in and, for pairs, the co-resident clusters: once per device
   const int max_clusters = per_device_once(reinterpret_cast<const void*>(kern), [&]() -> int {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -1;
@@ -387,14 +438,31 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
     if (ksplit > 1) return fail(c, GPT2_ERR_CONFIG, "gemm: split-K needs epilogue 4 and a workspace");
     ksplit = 1;
   } else if (ksplit == 0) {
-    const int tiles = tiles_m * tiles_n;
-    const int slots = pair ? c.num_sms / 2 : c.num_sms;  // tiles in flight at once
+    // Choose the split that minimises (waves of units) x (k-blocks per unit) plus the
+    // split-K reduction's traffic. A k-block of a 128-row x BN tile costs about
+    // 128 * BN * 64 * 2 / 8192 tensor cycles per SM (~0.14 us at BN 256 per 128 rows);
+    // the reduction moves (ksplit + 1 + accumulate) M N fp32 words at ~5 TB/s. Wave
+    // quantisation matters: 36 tiles split 5 ways are 180 units, 2.4 waves of 74 pairs
+    // (3 waves), where a split of 2 or 4 fills 1 or 2 waves exactly.
+    const long long tiles = (long long)tiles_m * tiles_n;
+    const long long slots = pair ? c.num_sms / 2 : c.num_sms;  // units in flight at once
+    const double kb_us = (double)(pair ? 2 * TC_BM : TC_BM) * BN * TC_BK * 2.0 / 8192.0 / (pair ? 2.0 : 1.0) / 1.8e3;
+    double best = 1e30;
     ksplit = 1;
-    if (tiles < 2 * slots) {
-      ksplit = (2 * slots + tiles - 1) / tiles;
-      if (ksplit > num_kb / 4) ksplit = num_kb / 4;
-      if (ksplit > 16) ksplit = 16;
-      if (ksplit < 1) ksplit = 1;
+    const int kmax = std::min(16, std::max(1, num_kb / 4));
+    for (int k = 1; k <= kmax; ++k) {
+      const int per = (num_kb + k - 1) / k;
+      const int kk = (num_kb + per - 1) / per;  // no empty slices
+      const long long waves = (tiles * kk + slots - 1) / slots;
+      double t = (double)waves * per * kb_us;
+      if (kk > 1) {
+        if ((size_t)kk * d.M * d.N > c.splitk_cap) continue;
+        t += (double)(kk + 1 + d.accumulate) * d.M * d.N * 4.0 / 5.0e6;  // us at 5 TB/s
+      }
+      if (t < best * 0.999) {
+        best = t;
+        ksplit = kk;
+      }
     }
   }
   int kb_per = (num_kb + ksplit - 1) / ksplit;
@@ -452,6 +520,10 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
     tm.o2 = tm.o;
   }
   if (!ok) return fail(c, GPT2_ERR_CUDA, "gemm: cuTensorMapEncodeTiled failed");
+  if (ksplit > 1) {  // the workspace's previous reduction has read it
+    const int rw = side_wait_free(c, c.ws_buf);
+    if (rw) return rw;
+  }
   int r;
   {
   ProfScope ps(c, d.role, 2.0 * d.M * d.N * d.K, 0.0);
@@ -470,13 +542,20 @@ inline int gemm_tc(const LaunchCtx& c, const GemmDesc& d) {
   }
   }
   if (r || ksplit == 1) return r;
-  ProfScope ps(c, CAT_SPLITK, 0.0, 4.0 * d.M * d.N * (ksplit + 1 + d.accumulate));
-  const long long n4 = (long long)d.M * (d.N / 4);
-  long long blocks = (n4 + 255) / 256;
-  if (blocks > 8LL * c.num_sms) blocks = 8LL * c.num_sms;
-  splitk_reduce_kernel<<<(int)blocks, 256, 0, c.stream>>>(c.splitk_ws, ksplit, d.M, d.N, (float*)d.out, d.ldo,
-                                                           d.accumulate);
-  return check_launch(c, "splitk_reduce");
+  const bool on_side = c.side && c.reduce_on_side && c.ws_buf >= 0;
+  const LaunchCtx rc = on_side ? side_ctx(c) : c;
+  {
+    ProfScope ps(rc, CAT_SPLITK, 0.0, 4.0 * d.M * d.N * (ksplit + 1 + d.accumulate));
+    const long long n4 = (long long)d.M * (d.N / 4);
+    long long blocks = (n4 + 255) / 256;
+    if (blocks > 8LL * c.num_sms) blocks = 8LL * c.num_sms;
+    splitk_reduce_kernel<<<(int)blocks, 256, 0, rc.stream>>>(c.splitk_ws, ksplit, d.M, d.N, (float*)d.out, d.ldo,
+                                                              d.accumulate);
+  }
+  r = check_launch(rc, "splitk_reduce");
+  if (on_side) side_mark_free(c, c.ws_buf);
+  else if (c.side && c.ws_buf >= 0) c.side->used[c.ws_buf] = false;  // read on the main stream already
+  return r;
 }
 
 inline int gemm_simt(const LaunchCtx& c, const GemmDesc& d) {
@@ -545,9 +624,10 @@ int layernorm_fwd_t(const LaunchCtx& c, const float* x, const float* g, const fl
   return check_launch(c, "layernorm_fwd");
 }
 
-// LayerNorm backward grid: at most the CTAs that are resident at once (each holds
-// LN_WARPS x 3 x C fp32 column accumulators in shared memory), so that no CTA waits
-// for a second wave.
+// LayerNorm backward grid: the CTAs resident at once (so that none waits for a second
+// wave). A CTA holds LN_WARPS x 3 x C fp32 column accumulators in shared memory and the
+// kernel is built for three CTAs per SM of registers: 3 per SM at C = 768, 2 at 1024,
+// 1 at 1600.
 inline int ln_bwd_grid(int N, int C, int num_sms) {
   const long long per_cta = (long long)LN_WARPS * 3 * C * 4 + 1024;
   long long resident = 233472 / per_cta;
@@ -576,30 +656,72 @@ void launch_ln_bwd(const LaunchCtx& c, int grid, size_t smem, const float* dy, c
                                                                        accumulate, part, with_rsum, N, C);
 }
 
+// Slots per warp of the staged backward: as many rows (dy, x, dres: 12 C bytes each) as
+// fit in the shared memory of one CTA, at most 3; 0 when fewer than 2 fit (the staged
+// kernel needs a row in flight while it computes one, so wide rows use the other kernel).
+inline int ln_ring_stages(int C) {
+  const long long slot = 12LL * C + 8;
+  long long st = (232448 - 1024) / ((long long)LNR_WARPS * slot);
+  if (st > 3) st = 3;
+  return st >= 2 ? (int)st : 0;
+}
+inline size_t ln_ring_smem(int C, int stages) { return (size_t)LNR_WARPS * stages * (12 * (size_t)C + 8); }
+
+template <class T, int NV>
+int launch_ln_bwd_ring(const LaunchCtx& c, int grid, int stages, const float* dy, const float* x, const float* g,
+                       const float* mean, const float* rstd, float* dres, T* dres_act, int accumulate, float* part,
+                       int with_rsum, int N, int C) {
+  const size_t smem = ln_ring_smem(C, stages);
+  // opted in once per device for the largest ring any C can ask for
+  if (!smem_optin(layernorm_bwd_ring_kernel<T, NV>, 232448 - 1024))
+    return fail(c, GPT2_ERR_CUDA, "layernorm_bwd: shared-memory opt-in");
+  layernorm_bwd_ring_kernel<T, NV><<<grid, LNR_WARPS * 32, smem, c.stream>>>(
+      dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C, stages, c.d_err, 4000000000ull);
+  return 0;
+}
+
 // LayerNorm backward plus the reduction of its parameter gradients: dg, db (+)=;
 // dbias_next (nullable) (+)= column sums of the updated dres.
 template <class T>
 int layernorm_bwd_t(const LaunchCtx& c, const float* dy, const float* x, const float* g, const float* mean,
                     const float* rstd, int N, int C, float* dres, T* dres_act, int accumulate,
-                    float* part /*3*grid*C*/, float* dg, float* db, float* dbias_next, int accumulate_params) {
-  const int grid = ln_bwd_grid(N, C, c.num_sms);
+                    float* part /*3*grid*C*/, float* dg, float* db, float* dbias_next, int accumulate_params,
+                    int side_buf = -1) {
+  const int stages = ln_ring_stages(C);
   const int nv = ln_nv(C);
+  // staged kernel: one CTA per SM (fewer if there are fewer row groups)
+  const int grid = stages && nv <= 8 ? (int)std::min<long long>(c.num_sms, ((long long)N + LNR_WARPS - 1) / LNR_WARPS)
+                                     : ln_bwd_grid(N, C, c.num_sms);
   const int with_rsum = dbias_next != nullptr;
+  {
+    const int rw = side_wait_free(c, side_buf);  // the partials' previous reduction has read them
+    if (rw) return rw;
+  }
   {
     ProfScope ps(c, CAT_LN_BWD, 0.0,
                  (double)N * C * (12 + 4 * accumulate + (dres_act ? sizeof(T) : 0)) + 8.0 * N +
                      4.0 * (2 + with_rsum) * grid * C);
     const size_t smem = (size_t)LN_WARPS * 3 * C * 4;
-    if (nv <= 1) launch_ln_bwd<T, 1>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    int rr = 0;
+    if (stages && nv <= 4) rr = launch_ln_bwd_ring<T, 4>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (stages && nv <= 6) rr = launch_ln_bwd_ring<T, 6>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (stages && nv <= 8) rr = launch_ln_bwd_ring<T, 8>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 1) launch_ln_bwd<T, 1>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
     else if (nv <= 2) launch_ln_bwd<T, 2>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
     else if (nv <= 4) launch_ln_bwd<T, 4>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
     else if (nv <= 6) launch_ln_bwd<T, 6>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
     else if (nv <= 8) launch_ln_bwd<T, 8>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
     else if (nv <= 13) launch_ln_bwd<T, 13>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
     else launch_ln_bwd<T, 16>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    if (rr) return rr;
   }
   int r = check_launch(c, "layernorm_bwd");
   if (r) return r;
+  if (c.side && side_buf >= 0) {  // the parameter-gradient reduction overlaps what follows
+    r = reduce_partials(side_ctx(c), part, grid, C, 2 + with_rsum, dg, db, dbias_next, accumulate_params);
+    side_mark_free(c, side_buf);
+    return r;
+  }
   return reduce_partials(c, part, grid, C, 2 + with_rsum, dg, db, dbias_next, accumulate_params);
 }
 

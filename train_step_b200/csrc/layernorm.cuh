@@ -180,6 +180,169 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
   }
 }
 
+// Backward, staged through shared memory (the same mathematics and partial layout as
+// layernorm_bwd_kernel). One CTA of LNR_WARPS warps per SM; warp w of CTA b takes rows
+// b * LNR_WARPS + w + k * gridDim.x * LNR_WARPS, k = 0, 1, ... Each warp owns a ring of
+// `stages` slots, a slot holding one row of dy, x and (when accumulating) dres; lane 0
+// fills slot k % stages with 1-D bulk copies `stages` rows ahead of the row computed, so
+// a warp always has rows in flight while it computes (an HBM-bound kernel needs bytes in
+// flight, not threads). Column accumulators live in registers (lane l owns the float4
+// columns i * 32 + l); at the end the warps' accumulators pass through shared memory and
+// are summed in warp order, so the reduction order is fixed.
+constexpr int LNR_WARPS = 8;
+template <class T, int NV>
+__global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
+    const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
+    const float* __restrict__ mean, const float* __restrict__ rstd, float* __restrict__ dres,
+    T* __restrict__ dres_act, int accumulate, float* __restrict__ part, int with_rsum, int N, int C, int stages,
+    int* err, unsigned long long limit_ns) {
+  extern __shared__ __align__(128) uint8_t lnr_smem[];
+  __shared__ int s_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C4 = C / 4;
+  const size_t slot_floats = (size_t)3 * C;  // dy | x | dres
+  float* ring = reinterpret_cast<float*>(lnr_smem);
+  float* mine = ring + (size_t)warp * stages * slot_floats;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(lnr_smem + (size_t)LNR_WARPS * stages * slot_floats * 4) + warp * stages;
+  if (threadIdx.x == 0) s_abort = 0;
+  if (lane == 0) {
+    for (int st = 0; st < stages; ++st) mbar_init(&bars[st], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const long long first = (long long)blockIdx.x * LNR_WARPS + warp;
+  const long long stride = (long long)gridDim.x * LNR_WARPS;
+  const uint32_t row_bytes = (uint32_t)C * 4;
+  const uint32_t slot_bytes = row_bytes * (accumulate ? 3u : 2u);
+  // lane 0: request row k of this warp into slot k % stages
+  auto issue = [&](long long k) {
+    const long long row = first + k * stride;
+    if (row >= N) return;
+    float* slot = mine + (size_t)(k % stages) * slot_floats;
+    uint64_t* bar = &bars[k % stages];
+    mbar_arrive_expect_tx(bar, slot_bytes);
+    bulk_load_1d(slot, dy + row * C, row_bytes, bar);
+    bulk_load_1d(slot + C, x + row * C, row_bytes, bar);
+    if (accumulate) bulk_load_1d(slot + 2 * C, dres + row * C, row_bytes, bar);
+  };
+  if (lane == 0)
+    for (int k = 0; k < stages; ++k) issue(k);
+  float4 gv[NV], ag[NV], ab[NV], ar[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c4 = i * 32 + lane;
+    gv[i] = c4 < C4 ? __ldg(reinterpret_cast<const float4*>(g) + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    ag[i] = ab[i] = ar[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  long long k = 0;
+  bool ok = true;
+  for (;; ++k) {
+    const long long row = first + k * stride;
+    if (row >= N) break;
+    const int st = (int)(k % stages);
+    const uint32_t par = (uint32_t)((k / stages) & 1);
+    int got = 1;
+    if (lane == 0) got = mbar_wait_bounded(&bars[st], par, &s_abort, limit_ns) ? 1 : 0;
+    got = __shfl_sync(0xffffffffu, got, 0);
+    if (!got) {
+      if (lane == 0) {
+        raise_device_error(err, DEV_TIMEOUT);
+        s_abort = 1;
+      }
+      ok = false;
+      break;
+    }
+    mbar_try_wait(&bars[st], par);  // every lane observes the completed phase
+    const float4* sdy = reinterpret_cast<const float4*>(mine + (size_t)st * slot_floats);
+    const float4* sx = sdy + C4;
+    const float4* sr = sdy + 2 * C4;
+    const float mu = mean[row], rs = rstd[row];
+    float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c4 = i * 32 + lane;
+      if (c4 < C4) {
+        const float4 d = sdy[c4], xx = sx[c4];
+        const float4 xh = make_float4((xx.x - mu) * rs, (xx.y - mu) * rs, (xx.z - mu) * rs, (xx.w - mu) * rs);
+        const float a = d.x * gv[i].x, b = d.y * gv[i].y, cc = d.z * gv[i].z, e = d.w * gv[i].w;
+        m1 += (a + b) + (cc + e);
+        m2 += (a * xh.x + b * xh.y) + (cc * xh.z + e * xh.w);
+        ag[i].x += d.x * xh.x;
+        ag[i].y += d.y * xh.y;
+        ag[i].z += d.z * xh.z;
+        ag[i].w += d.w * xh.w;
+        ab[i].x += d.x;
+        ab[i].y += d.y;
+        ab[i].z += d.z;
+        ab[i].w += d.w;
+      }
+    }
+    m1 = warp_sum(m1) / (float)C;
+    m2 = warp_sum(m2) / (float)C;
+    float* dr = dres + row * C;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int c4 = i * 32 + lane;
+      if (c4 < C4) {
+        const float4 d = sdy[c4], xx = sx[c4];
+        const float4 xh = make_float4((xx.x - mu) * rs, (xx.y - mu) * rs, (xx.z - mu) * rs, (xx.w - mu) * rs);
+        float4 o = make_float4(rs * (d.x * gv[i].x - m1 - xh.x * m2), rs * (d.y * gv[i].y - m1 - xh.y * m2),
+                               rs * (d.z * gv[i].z - m1 - xh.z * m2), rs * (d.w * gv[i].w - m1 - xh.w * m2));
+        if (accumulate) {
+          const float4 r = sr[c4];
+          o.x += r.x;
+          o.y += r.y;
+          o.z += r.z;
+          o.w += r.w;
+        }
+        reinterpret_cast<float4*>(dr)[c4] = o;
+        if (dres_act) store4<T>(dres_act + row * C + c4 * 4, o.x, o.y, o.z, o.w);
+        if (with_rsum) {
+          ar[i].x += o.x;
+          ar[i].y += o.y;
+          ar[i].z += o.z;
+          ar[i].w += o.w;
+        }
+      }
+    }
+    __syncwarp();  // every lane has read the slot before it is refilled
+    if (lane == 0) issue(k + stages);
+  }
+  if (!ok) {
+    // rows already requested land before the CTA exits: wait (bounded) for each
+    if (lane == 0) {
+      int never = 0;
+      for (long long kk = k + 1; kk < k + stages; ++kk)
+        if (first + kk * stride < N)
+          mbar_wait_bounded(&bars[kk % stages], (uint32_t)((kk / stages) & 1),
+                            reinterpret_cast<volatile int*>(&never), limit_ns);
+    }
+  }
+  __syncthreads();  // every warp arrives, including one that gave up (s_abort is set by then)
+  if (s_abort) return;
+  // every copy was consumed: the ring is free for the warps' accumulators [warp][3][C4]
+  float4* accs = reinterpret_cast<float4*>(lnr_smem) + (size_t)warp * 3 * C4;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c4 = i * 32 + lane;
+    if (c4 < C4) {
+      accs[c4] = ag[i];
+      accs[C4 + c4] = ab[i];
+      accs[2 * C4 + c4] = ar[i];
+    }
+  }
+  __syncthreads();
+  const int nsum = with_rsum ? 3 : 2;
+  const float* accf = reinterpret_cast<const float*>(lnr_smem);
+  for (int idx = threadIdx.x; idx < nsum * C; idx += blockDim.x) {
+    const int which = idx / C, col = idx - which * C;
+    float sacc = 0.f;
+#pragma unroll
+    for (int w = 0; w < LNR_WARPS; ++w) sacc += accf[((size_t)w * 3 + which) * C + col];
+    part[((long long)which * gridDim.x + blockIdx.x) * C + col] = sacc;
+  }
+}
+
 // Deterministic column reduction of up to three partial sets at once:
 // out_v[c] (+)= sum_{p < P} part[(v*P + p)*ncols + c] for v = blockIdx.y. Each CTA
 // owns 8 columns: thread t sums column t % 8 over rows p = t / 8, t / 8 + 32, ...

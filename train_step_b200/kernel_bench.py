@@ -127,7 +127,7 @@ def decode_bench(a) -> dict:
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["gemm", "attn", "attn_bwd", "ln", "ce", "decode", "gemv"])
+    ap.add_argument("kernel", choices=["gemm", "attn", "attn_bwd", "ln", "ln_bwd", "ce", "decode", "gemv"])
     ap.add_argument("--M", type=int, default=16384)
     ap.add_argument("--N", type=int, default=3072)
     ap.add_argument("--K", type=int, default=768)
@@ -194,6 +194,23 @@ def main() -> None:
         rstd = torch.zeros(N, device=dev)
         ms = timeit(lambda: tsb.layernorm_fwd(x, w, bb, y, mean, rstd), a.iters)
         res.update(shape=[N, C], ms=ms, gbs=N * C * 6 / (ms * 1e-3) / 1e9)
+    elif a.kernel == "ln_bwd":
+        N, C = a.M, a.C
+        x = torch.randn(N, C, device=dev, generator=g)
+        w = torch.ones(C, device=dev)
+        bb = torch.zeros(C, device=dev)
+        y = torch.zeros(N, C, device=dev, dtype=torch.bfloat16)
+        mean = torch.zeros(N, device=dev)
+        rstd = torch.zeros(N, device=dev)
+        tsb.layernorm_fwd(x, w, bb, y, mean, rstd)
+        dy = torch.randn(N, C, device=dev, generator=g)
+        dres = torch.randn(N, C, device=dev, generator=g)
+        dres_act = torch.zeros(N, C, device=dev, dtype=torch.bfloat16)
+        dg = torch.zeros(C, device=dev)
+        db = torch.zeros(C, device=dev)
+        ms = timeit(lambda: tsb.layernorm_bwd(dy, x, w, mean, rstd, dres, dres_act, dg, db, accumulate=True,
+                                              accumulate_params=True), a.iters)
+        res.update(shape=[N, C], ms=ms, gbs=N * C * 18 / (ms * 1e-3) / 1e9)
     elif a.kernel == "decode":
         res.update(decode_bench(a))
     elif a.kernel == "gemv":
