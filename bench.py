@@ -7,7 +7,8 @@ One step = `accum` micro-batches of forward + backward (gradient accumulation)
 followed by one global-norm-clipped AdamW update, on seeded synthetic Zipf(1.1)
 tokens (stand-in for the pages' BPE text corpora). For N > 1 (torchrun, one
 process per GPU) every rank runs its own micro-batches (weak scaling) and the
-gradients are averaged with one NCCL all-reduce before the step (data parallel).
+gradients are averaged with NCCL all-reduces, one per layer bucket, that overlap the
+last micro-batch's backward pass (data parallel).
 
 Prints one JSON line (rank 0). `value` is whole-job tokens/s with the inputs
 already resident in HBM; `e2e` is the same metric through the public C-ABI with
@@ -210,13 +211,6 @@ def run_reference(args, c):
     return 0
 
 
-class _CudaArray:
-    """Zero-copy view of a raw device buffer for torch.as_tensor."""
-
-    def __init__(self, ptr: int, n: int):
-        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<f4", "data": (ptr, False), "version": 3}
-
-
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -256,22 +250,26 @@ def main():
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
     model = tsb.GPT2(cfg, seed=42, stream=stream.cuda_stream)
-    gptr, glen = model.grad_buffer()
-    grads = torch.as_tensor(_CudaArray(gptr, glen), device="cuda")
 
     # inputs resident in HBM: this rank's micro-batches (weak scaling by rank)
     mbs = [synth.micro_batch(B, T, c["V"], index=i) for i in dp.micro_batch_indices(rank, world, accum)]
     dev_in = [(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()) for a, b in mbs]
 
-    def allreduce():
-        if dist is not None:
-            dp.allreduce_mean_(grads)
+    # data parallel: the gradient average runs bucket by bucket (a layer at a time) on its
+    # own stream while the last micro-batch's backward pass is still running
+    exchange = dp.BucketedAllReduce(model) if dist is not None else None
 
     def train_step(inputs, want_outputs=False):
         loss = None
         for j, (tok, tgt) in enumerate(inputs):
-            loss = model.forward_backward(tok, tgt, want_loss=want_outputs and j == len(inputs) - 1)
-        allreduce()
+            last = j == len(inputs) - 1
+            if exchange is not None and last:
+                exchange.arm()
+            loss = model.forward_backward(tok, tgt, want_loss=want_outputs and last and exchange is None)
+        if exchange is not None:
+            exchange.run()
+            if want_outputs:
+                loss = model.read_loss()
         gn = model.step(LR, WD, B1, B2, want_norm=want_outputs)
         return loss, gn
 
@@ -402,7 +400,6 @@ def main():
             "gpu_launches": launches, "clocks": clk,
         }
         print(json.dumps(line), flush=True)
-    del grads
     model.close()
     if dist is not None:
         dist.barrier()

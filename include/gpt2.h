@@ -109,6 +109,12 @@ int gpt2_forward_backward(gpt2* m, const int32_t* tokens, const int32_t* targets
  * estimate_loss on held-out batches). loss_out as above (nullable). */
 int gpt2_forward(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T, float* loss_out);
 
+/* The mean loss of the most recent gpt2_forward_backward or gpt2_forward call, read
+ * later (for a call made with loss_out = NULL so that it did not wait for the GPU).
+ * Synchronises the handle's stream; GPT2_ERR_CONFIG for a NULL loss_out; a device
+ * error raised since the last check is returned as in gpt2_forward_backward. */
+int gpt2_read_loss(gpt2* m, float* loss_out);
+
 /* Optimizer step ("AxonLM", Training Recipe: betas (0.9, 0.95), weight decay 0.1
  * on 2-D tensors only, gradient clip 1.0; "GPT From Scratch", Key decisions: AdamW
  * decays only parameters of two or more dimensions, clipping at 1.0) on the
@@ -184,6 +190,28 @@ int gpt2_set_adam(gpt2* m, const float* m_host, const float* v_host, int64_t n, 
  * Owned by the handle; valid until gpt2_destroy. */
 int gpt2_grad_buffer(gpt2* m, float** dev, int64_t* n);
 
+/* Storage layout, computed on the host from a configuration alone (no device, no
+ * handle): for canonical tensor i (the order of gpt2_tensor_info), its offset and
+ * length in floats in the flat device storage of parameters, gradients and Adam
+ * moments (vocabulary tensors include their padding rows), and its gradient bucket:
+ * layer l's tensors are bucket l, the embeddings, final LayerNorm and untied head
+ * bucket L. *n_store (nullable) receives the storage length, also for an i past the
+ * last tensor, which returns GPT2_ERR_CONFIG. The buckets exist for a data-parallel
+ * exchange that overlaps the backward pass ("AxonLM", Key Features and Quick Start:
+ * data-parallel training over several GPUs); see gpt2_set_grad_events. */
+int gpt2_storage_layout(const gpt2_config* cfg, int i, char* name, int name_len, int64_t* offset, int64_t* n,
+                        int* bucket, int64_t* n_store);
+
+/* One-shot completion events for the gradient buckets of the NEXT gpt2_forward_backward
+ * call (the last micro-batch before an exchange): events[b] (cudaEvent_t handles the
+ * caller created on this handle's device, caller-owned, n = L + 1) is recorded as soon
+ * as every gradient of bucket b is final in the gradient buffer, in the order L-1, ...,
+ * 0, then L. A stream that waits on events[b] may read (and all-reduce in place) bucket
+ * b's ranges while the rest of the backward pass runs; it must not write other buckets
+ * before their own events. n = 0 cancels. The events are recorded once, then
+ * forgotten. Returns GPT2_ERR_CONFIG for n other than 0 or L + 1, or a null event. */
+int gpt2_set_grad_events(gpt2* m, void* const* events, int n);
+
 /* Per-kernel-category timing with CUDA events on the handle's stream.
  * gpt2_profile(m, 1) clears old records and starts recording an event pair around
  * every launch; gpt2_profile(m, 0) stops. gpt2_profile_read(m, cat, ...) waits for
@@ -191,7 +219,9 @@ int gpt2_grad_buffer(gpt2* m, float** dev, int64_t* n);
  * milliseconds, launch count and the algorithmic FLOPs and bytes of those launches
  * (2*M*N*K per GEMM; causal attention 4*B*H*hd*T(T+1)/2 forward and 2.5 times
  * that backward; bytes a kernel must move for the memory-bound ones). Returns
- * GPT2_ERR_CONFIG past the last category. */
+ * GPT2_ERR_CONFIG past the last category. While recording, the gradient reductions
+ * that normally overlap on a second stream run in order on the handle's stream, so
+ * that each kernel's time is its own. */
 int gpt2_profile(gpt2* m, int enable);
 int gpt2_profile_read(gpt2* m, int cat, char* name, int name_len, double* ms, int64_t* launches, double* flops,
                       double* bytes);
@@ -282,7 +312,8 @@ int gpt2_op_gemm_bench(const void* A, int64_t lda, int a_mn, const void* B, int6
                        float* ms_out, void* stream);
 
 /* LayerNorm forward over rows of f32_x [N, C]: y(act) [N, C], f32 mean and rstd
- * [N]. eps 1e-5, biased variance. C % 4 == 0, C <= 2048. */
+ * [N]. eps 1e-5, biased variance. C % 4 == 0, C <= 2048, and x, g, b, y start on
+ * 16-byte boundaries; otherwise GPT2_ERR_CONFIG. */
 int gpt2_op_layernorm_fwd(int dtype, const float* f32_x, const float* f32_g, const float* f32_b, int N, int C, void* y,
                           float* f32_mean, float* f32_rstd, void* stream);
 

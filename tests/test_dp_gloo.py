@@ -270,3 +270,132 @@ def test_zero1_two_rank_gloo_matches_single_process(tmp_path):
         mr = np.load(tmp_path / f"zm{r}.npy")
         lo, hi = dp.shard_bounds(n, world, r)
         assert np.all(mr[:lo] == 0) and np.all(mr[hi:] == 0) and np.any(mr[lo:hi] != 0)
+
+
+def _tsb_cfg(cfg):
+    import train_step_b200 as tsb
+    return tsb.Config(L=cfg["L"], H=cfg["H"], C=cfg["C"], T=cfg["T"], V=cfg["V"], tied=cfg["tied"],
+                      qkv_bias=cfg["qkv_bias"])
+
+
+@pytest.mark.parametrize("cfg", [dict(CFG, C=64), dict(L=12, H=12, C=768, T=1024, V=50257, tied=1, qkv_bias=1),
+                                 dict(L=12, H=12, C=768, T=1024, V=50257, tied=0, qkv_bias=0),
+                                 dict(L=48, H=25, C=1600, T=1024, V=50257, tied=1, qkv_bias=1)])
+def test_gradient_buckets_cover_the_storage(cfg):
+    """The library's storage layout (a host-only query): each tensor lies inside one range
+    of its own bucket, the buckets' ranges are disjoint, and bucket l holds exactly layer
+    l's tensors."""
+    import train_step_b200 as tsb
+    c = _tsb_cfg(cfg)
+    layout, n_store = tsb.storage_layout(c)
+    ranges = tsb.bucket_ranges(c)
+    assert len(ranges) == c.L + 1
+    for name, off, n, b in layout:
+        assert b == (int(name[1:name.index(".")]) if name[0] == "h" and name[1].isdigit() else c.L)
+        assert sum(1 for o, m in ranges[b] if o <= off and off + n <= o + m) == 1, name
+    flat = sorted(r for rs in ranges for r in rs)
+    assert all(a[0] + a[1] <= b[0] for a, b in zip(flat, flat[1:]))
+    assert flat[-1][0] + flat[-1][1] <= n_store
+    covered = sum(n for _, _, n, _ in layout)
+    assert covered <= sum(m for _, m in flat) <= covered + 64 * len(layout)
+
+
+class _StorageOracleModel:
+    """The float64 oracle behind the library's gradient storage layout (CPU): gradients
+    accumulate into a flat buffer laid out as the library lays out its own (offsets and
+    padding from gpt2_storage_layout), which the bucketed exchange averages range by
+    range; the step gathers them back into canonical order for the oracle's AdamW."""
+
+    def __init__(self, seed):
+        import oracle
+        import train_step_b200 as tsb
+        self.cfg = _tsb_cfg(dict(CFG, C=64))
+        self.oc = oracle.Config(**dict(CFG, C=64))
+        self.p = oracle.init_params(self.oc, seed).astype(np.float64)
+        self.m = np.zeros_like(self.p)
+        self.v = np.zeros_like(self.p)
+        self.t = 0
+        self.k = 0
+        layout, n_store = tsb.storage_layout(self.cfg)
+        self.map = []  # (canonical offset, storage offset, logical length)
+        for (name, off, n, _), t in zip(layout, oracle.tensors(self.oc)):
+            assert name.split(".")[-1] == t.name.split(".")[-1] and t.size <= n
+            self.map.append((t.offset, off, t.size))
+        self.g = torch.zeros(n_store, dtype=torch.float64)
+        self.last = None
+
+    def grad_tensor(self):
+        return self.g
+
+    def set_grad_events(self, events):
+        pass
+
+    def forward_backward(self, tok, tgt, want_loss=True):
+        import oracle
+        loss, g = oracle.forward_backward(self.oc, self.p, tok, tgt)
+        for co, so, n in self.map:
+            self.g[so:so + n] += torch.from_numpy(g[co:co + n])
+        self.k += 1
+        self.last = loss
+        return loss if want_loss else None
+
+    def read_loss(self):
+        return self.last
+
+    def step(self, lr, wd, b1, b2):
+        import oracle
+        G = np.zeros_like(self.p)
+        for co, so, n in self.map:
+            G[co:co + n] = self.g[so:so + n].numpy()
+        self.t += 1
+        self.p, self.m, self.v, gn = oracle.adamw_step(self.oc, self.p, G / self.k, self.m, self.v, self.t, lr, wd,
+                                                       b1, b2)
+        self.g.zero_()
+        self.k = 0
+        return gn
+
+
+def _bucketed_rank(rank, world, port, out_dir):
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from train_step_b200 import dp, synth
+    from train_step_b200.schedule import CosineSchedule
+    from train_step_b200.trainer import Trainer
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    model = _StorageOracleModel(13)
+    tr = Trainer(model, CosineSchedule(1e-3, 1e-4, 1, 4), exchange=dp.BucketedAllReduce(model))
+    losses = []
+    for step in range(3):
+        mbs = [synth.micro_batch(2, CFG["T"], CFG["V"], index=i, dist="uniform")
+               for i in dp.micro_batch_indices(rank, world, ACCUM, step=step)]
+        losses.append(tr.train_step(mbs)["loss"])
+    np.save(os.path.join(out_dir, f"bp{rank}.npy"), model.p)
+    np.save(os.path.join(out_dir, f"bl{rank}.npy"), np.array(losses))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_bucketed_exchange_two_rank_gloo_matches_single_process(tmp_path):
+    """Three steps of the training driver with the bucketed exchange (gradients averaged
+    bucket by bucket, reverse layer order, over the library's storage layout) on two gloo
+    ranks equal one process accumulating every micro-batch; the reported loss is the mean
+    of the rank's own micro-batch losses."""
+    from train_step_b200 import dp, synth
+    from train_step_b200.schedule import CosineSchedule
+    from train_step_b200.trainer import Trainer
+    world = 2
+    mp.start_processes(_bucketed_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       start_method="spawn")
+    p_r = [np.load(tmp_path / f"bp{r}.npy") for r in range(world)]
+    assert np.array_equal(p_r[0], p_r[1])
+    model = _StorageOracleModel(13)
+    tr = Trainer(model, CosineSchedule(1e-3, 1e-4, 1, 4))
+    for step in range(3):
+        idx = [i for r in range(world) for i in dp.micro_batch_indices(r, world, ACCUM, step=step)]
+        tr.train_step([synth.micro_batch(2, CFG["T"], CFG["V"], index=i, dist="uniform") for i in idx])
+    assert np.max(np.abs(p_r[0] - model.p)) < 1e-12
+    l0 = np.load(tmp_path / "bl0.npy")
+    assert np.all(np.isfinite(l0)) and l0.shape == (3,)

@@ -180,7 +180,7 @@ def test_gemm_fp32_simt(a_mn, b_mn, epi):
 # LayerNorm
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("N,C", [(1000, 768), (77, 1600), (512, 128), (16384, 768), (3001, 1024), (5, 768),
-                                 (2371, 256)])
+                                 (2371, 256), (9999, 1024), (9473, 256)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_layernorm_fwd_bwd(N, C, dtype):
     x = randn((N, C), 20, torch.float32, scale=2.0) + 0.5

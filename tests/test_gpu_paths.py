@@ -244,3 +244,51 @@ def test_sharded_step_equals_the_full_step():
     assert abs(l1 - l0) <= 1e-5 * abs(l0)
     for mdl in models:
         mdl.close()
+
+
+# ---------------------------------------------------------------------------
+# Gradient-bucket events of the overlapped data-parallel exchange
+# ---------------------------------------------------------------------------
+def test_grad_bucket_events_and_the_overlapped_exchange():
+    """gpt2_set_grad_events: the next backward pass records one event per gradient bucket,
+    in the order L-1, ..., 0, L (device timestamps), leaves the gradients bit-identical to
+    a run without events and the loss readable later (gpt2_read_loss); the training
+    driver with the bucketed exchange (one process: the exchange only waits on the events)
+    takes the same steps as without it."""
+    from train_step_b200 import dp
+    from train_step_b200.schedule import CosineSchedule
+    from train_step_b200.trainer import Trainer
+    cfg = tsb.Config(L=3, H=2, C=128, T=128, V=1000, tied=1, qkv_bias=1, dtype=tsb.BF16, B_max=2)
+    stream = torch.cuda.current_stream().cuda_stream
+    a = tsb.GPT2(cfg, seed=3, stream=stream)
+    b = tsb.GPT2(cfg, seed=3, stream=stream)
+    tok, tgt = synth.micro_batch(2, cfg.T, cfg.V, index=7)
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(cfg.L + 1)]
+    for e in events:
+        e.record()
+    torch.cuda.synchronize()
+    a.set_grad_events(events)
+    a.forward_backward(tok, tgt, want_loss=False)
+    la = a.read_loss()
+    lb = b.forward_backward(tok, tgt)
+    torch.cuda.synchronize()
+    assert la == lb
+    order = list(range(cfg.L - 1, -1, -1)) + [cfg.L]
+    for x, y in zip(order, order[1:]):
+        assert events[x].elapsed_time(events[y]) >= 0.0, (x, y)
+    assert np.array_equal(a.get_grads(), b.get_grads())
+    with pytest.raises(tsb.Gpt2Error) as e:
+        a.set_grad_events(events[:2])
+    assert e.value.code == -1
+    a.zero_grad()
+    b.zero_grad()
+    sched = CosineSchedule(1e-3, 1e-4, 1, 4)
+    ta = Trainer(a, sched, exchange=dp.BucketedAllReduce(a))
+    tb = Trainer(b, sched)
+    for step in range(2):
+        mbs = [synth.micro_batch(2, cfg.T, cfg.V, index=10 + 2 * step + i) for i in range(2)]
+        ra, rb = ta.train_step(mbs), tb.train_step(mbs)
+        assert ra["loss"] == rb["loss"] and ra["grad_norm"] == rb["grad_norm"]
+    assert np.array_equal(a.get_params(), b.get_params())
+    a.close()
+    b.close()

@@ -100,6 +100,10 @@ _SYMBOLS = {
                          ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_param_buffer": ([ct.c_void_p, ct.POINTER(ct.c_void_p), ct.POINTER(ct.c_int64)], ct.c_int),
     "gpt2_refresh_shadow": ([ct.c_void_p], ct.c_int),
+    "gpt2_storage_layout": ([ct.POINTER(_Config), ct.c_int, ct.c_char_p, ct.c_int, ct.POINTER(ct.c_int64),
+                             ct.POINTER(ct.c_int64), ct.POINTER(ct.c_int), ct.POINTER(ct.c_int64)], ct.c_int),
+    "gpt2_set_grad_events": ([ct.c_void_p, ct.POINTER(ct.c_void_p), ct.c_int], ct.c_int),
+    "gpt2_read_loss": ([ct.c_void_p, ct.POINTER(ct.c_float)], ct.c_int),
     "gpt2_op_last_error": ([], ct.c_char_p),
 }
 
@@ -161,6 +165,38 @@ class Config:
         return _Config(self.L, self.H, self.C, self.T, self.V, self.tied, self.qkv_bias, self.dtype, self.B_max)
 
 
+def storage_layout(cfg: Config):
+    """Host-side storage layout of a configuration (no GPU needed): a list of
+    (name, offset, length, bucket) per tensor in canonical order, and the storage length."""
+    c = cfg.c()
+    name = ct.create_string_buffer(64)
+    off, n, ns = ct.c_int64(), ct.c_int64(), ct.c_int64()
+    b = ct.c_int()
+    out = []
+    i = 0
+    while lib().gpt2_storage_layout(ct.byref(c), i, name, 64, ct.byref(off), ct.byref(n), ct.byref(b),
+                                    ct.byref(ns)) == 0:
+        out.append((name.value.decode(), off.value, n.value, b.value))
+        i += 1
+    if not out:
+        raise Gpt2Error(-1, "invalid configuration")
+    return out, ns.value
+
+
+def bucket_ranges(cfg: Config):
+    """Storage ranges [(offset, length), ...] of each gradient bucket 0 .. L (adjacent
+    tensors of one bucket merged, the padding between them included)."""
+    layout, _ = storage_layout(cfg)
+    per = [[] for _ in range(cfg.L + 1)]
+    for _, off, n, b in sorted(layout, key=lambda t: t[1]):
+        r = per[b]
+        if r and r[-1][0] + r[-1][1] >= off - 63:  # contiguous up to the 64-float alignment
+            r[-1] = (r[-1][0], off + n - r[-1][0])
+        else:
+            r.append((off, n))
+    return per
+
+
 class GPT2:
     """One model handle: parameters, gradients, Adam state and activations on the GPU."""
 
@@ -199,6 +235,12 @@ class GPT2:
         self._check(lib().gpt2_forward_backward(self.h, _ptr(tokens), _ptr(targets), B, T,
                                                 ct.byref(loss) if want_loss else None))
         return loss.value if want_loss else None
+
+    def read_loss(self) -> float:
+        """Mean loss of the most recent forward_backward / forward (waits for the GPU)."""
+        loss = ct.c_float()
+        self._check(lib().gpt2_read_loss(self.h, ct.byref(loss)))
+        return loss.value
 
     def forward(self, tokens, targets):
         B, T = tokens.shape
@@ -278,6 +320,13 @@ class GPT2:
         v = _View()
         v.__cuda_array_interface__ = {"shape": (n,), "typestr": "<f4", "data": (ptr, False), "version": 3}
         return torch.as_tensor(v, device="cuda")
+
+    def set_grad_events(self, events) -> None:
+        """Arm the next forward_backward to record events[b] (torch.cuda.Event objects that
+        have been recorded once, or raw handles) as gradient bucket b completes; [] cancels."""
+        hs = [e.cuda_event if hasattr(e, "cuda_event") else int(e) for e in events]
+        arr = (ct.c_void_p * max(1, len(hs)))(*hs)
+        self._check(lib().gpt2_set_grad_events(self.h, arr, len(hs)))
 
     def grad_tensor(self):
         """Zero-copy fp32 CUDA tensor over the flat gradient storage (the library's padded

@@ -46,6 +46,8 @@ struct gpt2 {
   int act_bytes = 4;
   std::vector<TensorSlot> tensors;
   int64_t n_logical = 0, n_store = 0, n_decay = 0;
+  // one-shot: events the next backward pass records as gradient buckets complete
+  std::vector<cudaEvent_t> grad_events;
   // parameter state (device)
   float *p = nullptr, *g = nullptr, *m = nullptr, *v = nullptr;
   bf16* shadow = nullptr;
@@ -208,6 +210,29 @@ void build_tensors(gpt2* m) {
   m->n_store = (d + 4095) / 4096 * 4096;
 }
 
+// Gradient bucket of canonical tensor i: layer l's tensors form bucket l, everything else
+// (embeddings, final LayerNorm, untied head) bucket L. The backward pass completes the
+// buckets in the order L-1, ..., 0, L.
+int tensor_bucket(const gpt2* m, size_t i) {
+  const std::string& n = m->tensors[i].name;
+  if (n.size() > 1 && n[0] == 'h' && n[1] >= '0' && n[1] <= '9') return std::atoi(n.c_str() + 1);
+  return m->cfg.L;
+}
+
+// Record grad_events[b] once bucket b's gradients are complete: on the side stream (after
+// everything the main stream has enqueued) when there is one, so the main stream never waits.
+int mark_bucket(gpt2* m, const LaunchCtx& cb, int b) {
+  if (m->grad_events.empty()) return GPT2_OK;
+  cudaStream_t s = cb.stream;
+  if (cb.side) {
+    CK(m, cudaEventRecord(cb.side->ready, cb.stream));
+    CK(m, cudaStreamWaitEvent(cb.side->s, cb.side->ready, 0));
+    s = cb.side->s;
+  }
+  CK(m, cudaEventRecord(m->grad_events[b], s));
+  return GPT2_OK;
+}
+
 void host_init(const gpt2* m, uint64_t seed, std::vector<float>& out) {
   out.assign(m->n_logical, 0.f);
   for (size_t i = 0; i < m->tensors.size(); ++i) {
@@ -320,7 +345,9 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
   // ---------------- head + cross-entropy, chunk by chunk ----------------
   // bf16 backward: reductions of gradient partials run on the side stream (cb)
   LaunchCtx cb = c;
-  if (backward && dt == GPT2_BF16) cb.side = &m->side;
+  // the reductions overlap on the side stream, except while per-kernel times are being
+  // recorded (an event pair around a kernel that shares the GPU would charge it the overlap)
+  if (backward && dt == GPT2_BF16 && !m->prof.on) cb.side = &m->side;
   const float* headw = m->cfg.tied ? m->wte : m->head;
   float* g_head = m->cfg.tied ? m->g_wte : m->g_head;
   const int chunk = N < HEAD_CHUNK_ROWS ? N : HEAD_CHUNK_ROWS;
@@ -438,10 +465,14 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
                             nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
     RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b,
             l > 0 ? m->lg[l - 1].pj_b : nullptr));
+    RK(mark_bucket(m, cb, l));  // layer l's pj_b came from layer l + 1's LayerNorm (or ln_f)
   }
   EmbScratch es = emb_scratch_carve(m->emb_scratch, N, C);
   RK(embedding_bwd(c, m->tok, m->dres, B, T, C, m->cfg.V, m->g_wte, m->g_wpe, es));
-  return side_join(cb);  // every gradient is complete on the main stream from here on
+  RK(side_join(cb));  // every gradient is complete on the main stream from here on
+  RK(mark_bucket(m, c, L));
+  m->grad_events.clear();
+  return GPT2_OK;
 }
 
 int validate_batch(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, int T) {
@@ -648,6 +679,12 @@ int gpt2_forward(gpt2* m, const int32_t* tokens, const int32_t* targets, int B, 
     RK(check_device_error(m));
   }
   return GPT2_OK;
+}
+
+int gpt2_read_loss(gpt2* m, float* loss_out) {
+  if (!m || !loss_out) return GPT2_ERR_CONFIG;
+  CK(m, cudaMemcpyAsync(loss_out, m->d_loss, 4, cudaMemcpyDeviceToHost, m->stream));
+  return check_device_error(m);
 }
 
 int gpt2_step(gpt2* m, float lr, float wd, float beta1, float beta2, float* grad_norm_out) {
@@ -1017,6 +1054,37 @@ int gpt2_grad_buffer(gpt2* m, float** dev, int64_t* n) {
   return GPT2_OK;
 }
 
+int gpt2_storage_layout(const gpt2_config* cfg, int i, char* name, int name_len, int64_t* offset, int64_t* n,
+                        int* bucket, int64_t* n_store) {
+  if (!cfg || cfg->L <= 0 || cfg->C <= 0 || cfg->V <= 0 || cfg->T <= 0 || cfg->C % 64) return GPT2_ERR_CONFIG;
+  gpt2 m;  // host-side layout only: no device state
+  m.cfg = *cfg;
+  m.Vp = (cfg->V + 63) / 64 * 64;
+  build_tensors(&m);
+  if (n_store) *n_store = m.n_store;
+  if (i < 0 || i >= (int)m.tensors.size()) return GPT2_ERR_CONFIG;
+  const TensorSlot& t = m.tensors[i];
+  if (name && name_len > 0) std::snprintf(name, name_len, "%s", t.name.c_str());
+  if (offset) *offset = t.dev_off;
+  if (n) *n = t.dev_rows * t.cols;
+  if (bucket) *bucket = tensor_bucket(&m, i);
+  return GPT2_OK;
+}
+
+int gpt2_set_grad_events(gpt2* m, void* const* events, int n) {
+  if (!m) return GPT2_ERR_CONFIG;
+  if (n == 0) {
+    m->grad_events.clear();
+    return GPT2_OK;
+  }
+  if (n != m->cfg.L + 1 || !events) return set_err(m, GPT2_ERR_CONFIG, "expected L + 1 events");
+  for (int i = 0; i < n; ++i)
+    if (!events[i]) return set_err(m, GPT2_ERR_CONFIG, "null event");
+  m->grad_events.assign(reinterpret_cast<const cudaEvent_t*>(events),
+                        reinterpret_cast<const cudaEvent_t*>(events) + n);
+  return GPT2_OK;
+}
+
 int gpt2_profile(gpt2* m, int enable) {
   if (!m) return GPT2_ERR_CONFIG;
   if (enable) m->prof.reset();
@@ -1228,6 +1296,10 @@ int gpt2_op_layernorm_fwd(int dtype, const float* x, const float* g, const float
   OpCtx o(stream);
   if (C % 4 || C > 2048 || N <= 0) {
     g_op_error = "layernorm: C % 4 == 0, C <= 2048, N > 0 required";
+    return GPT2_ERR_CONFIG;
+  }
+  if (((uintptr_t)x | (uintptr_t)g | (uintptr_t)b | (uintptr_t)y) & 15) {
+    g_op_error = "layernorm: x, g, b and y must start on 16-byte boundaries";
     return GPT2_ERR_CONFIG;
   }
   return dtype == GPT2_BF16 ? layernorm_fwd_t<bf16>(o.c, x, g, b, N, C, (bf16*)y, mean, rstd)

@@ -42,6 +42,7 @@ def reduce_scatter_mean_(tensor, lo: int, hi: int, group=None) -> None:
     """tensor[lo:hi] <- the average over the ranks of their tensor[lo:hi] (this rank's
     shard of an equal split). NCCL reduces in place into the shard; gloo, which has no
     reduce-scatter, all-reduces the whole tensor (the same values in the shard)."""
+    import torch
     import torch.distributed as dist
     world = dist.get_world_size(group)
     if world == 1:
@@ -92,3 +93,70 @@ def zero1_step(model, lr: float, wd: float, beta1: float = 0.9, beta2: float = 0
     all_gather_shards_(model.param_tensor(), lo, hi, group)
     model.refresh_shadow()
     model.zero_grad()
+
+
+class BucketedAllReduce:
+    """Average of the accumulated gradients over the ranks, one bucket at a time (bucket l
+    holds layer l's tensors, bucket L the embeddings, final LayerNorm and untied head),
+    each bucket's all-reduce starting on a stream of its own as soon as the backward pass
+    of the last micro-batch has finished that bucket (gpt2_set_grad_events), so the
+    exchange overlaps the rest of that backward pass. Reverse layer order, as the
+    backward pass produces them.
+
+        ex = BucketedAllReduce(model)
+        for i, (tok, tgt) in enumerate(micro_batches):
+            if i == len(micro_batches) - 1:
+                ex.arm()
+            model.forward_backward(tok, tgt, want_loss=False)
+        ex.run()        # enqueues the exchange and orders the current stream after it
+        model.step(...)
+
+    The model must run on torch's current stream. Without CUDA (a CPU process group and
+    a CPU gradient tensor) run() reduces the buckets in the same order, synchronously.
+    """
+
+    def __init__(self, model, group=None, ranges=None):
+        import torch
+        from . import bucket_ranges
+        self.model, self.group = model, group
+        self.L = model.cfg.L
+        self.ranges = ranges if ranges is not None else bucket_ranges(model.cfg)
+        self.order = list(range(self.L - 1, -1, -1)) + [self.L]
+        self.cuda = torch.cuda.is_available() and model.grad_tensor().is_cuda
+        self.events = []
+        if self.cuda:
+            self.stream = torch.cuda.Stream()
+            self.events = [torch.cuda.Event() for _ in range(self.L + 1)]
+            for e in self.events:  # creates the CUDA events (completed at once)
+                e.record()
+        self.armed = False
+
+    def arm(self) -> None:
+        """Before the last micro-batch's forward_backward."""
+        if self.cuda:
+            self.model.set_grad_events(self.events)
+        self.armed = True
+
+    def run(self) -> None:
+        """After the last micro-batch's forward_backward has returned: the all-reduces,
+        each waiting for its bucket; then the current stream waits for all of them."""
+        import torch
+        import torch.distributed as dist
+        if not self.armed:
+            raise RuntimeError("arm() before the last micro-batch")
+        self.armed = False
+        g = self.model.grad_tensor()
+        world = dist.get_world_size(self.group) if dist.is_available() and dist.is_initialized() else 1
+        if not self.cuda:
+            if world > 1:
+                for b in self.order:
+                    for off, n in self.ranges[b]:
+                        allreduce_mean_(g[off:off + n], self.group)
+            return
+        with torch.cuda.stream(self.stream):
+            for b in self.order:
+                self.stream.wait_event(self.events[b])
+                if world > 1:
+                    for off, n in self.ranges[b]:
+                        allreduce_mean_(g[off:off + n], self.group)
+        torch.cuda.current_stream().wait_stream(self.stream)

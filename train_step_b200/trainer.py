@@ -22,19 +22,41 @@ def _sync_torch_stream() -> None:
 
 
 class Trainer:
+    """`exchange` (e.g. dp.BucketedAllReduce; the model on torch's current stream) averages
+    the gradients over data-parallel ranks while the last micro-batch's backward pass
+    runs, ordered by streams alone; `allreduce` (a callable run after the backward pass,
+    on torch's current stream) is the plain form, followed by a host synchronisation."""
+
     def __init__(self, model, schedule: Callable[[int], float] | None = None, weight_decay: float = 0.1,
-                 beta1: float = 0.9, beta2: float = 0.95, allreduce: Callable[[], None] | None = None):
+                 beta1: float = 0.9, beta2: float = 0.95, allreduce: Callable[[], None] | None = None,
+                 exchange=None):
         self.model = model
         self.schedule = schedule or CosineSchedule()
         self.weight_decay = weight_decay
         self.beta1 = beta1
         self.beta2 = beta2
         self.allreduce = allreduce
+        self.exchange = exchange
         self.step = 0
 
     def train_step(self, micro_batches: Iterable) -> dict:
         """One optimizer step over the (tokens, targets) micro-batches: returns the mean
         micro-batch loss, the pre-clip gradient norm and the learning rate used."""
+        if self.exchange is not None:
+            mbs = list(micro_batches)
+            losses = []
+            for i, (tok, tgt) in enumerate(mbs):
+                if i == len(mbs) - 1:
+                    self.exchange.arm()
+                    self.model.forward_backward(tok, tgt, want_loss=False)
+                    self.exchange.run()  # enqueued before the host waits for the loss
+                    losses.append(self.model.read_loss())
+                else:
+                    losses.append(self.model.forward_backward(tok, tgt))
+            lr = self.schedule(self.step)
+            gnorm = self.model.step(lr, self.weight_decay, self.beta1, self.beta2)
+            self.step += 1
+            return {"loss": sum(losses) / len(losses), "grad_norm": gnorm, "lr": lr, "step": self.step}
         losses = [self.model.forward_backward(tok, tgt) for tok, tgt in micro_batches]
         if self.allreduce is not None:
             # the gradients are complete (each forward_backward returned its loss); the
