@@ -339,15 +339,23 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
   auto rstd = [&](int i) { return m->stat_rstd + (int64_t)i * m->Nmax; };
   auto ACT = [&](char* base, int l, int64_t per) -> void* { return base + (int64_t)l * per * ab; };
 
+  // bf16 backward: reductions of gradient partials run on the side stream (cb); they
+  // overlap, except while per-kernel times are being recorded (an event pair around a
+  // kernel that shares the GPU would charge it the overlap)
+  LaunchCtx cb = c;
+  if (backward && dt == GPT2_BF16 && !m->prof.on) cb.side = &m->side;
+  EmbScratch es = emb_scratch_carve(m->emb_scratch, N, C);
+  if (backward && cb.side) {
+    // the embedding backward's sort of the token ids needs only the tokens: it runs on the
+    // side stream (one CTA) under the forward pass; the embedding backward waits for it
+    RK(token_sort(side_ctx(cb), m->tok, N, m->cfg.V, es));
+    side_mark_free(cb, SIDE_EMB);
+  }
+
   // ---------------- forward ----------------
   RK(forward_layers(m, B, T));
 
   // ---------------- head + cross-entropy, chunk by chunk ----------------
-  // bf16 backward: reductions of gradient partials run on the side stream (cb)
-  LaunchCtx cb = c;
-  // the reductions overlap on the side stream, except while per-kernel times are being
-  // recorded (an event pair around a kernel that shares the GPU would charge it the overlap)
-  if (backward && dt == GPT2_BF16 && !m->prof.on) cb.side = &m->side;
   const float* headw = m->cfg.tied ? m->wte : m->head;
   float* g_head = m->cfg.tied ? m->g_wte : m->g_head;
   const int chunk = N < HEAD_CHUNK_ROWS ? N : HEAD_CHUNK_ROWS;
@@ -467,8 +475,8 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
             l > 0 ? m->lg[l - 1].pj_b : nullptr));
     RK(mark_bucket(m, cb, l));  // layer l's pj_b came from layer l + 1's LayerNorm (or ln_f)
   }
-  EmbScratch es = emb_scratch_carve(m->emb_scratch, N, C);
-  RK(embedding_bwd(c, m->tok, m->dres, B, T, C, m->cfg.V, m->g_wte, m->g_wpe, es));
+  RK(side_wait_free(cb, SIDE_EMB));  // the token sort (side stream) has finished
+  RK(embedding_bwd(c, m->tok, m->dres, B, T, C, m->cfg.V, m->g_wte, m->g_wpe, es, cb.side != nullptr));
   RK(side_join(cb));  // every gradient is complete on the main stream from here on
   RK(mark_bucket(m, c, L));
   m->grad_events.clear();

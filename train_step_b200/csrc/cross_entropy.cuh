@@ -78,24 +78,44 @@ __global__ void __launch_bounds__(CE_STHREADS) cross_entropy_stats_kernel(
   __syncthreads();
   const int nvec = (int)(ld / 8);
   const int nrows = (int)min((long long)CE_SROWS, (long long)rows - r0);
-  for (int i = threadIdx.x; i < nrows * nvec; i += CE_STHREADS) {
-    const int rr = i / nvec, vi = i - rr * nvec;
-    uint4* ptr = reinterpret_cast<uint4*>(logits + (r0 + rr) * ld) + vi;
-    const uint4 u = *ptr;
+  for (int rr = 0; rr < nrows; ++rr) {
     const float lse2 = s_lse2[rr];
     const int t = s_tgt[rr];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t o[4];
+    uint4* rowv = reinterpret_cast<uint4*>(logits + (r0 + rr) * ld);
+    // dlogits of the 8 columns of vector vi
+    auto grad8 = [&](const uint4 u, int vi) -> uint4 {
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      uint32_t o[4];
+      const int c0 = vi * 8;
+      if (c0 + 8 <= V && (unsigned)(t - c0) >= 8u) {
+        // the common vector: all 8 columns inside the vocabulary, none of them the target
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 f = unpack_bf16x2(w[q]);
-      const int c = vi * 8 + 2 * q;
-      float a = 0.f, b = 0.f;
-      if (c < V) a = (ex2_approx(fmaf(f.x, LOG2E_CE, -lse2)) - (c == t ? 1.f : 0.f)) * scale;
-      if (c + 1 < V) b = (ex2_approx(fmaf(f.y, LOG2E_CE, -lse2)) - (c + 1 == t ? 1.f : 0.f)) * scale;
-      o[q] = pack_bf16x2(a, b);
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = unpack_bf16x2(w[q]);
+          o[q] = pack_bf16x2(ex2_approx(fmaf(f.x, LOG2E_CE, -lse2)) * scale,
+                             ex2_approx(fmaf(f.y, LOG2E_CE, -lse2)) * scale);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = unpack_bf16x2(w[q]);
+          const int c = c0 + 2 * q;
+          float a = 0.f, b = 0.f;
+          if (c < V) a = (ex2_approx(fmaf(f.x, LOG2E_CE, -lse2)) - (c == t ? 1.f : 0.f)) * scale;
+          if (c + 1 < V) b = (ex2_approx(fmaf(f.y, LOG2E_CE, -lse2)) - (c + 1 == t ? 1.f : 0.f)) * scale;
+          o[q] = pack_bf16x2(a, b);
+        }
+      }
+      return make_uint4(o[0], o[1], o[2], o[3]);
+    };
+    // two vectors per thread and iteration: both loads are in flight before either is used
+    for (int vi = threadIdx.x; vi < nvec; vi += 2 * CE_STHREADS) {
+      const int vj = vi + CE_STHREADS;
+      const uint4 u0 = rowv[vi];
+      const uint4 u1 = vj < nvec ? rowv[vj] : make_uint4(0u, 0u, 0u, 0u);
+      rowv[vi] = grad8(u0, vi);
+      if (vj < nvec) rowv[vj] = grad8(u1, vj);
     }
-    *ptr = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 

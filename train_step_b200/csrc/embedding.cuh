@@ -242,7 +242,9 @@ __global__ void __launch_bounds__(EMB_SORT_THREADS) token_sort_kernel(const int*
   }
 }
 
-// Stage 1: partial[c][:] = sum of dx0 rows of chunk c, in sorted order.
+// Stage 1: partial[c][:] = sum of dx0 rows of chunk c, in sorted order. The rows of a
+// chunk are fetched 8 at a time (independent loads in flight) and added in index order,
+// so the sum is the plain sequential one.
 __global__ void embed_chunk_sum_kernel(const float* __restrict__ dx0, const int* __restrict__ sorted_pos,
                                        const int* __restrict__ chunk_start, const int* __restrict__ counts, int C,
                                        float* __restrict__ partial) {
@@ -251,12 +253,19 @@ __global__ void embed_chunk_sum_kernel(const float* __restrict__ dx0, const int*
     const int a = chunk_start[ch], b = chunk_start[ch + 1];
     for (int c = threadIdx.x * 4; c < C; c += blockDim.x * 4) {
       float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int i = a; i < b; ++i) {
-        const float4 v = *reinterpret_cast<const float4*>(dx0 + (long long)sorted_pos[i] * C + c);
-        s.x += v.x;
-        s.y += v.y;
-        s.z += v.z;
-        s.w += v.w;
+      for (int i = a; i < b; i += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (i + u < b) v[u] = __ldg(reinterpret_cast<const float4*>(dx0 + (long long)sorted_pos[i + u] * C + c));
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (i + u < b) {
+            s.x += v[u].x;
+            s.y += v[u].y;
+            s.z += v[u].z;
+            s.w += v[u].w;
+          }
       }
       *reinterpret_cast<float4*>(partial + (long long)ch * C + c) = s;
     }
@@ -286,18 +295,25 @@ __global__ void embed_seg_sum_kernel(const float* __restrict__ partial, const in
   }
 }
 
-// dwpe[t, :] += sum_b dx0[b*T + t, :]
+// dwpe[t, :] += sum_b dx0[b*T + t, :] (the Bsz rows fetched 8 at a time, added in order)
 __global__ void embed_pos_grad_kernel(const float* __restrict__ dx0, int Bsz, int T, int C, float* __restrict__ dwpe) {
   const long long i = (blockIdx.x * (long long)blockDim.x + threadIdx.x) * 4;
   if (i >= (long long)T * C) return;
   const int t = (int)(i / C), c = (int)(i % C);
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int b = 0; b < Bsz; ++b) {
-    const float4 v = *reinterpret_cast<const float4*>(dx0 + ((long long)b * T + t) * C + c);
-    s.x += v.x;
-    s.y += v.y;
-    s.z += v.z;
-    s.w += v.w;
+  for (int b0 = 0; b0 < Bsz; b0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (b0 + u < Bsz) v[u] = __ldg(reinterpret_cast<const float4*>(dx0 + ((long long)(b0 + u) * T + t) * C + c));
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (b0 + u < Bsz) {
+        s.x += v[u].x;
+        s.y += v[u].y;
+        s.z += v[u].z;
+        s.w += v[u].w;
+      }
   }
   float4 o = *reinterpret_cast<float4*>(dwpe + i);
   *reinterpret_cast<float4*>(dwpe + i) = make_float4(o.x + s.x, o.y + s.y, o.z + s.z, o.w + s.w);

@@ -11,8 +11,8 @@
 //   warp 0      TMA producer: 128-byte-swizzled tiles into a STAGES-deep ring
 //   warp 1      one thread issues tcgen05.mma (M=128, N=BN, K=16) into TMEM;
 //               the warp also owns the TMEM allocation
-//   warps 2..9  epilogue: tcgen05.ld 32 lanes x 32 columns, fused bias / GELU /
-//               residual / GELU' math, global stores. Two TMEM accumulators
+//   warps 2..    epilogue (8 or 16 warps): tcgen05.ld 32 lanes x 32 columns, fused
+//               bias / GELU / residual / GELU' math, TMA stores. Two TMEM accumulators
 //               (2 x BN columns) let the epilogue of one tile overlap the main
 //               loop of the next.
 // No cluster multicast is used (tiles are fetched per CTA from L2).
@@ -56,8 +56,15 @@ struct GemmParams {
 
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
-constexpr int TC_THREADS = 320;
-constexpr int TC_EPI_WARPS = 8;
+// Epilogue warps: 8 (two per TMEM lane quarter, each draining half of the tile's columns),
+// or 16 where that measured faster on B200: the residual add (fp32 in and out, latency-bound
+// on its chunk chain; 16384 x 768 x 768: 39.1 -> 36.3 us) and GELU with two outputs (81.9 ->
+// 79.8 us). GELU backward with the bias column sums is issue-bound and lost with 16 (88.6 ->
+// 95.5 us), so it keeps 8.
+template <int EPI>
+__host__ __device__ constexpr int tc_epi_warps() {
+  return (EPI == EPI_BF16_GELU || EPI == EPI_F32_RESID) ? 16 : 8;
+}
 
 // PAIR: a 2-CTA cluster computes one (2 * TC_BM) x BN tile with M = 256 MMAs that
 // span both SMs' tensor cores. Each CTA stages its own 128 rows of A and its own
@@ -67,17 +74,21 @@ constexpr int TC_EPI_WARPS = 8;
 // four 2 KB chunk buffers per epilogue warp so that the auxiliary tile of chunk n + 3 is
 // in flight while chunk n is computed (one chunk of lookahead left the epilogue waiting
 // on every load), at the price of one main-loop stage.
-template <int BN, bool PAIR = false, bool AUX = false>
+template <int BN, bool PAIR = false, bool AUX = false, int EPW = 8>
 struct TcCfg {
+  static constexpr int THREADS = (2 + EPW) * 32;
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // B rows staged by one CTA
   static constexpr int B_BYTES = B_ROWS * TC_BK * 2;
   static constexpr int UNIT_M = PAIR ? 2 * TC_BM : TC_BM;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int NBUF = AUX ? 4 : 2;                   // 2 KB chunk buffers per epilogue warp
-  static constexpr int STAGING = TC_EPI_WARPS * NBUF * 2048;
+  // 2 KB chunk buffers per epilogue warp: with 8 warps an auxiliary tile gets 3 chunks of
+  // lookahead; 16 warps keep as many chunks in flight with one each
+  static constexpr int NBUF = (AUX && EPW == 8) ? 4 : 2;
+  static constexpr int STAGING = EPW * NBUF * 2048;
   static constexpr int BARS = 512;                           // mbarriers, TMEM slot, abort flag
   static constexpr int STAGES = (232448 - 1024 - BARS - STAGING) / STAGE;
+  static_assert(8 * (2 * STAGES + 6 + NBUF * EPW) <= BARS, "barrier space");
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
   static constexpr int SMEM = STAGES * STAGE + STAGING + 1024 + BARS;
 };
@@ -229,11 +240,12 @@ __device__ __forceinline__ void tc_decode_unit(const GemmParams& p, int unit, in
 // arrive on both ranks' `empty` / `tfull` barriers; both ranks' epilogue warps
 // arrive on the leader's `tempty`. No load is multicast.
 template <int BN, bool A_MN, bool B_MN, int EPI, bool PAIR>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__((2 + tc_epi_warps<EPI>()) * 32, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                    const GemmParams p) {
-  using Cfg = TcCfg<BN, PAIR, tc_has_aux<EPI>()>;
+  constexpr int EPW = tc_epi_warps<EPI>();
+  using Cfg = TcCfg<BN, PAIR, tc_has_aux<EPI>(), EPW>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int UNIT_M = Cfg::UNIT_M;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
@@ -249,7 +261,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint64_t* auxbar = drain + 2;  // [TC_EPI_WARPS][NBUF]: auxiliary tile landed in chunk buffer b
+  uint64_t* auxbar = drain + 2;  // [EPW][NBUF]: auxiliary tile landed in chunk buffer b
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -261,10 +273,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], PAIR ? 2 * TC_EPI_WARPS : TC_EPI_WARPS);
+      mbar_init(&tempty[a], PAIR ? 2 * EPW : EPW);
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < Cfg::NBUF * TC_EPI_WARPS; ++i) mbar_init(&auxbar[i], 1);
+    for (int i = 0; i < Cfg::NBUF * EPW; ++i) mbar_init(&auxbar[i], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -440,10 +452,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // ---------------- epilogue warps ----------------
     constexpr int CW = tc_chunk_cols<EPI>();
     constexpr bool HAS_AUX = tc_has_aux<EPI>();
-    const int ew = warp - 2;         // 0..7
+    constexpr int NPART = EPW / 4;   // column parts of the tile (one warp per lane quarter each)
+    const int ew = warp - 2;         // 0 .. EPW - 1
     const int q = warp & 3;          // TMEM lane quarter this warp may access
-    const int half = ew >> 2;        // which half of the BN columns
-    const int c_begin = half * (BN / 2), c_end = (half + 1) * (BN / 2);
+    const int part = ew >> 2;        // which part of the BN columns
+    const int c_begin = part * (BN / NPART), c_end = (part + 1) * (BN / NPART);
     constexpr int NBUF = Cfg::NBUF;
     uint8_t* wbuf = staging + ew * (NBUF * 2048);  // chunk buffers: wbuf + b * 2048
     uint64_t* abar = auxbar + NBUF * ew;
@@ -456,7 +469,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // lane 0 tracks the loads in flight (bit b: buffer b) for the abort path
     uint32_t aux_pending = 0, aux_par = 0;
     const int rbase = (int)rank * TC_BM + q * 32;  // this warp's first row within a unit
-    constexpr int CPU_ = (BN / 2) / CW;             // chunks per unit for this warp
+    constexpr int CPU_ = (BN / NPART) / CW;         // chunks per unit for this warp
     // issue the auxiliary load of this warp's chunk g (g counted over all its units)
     auto aux_load = [&](int g) {
       const int unit_g = cid + (g / CPU_) * ncl;
@@ -479,7 +492,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int unit = cid; unit < p.num_units && ok; unit += ncl) {
       int tm, tn, ks;
       tc_decode_unit(p, unit, tm, tn, ks);
-      float st_m = -INFINITY, st_s = 0.f;  // this lane's row over this warp's half of the tile
+      float st_m = -INFINITY, st_s = 0.f;  // this lane's row over this warp's part of the tile
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, lim)) {
         if (lane == 0) {
           raise_device_error(p.err, DEV_TIMEOUT);
@@ -596,7 +609,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             st_m = nm;
           }
           if (c + CW == c_end && row0 + lane < p.M)
-            p.rowstats[(long long)(row0 + lane) * (2 * p.tiles_n) + tn * 2 + half] = make_float2(st_m, st_s);
+            p.rowstats[(long long)(row0 + lane) * (NPART * p.tiles_n) + tn * NPART + part] = make_float2(st_m, st_s);
         }
         if (EPI == EPI_BF16_DGELU && CW == 32 && p.colsum != nullptr && col0 < p.N && row0 < p.M) {
           // the bias gradient of the layer that produced the GELU input: column sums of this

@@ -97,7 +97,7 @@ struct Profiler {
 // next GEMM (they fit beside a GEMM's CTA on each SM). A partial buffer is written again
 // only after the reduction that reads it has finished (its `freed` event); the main
 // stream joins the side stream at the end of a micro-batch's backward pass.
-enum SideBuf : int { SIDE_LN = 0, SIDE_BIAS = 1, SIDE_WS0 = 2, SIDE_WS1 = 3, SIDE_NBUF = 4 };
+enum SideBuf : int { SIDE_LN = 0, SIDE_BIAS = 1, SIDE_WS0 = 2, SIDE_WS1 = 3, SIDE_EMB = 4, SIDE_NBUF = 5 };
 struct SideStream {
   cudaStream_t s = nullptr;
   cudaEvent_t ready = nullptr;  // recorded on the main stream before side work is enqueued
@@ -351,7 +351,9 @@ struct GemmDesc {
 // Tile width of a tensor-core GEMM: 256 when N >= 256 unless forced.
 inline int gemm_bn(const GemmDesc& d) { return d.bn == 128 || d.bn == 256 ? d.bn : (d.N >= 256 ? 256 : 128); }
 // Softmax partials per row that a GEMM with rowstats writes.
-inline int gemm_rowstats_count(const GemmDesc& d) { return 2 * ((d.N + gemm_bn(d) - 1) / gemm_bn(d)); }
+inline int gemm_rowstats_count(const GemmDesc& d) {
+  return (tc_epi_warps<EPI_BF16>() / 4) * ((d.N + gemm_bn(d) - 1) / gemm_bn(d));
+}
 
 struct TcMaps {
   CUtensorMap a, b, o, o2;
@@ -360,14 +362,16 @@ struct TcMaps {
 template <int BN, bool AM, bool BM_, int EPI, bool PAIR>
 int launch_tc_inst(const LaunchCtx& c, const TcMaps& tm, const GemmParams& p) {
   auto kern = gemm_tc_kernel<BN, AM, BM_, EPI, PAIR>;
-  constexpr int smem = TcCfg<BN, PAIR, tc_has_aux<EPI>()>::SMEM;
+  using Cfg = TcCfg<BN, PAIR, tc_has_aux<EPI>(), tc_epi_warps<EPI>()>;
+  constexpr int smem = Cfg::SMEM;
+  constexpr int threads = Cfg::THREADS;
   // shared-memory opt-in and, for pairs, the co-resident clusters: once per device
   const int max_clusters = per_device_once(reinterpret_cast<const void*>(kern), [&]() -> int {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return -1;
     if (!PAIR) return 0;
     cudaLaunchConfig_t q{};
     q.gridDim = dim3(2 * (c.num_sms / 2));
-    q.blockDim = dim3(TC_THREADS);
+    q.blockDim = dim3(threads);
     q.dynamicSmemBytes = smem;
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;
@@ -384,13 +388,13 @@ int launch_tc_inst(const LaunchCtx& c, const TcMaps& tm, const GemmParams& p) {
   if (max_clusters < 0) return fail(c, GPT2_ERR_CUDA, "gemm_tc: no 2-CTA cluster fits");
   if (!PAIR) {
     const int grid = p.num_units < c.num_sms ? p.num_units : c.num_sms;
-    kern<<<grid, TC_THREADS, smem, c.stream>>>(tm.a, tm.b, tm.o, tm.o2, p);
+    kern<<<grid, threads, smem, c.stream>>>(tm.a, tm.b, tm.o, tm.o2, p);
     return check_launch(c, "gemm_tc");
   }
   const int clusters = p.num_units < max_clusters ? p.num_units : max_clusters;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(2 * clusters);
-  cfg.blockDim = dim3(TC_THREADS);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = c.stream;
   cudaLaunchAttribute attr[1];
@@ -880,17 +884,21 @@ inline int token_sort(const LaunchCtx& c, const int* tok, int N, int V, const Em
   return check_launch(c, "token_sort");
 }
 
+// sorted: the scratch already holds this batch's token sort (run earlier, e.g. on a side
+// stream that the caller has waited for)
 inline int embedding_bwd(const LaunchCtx& c, const int* tok, const float* dx0, int Bsz, int T, int C, int V,
-                         float* dwte, float* dwpe, const EmbScratch& s) {
+                         float* dwte, float* dwpe, const EmbScratch& s, bool sorted = false) {
   const int N = Bsz * T;
   if (C % 4) return fail(c, GPT2_ERR_CONFIG, "embedding: C % 4 != 0");
   ProfScope ps(c, CAT_EMB_BWD, 0.0, 8.0 * N * C + 8.0 * T * C + 4.0 * N);
-  int r = token_sort(c, tok, N, V, s);
+  int r = sorted ? GPT2_OK : token_sort(c, tok, N, V, s);
   if (r) return r;
   const int grid = 8 * c.num_sms;
-  embed_chunk_sum_kernel<<<grid, 128, 0, c.stream>>>(dx0, s.sorted_pos, s.chunk_start, s.counts, C, s.partial);
+  // a float4 of the row per thread: 192 threads cover C = 768 in one pass
+  const int threads = std::min(256, std::max(32, (C / 4 + 31) / 32 * 32));
+  embed_chunk_sum_kernel<<<grid, threads, 0, c.stream>>>(dx0, s.sorted_pos, s.chunk_start, s.counts, C, s.partial);
   if ((r = check_launch(c, "embed_chunk_sum"))) return r;
-  embed_seg_sum_kernel<<<grid, 128, 0, c.stream>>>(s.partial, s.seg_id, s.seg_chunk0, s.counts, C, dwte);
+  embed_seg_sum_kernel<<<grid, threads, 0, c.stream>>>(s.partial, s.seg_id, s.seg_chunk0, s.counts, C, dwte);
   if ((r = check_launch(c, "embed_seg_sum"))) return r;
   const long long n4 = (long long)T * C / 4;
   embed_pos_grad_kernel<<<(int)((n4 + 255) / 256), 256, 0, c.stream>>>(dx0, Bsz, T, C, dwpe);

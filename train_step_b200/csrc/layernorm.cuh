@@ -236,9 +236,16 @@ __global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
   }
   long long k = 0;
   bool ok = true;
+  // the row statistics are fetched one row ahead, so their latency is not on the row's path
+  float mu_next = first < N ? mean[first] : 0.f, rs_next = first < N ? rstd[first] : 0.f;
   for (;; ++k) {
     const long long row = first + k * stride;
     if (row >= N) break;
+    const float mu = mu_next, rs = rs_next;
+    if (row + stride < N) {
+      mu_next = mean[row + stride];
+      rs_next = rstd[row + stride];
+    }
     const int st = (int)(k % stages);
     const uint32_t par = (uint32_t)((k / stages) & 1);
     int got = 1;
@@ -256,7 +263,6 @@ __global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
     const float4* sdy = reinterpret_cast<const float4*>(mine + (size_t)st * slot_floats);
     const float4* sx = sdy + C4;
     const float4* sr = sdy + 2 * C4;
-    const float mu = mean[row], rs = rstd[row];
     float m1 = 0.f, m2 = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
