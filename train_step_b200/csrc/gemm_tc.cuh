@@ -93,20 +93,40 @@ struct TcCfg {
   static constexpr int SMEM = STAGES * STAGE + STAGING + 1024 + BARS;
 };
 
-__device__ __forceinline__ float gelu_tanh_fast(float u) {
-  const float k = 0.7978845608028654f;
-  float inner = k * (u + 0.044715f * u * u * u);
+// tanh-GELU and its derivative on a PAIR of values with the packed fp32 instructions of
+// sm_100 (f2_fma / f2_mul, common.cuh), t = u^2
+// shared, constants folded (k = sqrt(2/pi), c = 0.044715, z = u (k + k c t)):
+//   gelu(u)  = h + h tanh(z),  h = u / 2
+//   gelu'(u) = (1 + tanh z) / 2 + u (1 - tanh^2 z) (k + 3 k c t) / 2
+__device__ __forceinline__ float tanh_approx(float z) {
   float th;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(inner));
-  return 0.5f * u * (1.0f + th);
+  asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(z));
+  return th;
 }
-__device__ __forceinline__ float gelu_tanh_grad_fast(float u) {
-  const float k = 0.7978845608028654f;
-  float inner = k * (u + 0.044715f * u * u * u);
-  float th;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(inner));
-  float dinner = k * (1.0f + 3.0f * 0.044715f * u * u);
-  return 0.5f * (1.0f + th) + 0.5f * u * (1.0f - th * th) * dinner;
+constexpr float GELU_K = 0.7978845608028654f, GELU_KC = 0.7978845608028654f * 0.044715f;
+// tanh(z) of both lanes of Z
+__device__ __forceinline__ uint64_t f2_tanh(uint64_t Z) {
+  const float2 z = f2_unpack(Z);
+  return f2_pack(tanh_approx(z.x), tanh_approx(z.y));
+}
+__device__ __forceinline__ float2 gelu2_fast(float u0, float u1) {
+  const uint64_t U = f2_pack(u0, u1);
+  const uint64_t T = f2_mul(U, U);
+  const uint64_t TH = f2_tanh(f2_mul(U, f2_fma(T, f2_pack(GELU_KC, GELU_KC), f2_pack(GELU_K, GELU_K))));
+  const uint64_t H = f2_mul(U, f2_pack(0.5f, 0.5f));
+  return f2_unpack(f2_fma(H, TH, H));
+}
+// g * gelu'(u) for both lanes (g: the incoming gradient)
+__device__ __forceinline__ float2 gelu_grad2_mul(float u0, float u1, float g0, float g1) {
+  const uint64_t U = f2_pack(u0, u1);
+  const uint64_t T = f2_mul(U, U);
+  const uint64_t TH = f2_tanh(f2_mul(U, f2_fma(T, f2_pack(GELU_KC, GELU_KC), f2_pack(GELU_K, GELU_K))));
+  const uint64_t A = f2_fma(TH, f2_pack(0.5f, 0.5f), f2_pack(0.5f, 0.5f));             // (1 + th) / 2
+  const uint64_t NB = f2_fma(TH, TH, f2_pack(-1.0f, -1.0f));                           // th^2 - 1
+  const uint64_t NW = f2_mul(U, f2_fma(T, f2_pack(-1.5f * GELU_KC, -1.5f * GELU_KC),
+                                       f2_pack(-0.5f * GELU_K, -0.5f * GELU_K)));     // -u dz/2
+  const uint64_t GP = f2_fma(NW, NB, A);                                               // gelu'(u)
+  return f2_unpack(f2_mul(GP, f2_pack(g0, g1)));
 }
 
 // Epilogue chunks: each epilogue warp turns 32 accumulator rows (one per lane) into
@@ -184,9 +204,10 @@ __device__ __forceinline__ void tc_epilogue_chunk(const GemmParams& p, int col0,
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const float2 f = unpack_bf16x2(w[t]);
-        v[8 * k + 2 * t] *= gelu_tanh_grad_fast(f.x);  // kept in v for the column sums
-        v[8 * k + 2 * t + 1] *= gelu_tanh_grad_fast(f.y);
-        o[t] = pack_bf16x2(v[8 * k + 2 * t], v[8 * k + 2 * t + 1]);
+        const float2 d = gelu_grad2_mul(f.x, f.y, v[8 * k + 2 * t], v[8 * k + 2 * t + 1]);
+        v[8 * k + 2 * t] = d.x;  // kept in v for the column sums
+        v[8 * k + 2 * t + 1] = d.y;
+        o[t] = pack_bf16x2(d.x, d.y);
       }
       *q = make_uint4(o[0], o[1], o[2], o[3]);
     }
@@ -198,7 +219,11 @@ __device__ __forceinline__ void tc_epilogue_chunk(const GemmParams& p, int col0,
                      pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
     }
 #pragma unroll
-    for (int j = 0; j < CW; ++j) v[j] = gelu_tanh_fast(v[j]);
+    for (int j = 0; j < CW; j += 2) {
+      const float2 gg = gelu2_fast(v[j], v[j + 1]);
+      v[j] = gg.x;
+      v[j + 1] = gg.y;
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       *reinterpret_cast<uint4*>(row64_at(buf + 2048, lane, k)) =
@@ -574,7 +599,11 @@ __global__ void __launch_bounds__((2 + tc_epi_warps<EPI>()) * 32, 1)
           __syncwarp();
           if (col0 < p.N) {
 #pragma unroll
-            for (int j = 0; j < CW; ++j) v[j] = gelu_tanh_fast(v[j]);
+            for (int j = 0; j < CW; j += 2) {
+              const float2 gg = gelu2_fast(v[j], v[j + 1]);
+              v[j] = gg.x;
+              v[j + 1] = gg.y;
+            }
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               *reinterpret_cast<uint4*>(row64_at(cur + 2048, lane, k)) =
