@@ -71,7 +71,7 @@ constexpr int BK_THREADS = 32 * (BK_EW0 + FB_EW_WARPS);  // 640
 constexpr int BK_NST = 3;
 constexpr int BK_OFF_KV = 0;                            // K | V [2 items]
 constexpr int BK_OFF_ST = 4 * FA_TILE;                  // stages: Q_i | dO_i
-constexpr int BK_OFF_LD = BK_OFF_ST + BK_NST * FB_STAGE;  // per stage: lse*log2e [128] | D [128]
+constexpr int BK_OFF_LD = BK_OFF_ST + BK_NST * FB_STAGE;  // per stage: -lse*log2e [128] | -D [128]
 constexpr int BK_OFF_OUT = BK_OFF_LD + BK_NST * 1024;   // dK | dV staging for the TMA stores
 constexpr int BK_OFF_BAR = BK_OFF_OUT + 2 * FA_TILE;
 constexpr int BK_SMEM = BK_OFF_BAR + FB_BARS + 1024;
@@ -250,12 +250,12 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
         const int s = U % BK_NST;
         const uint32_t ph = (uint32_t)((U / BK_NST) & 1);
         if (!(ok = fb_warp_wait(&st_empty[s], ph ^ 1, abort_flag, lim, lane))) break;
-        float* ld = reinterpret_cast<float*>(sm + BK_OFF_LD + s * 1024);  // [lse*log2e 128][D 128]
+        float* ld = reinterpret_cast<float*>(sm + BK_OFF_LD + s * 1024);  // [-lse*log2e 128][-D 128]
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int c = lane * 4 + e, q = i * FA_BM + c;
-          ld[c] = q < T ? lse_bh[q] * LOG2E : INFINITY;  // P = 0 for queries past the end
-          ld[128 + c] = q < T ? D_bh[q] : 0.f;
+          ld[c] = q < T ? -lse_bh[q] * LOG2E : -INFINITY;  // P = 0 for queries past the end
+          ld[128 + c] = q < T ? -D_bh[q] : 0.f;
         }
         if (lane == 0) {
           uint8_t* d = sm + BK_OFF_ST + s * FB_STAGE;
@@ -409,24 +409,27 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
         const float* ld = reinterpret_cast<const float*>(sm + BK_OFF_LD + s * 1024) + cg * 32;
         uint32_t pw[16], dw[16];
         const bool diag = u == 0;  // the query block kb itself: queries before the key get P = 0
+        // pairs of columns on packed fp32 instructions: x = s scale log2e + (-lse log2e), then
+        // dS = P (dP + (-D)); the producer staged the negated lse and D
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           const float4 L4 = *reinterpret_cast<const float4*>(ld + 4 * e4);
           const float4 D4 = *reinterpret_cast<const float4*>(ld + 128 + 4 * e4);
-          const float Lv[4] = {L4.x, L4.y, L4.z, L4.w}, Dv[4] = {D4.x, D4.y, D4.z, D4.w};
-          float p[4], ds[4];
+          const uint64_t nl[2] = {f2_pack(L4.x, L4.y), f2_pack(L4.z, L4.w)};
+          const uint64_t nd[2] = {f2_pack(D4.x, D4.y), f2_pack(D4.z, D4.w)};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int e = 4 * e4 + i;
-            float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -Lv[i]));
-            if (diag && cg * 32 + e < r) pe = 0.f;
-            p[i] = pe;
-            ds[i] = pe * (__uint_as_float(dv[e]) - Dv[i]);
+          for (int h = 0; h < 2; ++h) {
+            const int e = 4 * e4 + 2 * h;
+            const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nl[h]));
+            float p0 = ex2_fast(x.x), p1 = ex2_fast(x.y);
+            if (diag && cg * 32 + e < r) p0 = 0.f;
+            if (diag && cg * 32 + e + 1 < r) p1 = 0.f;
+            const float2 ds = f2_unpack(
+                f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd[h])));
+            pw[2 * e4 + h] = pack_bf16x2(p0, p1);
+            dw[2 * e4 + h] = pack_bf16x2(ds.x, ds.y);
           }
-          pw[2 * e4] = pack_bf16x2(p[0], p[1]);
-          pw[2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
-          dw[2 * e4] = pack_bf16x2(ds[0], ds[1]);
-          dw[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
         // the previous unit's dV / dK products have finished reading P^T and dS^T
         if (!fb_warp_wait(p_free, (U & 1) ^ 1, abort_flag, lim, lane)) {
@@ -778,17 +781,19 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
         if (lane == 0) mbar_arrive(s_empty);
         uint32_t dw[16];
         const bool diag = u == nu - 1;  // the key block qb itself: keys after the query get P = 0
+        // pairs of columns on packed fp32 instructions: x = s scale log2e - lse log2e, then
+        // dS = P (dP - D)
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nl2 = f2_pack(-lse2, -lse2), nd2 = f2_pack(-Dr, -Dr);
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
-          float ds[2];
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int e = 2 * e2 + i;
-            float pe = ex2_fast(fmaf(__uint_as_float(sv[e]), sl2, -lse2));
-            if (diag && cg * 32 + e > r) pe = 0.f;
-            ds[i] = pe * (__uint_as_float(dv[e]) - Dr);
-          }
-          dw[e2] = pack_bf16x2(ds[0], ds[1]);
+          const int e = 2 * e2;
+          const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nl2));
+          float p0 = ex2_fast(x.x), p1 = ex2_fast(x.y);
+          if (diag && cg * 32 + e > r) p0 = 0.f;
+          if (diag && cg * 32 + e + 1 > r) p1 = 0.f;
+          const float2 ds = f2_unpack(
+              f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd2)));
+          dw[e2] = pack_bf16x2(ds.x, ds.y);
         }
         // the previous unit's dQ product has finished reading dS
         if (!fb_warp_wait(ds_free, (U & 1) ^ 1, abort_flag, lim, lane)) {
@@ -1147,7 +1152,8 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
         const bool rebase = m_blk > m_run + FX_REBASE;
         const float m_use = rebase ? m_blk : m_run;
         const float m_ref = m_use == -INFINITY ? 0.f : m_use;
-        // P = 2^(s * scale * log2e - m_ref) and the row sum, in registers as bf16 pairs
+        // P = 2^(s * scale * log2e - m_ref) and the row sum, in registers as bf16 pairs (the
+        // packed-pair form measured slower here: it spills under the 168-register cap)
         float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         uint32_t pw[64];
 #pragma unroll
