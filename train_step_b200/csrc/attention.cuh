@@ -43,20 +43,18 @@ __global__ void attn_bwd_dot_kernel(const T* __restrict__ out, const T* __restri
   }
 }
 
-// bf16, hd = 64: one thread per (row, head), 128-byte vector loads of O and dO.
+// bf16, hd = 64: eight threads per (row, head), each one 16-byte piece of O and of dO
+// (consecutive threads read consecutive 16 bytes, so a warp's loads are 512 contiguous
+// bytes of each tensor), the eight partial dot products combined by three shuffles in a
+// fixed order.
 __global__ void attn_bwd_dot64_bf16_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
                                            float* __restrict__ D, int Bsz, int Tn, int NH) {
-  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (i >= (long long)Bsz * Tn * NH) return;
-  const int h = (int)(i % NH);
-  const long long row = i / NH;
-  const long long off = row * NH * 64 + h * 64;
-  const uint4* o = reinterpret_cast<const uint4*>(out + off);
-  const uint4* d = reinterpret_cast<const uint4*>(dout + off);
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;  // 16-byte piece
+  const long long npieces = (long long)Bsz * Tn * NH * 8;
+  const bool in = i < npieces;
   float s = 0.f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint4 a = o[k], b = d[k];
+  if (in) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(out) + i), b = __ldg(reinterpret_cast<const uint4*>(dout) + i);
     const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -64,8 +62,16 @@ __global__ void attn_bwd_dot64_bf16_kernel(const bf16* __restrict__ out, const b
       s += fa.x * fb.x + fa.y * fb.y;
     }
   }
-  const int b = (int)(row / Tn), t = (int)(row % Tn);
-  D[((long long)b * NH + h) * Tn + t] = s;
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 4);
+  if (in && (i & 7) == 0) {
+    const long long rh = i >> 3;  // (row, head)
+    const int h = (int)(rh % NH);
+    const long long row = rh / NH;
+    const int b = (int)(row / Tn), t = (int)(row % Tn);
+    D[((long long)b * NH + h) * Tn + t] = s;
+  }
 }
 
 // ----------------------------------------------------------------------------

@@ -795,9 +795,10 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
   const int dblocks = (int)((warps * 32 + 255) / 256);
   if (dtype == GPT2_BF16) {
     if (hd != 64) return fail(c, GPT2_ERR_CONFIG, "attention (bf16): head dim must be 64");
-    if ((reinterpret_cast<uintptr_t>(qkv) & 15) || (reinterpret_cast<uintptr_t>(dout) & 15))
-      return fail(c, GPT2_ERR_CONFIG, "attention: qkv and dout must be 16-byte aligned");
-    attn_bwd_dot64_bf16_kernel<<<(int)((warps + 255) / 256), 256, 0, c.stream>>>((const bf16*)out, (const bf16*)dout,
+    if ((reinterpret_cast<uintptr_t>(qkv) & 15) || (reinterpret_cast<uintptr_t>(dout) & 15) ||
+        (reinterpret_cast<uintptr_t>(out) & 15))
+      return fail(c, GPT2_ERR_CONFIG, "attention: qkv, out and dout must be 16-byte aligned");
+    attn_bwd_dot64_bf16_kernel<<<(int)((warps * 8 + 255) / 256), 256, 0, c.stream>>>((const bf16*)out, (const bf16*)dout,
                                                                                   Dbuf, B, T, NH);
     int r = check_launch(c, "attn_bwd_dot");
     if (r) return r;
