@@ -465,3 +465,35 @@ def test_canonical_order_and_offsets():
         assert t.offset == off
         off += t.size
     assert off == oracle.num_params(cfg)
+
+
+def test_gpt2_124m_initial_loss_matches_a_library_model():
+    """The oracle at the real 124M shape and initialisation (seed 42), against the same
+    forward built from torch library routines in float64: the initial loss the GPU tests
+    compare with is pinned at full width, depth and vocabulary (one 64-token Zipf
+    sequence), not only on tiny shapes."""
+    cfg = oracle.Config(12, 12, 768, 1024, 50257, 1, 1)
+    p = oracle.init_params(cfg, 42).astype(np.float64)
+    T = 64
+    tok, tgt = synth.micro_batch(1, T, cfg.V, index=0)
+    loss = oracle.forward(cfg, p, tok, tgt)
+    P = {t.name: torch.from_numpy(p[t.offset:t.offset + t.size].reshape(t.shape)) for t in oracle.tensors(cfg)}
+    C, NH = cfg.C, cfg.H
+    with torch.no_grad():
+        x = P["wte"][torch.from_numpy(tok).long()] + P["wpe"][:T]
+        for l in range(cfg.L):
+            pre = f"h{l}."
+            hh = F.layer_norm(x, (C,), P[pre + "ln1_g"], P[pre + "ln1_b"], 1e-5)
+            qkv = F.linear(hh, P[pre + "qkv_w"], P[pre + "qkv_b"])
+            q, k, v = (qkv[..., i * C:(i + 1) * C].view(1, T, NH, C // NH).transpose(1, 2) for i in range(3))
+            y = F.scaled_dot_product_attention(q, k, v, is_causal=True).transpose(1, 2).reshape(1, T, C)
+            x = x + F.linear(y, P[pre + "ao_w"], P[pre + "ao_b"])
+            hh = F.layer_norm(x, (C,), P[pre + "ln2_g"], P[pre + "ln2_b"], 1e-5)
+            x = x + F.linear(F.gelu(F.linear(hh, P[pre + "fc_w"], P[pre + "fc_b"]), approximate="tanh"),
+                             P[pre + "pj_w"], P[pre + "pj_b"])
+        logits = F.linear(F.layer_norm(x, (C,), P["lnf_g"], P["lnf_b"], 1e-5), P["wte"])
+        ref = F.cross_entropy(logits.view(-1, cfg.V), torch.from_numpy(tgt).long().view(-1)).item()
+    assert abs(loss - ref) < 1e-9 * abs(ref), (loss, ref)
+    # near ln V: the initial logits are nearly uniform apart from the tied head's small
+    # preference for the input token itself
+    assert abs(ref - np.log(cfg.V)) < 0.3, ref
