@@ -49,9 +49,10 @@ constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 //       dQ += dS K_j                          (M=128 queries, N=64, K=128 keys; A = dS in TMEM)
 //
 // TMEM (512 columns). dK/dV: S^T | dP^T (128 + 128), P^T | dS^T (64 + 64, bf16 pairs),
-// dV | dK (64 + 64). dQ: S | dP (128 + 128), Q | dO operands (32 + 32), dS (64), dQ for two
-// items (64 + 64). The score tiles are single-buffered: the element-wise warps load them
-// into registers first thing, and the next unit's score products run while they compute.
+// dV | dK (64 + 64). dQ: S | dP (128 + 128), Q | dO operands (32 + 32), dS for two units in
+// turn (64 + 64: the next unit's dS is written while the dQ product reads this one), dQ (64).
+// The score tiles are single-buffered: the element-wise warps load them into registers
+// first thing, and the next unit's score products run while they compute.
 // MMA issue: a thread issues one tcgen05.mma every ~80-150 cycles (measured), so each
 // score product has its own issuing thread (lane 0 of its warp); dK/dV's two
 // accumulation products share one thread (a thread each measured slower: 21 warps
@@ -85,7 +86,7 @@ constexpr int BQ_OFF_ST = 4 * FA_TILE;                  // stages: K_j | V_j
 constexpr int BQ_OFF_OUT = BQ_OFF_ST + BQ_NST * FB_STAGE;
 constexpr int BQ_OFF_BAR = BQ_OFF_OUT + FA_TILE;
 constexpr int BQ_SMEM = BQ_OFF_BAR + FB_BARS + 1024;
-constexpr uint32_t BQ_TM_DP = 128, BQ_TM_Q = 256, BQ_TM_DS = 320, BQ_TM_ACC = 384;
+constexpr uint32_t BQ_TM_DP = 128, BQ_TM_Q = 256, BQ_TM_DS = 320, BQ_TM_ACC = 448;  // dS: 2 x 64
 static_assert(BK_SMEM <= 232448 && BQ_SMEM <= 232448, "shared memory per CTA");
 
 // Item of CTA `cta` in round k over G CTAs: zigzag over the longest-first order.
@@ -531,11 +532,11 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
   uint64_t* st_empty = st_full + BQ_NST;      // [BQ_NST]
   uint64_t* s_full = st_empty + BQ_NST;       // S and dP complete (2 commits)
   uint64_t* s_empty = s_full + 1;             // both read into registers (16 warps)
-  uint64_t* ds_full = s_empty + 1;            // dS written (16 warps)
-  uint64_t* ds_free = ds_full + 1;            // the dQ product has read it
-  uint64_t* acc_full = ds_free + 1;           // [2] the item's dQ complete
-  uint64_t* acc_empty = acc_full + 2;         // [2] read by the epilogue (16 warps)
-  uint64_t* out_full = acc_empty + 2;         // output tile staged (16 warps)
+  uint64_t* ds_full = s_empty + 1;            // [2] dS of a unit written (16 warps); units alternate
+  uint64_t* ds_free = ds_full + 2;            // [2] the dQ product has read it
+  uint64_t* acc_full = ds_free + 2;           // the item's dQ complete
+  uint64_t* acc_empty = acc_full + 1;         // read by the epilogue (16 warps)
+  uint64_t* out_full = acc_empty + 1;         // output tile staged (16 warps)
   uint64_t* out_free = out_full + 1;          // the previous item's TMA store has read the staging
   uint64_t* drain = out_free + 1;             // [3]: one per MMA thread (abort path)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
@@ -552,9 +553,11 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&qd_full[i], 1);
       mbar_init(&qd_empty[i], FB_EW_WARPS);
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], FB_EW_WARPS);
+      mbar_init(&ds_full[i], FB_EW_WARPS);
+      mbar_init(&ds_free[i], 1);
     }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, FB_EW_WARPS);
     mbar_init(qa_full, FB_EW_WARPS);
     for (int i = 0; i < BQ_NST; ++i) {
       mbar_init(&st_full[i], 1);
@@ -562,8 +565,6 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
     }
     mbar_init(s_full, 2);
     mbar_init(s_empty, FB_EW_WARPS);
-    mbar_init(ds_full, FB_EW_WARPS);
-    mbar_init(ds_free, 1);
     mbar_init(out_full, FB_EW_WARPS);
     mbar_init(out_free, 1);
     for (int i = 0; i < 3; ++i) mbar_init(&drain[i], 1);
@@ -681,29 +682,30 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
       for (int k = 0; ok; ++k) {
         const int item = fx_item(k, cta, G);
         if (item >= nitems) break;
-        const int ab = k & 1, nu = nqb - item / BH;
-        if (!mbar_wait_bounded(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag, lim)) {
+        const int nu = nqb - item / BH;
+        if (!mbar_wait_bounded(acc_empty, (k & 1) ^ 1, abort_flag, lim)) {
           ok = false;
           break;
         }
         for (int u = 0; u < nu; ++u, ++U) {
           const int s = U % BQ_NST;
           if (!mbar_wait_bounded(&st_full[s], (U / BQ_NST) & 1, abort_flag, lim) ||
-              !mbar_wait_bounded(ds_full, U & 1, abort_flag, lim)) {
+              !mbar_wait_bounded(&ds_full[U & 1], (U >> 1) & 1, abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t k_desc = make_sw128_desc(smem_u32(sm + BQ_OFF_ST + s * FB_STAGE), 8192, 1024);
-          const uint32_t acc = tmem + BQ_TM_ACC + (uint32_t)(ab * 64);
+          const uint32_t acc = tmem + BQ_TM_ACC;
+          const uint32_t dsb = tmem + BQ_TM_DS + (uint32_t)((U & 1) * 64);
           // K = 128 keys: A = dS (8 TMEM columns per 16 keys), B = 16 key rows of K_j per step
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_bf16_ts(acc, tmem + BQ_TM_DS + kk * 8, k_desc + 128 * kk, idesc_q, (u > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16_ts(acc, dsb + kk * 8, k_desc + 128 * kk, idesc_q, (u > 0 || kk > 0) ? 1u : 0u);
           any = true;
-          umma_commit(ds_free);
+          umma_commit(&ds_free[U & 1]);
           umma_commit(&st_empty[s]);  // the unit's score products completed before dS was written
-          if (u == nu - 1) umma_commit(&acc_full[ab]);
+          if (u == nu - 1) umma_commit(acc_full);
         }
       }
       if (!ok) {
@@ -795,16 +797,16 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
               f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd2)));
           dw[e2] = pack_bf16x2(ds.x, ds.y);
         }
-        // the previous unit's dQ product has finished reading dS
-        if (!fb_warp_wait(ds_free, (U & 1) ^ 1, abort_flag, lim, lane)) {
+        // the dQ product of two units ago has finished reading this dS buffer
+        if (!fb_warp_wait(&ds_free[U & 1], ((U >> 1) & 1) ^ 1, abort_flag, lim, lane)) {
           fail = true;
           break;
         }
-        tmem_st_32x32b_x16(tmem + lane_off + BQ_TM_DS + (uint32_t)(cg * 16), dw);
+        tmem_st_32x32b_x16(tmem + lane_off + BQ_TM_DS + (uint32_t)((U & 1) * 64 + cg * 16), dw);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(ds_full);
+        if (lane == 0) mbar_arrive(&ds_full[U & 1]);
       }
       if (fail) break;
       // the next item's operands first (lets its score products start), then this item's dQ
@@ -812,18 +814,17 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
         fail = true;
         break;
       }
-      const int ab = k & 1;
-      if (!fb_warp_wait(&acc_full[ab], (k >> 1) & 1, abort_flag, lim, lane)) {
+      if (!fb_warp_wait(acc_full, k & 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
       tc_fence_after();
       uint32_t v[16];
-      tmem_ld_32x32b_x16(tmem + lane_off + BQ_TM_ACC + (uint32_t)(ab * 64 + cg * 16), v);
+      tmem_ld_32x32b_x16(tmem + lane_off + BQ_TM_ACC + (uint32_t)(cg * 16), v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (lane == 0) mbar_arrive(acc_empty);
       if (colsum) {
         // column sums of dQ over this warp's 32 query rows (rows past T are zero here): the
         // query third of the qkv bias gradient, one partial per 32-row block
