@@ -54,9 +54,10 @@ constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 // The score tiles are single-buffered: the element-wise warps load them into registers
 // first thing, and the next unit's score products run while they compute.
 // MMA issue: a thread issues one tcgen05.mma every ~80-150 cycles (measured), so each
-// score product has its own issuing thread (lane 0 of its warp); dK/dV's two
-// accumulation products share one thread (a thread each measured slower: 21 warps
-// leave 80 registers per thread and the element-wise code spills).
+// score product has its own issuing thread (lane 0 of its warp); in dK/dV that thread also
+// issues one of the two accumulation products one unit behind (dV with S^T, dK with dP^T),
+// which splits them over two threads without another warp (a fifth warp for them measured
+// slower: 21 warps leave 80 registers per thread and the element-wise code spills).
 // Warps: 0 TMA producer, then the MMA issuers, then 16 element-wise warps: warp w reads
 // TMEM lane quarter w % 4 (32 rows) and column group (w - first) / 4 (32 of the 128
 // unit columns). D = rowsum(dO * O) comes precomputed. Every wait is bounded (device
@@ -67,8 +68,8 @@ constexpr int FB_BARS = 512;
 constexpr int FB_STAGE = 2 * FA_TILE;  // two 128-row tiles: 32 KB
 constexpr uint32_t FB_TMEM_COLS = 512;
 // dK/dV kernel
-constexpr int BK_EW0 = 4;  // producer, S^T, dP^T, (dV and dK) issuers, then element-wise warps
-constexpr int BK_THREADS = 32 * (BK_EW0 + FB_EW_WARPS);  // 640
+constexpr int BK_EW0 = 3;  // producer, (S^T and dV), (dP^T and dK) issuers, then element-wise warps
+constexpr int BK_THREADS = 32 * (BK_EW0 + FB_EW_WARPS);  // 608
 constexpr int BK_NST = 3;
 constexpr int BK_OFF_KV = 0;                            // K | V [2 items]
 constexpr int BK_OFF_ST = 4 * FA_TILE;                  // stages: Q_i | dO_i
@@ -172,12 +173,12 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
   uint64_t* kv_full = bar;                    // [2] K / V tiles landed
   uint64_t* kv_empty = kv_full + 2;           // [2] the item's S^T / dP^T products are complete (2 commits)
   uint64_t* st_full = kv_empty + 2;           // [BK_NST] Q_i / dO_i landed, lse / D staged (32 producer lanes)
-  uint64_t* st_empty = st_full + BK_NST;      // [BK_NST] the unit's dV and dK products are complete
+  uint64_t* st_empty = st_full + BK_NST;      // [BK_NST] the unit's dV and dK products are complete (2 commits)
   uint64_t* s_full = st_empty + BK_NST;       // S^T and dP^T complete (2 commits)
   uint64_t* s_empty = s_full + 1;             // both read into registers (16 warps)
   uint64_t* p_full = s_empty + 1;             // P^T and dS^T written (16 warps)
-  uint64_t* p_free = p_full + 1;              // the dV and dK products have read them
-  uint64_t* acc_full = p_free + 1;            // the item's dV and dK complete
+  uint64_t* p_free = p_full + 1;              // the dV and dK products have read them (2 commits)
+  uint64_t* acc_full = p_free + 1;            // the item's dV and dK complete (2 commits)
   uint64_t* acc_empty = acc_full + 1;         // dV and dK read by the epilogue (16 warps)
   uint64_t* out_full = acc_empty + 1;         // output tiles staged (16 warps)
   uint64_t* out_free = out_full + 1;          // the previous item's TMA stores have read the staging
@@ -199,13 +200,13 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
     }
     for (int i = 0; i < BK_NST; ++i) {
       mbar_init(&st_full[i], 32);
-      mbar_init(&st_empty[i], 1);
+      mbar_init(&st_empty[i], 2);
     }
     mbar_init(s_full, 2);
     mbar_init(s_empty, FB_EW_WARPS);
     mbar_init(p_full, FB_EW_WARPS);
-    mbar_init(p_free, 1);
-    mbar_init(acc_full, 1);
+    mbar_init(p_free, 2);
+    mbar_init(acc_full, 2);
     mbar_init(acc_empty, FB_EW_WARPS);
     mbar_init(out_full, FB_EW_WARPS);
     mbar_init(out_free, 1);
@@ -283,11 +284,37 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
     }
   } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
-      // ---------------- score MMAs: S^T = K Q_i^T (warp 1), dP^T = V dO_i^T (warp 2) ----------------
+      // ---------------- MMA issue, one thread per part: warp 1 S^T = K Q_i^T and dV += P^T dO_i,
+      // warp 2 dP^T = V dO_i^T and dK += dS^T Q_i. A thread issues the score product of unit U,
+      // then the accumulation of unit U - 1 (whose P^T / dS^T the element-wise warps finish
+      // while the new scores are computed), so the 16 accumulation MMAs of a unit are split
+      // over two issuing threads without adding a warp.
       const int part = warp - 1;
       constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_a = make_idesc_bf16(128, 64, false, true);  // B = dO_i / Q_i, MN-major
       bool ok = true, any = false;
       int U = 0;
+      // the unit whose accumulation is pending: global index, stage, item round, first / last
+      int pU = -1, pS = 0, pK = 0;
+      bool pFirst = false, pLast = false;
+      auto accumulate = [&]() -> bool {
+        if (pFirst && !mbar_wait_bounded(acc_empty, (pK & 1) ^ 1, abort_flag, lim)) return false;
+        if (!mbar_wait_bounded(p_full, pU & 1, abort_flag, lim)) return false;
+        tc_fence_after();
+        // K = 128 queries: A = P^T (dV) or dS^T (dK), 8 TMEM columns per 16 queries; B = 16
+        // query rows of dO_i (dV) or Q_i (dK) per step, descriptor base + 128 kk (2 KB)
+        const uint64_t b_desc =
+            make_sw128_desc(smem_u32(sm + BK_OFF_ST + pS * FB_STAGE + (1 - part) * FA_TILE), 8192, 1024);
+        const uint32_t a_tm = tmem + (part == 0 ? BK_TM_P : BK_TM_DS);
+        const uint32_t acc = tmem + (part == 0 ? BK_TM_DV : BK_TM_DK);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(acc, a_tm + kk * 8, b_desc + 128 * kk, idesc_a, (!pFirst || kk > 0) ? 1u : 0u);
+        umma_commit(p_free);
+        umma_commit(&st_empty[pS]);  // the unit's score products completed before P^T was written
+        if (pLast) umma_commit(acc_full);
+        return true;
+      };
       for (int k = 0; ok; ++k) {
         const int item = fx_item(k, cta, G);
         if (item >= nitems) break;
@@ -313,9 +340,19 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
             umma_bf16(tmem + part * BK_TM_DP, a_desc + 2 * kk, b_desc + 2 * kk, idesc_s, kk > 0 ? 1u : 0u);
           umma_commit(s_full);
           any = true;
+          if (pU >= 0 && !accumulate()) {
+            ok = false;
+            break;
+          }
+          pU = U;
+          pS = s;
+          pK = k;
+          pFirst = u == 0;
+          pLast = u == nu - 1;
         }
         if (ok) umma_commit(&kv_empty[kvb]);  // the item's K / V tile is no longer read
       }
+      if (ok && pU >= 0) ok = accumulate();  // the last unit
       if (!ok) {
         raise_device_error(err, DEV_TIMEOUT);
         *abort_flag = 1;
@@ -323,57 +360,6 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
           int never = 0;
           umma_commit(&drain[part]);
           mbar_wait_bounded(&drain[part], 0, reinterpret_cast<volatile int*>(&never), lim);
-        }
-      }
-    }
-  } else if (warp == 3) {
-    if (lane == 0) {
-      // ---------------- accumulation MMAs: dV += P^T dO_i, then dK += dS^T Q_i ----------------
-      constexpr uint32_t idesc_a = make_idesc_bf16(128, 64, false, true);  // B = dO_i / Q_i, MN-major
-      bool ok = true, any = false;
-      int U = 0;
-      for (int k = 0; ok; ++k) {
-        const int item = fx_item(k, cta, G);
-        if (item >= nitems) break;
-        const int nu = nqb - item / BH;
-        // the epilogue has read the previous item's dV / dK
-        if (!mbar_wait_bounded(acc_empty, (k & 1) ^ 1, abort_flag, lim)) {
-          ok = false;
-          break;
-        }
-        for (int u = 0; u < nu; ++u, ++U) {
-          const int s = U % BK_NST;
-          if (!mbar_wait_bounded(&st_full[s], (U / BK_NST) & 1, abort_flag, lim) ||
-              !mbar_wait_bounded(p_full, U & 1, abort_flag, lim)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // K = 128 queries: A = P^T (dV) or dS^T (dK), 8 TMEM columns per 16 queries; B = 16
-          // query rows of dO_i (dV) or Q_i (dK) per step, descriptor base + 128 kk (2 KB)
-#pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            const uint64_t b_desc =
-                make_sw128_desc(smem_u32(sm + BK_OFF_ST + s * FB_STAGE + (1 - part) * FA_TILE), 8192, 1024);
-            const uint32_t a_tm = tmem + (part == 0 ? BK_TM_P : BK_TM_DS);
-            const uint32_t acc = tmem + (part == 0 ? BK_TM_DV : BK_TM_DK);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_bf16_ts(acc, a_tm + kk * 8, b_desc + 128 * kk, idesc_a, (u > 0 || kk > 0) ? 1u : 0u);
-          }
-          any = true;
-          umma_commit(p_free);
-          umma_commit(&st_empty[s]);  // the unit's score products completed before P^T was written
-          if (u == nu - 1) umma_commit(acc_full);
-        }
-      }
-      if (!ok) {
-        raise_device_error(err, DEV_TIMEOUT);
-        *abort_flag = 1;
-        if (any) {
-          int never = 0;
-          umma_commit(&drain[2]);
-          mbar_wait_bounded(&drain[2], 0, reinterpret_cast<volatile int*>(&never), lim);
         }
       }
     }
