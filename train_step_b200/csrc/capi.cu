@@ -398,6 +398,15 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
                            : layernorm_bwd_t<float>(c, dy, x, gg, mu, rs, N, C, m->dres, (float*)nullptr, accumulate,
                                                     m->part, dg, db, dbias_next, 1);
   };
+  // bf16 mode: the dX GEMMs in front of the per-layer LayerNorms write dh in bf16 (half the
+  // bytes for the GEMM to store and the LayerNorm to read), in the fp32 dh buffer's storage;
+  // the final LayerNorm's dh stays fp32 (the head's dX accumulates over the logit chunks)
+  bf16* dh16 = reinterpret_cast<bf16*>(m->dh);
+  auto LN_B16 = [&](const float* x, const float* gg, float* mu, float* rs, float* dg, float* db,
+                    float* dbias_next) -> int {
+    return layernorm_bwd_t<bf16, bf16>(cb, dh16, x, gg, mu, rs, N, C, m->dres, (bf16*)m->dres_act, 1, m->part, dg,
+                                       db, dbias_next, 1, SIDE_LN);
+  };
   auto COLSUM_ACT = [&](const void* y, int ncols, float* out) -> int {
     return dt == GPT2_BF16 ? colsum_t<bf16>(c, (const bf16*)y, ncols, N, ncols, m->part, out)
                            : colsum_t<float>(c, (const float*)y, ncols, N, ncols, m->part, out);
@@ -451,9 +460,15 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     RK(DW(GemmDesc{m->du, F, true, h2, C, true, F, C, N, EPI_F32, gw.fc_w, C, nullptr, 0, nullptr, nullptr, 0,
                    1, 0, CAT_GEMM_DW}));
     if (dt != GPT2_BF16) RK(COLSUM_ACT(m->du, F, gw.fc_b));
-    RK(gemm(c, dt, GemmDesc{m->du, F, false, m->W(w.fc_w), C, true, N, C, F, EPI_F32, m->dh, C, nullptr, 0, nullptr,
-                            nullptr, 0, 0, 1, CAT_GEMM_DX}));
-    RK(LN_B(m->dh, xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), 1, gw.ln2_g, gw.ln2_b, gw.ao_b));
+    if (dt == GPT2_BF16) {
+      RK(gemm(c, dt, GemmDesc{m->du, F, false, m->W(w.fc_w), C, true, N, C, F, EPI_BF16, dh16, C, nullptr, 0,
+                              nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
+      RK(LN_B16(xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), gw.ln2_g, gw.ln2_b, gw.ao_b));
+    } else {
+      RK(gemm(c, dt, GemmDesc{m->du, F, false, m->W(w.fc_w), C, true, N, C, F, EPI_F32, m->dh, C, nullptr, 0,
+                              nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
+      RK(LN_B(m->dh, xs(2 * l + 1), w.ln2_g, mean(2 * l + 1), rstd(2 * l + 1), 1, gw.ln2_g, gw.ln2_b, gw.ao_b));
+    }
     // attention: x_mid = x_in + ao(attn(ln1(x_in)))
     RK(DW(GemmDesc{dres_act, C, true, att, C, true, C, C, N, EPI_F32, gw.ao_w, C, nullptr, 0, nullptr, nullptr,
                    0, 1, 0, CAT_GEMM_DW}));
@@ -469,10 +484,16 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     RK(DW(GemmDesc{m->dqkv, 3 * C, true, h1, C, true, 3 * C, C, N, EPI_F32, gw.qkv_w, C, nullptr, 0, nullptr,
                    nullptr, 0, 1, 0, CAT_GEMM_DW}));
     if (gw.qkv_b && !qkvb_fused) RK(COLSUM_ACT(m->dqkv, 3 * C, gw.qkv_b));
-    RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, false, m->W(w.qkv_w), C, true, N, C, 3 * C, EPI_F32, m->dh, C, nullptr, 0,
-                            nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
-    RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b,
-            l > 0 ? m->lg[l - 1].pj_b : nullptr));
+    if (dt == GPT2_BF16) {
+      RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, false, m->W(w.qkv_w), C, true, N, C, 3 * C, EPI_BF16, dh16, C, nullptr,
+                              0, nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
+      RK(LN_B16(xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), gw.ln1_g, gw.ln1_b, l > 0 ? m->lg[l - 1].pj_b : nullptr));
+    } else {
+      RK(gemm(c, dt, GemmDesc{m->dqkv, 3 * C, false, m->W(w.qkv_w), C, true, N, C, 3 * C, EPI_F32, m->dh, C, nullptr,
+                              0, nullptr, nullptr, 0, 0, 1, CAT_GEMM_DX}));
+      RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b,
+              l > 0 ? m->lg[l - 1].pj_b : nullptr));
+    }
     RK(mark_bucket(m, cb, l));  // layer l's pj_b came from layer l + 1's LayerNorm (or ln_f)
   }
   RK(side_wait_free(cb, SIDE_EMB));  // the token sort (side stream) has finished

@@ -651,13 +651,13 @@ inline int reduce_partials(const LaunchCtx& c, const float* part, int P, int nco
   return check_launch(c, "reduce_partials");
 }
 
-template <class T, int NV>
-void launch_ln_bwd(const LaunchCtx& c, int grid, size_t smem, const float* dy, const float* x, const float* g,
+template <class T, int NV, class DY>
+void launch_ln_bwd(const LaunchCtx& c, int grid, size_t smem, const DY* dy, const float* x, const float* g,
                    const float* mean, const float* rstd, float* dres, T* dres_act, int accumulate, float* part,
                    int with_rsum, int N, int C) {
-  smem_optin(layernorm_bwd_kernel<T, NV>, 200 * 1024);
-  layernorm_bwd_kernel<T, NV><<<grid, LN_WARPS * 32, smem, c.stream>>>(dy, x, g, mean, rstd, dres, dres_act,
-                                                                       accumulate, part, with_rsum, N, C);
+  smem_optin(layernorm_bwd_kernel<T, NV, DY>, 200 * 1024);
+  layernorm_bwd_kernel<T, NV, DY><<<grid, LN_WARPS * 32, smem, c.stream>>>(dy, x, g, mean, rstd, dres, dres_act,
+                                                                           accumulate, part, with_rsum, N, C);
 }
 
 // Slots per warp of the staged backward: as many rows (dy, x, dres: 12 C bytes each) as
@@ -671,23 +671,24 @@ inline int ln_ring_stages(int C) {
 }
 inline size_t ln_ring_smem(int C, int stages) { return (size_t)LNR_WARPS * stages * (12 * (size_t)C + 8); }
 
-template <class T, int NV>
-int launch_ln_bwd_ring(const LaunchCtx& c, int grid, int stages, const float* dy, const float* x, const float* g,
+template <class T, int NV, class DY>
+int launch_ln_bwd_ring(const LaunchCtx& c, int grid, int stages, const DY* dy, const float* x, const float* g,
                        const float* mean, const float* rstd, float* dres, T* dres_act, int accumulate, float* part,
                        int with_rsum, int N, int C) {
   const size_t smem = ln_ring_smem(C, stages);
   // opted in once per device for the largest ring any C can ask for
-  if (!smem_optin(layernorm_bwd_ring_kernel<T, NV>, 232448 - 1024))
+  if (!smem_optin(layernorm_bwd_ring_kernel<T, NV, DY>, 232448 - 1024))
     return fail(c, GPT2_ERR_CUDA, "layernorm_bwd: shared-memory opt-in");
-  layernorm_bwd_ring_kernel<T, NV><<<grid, LNR_WARPS * 32, smem, c.stream>>>(
+  layernorm_bwd_ring_kernel<T, NV, DY><<<grid, LNR_WARPS * 32, smem, c.stream>>>(
       dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C, stages, c.d_err, 4000000000ull);
   return 0;
 }
 
 // LayerNorm backward plus the reduction of its parameter gradients: dg, db (+)=;
 // dbias_next (nullable) (+)= column sums of the updated dres.
-template <class T>
-int layernorm_bwd_t(const LaunchCtx& c, const float* dy, const float* x, const float* g, const float* mean,
+// dy: fp32, or bf16 (the dX GEMMs' output in bf16 mode)
+template <class T, class DY = float>
+int layernorm_bwd_t(const LaunchCtx& c, const DY* dy, const float* x, const float* g, const float* mean,
                     const float* rstd, int N, int C, float* dres, T* dres_act, int accumulate,
                     float* part /*3*grid*C*/, float* dg, float* db, float* dbias_next, int accumulate_params,
                     int side_buf = -1) {
@@ -703,20 +704,20 @@ int layernorm_bwd_t(const LaunchCtx& c, const float* dy, const float* x, const f
   }
   {
     ProfScope ps(c, CAT_LN_BWD, 0.0,
-                 (double)N * C * (12 + 4 * accumulate + (dres_act ? sizeof(T) : 0)) + 8.0 * N +
+                 (double)N * C * (sizeof(DY) + 8 + 4 * accumulate + (dres_act ? sizeof(T) : 0)) + 8.0 * N +
                      4.0 * (2 + with_rsum) * grid * C);
     const size_t smem = (size_t)LN_WARPS * 3 * C * 4;
     int rr = 0;
-    if (stages && nv <= 4) rr = launch_ln_bwd_ring<T, 4>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else if (stages && nv <= 6) rr = launch_ln_bwd_ring<T, 6>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else if (stages && nv <= 8) rr = launch_ln_bwd_ring<T, 8>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else if (nv <= 1) launch_ln_bwd<T, 1>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else if (nv <= 2) launch_ln_bwd<T, 2>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else if (nv <= 4) launch_ln_bwd<T, 4>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else if (nv <= 6) launch_ln_bwd<T, 6>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else if (nv <= 8) launch_ln_bwd<T, 8>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else if (nv <= 13) launch_ln_bwd<T, 13>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
-    else launch_ln_bwd<T, 16>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    if (stages && nv <= 4) rr = launch_ln_bwd_ring<T, 4, DY>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (stages && nv <= 6) rr = launch_ln_bwd_ring<T, 6, DY>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (stages && nv <= 8) rr = launch_ln_bwd_ring<T, 8, DY>(c, grid, stages, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 1) launch_ln_bwd<T, 1, DY>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 2) launch_ln_bwd<T, 2, DY>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 4) launch_ln_bwd<T, 4, DY>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 6) launch_ln_bwd<T, 6, DY>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 8) launch_ln_bwd<T, 8, DY>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else if (nv <= 13) launch_ln_bwd<T, 13, DY>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
+    else launch_ln_bwd<T, 16, DY>(c, grid, smem, dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C);
     if (rr) return rr;
   }
   int r = check_launch(c, "layernorm_bwd");

@@ -21,6 +21,20 @@ __device__ __forceinline__ void store4<bf16>(bf16* dst, float a, float b, float 
   *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
 }
 
+// Four consecutive values of a row of type D as floats (16-byte fp32 or 8-byte bf16 load).
+template <class D>
+__device__ __forceinline__ float4 load4(const D* p);
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 load4<bf16>(const bf16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = unpack_bf16x2(u.x), b = unpack_bf16x2(u.y);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
 // x: fp32 [N, C]; y: T [N, C]; mean, rstd: fp32 [N]. C % 4 == 0, C <= 128 * NV.
 // PDL: launched as a programmatic dependent (generation steps), it waits for the
 // previous kernel before reading x.
@@ -85,9 +99,9 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_fwd_kernel(const floa
 // with_rsum, the updated dres itself (the bias gradient of the linear layer whose
 // output this residual is). Rows are assigned to CTAs in a fixed pattern, so the
 // reduction order never changes between runs.
-template <class T, int NV>
+template <class T, int NV, class DY = float>
 __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
-    const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
+    const DY* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
     const float* __restrict__ mean, const float* __restrict__ rstd, float* __restrict__ dres,
     T* __restrict__ dres_act, int accumulate, float* __restrict__ part, int with_rsum, int N, int C) {
   // per-warp column accumulators [warp][3][C] in dynamic shared memory; lane l owns
@@ -103,7 +117,7 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
   }
   for (long long row = (long long)blockIdx.x * LN_WARPS + warp; row < N; row += (long long)gridDim.x * LN_WARPS) {
     const float mu = mean[row], rs = rstd[row];
-    const float* dyr = dy + row * C;
+    const DY* dyr = dy + row * C;
     const float* xr = x + row * C;
     float4 vd[NV], vx[NV], vr[NV];
     float m1 = 0.f, m2 = 0.f;
@@ -119,7 +133,7 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
     for (int i = 0; i < NV; ++i) {
       const int c = (i * 32 + lane) * 4;
       if (c < C) {
-        vd[i] = *reinterpret_cast<const float4*>(dyr + c);
+        vd[i] = load4<DY>(dyr + c);
         float4 xx = *reinterpret_cast<const float4*>(xr + c);
         float4 gg = __ldg(reinterpret_cast<const float4*>(g + c));
         vx[i] = make_float4((xx.x - mu) * rs, (xx.y - mu) * rs, (xx.z - mu) * rs, (xx.w - mu) * rs);
@@ -190,9 +204,9 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_bwd_kernel(
 // columns i * 32 + l); at the end the warps' accumulators pass through shared memory and
 // are summed in warp order, so the reduction order is fixed.
 constexpr int LNR_WARPS = 8;
-template <class T, int NV>
+template <class T, int NV, class DY = float>
 __global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
-    const float* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
+    const DY* __restrict__ dy, const float* __restrict__ x, const float* __restrict__ g,
     const float* __restrict__ mean, const float* __restrict__ rstd, float* __restrict__ dres,
     T* __restrict__ dres_act, int accumulate, float* __restrict__ part, int with_rsum, int N, int C, int stages,
     int* err, unsigned long long limit_ns) {
@@ -212,8 +226,8 @@ __global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
   __syncthreads();
   const long long first = (long long)blockIdx.x * LNR_WARPS + warp;
   const long long stride = (long long)gridDim.x * LNR_WARPS;
-  const uint32_t row_bytes = (uint32_t)C * 4;
-  const uint32_t slot_bytes = row_bytes * (accumulate ? 3u : 2u);
+  const uint32_t row_bytes = (uint32_t)C * 4, dy_bytes = (uint32_t)(C * sizeof(DY));
+  const uint32_t slot_bytes = dy_bytes + row_bytes * (accumulate ? 2u : 1u);
   // lane 0: request row k of this warp into slot k % stages
   auto issue = [&](long long k) {
     const long long row = first + k * stride;
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
     float* slot = mine + (size_t)(k % stages) * slot_floats;
     uint64_t* bar = &bars[k % stages];
     mbar_arrive_expect_tx(bar, slot_bytes);
-    bulk_load_1d(slot, dy + row * C, row_bytes, bar);
+    bulk_load_1d(slot, dy + row * C, dy_bytes, bar);  // a bf16 row fills the first half of its part
     bulk_load_1d(slot + C, x + row * C, row_bytes, bar);
     if (accumulate) bulk_load_1d(slot + 2 * C, dres + row * C, row_bytes, bar);
   };
@@ -260,15 +274,15 @@ __global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
       break;
     }
     mbar_try_wait(&bars[st], par);  // every lane observes the completed phase
-    const float4* sdy = reinterpret_cast<const float4*>(mine + (size_t)st * slot_floats);
-    const float4* sx = sdy + C4;
-    const float4* sr = sdy + 2 * C4;
+    const DY* sdy = reinterpret_cast<const DY*>(mine + (size_t)st * slot_floats);
+    const float4* sx = reinterpret_cast<const float4*>(mine + (size_t)st * slot_floats) + C4;
+    const float4* sr = sx + C4;
     float m1 = 0.f, m2 = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int c4 = i * 32 + lane;
       if (c4 < C4) {
-        const float4 d = sdy[c4], xx = sx[c4];
+        const float4 d = load4<DY>(sdy + c4 * 4), xx = sx[c4];
         const float4 xh = make_float4((xx.x - mu) * rs, (xx.y - mu) * rs, (xx.z - mu) * rs, (xx.w - mu) * rs);
         const float a = d.x * gv[i].x, b = d.y * gv[i].y, cc = d.z * gv[i].z, e = d.w * gv[i].w;
         m1 += (a + b) + (cc + e);
@@ -290,7 +304,7 @@ __global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
     for (int i = 0; i < NV; ++i) {
       const int c4 = i * 32 + lane;
       if (c4 < C4) {
-        const float4 d = sdy[c4], xx = sx[c4];
+        const float4 d = load4<DY>(sdy + c4 * 4), xx = sx[c4];
         const float4 xh = make_float4((xx.x - mu) * rs, (xx.y - mu) * rs, (xx.z - mu) * rs, (xx.w - mu) * rs);
         float4 o = make_float4(rs * (d.x * gv[i].x - m1 - xh.x * m2), rs * (d.y * gv[i].y - m1 - xh.y * m2),
                                rs * (d.z * gv[i].z - m1 - xh.z * m2), rs * (d.w * gv[i].w - m1 - xh.w * m2));
