@@ -49,6 +49,8 @@ __global__ void attn_bwd_dot_kernel(const T* __restrict__ out, const T* __restri
 // fixed order.
 __global__ void attn_bwd_dot64_bf16_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
                                            float* __restrict__ D, int Bsz, int Tn, int NH) {
+  pdl_launch_dependents();
+  pdl_wait();
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;  // 16-byte piece
   const long long npieces = (long long)Bsz * Tn * NH * 8;
   const bool in = i < npieces;

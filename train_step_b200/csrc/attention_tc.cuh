@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
   const int C = NH * 64;
   const int nqb = (T + FA_BM - 1) / FA_BM;
   const int nitems = nqb * BH;  // item w: key block w / BH (the longest rows first), bh = w % BH
@@ -222,6 +223,7 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // programmatic dependent launch: global memory only from here on
 
   if (warp == 0) {
     // ---------------- producer: K/V per item; (Q_i, dO_i, lse, D) per unit ----------------
@@ -529,6 +531,7 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
   const int C = NH * 64;
   const int nqb = (T + FA_BM - 1) / FA_BM;
   const int nitems = nqb * BH;  // item w: query block nqb - 1 - w / BH (longest rows first), bh = w % BH
@@ -565,6 +568,7 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // programmatic dependent launch: global memory only from here on
 
   if (warp == 0) {
     if (lane == 0) {
@@ -921,6 +925,7 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
   static_assert((4 + 2 * FX_NST + 2 * 8 + 3) * 8 <= FB_BARS, "barrier space");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
   const int C = NH * 64;
   const int nqp = (T + 255) / 256;
   const int nitems = nqp * BH;  // item w: query pair nqp - 1 - w / BH, bh = w % BH
@@ -955,6 +960,7 @@ __global__ void __launch_bounds__(FX_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // programmatic dependent launch: global memory only from here on
 
   if (warp == 0) {
     if (lane == 0) {

@@ -285,6 +285,9 @@ int copy_tokens(gpt2* m, int* dst, const int32_t* src, size_t n) {
 int forward_layers(gpt2* m, int B, int T) {
   LaunchCtx c = m->ctx();
   const int dt = m->cfg.dtype;
+  // bf16: the tensor-core and LayerNorm kernels launch as programmatic dependents, so each
+  // one's set-up (barriers, TMEM allocation) overlaps the tail of the kernel before it
+  c.pdl = dt == GPT2_BF16 && !m->prof.on;
   const int N = B * T, C = m->C, F = m->F, L = m->L, NH = m->NH, hd = m->hd;
   const int64_t NC = (int64_t)m->Nmax * C, NF = (int64_t)m->Nmax * F, N3C = 3 * NC;
   const int64_t NLSE = (int64_t)m->cfg.B_max * NH * m->T;
@@ -330,6 +333,7 @@ int forward_layers(gpt2* m, int B, int T) {
 int run_micro_batch(gpt2* m, int B, int T, bool backward) {
   LaunchCtx c = m->ctx();
   const int dt = m->cfg.dtype;
+  c.pdl = dt == GPT2_BF16 && !m->prof.on;  // programmatic dependent launches, as in forward_layers
   const int N = B * T, C = m->C, F = m->F, L = m->L, NH = m->NH, hd = m->hd, Vp = m->Vp;
   const int64_t NC = (int64_t)m->Nmax * C, NF = (int64_t)m->Nmax * F, N3C = 3 * NC;
   const int64_t NLSE = (int64_t)m->cfg.B_max * NH * m->T;

@@ -47,6 +47,7 @@ __global__ void __launch_bounds__(CE_STHREADS) cross_entropy_stats_kernel(
     const float2* __restrict__ stats, int nstats, float* __restrict__ row_loss, int* err) {
   __shared__ float s_lse2[CE_SROWS];
   __shared__ int s_tgt[CE_SROWS];
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long r0 = (long long)blockIdx.x * CE_SROWS;
   if (warp < CE_SROWS && r0 + warp < rows) {

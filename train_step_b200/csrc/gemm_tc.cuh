@@ -290,6 +290,7 @@ __global__ void __launch_bounds__((2 + tc_epi_warps<EPI>()) * 32, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_launch_dependents();  // the next kernel may start its own set-up once every CTA is running
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -325,6 +326,10 @@ __global__ void __launch_bounds__((2 + tc_epi_warps<EPI>()) * 32, 1)
     __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // launched as a programmatic dependent (training step): the set-up above overlapped the
+  // previous kernel's tail; nothing in global memory is touched before this wait (a no-op
+  // for an ordinary launch)
+  pdl_wait();
   const uint64_t lim = p.timeout_ns;
 
   if (warp == 0) {

@@ -137,6 +137,7 @@ inline LaunchCtx side_ctx(const LaunchCtx& c) {
   cudaStreamWaitEvent(c.side->s, c.side->ready, 0);
   r.stream = c.side->s;
   r.side = nullptr;
+  r.pdl = false;
   return r;
 }
 // After the side-stream launches that read side buffer b.
@@ -388,7 +389,8 @@ int launch_tc_inst(const LaunchCtx& c, const TcMaps& tm, const GemmParams& p) {
   if (max_clusters < 0) return fail(c, GPT2_ERR_CUDA, "gemm_tc: no 2-CTA cluster fits");
   if (!PAIR) {
     const int grid = p.num_units < c.num_sms ? p.num_units : c.num_sms;
-    kern<<<grid, threads, smem, c.stream>>>(tm.a, tm.b, tm.o, tm.o2, p);
+    if (launch_k(c, kern, dim3(grid), dim3(threads), smem, tm.a, tm.b, tm.o, tm.o2, p) != cudaSuccess)
+      return fail(c, GPT2_ERR_CUDA, "gemm_tc: launch failed");
     return check_launch(c, "gemm_tc");
   }
   const int clusters = p.num_units < max_clusters ? p.num_units : max_clusters;
@@ -397,13 +399,15 @@ int launch_tc_inst(const LaunchCtx& c, const TcMaps& tm, const GemmParams& p) {
   cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = c.stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_k
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = c.pdl ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, kern, tm.a, tm.b, tm.o, tm.o2, p) != cudaSuccess)
     return fail(c, GPT2_ERR_CUDA, "gemm_tc: cluster launch failed");
   return check_launch(c, "gemm_tc_pair");
@@ -679,8 +683,10 @@ int launch_ln_bwd_ring(const LaunchCtx& c, int grid, int stages, const DY* dy, c
   // opted in once per device for the largest ring any C can ask for
   if (!smem_optin(layernorm_bwd_ring_kernel<T, NV, DY>, 232448 - 1024))
     return fail(c, GPT2_ERR_CUDA, "layernorm_bwd: shared-memory opt-in");
-  layernorm_bwd_ring_kernel<T, NV, DY><<<grid, LNR_WARPS * 32, smem, c.stream>>>(
-      dy, x, g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C, stages, c.d_err, 4000000000ull);
+  const cudaError_t e = launch_k(c, layernorm_bwd_ring_kernel<T, NV, DY>, dim3(grid), dim3(LNR_WARPS * 32), smem, dy, x,
+                                 g, mean, rstd, dres, dres_act, accumulate, part, with_rsum, N, C, stages, c.d_err,
+                                 4000000000ull);
+  if (e != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("layernorm_bwd: ") + cudaGetErrorString(e));
   return 0;
 }
 
@@ -773,8 +779,9 @@ inline int attention_fwd(const LaunchCtx& c, int dtype, const void* qkv, int B, 
     // persistent: one CTA per SM loops over (pair of query tiles, batch*head) items
     const long long items = (long long)((T + 255) / 256) * B * NH;
     const int grid = items < c.num_sms ? (int)items : c.num_sms;
-    attn_fwd_tc_kernel<<<grid, FX_THREADS, FX_SMEM, c.stream>>>(tqkv, tout, lse, T, NH, B * NH, scale, c.d_err,
-                                                                4000000000ull);
+    const cudaError_t e = launch_k(c, attn_fwd_tc_kernel, dim3(grid), dim3(FX_THREADS), FX_SMEM, tqkv, tout, lse, T,
+                                   NH, B * NH, scale, c.d_err, 4000000000ull);
+    if (e != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("attn_fwd_tc: ") + cudaGetErrorString(e));
     return check_launch(c, "attn_fwd_tc");
   }
   if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");
@@ -799,8 +806,9 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
     if ((reinterpret_cast<uintptr_t>(qkv) & 15) || (reinterpret_cast<uintptr_t>(dout) & 15) ||
         (reinterpret_cast<uintptr_t>(out) & 15))
       return fail(c, GPT2_ERR_CONFIG, "attention: qkv, out and dout must be 16-byte aligned");
-    attn_bwd_dot64_bf16_kernel<<<(int)((warps * 8 + 255) / 256), 256, 0, c.stream>>>((const bf16*)out, (const bf16*)dout,
-                                                                                  Dbuf, B, T, NH);
+    const cudaError_t e = launch_k(c, attn_bwd_dot64_bf16_kernel, dim3((unsigned)((warps * 8 + 255) / 256)), dim3(256), 0,
+                                   (const bf16*)out, (const bf16*)dout, Dbuf, B, T, NH);
+    if (e != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("attn_bwd_dot: ") + cudaGetErrorString(e));
     int r = check_launch(c, "attn_bwd_dot");
     if (r) return r;
     CUtensorMap tq, td, tout;  // 128-row tiles of qkv, dout and dqkv
@@ -813,12 +821,14 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
     // persistent: one CTA per SM loops over (block, batch*head) items
     const long long items = (long long)((T + FA_BM - 1) / FA_BM) * B * NH;
     const int grid = items < c.num_sms ? (int)items : c.num_sms;
-    attn_bwd_dkdv_tc_kernel<<<grid, BK_THREADS, BK_SMEM, c.stream>>>(tq, td, tout, lse, Dbuf, colsum, T, NH, B * NH,
-                                                                     scale, c.d_err, 4000000000ull);
+    cudaError_t e2 = launch_k(c, attn_bwd_dkdv_tc_kernel, dim3(grid), dim3(BK_THREADS), BK_SMEM, tq, td, tout, lse,
+                              (const float*)Dbuf, colsum, T, NH, B * NH, scale, c.d_err, 4000000000ull);
+    if (e2 != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("attn_bwd_dkdv_tc: ") + cudaGetErrorString(e2));
     r = check_launch(c, "attn_bwd_dkdv_tc");
     if (r) return r;
-    attn_bwd_dq_tc_kernel<<<grid, BQ_THREADS, BQ_SMEM, c.stream>>>(tq, td, tout, lse, Dbuf, colsum, T, NH, B * NH,
-                                                                   scale, c.d_err, 4000000000ull);
+    e2 = launch_k(c, attn_bwd_dq_tc_kernel, dim3(grid), dim3(BQ_THREADS), BQ_SMEM, tq, td, tout, lse, (const float*)Dbuf,
+                  colsum, T, NH, B * NH, scale, c.d_err, 4000000000ull);
+    if (e2 != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("attn_bwd_dq_tc: ") + cudaGetErrorString(e2));
     return check_launch(c, "attn_bwd_dq_tc");
   }
   if (hd % 32 || hd > 128) return fail(c, GPT2_ERR_CONFIG, "attention (fp32): head dim must be 32, 64, 96 or 128");

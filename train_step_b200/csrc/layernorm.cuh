@@ -45,10 +45,8 @@ __global__ void __launch_bounds__(LN_WARPS * 32) layernorm_fwd_kernel(const floa
                                                                       float* __restrict__ mean,
                                                                       float* __restrict__ rstd, int N, int C) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (PDL) {
-    pdl_launch_dependents();
-    pdl_wait();
-  }
+  pdl_launch_dependents();
+  if (PDL) pdl_wait();
   const long long row = (long long)blockIdx.x * LN_WARPS + warp;
   if (row >= N) return;
   const float* xr = x + row * C;
@@ -218,12 +216,14 @@ __global__ void __launch_bounds__(LNR_WARPS * 32, 1) layernorm_bwd_ring_kernel(
   float* ring = reinterpret_cast<float*>(lnr_smem);
   float* mine = ring + (size_t)warp * stages * slot_floats;
   uint64_t* bars = reinterpret_cast<uint64_t*>(lnr_smem + (size_t)LNR_WARPS * stages * slot_floats * 4) + warp * stages;
+  pdl_launch_dependents();
   if (threadIdx.x == 0) s_abort = 0;
   if (lane == 0) {
     for (int st = 0; st < stages; ++st) mbar_init(&bars[st], 1);
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_wait();  // programmatic dependent launch: global memory only from here on
   const long long first = (long long)blockIdx.x * LNR_WARPS + warp;
   const long long stride = (long long)gridDim.x * LNR_WARPS;
   const uint32_t row_bytes = (uint32_t)C * 4, dy_bytes = (uint32_t)(C * sizeof(DY));
