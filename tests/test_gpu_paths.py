@@ -292,3 +292,32 @@ def test_grad_bucket_events_and_the_overlapped_exchange():
     assert np.array_equal(a.get_params(), b.get_params())
     a.close()
     b.close()
+
+
+# ---------------------------------------------------------------------------
+# Overlap does not change a bit: side-stream reductions and programmatic dependent launches
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("C,H", [(256, 4), (1600, 25)], ids=["C256", "C1600"])
+def test_overlapped_and_in_order_runs_are_bitwise_equal(C, H):
+    """The bf16 step normally overlaps gradient reductions on a second stream and launches its
+    kernels as programmatic dependents; with per-kernel profiling on, everything runs in order
+    on one stream with ordinary launches. Every reduction has a fixed order, so the two must
+    agree bit for bit: losses, accumulated gradients and the parameters after a step. A missing
+    wait in either mechanism would show up here as a difference."""
+    cfg = tsb.Config(L=2, H=H, C=C, T=256, V=3001, tied=1, qkv_bias=1, dtype=tsb.BF16, B_max=4)
+    batches = [synth.micro_batch(4, cfg.T, cfg.V, index=60 + i) for i in range(3)]
+    out = []
+    for in_order in (False, True):
+        m = tsb.GPT2(cfg, seed=17)
+        if in_order:
+            m.profile(True)
+        losses = [m.forward_backward(tok, tgt) for tok, tgt in batches]
+        g = m.get_grads()
+        gn = m.step(1e-3, 0.1, 0.9, 0.95)
+        out.append((losses, g, gn, m.get_params()))
+        m.close()
+    (la, ga, na, pa), (lb, gb, nb, pb) = out
+    assert la == lb
+    assert np.array_equal(ga, gb)
+    assert na == nb
+    assert np.array_equal(pa, pb)
