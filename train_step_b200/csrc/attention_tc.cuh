@@ -41,7 +41,7 @@ constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 //       P^T = 2^(S^T*scale*log2e - lse*log2e), dS^T = P^T (dP^T - D)   (element-wise)
 //       dV += P^T dO_i, dK += dS^T Q_i        (M=128 keys, N=64, K=128 queries; A = P^T /
 //                                              dS^T in TMEM, B = dO_i / Q_i MN-major)
-//     lse*log2e and D of a unit's queries are staged in shared memory by the producer warp.
+//     -lse*log2e and -D of a unit's queries are staged in shared memory by the producer warp.
 //   dQ: item = (128-query block qb, batch*head); units = the key blocks 0 .. qb, in
 //     query-row orientation (lse and D of the thread's row are registers):
 //       S = Q K_j^T, dP = dO V_j^T            (M=128 queries, N=128 keys, K=64; A = Q / dO

@@ -221,15 +221,15 @@ int tensor_bucket(const gpt2* m, size_t i) {
 
 // Record grad_events[b] once bucket b's gradients are complete: on the side stream (after
 // everything the main stream has enqueued) when there is one, so the main stream never waits.
-int mark_bucket(gpt2* m, const LaunchCtx& cb, int b) {
-  if (m->grad_events.empty()) return GPT2_OK;
+int mark_bucket(gpt2* m, const std::vector<cudaEvent_t>& ev, const LaunchCtx& cb, int b) {
+  if (ev.empty()) return GPT2_OK;
   cudaStream_t s = cb.stream;
   if (cb.side) {
     CK(m, cudaEventRecord(cb.side->ready, cb.stream));
     CK(m, cudaStreamWaitEvent(cb.side->s, cb.side->ready, 0));
     s = cb.side->s;
   }
-  CK(m, cudaEventRecord(m->grad_events[b], s));
+  CK(m, cudaEventRecord(ev[b], s));
   return GPT2_OK;
 }
 
@@ -348,6 +348,10 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
   // kernel that shares the GPU would charge it the overlap)
   LaunchCtx cb = c;
   if (backward && dt == GPT2_BF16 && !m->prof.on) cb.side = &m->side;
+  // the gradient-bucket events armed for this backward pass (one-shot: taken now, so that a
+  // call that fails part-way leaves none behind for a later one)
+  std::vector<cudaEvent_t> bucket_ev;
+  if (backward) bucket_ev.swap(m->grad_events);
   EmbScratch es = emb_scratch_carve(m->emb_scratch, N, C);
   if (backward && cb.side) {
     // the embedding backward's sort of the token ids needs only the tokens: it runs on the
@@ -498,13 +502,12 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
       RK(LN_B(m->dh, xs(2 * l), w.ln1_g, mean(2 * l), rstd(2 * l), 1, gw.ln1_g, gw.ln1_b,
               l > 0 ? m->lg[l - 1].pj_b : nullptr));
     }
-    RK(mark_bucket(m, cb, l));  // layer l's pj_b came from layer l + 1's LayerNorm (or ln_f)
+    RK(mark_bucket(m, bucket_ev, cb, l));  // layer l's pj_b came from layer l + 1's LayerNorm (or ln_f)
   }
   RK(side_wait_free(cb, SIDE_EMB));  // the token sort (side stream) has finished
   RK(embedding_bwd(c, m->tok, m->dres, B, T, C, m->cfg.V, m->g_wte, m->g_wpe, es, cb.side != nullptr));
   RK(side_join(cb));  // every gradient is complete on the main stream from here on
-  RK(mark_bucket(m, c, L));
-  m->grad_events.clear();
+  RK(mark_bucket(m, bucket_ev, c, L));
   return GPT2_OK;
 }
 
