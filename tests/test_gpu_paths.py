@@ -277,6 +277,20 @@ def test_grad_bucket_events_and_the_overlapped_exchange():
     for x, y in zip(order, order[1:]):
         assert events[x].elapsed_time(events[y]) >= 0.0, (x, y)
     assert np.array_equal(a.get_grads(), b.get_grads())
+    # one-shot: a later backward pass does not record the events again (the marker recorded
+    # between the two calls stays after every bucket event)
+    marker = torch.cuda.Event(enable_timing=True)
+    marker.record()
+    a.forward_backward(tok, tgt, want_loss=False)
+    torch.cuda.synchronize()
+    assert all(e.elapsed_time(marker) >= 0.0 for e in events)
+    # armed, then a forward-only call: the events wait for the next backward pass
+    a.set_grad_events(events)
+    a.forward(tok, tgt)
+    marker.record()
+    a.forward_backward(tok, tgt, want_loss=False)
+    torch.cuda.synchronize()
+    assert all(marker.elapsed_time(e) >= 0.0 for e in events)
     with pytest.raises(tsb.Gpt2Error) as e:
         a.set_grad_events(events[:2])
     assert e.value.code == -1
