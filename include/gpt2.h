@@ -339,6 +339,23 @@ int gpt2_op_attention_fwd(int dtype, const void* qkv, int B, int T, int NH, int 
 int gpt2_op_attention_bwd(int dtype, const void* qkv, const void* out, const void* dout, const float* f32_lse, int B,
                           int T, int NH, int hd, void* dqkv, void* stream);
 
+/* The training step's form of the causal attention backward (bf16, hd == 64): the
+ * dK/dV kernel also stores the bf16 dS^T tiles it feeds to its dK product into the
+ * caller's workspace ds (DEVICE, gpt2_attention_ds_bytes(B, T, NH) bytes, 16-byte
+ * aligned: B*NH*nqb*nqb tiles of 32 KB, nqb = T / 128 rounded up, tile (b*NH + h, key
+ * block, query block) = two halves [128 keys][64 queries]; only the causal tiles are
+ * written), and dQ = dS K is then computed from them instead of
+ * recomputing the scores ("GPT From Scratch", Key decisions: the same gradients as the
+ * plain masked-softmax attention). Same arguments and results as gpt2_op_attention_bwd
+ * otherwise (deterministic, not bitwise equal to it: the dQ sums run in another order);
+ * ds == NULL returns GPT2_ERR_CONFIG. Synchronises the stream and reports a bounded wait
+ * that gave up as GPT2_ERR_TIMEOUT. */
+int gpt2_op_attention_bwd_stored(const void* qkv, const void* out, const void* dout, const float* f32_lse, int B,
+                                 int T, int NH, int hd, void* dqkv, void* ds, void* stream);
+
+/* Bytes of the dS^T workspace gpt2_op_attention_bwd_stored needs (0 for an empty shape). */
+size_t gpt2_attention_ds_bytes(int B, int T, int NH);
+
 /* Embedding forward: f32_x0[b*T + t, :] = wte[tokens[b*T + t], :] + wpe[t, :]
  * (wte [V, C], wpe [>= T, C], f32). Ids outside [0, V) raise
  * GPT2_ERR_TOKEN_RANGE (this call synchronises to report it). */

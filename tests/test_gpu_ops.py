@@ -238,9 +238,21 @@ def test_layernorm_bwd_overwrite(N, C):
 # ---------------------------------------------------------------------------
 # attention
 # ---------------------------------------------------------------------------
+def _attention_bwd_stored(qkv, out, dout, lse, dqkv, B, T, NH, hd):
+    """The training step's backward: dS^T tiles kept in a workspace, dQ computed from them.
+    The workspace starts as NaN so that a tile the dQ pass reads but nobody wrote shows."""
+    nbytes = tsb.attention_ds_bytes(B, T, NH)
+    nqb = (T + 127) // 128
+    assert nbytes == B * NH * nqb * nqb * 128 * 128 * 2
+    ds = torch.full((nbytes // 2,), float("nan"), dtype=torch.bfloat16, device=DEV)
+    tsb.attention_bwd_stored(qkv, out, dout, lse, dqkv, ds, B, T, NH, hd)
+    return ds
+
+
+@pytest.mark.parametrize("stored", [False, True])
 @pytest.mark.parametrize("B,T,NH", [(2, 200, 2), (1, 256, 3), (2, 64, 1), (1, 1024, 2), (1, 17, 2), (3, 300, 1),
                                     (1, 129, 2), (1, 385, 1), (2, 512, 2)])
-def test_attention_bf16(B, T, NH):
+def test_attention_bf16(B, T, NH, stored):
     hd = 64
     C = NH * hd
     qkv = randn((B * T, 3 * C), 30, torch.bfloat16)
@@ -254,12 +266,19 @@ def test_attention_bf16(B, T, NH):
     dout = randn((B * T, C), 31, torch.bfloat16)
     dqkv = torch.zeros_like(qkv)
     tsb.attention_bwd(qkv, out, dout, lse, dqkv, B, T, NH, hd)
+    if stored:
+        recomputed = dqkv.clone()
+        dqkv.fill_(float("nan"))
+        _attention_bwd_stored(qkv, out, dout, lse, dqkv, B, T, NH, hd)
     torch.cuda.synchronize()
     rd = oracle.attention_bwd(g64(qkv), g64(dout), B, T, NH, hd)
     got = g64(dqkv)
     for part in range(3):
         sl = slice(part * C, (part + 1) * C)
         assert rel_l2(got[:, sl], rd[:, sl]) < 2e-2, part
+    if stored:
+        # dK and dV come from the same kernel arithmetic in both forms
+        assert torch.equal(dqkv[:, C:], recomputed[:, C:])
 
 
 def test_attention_bf16_running_max_rebase():
@@ -301,7 +320,11 @@ def test_attention_bf16_full_size_sampled_heads():
     dout = randn((B * T, C), 34, torch.bfloat16)
     dqkv = torch.zeros_like(qkv)
     tsb.attention_bwd(qkv, out, dout, lse, dqkv, B, T, NH, hd)
+    dqkv_s = torch.zeros_like(qkv)
+    _attention_bwd_stored(qkv, out, dout, lse, dqkv_s, B, T, NH, hd)
     torch.cuda.synchronize()
+    assert torch.equal(dqkv_s[:, C:], dqkv[:, C:])
+    assert rel_l2(g64(dqkv_s[:, :C]), g64(dqkv[:, :C])) < 1e-2
     q3 = g64(qkv).reshape(B, T, 3, NH, hd)
     o3 = g64(out).reshape(B, T, NH, hd)
     d3 = g64(dout).reshape(B, T, NH, hd)
@@ -314,6 +337,9 @@ def test_attention_bf16_full_size_sampled_heads():
         rd = oracle.attention_bwd(qkv1, d3[b, :, h, :], 1, T, 1, hd).reshape(T, 3, hd)
         for part in range(3):
             assert rel_l2(g3[b, :, part, h, :], rd[:, part]) < 2e-2, (b, h, part)
+        # the stored-dS form's dQ (the training step's) against the oracle too
+        gs = g64(dqkv_s[:, :C]).reshape(B, T, NH, hd)
+        assert rel_l2(gs[b, :, h, :], rd[:, 0]) < 2e-2, (b, h)
 
 
 @pytest.mark.parametrize("B,T,NH,hd", [(2, 70, 2, 32), (1, 64, 4, 64), (2, 33, 1, 128)])

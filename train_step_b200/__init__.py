@@ -73,6 +73,9 @@ _SYMBOLS = {
                                ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_op_attention_bwd": ([ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int,
                                ct.c_int, ct.c_int, ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_op_attention_bwd_stored": ([ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int,
+                                      ct.c_int, ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p], ct.c_int),
+    "gpt2_attention_ds_bytes": ([ct.c_int, ct.c_int, ct.c_int], ct.c_size_t),
     "gpt2_op_embedding_fwd": ([ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_int, ct.c_int,
                                ct.c_void_p, ct.c_void_p], ct.c_int),
     "gpt2_op_token_buckets": ([ct.c_void_p, ct.c_int, ct.c_int, ct.c_void_p, ct.c_void_p, ct.c_void_p,
@@ -533,6 +536,17 @@ def attention_fwd(qkv, out, lse, B, T, NH, hd, stream=None):
 def attention_bwd(qkv, out, dout, lse, dqkv, B, T, NH, hd, stream=None):
     _op(lib().gpt2_op_attention_bwd(_dt(qkv), _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), B, T, NH, hd,
                                     _ptr(dqkv), _stream(stream)))
+
+
+def attention_ds_bytes(B, T, NH):
+    return lib().gpt2_attention_ds_bytes(B, T, NH)
+
+
+def attention_bwd_stored(qkv, out, dout, lse, dqkv, ds, B, T, NH, hd, stream=None):
+    """The training step's attention backward (bf16): dS^T tiles kept in ds
+    (attention_ds_bytes(B, T, NH) bytes of device memory) and dQ computed from them."""
+    _op(lib().gpt2_op_attention_bwd_stored(_ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), B, T, NH, hd, _ptr(dqkv),
+                                           _ptr(ds), _stream(stream)))
 
 
 def attention_bwd_noalloc(qkv, out, dout, lse, dqkv, B, T, NH, hd, stream=None):

@@ -47,6 +47,11 @@ constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 //       S = Q K_j^T, dP = dO V_j^T            (M=128 queries, N=128 keys, K=64; A = Q / dO
 //                                              copied into TMEM once per item)
 //       dQ += dS K_j                          (M=128 queries, N=64, K=128 keys; A = dS in TMEM)
+//   or, in the training step, dQ from the dS^T tiles the dK/dV kernel stored (bf16, the
+//     values its dK product used): attn_bwd_dq_stored_kernel streams them back, with K_j,
+//     through one accumulation product per unit. That replaces the recomputation of S, dP,
+//     P and dS (two thirds of the dQ kernel's tensor work and all of its exponentials) by
+//     2 x 32 KB of HBM traffic per unit, and the dQ pass becomes bandwidth-bound.
 //
 // TMEM (512 columns). dK/dV: S^T | dP^T (128 + 128), P^T | dS^T (64 + 64, bf16 pairs),
 // dV | dK (64 + 64). dQ: S | dP (128 + 128), Q | dO operands (32 + 32), dS for two units in
@@ -60,7 +65,11 @@ constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 // slower: 21 warps leave 80 registers per thread and the element-wise code spills).
 // Warps: 0 TMA producer, then the MMA issuers, then 16 element-wise warps: warp w reads
 // TMEM lane quarter w % 4 (32 rows) and column group (w - first) / 4 (32 of the 128
-// unit columns). D = rowsum(dO * O) comes precomputed. Every wait is bounded (device
+// unit columns); in dK/dV each element-wise warp stores what it holds (its 32 x 32 part of
+// a unit's dS^T when stored, its 32 x 16 parts of dK and dV) through a 2 KB shared-memory
+// buffer of its own and TMA stores issued by its lane 0, so that no warp waits for
+// another to store (one staging tile with a store-issuing warp measured 4 us slower per
+// launch at B = 16). D = rowsum(dO * O) comes precomputed. Every wait is bounded (device
 // error word, early exit, no trap).
 // ---------------------------------------------------------------------------
 constexpr int FB_EW_WARPS = 16;
@@ -74,7 +83,7 @@ constexpr int BK_NST = 3;
 constexpr int BK_OFF_KV = 0;                            // K | V [2 items]
 constexpr int BK_OFF_ST = 4 * FA_TILE;                  // stages: Q_i | dO_i
 constexpr int BK_OFF_LD = BK_OFF_ST + BK_NST * FB_STAGE;  // per stage: -lse*log2e [128] | -D [128]
-constexpr int BK_OFF_OUT = BK_OFF_LD + BK_NST * 1024;   // dK | dV staging for the TMA stores
+constexpr int BK_OFF_OUT = BK_OFF_LD + BK_NST * 1024;   // per element-wise warp 2 KB for its TMA stores
 constexpr int BK_OFF_BAR = BK_OFF_OUT + 2 * FA_TILE;
 constexpr int BK_SMEM = BK_OFF_BAR + FB_BARS + 1024;
 constexpr uint32_t BK_TM_DP = 128, BK_TM_P = 256, BK_TM_DS = 320, BK_TM_DV = 384, BK_TM_DK = 448;
@@ -102,6 +111,19 @@ __device__ __forceinline__ void fb_store16(uint8_t* tile, int r, int c16, const 
     uint4 w = make_uint4(pack_bf16x2(v[e], v[e + 1]), pack_bf16x2(v[e + 2], v[e + 3]),
                          pack_bf16x2(v[e + 4], v[e + 5]), pack_bf16x2(v[e + 6], v[e + 7]));
     *reinterpret_cast<uint4*>(tile + r * 128 + (((c16 + k) ^ (r & 7)) << 4)) = w;
+  }
+}
+
+// 16 accumulator values (x mul) as bf16 into a 32-byte row (an unswizzled box of 16 columns)
+__device__ __forceinline__ void fb_stage_row32b(uint8_t* row, const uint32_t (&v)[16], float mul) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int e = 8 * c;
+    *reinterpret_cast<uint4*>(row + 16 * c) =
+        make_uint4(pack_bf16x2(__uint_as_float(v[e]) * mul, __uint_as_float(v[e + 1]) * mul),
+                   pack_bf16x2(__uint_as_float(v[e + 2]) * mul, __uint_as_float(v[e + 3]) * mul),
+                   pack_bf16x2(__uint_as_float(v[e + 4]) * mul, __uint_as_float(v[e + 5]) * mul),
+                   pack_bf16x2(__uint_as_float(v[e + 6]) * mul, __uint_as_float(v[e + 7]) * mul));
   }
 }
 
@@ -162,11 +184,21 @@ __device__ __forceinline__ void fb_vals_to_tmem(const float (&v)[16], uint32_t t
 }
 
 
+// tm_out: dqkv [B][T][3C]; DS_OUT: in boxes of 16 columns x 32 rows (unswizzled), for the
+// per-warp dK and dV stores; otherwise in 128-row boxes (128-byte swizzle) for the two
+// staging tiles.
+// DS_OUT: also store every unit's dS^T tile (bf16, the values the dK product uses) through
+// tm_ds (boxes of 32 queries x 32 keys, 64-byte swizzle), for attn_bwd_dq_stored_kernel.
+// Tiles are contiguous: tile (bh, kb, i) is 32 KB at tile index (bh * nqb + kb) * nqb + i, as
+// two 16 KB halves (queries [0, 64) and [64, 128)) of 128 key rows x 64 queries (a 2-D view
+// with 64-element rows: row (2 tile + half) * 128 + key). Entries for keys or queries past T
+// are stored as zeros.
+template <bool DS_OUT>
 __global__ void __launch_bounds__(BK_THREADS, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                            const __grid_constant__ CUtensorMap tm_out, const float* __restrict__ lse,
-                            const float* __restrict__ Dg, float* __restrict__ colsum, int T, int NH, int BH,
-                            float scale, int* err, unsigned long long timeout_ns) {
+                            const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_ds,
+                            const float* __restrict__ lse, const float* __restrict__ Dg, float* __restrict__ colsum,
+                            int T, int NH, int BH, float scale, int* err, unsigned long long timeout_ns) {
   extern __shared__ uint8_t fb_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BK_OFF_BAR);
@@ -180,8 +212,8 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
   uint64_t* p_free = p_full + 1;              // the dV and dK products have read them (2 commits)
   uint64_t* acc_full = p_free + 1;            // the item's dV and dK complete (2 commits)
   uint64_t* acc_empty = acc_full + 1;         // dV and dK read by the epilogue (16 warps)
-  uint64_t* out_full = acc_empty + 1;         // output tiles staged (16 warps)
-  uint64_t* out_free = out_full + 1;          // the previous item's TMA stores have read the staging
+  uint64_t* out_full = acc_empty + 1;         // !DS_OUT: output tiles staged (16 warps)
+  uint64_t* out_free = out_full + 1;          // !DS_OUT: the previous item's TMA stores have read the staging
   uint64_t* drain = out_free + 1;             // [3]: one per MMA thread (abort path)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 4);
@@ -369,9 +401,9 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
     // ---------------- element-wise warps: key row r, query columns [cg*32, cg*32 + 32) of each unit ----------------
     const int q4 = warp & 3, cg = (warp - BK_EW0) >> 2;
     const int r = q4 * 32 + lane;
-    const bool issuer = (warp == BK_EW0 && lane == 0);  // issues the output tiles' TMA stores
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * LOG2E;
+    const bool issuer = !DS_OUT && warp == BK_EW0 && lane == 0;  // stores the staging tiles
     bool fail = false;
     int U = 0;
     for (int k = 0; !fail; ++k) {
@@ -431,6 +463,24 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
+        if (DS_OUT) {
+          // the same bf16 dS^T values, this warp's 32 keys x 32 queries, through its own 2 KB
+          // buffer (64-byte rows, 64-byte swizzle) and one TMA store issued by lane 0
+          uint8_t* buf = sm + BK_OFF_OUT + (warp - BK_EW0) * 2048;
+          if (lane == 0) bulk_wait_read<0>();  // the warp's previous store has read the buffer
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(dw[4 * c], dw[4 * c + 1], dw[4 * c + 2], dw[4 * c + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int i = kb + u, tile = (bh * nqb + kb) * nqb + i;
+            tma_store_2d(&tm_ds, buf, (cg & 1) * 32, (tile * 2 + (cg >> 1)) * 128 + q4 * 32);
+            bulk_commit();
+          }
+        }
       }
       if (fail) break;
       if (!fb_warp_wait(acc_full, k & 1, abort_flag, lim, lane)) {
@@ -462,35 +512,53 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
           row[2 * C] = sv2;
         }
       }
-      // dK (scaled) and dV through shared memory, one TMA store per tile (rows past T are clipped)
-      if (issuer && k > 0) {
-        bulk_wait_read<0>();
-        mbar_arrive(out_free);
-      }
-      if (!fb_warp_wait(out_free, (k & 1) ^ 1, abort_flag, lim, lane)) {
-        fail = true;
-        break;
-      }
-      fb_stage_row16(sm + BK_OFF_OUT, r, cg, kg, scale);
-      fb_stage_row16(sm + BK_OFF_OUT + FA_TILE, r, cg, v, 1.0f);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(out_full);
-      if (issuer) {
-        if (mbar_wait_bounded(out_full, k & 1, abort_flag, lim)) {
-          tma_store_3d(&tm_out, sm + BK_OFF_OUT, C + h * 64, kb * FA_BN, b);
-          tma_store_3d(&tm_out, sm + BK_OFF_OUT + FA_TILE, 2 * C + h * 64, kb * FA_BN, b);
+      if (DS_OUT) {
+        // dK (scaled) and dV of the warp's 32 keys x 16 columns through its buffer (32-byte
+        // rows), two TMA stores by lane 0 (rows past T are clipped)
+        uint8_t* buf = sm + BK_OFF_OUT + (warp - BK_EW0) * 2048;
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        fb_stage_row32b(buf + lane * 32, kg, scale);
+        fb_stage_row32b(buf + 1024 + lane * 32, v, 1.0f);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_out, buf, C + h * 64 + cg * 16, kb * FA_BN + q4 * 32, b);
+          tma_store_3d(&tm_out, buf + 1024, 2 * C + h * 64 + cg * 16, kb * FA_BN + q4 * 32, b);
           bulk_commit();
-        } else {
+        }
+      } else {
+        // dK (scaled) and dV through the two 128-row staging tiles, one TMA store per tile by
+        // the issuer (rows past T are clipped)
+        if (issuer && k > 0) {
+          bulk_wait_read<0>();
+          mbar_arrive(out_free);
+        }
+        if (!fb_warp_wait(out_free, (k & 1) ^ 1, abort_flag, lim, lane)) {
           fail = true;
+          break;
+        }
+        fb_stage_row16(sm + BK_OFF_OUT, r, cg, kg, scale);
+        fb_stage_row16(sm + BK_OFF_OUT + FA_TILE, r, cg, v, 1.0f);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(out_full);
+        if (issuer) {
+          if (mbar_wait_bounded(out_full, k & 1, abort_flag, lim)) {
+            tma_store_3d(&tm_out, sm + BK_OFF_OUT, C + h * 64, kb * FA_BN, b);
+            tma_store_3d(&tm_out, sm + BK_OFF_OUT + FA_TILE, 2 * C + h * 64, kb * FA_BN, b);
+            bulk_commit();
+          } else {
+            fail = true;
+          }
+        }
+        if (__shfl_sync(0xffffffffu, fail ? 1 : 0, 0)) {  // the issuer's warp leaves together
+          fail = true;
+          break;
         }
       }
-      if (__shfl_sync(0xffffffffu, fail ? 1 : 0, 0)) {  // the issuer's warp leaves together
-        fail = true;
-        break;
-      }
     }
-    if (issuer) bulk_wait_all();  // the staging must outlive the stores' reads
+    if (lane == 0) bulk_wait_all();  // the staging must outlive the stores' reads
     if (fail && lane == 0) {
       raise_device_error(err, DEV_TIMEOUT);
       *abort_flag = 1;
@@ -864,6 +932,232 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, FB_TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ from the stored dS^T tiles: dQ_qb = scale * sum_{j <= qb} dS_{qb,j} K_j. Item =
+// (128-query block qb, batch*head), longest first in the zigzag; unit = key block j.
+// Per unit the producer loads the dS^T tile (keys j*128.., queries qb*128..: 32 contiguous
+// KB, as four boxes of 64 queries x 64 keys, so that A = dS is the MN-major operand the
+// GEMM's dX role uses)
+// and K_j (128 keys x 64, MN-major B), and one thread issues the 8 products of K = 16
+// keys into a 64-column TMEM accumulator (two, alternating between items, so that the
+// epilogue of one item overlaps the next). Warps: 0 producer, 1 MMA issuer (and the TMEM
+// allocation), 2-5 epilogue (warp w drains TMEM lane quarter w % 4: 32 query rows x 64).
+// Bound by the dS^T bytes (2 per element of the causal half); every wait is bounded.
+// ---------------------------------------------------------------------------
+constexpr int DQS_THREADS = 192;
+constexpr int DQS_NST = 4;
+constexpr int DQS_STAGE = 3 * FA_TILE;  // dS^T tile (2 x 2 boxes of 8 KB) | K_j (16 KB)
+constexpr int DQS_OFF_OUT = DQS_NST * DQS_STAGE;
+constexpr int DQS_OFF_BAR = DQS_OFF_OUT + FA_TILE;
+constexpr int DQS_SMEM = DQS_OFF_BAR + FB_BARS + 1024;
+constexpr uint32_t DQS_TMEM_COLS = 128;
+static_assert(DQS_SMEM <= 232448, "shared memory per CTA");
+
+__global__ void __launch_bounds__(DQS_THREADS, 1)
+    attn_bwd_dq_stored_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_ds,
+                              const __grid_constant__ CUtensorMap tm_out, float* __restrict__ colsum, int T, int NH,
+                              int BH, float scale, int* err, unsigned long long timeout_ns) {
+  extern __shared__ uint8_t fb_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fb_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + DQS_OFF_BAR);
+  uint64_t* st_full = bar;                    // [DQS_NST] dS^T tile and K_j landed
+  uint64_t* st_empty = st_full + DQS_NST;     // [DQS_NST] the unit's products are complete
+  uint64_t* acc_full = st_empty + DQS_NST;    // [2] the item's dQ complete
+  uint64_t* acc_empty = acc_full + 2;         // [2] read by the epilogue (4 warps)
+  uint64_t* out_full = acc_empty + 2;         // output tile staged (4 warps)
+  uint64_t* out_free = out_full + 1;          // the previous item's TMA store has read the staging
+  uint64_t* drain = out_free + 1;             // the MMA thread's abort path
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  const int C = NH * 64;
+  const int nqb = (T + FA_BM - 1) / FA_BM;
+  const int nitems = nqb * BH;  // item w: query block nqb - 1 - w / BH (longest first), bh = w % BH
+  const int G = gridDim.x, cta = blockIdx.x;
+  const uint64_t lim = timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < DQS_NST; ++i) {
+      mbar_init(&st_full[i], 1);
+      mbar_init(&st_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(out_full, 4);
+    mbar_init(out_free, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, DQS_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // programmatic dependent launch: global memory only from here on
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- producer: (dS^T tile, K_j) per unit ----------------
+      tma_prefetch_desc(&tm_qkv);
+      tma_prefetch_desc(&tm_ds);
+      bool ok = true;
+      uint32_t st_iss = 0, st_par = 0;  // copies in flight, for the abort path
+      int U = 0;
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
+        const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
+        for (int j = 0; j <= qb; ++j, ++U) {
+          const int s = U % DQS_NST;
+          const uint32_t ph = (uint32_t)((U / DQS_NST) & 1);
+          if (!(ok = mbar_wait_bounded(&st_empty[s], ph ^ 1, abort_flag, lim))) break;
+          uint8_t* d = sm + s * DQS_STAGE;
+          const int tile = (bh * nqb + j) * nqb + qb;  // stored by the dK/dV kernel's item (bh, j), unit qb
+          mbar_arrive_expect_tx(&st_full[s], DQS_STAGE);
+#pragma unroll
+          for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+            for (int qh = 0; qh < 2; ++qh)
+              tma_load_2d(d + kh * FA_TILE + qh * 8192, &tm_ds, &st_full[s], 0, (tile * 2 + qh) * 128 + kh * 64);
+          tma_load_3d(d + 2 * FA_TILE, &tm_qkv, &st_full[s], C + h * 64, j * FA_BN, b);
+          st_iss |= 1u << s;
+          st_par = (st_par & ~(1u << s)) | (ph << s);
+        }
+      }
+      if (!ok) {
+        raise_device_error(err, DEV_TIMEOUT);
+        *abort_flag = 1;
+        int never = 0;  // let the copies in flight land before the CTA's shared memory goes away
+        for (int i = 0; i < DQS_NST; ++i)
+          if ((st_iss >> i) & 1u)
+            mbar_wait_bounded(&st_full[i], (st_par >> i) & 1u, reinterpret_cast<volatile int*>(&never), lim);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- dQ += dS K_j: A = dS (MN-major: queries contiguous), B = K_j (MN-major) ----------------
+      constexpr uint32_t idesc = make_idesc_bf16(128, 64, true, true);
+      bool ok = true, any = false;
+      int U = 0;
+      for (int k = 0; ok; ++k) {
+        const int item = fx_item(k, cta, G);
+        if (item >= nitems) break;
+        const int nu = nqb - item / BH, ab = k & 1;
+        if (!(ok = mbar_wait_bounded(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag, lim))) break;
+        for (int u = 0; u < nu; ++u, ++U) {
+          const int s = U % DQS_NST;
+          if (!(ok = mbar_wait_bounded(&st_full[s], (U / DQS_NST) & 1, abort_flag, lim))) break;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(sm + s * DQS_STAGE), sb = sa + 2 * FA_TILE;
+          // 16 keys per product: key rows 16 kk.. of the box pair kk / 4 (boxes of 64 keys),
+          // the two 64-query halves 8 KB apart; K_j rows 16 kk..
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16(tmem + (uint32_t)(ab * 64), make_sw128_desc(sa + (kk >> 2) * FA_TILE + (kk & 3) * 2048, 8192, 1024),
+                      make_sw128_desc(sb + kk * 2048, 8192, 1024), idesc, (u > 0 || kk > 0) ? 1u : 0u);
+          any = true;
+          umma_commit(&st_empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[ab]);
+      }
+      if (!ok) {
+        raise_device_error(err, DEV_TIMEOUT);
+        *abort_flag = 1;
+        if (any) {  // wait for the products already issued before the TMEM is freed
+          int never = 0;
+          umma_commit(drain);
+          mbar_wait_bounded(drain, 0, reinterpret_cast<volatile int*>(&never), lim);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: query row r, the 64 columns of dQ ----------------
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const bool issuer = (warp == 2 && lane == 0);  // issues the output tile's TMA store
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    bool fail = false;
+    for (int k = 0; !fail; ++k) {
+      const int item = fx_item(k, cta, G);
+      if (item >= nitems) break;
+      const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
+      const int ab = k & 1;
+      if (!fb_warp_wait(&acc_full[ab], (k >> 1) & 1, abort_flag, lim, lane)) {
+        fail = true;
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[4][16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(ab * 64 + g * 16), v[g]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (colsum) {
+        // column sums of dQ over this warp's 32 query rows (rows past T are zero: their dS
+        // entries are): the query third of the qkv bias gradient, one partial per 32-row block
+        float* row = colsum + (long long)((b * nqb + qb) * 4 + q4) * (3 * C) + h * 64;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          float cq[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) cq[e] = __uint_as_float(v[g][e]) * scale;
+          const float sq = warp_colsum16(cq, lane);
+          if (lane < 16) row[g * 16 + lane] = sq;
+        }
+      }
+      // dQ (scaled) through shared memory, one TMA store (rows past T are clipped)
+      if (issuer && k > 0) {
+        bulk_wait_read<0>();
+        mbar_arrive(out_free);
+      }
+      if (!fb_warp_wait(out_free, (k & 1) ^ 1, abort_flag, lim, lane)) {
+        fail = true;
+        break;
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) fb_stage_row16(sm + DQS_OFF_OUT, r, g, v[g], scale);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(out_full);
+      if (issuer) {
+        if (mbar_wait_bounded(out_full, k & 1, abort_flag, lim)) {
+          tma_store_3d(&tm_out, sm + DQS_OFF_OUT, h * 64, qb * FA_BM, b);
+          bulk_commit();
+        } else {
+          fail = true;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, fail ? 1 : 0, 0)) {  // the issuer's warp leaves together
+        fail = true;
+        break;
+      }
+    }
+    if (issuer) bulk_wait_all();  // the staging must outlive the store's read
+    if (fail && lane == 0) {
+      raise_device_error(err, DEV_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, DQS_TMEM_COLS);
   }
 }
 

@@ -65,6 +65,7 @@ struct gpt2 {
   float2* ce_stats = nullptr;  // softmax partials of one head chunk, [chunk rows][2 * ceil(Vp / 128)]
   float* splitk2 = nullptr;    // second split-K workspace (dW reductions alternate on the side stream)
   float* part_bias = nullptr;  // bias-gradient column-sum partials (GELU-backward epilogue, attention backward)
+  void* attn_ds = nullptr;     // bf16: the attention backward's stored dS^T tiles (one layer at a time)
   size_t part_bias_floats = 0;
   SideStream side;             // reductions of gradient partials overlapping the backward pass
   size_t part_floats = 0, splitk_floats = 0;
@@ -487,7 +488,7 @@ int run_micro_batch(gpt2* m, int B, int T, bool backward) {
     const bool qkvb_fused = gw.qkv_b && dt == GPT2_BF16;
     if (qkvb_fused) RK(side_wait_free(cb, SIDE_BIAS));
     RK(attention_bwd(c, dt, qkv, att, m->datt, lse, B, T, NH, hd, m->dqkv, m->Dattn,
-                     qkvb_fused ? m->part_bias : nullptr));
+                     qkvb_fused ? m->part_bias : nullptr, dt == GPT2_BF16 ? m->attn_ds : nullptr));
     if (qkvb_fused) RK(BIAS_RED(attn_colsum_blocks(B, T), 3 * C, gw.qkv_b));
     RK(DW(GemmDesc{m->dqkv, 3 * C, true, h1, C, true, 3 * C, C, N, EPI_F32, gw.qkv_w, C, nullptr, 0, nullptr,
                    nullptr, 0, 1, 0, CAT_GEMM_DW}));
@@ -634,6 +635,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out) {
       {(void**)&m->dres, (size_t)N * C * 4},
       {(void**)&m->dh, (size_t)N * C * 4},
       {(void**)&m->Dattn, (size_t)c.B_max * c.H * c.T * 4},
+      {(void**)&m->attn_ds, c.dtype == GPT2_BF16 ? attn_ds_bytes(c.B_max, c.T, c.H) : 0},
       {(void**)&m->row_loss, (size_t)N * 4},
       {(void**)&m->part, m->part_floats * 4},
       {(void**)&m->splitk, m->splitk_floats * 4},
@@ -1399,6 +1401,33 @@ int gpt2_op_attention_bwd(int dtype, const void* qkv, const void* out, const voi
   cudaFreeAsync(D, o.s);
   int r2 = o.finish();
   return r ? r : r2;
+}
+
+int gpt2_op_attention_bwd_stored(const void* qkv, const void* out, const void* dout, const float* lse, int B, int T,
+                                 int NH, int hd, void* dqkv, void* ds, void* stream) {
+  OpCtx o(stream);
+  if (B <= 0 || T <= 0 || NH <= 0) {
+    g_op_error = "attention: empty shape";
+    return GPT2_ERR_CONFIG;
+  }
+  if (!ds) {
+    g_op_error = "attention_bwd_stored: no dS workspace";
+    return GPT2_ERR_CONFIG;
+  }
+  RK(o.alloc_err());
+  float* D = nullptr;
+  if (cudaMallocAsync((void**)&D, (size_t)B * NH * T * 4, o.s) != cudaSuccess) {
+    o.finish();
+    return GPT2_ERR_OOM;
+  }
+  int r = attention_bwd(o.c, GPT2_BF16, qkv, out, dout, lse, B, T, NH, hd, dqkv, D, nullptr, ds);
+  cudaFreeAsync(D, o.s);
+  int r2 = o.finish();
+  return r ? r : r2;
+}
+
+size_t gpt2_attention_ds_bytes(int B, int T, int NH) {
+  return B > 0 && T > 0 && NH > 0 ? attn_ds_bytes(B, T, NH) : 0;
 }
 
 int gpt2_op_embedding_fwd(const int32_t* tokens, const float* wte, const float* wpe, int B, int T, int C, int V,

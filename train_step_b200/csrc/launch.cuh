@@ -307,15 +307,17 @@ inline bool encode_partial_map(CUtensorMap* map, const void* ptr, long long cols
 // qkv [B][T][3C] bf16 as a 3-D map {3C, T, B}; box {64, rows, 1} (one head's 64
 // columns of `rows` positions), 128-byte swizzle; positions past T read as zero.
 inline bool encode_qkv_map(CUtensorMap* map, const void* ptr, long long cols, long long T, long long B,
-                           unsigned rows = 128) {
+                           unsigned rows = 128, unsigned box_cols = 64) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), (cuuint64_t)(T * cols * 2)};
-  cuuint32_t box[3] = {64u, rows, 1u};
+  cuuint32_t box[3] = {box_cols, rows, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
+  // 64-column boxes: 128-byte rows, 128-byte swizzle; 16-column boxes: 32-byte rows, unswizzled
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   box_cols == 64 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -794,9 +796,18 @@ inline int attention_fwd(const LaunchCtx& c, int dtype, const void* qkv, int B, 
 // colsum (nullable, bf16 only): the kernels also leave the column sums of dqkv per 32-row
 // block, [B * ceil(T / 128) * 4][3 * NH * hd] (the qkv bias gradient after a reduction).
 inline int attn_colsum_blocks(int B, int T) { return B * ((T + FA_BM - 1) / FA_BM) * 4; }
+// dS^T workspace of the stored-dS backward: B*NH*nqb*nqb contiguous 32 KB tiles (nqb = T / 128
+// rounded up), tile (bh, key block, query block) = two halves of [128 keys][64 queries] bf16
+inline size_t attn_ds_bytes(int B, int T, int NH) {
+  const size_t nqb = (size_t)((T + FA_BM - 1) / FA_BM);
+  return (size_t)B * NH * nqb * nqb * 2 * FA_BN * 64 * 2;
+}
+// ds (nullable, bf16 only, attn_ds_bytes(B, T, NH) bytes, 16-byte aligned): when given, the
+// dK/dV kernel stores its dS^T tiles there and dQ is computed from them
+// (attn_bwd_dq_stored_kernel); otherwise the dQ kernel recomputes S, dP and dS.
 inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const void* out, const void* dout,
                          const float* lse, int B, int T, int NH, int hd, void* dqkv, float* Dbuf,
-                         float* colsum = nullptr) {
+                         float* colsum = nullptr, void* ds = nullptr) {
   const float scale = 1.0f / sqrtf((float)hd);
   ProfScope ps(c, CAT_ATTN_BWD, 2.5 * 4.0 * B * NH * hd * (0.5 * T * (T + 1.0)), 0.0);
   const long long warps = (long long)B * NH * T;
@@ -816,16 +827,34 @@ inline int attention_bwd(const LaunchCtx& c, int dtype, const void* qkv, const v
         !encode_qkv_map(&tout, dqkv, 3LL * NH * 64, T, B))
       return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
     if (reinterpret_cast<uintptr_t>(dqkv) & 15) return fail(c, GPT2_ERR_CONFIG, "attention: dqkv must be 16-byte aligned");
-    if (!smem_optin(attn_bwd_dkdv_tc_kernel, BK_SMEM) || !smem_optin(attn_bwd_dq_tc_kernel, BQ_SMEM))
+    if (reinterpret_cast<uintptr_t>(ds) & 15) return fail(c, GPT2_ERR_CONFIG, "attention: dS workspace must be 16-byte aligned");
+    // dS^T tiles as rows of 64 bf16: 128-key boxes for the dK/dV kernel's stores, 64-key
+    // boxes for the loads
+    const long long nqb = (T + FA_BM - 1) / FA_BM, ds_rows = (long long)B * NH * nqb * nqb * 2 * FA_BN;
+    if (ds && ds_rows >= (1LL << 31)) return fail(c, GPT2_ERR_CONFIG, "attention: dS workspace too large");
+    CUtensorMap tds_st = tq, tds_ld = tq;  // placeholders when dS is not stored (never read)
+    if (ds && (!encode_out_map(&tds_st, ds, 64, ds_rows, 64, false, 32) || !encode_bf16_map(&tds_ld, ds, 64, ds_rows, 64, 64)))
+      return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
+    CUtensorMap tout16;  // dqkv in boxes of 16 columns x 32 rows: the dK/dV kernel's per-warp stores
+    if (!encode_qkv_map(&tout16, dqkv, 3LL * NH * 64, T, B, 32, 16)) return fail(c, GPT2_ERR_CUDA, "attention: tensor map");
+    if (!smem_optin(attn_bwd_dkdv_tc_kernel<true>, BK_SMEM) || !smem_optin(attn_bwd_dkdv_tc_kernel<false>, BK_SMEM) ||
+        !smem_optin(attn_bwd_dq_tc_kernel, BQ_SMEM) || !smem_optin(attn_bwd_dq_stored_kernel, DQS_SMEM))
       return fail(c, GPT2_ERR_CUDA, "attention: shared-memory opt-in");
     // persistent: one CTA per SM loops over (block, batch*head) items
     const long long items = (long long)((T + FA_BM - 1) / FA_BM) * B * NH;
     const int grid = items < c.num_sms ? (int)items : c.num_sms;
-    cudaError_t e2 = launch_k(c, attn_bwd_dkdv_tc_kernel, dim3(grid), dim3(BK_THREADS), BK_SMEM, tq, td, tout, lse,
-                              (const float*)Dbuf, colsum, T, NH, B * NH, scale, c.d_err, 4000000000ull);
+    cudaError_t e2 = launch_k(c, ds ? attn_bwd_dkdv_tc_kernel<true> : attn_bwd_dkdv_tc_kernel<false>, dim3(grid),
+                              dim3(BK_THREADS), BK_SMEM, tq, td, ds ? tout16 : tout, tds_st, lse, (const float*)Dbuf,
+                              colsum, T, NH, B * NH, scale, c.d_err, 4000000000ull);
     if (e2 != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("attn_bwd_dkdv_tc: ") + cudaGetErrorString(e2));
     r = check_launch(c, "attn_bwd_dkdv_tc");
     if (r) return r;
+    if (ds) {
+      e2 = launch_k(c, attn_bwd_dq_stored_kernel, dim3(grid), dim3(DQS_THREADS), DQS_SMEM, tq, tds_ld, tout, colsum, T,
+                    NH, B * NH, scale, c.d_err, 4000000000ull);
+      if (e2 != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("attn_bwd_dq_stored: ") + cudaGetErrorString(e2));
+      return check_launch(c, "attn_bwd_dq_stored");
+    }
     e2 = launch_k(c, attn_bwd_dq_tc_kernel, dim3(grid), dim3(BQ_THREADS), BQ_SMEM, tq, td, tout, lse, (const float*)Dbuf,
                   colsum, T, NH, B * NH, scale, c.d_err, 4000000000ull);
     if (e2 != cudaSuccess) return fail(c, GPT2_ERR_CUDA, std::string("attn_bwd_dq_tc: ") + cudaGetErrorString(e2));

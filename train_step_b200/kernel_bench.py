@@ -143,6 +143,7 @@ def main() -> None:
     ap.add_argument("--C", type=int, default=768)
     ap.add_argument("--V", type=int, default=50257)
     ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--stored", action="store_true", help="attn_bwd: the training step's stored-dS form")
     ap.add_argument("--T0", type=int, default=512, help="decode: prompt length")
     ap.add_argument("--steps", type=int, default=64, help="decode: generated tokens per sequence")
     ap.add_argument("--topk", type=int, default=50, help="decode: k of the sampler")
@@ -180,6 +181,10 @@ def main() -> None:
         if a.kernel == "attn":
             ms = timeit(lambda: tsb.attention_fwd(qkv, out, lse, B, T, H, hd), a.iters)
             fl = 4.0 * B * H * hd * T * (T + 1) / 2
+        elif a.stored:
+            ds = torch.empty(tsb.attention_ds_bytes(B, T, H) // 2, dtype=torch.bfloat16, device=dev)
+            ms = timeit(lambda: tsb.attention_bwd_stored(qkv, out, dout, lse, dqkv, ds, B, T, H, hd), a.iters)
+            fl = 2.5 * 4.0 * B * H * hd * T * (T + 1) / 2
         else:
             ms = timeit(lambda: tsb.attention_bwd(qkv, out, dout, lse, dqkv, B, T, H, hd), a.iters)
             fl = 2.5 * 4.0 * B * H * hd * T * (T + 1) / 2
