@@ -20,6 +20,8 @@
 //  * outputs leave through a swizzled shared-memory tile and one TMA store per tile.
 // Every mbarrier wait is bounded (device error word, early exit, no trap).
 #pragma once
+#include <type_traits>
+
 #include "attention.cuh"
 #include "common.cuh"
 
@@ -420,37 +422,56 @@ __global__ void __launch_bounds__(BK_THREADS, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sv[32], dv[32];
-        tmem_ld_32x32b_x32(tmem + lane_off + (uint32_t)(cg * 32), sv);
-        tmem_ld_32x32b_x32(tmem + lane_off + BK_TM_DP + (uint32_t)(cg * 32), dv);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_empty);
         const float* ld = reinterpret_cast<const float*>(sm + BK_OFF_LD + s * 1024) + cg * 32;
         uint32_t pw[16], dw[16];
-        const bool diag = u == 0;  // the query block kb itself: queries before the key get P = 0
-        // pairs of columns on packed fp32 instructions: x = s scale log2e + (-lse log2e), then
-        // dS = P (dP + (-D)); the producer staged the negated lse and D
+        // The thread's 32 columns in two halves of 16 (scores and dP^T of a half loaded, then
+        // turned into P^T and dS^T): 32 loaded values live at a time instead of 64 keep the
+        // warp within its 96 registers without spills (measured: 122 -> 118 us per launch at
+        // B = 16 for the stored-dS form, 118 -> 103 us for the other). The score columns are
+        // released to the next unit's products once the second half is in registers.
+        // Pairs of columns run on packed fp32 instructions: x = s scale log2e + (-lse log2e),
+        // then dS = P (dP + (-D)); the producer staged the negated lse and D. In the query
+        // block kb itself (u == 0, a warp-uniform branch) queries before the key get P = 0;
+        // the other units run without the per-element test.
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 L4 = *reinterpret_cast<const float4*>(ld + 4 * e4);
-          const float4 D4 = *reinterpret_cast<const float4*>(ld + 128 + 4 * e4);
-          const uint64_t nl[2] = {f2_pack(L4.x, L4.y), f2_pack(L4.z, L4.w)};
-          const uint64_t nd[2] = {f2_pack(D4.x, D4.y), f2_pack(D4.z, D4.w)};
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int e = 4 * e4 + 2 * h;
-            const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nl[h]));
-            float p0 = ex2_fast(x.x), p1 = ex2_fast(x.y);
-            if (diag && cg * 32 + e < r) p0 = 0.f;
-            if (diag && cg * 32 + e + 1 < r) p1 = 0.f;
-            const float2 ds = f2_unpack(
-                f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd[h])));
-            pw[2 * e4 + h] = pack_bf16x2(p0, p1);
-            dw[2 * e4 + h] = pack_bf16x2(ds.x, ds.y);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sv[16], dv[16];
+          tmem_ld_32x32b_x16(tmem + lane_off + (uint32_t)(cg * 32 + half * 16), sv);
+          tmem_ld_32x32b_x16(tmem + lane_off + BK_TM_DP + (uint32_t)(cg * 32 + half * 16), dv);
+          tmem_ld_wait();
+          if (half == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_empty);
           }
+          auto p_ds = [&](auto diag_tag) {
+            constexpr bool DIAG = decltype(diag_tag)::value;
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) {
+              const float4 L4 = *reinterpret_cast<const float4*>(ld + half * 16 + 4 * e4);
+              const float4 D4 = *reinterpret_cast<const float4*>(ld + 128 + half * 16 + 4 * e4);
+              const uint64_t nl[2] = {f2_pack(L4.x, L4.y), f2_pack(L4.z, L4.w)};
+              const uint64_t nd[2] = {f2_pack(D4.x, D4.y), f2_pack(D4.z, D4.w)};
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int e = 4 * e4 + 2 * h, q = cg * 32 + half * 16 + e;  // q: query column in the unit
+                const float2 x =
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nl[h]));
+                float p0 = ex2_fast(x.x), p1 = ex2_fast(x.y);
+                if (DIAG && q < r) p0 = 0.f;
+                if (DIAG && q + 1 < r) p1 = 0.f;
+                const float2 ds = f2_unpack(f2_mul(
+                    f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd[h])));
+                pw[half * 8 + 2 * e4 + h] = pack_bf16x2(p0, p1);
+                dw[half * 8 + 2 * e4 + h] = pack_bf16x2(ds.x, ds.y);
+              }
+            }
+          };
+          if (u == 0)
+            p_ds(std::true_type{});
+          else
+            p_ds(std::false_type{});
         }
         // the previous unit's dV / dK products have finished reading P^T and dS^T
         if (!fb_warp_wait(p_free, (U & 1) ^ 1, abort_flag, lim, lane)) {
@@ -840,21 +861,29 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(s_empty);
         uint32_t dw[16];
-        const bool diag = u == nu - 1;  // the key block qb itself: keys after the query get P = 0
         // pairs of columns on packed fp32 instructions: x = s scale log2e - lse log2e, then
-        // dS = P (dP - D)
+        // dS = P (dP - D). In the key block qb itself (u == nu - 1, a warp-uniform branch) keys
+        // after the query get P = 0; the other units run without the per-element test.
         const uint64_t sl2x2 = f2_pack(sl2, sl2), nl2 = f2_pack(-lse2, -lse2), nd2 = f2_pack(-Dr, -Dr);
+        auto ds_row = [&](auto diag_tag) {
+          constexpr bool DIAG = decltype(diag_tag)::value;
 #pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          const int e = 2 * e2;
-          const float2 x = f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nl2));
-          float p0 = ex2_fast(x.x), p1 = ex2_fast(x.y);
-          if (diag && cg * 32 + e > r) p0 = 0.f;
-          if (diag && cg * 32 + e + 1 > r) p1 = 0.f;
-          const float2 ds = f2_unpack(
-              f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd2)));
-          dw[e2] = pack_bf16x2(ds.x, ds.y);
-        }
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const int e = 2 * e2;
+            const float2 x =
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sl2x2, nl2));
+            float p0 = ex2_fast(x.x), p1 = ex2_fast(x.y);
+            if (DIAG && cg * 32 + e > r) p0 = 0.f;
+            if (DIAG && cg * 32 + e + 1 > r) p1 = 0.f;
+            const float2 ds = f2_unpack(
+                f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), nd2)));
+            dw[e2] = pack_bf16x2(ds.x, ds.y);
+          }
+        };
+        if (u == nu - 1)
+          ds_row(std::true_type{});
+        else
+          ds_row(std::false_type{});
         // the dQ product of two units ago has finished reading this dS buffer
         if (!fb_warp_wait(&ds_free[U & 1], ((U >> 1) & 1) ^ 1, abort_flag, lim, lane)) {
           fail = true;
@@ -943,18 +972,22 @@ __global__ void __launch_bounds__(BQ_THREADS, 1)
 // GEMM's dX role uses)
 // and K_j (128 keys x 64, MN-major B), and one thread issues the 8 products of K = 16
 // keys into a 64-column TMEM accumulator (two, alternating between items, so that the
-// epilogue of one item overlaps the next). Warps: 0 producer, 1 MMA issuer (and the TMEM
-// allocation), 2-5 epilogue (warp w drains TMEM lane quarter w % 4: 32 query rows x 64).
-// Bound by the dS^T bytes (2 per element of the causal half); every wait is bounded.
+// epilogue of one item overlaps the next; four accumulators and eight epilogue warps
+// measured the same). Warps: 0 producer, 1 MMA issuer (and the TMEM allocation), 2-5
+// epilogue (warp w drains TMEM lane quarter w % 4: 32 query rows x 64). Bound by the dS^T
+// bytes (2 per element of the causal half): ~4.7 TB/s measured, the 4-stage ring being held
+// for a load's latency plus the products' completion latency per unit. Every wait is bounded.
 // ---------------------------------------------------------------------------
-constexpr int DQS_THREADS = 192;
+constexpr int DQS_EPI_WARPS = 4;
+constexpr int DQS_THREADS = 32 * (2 + DQS_EPI_WARPS);  // 192
+constexpr int DQS_ACC = 2;                             // TMEM accumulators of 64 columns
 constexpr int DQS_NST = 4;
 constexpr int DQS_STAGE = 3 * FA_TILE;  // dS^T tile (2 x 2 boxes of 8 KB) | K_j (16 KB)
 constexpr int DQS_OFF_OUT = DQS_NST * DQS_STAGE;
 constexpr int DQS_OFF_BAR = DQS_OFF_OUT + FA_TILE;
 constexpr int DQS_SMEM = DQS_OFF_BAR + FB_BARS + 1024;
-constexpr uint32_t DQS_TMEM_COLS = 128;
-static_assert(DQS_SMEM <= 232448, "shared memory per CTA");
+constexpr uint32_t DQS_TMEM_COLS = 64 * DQS_ACC;
+static_assert(DQS_SMEM <= 232448 && (4 * DQS_NST + 4 * DQS_ACC + 4) * 8 <= FB_BARS, "shared memory per CTA");
 
 __global__ void __launch_bounds__(DQS_THREADS, 1)
     attn_bwd_dq_stored_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_ds,
@@ -965,9 +998,9 @@ __global__ void __launch_bounds__(DQS_THREADS, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + DQS_OFF_BAR);
   uint64_t* st_full = bar;                    // [DQS_NST] dS^T tile and K_j landed
   uint64_t* st_empty = st_full + DQS_NST;     // [DQS_NST] the unit's products are complete
-  uint64_t* acc_full = st_empty + DQS_NST;    // [2] the item's dQ complete
-  uint64_t* acc_empty = acc_full + 2;         // [2] read by the epilogue (4 warps)
-  uint64_t* out_full = acc_empty + 2;         // output tile staged (4 warps)
+  uint64_t* acc_full = st_empty + DQS_NST;    // [DQS_ACC] the item's dQ complete
+  uint64_t* acc_empty = acc_full + DQS_ACC;   // [DQS_ACC] read by the epilogue warps
+  uint64_t* out_full = acc_empty + DQS_ACC;   // output tile staged (the epilogue warps)
   uint64_t* out_free = out_full + 1;          // the previous item's TMA store has read the staging
   uint64_t* drain = out_free + 1;             // the MMA thread's abort path
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -986,11 +1019,11 @@ __global__ void __launch_bounds__(DQS_THREADS, 1)
       mbar_init(&st_full[i], 1);
       mbar_init(&st_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < DQS_ACC; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
+      mbar_init(&acc_empty[i], DQS_EPI_WARPS);
     }
-    mbar_init(out_full, 4);
+    mbar_init(out_full, DQS_EPI_WARPS);
     mbar_init(out_free, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -1053,8 +1086,8 @@ __global__ void __launch_bounds__(DQS_THREADS, 1)
       for (int k = 0; ok; ++k) {
         const int item = fx_item(k, cta, G);
         if (item >= nitems) break;
-        const int nu = nqb - item / BH, ab = k & 1;
-        if (!(ok = mbar_wait_bounded(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag, lim))) break;
+        const int nu = nqb - item / BH, ab = k % DQS_ACC;
+        if (!(ok = mbar_wait_bounded(&acc_empty[ab], ((k / DQS_ACC) & 1) ^ 1, abort_flag, lim))) break;
         for (int u = 0; u < nu; ++u, ++U) {
           const int s = U % DQS_NST;
           if (!(ok = mbar_wait_bounded(&st_full[s], (U / DQS_NST) & 1, abort_flag, lim))) break;
@@ -1093,8 +1126,8 @@ __global__ void __launch_bounds__(DQS_THREADS, 1)
       const int item = fx_item(k, cta, G);
       if (item >= nitems) break;
       const int qb = nqb - 1 - item / BH, bh = item % BH, b = bh / NH, h = bh - b * NH;
-      const int ab = k & 1;
-      if (!fb_warp_wait(&acc_full[ab], (k >> 1) & 1, abort_flag, lim, lane)) {
+      const int ab = k % DQS_ACC;
+      if (!fb_warp_wait(&acc_full[ab], (k / DQS_ACC) & 1, abort_flag, lim, lane)) {
         fail = true;
         break;
       }
