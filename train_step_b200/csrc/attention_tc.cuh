@@ -5,10 +5,12 @@
 // "GPT From Scratch", Key decisions): per (batch, head), online softmax over key
 // blocks; lse = logsumexp of the scaled scores; the backward recomputes P from lse.
 //
-// Three persistent kernels (one CTA per SM looping over (block, batch*head) items,
-// longest first): the forward, and a deterministic backward split into a dK/dV
-// kernel (per key block) and a dQ kernel (per query block). They share one design,
-// set by what B200 measurements showed:
+// Persistent kernels (one CTA per SM looping over (block, batch*head) items, longest
+// first): the forward, and a deterministic backward split into a dK/dV kernel (per key
+// block) and a dQ kernel (per query block) -- in the training step the dK/dV kernel also
+// stores its dS^T tiles and the dQ kernel only multiplies them by K; the op-level calls
+// recompute dS in the dQ kernel instead. They share one design, set by what B200
+// measurements showed:
 //  * a thread can issue a 1-SM tcgen05.mma only every ~80-150 cycles, while the
 //    tensor pipe overlaps the streams of several threads, so each product (or pair of
 //    products that always run together) has its own issuing thread;
@@ -17,7 +19,7 @@
 //  * P and dS are written to TMEM by the element-wise warps and used there as the A
 //    operand of the following product; tiles are streamed through a TMA ring several
 //    units deep;
-//  * outputs leave through a swizzled shared-memory tile and one TMA store per tile.
+//  * outputs leave through swizzled shared-memory tiles and TMA stores.
 // Every mbarrier wait is bounded (device error word, early exit, no trap).
 #pragma once
 #include <type_traits>
