@@ -251,7 +251,7 @@ def _attention_bwd_stored(qkv, out, dout, lse, dqkv, B, T, NH, hd):
 
 @pytest.mark.parametrize("stored", [False, True])
 @pytest.mark.parametrize("B,T,NH", [(2, 200, 2), (1, 256, 3), (2, 64, 1), (1, 1024, 2), (1, 17, 2), (3, 300, 1),
-                                    (1, 129, 2), (1, 385, 1), (2, 512, 2)])
+                                    (1, 129, 2), (1, 385, 1), (2, 512, 2), (1, 1024, 16), (1, 640, 25)])
 def test_attention_bf16(B, T, NH, stored):
     hd = 64
     C = NH * hd
