@@ -69,12 +69,13 @@ constexpr int FA_TILE = FA_BM * 64 * 2;  // 16 KB: 128 rows x 64 bf16
 // slower: 21 warps leave 80 registers per thread and the element-wise code spills).
 // Warps: 0 TMA producer, then the MMA issuers, then 16 element-wise warps: warp w reads
 // TMEM lane quarter w % 4 (32 rows) and column group (w - first) / 4 (32 of the 128
-// unit columns); in dK/dV each element-wise warp stores what it holds (its 32 x 32 part of
-// a unit's dS^T when stored, its 32 x 16 parts of dK and dV) through a 2 KB shared-memory
-// buffer of its own and TMA stores issued by its lane 0, so that no warp waits for
-// another to store (one staging tile with a store-issuing warp measured 4 us slower per
-// launch at B = 16). D = rowsum(dO * O) comes precomputed. Every wait is bounded (device
-// error word, early exit, no trap).
+// unit columns). In dK/dV with dS stored, each element-wise warp stores what it holds (its
+// 32 x 32 part of a unit's dS^T, its 32 x 16 parts of dK and dV) through a 2 KB shared-memory
+// buffer of its own and TMA stores issued by its lane 0, so that no warp waits for another
+// to store (one staging tile with a store-issuing warp measured 4 us slower per launch at
+// B = 16); without, dK and dV leave through two 128-row staging tiles and one TMA store each.
+// D = rowsum(dO * O) comes precomputed. Every wait is bounded (device error word, early
+// exit, no trap).
 // ---------------------------------------------------------------------------
 constexpr int FB_EW_WARPS = 16;
 constexpr int FB_BARS = 512;
