@@ -281,6 +281,33 @@ def test_attention_bf16(B, T, NH, stored):
         assert torch.equal(dqkv[:, C:], recomputed[:, C:])
 
 
+def test_attention_bwd_stored_rejects_a_bad_workspace():
+    """The stored-dS entry point: no workspace, or one that is not 16-byte aligned, is a
+    configuration error reported before any dS tile is written; the next call works."""
+    B, T, NH, hd = 1, 256, 2, 64
+    C = NH * hd
+    qkv = randn((B * T, 3 * C), 35, torch.bfloat16)
+    out = torch.zeros(B * T, C, dtype=torch.bfloat16, device=DEV)
+    lse = torch.zeros(B, NH, T, device=DEV)
+    tsb.attention_fwd(qkv, out, lse, B, T, NH, hd)
+    dout = randn((B * T, C), 36, torch.bfloat16)
+    dqkv = torch.zeros_like(qkv)
+    with pytest.raises(tsb.Gpt2Error) as e:
+        tsb.attention_bwd_stored(qkv, out, dout, lse, dqkv, None, B, T, NH, hd)
+    assert e.value.code == -1
+    nbytes = tsb.attention_ds_bytes(B, T, NH)
+    raw = torch.zeros(nbytes // 2 + 8, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(tsb.Gpt2Error) as e:
+        tsb.attention_bwd_stored(qkv, out, dout, lse, dqkv, raw[1:], B, T, NH, hd)  # 2-byte offset
+    assert e.value.code == -1
+    ref = torch.zeros_like(qkv)
+    tsb.attention_bwd(qkv, out, dout, lse, ref, B, T, NH, hd)
+    _attention_bwd_stored(qkv, out, dout, lse, dqkv, B, T, NH, hd)
+    torch.cuda.synchronize()
+    assert torch.equal(dqkv[:, C:], ref[:, C:])
+    assert rel_l2(g64(dqkv[:, :C]), g64(ref[:, :C])) < 1e-2
+
+
 def test_attention_bf16_running_max_rebase():
     """Scores that grow by ~12 (log2 units) per 64 keys on odd query rows and stay flat
     on even rows: the odd rows re-base their running maximum (rescaling their output
