@@ -80,7 +80,10 @@ typedef struct gpt2 gpt2; /* opaque; the library owns all device memory it uses 
  * ^ (2j + 1), maps them to u1 in (0, 1] and u2 in [0, 1), and uses the cos branch
  * of Box-Muller, computed on the host in double and rounded to fp32.
  * Allocates parameters, gradients, Adam state, the bf16 shadow and the
- * activation arena for B_max * T tokens. On failure *out is NULL. */
+ * activation arena for B_max * T tokens (in bf16 mode it includes one layer's
+ * attention dS workspace, gpt2_attention_ds_bytes(B_max, T, H) bytes, which grows
+ * with T^2: 384 MiB at B_max = 16, T = 1024, H = 12). On failure *out is NULL and an
+ * arena larger than the free device memory returns GPT2_ERR_OOM. */
 int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2** out);
 
 /* Use `stream` (a cudaStream_t, e.g. torch.cuda.current_stream().cuda_stream) for
